@@ -1,0 +1,367 @@
+"""FP64 CPU oracle for Flint's sink-aware attention.
+
+TEST INFRASTRUCTURE ONLY. Only ``tests/``, ``__graft_entry__.smoke()`` and
+``bench.py``'s CPU-baseline leg may import this module. The CUDA library never
+calls it, and it shares no code with the CUDA library.
+
+What it computes, step by step, with the passage each step follows:
+
+* Per-head RMSNorm on q and k: Flint layers page
+  (nemo_automodel.components.models.flint.layers), ``FlintAttention`` class
+  summary ("per-head RMSNorm") and its ``q_norm``/``k_norm``/``eps`` attributes;
+  the epsilon is ``rms_norm_eps`` = 1e-6 on the Flint config page
+  (nemo_automodel.components.models.flint.config, ``FlintConfig``).
+* NeoX RoPE: Flint layers page, ``FlintAttention._apply_rope`` (each channel in
+  the first half of a head rotates with the matching channel of the second
+  half), applied to all head channels on sliding layers and not at all on full
+  layers (Flint config page, ``FlintConfig`` docstring; ``use_rope`` on the
+  layers page). Positions are document-local for THD (``FlintAttention.forward``,
+  ``position_ids``).
+* Causal window that counts the current token (``FlintConfig`` docstring;
+  attention utils page, ``preprocess_args_and_kwargs_for_attn``: a positive
+  left window counts visible keys including the current token, negative or
+  None is unbounded).
+* Block-diagonal document mask over THD packing (``cu_seqlens`` [documents+1]
+  on the attention utils page; the causal document mask of ``SequenceLayout.allowed``
+  on the mistral_large4 attention page).
+* A learned, unscaled FP32 sink logit per query head that enters only the
+  softmax denominator, with a zero value: ``_FlintSinkParameters.forward`` and
+  ``FlintAttention.forward`` ("causal attention with a zero-value sink
+  category") on the Flint layers page.
+* GQA with contiguous groups: head h reads KV head floor(h / (H / Hk)).
+
+Readings where the pages are silent: the softmax scale is 1/sqrt(head_dim);
+the norm weight is one [D] vector shared by all heads of q (and one for k),
+applied as w * x / sqrt(mean(x^2) + eps); norm comes before RoPE; RoPE
+frequencies are theta^(-2j/D) for j < D/2; W <= 0 is unbounded.
+
+The forward is the plain definition of softmax attention over the visible set
+plus the sink category. To keep memory bounded it is evaluated for blocks of at
+most ``BLOCK`` query rows at a time; nothing else is reordered. The backward is
+the analytic gradient of the same definition.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+BLOCK = 512
+
+
+# ----------------------------------------------------------------------------
+# Document layout
+# ----------------------------------------------------------------------------
+
+def doc_bounds(cu_doc_lens):
+    """List of (start, end) token ranges, one per document (THD ``cu_seqlens``)."""
+    cu = np.asarray(cu_doc_lens, dtype=np.int64)
+    return [(int(cu[d]), int(cu[d + 1])) for d in range(len(cu) - 1)]
+
+
+def doc_positions(cu_doc_lens):
+    """Document-local positions: 0, 1, ... restarting at every document start."""
+    cu = np.asarray(cu_doc_lens, dtype=np.int64)
+    pos = np.zeros(int(cu[-1]), dtype=np.int64)
+    for a, b in doc_bounds(cu):
+        pos[a:b] = np.arange(b - a)
+    return pos
+
+
+def visible_keys(i, d0, window):
+    """Key range [lo, i] visible from query token i of a document starting at d0.
+
+    The window counts the current token: key j is visible iff d0 <= j <= i and
+    (window <= 0 or i - j < window).
+    """
+    lo = d0 if window <= 0 else max(d0, i - window + 1)
+    return lo, i
+
+
+# ----------------------------------------------------------------------------
+# Prologue: per-head RMSNorm, then NeoX RoPE
+# ----------------------------------------------------------------------------
+
+def rms_norm(x, w, eps):
+    """w * x / sqrt(mean_c x_c^2 + eps) over the last (head_dim) axis.
+
+    Returns the normalised tensor and the per-row factor r = (mean x^2 + eps)^-1/2.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    r = 1.0 / np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + eps)
+    return x * r * np.asarray(w, dtype=np.float64), r
+
+
+def rope_angles(pos, head_dim, theta):
+    """Angles [T, D/2]: position times theta^(-2j/D) for frequency index j."""
+    j = np.arange(head_dim // 2, dtype=np.float64)
+    inv_freq = float(theta) ** (-2.0 * j / head_dim)
+    return np.asarray(pos, dtype=np.float64)[:, None] * inv_freq[None, :]
+
+
+def rope_neox(x, ang):
+    """Rotate channel j with channel j + D/2 of every head by angle ang[t, j].
+
+    x: [T, heads, D]; ang: [T, D/2].
+    """
+    h = x.shape[-1] // 2
+    c = np.cos(ang)[:, None, :]
+    s = np.sin(ang)[:, None, :]
+    x1, x2 = x[..., :h], x[..., h:]
+    return np.concatenate([x1 * c - x2 * s, x2 * c + x1 * s], axis=-1)
+
+
+def rope_neox_transpose(g, ang):
+    """Transpose (= inverse) of ``rope_neox``: rotation by the negated angle."""
+    h = g.shape[-1] // 2
+    c = np.cos(ang)[:, None, :]
+    s = np.sin(ang)[:, None, :]
+    g1, g2 = g[..., :h], g[..., h:]
+    return np.concatenate([g1 * c + g2 * s, g2 * c - g1 * s], axis=-1)
+
+
+def prologue(x, w, pos, use_rope, theta, eps):
+    """x [T, heads, D] -> x_hat: RMSNorm with weight w, then RoPE at positions pos [T]."""
+    y, _ = rms_norm(x, w, eps)
+    if use_rope:
+        y = rope_neox(y, rope_angles(pos, x.shape[-1], theta))
+    return y
+
+
+def prologue_backward(x, w, g_hat, pos, use_rope, theta, eps):
+    """Gradients of ``prologue`` w.r.t. x and w, given the gradient g_hat of x_hat.
+
+    With y = x r w, r = (mean x^2 + eps)^-1/2 and u = dy * w:
+    dx = r u - x r^3 (1/D) sum_c u_c x_c, and dw = sum over rows of dy * x r.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    w = np.asarray(w, dtype=np.float64)
+    D = x.shape[-1]
+    dy = g_hat
+    if use_rope:
+        dy = rope_neox_transpose(g_hat, rope_angles(pos, D, theta))
+    r = 1.0 / np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + eps)
+    dw = np.sum(dy * x * r, axis=tuple(range(x.ndim - 1)))
+    u = dy * w
+    dx = r * u - x * (r ** 3) * np.sum(u * x, axis=-1, keepdims=True) / D
+    return dx, dw
+
+
+# ----------------------------------------------------------------------------
+# Attention core with a sink category
+# ----------------------------------------------------------------------------
+
+def _group(h, H, Hk):
+    return h // (H // Hk)
+
+
+def _block_logits(q_hat, k_hat, a, b, lo, window, h_list, kv, scale):
+    """Scaled logits [len(h_list), b-a, b-lo] with -inf outside the visible set."""
+    q = q_hat[a:b][:, h_list, :]                       # [n, g, D]
+    k = k_hat[lo:b, kv, :]                             # [m, D]
+    z = scale * np.einsum("ngd,md->gnm", q, k)
+    i = np.arange(a, b)[:, None]
+    j = np.arange(lo, b)[None, :]
+    vis = j <= i
+    if window > 0:
+        vis &= (i - j) < window
+    z = np.where(vis[None, :, :], z, -np.inf)
+    return z
+
+
+def _sink_softmax(z, sink_g):
+    """Softmax over [z_i., s_h]: returns p [g,n,m], p_sink [g,n], lse [g,n]."""
+    s = sink_g[:, None]                                # [g, 1]
+    m = np.maximum(np.max(z, axis=-1), s)              # [g, n]
+    e = np.exp(z - m[..., None])
+    es = np.exp(s - m)
+    Z = es + np.sum(e, axis=-1)
+    p = e / Z[..., None]
+    return p, es / Z, m + np.log(Z)
+
+
+def attention_forward(q_hat, k_hat, v, sink, cu_doc_lens, window, scale=None):
+    """Sink-aware causal (windowed) GQA attention over THD documents.
+
+    q_hat [T,H,D], k_hat/v [T,Hk,D], sink [H] (unscaled logits).
+    Returns O [T,H,D] and LSE [H,T] = ln(e^{s_h} + sum_j e^{z_ij}).
+    """
+    T, H, D = q_hat.shape
+    Hk = k_hat.shape[1]
+    G = H // Hk
+    scale = 1.0 / np.sqrt(D) if scale is None else scale
+    sink = np.asarray(sink, dtype=np.float64)
+    O = np.zeros((T, H, v.shape[-1]))
+    lse = np.zeros((H, T))
+    for d0, d1 in doc_bounds(cu_doc_lens):
+        for a in range(d0, d1, BLOCK):
+            b = min(a + BLOCK, d1)
+            lo = d0 if window <= 0 else max(d0, a - window + 1)
+            for kv in range(Hk):
+                hs = list(range(kv * G, (kv + 1) * G))
+                z = _block_logits(q_hat, k_hat, a, b, lo, window, hs, kv, scale)
+                p, _, l = _sink_softmax(z, sink[hs])
+                O[a:b, kv * G:(kv + 1) * G, :] = np.einsum("gnm,md->ngd", p, v[lo:b, kv, :])
+                lse[kv * G:(kv + 1) * G, a:b] = l
+    return O, lse
+
+
+def attention_backward(q_hat, k_hat, v, sink, cu_doc_lens, window, dO, scale=None):
+    """Analytic gradients of ``attention_forward`` for the loss sum(dO * O).
+
+    D_i = dO_i . O_i; dv_j = sum_i p_ij dO_i; dz_ij = p_ij (dO_i . v_j - D_i);
+    dq_hat_i = scale sum_j dz_ij k_hat_j; dk_hat_j = scale sum_i dz_ij q_hat_i;
+    d sink_h = -sum_i p_sink_i D_i (the sink's value is zero).
+    Returns dq_hat, dk_hat, dv, dsink.
+    """
+    T, H, D = q_hat.shape
+    Hk = k_hat.shape[1]
+    G = H // Hk
+    scale = 1.0 / np.sqrt(D) if scale is None else scale
+    sink = np.asarray(sink, dtype=np.float64)
+    dO = np.asarray(dO, dtype=np.float64)
+    O, _ = attention_forward(q_hat, k_hat, v, sink, cu_doc_lens, window, scale)
+    Dvec = np.sum(dO * O, axis=-1)                     # [T, H]
+    dq = np.zeros_like(q_hat)
+    dk = np.zeros_like(k_hat)
+    dv = np.zeros_like(v, dtype=np.float64)
+    dsink = np.zeros(H)
+    for d0, d1 in doc_bounds(cu_doc_lens):
+        for a in range(d0, d1, BLOCK):
+            b = min(a + BLOCK, d1)
+            lo = d0 if window <= 0 else max(d0, a - window + 1)
+            for kv in range(Hk):
+                hs = list(range(kv * G, (kv + 1) * G))
+                z = _block_logits(q_hat, k_hat, a, b, lo, window, hs, kv, scale)
+                p, ps, _ = _sink_softmax(z, sink[hs])            # [g,n,m], [g,n]
+                dOb = dO[a:b, kv * G:(kv + 1) * G, :]             # [n,g,D]
+                Di = Dvec[a:b, kv * G:(kv + 1) * G].T             # [g,n]
+                dv[lo:b, kv, :] += np.einsum("gnm,ngd->md", p, dOb)
+                dp = np.einsum("ngd,md->gnm", dOb, v[lo:b, kv, :])
+                dz = p * (dp - Di[..., None])
+                dq[a:b, kv * G:(kv + 1) * G, :] += scale * np.einsum(
+                    "gnm,md->ngd", dz, k_hat[lo:b, kv, :])
+                dk[lo:b, kv, :] += scale * np.einsum(
+                    "gnm,ngd->md", dz, q_hat[a:b][:, hs, :])
+                dsink[hs] -= np.sum(ps * Di, axis=-1)
+    return dq, dk, dv, dsink
+
+
+# ----------------------------------------------------------------------------
+# Whole layer: prologue + attention (+ backward)
+# ----------------------------------------------------------------------------
+
+def _f64(x):
+    if hasattr(x, "detach"):
+        x = x.detach().to("cpu").double().numpy()
+    return np.asarray(x, dtype=np.float64)
+
+
+def flint_attn_fwd(q, k, v, w_q, w_k, sink, cu_doc_lens, window, use_rope,
+                   rope_theta, eps=1e-6, scale=None):
+    """Prologue on q and k, then sink-aware attention. Returns O [T,H,D], LSE [H,T]."""
+    q, k, v, w_q, w_k, sink = map(_f64, (q, k, v, w_q, w_k, sink))
+    cu = np.asarray(_f64(cu_doc_lens), dtype=np.int64)
+    pos = doc_positions(cu)
+    q_hat = prologue(q, w_q, pos, use_rope, rope_theta, eps)
+    k_hat = prologue(k, w_k, pos, use_rope, rope_theta, eps)
+    return attention_forward(q_hat, k_hat, v, sink, cu, window, scale)
+
+
+def flint_attn_bwd(q, k, v, w_q, w_k, sink, cu_doc_lens, window, use_rope,
+                   rope_theta, dO, eps=1e-6, scale=None):
+    """Gradients of sum(dO * O) w.r.t. the raw q, k, v, both norm weights and the sinks.
+
+    Returns a dict with dq, dk, dv, dw_q, dw_k, dsink.
+    """
+    q, k, v, w_q, w_k, sink, dO = map(_f64, (q, k, v, w_q, w_k, sink, dO))
+    cu = np.asarray(_f64(cu_doc_lens), dtype=np.int64)
+    pos = doc_positions(cu)
+    q_hat = prologue(q, w_q, pos, use_rope, rope_theta, eps)
+    k_hat = prologue(k, w_k, pos, use_rope, rope_theta, eps)
+    dqh, dkh, dv, dsink = attention_backward(q_hat, k_hat, v, sink, cu, window, dO, scale)
+    dq, dwq = prologue_backward(q, w_q, dqh, pos, use_rope, rope_theta, eps)
+    dk, dwk = prologue_backward(k, w_k, dkh, pos, use_rope, rope_theta, eps)
+    return {"dq": dq, "dk": dk, "dv": dv, "dw_q": dwq, "dw_k": dwk, "dsink": dsink}
+
+
+# ----------------------------------------------------------------------------
+# Sampled rows, for sizes where the whole layer is too slow on a CPU
+# ----------------------------------------------------------------------------
+
+def _doc_of(cu, t):
+    """(start, end) of the document holding token t."""
+    d = int(np.searchsorted(cu, t, side="right") - 1)
+    while cu[d + 1] <= t:          # skip empty documents that share a start
+        d += 1
+    return int(cu[d]), int(cu[d + 1])
+
+
+class RowOracle:
+    """Selected outputs of one layer, each computed on its own from the definition.
+
+    Used where the whole layer is too large for a CPU: a query row (t, h) needs
+    only its own visible keys; a key row (j, kv) needs the query rows that see it.
+    The normalised keys of the whole input are computed once (T * Hk * D work).
+    """
+
+    def __init__(self, q, k, v, w_q, w_k, sink, cu_doc_lens, window, use_rope,
+                 rope_theta, dO=None, eps=1e-6, scale=None):
+        self.q, self.k, self.v, self.w_q, self.w_k, self.sink = map(
+            _f64, (q, k, v, w_q, w_k, sink))
+        self.dO = None if dO is None else _f64(dO)
+        self.cu = np.asarray(_f64(cu_doc_lens), dtype=np.int64)
+        self.pos = doc_positions(self.cu)
+        self.window, self.use_rope, self.theta, self.eps = window, use_rope, rope_theta, eps
+        T, H, D = self.q.shape
+        self.H, self.Hk, self.D = H, self.k.shape[1], D
+        self.scale = 1.0 / np.sqrt(D) if scale is None else scale
+        self.k_hat = prologue(self.k, self.w_k, self.pos, use_rope, rope_theta, eps)
+
+    def _q_hat(self, t, h):
+        return prologue(self.q[t:t + 1, h:h + 1, :], self.w_q, self.pos[t:t + 1],
+                        self.use_rope, self.theta, self.eps)[0, 0]
+
+    def _row(self, t, h):
+        """Visible key range, probabilities over it, p_sink, LSE and O for row (t, h)."""
+        d0, _ = _doc_of(self.cu, t)
+        lo, hi = visible_keys(t, d0, self.window)
+        kv = _group(h, self.H, self.Hk)
+        z = self.scale * (self.k_hat[lo:hi + 1, kv, :] @ self._q_hat(t, h))
+        m = max(float(np.max(z)), float(self.sink[h]))
+        e = np.exp(z - m)
+        Z = np.exp(self.sink[h] - m) + np.sum(e)
+        p = e / Z
+        return lo, hi, kv, p, np.exp(self.sink[h] - m) / Z, m + np.log(Z), p @ self.v[lo:hi + 1, kv, :]
+
+    def forward_row(self, t, h):
+        """(O[t, h, :], LSE[h, t])."""
+        _, _, _, _, _, lse, o = self._row(t, h)
+        return o, lse
+
+    def dq_row(self, t, h):
+        """Gradient of sum(dO * O) w.r.t. the raw q[t, h, :]."""
+        lo, hi, kv, p, _, _, o = self._row(t, h)
+        Di = float(self.dO[t, h] @ o)
+        dz = p * (self.v[lo:hi + 1, kv, :] @ self.dO[t, h] - Di)
+        g_hat = self.scale * (dz @ self.k_hat[lo:hi + 1, kv, :])
+        dx, _ = prologue_backward(self.q[t:t + 1, h:h + 1, :], self.w_q, g_hat[None, None, :],
+                                  self.pos[t:t + 1], self.use_rope, self.theta, self.eps)
+        return dx[0, 0]
+
+    def dkv_row(self, j, kv):
+        """Gradients w.r.t. the raw k[j, kv, :] and v[j, kv, :]."""
+        d0, d1 = _doc_of(self.cu, j)
+        hi = d1 if self.window <= 0 else min(d1, j + self.window)
+        G = self.H // self.Hk
+        dk_hat = np.zeros(self.D)
+        dv = np.zeros(self.v.shape[-1])
+        for i in range(j, hi):
+            for h in range(kv * G, (kv + 1) * G):
+                lo, _, _, p, _, _, o = self._row(i, h)
+                pij = p[j - lo]
+                Di = float(self.dO[i, h] @ o)
+                dv += pij * self.dO[i, h]
+                dz = pij * (float(self.dO[i, h] @ self.v[j, kv]) - Di)
+                dk_hat += self.scale * dz * self._q_hat(i, h)
+        dx, _ = prologue_backward(self.k[j:j + 1, kv:kv + 1, :], self.w_k, dk_hat[None, None, :],
+                                  self.pos[j:j + 1], self.use_rope, self.theta, self.eps)
+        return dx[0, 0], dv
