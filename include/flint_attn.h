@@ -1,0 +1,138 @@
+/*
+ * flint_attn.h - C ABI of a B200 (sm_100a) library for Flint's sink-aware
+ * sliding/full GQA attention, forward and backward.
+ *
+ * What the calls compute (the passages that define it):
+ *   - Per-head RMSNorm of q and k with eps = rms_norm_eps (1e-6 by default):
+ *     Flint layers page (nemo_automodel.components.models.flint.layers),
+ *     FlintAttention ("Separate Q/K/V, per-head RMSNorm, selective Neox RoPE
+ *     and learned sinks"), attributes q_norm, k_norm, eps; Flint config page
+ *     (nemo_automodel.components.models.flint.config), FlintConfig.rms_norm_eps.
+ *     Reading: one weight vector [D] for q and one for k, shared by all heads,
+ *     applied as w * x / sqrt(mean(x^2) + eps).
+ *   - NeoX RoPE over all head channels on sliding layers, none on full layers:
+ *     FlintAttention._apply_rope (channel j rotates with channel j + D/2) and the
+ *     FlintConfig docstring. Frequencies theta^(-2j/D); positions restart at 0
+ *     in every document (FlintAttention.forward, position_ids for THD).
+ *     RMSNorm is applied first, then RoPE.
+ *   - Causal window that counts the current token; window <= 0 is unbounded:
+ *     FlintConfig docstring and sliding_window; attention utils page
+ *     (nemo_automodel.components.attention.utils),
+ *     preprocess_args_and_kwargs_for_attn ("window_size" semantics).
+ *   - THD packing: documents given by cu_doc_lens int32 [num_docs + 1], the
+ *     cu_seqlens format of preprocess_args_and_kwargs_for_attn; attention never
+ *     crosses a document boundary.
+ *   - GQA: query head h reads KV head h / (H / Hk).
+ *   - One learned FP32 sink logit per query head, unscaled, entering only the
+ *     softmax denominator with a zero value: _FlintSinkParameters.forward and
+ *     FlintAttention.forward ("causal attention with a zero-value sink
+ *     category").
+ *     LSE_i = ln(e^{sink_h} + sum_j e^{z_ij}),  O_i = sum_j e^{z_ij - LSE_i} v_j,
+ *     z_ij = softmax_scale * q_hat_i . k_hat_j.
+ *   - Backward: gradients of sum(dO * O) w.r.t. q, k, v (raw inputs, before
+ *     norm and RoPE), both norm weights and the sinks. The learned-sink training
+ *     kernel is named on the Flint layers page (module docstring).
+ *     d sink_h = -sum_i e^{sink_h - LSE_i} (dO_i . O_i).
+ *
+ * Conventions for every call:
+ *   - All tensor arguments are DEVICE pointers owned by the caller, contiguous,
+ *     row-major, 16-byte aligned. The library allocates no memory and keeps no
+ *     state between calls except a cached device property (SM count).
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream). Results are ready when the stream is synchronised.
+ *   - Argument errors are returned before any launch (no GPU work is queued).
+ *     A failed launch returns FLINT_ERR_CUDA. Device-side waits are bounded:
+ *     a wait that runs out sets a status word in the workspace, which
+ *     flint_attn_check_status() turns into FLINT_ERR_TIMEOUT.
+ *   - Layouts: q, out, dout, dq [T, H, D]; k, v, dk, dv [T, Hk, D];
+ *     q_norm_w, k_norm_w [D]; sink, dsink [H] fp32; lse [H, T] fp32;
+ *     dq_norm_w, dk_norm_w [D] fp32.
+ *   - dtype FLINT_BF16: q, k, v, out, dout, dq, dk, dv and the norm weights are
+ *     bfloat16; the attention contractions run on tcgen05 tensor cores with
+ *     FP32 accumulation. dtype FLINT_FP32: those tensors are float32 and every
+ *     step runs in FP32 on CUDA cores.
+ */
+#ifndef FLINT_ATTN_H
+#define FLINT_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FLINT_OK = 0,
+  FLINT_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, bad size, bad cu_doc_lens bound */
+  FLINT_ERR_UNSUPPORTED = 2,   /* valid but not implemented: head_dim != 128, G not in {1,2,4,8,16} */
+  FLINT_ERR_WORKSPACE = 3,     /* workspace smaller than flint_attn_workspace_bytes() */
+  FLINT_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed */
+  FLINT_ERR_TIMEOUT = 5        /* a device-side wait ran out (see flint_attn_check_status) */
+} flint_status_t;
+
+typedef enum { FLINT_BF16 = 0, FLINT_FP32 = 1 } flint_dtype_t;
+
+typedef struct {
+  int32_t total_tokens;   /* T = cu_doc_lens[num_docs]; 0 <= T < 2^31 / H / D */
+  int32_t num_docs;       /* N >= 1; zero-length documents are allowed */
+  int32_t num_q_heads;    /* H, a multiple of num_kv_heads */
+  int32_t num_kv_heads;   /* Hk >= 1; G = H / Hk must be 1, 2, 4, 8 or 16 */
+  int32_t head_dim;       /* D; must be 128 */
+  int32_t window;         /* > 0: key j visible from query i iff 0 <= i - j < window
+                             (counts the current token); <= 0: full causal */
+  int32_t use_rope;       /* nonzero: NeoX RoPE on all D channels after RMSNorm */
+  float rope_theta;       /* RoPE base (> 0 when use_rope) */
+  float rms_eps;          /* RMSNorm epsilon (Flint: 1e-6) */
+  float softmax_scale;    /* 0 => 1/sqrt(head_dim) */
+  int32_t dtype;          /* flint_dtype_t */
+} flint_attn_params_t;
+
+/* Bytes of device workspace a call needs (backward = 0 for flint_attn_fwd,
+ * 1 for flint_attn_bwd). Returns 0 if the params are invalid. The workspace
+ * must be 256-byte aligned and is not used after the call's kernels finish. */
+size_t flint_attn_workspace_bytes(const flint_attn_params_t* params, int backward);
+
+/* Forward: O and LSE.
+ *   q [T,H,D], k [T,Hk,D], v [T,Hk,D], q_norm_w [D], k_norm_w [D]  (dtype)
+ *   sink [H] fp32, cu_doc_lens [num_docs+1] int32 (device, non-decreasing,
+ *   cu_doc_lens[0] = 0, cu_doc_lens[num_docs] = T; not checked on the device)
+ *   out [T,H,D] (dtype), lse [H,T] fp32 (natural log). */
+flint_status_t flint_attn_fwd(const flint_attn_params_t* params,
+                              const void* q, const void* k, const void* v,
+                              const void* q_norm_w, const void* k_norm_w,
+                              const float* sink, const int32_t* cu_doc_lens,
+                              void* out, float* lse,
+                              void* workspace, size_t workspace_bytes, void* stream);
+
+/* Backward of sum(dout * out) for out = flint_attn_fwd(...).
+ *   out, lse: the forward's results for the same inputs; dout [T,H,D] (dtype).
+ *   Writes dq [T,H,D], dk [T,Hk,D], dv [T,Hk,D] (dtype; gradients w.r.t. the RAW
+ *   q, k, v), dq_norm_w, dk_norm_w [D] fp32, dsink [H] fp32. Outputs are
+ *   overwritten, not accumulated. q and k are re-normalised and re-rotated
+ *   inside (nothing from the forward besides out and lse is needed). */
+flint_status_t flint_attn_bwd(const flint_attn_params_t* params,
+                              const void* q, const void* k, const void* v,
+                              const void* q_norm_w, const void* k_norm_w,
+                              const float* sink, const int32_t* cu_doc_lens,
+                              const void* out, const float* lse, const void* dout,
+                              void* dq, void* dk, void* dv,
+                              float* dq_norm_w, float* dk_norm_w, float* dsink,
+                              void* workspace, size_t workspace_bytes, void* stream);
+
+/* Synchronises `stream`, reads and clears the device status word in
+ * `workspace` (written by bounded device waits), and returns FLINT_OK or
+ * FLINT_ERR_TIMEOUT (FLINT_ERR_CUDA if the stream itself reports an error). */
+flint_status_t flint_attn_check_status(void* workspace, void* stream);
+
+/* Static description of a status code. */
+const char* flint_status_string(flint_status_t status);
+
+/* Library version string, e.g. "flint_attn 0.1 sm_100a". */
+const char* flint_attn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FLINT_ATTN_H */

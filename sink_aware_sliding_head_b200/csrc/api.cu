@@ -1,0 +1,274 @@
+// api.cu - the C ABI declared in include/flint_attn.h: argument validation,
+// workspace carving, TMA tensor-map encoding and the launch sequence of each
+// call. Everything here is host code; it allocates nothing and launches only
+// this library's kernels on the caller's stream.
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "common.cuh"
+#include "sm100_primitives.cuh"
+
+namespace flint {
+
+cudaError_t launch_reduce_rows(const float* part, int nrows, int width, float* out,
+                               cudaStream_t st);
+cudaError_t launch_attn_fwd_sm100_impl(const CUtensorMap& tq, const CUtensorMap& tk,
+                                       const CUtensorMap& tv, const Resolved& p, const float* sink,
+                                       const int4* items, const int* n_items, int max_items,
+                                       void* out, float* lse, int* status, int num_sms,
+                                       cudaStream_t st);
+cudaError_t launch_attn_bwd_sm100_impl(const CUtensorMap& tq, const CUtensorMap& tk,
+                                       const CUtensorMap& tv, const CUtensorMap& tdo,
+                                       const Resolved& p, const float* lse, const float* dvec,
+                                       const int4* items_kv, const int* n_kv, int max_kv,
+                                       const int4* items_q, const int* n_q, int max_q,
+                                       float* dq_acc, float* dk_acc, void* dv, int* status,
+                                       int num_sms, cudaStream_t st);
+
+namespace {
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+flint_status_t resolve(const flint_attn_params_t* in, Resolved* p) {
+  if (!in) return FLINT_ERR_INVALID_ARG;
+  if (in->dtype != FLINT_BF16 && in->dtype != FLINT_FP32) return FLINT_ERR_INVALID_ARG;
+  if (in->total_tokens < 0 || in->num_docs < 1 || in->num_q_heads < 1 || in->num_kv_heads < 1)
+    return FLINT_ERR_INVALID_ARG;
+  if (in->num_q_heads % in->num_kv_heads != 0) return FLINT_ERR_INVALID_ARG;
+  if (in->head_dim != kHeadDim) return FLINT_ERR_UNSUPPORTED;
+  const int G = in->num_q_heads / in->num_kv_heads;
+  if (in->dtype == FLINT_BF16 && !(G == 1 || G == 2 || G == 4 || G == 8 || G == 16))
+    return FLINT_ERR_UNSUPPORTED;
+  if ((long long)in->total_tokens * in->num_q_heads * in->head_dim > 0x7fffffffLL)
+    return FLINT_ERR_INVALID_ARG;
+  if (!(std::isfinite(in->rms_eps) && in->rms_eps >= 0.f)) return FLINT_ERR_INVALID_ARG;
+  if (in->use_rope && !(std::isfinite(in->rope_theta) && in->rope_theta > 0.f))
+    return FLINT_ERR_INVALID_ARG;
+  if (!std::isfinite(in->softmax_scale) || in->softmax_scale < 0.f) return FLINT_ERR_INVALID_ARG;
+  p->T = in->total_tokens;
+  p->N = in->num_docs;
+  p->H = in->num_q_heads;
+  p->Hk = in->num_kv_heads;
+  p->D = in->head_dim;
+  p->G = G;
+  p->W = in->window > 0 ? in->window : 0;
+  p->rope = in->use_rope ? 1 : 0;
+  p->theta = in->rope_theta;
+  p->eps = in->rms_eps;
+  p->scale = in->softmax_scale > 0.f ? in->softmax_scale : 1.0f / std::sqrt((float)kHeadDim);
+  p->dtype = in->dtype;
+  p->R = kTileRows / (G <= 128 ? G : 128);
+  if (p->R < 1) p->R = 1;
+  return FLINT_OK;
+}
+
+int sm_count() {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (cached[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+// 3-D bf16 tensor [T][heads][128] with a (64, box_heads, box_tokens) box and
+// 128-byte swizzle: one box fills one 128-row K-major operand panel.
+bool encode_3d(CUtensorMap* m, const void* base, int T, int heads, int box_heads, int box_tokens) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)kHeadDim, (cuuint64_t)heads, (cuuint64_t)(T > 0 ? T : 1)};
+  cuuint64_t strides[2] = {(cuuint64_t)kHeadDim * 2, (cuuint64_t)heads * kHeadDim * 2};
+  cuuint32_t box[3] = {64, (cuuint32_t)box_heads, (cuuint32_t)box_tokens};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <typename T>
+T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
+}
+
+flint_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? FLINT_OK : FLINT_ERR_CUDA; }
+
+#define FLINT_TRY(expr)                                    \
+  do {                                                     \
+    cudaError_t e_ = (expr);                               \
+    if (e_ != cudaSuccess) return FLINT_ERR_CUDA;          \
+  } while (0)
+
+}  // namespace
+}  // namespace flint
+
+using namespace flint;
+
+extern "C" size_t flint_attn_workspace_bytes(const flint_attn_params_t* params, int backward) {
+  Resolved p;
+  if (resolve(params, &p) != FLINT_OK) return 0;
+  return make_layout(p, backward != 0).total;
+}
+
+extern "C" flint_status_t flint_attn_fwd(const flint_attn_params_t* params, const void* q,
+                                         const void* k, const void* v, const void* q_norm_w,
+                                         const void* k_norm_w, const float* sink,
+                                         const int32_t* cu_doc_lens, void* out, float* lse,
+                                         void* workspace, size_t workspace_bytes, void* stream) {
+  Resolved p;
+  flint_status_t s = resolve(params, &p);
+  if (s != FLINT_OK) return s;
+  const void* vec16[] = {q, k, v, q_norm_w, k_norm_w, out};
+  for (const void* ptr : vec16)
+    if (!ptr || !aligned(ptr, 16)) return FLINT_ERR_INVALID_ARG;
+  if (!sink || !aligned(sink, 4) || !cu_doc_lens || !aligned(cu_doc_lens, 4) || !lse ||
+      !aligned(lse, 4))
+    return FLINT_ERR_INVALID_ARG;
+  const WsLayout L = make_layout(p, false);
+  if (!workspace || !aligned(workspace, 256)) return FLINT_ERR_INVALID_ARG;
+  if (workspace_bytes < L.total) return FLINT_ERR_WORKSPACE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  int* status = at<int>(workspace, L.status);
+  FLINT_TRY(cudaMemsetAsync(status, 0, 64 * sizeof(int), st));
+  if (p.T == 0) return FLINT_OK;
+  void* qh = at<void>(workspace, L.qhat);
+  void* kh = at<void>(workspace, L.khat);
+  FLINT_TRY(launch_prologue(p, q, q_norm_w, qh, p.H, cu_doc_lens, st));
+  FLINT_TRY(launch_prologue(p, k, k_norm_w, kh, p.Hk, cu_doc_lens, st));
+  if (p.dtype == FLINT_FP32) {
+    return cuda_status(launch_attn_fwd_fp32(p, (const float*)qh, (const float*)kh,
+                                            (const float*)v, sink, cu_doc_lens, (float*)out, lse,
+                                            st));
+  }
+  int4* items = at<int4>(workspace, L.items_q);
+  FLINT_TRY(launch_build_worklist(cu_doc_lens, p, kModeQuery, 2 * p.R, items, status + 1,
+                                  at<void>(workspace, L.sched_tmp), L.max_items_q, st));
+  CUtensorMap tq, tk, tv;
+  if (!encode_3d(&tq, qh, p.T, p.H, p.G, p.R) || !encode_3d(&tk, kh, p.T, p.Hk, 1, kTileKeys) ||
+      !encode_3d(&tv, v, p.T, p.Hk, 1, kTileKeys))
+    return FLINT_ERR_CUDA;
+  return cuda_status(launch_attn_fwd_sm100_impl(tq, tk, tv, p, sink, items, status + 1,
+                                                L.max_items_q, out, lse, status, sm_count(), st));
+}
+
+extern "C" flint_status_t flint_attn_bwd(const flint_attn_params_t* params, const void* q,
+                                         const void* k, const void* v, const void* q_norm_w,
+                                         const void* k_norm_w, const float* sink,
+                                         const int32_t* cu_doc_lens, const void* out,
+                                         const float* lse, const void* dout, void* dq, void* dk,
+                                         void* dv, float* dq_norm_w, float* dk_norm_w,
+                                         float* dsink, void* workspace, size_t workspace_bytes,
+                                         void* stream) {
+  Resolved p;
+  flint_status_t s = resolve(params, &p);
+  if (s != FLINT_OK) return s;
+  const void* vec16[] = {q, k, v, q_norm_w, k_norm_w, out, dout, dq, dk, dv};
+  for (const void* ptr : vec16)
+    if (!ptr || !aligned(ptr, 16)) return FLINT_ERR_INVALID_ARG;
+  const void* vec4[] = {sink, cu_doc_lens, lse, dq_norm_w, dk_norm_w, dsink};
+  for (const void* ptr : vec4)
+    if (!ptr || !aligned(ptr, 4)) return FLINT_ERR_INVALID_ARG;
+  const WsLayout L = make_layout(p, true);
+  if (!workspace || !aligned(workspace, 256)) return FLINT_ERR_INVALID_ARG;
+  if (workspace_bytes < L.total) return FLINT_ERR_WORKSPACE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  int* status = at<int>(workspace, L.status);
+  FLINT_TRY(cudaMemsetAsync(status, 0, 64 * sizeof(int), st));
+  if (p.T == 0) {
+    FLINT_TRY(cudaMemsetAsync(dsink, 0, p.H * sizeof(float), st));
+    FLINT_TRY(cudaMemsetAsync(dq_norm_w, 0, kHeadDim * sizeof(float), st));
+    FLINT_TRY(cudaMemsetAsync(dk_norm_w, 0, kHeadDim * sizeof(float), st));
+    return FLINT_OK;
+  }
+  void* qh = at<void>(workspace, L.qhat);
+  void* kh = at<void>(workspace, L.khat);
+  float* dvec = at<float>(workspace, L.dvec);
+  float* part = at<float>(workspace, L.part);
+  float* dq_acc = at<float>(workspace, L.dq_acc);
+  float* dk_acc = at<float>(workspace, L.dk_acc);
+  FLINT_TRY(launch_prologue(p, q, q_norm_w, qh, p.H, cu_doc_lens, st));
+  FLINT_TRY(launch_prologue(p, k, k_norm_w, kh, p.Hk, cu_doc_lens, st));
+  FLINT_TRY(launch_bwd_preprocess(p, out, dout, lse, sink, dvec, part, dsink, st));
+  if (p.dtype == FLINT_FP32) {
+    FLINT_TRY(launch_attn_bwd_fp32(p, (const float*)qh, (const float*)kh, (const float*)v,
+                                   (const float*)dout, lse, dvec, cu_doc_lens, dq_acc, dk_acc,
+                                   (float*)dv, st));
+  } else {
+    int4* items_kv = at<int4>(workspace, L.items_kv);
+    int4* items_q1 = at<int4>(workspace, L.items_q1);
+    void* tmp = at<void>(workspace, L.sched_tmp);
+    FLINT_TRY(launch_build_worklist(cu_doc_lens, p, kModeKey, kTileKeys, items_kv, status + 2, tmp,
+                                    L.max_items_kv, st));
+    FLINT_TRY(launch_build_worklist(cu_doc_lens, p, kModeQuery, p.R, items_q1, status + 3, tmp,
+                                    L.max_items_q1, st));
+    CUtensorMap tq, tk, tv, tdo;
+    if (!encode_3d(&tq, qh, p.T, p.H, p.G, p.R) || !encode_3d(&tk, kh, p.T, p.Hk, 1, kTileKeys) ||
+        !encode_3d(&tv, v, p.T, p.Hk, 1, kTileKeys) || !encode_3d(&tdo, dout, p.T, p.H, p.G, p.R))
+      return FLINT_ERR_CUDA;
+    FLINT_TRY(launch_attn_bwd_sm100_impl(tq, tk, tv, tdo, p, lse, dvec, items_kv, status + 2,
+                                         L.max_items_kv, items_q1, status + 3, L.max_items_q1,
+                                         dq_acc, dk_acc, dv, status, sm_count(), st));
+  }
+  float* part_q = part + (size_t)kPartBlocks * p.H;
+  float* part_k = part_q + (size_t)kPartBlocks * kHeadDim;
+  FLINT_TRY(launch_bwd_epilogue(p, q, q_norm_w, dq_acc, dq, dq_norm_w, part_q, p.H, cu_doc_lens,
+                                st));
+  FLINT_TRY(launch_bwd_epilogue(p, k, k_norm_w, dk_acc, dk, dk_norm_w, part_k, p.Hk, cu_doc_lens,
+                                st));
+  return FLINT_OK;
+}
+
+extern "C" flint_status_t flint_attn_check_status(void* workspace, void* stream) {
+  if (!workspace || !aligned(workspace, 256)) return FLINT_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return FLINT_ERR_CUDA;
+  int host = 0;
+  if (cudaMemcpy(&host, workspace, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return FLINT_ERR_CUDA;
+  if (host != 0) {
+    const int zero = 0;
+    if (cudaMemcpy(workspace, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
+      return FLINT_ERR_CUDA;
+    return FLINT_ERR_TIMEOUT;
+  }
+  return FLINT_OK;
+}
+
+extern "C" const char* flint_status_string(flint_status_t s) {
+  switch (s) {
+    case FLINT_OK: return "ok";
+    case FLINT_ERR_INVALID_ARG: return "invalid argument";
+    case FLINT_ERR_UNSUPPORTED: return "unsupported configuration";
+    case FLINT_ERR_WORKSPACE: return "workspace too small";
+    case FLINT_ERR_CUDA: return "CUDA error";
+    case FLINT_ERR_TIMEOUT: return "device wait timed out";
+  }
+  return "unknown status";
+}
+
+extern "C" const char* flint_attn_version(void) { return "flint_attn 0.1 sm_100a"; }

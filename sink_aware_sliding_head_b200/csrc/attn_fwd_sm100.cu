@@ -1,0 +1,432 @@
+// attn_fwd_sm100.cu - sink-aware sliding/full GQA attention forward on
+// Blackwell tensor cores (tcgen05 + TMEM + TMA), BF16 in, FP32 accumulate.
+//
+// What it computes (Flint layers page, nemo_automodel.components.models.flint.
+// layers, FlintAttention.forward: causal attention with a zero-value sink
+// category; _FlintSinkParameters.forward: unscaled FP32 sink logits; Flint
+// config page: the window counts the current token):
+//   O_i = sum_j e^{z_ij - LSE_i} v_j,  LSE_i = ln(e^{s_h} + sum_j e^{z_ij}),
+//   over keys j of the same document with 0 <= i - j < W (W <= 0: unbounded).
+//
+// Design:
+//   * A 128-row tile is R = 128/G tokens x the G query heads of one KV group,
+//     so every K/V tile staged by TMA feeds all G heads of the group (GQA
+//     sharing inside the CTA, no multicast). A CTA works on two such tiles at
+//     once ("tile 0" and "tile 1": 2R consecutive tokens) that share every K/V
+//     tile, so each K/V byte brought on chip serves 256 query rows.
+//   * Persistent grid (one CTA per SM) striding over an LPT-sorted work list
+//     built on the device; only key tiles inside the window and the document
+//     are visited, and only edge tiles are masked.
+//   * Warp roles: warps 0-3 run the softmax of tile 0, warps 4-7 of tile 1
+//     (thread = TMEM lane = query row), warp 8 issues TMA loads, warp 9 issues
+//     tcgen05.mma from one thread and owns the TMEM allocation.
+//   * TMEM (512 columns): S0 [0,128), S1 [128,256), O0 [256,384), O1 [384,512).
+//     P_i (bf16, two per column) overwrites the first 64 columns of S_i and is
+//     the A operand of the PV MMA straight from TMEM. Before the next QK MMA of
+//     tile i overwrites S_i, the issuer waits until the PV MMA of tile i has
+//     completed (a commit barrier), so no ordering between MMAs writing
+//     different accumulators is assumed.
+//   * Sink folding: the running max starts at the sink logit and the running
+//     sum at 1 (the sink's own weight), so there is no extra pass and a row is
+//     never all -inf. The max is updated lazily: O and l are rescaled only when
+//     the max grows by more than 2^8.
+#include "common.cuh"
+#include "sm100_primitives.cuh"
+
+namespace flint {
+
+namespace {
+
+constexpr int kStages = 2;
+constexpr int kThreads = 320;
+constexpr int kWarpTma = 8;
+constexpr int kWarpMma = 9;
+constexpr uint32_t kChunkBytes = 128 * 64 * 2;     // 128 rows x 64 bf16 (one 128B-swizzle panel)
+constexpr uint32_t kTileBytes = 2 * kChunkBytes;   // 128 rows x 128 bf16
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kRescaleThreshold = 8.0f;          // log2 units
+
+struct FwdArgs {
+  int T, H, Hk, G, R, W;
+  float scale_log2;
+  const float* sink;
+  const int4* items;
+  const int* n_items;
+  int max_items;
+  __nv_bfloat16* out;
+  float* lse;
+  int* status;
+};
+
+struct __align__(8) Barriers {
+  uint64_t q_full, q_empty;
+  uint64_t k_full[kStages], k_empty[kStages], v_full[kStages], v_empty[kStages];
+  uint64_t s_full[2], p_full[2], pv_done[2], o_full[2], o_empty[2];
+  uint64_t drain;
+};
+
+// Dynamic shared memory: [Q0 | Q1 | K stages | V stages | barriers | tmem addr | abort flag]
+constexpr uint32_t kOffQ = 0;
+constexpr uint32_t kOffK = 2 * kTileBytes;
+constexpr uint32_t kOffV = kOffK + kStages * kTileBytes;
+constexpr uint32_t kOffBar = kOffV + kStages * kTileBytes;
+constexpr uint32_t kOffTmem = kOffBar + sizeof(Barriers);
+constexpr uint32_t kOffAbort = kOffTmem + 16;
+constexpr uint32_t kSmemBytes = kOffAbort + 16 + 1024;   // + alignment slack
+
+struct Item {
+  int q0, d0, d1, g, kend, kbeg, ntiles;
+};
+
+__device__ __forceinline__ Item decode(const FwdArgs& a, int idx) {
+  const int4 it = a.items[idx];
+  Item r;
+  r.q0 = it.x; r.d0 = it.y; r.d1 = it.z; r.g = it.w;
+  r.kend = min(r.q0 + 2 * a.R, r.d1);
+  r.kbeg = a.W > 0 ? max(r.d0, r.q0 - a.W + 1) : r.d0;
+  r.ntiles = (r.kend - r.kbeg + kTileKeys - 1) / kTileKeys;
+  return r;
+}
+
+// K-major operand panel with 128-byte swizzle: rows of 128 bytes, 8-row groups
+// 1024 bytes apart. kk selects the 16-element K slice (of 8) across two panels.
+__device__ __forceinline__ uint64_t kmajor_desc(uint32_t tile_base, int kk) {
+  return make_sdesc(tile_base + (kk >> 2) * kChunkBytes + (kk & 3) * 32, 16, 1024);
+}
+// MN-major operand (V: keys x D with D contiguous), 128-byte swizzle: the two
+// 64-column panels are kChunkBytes apart (LBO), 8-key groups 1024 bytes (SBO);
+// kk selects keys [16kk, 16kk+16).
+__device__ __forceinline__ uint64_t mnmajor_desc(uint32_t tile_base, int kk) {
+  return make_sdesc(tile_base + kk * 2048, kChunkBytes, 1024);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
+                      const __grid_constant__ CUtensorMap tm_k,
+                      const __grid_constant__ CUtensorMap tm_v, const FwdArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  Barriers* bars = reinterpret_cast<Barriers*>(smem + kOffBar);
+  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + kOffTmem);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffAbort);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const WaitCtx wc{abort_flag, a.status, kStatusTimeoutFwd};
+
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    mbar_init(smem_u32(&bars->q_full), 1);
+    mbar_init(smem_u32(&bars->q_empty), 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(smem_u32(&bars->k_full[s]), 1);
+      mbar_init(smem_u32(&bars->k_empty[s]), 1);
+      mbar_init(smem_u32(&bars->v_full[s]), 1);
+      mbar_init(smem_u32(&bars->v_empty[s]), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&bars->s_full[i]), 1);
+      mbar_init(smem_u32(&bars->p_full[i]), 4);
+      mbar_init(smem_u32(&bars->pv_done[i]), 1);
+      mbar_init(smem_u32(&bars->o_full[i]), 1);
+      mbar_init(smem_u32(&bars->o_empty[i]), 4);
+    }
+    mbar_init(smem_u32(&bars->drain), 1);
+    fence_mbar_init();
+  }
+  if (warp == kWarpMma) {
+    tmem_alloc(smem_u32((const void*)tmem_slot), 512);
+    tmem_relinquish();
+  }
+  if (warp == kWarpTma && lane == 0) {
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int n_items = min(*a.n_items, a.max_items);
+
+  if (warp == kWarpTma) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      uint32_t kv_iter = 0, item_count = 0, q_arm = 0, k_arm[kStages] = {}, v_arm[kStages] = {};
+      bool ok = true;
+      for (int idx = blockIdx.x; idx < n_items && ok; idx += gridDim.x) {
+        const Item it = decode(a, idx);
+        if (item_count > 0) ok = mbar_wait(smem_u32(&bars->q_empty), (item_count - 1) & 1, wc);
+        if (!ok) break;
+        const uint32_t qf = smem_u32(&bars->q_full);
+        mbar_arrive_expect_tx(qf, 2 * kTileBytes);
+        ++q_arm;
+        for (int i = 0; i < 2; ++i)
+          for (int c = 0; c < 2; ++c)
+            tma_load_3d(sbase + kOffQ + i * kTileBytes + c * kChunkBytes, &tm_q, qf, c * 64,
+                        it.g * a.G, it.q0 + i * a.R);
+        for (int n = 0; n < it.ntiles && ok; ++n, ++kv_iter) {
+          const int ks = it.kend - kTileKeys * (n + 1);
+          const uint32_t s = kv_iter % kStages, ph = (kv_iter / kStages) & 1;
+          if (kv_iter >= kStages) ok = mbar_wait(smem_u32(&bars->k_empty[s]), ph ^ 1, wc);
+          if (!ok) break;
+          const uint32_t kf = smem_u32(&bars->k_full[s]);
+          mbar_arrive_expect_tx(kf, kTileBytes);
+          ++k_arm[s];
+          for (int c = 0; c < 2; ++c)
+            tma_load_3d(sbase + kOffK + s * kTileBytes + c * kChunkBytes, &tm_k, kf, c * 64, it.g,
+                        ks);
+          if (kv_iter >= kStages) ok = mbar_wait(smem_u32(&bars->v_empty[s]), ph ^ 1, wc);
+          if (!ok) break;
+          const uint32_t vf = smem_u32(&bars->v_full[s]);
+          mbar_arrive_expect_tx(vf, kTileBytes);
+          ++v_arm[s];
+          for (int c = 0; c < 2; ++c)
+            tma_load_3d(sbase + kOffV + s * kTileBytes + c * kChunkBytes, &tm_v, vf, c * 64, it.g,
+                        ks);
+        }
+        ++item_count;
+      }
+      // Every copy this thread started has landed before the CTA can exit
+      // (immediate on the normal path: the consumer already saw each one).
+      volatile int no_abort = 0;
+      const WaitCtx drain{&no_abort, a.status, kStatusTimeoutFwd};
+      if (q_arm) mbar_wait(smem_u32(&bars->q_full), (q_arm - 1) & 1, drain);
+      for (int s = 0; s < kStages; ++s) {
+        if (k_arm[s]) mbar_wait(smem_u32(&bars->k_full[s]), (k_arm[s] - 1) & 1, drain);
+        if (v_arm[s]) mbar_wait(smem_u32(&bars->v_full[s]), (v_arm[s] - 1) & 1, drain);
+      }
+    }
+  } else if (warp == kWarpMma) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc_qk = make_idesc_bf16(128, 128, 0, 0);
+      const uint32_t idesc_pv = make_idesc_bf16(128, 128, 0, 1);
+      uint32_t kv_iter = 0, item_count = 0, pv_count[2] = {0, 0}, p_count[2] = {0, 0};
+      bool ok = true;
+      for (int idx = blockIdx.x; idx < n_items && ok; idx += gridDim.x) {
+        const Item it = decode(a, idx);
+        ok = mbar_wait(smem_u32(&bars->q_full), item_count & 1, wc);
+        if (!ok) break;
+        tc_fence_after();
+        for (int n = 0; n < it.ntiles && ok; ++n, ++kv_iter) {
+          const uint32_t s = kv_iter % kStages, ph = (kv_iter / kStages) & 1;
+          ok = mbar_wait(smem_u32(&bars->k_full[s]), ph, wc);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t kt = sbase + kOffK + s * kTileBytes;
+          for (int i = 0; i < 2 && ok; ++i) {
+            if (pv_count[i] > 0) {
+              ok = mbar_wait(smem_u32(&bars->pv_done[i]), (pv_count[i] - 1) & 1, wc);
+              if (!ok) break;
+              tc_fence_after();
+            }
+            const uint32_t qt = sbase + kOffQ + i * kTileBytes;
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+              mma_ss(tmem + i * 128, kmajor_desc(qt, kk), kmajor_desc(kt, kk), idesc_qk, kk > 0);
+            mma_commit(smem_u32(&bars->s_full[i]));
+          }
+          if (!ok) break;
+          mma_commit(smem_u32(&bars->k_empty[s]));
+          if (n == it.ntiles - 1) mma_commit(smem_u32(&bars->q_empty));
+          ok = mbar_wait(smem_u32(&bars->v_full[s]), ph, wc);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t vt = sbase + kOffV + s * kTileBytes;
+          for (int i = 0; i < 2 && ok; ++i) {
+            ok = mbar_wait(smem_u32(&bars->p_full[i]), p_count[i] & 1, wc);
+            ++p_count[i];
+            if (!ok) break;
+            if (n == 0 && item_count > 0) {
+              ok = mbar_wait(smem_u32(&bars->o_empty[i]), (item_count - 1) & 1, wc);
+              if (!ok) break;
+            }
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+              mma_ts(tmem + 256 + i * 128, tmem + i * 128 + kk * 8, mnmajor_desc(vt, kk),
+                     idesc_pv, (n > 0 || kk > 0) ? 1u : 0u);
+            mma_commit(smem_u32(&bars->pv_done[i]));
+            ++pv_count[i];
+            if (n == it.ntiles - 1) mma_commit(smem_u32(&bars->o_full[i]));
+          }
+          if (!ok) break;
+          mma_commit(smem_u32(&bars->v_empty[s]));
+        }
+        ++item_count;
+      }
+      // Every MMA this thread issued has finished before TMEM is released.
+      mma_commit(smem_u32(&bars->drain));
+      volatile int no_abort = 0;
+      const WaitCtx drain{&no_abort, a.status, kStatusTimeoutFwd};
+      mbar_wait(smem_u32(&bars->drain), 0, drain);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax + epilogue
+    const int i = warp >> 2;               // which query tile of the pair
+    const int wq = warp & 3;               // TMEM lane quarter
+    const int r = wq * 32 + lane;          // row of the tile = TMEM lane
+    const uint32_t t_row = tmem + ((uint32_t)(wq * 32) << 16);
+    const uint32_t s_col = i * 128, o_col = 256 + i * 128;
+    uint32_t s_count = 0, item_count = 0;
+    bool ok = true;
+    for (int idx = blockIdx.x; idx < n_items && ok; idx += gridDim.x) {
+      const Item it = decode(a, idx);
+      const int tok = it.q0 + i * a.R + r / a.G;
+      const int h = it.g * a.G + r % a.G;
+      const bool valid = tok < it.d1;
+      const int lo_r = a.W > 0 ? max(it.d0, tok - a.W + 1) : it.d0;
+      const float sink2 = __ldg(a.sink + h) * kLog2e;
+      float m = sink2;                     // running max (log2 units)
+      float l = 1.f;                       // running sum, sink included
+      for (int n = 0; n < it.ntiles; ++n) {
+        const int ks = it.kend - kTileKeys * (n + 1);
+        ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->s_full[i]), s_count & 1, wc));
+        ++s_count;
+        if (!ok) break;
+        tc_fence_after();
+        float sv[128];
+        {
+          uint32_t u0[32], u1[32], u2[32], u3[32];
+          tmem_ld32(t_row + s_col + 0, u0);
+          tmem_ld32(t_row + s_col + 32, u1);
+          tmem_ld32(t_row + s_col + 64, u2);
+          tmem_ld32(t_row + s_col + 96, u3);
+          tc_wait_ld_dep(u0);
+          tc_wait_ld_dep(u1);
+          tc_wait_ld_dep(u2);
+          tc_wait_ld_dep(u3);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            sv[e] = __uint_as_float(u0[e]);
+            sv[32 + e] = __uint_as_float(u1[e]);
+            sv[64 + e] = __uint_as_float(u2[e]);
+            sv[96 + e] = __uint_as_float(u3[e]);
+          }
+        }
+        const bool needs_mask = (ks + kTileKeys - 1 > it.q0) || (ks < it.d0) ||
+                                (a.W > 0 && ks < it.q0 + 2 * a.R - a.W);
+        if (needs_mask) {
+          const int c_lo = lo_r - ks, c_hi = tok - ks;
+#pragma unroll
+          for (int c = 0; c < 128; ++c)
+            if (c < c_lo || c > c_hi) sv[c] = -INFINITY;
+        }
+        float mx = sv[0];
+#pragma unroll
+        for (int c = 1; c < 128; ++c) mx = fmaxf(mx, sv[c]);
+        const float m_tile = mx * a.scale_log2;
+        float alpha = 1.f;
+        bool rescale_o = false;
+        if (n == 0) {
+          if (m_tile > m) { alpha = ex2_approx(m - m_tile); m = m_tile; }
+        } else if (m_tile > m + kRescaleThreshold) {
+          alpha = ex2_approx(m - m_tile);
+          m = m_tile;
+          rescale_o = true;
+        }
+        l *= alpha;
+        if (__any_sync(0xffffffffu, rescale_o)) {
+          // PV of the previous tile has completed (it was issued before this
+          // tile's QK, whose completion was just observed), so O is stable.
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint32_t u[32];
+            tmem_ld32(t_row + o_col + c * 32, u);
+            tc_wait_ld_dep(u);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) u[e] = __float_as_uint(__uint_as_float(u[e]) * alpha);
+            tmem_st32(t_row + o_col + c * 32, u);
+          }
+        }
+        const float mb = (m == -INFINITY) ? 0.f : m;
+        float rs = 0.f;
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          uint32_t pk[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const float p0 = ex2_approx(fmaf(sv[hf * 64 + 2 * e], a.scale_log2, -mb));
+            const float p1 = ex2_approx(fmaf(sv[hf * 64 + 2 * e + 1], a.scale_log2, -mb));
+            rs += p0 + p1;
+            pk[e] = pack_bf16x2(p0, p1);
+          }
+          tmem_st32(t_row + s_col + hf * 32, pk);
+        }
+        l += rs;
+        tc_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&bars->p_full[i]));
+      }
+      if (!ok) break;
+      // epilogue: O / l -> bf16, LSE
+      ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->o_full[i]), item_count & 1, wc));
+      if (!ok) break;
+      tc_fence_after();
+      const float inv_l = 1.f / l;
+      __nv_bfloat16* orow = a.out + ((size_t)tok * a.H + h) * kHeadDim;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t u[32];
+        tmem_ld32(t_row + o_col + c * 32, u);
+        tc_wait_ld_dep(u);
+        if (c == 3) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(smem_u32(&bars->o_empty[i]));
+        }
+        if (valid) {
+#pragma unroll
+          for (int v4 = 0; v4 < 4; ++v4) {
+            uint4 pk;
+            pk.x = pack_bf16x2(__uint_as_float(u[v4 * 8 + 0]) * inv_l, __uint_as_float(u[v4 * 8 + 1]) * inv_l);
+            pk.y = pack_bf16x2(__uint_as_float(u[v4 * 8 + 2]) * inv_l, __uint_as_float(u[v4 * 8 + 3]) * inv_l);
+            pk.z = pack_bf16x2(__uint_as_float(u[v4 * 8 + 4]) * inv_l, __uint_as_float(u[v4 * 8 + 5]) * inv_l);
+            pk.w = pack_bf16x2(__uint_as_float(u[v4 * 8 + 6]) * inv_l, __uint_as_float(u[v4 * 8 + 7]) * inv_l);
+            *reinterpret_cast<uint4*>(orow + c * 32 + v4 * 8) = pk;
+          }
+        }
+      }
+      if (valid) a.lse[(size_t)h * a.T + tok] = (m + log2f(l)) * kLn2;
+      ++item_count;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == kWarpMma) tmem_dealloc(tmem, 512);
+}
+
+}  // namespace
+
+cudaError_t launch_attn_fwd_sm100_impl(const CUtensorMap& tq, const CUtensorMap& tk,
+                                       const CUtensorMap& tv, const Resolved& p, const float* sink,
+                                       const int4* items, const int* n_items, int max_items,
+                                       void* out, float* lse, int* status, int num_sms,
+                                       cudaStream_t st) {
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(attn_fwd_sm100_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  FwdArgs a;
+  a.T = p.T; a.H = p.H; a.Hk = p.Hk; a.G = p.G; a.R = p.R; a.W = p.W;
+  a.scale_log2 = p.scale * kLog2e;
+  a.sink = sink; a.items = items; a.n_items = n_items; a.max_items = max_items;
+  a.out = reinterpret_cast<__nv_bfloat16*>(out);
+  a.lse = lse;
+  a.status = status;
+  int grid = num_sms;
+  if (grid > max_items) grid = max_items;
+  if (grid < 1) grid = 1;
+  attn_fwd_sm100_kernel<<<grid, kThreads, kSmemBytes, st>>>(tq, tk, tv, a);
+  return cudaGetLastError();
+}
+
+}  // namespace flint

@@ -1,0 +1,92 @@
+// bwd_preprocess.cu - per-row D_i = dO_i . O_i and the sink-logit gradient.
+//
+// The sink is a softmax category with a zero value (Flint layers page,
+// nemo_automodel.components.models.flint.layers, FlintAttention.forward and
+// _FlintSinkParameters.forward), so with p_sink_i = e^{s_h - LSE_i}:
+//   d s_h = sum_i p_sink_i (0 - dO_i . O_i) = -sum_i e^{s_h - LSE_i} D_i.
+// One 16-lane half-warp reduces one (token, head) row with warp shuffles; the
+// sink sum is kept per half-warp and per head in shared memory (no atomics),
+// summed per block in a fixed order, and the per-block partials are summed in a
+// fixed order by a second tiny launch, so the result is deterministic.
+#include "common.cuh"
+
+namespace flint {
+
+cudaError_t launch_reduce_rows(const float* part, int nrows, int width, float* out,
+                               cudaStream_t st);
+
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kGroups = kThreads / 16;
+constexpr int kTok = 4;
+
+template <typename T>
+__global__ void __launch_bounds__(kThreads)
+bwd_pre_kernel(const T* __restrict__ out, const T* __restrict__ dout,
+               const float* __restrict__ lse, const float* __restrict__ sink,
+               float* __restrict__ dvec, float* __restrict__ part, int ntok, int H) {
+  extern __shared__ float acc[];   // [kGroups][H]
+  const int lane16 = threadIdx.x & 15, grp = threadIdx.x >> 4;
+  const int c0 = lane16 * 8;
+  for (int e = threadIdx.x; e < kGroups * H; e += kThreads) acc[e] = 0.f;
+  __syncthreads();
+  const int rows = kTok * H;
+  const int iters = (rows + kGroups - 1) / kGroups;
+  for (int t0 = blockIdx.x * kTok; t0 < ntok; t0 += gridDim.x * kTok) {
+    for (int it = 0; it < iters; ++it) {
+      const int rr = grp + it * kGroups;
+      const int t = t0 + rr / H, h = rr % H;
+      const bool valid = rr < rows && t < ntok;
+      float a[8], b[8];
+      if (valid) {
+        const size_t base = ((size_t)t * H + h) * kHeadDim + c0;
+        load8(out + base, a);
+        load8(dout + base, b);
+      } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) { a[e] = 0.f; b[e] = 0.f; }
+      }
+      float d = 0.f;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) d = fmaf(a[e], b[e], d);
+#pragma unroll
+      for (int o = 8; o >= 1; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
+      if (valid && lane16 == 0) {
+        dvec[(size_t)h * ntok + t] = d;
+        acc[grp * H + h] -= expf(sink[h] - lse[(size_t)h * ntok + t]) * d;
+      }
+    }
+  }
+  __syncthreads();
+  for (int h = threadIdx.x; h < H; h += kThreads) {
+    float s = 0.f;
+    for (int g = 0; g < kGroups; ++g) s += acc[g * H + h];
+    part[(size_t)blockIdx.x * H + h] = s;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_bwd_preprocess(const Resolved& p, const void* out, const void* dout,
+                                  const float* lse, const float* sink, float* dvec, float* part,
+                                  float* dsink, cudaStream_t st) {
+  if (p.T == 0) {
+    cudaMemsetAsync(dsink, 0, p.H * sizeof(float), st);
+    return cudaGetLastError();
+  }
+  int blocks = (p.T + kTok - 1) / kTok;
+  if (blocks > kPartBlocks) blocks = kPartBlocks;
+  const size_t smem = (size_t)kGroups * p.H * sizeof(float);
+  if (p.dtype == FLINT_BF16)
+    bwd_pre_kernel<__nv_bfloat16><<<blocks, kThreads, smem, st>>>(
+        (const __nv_bfloat16*)out, (const __nv_bfloat16*)dout, lse, sink, dvec, part, p.T, p.H);
+  else
+    bwd_pre_kernel<float><<<blocks, kThreads, smem, st>>>((const float*)out, (const float*)dout,
+                                                          lse, sink, dvec, part, p.T, p.H);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  return launch_reduce_rows(part, blocks, p.H, dsink, st);
+}
+
+}  // namespace flint

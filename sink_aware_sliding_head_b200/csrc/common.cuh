@@ -1,0 +1,168 @@
+// common.cuh - internal definitions shared by the library's kernels and its
+// C-ABI layer: resolved parameters, workspace layout, status bits, and small
+// device helpers (document lookup, bf16/fp32 loads and stores).
+#pragma once
+#include <cstddef>
+#include <cstdint>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "../../include/flint_attn.h"
+
+namespace flint {
+
+constexpr int kHeadDim = 128;
+constexpr int kTileRows = 128;   // query rows per tensor-core tile (tokens x heads-of-group)
+constexpr int kTileKeys = 128;   // keys per tensor-core tile
+
+// Status bits written into the workspace's status word by bounded device waits.
+enum : int {
+  kStatusTimeoutFwd = 1,
+  kStatusTimeoutBwdKV = 2,
+  kStatusTimeoutBwdQ = 4,
+};
+
+// Parameters after validation and defaulting.
+struct Resolved {
+  int T, N, H, Hk, D, G, W, rope;
+  float theta, eps, scale;
+  int dtype;
+  int R;            // tokens per 128-row tile = 128 / G
+};
+
+// Offsets (bytes) of every region of the workspace. All regions are 256-byte aligned.
+struct WsLayout {
+  size_t status;        // int[64]: [0] status bits, [1..3] work-list lengths
+  size_t qhat, khat;    // normalised+rotated q [T,H,D], k [T,Hk,D] (dtype)
+  size_t items_q;       // int4 work items, query-major (forward: pairs of tiles)
+  size_t items_q1;      // int4 work items, query-major single tiles (backward dQ)
+  size_t items_kv;      // int4 work items, key-major (backward dK/dV)
+  size_t sched_tmp;     // int4 + int per item, scratch for the LPT sort
+  size_t dvec;          // [H,T] fp32 rowsum(dO * O)      (backward)
+  size_t part;          // fp32 partial sums (d sink, d norm weights)
+  size_t dq_acc;        // [T,H,D] fp32 gradient w.r.t. q_hat (backward)
+  size_t dk_acc;        // [T,Hk,D] fp32 gradient w.r.t. k_hat (backward)
+  size_t total;
+  int max_items_q, max_items_q1, max_items_kv, max_items_any;
+  int part_blocks;      // number of partial-sum rows per reduced quantity
+};
+
+__host__ __device__ inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+inline int elem_bytes(int dtype) { return dtype == FLINT_BF16 ? 2 : 4; }
+
+constexpr int kPartBlocks = 1184;   // 148 SMs x 8: rows of partial sums for reductions
+
+inline WsLayout make_layout(const Resolved& p, bool backward) {
+  WsLayout L{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) { size_t o = off; off = align256(off + bytes); return o; };
+  const size_t eb = elem_bytes(p.dtype);
+  L.status = take(64 * sizeof(int));
+  L.qhat = take((size_t)p.T * p.H * p.D * eb);
+  L.khat = take((size_t)p.T * p.Hk * p.D * eb);
+  L.max_items_q = p.Hk * ((p.T + 2 * p.R - 1) / (2 * p.R) + p.N);
+  L.max_items_q1 = p.Hk * ((p.T + p.R - 1) / p.R + p.N);
+  L.max_items_kv = p.Hk * ((p.T + kTileKeys - 1) / kTileKeys + p.N);
+  L.max_items_any = L.max_items_q1;
+  if (L.max_items_q > L.max_items_any) L.max_items_any = L.max_items_q;
+  if (L.max_items_kv > L.max_items_any) L.max_items_any = L.max_items_kv;
+  L.items_q = take((size_t)L.max_items_q * 16);
+  L.items_q1 = backward ? take((size_t)L.max_items_q1 * 16) : off;
+  L.items_kv = backward ? take((size_t)L.max_items_kv * 16) : off;
+  L.sched_tmp = take((size_t)L.max_items_any * 20);
+  L.part_blocks = kPartBlocks;
+  if (backward) {
+    L.dvec = take((size_t)p.H * p.T * 4);
+    L.part = take((size_t)kPartBlocks * (p.H + 2 * p.D) * 4);
+    L.dq_acc = take((size_t)p.T * p.H * p.D * 4);
+    L.dk_acc = take((size_t)p.T * p.Hk * p.D * 4);
+  }
+  L.total = off;
+  return L;
+}
+
+// ------------------------------------------------------------------ device helpers
+
+// Index of the document that holds token t (cu non-decreasing, cu[0] = 0,
+// cu[N] = T, t < T). Empty documents are skipped.
+__device__ __forceinline__ int doc_of(const int32_t* __restrict__ cu, int N, int t) {
+  int lo = 0, hi = N;           // invariant: cu[lo] <= t < cu[hi]
+  while (hi - lo > 1) {
+    int mid = (lo + hi) >> 1;
+    if (__ldg(cu + mid) <= t) lo = mid; else hi = mid;
+  }
+  return lo;
+}
+
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+  return __float2bfloat16_rn(x);
+}
+
+// 8 consecutive elements <-> 8 floats (16-byte loads for bf16, 2 x 16 bytes for fp32).
+__device__ __forceinline__ void load8(const __nv_bfloat16* p, float (&f)[8]) {
+  uint4 u = *reinterpret_cast<const uint4*>(p);
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float2 t = __bfloat1622float2(h[i]);
+    f[2 * i] = t.x;
+    f[2 * i + 1] = t.y;
+  }
+}
+__device__ __forceinline__ void load8(const float* p, float (&f)[8]) {
+  float4 a = *reinterpret_cast<const float4*>(p);
+  float4 b = *reinterpret_cast<const float4*>(p + 4);
+  f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
+  f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+}
+__device__ __forceinline__ void store8(__nv_bfloat16* p, const float (&f)[8]) {
+  uint4 u;
+  __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(f[2 * i], f[2 * i + 1]);
+  *reinterpret_cast<uint4*>(p) = u;
+}
+__device__ __forceinline__ void store8(float* p, const float (&f)[8]) {
+  *reinterpret_cast<float4*>(p) = make_float4(f[0], f[1], f[2], f[3]);
+  *reinterpret_cast<float4*>(p + 4) = make_float4(f[4], f[5], f[6], f[7]);
+}
+
+// ------------------------------------------------------------------ launchers
+// (defined in the .cu files; all return cudaGetLastError() of their launch)
+cudaError_t launch_build_worklist(const int32_t* cu, const Resolved& p, int mode, int span,
+                                  int4* items, int* count, void* tmp, int max_items,
+                                  cudaStream_t st);
+cudaError_t launch_prologue(const Resolved& p, const void* x, const void* w, void* y, int heads,
+                            const int32_t* cu, cudaStream_t st);
+cudaError_t launch_attn_fwd_fp32(const Resolved& p, const float* qh, const float* kh,
+                                 const float* v, const float* sink, const int32_t* cu, float* out,
+                                 float* lse, cudaStream_t st);
+cudaError_t launch_attn_bwd_fp32(const Resolved& p, const float* qh, const float* kh,
+                                 const float* v, const float* dout, const float* lse,
+                                 const float* dvec, const int32_t* cu, float* dq_acc,
+                                 float* dk_acc, float* dv, cudaStream_t st);
+cudaError_t launch_bwd_preprocess(const Resolved& p, const void* out, const void* dout,
+                                  const float* lse, const float* sink, float* dvec, float* part,
+                                  float* dsink, cudaStream_t st);
+cudaError_t launch_bwd_epilogue(const Resolved& p, const void* x, const void* w,
+                                const float* g_hat, void* dx, float* dw, float* part, int heads,
+                                const int32_t* cu, cudaStream_t st);
+cudaError_t launch_attn_fwd_sm100(const Resolved& p, const void* qh, const void* kh,
+                                  const void* v, const float* sink, const int4* items,
+                                  const int* n_items, int max_items, void* out, float* lse,
+                                  int* status, int num_sms, cudaStream_t st);
+cudaError_t launch_attn_bwd_sm100(const Resolved& p, const void* qh, const void* kh,
+                                  const void* v, const void* dout, const float* lse,
+                                  const float* dvec, const int4* items_kv, const int* n_kv,
+                                  int max_kv, const int4* items_q, const int* n_q, int max_q,
+                                  float* dq_acc, float* dk_acc, void* dv, int* status,
+                                  int num_sms, cudaStream_t st);
+
+enum { kModeQuery = 0, kModeKey = 1 };
+
+}  // namespace flint

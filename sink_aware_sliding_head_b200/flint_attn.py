@@ -1,0 +1,186 @@
+"""Python binding of the C ABI in ``include/flint_attn.h`` (ctypes).
+
+Argument marshalling only: tensors are allocated with torch on the current CUDA
+device and passed as raw device pointers together with torch's current stream.
+Every step of the computation runs in the library's CUDA kernels. There is no
+CPU or PyTorch fallback: if the library is missing or a call fails, an error is
+raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libflint_attn.so")
+
+FLINT_BF16 = 0
+FLINT_FP32 = 1
+
+STATUS = {0: "FLINT_OK", 1: "FLINT_ERR_INVALID_ARG", 2: "FLINT_ERR_UNSUPPORTED",
+          3: "FLINT_ERR_WORKSPACE", 4: "FLINT_ERR_CUDA", 5: "FLINT_ERR_TIMEOUT"}
+
+EXPORTED = ["flint_attn_workspace_bytes", "flint_attn_fwd", "flint_attn_bwd",
+            "flint_attn_check_status", "flint_status_string", "flint_attn_version"]
+
+
+class Params(ctypes.Structure):
+    """Mirror of ``flint_attn_params_t``."""
+    _fields_ = [
+        ("total_tokens", ctypes.c_int32),
+        ("num_docs", ctypes.c_int32),
+        ("num_q_heads", ctypes.c_int32),
+        ("num_kv_heads", ctypes.c_int32),
+        ("head_dim", ctypes.c_int32),
+        ("window", ctypes.c_int32),
+        ("use_rope", ctypes.c_int32),
+        ("rope_theta", ctypes.c_float),
+        ("rms_eps", ctypes.c_float),
+        ("softmax_scale", ctypes.c_float),
+        ("dtype", ctypes.c_int32),
+    ]
+
+
+class FlintError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        super().__init__(f"{where}: {STATUS.get(code, code)}")
+        self.code = code
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH):
+    """Load (once) and return the ctypes handle; raises if the library is missing."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise ImportError(f"CUDA library not built: {path} (run python -m "
+                          "sink_aware_sliding_head_b200.build)")
+    lib = ctypes.CDLL(path)
+    vp, sz = ctypes.c_void_p, ctypes.c_size_t
+    P = ctypes.POINTER(Params)
+    lib.flint_attn_workspace_bytes.argtypes = [P, ctypes.c_int]
+    lib.flint_attn_workspace_bytes.restype = sz
+    lib.flint_attn_fwd.argtypes = [P] + [vp] * 9 + [vp, sz, vp]
+    lib.flint_attn_fwd.restype = ctypes.c_int
+    lib.flint_attn_bwd.argtypes = [P] + [vp] * 16 + [vp, sz, vp]
+    lib.flint_attn_bwd.restype = ctypes.c_int
+    lib.flint_attn_check_status.argtypes = [vp, vp]
+    lib.flint_attn_check_status.restype = ctypes.c_int
+    lib.flint_status_string.argtypes = [ctypes.c_int]
+    lib.flint_status_string.restype = ctypes.c_char_p
+    lib.flint_attn_version.argtypes = []
+    lib.flint_attn_version.restype = ctypes.c_char_p
+    _lib = lib
+    return lib
+
+
+def make_params(total_tokens, num_docs, num_q_heads, num_kv_heads, window, use_rope,
+                rope_theta, dtype, head_dim=128, rms_eps=1e-6, softmax_scale=0.0) -> Params:
+    return Params(int(total_tokens), int(num_docs), int(num_q_heads), int(num_kv_heads),
+                  int(head_dim), int(window), 1 if use_rope else 0, float(rope_theta),
+                  float(rms_eps), float(softmax_scale), int(dtype))
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return FLINT_BF16
+    if t.dtype == torch.float32:
+        return FLINT_FP32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _stream_ptr(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(code: int, where: str):
+    if code != 0:
+        raise FlintError(code, where)
+
+
+def params_for(q, k, cu_doc_lens, window, use_rope, rope_theta, rms_eps=1e-6,
+               softmax_scale=0.0) -> Params:
+    T, H, D = q.shape
+    return make_params(T, cu_doc_lens.numel() - 1, H, k.shape[1], window, use_rope, rope_theta,
+                       _dtype_code(q), head_dim=D, rms_eps=rms_eps, softmax_scale=softmax_scale)
+
+
+def workspace_bytes(params: Params, backward: bool) -> int:
+    return int(load_library().flint_attn_workspace_bytes(ctypes.byref(params), int(backward)))
+
+
+def alloc_workspace(params: Params, backward: bool, device=None) -> torch.Tensor:
+    n = workspace_bytes(params, backward)
+    if n == 0:
+        raise FlintError(1, "flint_attn_workspace_bytes")
+    return torch.empty(n, dtype=torch.uint8, device=device or "cuda")
+
+
+def fwd(q, k, v, q_norm_w, k_norm_w, sink, cu_doc_lens, window, use_rope, rope_theta,
+        rms_eps=1e-6, softmax_scale=0.0, out=None, lse=None, workspace=None, stream=None,
+        check_status=False):
+    """Forward through ``flint_attn_fwd``. Returns (out [T,H,D], lse [H,T] fp32)."""
+    lib = load_library()
+    p = params_for(q, k, cu_doc_lens, window, use_rope, rope_theta, rms_eps, softmax_scale)
+    T, H, D = q.shape
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty(H, T, dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = alloc_workspace(p, False, q.device)
+    st = _stream_ptr(stream)
+    code = lib.flint_attn_fwd(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(q_norm_w),
+                              _ptr(k_norm_w), _ptr(sink), _ptr(cu_doc_lens), _ptr(out), _ptr(lse),
+                              _ptr(workspace), workspace.numel(), st)
+    _check(code, "flint_attn_fwd")
+    if check_status:
+        _check(lib.flint_attn_check_status(_ptr(workspace), st), "flint_attn_fwd (device)")
+    return out, lse
+
+
+def bwd(q, k, v, q_norm_w, k_norm_w, sink, cu_doc_lens, out, lse, dout, window, use_rope,
+        rope_theta, rms_eps=1e-6, softmax_scale=0.0, grads=None, workspace=None, stream=None,
+        check_status=False):
+    """Backward through ``flint_attn_bwd``.
+
+    Returns a dict with dq, dk, dv (input dtype), dw_q, dw_k, dsink (fp32).
+    """
+    lib = load_library()
+    p = params_for(q, k, cu_doc_lens, window, use_rope, rope_theta, rms_eps, softmax_scale)
+    T, H, D = q.shape
+    if grads is None:
+        grads = {
+            "dq": torch.empty_like(q), "dk": torch.empty_like(k), "dv": torch.empty_like(v),
+            "dw_q": torch.empty(D, dtype=torch.float32, device=q.device),
+            "dw_k": torch.empty(D, dtype=torch.float32, device=q.device),
+            "dsink": torch.empty(H, dtype=torch.float32, device=q.device),
+        }
+    if workspace is None:
+        workspace = alloc_workspace(p, True, q.device)
+    st = _stream_ptr(stream)
+    code = lib.flint_attn_bwd(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(q_norm_w),
+                              _ptr(k_norm_w), _ptr(sink), _ptr(cu_doc_lens), _ptr(out), _ptr(lse),
+                              _ptr(dout), _ptr(grads["dq"]), _ptr(grads["dk"]), _ptr(grads["dv"]),
+                              _ptr(grads["dw_q"]), _ptr(grads["dw_k"]), _ptr(grads["dsink"]),
+                              _ptr(workspace), workspace.numel(), st)
+    _check(code, "flint_attn_bwd")
+    if check_status:
+        _check(lib.flint_attn_check_status(_ptr(workspace), st), "flint_attn_bwd (device)")
+    return grads
+
+
+def version() -> str:
+    return load_library().flint_attn_version().decode()

@@ -1,0 +1,48 @@
+"""Helpers shared by the GPU parity tests: run the library, compare with the oracle."""
+import numpy as np
+import torch
+
+# Tolerances of the parity bar: FP32 inputs max-abs 1e-4; BF16 inputs max-abs
+# 2e-2 and relative RMS 1e-2.
+FP32_MAX_ABS = 1e-4
+BF16_MAX_ABS = 2e-2
+BF16_REL_RMS = 1e-2
+
+
+def to_dev(inp, device="cuda"):
+    out = {}
+    for k, v in inp.items():
+        out[k] = v.to(device) if torch.is_tensor(v) else v
+    return out
+
+
+def f64(t):
+    return t.detach().to("cpu").double().numpy() if torch.is_tensor(t) else np.asarray(t, np.float64)
+
+
+def compare(gpu, ref, dtype, name=""):
+    """Assert the parity bar; returns (max_abs, rel_rms)."""
+    g = f64(gpu)
+    r = np.asarray(ref, dtype=np.float64)
+    assert g.shape == r.shape, (name, g.shape, r.shape)
+    assert np.all(np.isfinite(g)), f"{name}: non-finite GPU values"
+    err = g - r
+    max_abs = float(np.max(np.abs(err))) if err.size else 0.0
+    denom = float(np.sqrt(np.mean(r * r))) if r.size else 1.0
+    rel_rms = float(np.sqrt(np.mean(err * err)) / denom) if r.size and denom > 0 else 0.0
+    if dtype == "fp32":
+        assert max_abs <= FP32_MAX_ABS, f"{name}: max_abs {max_abs:.3e}"
+    else:
+        assert max_abs <= BF16_MAX_ABS, f"{name}: max_abs {max_abs:.3e}"
+        assert rel_rms <= BF16_REL_RMS, f"{name}: rel_rms {rel_rms:.3e}"
+    return max_abs, rel_rms
+
+
+def run_fwd(fa, d, window, rope, theta, check=True):
+    return fa.fwd(d["q"], d["k"], d["v"], d["w_q"], d["w_k"], d["sink"], d["cu_doc_lens"],
+                  window, rope, theta, check_status=check)
+
+
+def run_bwd(fa, d, out, lse, window, rope, theta, check=True):
+    return fa.bwd(d["q"], d["k"], d["v"], d["w_q"], d["w_k"], d["sink"], d["cu_doc_lens"],
+                  out, lse, d["dout"], window, rope, theta, check_status=check)

@@ -1,0 +1,84 @@
+"""The C-ABI library loads, exports every declared symbol, and rejects bad
+arguments before any CUDA call (these run without a GPU)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from sink_aware_sliding_head_b200 import build as build_mod
+from sink_aware_sliding_head_b200 import flint_attn as fa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build_mod.build()
+    return fa.load_library()
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "flint_attn.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(flint_\w+)\s*\(", src)))
+
+
+def test_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    assert set(names) == set(fa.EXPORTED)
+    for n in names:
+        assert hasattr(lib, n), n
+    out = os.popen(f"nm -D --defined-only {fa.LIB_PATH}").read()
+    for n in names:
+        assert re.search(rf"\bT {n}\b", out), n
+
+
+def test_version_and_status_strings(lib):
+    assert "sm_100a" in fa.version()
+    for code in range(6):
+        assert lib.flint_status_string(code)
+
+
+def params(**kw):
+    d = dict(total_tokens=256, num_docs=1, num_q_heads=32, num_kv_heads=4, window=0,
+             use_rope=False, rope_theta=1e6, dtype=fa.FLINT_BF16)
+    d.update(kw)
+    return fa.make_params(**d)
+
+
+def test_workspace_bytes(lib):
+    n_fwd = fa.workspace_bytes(params(), False)
+    n_bwd = fa.workspace_bytes(params(), True)
+    # q_hat + k_hat at least, backward adds fp32 gradient accumulators
+    assert n_fwd >= 256 * (32 + 4) * 128 * 2
+    assert n_bwd >= n_fwd + 256 * (32 + 4) * 128 * 4
+    assert fa.workspace_bytes(params(head_dim=64), False) == 0
+    assert fa.workspace_bytes(params(num_q_heads=30), False) == 0
+
+
+def _fwd(lib, p, ptr=0x1000, ws=0x100000, ws_bytes=1 << 40):
+    P = ctypes.c_void_p
+    return lib.flint_attn_fwd(ctypes.byref(p), P(ptr), P(ptr), P(ptr), P(ptr), P(ptr), P(ptr),
+                              P(ptr), P(ptr), P(ptr), P(ws), ws_bytes, None)
+
+
+def test_argument_errors_return_before_any_launch(lib):
+    assert _fwd(lib, params(head_dim=64)) == 2              # FLINT_ERR_UNSUPPORTED
+    assert _fwd(lib, params(num_q_heads=12, num_kv_heads=1)) == 2   # G = 12
+    assert _fwd(lib, params(num_q_heads=30)) == 1           # H % Hk != 0
+    assert _fwd(lib, params(num_docs=0)) == 1
+    assert _fwd(lib, params(total_tokens=-1)) == 1
+    assert _fwd(lib, params(use_rope=True, rope_theta=0.0)) == 1
+    assert _fwd(lib, params(dtype=7)) == 1
+    assert _fwd(lib, params(), ptr=0) == 1                  # null pointers
+    assert _fwd(lib, params(), ptr=0x1008) == 1             # not 16-byte aligned
+    assert _fwd(lib, params(), ws=0x100010) == 1            # workspace not 256-byte aligned
+    assert _fwd(lib, params(), ws_bytes=16) == 3            # FLINT_ERR_WORKSPACE
+    assert lib.flint_attn_fwd(None, *([None] * 9), None, 0, None) == 1
+
+
+def test_fp32_any_group_size_is_accepted_by_validation(lib):
+    # FP32 runs on CUDA cores and takes any H/Hk; only workspace sizing is checked here
+    assert fa.workspace_bytes(params(num_q_heads=12, num_kv_heads=1, dtype=fa.FLINT_FP32),
+                              False) > 0

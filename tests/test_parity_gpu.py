@@ -1,0 +1,140 @@
+"""GPU parity: the CUDA library (through its C ABI) against the FP64 oracle.
+
+Small cases compare every output element; the full-size workloads compare
+sampled rows that the oracle computes one by one.
+"""
+import numpy as np
+import pytest
+import torch
+
+import flint_inputs as fi
+from oracle import flint_oracle as fo
+from parity_util import compare, f64, run_bwd, run_fwd, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+def oracle_full(d, w: fi.Workload, backward):
+    O, lse = fo.flint_attn_fwd(d["q"], d["k"], d["v"], d["w_q"], d["w_k"], d["sink"],
+                               d["cu_doc_lens"], w.window, w.use_rope, w.rope_theta)
+    g = None
+    if backward:
+        g = fo.flint_attn_bwd(d["q"], d["k"], d["v"], d["w_q"], d["w_k"], d["sink"],
+                              d["cu_doc_lens"], w.window, w.use_rope, w.rope_theta, d["dout"])
+    return O, lse, g
+
+
+# ----------------------------------------------------------------------- FP32 tiny layer
+
+def test_tiny_sliding_fp32_forward_backward(cuda_lib):
+    w = fi.TINY_SLIDING_FP32
+    cpu = fi.make_inputs(w)
+    d = to_dev(cpu)
+    out, lse = run_fwd(cuda_lib, d, w.window, w.use_rope, w.rope_theta)
+    O, L, g = oracle_full(cpu, w, True)
+    compare(out, O, "fp32", "out")
+    compare(lse, L, "fp32", "lse")
+    gr = run_bwd(cuda_lib, d, out, lse, w.window, w.use_rope, w.rope_theta)
+    torch.cuda.synchronize()
+    for name in ["dq", "dk", "dv", "dw_q", "dw_k", "dsink"]:
+        compare(gr[name], g[name], "fp32", name)
+
+
+# ----------------------------------------------------------------------- BF16 small sweeps
+
+SMALL_CASES = [
+    # doc lengths, H, Hk, window, rope
+    ([300], 32, 4, 64, True),
+    ([257, 1, 130, 7], 32, 4, 63, True),
+    ([200, 0, 333], 32, 4, 65, False),
+    ([513], 32, 4, 1, True),
+    ([129, 64], 32, 4, 2, False),
+    ([600], 32, 4, 0, False),
+    ([450], 32, 4, 10_000, True),
+    ([31, 17, 290], 16, 2, 100, True),
+    ([160, 96], 8, 1, 0, True),
+    ([384], 16, 4, 128, False),      # G = 4
+    ([70, 260], 4, 4, 50, True),     # G = 1
+]
+
+
+@pytest.mark.parametrize("lens,H,Hk,W,rope", SMALL_CASES)
+def test_bf16_forward_small(cuda_lib, lens, H, Hk, W, rope):
+    cpu = fi.make_custom(lens, H, Hk, dtype="bf16", seed=len(lens) * 7 + W % 97)
+    d = to_dev(cpu)
+    out, lse = run_fwd(cuda_lib, d, W, rope, 1e6)
+    O, L = fo.flint_attn_fwd(cpu["q"], cpu["k"], cpu["v"], cpu["w_q"], cpu["w_k"], cpu["sink"],
+                             cpu["cu_doc_lens"], W, rope, 1e6)
+    compare(out, O, "bf16", "out")
+    compare(lse, L, "bf16", "lse")
+
+
+def test_bf16_forward_is_deterministic(cuda_lib):
+    cpu = fi.make_custom([700, 300], 32, 4, dtype="bf16", seed=3)
+    d = to_dev(cpu)
+    o1, l1 = run_fwd(cuda_lib, d, 256, True, 1e6)
+    o2, l2 = run_fwd(cuda_lib, d, 256, True, 1e6)
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_bf16_sink_minus_inf_and_large_logits(cuda_lib):
+    """Sinks at -inf reduce to plain softmax attention; large sinks dominate the row."""
+    cpu = fi.make_custom([260, 140], 32, 4, dtype="bf16", seed=5)
+    cpu["sink"][:8] = -float("inf")
+    cpu["sink"][8:16] = 30.0
+    d = to_dev(cpu)
+    out, lse = run_fwd(cuda_lib, d, 90, True, 1e6)
+    O, L = fo.flint_attn_fwd(cpu["q"], cpu["k"], cpu["v"], cpu["w_q"], cpu["w_k"], cpu["sink"],
+                             cpu["cu_doc_lens"], 90, True, 1e6)
+    compare(out, O, "bf16", "out")
+    compare(lse, L, "bf16", "lse")
+
+
+# ----------------------------------------------------------------------- full-size workloads
+
+def sample_rows(cu, H, n, seed):
+    """Rows at document edges and tile edges, plus random ones."""
+    rng = np.random.default_rng(seed)
+    cu = [int(c) for c in cu]
+    T = cu[-1]
+    toks = {0, T - 1, 15, 16, 31, 32, 127, 128, 255}
+    for a, b in zip(cu[:-1], cu[1:]):
+        if b > a:
+            toks |= {a, b - 1}
+    toks = [t for t in toks if 0 <= t < T]
+    toks += list(rng.integers(0, T, size=max(0, n - len(toks))))
+    return [(int(t), int(rng.integers(0, H))) for t in toks[:n]]
+
+
+@pytest.mark.parametrize("wl", [fi.SLIDING_BF16, fi.FULL_BF16, fi.PACKED_BF16, fi.LONG_FULL_BF16],
+                         ids=lambda w: w.name)
+def test_bf16_forward_full_size_sampled(cuda_lib, wl):
+    cpu = fi.make_inputs(wl, with_grad_out=False)
+    d = to_dev(cpu)
+    out, lse = run_fwd(cuda_lib, d, wl.window, wl.use_rope, wl.rope_theta)
+    torch.cuda.synchronize()
+    ro = fo.RowOracle(cpu["q"], cpu["k"], cpu["v"], cpu["w_q"], cpu["w_k"], cpu["sink"],
+                      cpu["cu_doc_lens"], wl.window, wl.use_rope, wl.rope_theta)
+    rows = sample_rows(cpu["cu_doc_lens"], wl.num_q_heads, 48 if wl.total_tokens > 40000 else 96,
+                       seed=1)
+    ref_o = np.stack([ro.forward_row(t, h)[0] for t, h in rows])
+    ref_l = np.array([ro.forward_row(t, h)[1] for t, h in rows])
+    got_o = torch.stack([out[t, h] for t, h in rows])
+    got_l = torch.stack([lse[h, t] for t, h in rows])
+    compare(got_o, ref_o, "bf16", "out rows")
+    compare(got_l, ref_l, "bf16", "lse rows")
+    # properties that hold at every row: finite, |O| bounded by max |v| of the KV head
+    assert torch.isfinite(out).all() and torch.isfinite(lse).all()
+    vmax = d["v"].float().abs().amax().item()
+    assert out.float().abs().amax().item() <= vmax * 1.01
+
+
+def test_bf16_sliding_forward_full_oracle(cuda_lib):
+    """The 2 x 4096, W=512 layer against the whole-layer oracle (every element)."""
+    wl = fi.SLIDING_BF16
+    cpu = fi.make_inputs(wl, with_grad_out=False)
+    d = to_dev(cpu)
+    out, lse = run_fwd(cuda_lib, d, wl.window, wl.use_rope, wl.rope_theta)
+    O, L, _ = oracle_full(cpu, wl, False)
+    compare(out, O, "bf16", "out")
+    compare(lse, L, "bf16", "lse")
