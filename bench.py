@@ -1,0 +1,471 @@
+#!/usr/bin/env python
+"""Benchmark of Flint's sink-aware attention (forward + backward) on B200.
+
+One step = the whole hot path over one batch: RMSNorm+RoPE prologue, work
+list, tcgen05 attention forward, backward preprocess (D, d_sink), tcgen05
+backward (dK/dV and dQ) and the prologue backward - both C-ABI calls
+(flint_attn_fwd, flint_attn_bwd). The metric counts masked FLOPs: 4*D*H*pairs
+for the forward and 10*D*H*pairs for the backward (five GEMMs).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Multi-GPU (torchrun, one process per GPU): every rank runs its own batch
+(replicas, weak scaling); no data-path collective exists in this path. The
+step time is the max over ranks of CUDA-event time. Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+import flint_inputs as fi  # noqa: E402
+
+METRIC = "sink-attention fwd/bwd TFLOP/s (masked FLOPs) and % of B200 BF16 tensor peak"
+UNIT = "TFLOP/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+WORKLOADS = {w.name: w for w in fi.WORKLOADS}
+DEFAULT_WORKLOAD = fi.FULL_BF16.name
+L2_FLUSH_BYTES = 256 << 20
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="flint", choices=["flint", "reference"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0,
+                    help="target CPU time of the oracle baseline sample")
+    return ap.parse_args(argv)
+
+
+# --------------------------------------------------------------------------- helpers
+
+def flops_of(doc_lens, window, H, D=128):
+    pairs = fi.visible_pairs(doc_lens, window)
+    return pairs, 4.0 * D * H * pairs, 10.0 * D * H * pairs
+
+
+def read_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def config_of(w, pairs, flops_step):
+    return {
+        "workload": f"{w.name} fwd+bwd",
+        "tokens": w.total_tokens,
+        "docs": "drawn U[128,8192]" if w.doc_lens is None else len(w.doc_lens),
+        "heads_q": w.num_q_heads, "heads_kv": w.num_kv_heads, "head_dim": w.head_dim,
+        "window": w.window if w.window > 0 else "full causal",
+        "rope": bool(w.use_rope), "rope_theta": w.rope_theta if w.use_rope else None,
+        "sink_std": w.sink_std,
+        "masked_pairs_per_head": pairs, "flops_per_step": flops_step,
+        "l2": "inputs larger than L2 (126 MB), plus a 256 MB L2 flush before every step",
+        "parallelism": "replicas (one independent batch per GPU)",
+        "gradients": "dq, dk, dv in float32; dw_q, dw_k, d_sink float32",
+    }
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples taken while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self):
+        self.proc = None
+        self.path = os.path.join("/tmp", f"flint_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self, device_index=None):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    idx, clk, cmax, pw = int(parts[0]), float(parts[1]), float(parts[2]), float(parts[3])
+                except ValueError:
+                    continue
+                if device_index is not None and idx != device_index:
+                    continue
+                mx = max(mx, cmax)
+                if pw > 250.0:          # under load
+                    sm.append(clk)
+                for n, v in zip(names, parts[5:9]):
+                    if v.lower().startswith("active"):
+                        reasons.add(n)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx or None,
+                "reasons": sorted(reasons), "samples_under_load": len(sm)}
+
+
+def kernel_source_sha(name):
+    path = os.path.join(ROOT, "sink_aware_sliding_head_b200", "csrc", name)
+    try:
+        with open(path, "rb") as f:
+            return hashlib.sha256(f.read()).hexdigest()[:16]
+    except OSError:
+        return None
+
+
+def traffic_for(kernel, workload):
+    """DRAM bytes per launch from the committed ncu summary, if the kernel is unchanged."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    try:
+        with open(path) as f:
+            entries = json.load(f)
+    except Exception:
+        return None
+    for e in entries:
+        if e.get("kernel") == kernel and e.get("workload") == workload and \
+                e.get("source_sha") == kernel_source_sha(e.get("source", "")):
+            return e.get("dram_bytes_per_launch")
+    return None
+
+
+# --------------------------------------------------------------------------- CPU oracle
+
+def oracle_sample(w, inp, seconds):
+    """Time the FP64 oracle fwd+bwd on a prefix of the workload sized for ~seconds.
+
+    Returns (flops, wall seconds, description). The prefix keeps the workload's
+    heads, window and RoPE; for packed workloads it takes whole leading documents.
+    """
+    from oracle import flint_oracle as fo   # test infrastructure: CPU baseline leg only
+
+    def run(n_tok):
+        cu = [int(c) for c in inp["cu_doc_lens"]]
+        lens, acc = [], 0
+        for a, b in zip(cu[:-1], cu[1:]):
+            if acc >= n_tok:
+                break
+            take = min(b - a, n_tok - acc)
+            lens.append(take)
+            acc += take
+        n_tok = acc
+        cu_p = [0]
+        for L in lens:
+            cu_p.append(cu_p[-1] + L)
+        sl = slice(0, n_tok)
+        t0 = time.perf_counter()
+        fo.flint_attn_bwd(inp["q"][sl], inp["k"][sl], inp["v"][sl], inp["w_q"], inp["w_k"],
+                          inp["sink"], cu_p, w.window, w.use_rope, w.rope_theta, inp["dout"][sl])
+        fo.flint_attn_fwd(inp["q"][sl], inp["k"][sl], inp["v"][sl], inp["w_q"], inp["w_k"],
+                          inp["sink"], cu_p, w.window, w.use_rope, w.rope_theta)
+        dt = time.perf_counter() - t0
+        pairs, ff, fb = flops_of(lens, w.window, w.num_q_heads)
+        return ff + fb, dt, n_tok
+
+    f0, t0, n0 = run(256)
+    # work grows ~quadratically (full causal) or linearly (windowed) with the prefix
+    grow = 2.0 if w.window <= 0 else 1.0
+    n = int(256 * max(1.0, seconds / max(t0, 1e-3)) ** (1.0 / grow))
+    n = max(256, min(w.total_tokens, (n // 128) * 128))
+    f, t, n = run(n)
+    desc = (f"oracle fwd+bwd (FP64 NumPy) on the first {n} tokens of {w.name} "
+            f"({w.num_q_heads}/{w.num_kv_heads} heads, same window/RoPE); masked FLOPs of that prefix")
+    return f, t, desc
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+# --------------------------------------------------------------------------- reference arm
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    w = WORKLOADS[args.workload]
+    inp = fi.make_inputs(w, with_grad_out=True)
+    pairs, ff, fb = flops_of(inp["doc_lens"], w.window, w.num_q_heads)
+    per_step = max(2.0, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
+    total_f, total_t, desc = 0.0, 0.0, ""
+    for i in range(args.warmup + args.steps):
+        f, t, desc = oracle_sample(w, inp, per_step)
+        if i >= args.warmup:
+            total_f += f
+            total_t += t
+    value = total_f / total_t / 1e12
+    cores = blas_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total_t / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_of(w, pairs, ff + fb),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# --------------------------------------------------------------------------- GPU arm
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        run_reference(args)
+        return
+    from sink_aware_sliding_head_b200 import flint_attn as fa
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=dev)
+        pg = dist
+
+    def barrier():
+        if pg is not None:
+            pg.barrier()
+
+    w = WORKLOADS[args.workload]
+    cpu = fi.make_inputs(w, seed=w.seed + rank, with_grad_out=True)
+    pairs, ff, fb = flops_of(cpu["doc_lens"], w.window, w.num_q_heads)
+    flops_step = ff + fb
+    d = {k: (v.to(dev) if torch.is_tensor(v) else v) for k, v in cpu.items()}
+    T, H, D = d["q"].shape
+    p = fa.params_for(d["q"], d["k"], d["cu_doc_lens"], w.window, w.use_rope, w.rope_theta,
+                      fp32_grads=True)
+    ws_f = fa.alloc_workspace(p, False, dev)
+    ws_b = fa.alloc_workspace(p, True, dev)
+    out = torch.empty_like(d["q"])
+    lse = torch.empty(H, T, dtype=torch.float32, device=dev)
+    # gradients w.r.t. q, k, v in float32 (the configuration the parity tests hold
+    # to max-abs 2e-2; bfloat16 storage alone would exceed that for |grad| > 10)
+    f32 = torch.float32
+    grads = {"dq": torch.empty(d["q"].shape, dtype=f32, device=dev),
+             "dk": torch.empty(d["k"].shape, dtype=f32, device=dev),
+             "dv": torch.empty(d["v"].shape, dtype=f32, device=dev),
+             "dw_q": torch.empty(D, dtype=torch.float32, device=dev),
+             "dw_k": torch.empty(D, dtype=torch.float32, device=dev),
+             "dsink": torch.empty(H, dtype=torch.float32, device=dev)}
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def fwd_call(src):
+        fa.fwd(src["q"], src["k"], src["v"], src["w_q"], src["w_k"], src["sink"],
+               src["cu_doc_lens"], w.window, w.use_rope, w.rope_theta, out=out, lse=lse,
+               workspace=ws_f)
+
+    def bwd_call(src):
+        fa.bwd(src["q"], src["k"], src["v"], src["w_q"], src["w_k"], src["sink"],
+               src["cu_doc_lens"], out, lse, src["dout"], w.window, w.use_rope, w.rope_theta,
+               grads=grads, workspace=ws_b, fp32_grads=True)
+
+    # ---- warm-up (also surfaces device-side timeouts before timing)
+    for _ in range(args.warmup):
+        flush.zero_()
+        fwd_call(d)
+        bwd_call(d)
+    torch.cuda.synchronize(dev)
+    lib = fa.load_library()
+    for ws in (ws_f, ws_b):
+        code = lib.flint_attn_check_status(fa._ptr(ws), fa._stream_ptr())
+        if code != 0:
+            raise RuntimeError(f"device status {fa.STATUS.get(code, code)} during warm-up")
+
+    # ---- timed region: device-resident inputs
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    clocks = ClockSampler() if rank == 0 else None
+    if clocks:
+        clocks.start()
+    fa.profile_reset()
+    fa.profile_collect()
+    fa.profile_reset()
+    fa.profile_enable(True)
+    n0 = fa.launch_count()
+    barrier()
+    torch.cuda.synchronize(dev)
+    for i in range(args.steps):
+        flush.zero_()
+        ev[i][0].record(stream)
+        fwd_call(d)
+        ev[i][1].record(stream)
+        bwd_call(d)
+        ev[i][2].record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    launches = fa.launch_count() - n0
+    fa.profile_enable(False)
+    kern = fa.profile_collect()
+    clk = clocks.stop() if clocks else None
+    fwd_ms = sum(e[0].elapsed_time(e[1]) for e in ev)
+    bwd_ms = sum(e[1].elapsed_time(e[2]) for e in ev)
+    tot_ms = fwd_ms + bwd_ms
+    t_local = torch.tensor([tot_ms, fwd_ms, bwd_ms], dtype=torch.float64, device=dev)
+    if pg is not None:
+        pg.all_reduce(t_local, op=pg.ReduceOp.MAX)
+    tot_ms, fwd_ms, bwd_ms = [float(x) for x in t_local.tolist()]
+    ms_step = tot_ms / args.steps
+    value = world * flops_step * args.steps / (tot_ms * 1e-3) / 1e12
+
+    # ---- end to end: host (pinned) inputs -> device -> both calls -> host results
+    e2e = None
+    if not args.no_e2e:
+        names_in = ["q", "k", "v", "w_q", "w_k", "sink", "cu_doc_lens", "dout"]
+        host_in = {k: cpu[k].pin_memory() for k in names_in}
+        dev_in = {k: torch.empty_like(d[k]) for k in names_in}
+        host_out = {"out": torch.empty(out.shape, dtype=out.dtype, pin_memory=True),
+                    "lse": torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)}
+        for k, v in grads.items():
+            host_out[k] = torch.empty(v.shape, dtype=v.dtype, pin_memory=True)
+        h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+        d2h = sum(t.numel() * t.element_size() for t in host_out.values())
+
+        def e2e_step():
+            for k in names_in:
+                dev_in[k].copy_(host_in[k], non_blocking=True)
+            fwd_call(dev_in)
+            bwd_call(dev_in)
+            host_out["out"].copy_(out, non_blocking=True)
+            host_out["lse"].copy_(lse, non_blocking=True)
+            for k, v in grads.items():
+                host_out[k].copy_(v, non_blocking=True)
+
+        for _ in range(max(1, args.warmup)):
+            e2e_step()
+        torch.cuda.synchronize(dev)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        barrier()
+        torch.cuda.synchronize(dev)
+        e0.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+        t_e2e = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+        if pg is not None:
+            pg.all_reduce(t_e2e, op=pg.ReduceOp.MAX)
+        e2e = {"value": world * flops_step * args.steps / (float(t_e2e.item()) * 1e-3) / 1e12,
+               "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "ms_per_step": float(t_e2e.item()) / args.steps}
+
+    if rank != 0:
+        if pg is not None:
+            pg.destroy_process_group()
+        return
+
+    # ---- roofline of the dominant kernel (live CUDA-event time per launch)
+    peaks, peak_src = read_peaks()
+    algo = {  # algorithmic work per launch
+        "attn_fwd_sm100": ("tensor", 4.0 * D * H * pairs),
+        "attn_bwd_dkv_sm100": ("tensor", 8.0 * D * H * pairs),
+        "attn_bwd_dq_sm100": ("tensor", 2.0 * D * H * pairs),
+        "prologue_rmsnorm_rope": ("hbm", None),
+    }
+    dom = max(kern.items(), key=lambda kv: kv[1][0])
+    dname, (dms, dn) = dom
+    per_launch_ms = dms / max(dn, 1)
+    roofline = None
+    if dname in algo and algo[dname][1] is not None:
+        achieved = algo[dname][1] / (per_launch_ms * 1e-3) / 1e12
+        peak = peaks["bf16_tflops_sustained"]
+        src = {"attn_fwd_sm100": "attn_fwd_sm100.cu"}.get(dname, "attn_bwd_sm100.cu")
+        roofline = {"kernel": dname, "bound": "tensor", "achieved": achieved, "peak": peak,
+                    "unit": "TFLOP/s", "frac": achieved / peak,
+                    "peak_kind": f"bf16 sustained ({peak_src})",
+                    "frac_of_burst": achieved / peaks["bf16_tflops"],
+                    "traffic": traffic_for(dname, w.name),
+                    "algorithmic_flops_per_launch": algo[dname][1],
+                    "ms_per_launch": per_launch_ms, "source": src}
+    kernels = {k: {"ms_per_step": v[0] / args.steps, "launches": v[1],
+                   "share": v[0] / max(sum(x[0] for x in kern.values()), 1e-9)}
+               for k, v in kern.items() if v[1] > 0}
+    fwd_attn = kern.get("attn_fwd_sm100", (0.0, 0))
+    fwd_kernel_tflops = (4.0 * D * H * pairs * fwd_attn[1] / (fwd_attn[0] * 1e-3) / 1e12
+                         if fwd_attn[1] else None)
+
+    cpu_baseline = None
+    if world == 1 and not args.no_cpu_baseline:
+        f, t, desc = oracle_sample(w, cpu, args.cpu_seconds)
+        cpu_baseline = {"value": f / t / 1e12, "unit": UNIT, "cores": blas_threads(),
+                        "kind": "oracle", "sample": desc, "seconds": t}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) q/k/v/dO, norm weights 1+0.1N, FP32 sinks)",
+        "config": config_of(w, pairs, flops_step),
+        "fwd_tflops": world * ff * args.steps / (fwd_ms * 1e-3) / 1e12,
+        "bwd_tflops": world * fb * args.steps / (bwd_ms * 1e-3) / 1e12,
+        "fwd_ms": fwd_ms / args.steps, "bwd_ms": bwd_ms / args.steps,
+        "fwd_kernel_tflops": fwd_kernel_tflops,
+        "pct_of_peak": {
+            "step_vs_bf16_sustained": value / world / peaks["bf16_tflops_sustained"],
+            "fwd_kernel_vs_bf16_burst": (fwd_kernel_tflops or 0) / peaks["bf16_tflops"],
+            "fwd_kernel_vs_nominal_2250": (fwd_kernel_tflops or 0) / 2250.0,
+            "peaks": peak_src},
+        "roofline": roofline,
+        "kernels": kernels,
+        "gpu_launches": launches,
+        "clocks": clk,
+        "e2e": e2e,
+        "cpu_baseline": cpu_baseline,
+    }
+    print(json.dumps(line), flush=True)
+    if pg is not None:
+        pg.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -86,6 +86,8 @@ typedef struct {
   float rms_eps;          /* RMSNorm epsilon (Flint: 1e-6) */
   float softmax_scale;    /* 0 => 1/sqrt(head_dim) */
   int32_t dtype;          /* flint_dtype_t */
+  int32_t fp32_grads;     /* backward only: nonzero => dq, dk, dv are float32 (FP32 inputs
+                             always give float32 gradients); zero => same type as q */
 } flint_attn_params_t;
 
 /* Bytes of device workspace a call needs (backward = 0 for flint_attn_fwd,
@@ -107,10 +109,14 @@ flint_status_t flint_attn_fwd(const flint_attn_params_t* params,
 
 /* Backward of sum(dout * out) for out = flint_attn_fwd(...).
  *   out, lse: the forward's results for the same inputs; dout [T,H,D] (dtype).
- *   Writes dq [T,H,D], dk [T,Hk,D], dv [T,Hk,D] (dtype; gradients w.r.t. the RAW
- *   q, k, v), dq_norm_w, dk_norm_w [D] fp32, dsink [H] fp32. Outputs are
- *   overwritten, not accumulated. q and k are re-normalised and re-rotated
- *   inside (nothing from the forward besides out and lse is needed). */
+ *   Writes dq [T,H,D], dk [T,Hk,D], dv [T,Hk,D] (gradients w.r.t. the RAW q, k,
+ *   v; float32 when params->fp32_grads or dtype is FLINT_FP32, else bfloat16),
+ *   dq_norm_w, dk_norm_w [D] fp32, dsink [H] fp32. Outputs are overwritten, not
+ *   accumulated. q and k are re-normalised and re-rotated inside (nothing from
+ *   the forward besides out and lse is needed).
+ *   BF16 inputs: the backward's tensor-core operands (q_hat, k_hat, v, dout, P,
+ *   dS) are IEEE fp16 for their 10-bit mantissa; |v| and |dout| must stay below
+ *   65504 (larger values saturate to +-65504). Accumulation is FP32. */
 flint_status_t flint_attn_bwd(const flint_attn_params_t* params,
                               const void* q, const void* k, const void* v,
                               const void* q_norm_w, const void* k_norm_w,
@@ -124,6 +130,22 @@ flint_status_t flint_attn_bwd(const flint_attn_params_t* params,
  * `workspace` (written by bounded device waits), and returns FLINT_OK or
  * FLINT_ERR_TIMEOUT (FLINT_ERR_CUDA if the stream itself reports an error). */
 flint_status_t flint_attn_check_status(void* workspace, void* stream);
+
+/* ---- Measurement aids (not needed to compute anything) --------------------
+ * flint_attn_profile_enable(1): later calls bracket each of their kernel
+ * launches with a pair of CUDA events recorded on the call's stream (events are
+ * created on first use and reused; no device memory is allocated).
+ * flint_attn_profile_collect(): synchronises the recorded events, adds each
+ * launch's duration into per-kernel totals and frees the event slots; then
+ * fills up to max_kernels entries of names / total_ms / launches and returns
+ * the number of kernel kinds. flint_attn_profile_reset() zeroes the totals.
+ * flint_attn_launch_count(): kernels this library has launched since it was
+ * loaded (counted whether or not profiling is enabled). Host-thread-safe. */
+void flint_attn_profile_enable(int enable);
+int flint_attn_profile_collect(int max_kernels, const char** names, double* total_ms,
+                               long long* launches);
+void flint_attn_profile_reset(void);
+long long flint_attn_launch_count(void);
 
 /* Static description of a status code. */
 const char* flint_status_string(flint_status_t status);

@@ -157,7 +157,7 @@ def _block_logits(q_hat, k_hat, a, b, lo, window, h_list, kv, scale):
     """Scaled logits [len(h_list), b-a, b-lo] with -inf outside the visible set."""
     q = q_hat[a:b][:, h_list, :]                       # [n, g, D]
     k = k_hat[lo:b, kv, :]                             # [m, D]
-    z = scale * np.einsum("ngd,md->gnm", q, k)
+    z = scale * (q.transpose(1, 0, 2) @ k.T)         # [g, n, m]
     i = np.arange(a, b)[:, None]
     j = np.arange(lo, b)[None, :]
     vis = j <= i
@@ -199,7 +199,7 @@ def attention_forward(q_hat, k_hat, v, sink, cu_doc_lens, window, scale=None):
                 hs = list(range(kv * G, (kv + 1) * G))
                 z = _block_logits(q_hat, k_hat, a, b, lo, window, hs, kv, scale)
                 p, _, l = _sink_softmax(z, sink[hs])
-                O[a:b, kv * G:(kv + 1) * G, :] = np.einsum("gnm,md->ngd", p, v[lo:b, kv, :])
+                O[a:b, kv * G:(kv + 1) * G, :] = (p @ v[lo:b, kv, :]).transpose(1, 0, 2)
                 lse[kv * G:(kv + 1) * G, a:b] = l
     return O, lse
 
@@ -234,13 +234,13 @@ def attention_backward(q_hat, k_hat, v, sink, cu_doc_lens, window, dO, scale=Non
                 p, ps, _ = _sink_softmax(z, sink[hs])            # [g,n,m], [g,n]
                 dOb = dO[a:b, kv * G:(kv + 1) * G, :]             # [n,g,D]
                 Di = Dvec[a:b, kv * G:(kv + 1) * G].T             # [g,n]
-                dv[lo:b, kv, :] += np.einsum("gnm,ngd->md", p, dOb)
-                dp = np.einsum("ngd,md->gnm", dOb, v[lo:b, kv, :])
+                dOg = dOb.transpose(1, 0, 2)                      # [g,n,D]
+                dv[lo:b, kv, :] += (p.transpose(0, 2, 1) @ dOg).sum(axis=0)
+                dp = dOg @ v[lo:b, kv, :].T                       # [g,n,m]
                 dz = p * (dp - Di[..., None])
-                dq[a:b, kv * G:(kv + 1) * G, :] += scale * np.einsum(
-                    "gnm,md->ngd", dz, k_hat[lo:b, kv, :])
-                dk[lo:b, kv, :] += scale * np.einsum(
-                    "gnm,ngd->md", dz, q_hat[a:b][:, hs, :])
+                dq[a:b, kv * G:(kv + 1) * G, :] += scale * (dz @ k_hat[lo:b, kv, :]).transpose(1, 0, 2)
+                dk[lo:b, kv, :] += scale * (dz.transpose(0, 2, 1) @
+                                            q_hat[a:b][:, hs, :].transpose(1, 0, 2)).sum(axis=0)
                 dsink[hs] -= np.sum(ps * Di, axis=-1)
     return dq, dk, dv, dsink
 
@@ -305,19 +305,29 @@ class RowOracle:
 
     def __init__(self, q, k, v, w_q, w_k, sink, cu_doc_lens, window, use_rope,
                  rope_theta, dO=None, eps=1e-6, scale=None):
-        self.q, self.k, self.v, self.w_q, self.w_k, self.sink = map(
-            _f64, (q, k, v, w_q, w_k, sink))
-        self.dO = None if dO is None else _f64(dO)
+        # q and dO rows are converted to float64 when a row needs them (the
+        # whole tensors can be several GB in float64); k, v are converted once.
+        self._q_src, self._dO_src = q, dO
+        self.k, self.v, self.w_q, self.w_k, self.sink = map(_f64, (k, v, w_q, w_k, sink))
         self.cu = np.asarray(_f64(cu_doc_lens), dtype=np.int64)
         self.pos = doc_positions(self.cu)
         self.window, self.use_rope, self.theta, self.eps = window, use_rope, rope_theta, eps
-        T, H, D = self.q.shape
+        T, H, D = q.shape
         self.H, self.Hk, self.D = H, self.k.shape[1], D
         self.scale = 1.0 / np.sqrt(D) if scale is None else scale
         self.k_hat = prologue(self.k, self.w_k, self.pos, use_rope, rope_theta, eps)
+        # contiguous copy per KV head: row products then read memory in order
+        self.k_hat_kv = [np.ascontiguousarray(self.k_hat[:, g, :]) for g in range(self.Hk)]
+        self.v_kv = [np.ascontiguousarray(self.v[:, g, :]) for g in range(self.Hk)]
+
+    def _q_row(self, t, h):
+        return _f64(self._q_src[t:t + 1, h:h + 1, :])
+
+    def _dO_row(self, t, h):
+        return _f64(self._dO_src[t, h, :])
 
     def _q_hat(self, t, h):
-        return prologue(self.q[t:t + 1, h:h + 1, :], self.w_q, self.pos[t:t + 1],
+        return prologue(self._q_row(t, h), self.w_q, self.pos[t:t + 1],
                         self.use_rope, self.theta, self.eps)[0, 0]
 
     def _row(self, t, h):
@@ -325,12 +335,12 @@ class RowOracle:
         d0, _ = _doc_of(self.cu, t)
         lo, hi = visible_keys(t, d0, self.window)
         kv = _group(h, self.H, self.Hk)
-        z = self.scale * (self.k_hat[lo:hi + 1, kv, :] @ self._q_hat(t, h))
+        z = self.scale * (self.k_hat_kv[kv][lo:hi + 1] @ self._q_hat(t, h))
         m = max(float(np.max(z)), float(self.sink[h]))
         e = np.exp(z - m)
         Z = np.exp(self.sink[h] - m) + np.sum(e)
         p = e / Z
-        return lo, hi, kv, p, np.exp(self.sink[h] - m) / Z, m + np.log(Z), p @ self.v[lo:hi + 1, kv, :]
+        return lo, hi, kv, p, np.exp(self.sink[h] - m) / Z, m + np.log(Z), p @ self.v_kv[kv][lo:hi + 1]
 
     def forward_row(self, t, h):
         """(O[t, h, :], LSE[h, t])."""
@@ -340,10 +350,11 @@ class RowOracle:
     def dq_row(self, t, h):
         """Gradient of sum(dO * O) w.r.t. the raw q[t, h, :]."""
         lo, hi, kv, p, _, _, o = self._row(t, h)
-        Di = float(self.dO[t, h] @ o)
-        dz = p * (self.v[lo:hi + 1, kv, :] @ self.dO[t, h] - Di)
-        g_hat = self.scale * (dz @ self.k_hat[lo:hi + 1, kv, :])
-        dx, _ = prologue_backward(self.q[t:t + 1, h:h + 1, :], self.w_q, g_hat[None, None, :],
+        dO = self._dO_row(t, h)
+        Di = float(dO @ o)
+        dz = p * (self.v_kv[kv][lo:hi + 1] @ dO - Di)
+        g_hat = self.scale * (dz @ self.k_hat_kv[kv][lo:hi + 1])
+        dx, _ = prologue_backward(self._q_row(t, h), self.w_q, g_hat[None, None, :],
                                   self.pos[t:t + 1], self.use_rope, self.theta, self.eps)
         return dx[0, 0]
 
@@ -358,9 +369,10 @@ class RowOracle:
             for h in range(kv * G, (kv + 1) * G):
                 lo, _, _, p, _, _, o = self._row(i, h)
                 pij = p[j - lo]
-                Di = float(self.dO[i, h] @ o)
-                dv += pij * self.dO[i, h]
-                dz = pij * (float(self.dO[i, h] @ self.v[j, kv]) - Di)
+                dO = self._dO_row(i, h)
+                Di = float(dO @ o)
+                dv += pij * dO
+                dz = pij * (float(dO @ self.v[j, kv]) - Di)
                 dk_hat += self.scale * dz * self._q_hat(i, h)
         dx, _ = prologue_backward(self.k[j:j + 1, kv:kv + 1, :], self.w_k, dk_hat[None, None, :],
                                   self.pos[j:j + 1], self.use_rope, self.theta, self.eps)

@@ -6,6 +6,7 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "common.cuh"
 #include "sm100_primitives.cuh"
@@ -26,6 +27,53 @@ cudaError_t launch_attn_bwd_sm100_impl(const CUtensorMap& tq, const CUtensorMap&
                                        const int4* items_q, const int* n_q, int max_q,
                                        float* dq_acc, float* dk_acc, void* dv, int* status,
                                        int num_sms, cudaStream_t st);
+
+// ------------------------------------------------------------------ kernel timing
+namespace {
+const char* const kKernelNames[kNumKernelIds] = {
+    "prologue_rmsnorm_rope", "build_worklist", "attn_fwd_sm100", "attn_fwd_fp32",
+    "bwd_preprocess", "reduce_rows", "attn_bwd_dkv_sm100", "attn_bwd_dq_sm100",
+    "attn_bwd_dq_fp32", "attn_bwd_dkv_fp32", "prologue_bwd", "convert_f16"};
+constexpr int kMaxSlots = 1 << 15;
+struct Prof {
+  std::mutex mu;
+  bool enabled = false;
+  long long launches_total = 0;
+  std::vector<cudaEvent_t> ev0, ev1;
+  std::vector<int> slot_id;
+  int used = 0;
+  double total_ms[kNumKernelIds] = {};
+  long long launches[kNumKernelIds] = {};
+};
+Prof& prof() {
+  static Prof p;
+  return p;
+}
+}  // namespace
+
+ProfScope::ProfScope(int id_, cudaStream_t st_) : id(id_), st(st_), slot(-1) {
+  Prof& P = prof();
+  std::lock_guard<std::mutex> g(P.mu);
+  ++P.launches_total;
+  if (!P.enabled || P.used >= kMaxSlots) return;
+  if (P.used == (int)P.ev0.size()) {
+    cudaEvent_t a, b;
+    if (cudaEventCreate(&a) != cudaSuccess) return;
+    if (cudaEventCreate(&b) != cudaSuccess) { cudaEventDestroy(a); return; }
+    P.ev0.push_back(a);
+    P.ev1.push_back(b);
+    P.slot_id.push_back(0);
+  }
+  slot = P.used++;
+  P.slot_id[slot] = id;
+  cudaEventRecord(P.ev0[slot], st);
+}
+ProfScope::~ProfScope() {
+  if (slot < 0) return;
+  Prof& P = prof();
+  std::lock_guard<std::mutex> g(P.mu);
+  cudaEventRecord(P.ev1[slot], st);
+}
 
 namespace {
 
@@ -59,6 +107,7 @@ flint_status_t resolve(const flint_attn_params_t* in, Resolved* p) {
   p->eps = in->rms_eps;
   p->scale = in->softmax_scale > 0.f ? in->softmax_scale : 1.0f / std::sqrt((float)kHeadDim);
   p->dtype = in->dtype;
+  p->fp32_grads = (in->fp32_grads != 0 || in->dtype == FLINT_FP32) ? 1 : 0;
   p->R = kTileRows / (G <= 128 ? G : 128);
   if (p->R < 1) p->R = 1;
   return FLINT_OK;
@@ -96,16 +145,17 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 3-D bf16 tensor [T][heads][128] with a (64, box_heads, box_tokens) box and
-// 128-byte swizzle: one box fills one 128-row K-major operand panel.
-bool encode_3d(CUtensorMap* m, const void* base, int T, int heads, int box_heads, int box_tokens) {
+// 3-D 16-bit tensor [T][heads][128] (bf16 or fp16) with a (64, box_heads,
+// box_tokens) box and 128-byte swizzle: one box fills one 128-row operand panel.
+bool encode_3d(CUtensorMap* m, const void* base, int T, int heads, int box_heads, int box_tokens,
+               CUtensorMapDataType type = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[3] = {(cuuint64_t)kHeadDim, (cuuint64_t)heads, (cuuint64_t)(T > 0 ? T : 1)};
   cuuint64_t strides[2] = {(cuuint64_t)kHeadDim * 2, (cuuint64_t)heads * kHeadDim * 2};
   cuuint32_t box[3] = {64, (cuuint32_t)box_heads, (cuuint32_t)box_tokens};
   cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+  CUresult r = fn(m, type, 3, const_cast<void*>(base), dims, strides,
                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
@@ -211,9 +261,12 @@ extern "C" flint_status_t flint_attn_bwd(const flint_attn_params_t* params, cons
   float* part = at<float>(workspace, L.part);
   float* dq_acc = at<float>(workspace, L.dq_acc);
   float* dk_acc = at<float>(workspace, L.dk_acc);
-  FLINT_TRY(launch_prologue(p, q, q_norm_w, qh, p.H, cu_doc_lens, st));
-  FLINT_TRY(launch_prologue(p, k, k_norm_w, kh, p.Hk, cu_doc_lens, st));
-  FLINT_TRY(launch_bwd_preprocess(p, out, dout, lse, sink, dvec, part, dsink, st));
+  const bool f16 = p.dtype == FLINT_BF16;   // tensor-core operands of the backward are fp16
+  __half* dout16 = f16 ? at<__half>(workspace, L.dout16) : nullptr;
+  __half* v16 = f16 ? at<__half>(workspace, L.v16) : nullptr;
+  FLINT_TRY(launch_prologue(p, q, q_norm_w, qh, p.H, cu_doc_lens, st, f16));
+  FLINT_TRY(launch_prologue(p, k, k_norm_w, kh, p.Hk, cu_doc_lens, st, f16));
+  FLINT_TRY(launch_bwd_preprocess(p, out, dout, lse, sink, dvec, part, dsink, dout16, st));
   if (p.dtype == FLINT_FP32) {
     FLINT_TRY(launch_attn_bwd_fp32(p, (const float*)qh, (const float*)kh, (const float*)v,
                                    (const float*)dout, lse, dvec, cu_doc_lens, dq_acc, dk_acc,
@@ -226,9 +279,14 @@ extern "C" flint_status_t flint_attn_bwd(const flint_attn_params_t* params, cons
                                     L.max_items_kv, st));
     FLINT_TRY(launch_build_worklist(cu_doc_lens, p, kModeQuery, p.R, items_q1, status + 3, tmp,
                                     L.max_items_q1, st));
+    FLINT_TRY(launch_convert_f16(static_cast<const __nv_bfloat16*>(v), v16,
+                                 (size_t)p.T * p.Hk * kHeadDim, st));
+    const CUtensorMapDataType f16t = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
     CUtensorMap tq, tk, tv, tdo;
-    if (!encode_3d(&tq, qh, p.T, p.H, p.G, p.R) || !encode_3d(&tk, kh, p.T, p.Hk, 1, kTileKeys) ||
-        !encode_3d(&tv, v, p.T, p.Hk, 1, kTileKeys) || !encode_3d(&tdo, dout, p.T, p.H, p.G, p.R))
+    if (!encode_3d(&tq, qh, p.T, p.H, p.G, p.R, f16t) ||
+        !encode_3d(&tk, kh, p.T, p.Hk, 1, kTileKeys, f16t) ||
+        !encode_3d(&tv, v16, p.T, p.Hk, 1, kTileKeys, f16t) ||
+        !encode_3d(&tdo, dout16, p.T, p.H, p.G, p.R, f16t))
       return FLINT_ERR_CUDA;
     FLINT_TRY(launch_attn_bwd_sm100_impl(tq, tk, tv, tdo, p, lse, dvec, items_kv, status + 2,
                                          L.max_items_kv, items_q1, status + 3, L.max_items_q1,
@@ -257,6 +315,48 @@ extern "C" flint_status_t flint_attn_check_status(void* workspace, void* stream)
     return FLINT_ERR_TIMEOUT;
   }
   return FLINT_OK;
+}
+
+extern "C" void flint_attn_profile_enable(int enable) {
+  Prof& P = prof();
+  std::lock_guard<std::mutex> g(P.mu);
+  P.enabled = enable != 0;
+}
+
+extern "C" int flint_attn_profile_collect(int max_kernels, const char** names, double* total_ms,
+                                          long long* launches) {
+  Prof& P = prof();
+  std::lock_guard<std::mutex> g(P.mu);
+  for (int i = 0; i < P.used; ++i) {
+    float ms = 0.f;
+    if (cudaEventSynchronize(P.ev1[i]) == cudaSuccess &&
+        cudaEventElapsedTime(&ms, P.ev0[i], P.ev1[i]) == cudaSuccess) {
+      P.total_ms[P.slot_id[i]] += ms;
+      P.launches[P.slot_id[i]] += 1;
+    }
+  }
+  P.used = 0;
+  for (int k = 0; k < kNumKernelIds && k < max_kernels; ++k) {
+    if (names) names[k] = kKernelNames[k];
+    if (total_ms) total_ms[k] = P.total_ms[k];
+    if (launches) launches[k] = P.launches[k];
+  }
+  return kNumKernelIds;
+}
+
+extern "C" void flint_attn_profile_reset(void) {
+  Prof& P = prof();
+  std::lock_guard<std::mutex> g(P.mu);
+  for (int k = 0; k < kNumKernelIds; ++k) {
+    P.total_ms[k] = 0.0;
+    P.launches[k] = 0;
+  }
+}
+
+extern "C" long long flint_attn_launch_count(void) {
+  Prof& P = prof();
+  std::lock_guard<std::mutex> g(P.mu);
+  return P.launches_total;
 }
 
 extern "C" const char* flint_status_string(flint_status_t s) {

@@ -1,13 +1,730 @@
-// attn_bwd_sm100.cu - placeholder until the tcgen05 backward lands.
+// attn_bwd_sm100.cu - backward of the sink-aware attention on Blackwell tensor
+// cores (tcgen05 + TMEM + TMA), FP16 operands, FP32 accumulation.
+//
+// Gradients of sum(dO * O) (Flint layers page, nemo_automodel.components.
+// models.flint.layers: the learned-sink training kernel named in the module
+// docstring; FlintAttention.forward defines O). With P_ij = e^{z_ij - LSE_i}
+// over visible keys (the sink's share needs no term: its value is zero) and
+// D_i = dO_i . O_i (computed by the preprocess kernel):
+//   dV_j   = sum_i P_ij dO_i
+//   dS_ij  = P_ij (dO_i . v_j - D_i)
+//   dK^_j  = scale sum_i dS_ij q^_i        dQ^_i = scale sum_j dS_ij k^_j
+// The sink gradient itself comes from the preprocess kernel.
+//
+// Operands: q_hat, k_hat (recomputed by the prologue in fp16), fp16 copies of v
+// and dO, and P, dS rounded to fp16 - fp16's 10-bit mantissa keeps the bf16
+// rounding of these intermediates from dominating the gradient error.
+//
+// Two persistent kernels share one warp layout (warps 0-3: elementwise math,
+// thread = TMEM lane; warp 4: TMA; warp 5: MMA issue + TMEM owner):
+//  * dkv: key-major. A CTA owns 128 keys of one KV head and streams the
+//    128-row query tiles (R tokens x G heads) that see them. Per tile:
+//    S^T = K Q^T and dP^T = V dO^T (TMEM), then P^T and dS^T in fp16 overwrite
+//    their first 64 columns and feed dV += P^T dO and dK += dS^T Q as TMEM A
+//    operands. dK and dV stay in TMEM for the whole key tile, so the G heads
+//    of a group are summed without atomics. TMEM: S^T, dP^T, dV, dK = 512 cols.
+//  * dq: query-major. A CTA owns one 128-row query tile and streams its key
+//    tiles: S = Q K^T, dP = dO V^T, dS (fp16) over S, dQ += dS K. TMEM 384 cols.
+// Before an MMA overwrites a TMEM region that a previous MMA reads as its A
+// operand, the issuer waits for that MMA's completion barrier.
 #include "common.cuh"
 #include "sm100_primitives.cuh"
 
 namespace flint {
-cudaError_t launch_attn_bwd_sm100_impl(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,
-                                       const CUtensorMap&, const Resolved&, const float*,
-                                       const float*, const int4*, const int*, int, const int4*,
-                                       const int*, int, float*, float*, void*, int*, int,
-                                       cudaStream_t) {
-  return cudaErrorNotSupported;
+
+namespace {
+
+constexpr int kThreads = 192;
+constexpr int kWarpTma = 4;
+constexpr int kWarpMma = 5;
+constexpr uint32_t kChunkBytes = 128 * 64 * 2;
+constexpr uint32_t kTileBytes = 2 * kChunkBytes;
+constexpr float kLog2e = 1.4426950408889634f;
+
+struct BwdArgs {
+  int T, H, Hk, G, R, W, logG;
+  float scale, scale_log2;
+  const float* lse;
+  const float* dvec;
+  const int4* items;
+  const int* n_items;
+  int max_items;
+  float* dq_acc;
+  float* dk_acc;
+  void* dv;          // float or bf16, per dv_f32
+  int dv_f32;
+  int* status;
+};
+
+__device__ __forceinline__ uint64_t kmajor_desc(uint32_t tile_base, int kk) {
+  return make_sdesc(tile_base + (kk >> 2) * kChunkBytes + (kk & 3) * 32, 16, 1024);
 }
+__device__ __forceinline__ uint64_t mnmajor_desc(uint32_t tile_base, int kk) {
+  return make_sdesc(tile_base + kk * 2048, kChunkBytes, 1024);
+}
+
+// 128 fp32 TMEM columns of this thread's lane -> v[128]
+__device__ __forceinline__ void tmem_row128(uint32_t taddr, float (&v)[128]) {
+  uint32_t u0[32], u1[32], u2[32], u3[32];
+  tmem_ld32(taddr + 0, u0);
+  tmem_ld32(taddr + 32, u1);
+  tmem_ld32(taddr + 64, u2);
+  tmem_ld32(taddr + 96, u3);
+  tc_wait_ld_dep(u0);
+  tc_wait_ld_dep(u1);
+  tc_wait_ld_dep(u2);
+  tc_wait_ld_dep(u3);
+#pragma unroll
+  for (int e = 0; e < 32; ++e) {
+    v[e] = __uint_as_float(u0[e]);
+    v[32 + e] = __uint_as_float(u1[e]);
+    v[64 + e] = __uint_as_float(u2[e]);
+    v[96 + e] = __uint_as_float(u3[e]);
+  }
+}
+
+__device__ __forceinline__ float2 unpack_f16x2(uint32_t u) {
+  __half2 h = *reinterpret_cast<__half2*>(&u);
+  return __half22float2(h);
+}
+
+// ============================================================================
+// dK / dV : key-major
+// ============================================================================
+struct __align__(8) KvBars {
+  uint64_t kv_full, kv_empty;
+  uint64_t qd_full[2], qd_empty[2];
+  uint64_t s_full, dp_full, p_full, ds_full, dv_done, dk_done, acc_full, acc_empty;
+  uint64_t drain;
+};
+constexpr uint32_t kKvOffK = 0;
+constexpr uint32_t kKvOffV = kTileBytes;
+constexpr uint32_t kKvOffQ = 2 * kTileBytes;                 // 2 stages
+constexpr uint32_t kKvOffDO = kKvOffQ + 2 * kTileBytes;      // 2 stages
+constexpr uint32_t kKvOffStats = kKvOffDO + 2 * kTileBytes;  // [2][2][128] fp32
+constexpr uint32_t kKvOffBar = kKvOffStats + 2 * 2 * 128 * 4;
+constexpr uint32_t kKvOffTmem = kKvOffBar + sizeof(KvBars);
+constexpr uint32_t kKvOffAbort = kKvOffTmem + 16;
+constexpr uint32_t kKvSmem = kKvOffAbort + 16 + 1024;
+
+struct KvItem {
+  int k0, d0, d1, g, qend, nq;
+};
+__device__ __forceinline__ KvItem decode_kv(const BwdArgs& a, int idx) {
+  const int4 it = a.items[idx];
+  KvItem r;
+  r.k0 = it.x; r.d0 = it.y; r.d1 = it.z; r.g = it.w;
+  r.qend = a.W > 0 ? min(r.d1, r.k0 + kTileKeys - 1 + a.W) : r.d1;
+  r.nq = (r.qend - r.k0 + a.R - 1) / a.R;
+  return r;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_q,
+                    const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v,
+                    const __grid_constant__ CUtensorMap tm_do, const BwdArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  KvBars* bars = reinterpret_cast<KvBars*>(smem + kKvOffBar);
+  float* stats = reinterpret_cast<float*>(smem + kKvOffStats);   // [buf][lse2|D][128]
+  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + kKvOffTmem);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kKvOffAbort);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const WaitCtx wc{abort_flag, a.status, kStatusTimeoutBwdKV};
+
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    mbar_init(smem_u32(&bars->kv_full), 1);
+    mbar_init(smem_u32(&bars->kv_empty), 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(smem_u32(&bars->qd_full[s]), 2);   // TMA bytes + per-row statistics
+      mbar_init(smem_u32(&bars->qd_empty[s]), 1);
+    }
+    mbar_init(smem_u32(&bars->s_full), 1);
+    mbar_init(smem_u32(&bars->dp_full), 1);
+    mbar_init(smem_u32(&bars->p_full), 4);
+    mbar_init(smem_u32(&bars->ds_full), 4);
+    mbar_init(smem_u32(&bars->dv_done), 1);
+    mbar_init(smem_u32(&bars->dk_done), 1);
+    mbar_init(smem_u32(&bars->acc_full), 1);
+    mbar_init(smem_u32(&bars->acc_empty), 4);
+    mbar_init(smem_u32(&bars->drain), 1);
+    fence_mbar_init();
+  }
+  if (warp == kWarpMma) {
+    tmem_alloc(smem_u32((const void*)tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int n_items = min(*a.n_items, a.max_items);
+
+  if (warp == kWarpTma) {
+    // TMA issue from lane 0; the whole warp stages each query tile's per-row
+    // log2-LSE and D into shared memory and completes qd_full's second arrival.
+    uint32_t item_count = 0, qd_iter = 0, kv_arm = 0, qd_arm[2] = {0, 0};
+    bool ok = true;
+    for (int idx = blockIdx.x; idx < n_items && ok; idx += gridDim.x) {
+      const KvItem it = decode_kv(a, idx);
+      if (lane == 0) {
+        if (item_count > 0) ok = mbar_wait(smem_u32(&bars->kv_empty), (item_count - 1) & 1, wc);
+        if (ok) {
+          const uint32_t kf = smem_u32(&bars->kv_full);
+          mbar_arrive_expect_tx(kf, 2 * kTileBytes);
+          ++kv_arm;
+          for (int c = 0; c < 2; ++c) {
+            tma_load_3d(sbase + kKvOffK + c * kChunkBytes, &tm_k, kf, c * 64, it.g, it.k0);
+            tma_load_3d(sbase + kKvOffV + c * kChunkBytes, &tm_v, kf, c * 64, it.g, it.k0);
+          }
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      for (int m = 0; m < it.nq && ok; ++m, ++qd_iter) {
+        const int qs = it.k0 + m * a.R;
+        const uint32_t s = qd_iter & 1, ph = (qd_iter >> 1) & 1;
+        if (lane == 0 && qd_iter >= 2) ok = mbar_wait(smem_u32(&bars->qd_empty[s]), ph ^ 1, wc);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        const uint32_t qf = smem_u32(&bars->qd_full[s]);
+        if (lane == 0) {
+          mbar_arrive_expect_tx(qf, 2 * kTileBytes);
+          ++qd_arm[s];
+          for (int c = 0; c < 2; ++c) {
+            tma_load_3d(sbase + kKvOffQ + s * kTileBytes + c * kChunkBytes, &tm_q, qf, c * 64,
+                        it.g * a.G, qs);
+            tma_load_3d(sbase + kKvOffDO + s * kTileBytes + c * kChunkBytes, &tm_do, qf, c * 64,
+                        it.g * a.G, qs);
+          }
+        }
+        float* st = stats + s * 256;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int r = lane + 32 * e;
+          const int tok = qs + (r >> a.logG), h = it.g * a.G + (r & (a.G - 1));
+          const bool vr = tok < it.d1;
+          st[r] = vr ? __ldg(a.lse + (size_t)h * a.T + tok) * kLog2e : 0.f;
+          st[128 + r] = vr ? __ldg(a.dvec + (size_t)h * a.T + tok) : 0.f;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(qf);
+      }
+      ++item_count;
+    }
+    if (lane == 0) {
+      volatile int no_abort = 0;
+      const WaitCtx drain{&no_abort, a.status, kStatusTimeoutBwdKV};
+      if (kv_arm) mbar_wait(smem_u32(&bars->kv_full), (kv_arm - 1) & 1, drain);
+      if (qd_arm[0]) mbar_wait(smem_u32(&bars->qd_full[0]), (qd_arm[0] - 1) & 1, drain);
+      if (qd_arm[1]) mbar_wait(smem_u32(&bars->qd_full[1]), (qd_arm[1] - 1) & 1, drain);
+    }
+  } else if (warp == kWarpMma) {
+    if (lane == 0) {
+      const uint32_t idesc_ss = make_idesc_f16(128, 128, 0, 0);
+      const uint32_t idesc_ts = make_idesc_f16(128, 128, 0, 1);
+      uint32_t item_count = 0, qd_iter = 0, dv_count = 0, dk_count = 0, p_cnt = 0, ds_cnt = 0;
+      bool ok = true;
+      const uint32_t kt = sbase + kKvOffK, vt = sbase + kKvOffV;
+      for (int idx = blockIdx.x; idx < n_items && ok; idx += gridDim.x) {
+        const KvItem it = decode_kv(a, idx);
+        ok = mbar_wait(smem_u32(&bars->kv_full), item_count & 1, wc);
+        if (!ok) break;
+        tc_fence_after();
+        for (int m = 0; m < it.nq && ok; ++m, ++qd_iter) {
+          const uint32_t s = qd_iter & 1, ph = (qd_iter >> 1) & 1;
+          const uint32_t qt = sbase + kKvOffQ + s * kTileBytes;
+          const uint32_t dot = sbase + kKvOffDO + s * kTileBytes;
+          ok = mbar_wait(smem_u32(&bars->qd_full[s]), ph, wc);
+          if (!ok) break;
+          if (dv_count > 0) ok = mbar_wait(smem_u32(&bars->dv_done), (dv_count - 1) & 1, wc);
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ss(tmem + 0, kmajor_desc(kt, kk), kmajor_desc(qt, kk), idesc_ss, kk > 0);
+          mma_commit(smem_u32(&bars->s_full));
+          if (dk_count > 0) ok = mbar_wait(smem_u32(&bars->dk_done), (dk_count - 1) & 1, wc);
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ss(tmem + 128, kmajor_desc(vt, kk), kmajor_desc(dot, kk), idesc_ss, kk > 0);
+          mma_commit(smem_u32(&bars->dp_full));
+          ok = mbar_wait(smem_u32(&bars->p_full), p_cnt & 1, wc);
+          ++p_cnt;
+          if (!ok) break;
+          if (m == 0 && item_count > 0)
+            ok = mbar_wait(smem_u32(&bars->acc_empty), (item_count - 1) & 1, wc);
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ts(tmem + 256, tmem + 0 + kk * 8, mnmajor_desc(dot, kk), idesc_ts,
+                   (m > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(smem_u32(&bars->dv_done));
+          ++dv_count;
+          ok = mbar_wait(smem_u32(&bars->ds_full), ds_cnt & 1, wc);
+          ++ds_cnt;
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ts(tmem + 384, tmem + 128 + kk * 8, mnmajor_desc(qt, kk), idesc_ts,
+                   (m > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(smem_u32(&bars->dk_done));
+          ++dk_count;
+          mma_commit(smem_u32(&bars->qd_empty[s]));
+        }
+        if (!ok) break;
+        mma_commit(smem_u32(&bars->kv_empty));
+        mma_commit(smem_u32(&bars->acc_full));
+        ++item_count;
+      }
+      mma_commit(smem_u32(&bars->drain));
+      volatile int no_abort = 0;
+      const WaitCtx drain{&no_abort, a.status, kStatusTimeoutBwdKV};
+      mbar_wait(smem_u32(&bars->drain), 0, drain);
+    }
+  } else {
+    // ---------------------------------------------------------------- math warps
+    const int kl = warp * 32 + lane;               // key row of the tile = TMEM lane
+    const uint32_t t_row = tmem + ((uint32_t)(warp * 32) << 16);
+    uint32_t item_count = 0, s_cnt = 0, dp_cnt = 0, tile_count = 0;
+    bool ok = true;
+    for (int idx = blockIdx.x; idx < n_items && ok; idx += gridDim.x) {
+      const KvItem it = decode_kv(a, idx);
+      const int j = it.k0 + kl;
+      const bool valid_key = j < it.d1;
+      for (int m = 0; m < it.nq; ++m, ++tile_count) {
+        const int qs = it.k0 + m * a.R;
+        const uint32_t stg = tile_count & 1, ph = (tile_count >> 1) & 1;
+        const float* st = stats + stg * 256;
+        const bool needs_mask = (it.k0 + kTileKeys - 1 > qs) || (it.k0 + kTileKeys > it.d1) ||
+                                (qs + a.R > it.d1) || (a.W > 0 && qs + a.R - 1 - it.k0 >= a.W);
+        // the tile's statistics are in shared memory once qd_full completes
+        ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->qd_full[stg]), ph, wc));
+        if (!ok) break;
+        ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->s_full), s_cnt & 1, wc));
+        ++s_cnt;
+        if (!ok) break;
+        tc_fence_after();
+        uint32_t pk[64];
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          uint32_t u0[32], u1[32];
+          tmem_ld32(t_row + hf * 64, u0);
+          tmem_ld32(t_row + hf * 64 + 32, u1);
+          tc_wait_ld_dep(u0);
+          tc_wait_ld_dep(u1);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const int c = hf * 64 + 2 * e;
+            const float s0 = __uint_as_float(e < 16 ? u0[2 * e] : u1[2 * e - 32]);
+            const float s1 = __uint_as_float(e < 16 ? u0[2 * e + 1] : u1[2 * e - 31]);
+            float p0 = ex2_approx(fmaf(s0, a.scale_log2, -st[c]));
+            float p1 = ex2_approx(fmaf(s1, a.scale_log2, -st[c + 1]));
+            if (needs_mask) {
+              const int t0 = qs + (c >> a.logG), t1 = qs + ((c + 1) >> a.logG);
+              const bool v0 = valid_key && j <= t0 && t0 < it.d1 && (a.W <= 0 || t0 - j < a.W);
+              const bool v1 = valid_key && j <= t1 && t1 < it.d1 && (a.W <= 0 || t1 - j < a.W);
+              p0 = v0 ? p0 : 0.f;
+              p1 = v1 ? p1 : 0.f;
+            }
+            pk[hf * 32 + e] = pack_f16x2(p0, p1);
+          }
+        }
+        tmem_st32(t_row + 0, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
+        tmem_st32(t_row + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
+        tc_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&bars->p_full));
+        ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->dp_full), dp_cnt & 1, wc));
+        ++dp_cnt;
+        if (!ok) break;
+        tc_fence_after();
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          uint32_t u0[32], u1[32], ds[32];
+          tmem_ld32(t_row + 128 + hf * 64, u0);
+          tmem_ld32(t_row + 128 + hf * 64 + 32, u1);
+          tc_wait_ld_dep(u0);
+          tc_wait_ld_dep(u1);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const int c = hf * 64 + 2 * e;
+            const float d0 = __uint_as_float(e < 16 ? u0[2 * e] : u1[2 * e - 32]);
+            const float d1 = __uint_as_float(e < 16 ? u0[2 * e + 1] : u1[2 * e - 31]);
+            const float2 p = unpack_f16x2(pk[hf * 32 + e]);
+            ds[e] = pack_f16x2(p.x * (d0 - st[128 + c]), p.y * (d1 - st[128 + c + 1]));
+          }
+          // dS^T columns [hf*32, hf*32+32) of the fp16 region; this thread's
+          // dP^T row for these keys was fully read above.
+          tmem_st32(t_row + 128 + hf * 32, ds);
+        }
+        tc_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&bars->ds_full));
+      }
+      if (!ok) break;
+      ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->acc_full), item_count & 1, wc));
+      if (!ok) break;
+      tc_fence_after();
+      {
+        const size_t rb = ((size_t)j * a.Hk + it.g) * kHeadDim;
+        {  // dV: fp32 or bf16
+          float acc[128];
+          tmem_row128(t_row + 256, acc);
+          if (valid_key) {
+#pragma unroll
+            for (int c = 0; c < 128; c += 8) {
+              if (a.dv_f32) {
+                float* dvrow = reinterpret_cast<float*>(a.dv) + rb;
+                *reinterpret_cast<float4*>(dvrow + c) =
+                    make_float4(acc[c], acc[c + 1], acc[c + 2], acc[c + 3]);
+                *reinterpret_cast<float4*>(dvrow + c + 4) =
+                    make_float4(acc[c + 4], acc[c + 5], acc[c + 6], acc[c + 7]);
+              } else {
+                __nv_bfloat16* dvrow = reinterpret_cast<__nv_bfloat16*>(a.dv) + rb;
+                uint4 pkv;
+                pkv.x = pack_bf16x2(acc[c + 0], acc[c + 1]);
+                pkv.y = pack_bf16x2(acc[c + 2], acc[c + 3]);
+                pkv.z = pack_bf16x2(acc[c + 4], acc[c + 5]);
+                pkv.w = pack_bf16x2(acc[c + 6], acc[c + 7]);
+                *reinterpret_cast<uint4*>(dvrow + c) = pkv;
+              }
+            }
+          }
+        }
+        {  // dK_hat (scaled) into the fp32 workspace
+          float dkv[128];
+          tmem_row128(t_row + 384, dkv);
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(smem_u32(&bars->acc_empty));
+          if (valid_key) {
+            float* dkrow = a.dk_acc + rb;
+#pragma unroll
+            for (int c = 0; c < 128; c += 4)
+              *reinterpret_cast<float4*>(dkrow + c) =
+                  make_float4(dkv[c] * a.scale, dkv[c + 1] * a.scale, dkv[c + 2] * a.scale,
+                              dkv[c + 3] * a.scale);
+          }
+        }
+      }
+      ++item_count;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == kWarpMma) tmem_dealloc(tmem, 512);
+}
+
+// ============================================================================
+// dQ : query-major
+// ============================================================================
+struct __align__(8) QBars {
+  uint64_t qd_full, qd_empty;
+  uint64_t kv_full[2], kv_empty[2];
+  uint64_t s_full, dp_full, ds_full, dq_done, acc_full, acc_empty;
+  uint64_t drain;
+};
+constexpr uint32_t kQOffQ = 0;
+constexpr uint32_t kQOffDO = kTileBytes;
+constexpr uint32_t kQOffK = 2 * kTileBytes;                  // 2 stages
+constexpr uint32_t kQOffV = kQOffK + 2 * kTileBytes;         // 2 stages
+constexpr uint32_t kQOffBar = kQOffV + 2 * kTileBytes;
+constexpr uint32_t kQOffTmem = kQOffBar + sizeof(QBars);
+constexpr uint32_t kQOffAbort = kQOffTmem + 16;
+constexpr uint32_t kQSmem = kQOffAbort + 16 + 1024;
+
+struct QItem {
+  int q0, d0, d1, g, kend, kbeg, ntiles;
+};
+__device__ __forceinline__ QItem decode_q(const BwdArgs& a, int idx) {
+  const int4 it = a.items[idx];
+  QItem r;
+  r.q0 = it.x; r.d0 = it.y; r.d1 = it.z; r.g = it.w;
+  r.kend = min(r.q0 + a.R, r.d1);
+  r.kbeg = a.W > 0 ? max(r.d0, r.q0 - a.W + 1) : r.d0;
+  r.ntiles = (r.kend - r.kbeg + kTileKeys - 1) / kTileKeys;
+  return r;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q,
+                   const __grid_constant__ CUtensorMap tm_k,
+                   const __grid_constant__ CUtensorMap tm_v,
+                   const __grid_constant__ CUtensorMap tm_do, const BwdArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  QBars* bars = reinterpret_cast<QBars*>(smem + kQOffBar);
+  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + kQOffTmem);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kQOffAbort);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const WaitCtx wc{abort_flag, a.status, kStatusTimeoutBwdQ};
+
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    mbar_init(smem_u32(&bars->qd_full), 1);
+    mbar_init(smem_u32(&bars->qd_empty), 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(smem_u32(&bars->kv_full[s]), 1);
+      mbar_init(smem_u32(&bars->kv_empty[s]), 1);
+    }
+    mbar_init(smem_u32(&bars->s_full), 1);
+    mbar_init(smem_u32(&bars->dp_full), 1);
+    mbar_init(smem_u32(&bars->ds_full), 4);
+    mbar_init(smem_u32(&bars->dq_done), 1);
+    mbar_init(smem_u32(&bars->acc_full), 1);
+    mbar_init(smem_u32(&bars->acc_empty), 4);
+    mbar_init(smem_u32(&bars->drain), 1);
+    fence_mbar_init();
+  }
+  if (warp == kWarpMma) {
+    tmem_alloc(smem_u32((const void*)tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int n_items = min(*a.n_items, a.max_items);
+
+  if (warp == kWarpTma) {
+    if (lane == 0) {
+      uint32_t item_count = 0, kv_iter = 0, qd_arm = 0, kv_arm[2] = {0, 0};
+      bool ok = true;
+      for (int idx = blockIdx.x; idx < n_items && ok; idx += gridDim.x) {
+        const QItem it = decode_q(a, idx);
+        if (item_count > 0) ok = mbar_wait(smem_u32(&bars->qd_empty), (item_count - 1) & 1, wc);
+        if (!ok) break;
+        const uint32_t qf = smem_u32(&bars->qd_full);
+        mbar_arrive_expect_tx(qf, 2 * kTileBytes);
+        ++qd_arm;
+        for (int c = 0; c < 2; ++c) {
+          tma_load_3d(sbase + kQOffQ + c * kChunkBytes, &tm_q, qf, c * 64, it.g * a.G, it.q0);
+          tma_load_3d(sbase + kQOffDO + c * kChunkBytes, &tm_do, qf, c * 64, it.g * a.G, it.q0);
+        }
+        for (int n = 0; n < it.ntiles && ok; ++n, ++kv_iter) {
+          const int ks = it.kend - kTileKeys * (n + 1);
+          const uint32_t s = kv_iter & 1, ph = (kv_iter >> 1) & 1;
+          if (kv_iter >= 2) ok = mbar_wait(smem_u32(&bars->kv_empty[s]), ph ^ 1, wc);
+          if (!ok) break;
+          const uint32_t kf = smem_u32(&bars->kv_full[s]);
+          mbar_arrive_expect_tx(kf, 2 * kTileBytes);
+          ++kv_arm[s];
+          for (int c = 0; c < 2; ++c) {
+            tma_load_3d(sbase + kQOffK + s * kTileBytes + c * kChunkBytes, &tm_k, kf, c * 64, it.g,
+                        ks);
+            tma_load_3d(sbase + kQOffV + s * kTileBytes + c * kChunkBytes, &tm_v, kf, c * 64, it.g,
+                        ks);
+          }
+        }
+        ++item_count;
+      }
+      volatile int no_abort = 0;
+      const WaitCtx drain{&no_abort, a.status, kStatusTimeoutBwdQ};
+      if (qd_arm) mbar_wait(smem_u32(&bars->qd_full), (qd_arm - 1) & 1, drain);
+      if (kv_arm[0]) mbar_wait(smem_u32(&bars->kv_full[0]), (kv_arm[0] - 1) & 1, drain);
+      if (kv_arm[1]) mbar_wait(smem_u32(&bars->kv_full[1]), (kv_arm[1] - 1) & 1, drain);
+    }
+  } else if (warp == kWarpMma) {
+    if (lane == 0) {
+      const uint32_t idesc_ss = make_idesc_f16(128, 128, 0, 0);
+      const uint32_t idesc_ts = make_idesc_f16(128, 128, 0, 1);
+      uint32_t item_count = 0, kv_iter = 0, dq_count = 0, ds_cnt = 0;
+      bool ok = true;
+      const uint32_t qt = sbase + kQOffQ, dot = sbase + kQOffDO;
+      for (int idx = blockIdx.x; idx < n_items && ok; idx += gridDim.x) {
+        const QItem it = decode_q(a, idx);
+        ok = mbar_wait(smem_u32(&bars->qd_full), item_count & 1, wc);
+        if (!ok) break;
+        tc_fence_after();
+        for (int n = 0; n < it.ntiles && ok; ++n, ++kv_iter) {
+          const uint32_t s = kv_iter & 1, ph = (kv_iter >> 1) & 1;
+          const uint32_t kt = sbase + kQOffK + s * kTileBytes;
+          const uint32_t vt = sbase + kQOffV + s * kTileBytes;
+          ok = mbar_wait(smem_u32(&bars->kv_full[s]), ph, wc);
+          if (!ok) break;
+          if (dq_count > 0) ok = mbar_wait(smem_u32(&bars->dq_done), (dq_count - 1) & 1, wc);
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ss(tmem + 0, kmajor_desc(qt, kk), kmajor_desc(kt, kk), idesc_ss, kk > 0);
+          mma_commit(smem_u32(&bars->s_full));
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ss(tmem + 128, kmajor_desc(dot, kk), kmajor_desc(vt, kk), idesc_ss, kk > 0);
+          mma_commit(smem_u32(&bars->dp_full));
+          ok = mbar_wait(smem_u32(&bars->ds_full), ds_cnt & 1, wc);
+          ++ds_cnt;
+          if (!ok) break;
+          if (n == 0 && item_count > 0)
+            ok = mbar_wait(smem_u32(&bars->acc_empty), (item_count - 1) & 1, wc);
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ts(tmem + 256, tmem + 0 + kk * 8, mnmajor_desc(kt, kk), idesc_ts,
+                   (n > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(smem_u32(&bars->dq_done));
+          ++dq_count;
+          mma_commit(smem_u32(&bars->kv_empty[s]));
+        }
+        if (!ok) break;
+        mma_commit(smem_u32(&bars->qd_empty));
+        mma_commit(smem_u32(&bars->acc_full));
+        ++item_count;
+      }
+      mma_commit(smem_u32(&bars->drain));
+      volatile int no_abort = 0;
+      const WaitCtx drain{&no_abort, a.status, kStatusTimeoutBwdQ};
+      mbar_wait(smem_u32(&bars->drain), 0, drain);
+    }
+  } else {
+    // ---------------------------------------------------------------- math warps
+    const int r = warp * 32 + lane;                // query row of the tile = TMEM lane
+    const uint32_t t_row = tmem + ((uint32_t)(warp * 32) << 16);
+    uint32_t item_count = 0, s_cnt = 0, dp_cnt = 0;
+    bool ok = true;
+    for (int idx = blockIdx.x; idx < n_items && ok; idx += gridDim.x) {
+      const QItem it = decode_q(a, idx);
+      const int tok = it.q0 + r / a.G;
+      const int h = it.g * a.G + r % a.G;
+      const bool valid = tok < it.d1;
+      const int lo_r = a.W > 0 ? max(it.d0, tok - a.W + 1) : it.d0;
+      const float lse2 = valid ? __ldg(a.lse + (size_t)h * a.T + tok) * kLog2e : 0.f;
+      const float Di = valid ? __ldg(a.dvec + (size_t)h * a.T + tok) : 0.f;
+      for (int n = 0; n < it.ntiles; ++n) {
+        const int ks = it.kend - kTileKeys * (n + 1);
+        const bool needs_mask = (ks + kTileKeys - 1 > it.q0) || (ks < it.d0) ||
+                                (a.W > 0 && ks < it.q0 + a.R - a.W);
+        ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->s_full), s_cnt & 1, wc));
+        ++s_cnt;
+        if (!ok) break;
+        tc_fence_after();
+        uint32_t pk[64];
+        {
+          float sv[128];
+          tmem_row128(t_row + 0, sv);
+          const int c_lo = lo_r - ks, c_hi = tok - ks;
+#pragma unroll
+          for (int c = 0; c < 128; c += 2) {
+            float p0 = ex2_approx(fmaf(sv[c], a.scale_log2, -lse2));
+            float p1 = ex2_approx(fmaf(sv[c + 1], a.scale_log2, -lse2));
+            if (needs_mask) {
+              p0 = (valid && c >= c_lo && c <= c_hi) ? p0 : 0.f;
+              p1 = (valid && c + 1 >= c_lo && c + 1 <= c_hi) ? p1 : 0.f;
+            }
+            pk[c >> 1] = pack_f16x2(p0, p1);
+          }
+        }
+        ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->dp_full), dp_cnt & 1, wc));
+        ++dp_cnt;
+        if (!ok) break;
+        tc_fence_after();
+        {
+          float dp[128];
+          tmem_row128(t_row + 128, dp);
+          uint32_t ds[64];
+#pragma unroll
+          for (int c = 0; c < 128; c += 2) {
+            const float2 p = unpack_f16x2(pk[c >> 1]);
+            ds[c >> 1] = pack_f16x2(p.x * (dp[c] - Di), p.y * (dp[c + 1] - Di));
+          }
+          tmem_st32(t_row + 0, *reinterpret_cast<uint32_t(*)[32]>(&ds[0]));
+          tmem_st32(t_row + 32, *reinterpret_cast<uint32_t(*)[32]>(&ds[32]));
+        }
+        tc_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&bars->ds_full));
+      }
+      if (!ok) break;
+      ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->acc_full), item_count & 1, wc));
+      if (!ok) break;
+      tc_fence_after();
+      {
+        float acc[128];
+        tmem_row128(t_row + 256, acc);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&bars->acc_empty));
+        if (valid) {
+          float* row = a.dq_acc + ((size_t)tok * a.H + h) * kHeadDim;
+#pragma unroll
+          for (int c = 0; c < 128; c += 4)
+            *reinterpret_cast<float4*>(row + c) = make_float4(acc[c] * a.scale, acc[c + 1] * a.scale,
+                                                              acc[c + 2] * a.scale,
+                                                              acc[c + 3] * a.scale);
+        }
+      }
+      ++item_count;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == kWarpMma) tmem_dealloc(tmem, 512);
+}
+
+}  // namespace
+
+cudaError_t launch_attn_bwd_sm100_impl(const CUtensorMap& tq, const CUtensorMap& tk,
+                                       const CUtensorMap& tv, const CUtensorMap& tdo,
+                                       const Resolved& p, const float* lse, const float* dvec,
+                                       const int4* items_kv, const int* n_kv, int max_kv,
+                                       const int4* items_q, const int* n_q, int max_q,
+                                       float* dq_acc, float* dk_acc, void* dv, int* status,
+                                       int num_sms, cudaStream_t st) {
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(attn_bwd_dkv_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kKvSmem);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(attn_bwd_dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kQSmem);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  BwdArgs a;
+  a.T = p.T; a.H = p.H; a.Hk = p.Hk; a.G = p.G; a.R = p.R; a.W = p.W;
+  a.logG = 0;
+  while ((1 << a.logG) < p.G) ++a.logG;
+  a.scale = p.scale;
+  a.scale_log2 = p.scale * kLog2e;
+  a.lse = lse; a.dvec = dvec;
+  a.dq_acc = dq_acc; a.dk_acc = dk_acc;
+  a.dv = dv;
+  a.dv_f32 = p.fp32_grads || p.dtype == FLINT_FP32;
+  a.status = status;
+
+  a.items = items_kv; a.n_items = n_kv; a.max_items = max_kv;
+  int grid = num_sms < max_kv ? num_sms : max_kv;
+  {
+    ProfScope prof(kKBwdDkvSm100, st);
+    attn_bwd_dkv_kernel<<<grid > 0 ? grid : 1, kThreads, kKvSmem, st>>>(tq, tk, tv, tdo, a);
+  }
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+
+  a.items = items_q; a.n_items = n_q; a.max_items = max_q;
+  grid = num_sms < max_q ? num_sms : max_q;
+  ProfScope prof(kKBwdDqSm100, st);
+  attn_bwd_dq_kernel<<<grid > 0 ? grid : 1, kThreads, kQSmem, st>>>(tq, tk, tv, tdo, a);
+  return cudaGetLastError();
+}
+
 }  // namespace flint

@@ -276,6 +276,7 @@ cudaError_t launch_attn_fwd_fp32(const Resolved& p, const float* qh, const float
                                  float* lse, cudaStream_t st) {
   if (p.T == 0) return cudaSuccess;
   dim3 grid((p.T + kRows - 1) / kRows, p.H);
+  ProfScope prof(kKFwdFp32, st);
   fwd_fp32_kernel<<<grid, kThreads, 0, st>>>(qh, kh, v, sink, cu, p.N, p.T, p.H, p.Hk, p.W,
                                              p.scale, out, lse);
   return cudaGetLastError();
@@ -287,11 +288,15 @@ cudaError_t launch_attn_bwd_fp32(const Resolved& p, const float* qh, const float
                                  float* dk_acc, float* dv, cudaStream_t st) {
   if (p.T == 0) return cudaSuccess;
   dim3 gq((p.T + kRows - 1) / kRows, p.H);
-  bwd_dq_fp32_kernel<<<gq, kThreads, 0, st>>>(qh, kh, v, dout, lse, dvec, cu, p.N, p.T, p.H, p.Hk,
-                                              p.W, p.scale, dq_acc);
+  {
+    ProfScope prof(kKBwdDqFp32, st);
+    bwd_dq_fp32_kernel<<<gq, kThreads, 0, st>>>(qh, kh, v, dout, lse, dvec, cu, p.N, p.T, p.H,
+                                                p.Hk, p.W, p.scale, dq_acc);
+  }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   dim3 gk((p.T + kRows - 1) / kRows, p.Hk);
+  ProfScope prof(kKBwdDkvFp32, st);
   bwd_dkv_fp32_kernel<<<gk, kThreads, 0, st>>>(qh, kh, v, dout, lse, dvec, cu, p.N, p.T, p.H,
                                                p.Hk, p.W, p.scale, dk_acc, dv);
   return cudaGetLastError();

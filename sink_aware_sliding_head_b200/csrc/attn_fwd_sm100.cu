@@ -200,61 +200,105 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
     }
   } else if (warp == kWarpMma) {
     // ------------------------------------------------------------ MMA issuer
+    // Issue order per key tile n: PV0(n), QK0(n+1), PV1(n), QK1(n+1). Tile 1
+    // runs half a period behind tile 0, so each tile's softmax overlaps the
+    // other tile's MMAs. QK_i(n+1) overwrites S_i, which holds P_i(n), so it
+    // is issued only after PV_i(n) has completed.
     if (lane == 0) {
       const uint32_t idesc_qk = make_idesc_bf16(128, 128, 0, 0);
       const uint32_t idesc_pv = make_idesc_bf16(128, 128, 0, 1);
-      uint32_t kv_iter = 0, item_count = 0, pv_count[2] = {0, 0}, p_count[2] = {0, 0};
+      uint32_t kv_iter = 0, item_count = 0;
+      uint32_t pv0 = 0, pv1 = 0, pc0 = 0, pc1 = 0;   // PV commits / P arrivals seen, per tile
       bool ok = true;
+      const uint32_t q0t = sbase + kOffQ, q1t = sbase + kOffQ + kTileBytes;
       for (int idx = blockIdx.x; idx < n_items && ok; idx += gridDim.x) {
         const Item it = decode(a, idx);
         ok = mbar_wait(smem_u32(&bars->q_full), item_count & 1, wc);
         if (!ok) break;
         tc_fence_after();
-        for (int n = 0; n < it.ntiles && ok; ++n, ++kv_iter) {
+        {  // QK of the first key tile for both query tiles
           const uint32_t s = kv_iter % kStages, ph = (kv_iter / kStages) & 1;
           ok = mbar_wait(smem_u32(&bars->k_full[s]), ph, wc);
           if (!ok) break;
-          tc_fence_after();
           const uint32_t kt = sbase + kOffK + s * kTileBytes;
-          for (int i = 0; i < 2 && ok; ++i) {
-            if (pv_count[i] > 0) {
-              ok = mbar_wait(smem_u32(&bars->pv_done[i]), (pv_count[i] - 1) & 1, wc);
-              if (!ok) break;
-              tc_fence_after();
-            }
-            const uint32_t qt = sbase + kOffQ + i * kTileBytes;
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk)
-              mma_ss(tmem + i * 128, kmajor_desc(qt, kk), kmajor_desc(kt, kk), idesc_qk, kk > 0);
-            mma_commit(smem_u32(&bars->s_full[i]));
-          }
-          if (!ok) break;
-          mma_commit(smem_u32(&bars->k_empty[s]));
-          if (n == it.ntiles - 1) mma_commit(smem_u32(&bars->q_empty));
-          ok = mbar_wait(smem_u32(&bars->v_full[s]), ph, wc);
+          if (pv0 > 0) ok = mbar_wait(smem_u32(&bars->pv_done[0]), (pv0 - 1) & 1, wc);
           if (!ok) break;
           tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ss(tmem + 0, kmajor_desc(q0t, kk), kmajor_desc(kt, kk), idesc_qk, kk > 0);
+          mma_commit(smem_u32(&bars->s_full[0]));
+          if (pv1 > 0) ok = mbar_wait(smem_u32(&bars->pv_done[1]), (pv1 - 1) & 1, wc);
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ss(tmem + 128, kmajor_desc(q1t, kk), kmajor_desc(kt, kk), idesc_qk, kk > 0);
+          mma_commit(smem_u32(&bars->s_full[1]));
+          mma_commit(smem_u32(&bars->k_empty[s]));
+          if (it.ntiles == 1) mma_commit(smem_u32(&bars->q_empty));
+        }
+        for (int n = 0; n < it.ntiles; ++n) {
+          const uint32_t cur = kv_iter + n, nxt = cur + 1;
+          const uint32_t s = cur % kStages, ph = (cur / kStages) & 1;
+          const uint32_t s2 = nxt % kStages, ph2 = (nxt / kStages) & 1;
+          const bool has_next = n + 1 < it.ntiles;
           const uint32_t vt = sbase + kOffV + s * kTileBytes;
-          for (int i = 0; i < 2 && ok; ++i) {
-            ok = mbar_wait(smem_u32(&bars->p_full[i]), p_count[i] & 1, wc);
-            ++p_count[i];
+          const uint32_t kt2 = sbase + kOffK + s2 * kTileBytes;
+          ok = mbar_wait(smem_u32(&bars->v_full[s]), ph, wc);
+          if (ok && has_next) ok = mbar_wait(smem_u32(&bars->k_full[s2]), ph2, wc);
+          // ---- tile 0
+          if (ok) ok = mbar_wait(smem_u32(&bars->p_full[0]), pc0 & 1, wc);
+          ++pc0;
+          if (ok && n == 0 && item_count > 0)
+            ok = mbar_wait(smem_u32(&bars->o_empty[0]), (item_count - 1) & 1, wc);
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ts(tmem + 256, tmem + 0 + kk * 8, mnmajor_desc(vt, kk), idesc_pv,
+                   (n > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(smem_u32(&bars->pv_done[0]));
+          ++pv0;
+          if (!has_next) mma_commit(smem_u32(&bars->o_full[0]));
+          if (has_next) {
+            ok = mbar_wait(smem_u32(&bars->pv_done[0]), (pv0 - 1) & 1, wc);
             if (!ok) break;
-            if (n == 0 && item_count > 0) {
-              ok = mbar_wait(smem_u32(&bars->o_empty[i]), (item_count - 1) & 1, wc);
-              if (!ok) break;
-            }
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
-              mma_ts(tmem + 256 + i * 128, tmem + i * 128 + kk * 8, mnmajor_desc(vt, kk),
-                     idesc_pv, (n > 0 || kk > 0) ? 1u : 0u);
-            mma_commit(smem_u32(&bars->pv_done[i]));
-            ++pv_count[i];
-            if (n == it.ntiles - 1) mma_commit(smem_u32(&bars->o_full[i]));
+              mma_ss(tmem + 0, kmajor_desc(q0t, kk), kmajor_desc(kt2, kk), idesc_qk, kk > 0);
+            mma_commit(smem_u32(&bars->s_full[0]));
           }
+          // ---- tile 1
+          ok = mbar_wait(smem_u32(&bars->p_full[1]), pc1 & 1, wc);
+          ++pc1;
+          if (ok && n == 0 && item_count > 0)
+            ok = mbar_wait(smem_u32(&bars->o_empty[1]), (item_count - 1) & 1, wc);
           if (!ok) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ts(tmem + 384, tmem + 128 + kk * 8, mnmajor_desc(vt, kk), idesc_pv,
+                   (n > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(smem_u32(&bars->pv_done[1]));
+          ++pv1;
+          if (!has_next) mma_commit(smem_u32(&bars->o_full[1]));
           mma_commit(smem_u32(&bars->v_empty[s]));
+          if (has_next) {
+            ok = mbar_wait(smem_u32(&bars->pv_done[1]), (pv1 - 1) & 1, wc);
+            if (!ok) break;
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+              mma_ss(tmem + 128, kmajor_desc(q1t, kk), kmajor_desc(kt2, kk), idesc_qk, kk > 0);
+            mma_commit(smem_u32(&bars->s_full[1]));
+            mma_commit(smem_u32(&bars->k_empty[s2]));
+            if (n + 2 == it.ntiles) mma_commit(smem_u32(&bars->q_empty));
+          }
         }
+        if (!ok) break;
+        kv_iter += it.ntiles;
         ++item_count;
       }
       // Every MMA this thread issued has finished before TMEM is released.
@@ -287,36 +331,36 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         ++s_count;
         if (!ok) break;
         tc_fence_after();
-        float sv[128];
-        {
-          uint32_t u0[32], u1[32], u2[32], u3[32];
-          tmem_ld32(t_row + s_col + 0, u0);
-          tmem_ld32(t_row + s_col + 32, u1);
-          tmem_ld32(t_row + s_col + 64, u2);
-          tmem_ld32(t_row + s_col + 96, u3);
-          tc_wait_ld_dep(u0);
-          tc_wait_ld_dep(u1);
-          tc_wait_ld_dep(u2);
-          tc_wait_ld_dep(u3);
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            sv[e] = __uint_as_float(u0[e]);
-            sv[32 + e] = __uint_as_float(u1[e]);
-            sv[64 + e] = __uint_as_float(u2[e]);
-            sv[96 + e] = __uint_as_float(u3[e]);
-          }
-        }
         const bool needs_mask = (ks + kTileKeys - 1 > it.q0) || (ks < it.d0) ||
                                 (a.W > 0 && ks < it.q0 + 2 * a.R - a.W);
-        if (needs_mask) {
-          const int c_lo = lo_r - ks, c_hi = tok - ks;
+        const int c_lo = needs_mask ? lo_r - ks : 0;
+        const int c_hi = needs_mask ? tok - ks : 127;
+        // pass 1: row max over the 128 columns, two 64-column halves
+        float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
 #pragma unroll
-          for (int c = 0; c < 128; ++c)
-            if (c < c_lo || c > c_hi) sv[c] = -INFINITY;
+        for (int hf = 0; hf < 2; ++hf) {
+          uint32_t u0[32], u1[32];
+          tmem_ld32(t_row + s_col + hf * 64, u0);
+          tmem_ld32(t_row + s_col + hf * 64 + 32, u1);
+          tc_wait_ld_dep(u0);
+          tc_wait_ld_dep(u1);
+          if (needs_mask) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              const int c0 = hf * 64 + e, c1 = hf * 64 + 32 + e;
+              if (c0 < c_lo || c0 > c_hi) u0[e] = 0xff800000u;   // -inf
+              if (c1 < c_lo || c1 > c_hi) u1[e] = 0xff800000u;
+            }
+          }
+#pragma unroll
+          for (int e = 0; e < 32; e += 4) {
+            mx0 = fmax3(mx0, __uint_as_float(u0[e]), __uint_as_float(u0[e + 1]));
+            mx1 = fmax3(mx1, __uint_as_float(u0[e + 2]), __uint_as_float(u0[e + 3]));
+            mx2 = fmax3(mx2, __uint_as_float(u1[e]), __uint_as_float(u1[e + 1]));
+            mx3 = fmax3(mx3, __uint_as_float(u1[e + 2]), __uint_as_float(u1[e + 3]));
+          }
         }
-        float mx = sv[0];
-#pragma unroll
-        for (int c = 1; c < 128; ++c) mx = fmaxf(mx, sv[c]);
+        const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
         const float m_tile = mx * a.scale_log2;
         float alpha = 1.f;
         bool rescale_o = false;
@@ -329,32 +373,62 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         }
         l *= alpha;
         if (__any_sync(0xffffffffu, rescale_o)) {
-          // PV of the previous tile has completed (it was issued before this
-          // tile's QK, whose completion was just observed), so O is stable.
+          // PV of the previous tile has completed (the QK that produced this
+          // S was issued after it completed), so O is stable here.
+          const uint64_t a2 = f2(alpha, alpha);
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
             uint32_t u[32];
             tmem_ld32(t_row + o_col + c * 32, u);
             tc_wait_ld_dep(u);
 #pragma unroll
-            for (int e = 0; e < 32; ++e) u[e] = __float_as_uint(__uint_as_float(u[e]) * alpha);
+            for (int e = 0; e < 32; e += 2) {
+              float x0, x1;
+              f2_split(fmul2(f2(__uint_as_float(u[e]), __uint_as_float(u[e + 1])), a2), x0, x1);
+              u[e] = __float_as_uint(x0);
+              u[e + 1] = __float_as_uint(x1);
+            }
             tmem_st32(t_row + o_col + c * 32, u);
           }
         }
         const float mb = (m == -INFINITY) ? 0.f : m;
-        float rs = 0.f;
+        const uint64_t sc2 = f2(a.scale_log2, a.scale_log2);
+        const uint64_t nm2 = f2(-mb, -mb);
+        uint64_t rs2 = f2(0.f, 0.f);
+        // pass 2: P = 2^(s*scale - m) in bf16 over the first 64 columns of S.
+        // Half hf re-reads S columns [64hf, 64hf+64) and writes P columns
+        // [32hf, 32hf+32), which this thread has already read.
 #pragma unroll
         for (int hf = 0; hf < 2; ++hf) {
-          uint32_t pk[32];
+          uint32_t u0[32], u1[32], pk[32];
+          tmem_ld32(t_row + s_col + hf * 64, u0);
+          tmem_ld32(t_row + s_col + hf * 64 + 32, u1);
+          tc_wait_ld_dep(u0);
+          tc_wait_ld_dep(u1);
+          if (needs_mask) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              const int c0 = hf * 64 + e, c1 = hf * 64 + 32 + e;
+              if (c0 < c_lo || c0 > c_hi) u0[e] = 0xff800000u;
+              if (c1 < c_lo || c1 > c_hi) u1[e] = 0xff800000u;
+            }
+          }
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
-            const float p0 = ex2_approx(fmaf(sv[hf * 64 + 2 * e], a.scale_log2, -mb));
-            const float p1 = ex2_approx(fmaf(sv[hf * 64 + 2 * e + 1], a.scale_log2, -mb));
-            rs += p0 + p1;
+            const uint32_t a0 = e < 16 ? u0[2 * e] : u1[2 * e - 32];
+            const uint32_t a1 = e < 16 ? u0[2 * e + 1] : u1[2 * e - 31];
+            float x0, x1;
+            f2_split(ffma2(f2(__uint_as_float(a0), __uint_as_float(a1)), sc2, nm2), x0, x1);
+            const float p0 = ex2_approx(x0);
+            const float p1 = ex2_approx(x1);
+            rs2 = fadd2(rs2, f2(p0, p1));
             pk[e] = pack_bf16x2(p0, p1);
           }
           tmem_st32(t_row + s_col + hf * 32, pk);
         }
+        float rs_lo, rs_hi;
+        f2_split(rs2, rs_lo, rs_hi);
+        const float rs = rs_lo + rs_hi;
         l += rs;
         tc_wait_st();
         tc_fence_before();
@@ -425,6 +499,7 @@ cudaError_t launch_attn_fwd_sm100_impl(const CUtensorMap& tq, const CUtensorMap&
   int grid = num_sms;
   if (grid > max_items) grid = max_items;
   if (grid < 1) grid = 1;
+  ProfScope prof(kKFwdSm100, st);
   attn_fwd_sm100_kernel<<<grid, kThreads, kSmemBytes, st>>>(tq, tk, tv, a);
   return cudaGetLastError();
 }

@@ -21,11 +21,14 @@ constexpr int kThreads = 256;
 constexpr int kGroups = kThreads / 16;
 constexpr int kTok = 4;
 
+// Also writes an fp16 copy of dO (dout16, when non-null): the BF16 backward's
+// tensor-core operands are fp16.
 template <typename T>
 __global__ void __launch_bounds__(kThreads)
 bwd_pre_kernel(const T* __restrict__ out, const T* __restrict__ dout,
                const float* __restrict__ lse, const float* __restrict__ sink,
-               float* __restrict__ dvec, float* __restrict__ part, int ntok, int H) {
+               float* __restrict__ dvec, float* __restrict__ part, __half* __restrict__ dout16,
+               int ntok, int H) {
   extern __shared__ float acc[];   // [kGroups][H]
   const int lane16 = threadIdx.x & 15, grp = threadIdx.x >> 4;
   const int c0 = lane16 * 8;
@@ -43,6 +46,12 @@ bwd_pre_kernel(const T* __restrict__ out, const T* __restrict__ dout,
         const size_t base = ((size_t)t * H + h) * kHeadDim + c0;
         load8(out + base, a);
         load8(dout + base, b);
+        if (dout16) {
+          float s8[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) s8[e] = sat_f16(b[e]);
+          store8(dout16 + base, s8);
+        }
       } else {
 #pragma unroll
         for (int e = 0; e < 8; ++e) { a[e] = 0.f; b[e] = 0.f; }
@@ -66,11 +75,34 @@ bwd_pre_kernel(const T* __restrict__ out, const T* __restrict__ dout,
   }
 }
 
+// dst[i] = fp16(src[i]) for n elements (n a multiple of 8), saturating at +-65504.
+__global__ void convert_f16_kernel(const __nv_bfloat16* __restrict__ src, __half* __restrict__ dst,
+                                   size_t n8) {
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n8;
+       i += (size_t)gridDim.x * blockDim.x) {
+    float f[8];
+    load8(src + 8 * i, f);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) f[e] = sat_f16(f[e]);
+    store8(dst + 8 * i, f);
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_convert_f16(const __nv_bfloat16* src, __half* dst, size_t n, cudaStream_t st) {
+  const size_t n8 = n / 8;
+  if (n8 == 0) return cudaSuccess;
+  size_t blocks = (n8 + 255) / 256;
+  if (blocks > 148 * 16) blocks = 148 * 16;
+  ProfScope prof(kKConvert, st);
+  convert_f16_kernel<<<(unsigned)blocks, 256, 0, st>>>(src, dst, n8);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_bwd_preprocess(const Resolved& p, const void* out, const void* dout,
                                   const float* lse, const float* sink, float* dvec, float* part,
-                                  float* dsink, cudaStream_t st) {
+                                  float* dsink, __half* dout16, cudaStream_t st) {
   if (p.T == 0) {
     cudaMemsetAsync(dsink, 0, p.H * sizeof(float), st);
     return cudaGetLastError();
@@ -78,12 +110,17 @@ cudaError_t launch_bwd_preprocess(const Resolved& p, const void* out, const void
   int blocks = (p.T + kTok - 1) / kTok;
   if (blocks > kPartBlocks) blocks = kPartBlocks;
   const size_t smem = (size_t)kGroups * p.H * sizeof(float);
+  {
+  ProfScope prof(kKBwdPre, st);
   if (p.dtype == FLINT_BF16)
     bwd_pre_kernel<__nv_bfloat16><<<blocks, kThreads, smem, st>>>(
-        (const __nv_bfloat16*)out, (const __nv_bfloat16*)dout, lse, sink, dvec, part, p.T, p.H);
+        (const __nv_bfloat16*)out, (const __nv_bfloat16*)dout, lse, sink, dvec, part, dout16,
+        p.T, p.H);
   else
     bwd_pre_kernel<float><<<blocks, kThreads, smem, st>>>((const float*)out, (const float*)dout,
-                                                          lse, sink, dvec, part, p.T, p.H);
+                                                          lse, sink, dvec, part, nullptr, p.T,
+                                                          p.H);
+  }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   return launch_reduce_rows(part, blocks, p.H, dsink, st);

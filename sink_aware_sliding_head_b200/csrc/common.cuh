@@ -5,6 +5,7 @@
 #include <cstddef>
 #include <cstdint>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include "../../include/flint_attn.h"
@@ -27,6 +28,7 @@ struct Resolved {
   int T, N, H, Hk, D, G, W, rope;
   float theta, eps, scale;
   int dtype;
+  int fp32_grads;   // dq, dk, dv written as float32 (always for FP32 inputs)
   int R;            // tokens per 128-row tile = 128 / G
 };
 
@@ -42,6 +44,8 @@ struct WsLayout {
   size_t part;          // fp32 partial sums (d sink, d norm weights)
   size_t dq_acc;        // [T,H,D] fp32 gradient w.r.t. q_hat (backward)
   size_t dk_acc;        // [T,Hk,D] fp32 gradient w.r.t. k_hat (backward)
+  size_t dout16;        // [T,H,D] fp16 copy of dO (backward, BF16 inputs)
+  size_t v16;           // [T,Hk,D] fp16 copy of v (backward, BF16 inputs)
   size_t total;
   int max_items_q, max_items_q1, max_items_kv, max_items_any;
   int part_blocks;      // number of partial-sum rows per reduced quantity
@@ -77,6 +81,10 @@ inline WsLayout make_layout(const Resolved& p, bool backward) {
     L.part = take((size_t)kPartBlocks * (p.H + 2 * p.D) * 4);
     L.dq_acc = take((size_t)p.T * p.H * p.D * 4);
     L.dk_acc = take((size_t)p.T * p.Hk * p.D * 4);
+    if (p.dtype == FLINT_BF16) {
+      L.dout16 = take((size_t)p.T * p.H * p.D * 2);
+      L.v16 = take((size_t)p.T * p.Hk * p.D * 2);
+    }
   }
   L.total = off;
   return L;
@@ -127,18 +135,45 @@ __device__ __forceinline__ void store8(__nv_bfloat16* p, const float (&f)[8]) {
   for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(f[2 * i], f[2 * i + 1]);
   *reinterpret_cast<uint4*>(p) = u;
 }
+__device__ __forceinline__ void store8(__half* p, const float (&f)[8]) {
+  uint4 u;
+  __half2* h = reinterpret_cast<__half2*>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) h[i] = __floats2half2_rn(f[2 * i], f[2 * i + 1]);
+  *reinterpret_cast<uint4*>(p) = u;
+}
+// fp16 range: values beyond +-65504 saturate instead of becoming infinite
+__device__ __forceinline__ float sat_f16(float x) { return fminf(fmaxf(x, -65504.f), 65504.f); }
 __device__ __forceinline__ void store8(float* p, const float (&f)[8]) {
   *reinterpret_cast<float4*>(p) = make_float4(f[0], f[1], f[2], f[3]);
   *reinterpret_cast<float4*>(p + 4) = make_float4(f[4], f[5], f[6], f[7]);
 }
+
+// ------------------------------------------------------------------ kernel timing
+// Every kernel launch of the library sits inside a ProfScope: it counts the
+// launch and, when profiling is enabled, records a CUDA event pair around it
+// on the launching stream (see flint_attn_profile_* in the public header).
+enum KernelId {
+  kKPrologue = 0, kKWorklist, kKFwdSm100, kKFwdFp32, kKBwdPre, kKReduce, kKBwdDkvSm100,
+  kKBwdDqSm100, kKBwdDqFp32, kKBwdDkvFp32, kKPrologueBwd, kKConvert, kNumKernelIds
+};
+struct ProfScope {
+  int id;
+  cudaStream_t st;
+  int slot;
+  ProfScope(int id, cudaStream_t st);
+  ~ProfScope();
+};
 
 // ------------------------------------------------------------------ launchers
 // (defined in the .cu files; all return cudaGetLastError() of their launch)
 cudaError_t launch_build_worklist(const int32_t* cu, const Resolved& p, int mode, int span,
                                   int4* items, int* count, void* tmp, int max_items,
                                   cudaStream_t st);
+// out_f16: write x_hat as fp16 (backward operands of BF16 inputs) instead of the input type
 cudaError_t launch_prologue(const Resolved& p, const void* x, const void* w, void* y, int heads,
-                            const int32_t* cu, cudaStream_t st);
+                            const int32_t* cu, cudaStream_t st, bool out_f16 = false);
+cudaError_t launch_convert_f16(const __nv_bfloat16* src, __half* dst, size_t n, cudaStream_t st);
 cudaError_t launch_attn_fwd_fp32(const Resolved& p, const float* qh, const float* kh,
                                  const float* v, const float* sink, const int32_t* cu, float* out,
                                  float* lse, cudaStream_t st);
@@ -148,7 +183,7 @@ cudaError_t launch_attn_bwd_fp32(const Resolved& p, const float* qh, const float
                                  float* dk_acc, float* dv, cudaStream_t st);
 cudaError_t launch_bwd_preprocess(const Resolved& p, const void* out, const void* dout,
                                   const float* lse, const float* sink, float* dvec, float* part,
-                                  float* dsink, cudaStream_t st);
+                                  float* dsink, __half* dout16, cudaStream_t st);
 cudaError_t launch_bwd_epilogue(const Resolved& p, const void* x, const void* w,
                                 const float* g_hat, void* dx, float* dw, float* part, int heads,
                                 const int32_t* cu, cudaStream_t st);

@@ -46,9 +46,9 @@ __device__ void build_rope_table(const int32_t* __restrict__ cu, int N, int T, i
   __syncthreads();
 }
 
-template <typename T>
+template <typename T, typename TO>
 __global__ void __launch_bounds__(kThreads)
-prologue_kernel(const T* __restrict__ x, const T* __restrict__ w, T* __restrict__ y, int ntok,
+prologue_kernel(const T* __restrict__ x, const T* __restrict__ w, TO* __restrict__ y, int ntok,
                 int heads, const int32_t* __restrict__ cu, int N, int rope, float theta,
                 float eps) {
   __shared__ float cs[kTok][kHalf], sn[kTok][kHalf];
@@ -105,10 +105,10 @@ prologue_kernel(const T* __restrict__ x, const T* __restrict__ w, T* __restrict_
 // Gradient of the prologue. g_hat: fp32 gradient w.r.t. the normalised (and
 // rotated) rows. dx = r*u - x*r^3*(1/D)*sum(u*x) with u = RoPE^T(g_hat)*w and
 // r = (mean x^2 + eps)^-1/2; partial d w = sum over rows of RoPE^T(g_hat)*x*r.
-template <typename T>
+template <typename T, typename TD>
 __global__ void __launch_bounds__(kThreads)
 prologue_bwd_kernel(const T* __restrict__ x, const T* __restrict__ w,
-                    const float* __restrict__ g_hat, T* __restrict__ dx,
+                    const float* __restrict__ g_hat, TD* __restrict__ dx,
                     float* __restrict__ dw_part, int ntok, int heads,
                     const int32_t* __restrict__ cu, int N, int rope, float theta, float eps) {
   __shared__ float cs[kTok][kHalf], sn[kTok][kHalf];
@@ -199,16 +199,20 @@ __global__ void reduce_rows_kernel(const float* __restrict__ part, int nrows, in
 }  // namespace
 
 cudaError_t launch_prologue(const Resolved& p, const void* x, const void* w, void* y, int heads,
-                            const int32_t* cu, cudaStream_t st) {
+                            const int32_t* cu, cudaStream_t st, bool out_f16) {
   if (p.T == 0) return cudaSuccess;
   dim3 grid((p.T + kTok - 1) / kTok);
-  if (p.dtype == FLINT_BF16)
-    prologue_kernel<__nv_bfloat16><<<grid, kThreads, 0, st>>>(
-        (const __nv_bfloat16*)x, (const __nv_bfloat16*)w, (__nv_bfloat16*)y, p.T, heads, cu, p.N,
-        p.rope, p.theta, p.eps);
+  ProfScope prof(kKPrologue, st);
+  typedef __nv_bfloat16 bf;
+  if (p.dtype == FLINT_BF16 && out_f16)
+    prologue_kernel<bf, __half><<<grid, kThreads, 0, st>>>(
+        (const bf*)x, (const bf*)w, (__half*)y, p.T, heads, cu, p.N, p.rope, p.theta, p.eps);
+  else if (p.dtype == FLINT_BF16)
+    prologue_kernel<bf, bf><<<grid, kThreads, 0, st>>>(
+        (const bf*)x, (const bf*)w, (bf*)y, p.T, heads, cu, p.N, p.rope, p.theta, p.eps);
   else
-    prologue_kernel<float><<<grid, kThreads, 0, st>>>((const float*)x, (const float*)w, (float*)y,
-                                                      p.T, heads, cu, p.N, p.rope, p.theta, p.eps);
+    prologue_kernel<float, float><<<grid, kThreads, 0, st>>>(
+        (const float*)x, (const float*)w, (float*)y, p.T, heads, cu, p.N, p.rope, p.theta, p.eps);
   return cudaGetLastError();
 }
 
@@ -222,22 +226,32 @@ cudaError_t launch_bwd_epilogue(const Resolved& p, const void* x, const void* w,
     cudaMemsetAsync(dw, 0, kHeadDim * sizeof(float), st);
     return cudaGetLastError();
   }
-  if (p.dtype == FLINT_BF16)
-    prologue_bwd_kernel<__nv_bfloat16><<<blocks, kThreads, 0, st>>>(
-        (const __nv_bfloat16*)x, (const __nv_bfloat16*)w, g_hat, (__nv_bfloat16*)dx, part, p.T,
-        heads, cu, p.N, p.rope, p.theta, p.eps);
+  {
+  ProfScope prof(kKPrologueBwd, st);
+  typedef __nv_bfloat16 bf;
+  if (p.dtype == FLINT_BF16 && p.fp32_grads)
+    prologue_bwd_kernel<bf, float><<<blocks, kThreads, 0, st>>>(
+        (const bf*)x, (const bf*)w, g_hat, (float*)dx, part, p.T, heads, cu, p.N, p.rope, p.theta,
+        p.eps);
+  else if (p.dtype == FLINT_BF16)
+    prologue_bwd_kernel<bf, bf><<<blocks, kThreads, 0, st>>>(
+        (const bf*)x, (const bf*)w, g_hat, (bf*)dx, part, p.T, heads, cu, p.N, p.rope, p.theta,
+        p.eps);
   else
-    prologue_bwd_kernel<float><<<blocks, kThreads, 0, st>>>((const float*)x, (const float*)w,
-                                                            g_hat, (float*)dx, part, p.T, heads,
-                                                            cu, p.N, p.rope, p.theta, p.eps);
+    prologue_bwd_kernel<float, float><<<blocks, kThreads, 0, st>>>(
+        (const float*)x, (const float*)w, g_hat, (float*)dx, part, p.T, heads, cu, p.N, p.rope,
+        p.theta, p.eps);
+  }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
+  ProfScope prof(kKReduce, st);
   reduce_rows_kernel<<<1, kHeadDim, 0, st>>>(part, blocks, kHeadDim, dw);
   return cudaGetLastError();
 }
 
 cudaError_t launch_reduce_rows(const float* part, int nrows, int width, float* out,
                                cudaStream_t st) {
+  ProfScope prof(kKReduce, st);
   reduce_rows_kernel<<<(width + 127) / 128, 128, 0, st>>>(part, nrows, width, out);
   return cudaGetLastError();
 }

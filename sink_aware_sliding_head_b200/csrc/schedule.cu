@@ -143,6 +143,7 @@ cudaError_t launch_build_worklist(const int32_t* cu, const Resolved& p, int mode
                                   cudaStream_t st) {
   int4* tmp_items = reinterpret_cast<int4*>(tmp);
   int* tmp_cost = reinterpret_cast<int*>(tmp_items + max_items);
+  ProfScope prof(kKWorklist, st);
   build_worklist_kernel<<<1, kThreads, 0, st>>>(cu, p.N, mode, span, p.W, p.R, p.Hk, items, count,
                                                 tmp_items, tmp_cost, max_items);
   return cudaGetLastError();

@@ -25,7 +25,9 @@ STATUS = {0: "FLINT_OK", 1: "FLINT_ERR_INVALID_ARG", 2: "FLINT_ERR_UNSUPPORTED",
           3: "FLINT_ERR_WORKSPACE", 4: "FLINT_ERR_CUDA", 5: "FLINT_ERR_TIMEOUT"}
 
 EXPORTED = ["flint_attn_workspace_bytes", "flint_attn_fwd", "flint_attn_bwd",
-            "flint_attn_check_status", "flint_status_string", "flint_attn_version"]
+            "flint_attn_check_status", "flint_status_string", "flint_attn_version",
+            "flint_attn_profile_enable", "flint_attn_profile_collect",
+            "flint_attn_profile_reset", "flint_attn_launch_count"]
 
 
 class Params(ctypes.Structure):
@@ -42,6 +44,7 @@ class Params(ctypes.Structure):
         ("rms_eps", ctypes.c_float),
         ("softmax_scale", ctypes.c_float),
         ("dtype", ctypes.c_int32),
+        ("fp32_grads", ctypes.c_int32),
     ]
 
 
@@ -77,15 +80,26 @@ def load_library(path: str = LIB_PATH):
     lib.flint_status_string.restype = ctypes.c_char_p
     lib.flint_attn_version.argtypes = []
     lib.flint_attn_version.restype = ctypes.c_char_p
+    lib.flint_attn_profile_enable.argtypes = [ctypes.c_int]
+    lib.flint_attn_profile_enable.restype = None
+    lib.flint_attn_profile_collect.argtypes = [ctypes.c_int, ctypes.POINTER(ctypes.c_char_p),
+                                               ctypes.POINTER(ctypes.c_double),
+                                               ctypes.POINTER(ctypes.c_longlong)]
+    lib.flint_attn_profile_collect.restype = ctypes.c_int
+    lib.flint_attn_profile_reset.argtypes = []
+    lib.flint_attn_profile_reset.restype = None
+    lib.flint_attn_launch_count.argtypes = []
+    lib.flint_attn_launch_count.restype = ctypes.c_longlong
     _lib = lib
     return lib
 
 
 def make_params(total_tokens, num_docs, num_q_heads, num_kv_heads, window, use_rope,
-                rope_theta, dtype, head_dim=128, rms_eps=1e-6, softmax_scale=0.0) -> Params:
+                rope_theta, dtype, head_dim=128, rms_eps=1e-6, softmax_scale=0.0,
+                fp32_grads=False) -> Params:
     return Params(int(total_tokens), int(num_docs), int(num_q_heads), int(num_kv_heads),
                   int(head_dim), int(window), 1 if use_rope else 0, float(rope_theta),
-                  float(rms_eps), float(softmax_scale), int(dtype))
+                  float(rms_eps), float(softmax_scale), int(dtype), 1 if fp32_grads else 0)
 
 
 def _ptr(t: Optional[torch.Tensor]):
@@ -111,10 +125,11 @@ def _check(code: int, where: str):
 
 
 def params_for(q, k, cu_doc_lens, window, use_rope, rope_theta, rms_eps=1e-6,
-               softmax_scale=0.0) -> Params:
+               softmax_scale=0.0, fp32_grads=False) -> Params:
     T, H, D = q.shape
     return make_params(T, cu_doc_lens.numel() - 1, H, k.shape[1], window, use_rope, rope_theta,
-                       _dtype_code(q), head_dim=D, rms_eps=rms_eps, softmax_scale=softmax_scale)
+                       _dtype_code(q), head_dim=D, rms_eps=rms_eps, softmax_scale=softmax_scale,
+                       fp32_grads=fp32_grads)
 
 
 def workspace_bytes(params: Params, backward: bool) -> int:
@@ -153,17 +168,22 @@ def fwd(q, k, v, q_norm_w, k_norm_w, sink, cu_doc_lens, window, use_rope, rope_t
 
 def bwd(q, k, v, q_norm_w, k_norm_w, sink, cu_doc_lens, out, lse, dout, window, use_rope,
         rope_theta, rms_eps=1e-6, softmax_scale=0.0, grads=None, workspace=None, stream=None,
-        check_status=False):
+        check_status=False, fp32_grads=False):
     """Backward through ``flint_attn_bwd``.
 
-    Returns a dict with dq, dk, dv (input dtype), dw_q, dw_k, dsink (fp32).
+    Returns a dict with dq, dk, dv (input dtype, or float32 with ``fp32_grads``),
+    dw_q, dw_k, dsink (fp32).
     """
     lib = load_library()
-    p = params_for(q, k, cu_doc_lens, window, use_rope, rope_theta, rms_eps, softmax_scale)
+    p = params_for(q, k, cu_doc_lens, window, use_rope, rope_theta, rms_eps, softmax_scale,
+                   fp32_grads)
     T, H, D = q.shape
+    gdt = torch.float32 if (fp32_grads or q.dtype == torch.float32) else q.dtype
     if grads is None:
         grads = {
-            "dq": torch.empty_like(q), "dk": torch.empty_like(k), "dv": torch.empty_like(v),
+            "dq": torch.empty(q.shape, dtype=gdt, device=q.device),
+            "dk": torch.empty(k.shape, dtype=gdt, device=q.device),
+            "dv": torch.empty(v.shape, dtype=gdt, device=q.device),
             "dw_q": torch.empty(D, dtype=torch.float32, device=q.device),
             "dw_k": torch.empty(D, dtype=torch.float32, device=q.device),
             "dsink": torch.empty(H, dtype=torch.float32, device=q.device),
@@ -180,6 +200,31 @@ def bwd(q, k, v, q_norm_w, k_norm_w, sink, cu_doc_lens, out, lse, dout, window, 
     if check_status:
         _check(lib.flint_attn_check_status(_ptr(workspace), st), "flint_attn_bwd (device)")
     return grads
+
+
+def profile_enable(on: bool = True):
+    """Bracket each later kernel launch with CUDA events on its stream."""
+    load_library().flint_attn_profile_enable(1 if on else 0)
+
+
+def profile_reset():
+    load_library().flint_attn_profile_reset()
+
+
+def profile_collect():
+    """{kernel name: (total ms, launches)} over the launches timed so far."""
+    lib = load_library()
+    n = 32
+    names = (ctypes.c_char_p * n)()
+    ms = (ctypes.c_double * n)()
+    cnt = (ctypes.c_longlong * n)()
+    k = lib.flint_attn_profile_collect(n, names, ms, cnt)
+    return {names[i].decode(): (ms[i], cnt[i]) for i in range(min(k, n))}
+
+
+def launch_count() -> int:
+    """Kernels the library has launched since it was loaded."""
+    return int(load_library().flint_attn_launch_count())
 
 
 def version() -> str:

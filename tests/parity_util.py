@@ -20,8 +20,14 @@ def f64(t):
     return t.detach().to("cpu").double().numpy() if torch.is_tensor(t) else np.asarray(t, np.float64)
 
 
-def compare(gpu, ref, dtype, name=""):
-    """Assert the parity bar; returns (max_abs, rel_rms)."""
+def compare(gpu, ref, dtype, name="", out_bf16=False):
+    """Assert the parity bar; returns (max_abs, rel_rms).
+
+    out_bf16: the GPU result is stored in bfloat16 and compared as such. Rounding
+    to bfloat16 alone moves a value by up to 2^-9 of its magnitude (half an ulp),
+    which exceeds 2e-2 for |values| > ~10; the bar then becomes
+    2e-2 + 2^-8 |ref| per element (the stated bar plus one bf16 ulp).
+    """
     g = f64(gpu)
     r = np.asarray(ref, dtype=np.float64)
     assert g.shape == r.shape, (name, g.shape, r.shape)
@@ -32,6 +38,11 @@ def compare(gpu, ref, dtype, name=""):
     rel_rms = float(np.sqrt(np.mean(err * err)) / denom) if r.size and denom > 0 else 0.0
     if dtype == "fp32":
         assert max_abs <= FP32_MAX_ABS, f"{name}: max_abs {max_abs:.3e}"
+    elif out_bf16:
+        bound = BF16_MAX_ABS + np.abs(r) * 2.0 ** -8
+        worst = float(np.max(np.abs(err) - bound)) if err.size else -1.0
+        assert worst <= 0, f"{name}: exceeds 2e-2 + 2^-8|ref| by {worst:.3e} (max_abs {max_abs:.3e})"
+        assert rel_rms <= BF16_REL_RMS, f"{name}: rel_rms {rel_rms:.3e}"
     else:
         assert max_abs <= BF16_MAX_ABS, f"{name}: max_abs {max_abs:.3e}"
         assert rel_rms <= BF16_REL_RMS, f"{name}: rel_rms {rel_rms:.3e}"
@@ -43,6 +54,7 @@ def run_fwd(fa, d, window, rope, theta, check=True):
                   window, rope, theta, check_status=check)
 
 
-def run_bwd(fa, d, out, lse, window, rope, theta, check=True):
+def run_bwd(fa, d, out, lse, window, rope, theta, check=True, fp32_grads=True):
     return fa.bwd(d["q"], d["k"], d["v"], d["w_q"], d["w_k"], d["sink"], d["cu_doc_lens"],
-                  out, lse, d["dout"], window, rope, theta, check_status=check)
+                  out, lse, d["dout"], window, rope, theta, check_status=check,
+                  fp32_grads=fp32_grads)

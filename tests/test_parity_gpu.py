@@ -138,3 +138,107 @@ def test_bf16_sliding_forward_full_oracle(cuda_lib):
     O, L, _ = oracle_full(cpu, wl, False)
     compare(out, O, "bf16", "out")
     compare(lse, L, "bf16", "lse")
+
+
+# ----------------------------------------------------------------------- BF16 backward
+
+BWD_CASES = [c for i, c in enumerate(SMALL_CASES) if i in (0, 1, 2, 3, 5, 7, 9, 10)]
+
+
+@pytest.mark.parametrize("lens,H,Hk,W,rope", BWD_CASES)
+def test_bf16_backward_small(cuda_lib, lens, H, Hk, W, rope):
+    cpu = fi.make_custom(lens, H, Hk, dtype="bf16", seed=len(lens) * 11 + W % 89)
+    d = to_dev(cpu)
+    out, lse = run_fwd(cuda_lib, d, W, rope, 1e6)
+    g = run_bwd(cuda_lib, d, out, lse, W, rope, 1e6)
+    torch.cuda.synchronize()
+    ref = fo.flint_attn_bwd(cpu["q"], cpu["k"], cpu["v"], cpu["w_q"], cpu["w_k"], cpu["sink"],
+                            cpu["cu_doc_lens"], W, rope, 1e6, cpu["dout"])
+    for name in ["dq", "dk", "dv", "dw_q", "dw_k", "dsink"]:
+        compare(g[name], ref[name], "bf16", name)
+
+
+def test_bf16_backward_bf16_gradients(cuda_lib):
+    """Gradients stored in bfloat16: the stated bar plus one bf16 ulp of the value."""
+    lens, H, Hk, W, rope = [300, 77], 32, 4, 96, True
+    cpu = fi.make_custom(lens, H, Hk, dtype="bf16", seed=21)
+    d = to_dev(cpu)
+    out, lse = run_fwd(cuda_lib, d, W, rope, 1e6)
+    g = run_bwd(cuda_lib, d, out, lse, W, rope, 1e6, fp32_grads=False)
+    torch.cuda.synchronize()
+    assert g["dq"].dtype == torch.bfloat16 and g["dv"].dtype == torch.bfloat16
+    ref = fo.flint_attn_bwd(cpu["q"], cpu["k"], cpu["v"], cpu["w_q"], cpu["w_k"], cpu["sink"],
+                            cpu["cu_doc_lens"], W, rope, 1e6, cpu["dout"])
+    for name in ["dq", "dk", "dv"]:
+        compare(g[name], ref[name], "bf16", name, out_bf16=True)
+    for name in ["dw_q", "dw_k", "dsink"]:
+        compare(g[name], ref[name], "bf16", name)
+
+
+def test_bf16_backward_is_deterministic(cuda_lib):
+    cpu = fi.make_custom([500, 260], 32, 4, dtype="bf16", seed=9)
+    d = to_dev(cpu)
+    out, lse = run_fwd(cuda_lib, d, 200, True, 1e6)
+    g1 = run_bwd(cuda_lib, d, out, lse, 200, True, 1e6)
+    g1 = {k: v.clone() for k, v in g1.items()}
+    g2 = run_bwd(cuda_lib, d, out, lse, 200, True, 1e6)
+    for k in g1:
+        assert torch.equal(g1[k], g2[k]), k
+
+
+def _prefix(cpu, n_tok, n_docs):
+    p = {k: (v[:n_tok] if torch.is_tensor(v) and v.dim() == 3 else v) for k, v in cpu.items()}
+    p["cu_doc_lens"] = cpu["cu_doc_lens"][:n_docs + 1].clone()
+    p["cu_doc_lens"][-1] = n_tok
+    p["doc_lens"] = None
+    return p
+
+
+@pytest.mark.parametrize("wl", [fi.PACKED_BF16, fi.LONG_FULL_BF16], ids=lambda w: w.name)
+def test_bf16_backward_full_size_sampled(cuda_lib, wl):
+    cpu = fi.make_inputs(wl)
+    d = to_dev(cpu)
+    out, lse = run_fwd(cuda_lib, d, wl.window, wl.use_rope, wl.rope_theta)
+    g = run_bwd(cuda_lib, d, out, lse, wl.window, wl.use_rope, wl.rope_theta)
+    torch.cuda.synchronize()
+    for name in ["dq", "dk", "dv", "dw_q", "dw_k", "dsink"]:
+        assert torch.isfinite(g[name]).all(), name
+    ro = fo.RowOracle(cpu["q"], cpu["k"], cpu["v"], cpu["w_q"], cpu["w_k"], cpu["sink"],
+                      cpu["cu_doc_lens"], wl.window, wl.use_rope, wl.rope_theta, dO=cpu["dout"])
+    rows = sample_rows(cpu["cu_doc_lens"], wl.num_q_heads, 24, seed=2)
+    compare(torch.stack([g["dq"][t, h] for t, h in rows]),
+            np.stack([ro.dq_row(t, h) for t, h in rows]), "bf16", "dq rows")
+    T = wl.total_tokens
+    cu = [int(c) for c in cpu["cu_doc_lens"]]
+    # key rows whose viewing queries are few enough for the oracle: the ends of documents
+    offs = (0, 3, 40) if wl.window > 0 else (0, 5)
+    keys = [(b - 1 - o, kv) for b in cu[1:4] for o in offs for kv in (0, 3)]
+    keys = [(j, kv) for j, kv in keys if 0 <= j < T]
+    ref = [ro.dkv_row(j, kv) for j, kv in keys]
+    compare(torch.stack([g["dk"][j, kv] for j, kv in keys]), np.stack([r[0] for r in ref]),
+            "bf16", "dk rows")
+    compare(torch.stack([g["dv"][j, kv] for j, kv in keys]), np.stack([r[1] for r in ref]),
+            "bf16", "dv rows")
+
+
+@pytest.mark.parametrize("wl,n_tok,n_docs", [(fi.LONG_FULL_BF16, 4096, 1),
+                                             (fi.PACKED_BF16, None, 2)],
+                         ids=["long_full_prefix4096", "packed_first2docs"])
+def test_bf16_backward_prefix_whole_layer(cuda_lib, wl, n_tok, n_docs):
+    """d_sink, d norm weights and every gradient element on a prefix of the workload."""
+    cpu = fi.make_inputs(wl)
+    if n_tok is None:
+        n_tok = int(cpu["cu_doc_lens"][n_docs])
+    p = _prefix(cpu, n_tok, n_docs)
+    d = to_dev(p)
+    out, lse = run_fwd(cuda_lib, d, wl.window, wl.use_rope, wl.rope_theta)
+    g = run_bwd(cuda_lib, d, out, lse, wl.window, wl.use_rope, wl.rope_theta)
+    torch.cuda.synchronize()
+    O, L = fo.flint_attn_fwd(p["q"], p["k"], p["v"], p["w_q"], p["w_k"], p["sink"],
+                             p["cu_doc_lens"], wl.window, wl.use_rope, wl.rope_theta)
+    compare(out, O, "bf16", "out")
+    compare(lse, L, "bf16", "lse")
+    ref = fo.flint_attn_bwd(p["q"], p["k"], p["v"], p["w_q"], p["w_k"], p["sink"],
+                            p["cu_doc_lens"], wl.window, wl.use_rope, wl.rope_theta, p["dout"])
+    for name in ["dq", "dk", "dv", "dw_q", "dw_k", "dsink"]:
+        compare(g[name], ref[name], "bf16", name)
