@@ -82,7 +82,7 @@ def config_of(w, pairs, flops_step):
         "masked_pairs_per_head": pairs, "flops_per_step": flops_step,
         "l2": "inputs larger than L2 (126 MB), plus a 256 MB L2 flush before every step",
         "parallelism": "replicas (one independent batch per GPU)",
-        "gradients": "dq, dk, dv in float32; dw_q, dw_k, d_sink float32",
+        "outputs": "O, dq, dk, dv in float32 (fp32_out); LSE, dw_q, dw_k, d_sink float32",
     }
 
 
@@ -282,13 +282,14 @@ def main(argv=None):
     d = {k: (v.to(dev) if torch.is_tensor(v) else v) for k, v in cpu.items()}
     T, H, D = d["q"].shape
     p = fa.params_for(d["q"], d["k"], d["cu_doc_lens"], w.window, w.use_rope, w.rope_theta,
-                      fp32_grads=True)
+                      fp32_out=True)
     ws_f = fa.alloc_workspace(p, False, dev)
     ws_b = fa.alloc_workspace(p, True, dev)
-    out = torch.empty_like(d["q"])
+    out = torch.empty(d["q"].shape, dtype=torch.float32, device=dev)
     lse = torch.empty(H, T, dtype=torch.float32, device=dev)
-    # gradients w.r.t. q, k, v in float32 (the configuration the parity tests hold
-    # to max-abs 2e-2; bfloat16 storage alone would exceed that for |grad| > 10)
+    # O and the gradients w.r.t. q, k, v in float32 (fp32_out): the configuration
+    # the parity tests hold to max-abs 2e-2; bfloat16 storage alone exceeds that
+    # for |grad| > 10, and bf16 O feeds D = dO . O of the sink gradient
     f32 = torch.float32
     grads = {"dq": torch.empty(d["q"].shape, dtype=f32, device=dev),
              "dk": torch.empty(d["k"].shape, dtype=f32, device=dev),
@@ -302,12 +303,12 @@ def main(argv=None):
     def fwd_call(src):
         fa.fwd(src["q"], src["k"], src["v"], src["w_q"], src["w_k"], src["sink"],
                src["cu_doc_lens"], w.window, w.use_rope, w.rope_theta, out=out, lse=lse,
-               workspace=ws_f)
+               workspace=ws_f, fp32_out=True)
 
     def bwd_call(src):
         fa.bwd(src["q"], src["k"], src["v"], src["w_q"], src["w_k"], src["sink"],
                src["cu_doc_lens"], out, lse, src["dout"], w.window, w.use_rope, w.rope_theta,
-               grads=grads, workspace=ws_b, fp32_grads=True)
+               grads=grads, workspace=ws_b, fp32_out=True)
 
     # ---- warm-up (also surfaces device-side timeouts before timing)
     for _ in range(args.warmup):

@@ -47,10 +47,14 @@
  *   - Layouts: q, out, dout, dq [T, H, D]; k, v, dk, dv [T, Hk, D];
  *     q_norm_w, k_norm_w [D]; sink, dsink [H] fp32; lse [H, T] fp32;
  *     dq_norm_w, dk_norm_w [D] fp32.
- *   - dtype FLINT_BF16: q, k, v, out, dout, dq, dk, dv and the norm weights are
- *     bfloat16; the attention contractions run on tcgen05 tensor cores with
- *     FP32 accumulation. dtype FLINT_FP32: those tensors are float32 and every
- *     step runs in FP32 on CUDA cores.
+ *   - dtype FLINT_BF16: q, k, v, dout and the norm weights are bfloat16; out,
+ *     dq, dk, dv are bfloat16, or float32 with params->fp32_out. The attention
+ *     contractions run on tcgen05 tensor cores with FP32 accumulation; their
+ *     operands (q_hat, k_hat, v, P, and in the backward dout and dS) are IEEE
+ *     fp16, whose 10-bit mantissa keeps their rounding well below bf16's.
+ *     |v| and |dout| must stay below 65504 (larger values saturate).
+ *     dtype FLINT_FP32: all tensors are float32 and every step runs in FP32 on
+ *     CUDA cores.
  */
 #ifndef FLINT_ATTN_H
 #define FLINT_ATTN_H
@@ -86,8 +90,9 @@ typedef struct {
   float rms_eps;          /* RMSNorm epsilon (Flint: 1e-6) */
   float softmax_scale;    /* 0 => 1/sqrt(head_dim) */
   int32_t dtype;          /* flint_dtype_t */
-  int32_t fp32_grads;     /* backward only: nonzero => dq, dk, dv are float32 (FP32 inputs
-                             always give float32 gradients); zero => same type as q */
+  int32_t fp32_out;       /* nonzero => out (forward, and as passed to the backward) and
+                             dq, dk, dv are float32; zero => same type as q. FP32 inputs
+                             always use float32. */
 } flint_attn_params_t;
 
 /* Bytes of device workspace a call needs (backward = 0 for flint_attn_fwd,
@@ -99,7 +104,7 @@ size_t flint_attn_workspace_bytes(const flint_attn_params_t* params, int backwar
  *   q [T,H,D], k [T,Hk,D], v [T,Hk,D], q_norm_w [D], k_norm_w [D]  (dtype)
  *   sink [H] fp32, cu_doc_lens [num_docs+1] int32 (device, non-decreasing,
  *   cu_doc_lens[0] = 0, cu_doc_lens[num_docs] = T; not checked on the device)
- *   out [T,H,D] (dtype), lse [H,T] fp32 (natural log). */
+ *   out [T,H,D] (dtype, or float32 with fp32_out), lse [H,T] fp32 (natural log). */
 flint_status_t flint_attn_fwd(const flint_attn_params_t* params,
                               const void* q, const void* k, const void* v,
                               const void* q_norm_w, const void* k_norm_w,
@@ -109,14 +114,14 @@ flint_status_t flint_attn_fwd(const flint_attn_params_t* params,
 
 /* Backward of sum(dout * out) for out = flint_attn_fwd(...).
  *   out, lse: the forward's results for the same inputs; dout [T,H,D] (dtype).
+ *   out must have the type the forward wrote (float32 with fp32_out): D = dO . O
+ *   is formed from it, and the bf16 rounding of O is the largest error source
+ *   of the sink and norm-weight gradients.
  *   Writes dq [T,H,D], dk [T,Hk,D], dv [T,Hk,D] (gradients w.r.t. the RAW q, k,
- *   v; float32 when params->fp32_grads or dtype is FLINT_FP32, else bfloat16),
- *   dq_norm_w, dk_norm_w [D] fp32, dsink [H] fp32. Outputs are overwritten, not
- *   accumulated. q and k are re-normalised and re-rotated inside (nothing from
- *   the forward besides out and lse is needed).
- *   BF16 inputs: the backward's tensor-core operands (q_hat, k_hat, v, dout, P,
- *   dS) are IEEE fp16 for their 10-bit mantissa; |v| and |dout| must stay below
- *   65504 (larger values saturate to +-65504). Accumulation is FP32. */
+ *   v; float32 with fp32_out, else the input type), dq_norm_w, dk_norm_w [D]
+ *   fp32, dsink [H] fp32. Outputs are overwritten, not accumulated. q and k are
+ *   re-normalised and re-rotated inside (nothing from the forward besides out
+ *   and lse is needed). */
 flint_status_t flint_attn_bwd(const flint_attn_params_t* params,
                               const void* q, const void* k, const void* v,
                               const void* q_norm_w, const void* k_norm_w,

@@ -107,7 +107,7 @@ flint_status_t resolve(const flint_attn_params_t* in, Resolved* p) {
   p->eps = in->rms_eps;
   p->scale = in->softmax_scale > 0.f ? in->softmax_scale : 1.0f / std::sqrt((float)kHeadDim);
   p->dtype = in->dtype;
-  p->fp32_grads = (in->fp32_grads != 0 || in->dtype == FLINT_FP32) ? 1 : 0;
+  p->fp32_out = (in->fp32_out != 0 || in->dtype == FLINT_FP32) ? 1 : 0;
   p->R = kTileRows / (G <= 128 ? G : 128);
   if (p->R < 1) p->R = 1;
   return FLINT_OK;
@@ -208,8 +208,9 @@ extern "C" flint_status_t flint_attn_fwd(const flint_attn_params_t* params, cons
   if (p.T == 0) return FLINT_OK;
   void* qh = at<void>(workspace, L.qhat);
   void* kh = at<void>(workspace, L.khat);
-  FLINT_TRY(launch_prologue(p, q, q_norm_w, qh, p.H, cu_doc_lens, st));
-  FLINT_TRY(launch_prologue(p, k, k_norm_w, kh, p.Hk, cu_doc_lens, st));
+  const bool f16 = p.dtype == FLINT_BF16;   // tensor-core operands are fp16
+  FLINT_TRY(launch_prologue(p, q, q_norm_w, qh, p.H, cu_doc_lens, st, f16));
+  FLINT_TRY(launch_prologue(p, k, k_norm_w, kh, p.Hk, cu_doc_lens, st, f16));
   if (p.dtype == FLINT_FP32) {
     return cuda_status(launch_attn_fwd_fp32(p, (const float*)qh, (const float*)kh,
                                             (const float*)v, sink, cu_doc_lens, (float*)out, lse,
@@ -218,9 +219,14 @@ extern "C" flint_status_t flint_attn_fwd(const flint_attn_params_t* params, cons
   int4* items = at<int4>(workspace, L.items_q);
   FLINT_TRY(launch_build_worklist(cu_doc_lens, p, kModeQuery, 2 * p.R, items, status + 1,
                                   at<void>(workspace, L.sched_tmp), L.max_items_q, st));
+  __half* v16 = at<__half>(workspace, L.v16);
+  FLINT_TRY(launch_convert_f16(static_cast<const __nv_bfloat16*>(v), v16,
+                               (size_t)p.T * p.Hk * kHeadDim, st));
+  const CUtensorMapDataType f16t = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
   CUtensorMap tq, tk, tv;
-  if (!encode_3d(&tq, qh, p.T, p.H, p.G, p.R) || !encode_3d(&tk, kh, p.T, p.Hk, 1, kTileKeys) ||
-      !encode_3d(&tv, v, p.T, p.Hk, 1, kTileKeys))
+  if (!encode_3d(&tq, qh, p.T, p.H, p.G, p.R, f16t) ||
+      !encode_3d(&tk, kh, p.T, p.Hk, 1, kTileKeys, f16t) ||
+      !encode_3d(&tv, v16, p.T, p.Hk, 1, kTileKeys, f16t))
     return FLINT_ERR_CUDA;
   return cuda_status(launch_attn_fwd_sm100_impl(tq, tk, tv, p, sink, items, status + 1,
                                                 L.max_items_q, out, lse, status, sm_count(), st));

@@ -708,7 +708,7 @@ cudaError_t launch_attn_bwd_sm100_impl(const CUtensorMap& tq, const CUtensorMap&
   a.lse = lse; a.dvec = dvec;
   a.dq_acc = dq_acc; a.dk_acc = dk_acc;
   a.dv = dv;
-  a.dv_f32 = p.fp32_grads || p.dtype == FLINT_FP32;
+  a.dv_f32 = p.fp32_out || p.dtype == FLINT_FP32;
   a.status = status;
 
   a.items = items_kv; a.n_items = n_kv; a.max_items = max_kv;

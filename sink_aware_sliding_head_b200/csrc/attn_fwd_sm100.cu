@@ -1,5 +1,7 @@
 // attn_fwd_sm100.cu - sink-aware sliding/full GQA attention forward on
-// Blackwell tensor cores (tcgen05 + TMEM + TMA), BF16 in, FP32 accumulate.
+// Blackwell tensor cores (tcgen05 + TMEM + TMA): BF16 inputs, FP16 tensor-core
+// operands (q_hat, k_hat from the prologue, an fp16 copy of v, P), FP32
+// accumulation, output in bf16 or fp32.
 //
 // What it computes (Flint layers page, nemo_automodel.components.models.flint.
 // layers, FlintAttention.forward: causal attention with a zero-value sink
@@ -54,7 +56,8 @@ struct FwdArgs {
   const int4* items;
   const int* n_items;
   int max_items;
-  __nv_bfloat16* out;
+  void* out;        // bf16 or float, per out_f32
+  int out_f32;
   float* lse;
   int* status;
 };
@@ -205,8 +208,8 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
     // other tile's MMAs. QK_i(n+1) overwrites S_i, which holds P_i(n), so it
     // is issued only after PV_i(n) has completed.
     if (lane == 0) {
-      const uint32_t idesc_qk = make_idesc_bf16(128, 128, 0, 0);
-      const uint32_t idesc_pv = make_idesc_bf16(128, 128, 0, 1);
+      const uint32_t idesc_qk = make_idesc_f16(128, 128, 0, 0);
+      const uint32_t idesc_pv = make_idesc_f16(128, 128, 0, 1);
       uint32_t kv_iter = 0, item_count = 0;
       uint32_t pv0 = 0, pv1 = 0, pc0 = 0, pc1 = 0;   // PV commits / P arrivals seen, per tile
       bool ok = true;
@@ -422,7 +425,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
             const float p0 = ex2_approx(x0);
             const float p1 = ex2_approx(x1);
             rs2 = fadd2(rs2, f2(p0, p1));
-            pk[e] = pack_bf16x2(p0, p1);
+            pk[e] = pack_f16x2(p0, p1);
           }
           tmem_st32(t_row + s_col + hf * 32, pk);
         }
@@ -441,7 +444,8 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       if (!ok) break;
       tc_fence_after();
       const float inv_l = 1.f / l;
-      __nv_bfloat16* orow = a.out + ((size_t)tok * a.H + h) * kHeadDim;
+      const uint64_t il2 = f2(inv_l, inv_l);
+      const size_t obase = ((size_t)tok * a.H + h) * kHeadDim;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t u[32];
@@ -453,14 +457,28 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
           if (lane == 0) mbar_arrive(smem_u32(&bars->o_empty[i]));
         }
         if (valid) {
+          float o[32];
 #pragma unroll
-          for (int v4 = 0; v4 < 4; ++v4) {
-            uint4 pk;
-            pk.x = pack_bf16x2(__uint_as_float(u[v4 * 8 + 0]) * inv_l, __uint_as_float(u[v4 * 8 + 1]) * inv_l);
-            pk.y = pack_bf16x2(__uint_as_float(u[v4 * 8 + 2]) * inv_l, __uint_as_float(u[v4 * 8 + 3]) * inv_l);
-            pk.z = pack_bf16x2(__uint_as_float(u[v4 * 8 + 4]) * inv_l, __uint_as_float(u[v4 * 8 + 5]) * inv_l);
-            pk.w = pack_bf16x2(__uint_as_float(u[v4 * 8 + 6]) * inv_l, __uint_as_float(u[v4 * 8 + 7]) * inv_l);
-            *reinterpret_cast<uint4*>(orow + c * 32 + v4 * 8) = pk;
+          for (int e = 0; e < 32; e += 2)
+            f2_split(fmul2(f2(__uint_as_float(u[e]), __uint_as_float(u[e + 1])), il2), o[e],
+                     o[e + 1]);
+          if (a.out_f32) {
+            float* orow = reinterpret_cast<float*>(a.out) + obase + c * 32;
+#pragma unroll
+            for (int v4 = 0; v4 < 8; ++v4)
+              *reinterpret_cast<float4*>(orow + 4 * v4) =
+                  make_float4(o[4 * v4], o[4 * v4 + 1], o[4 * v4 + 2], o[4 * v4 + 3]);
+          } else {
+            __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.out) + obase + c * 32;
+#pragma unroll
+            for (int v4 = 0; v4 < 4; ++v4) {
+              uint4 pk;
+              pk.x = pack_bf16x2(o[v4 * 8 + 0], o[v4 * 8 + 1]);
+              pk.y = pack_bf16x2(o[v4 * 8 + 2], o[v4 * 8 + 3]);
+              pk.z = pack_bf16x2(o[v4 * 8 + 4], o[v4 * 8 + 5]);
+              pk.w = pack_bf16x2(o[v4 * 8 + 6], o[v4 * 8 + 7]);
+              *reinterpret_cast<uint4*>(orow + v4 * 8) = pk;
+            }
           }
         }
       }
@@ -493,7 +511,8 @@ cudaError_t launch_attn_fwd_sm100_impl(const CUtensorMap& tq, const CUtensorMap&
   a.T = p.T; a.H = p.H; a.Hk = p.Hk; a.G = p.G; a.R = p.R; a.W = p.W;
   a.scale_log2 = p.scale * kLog2e;
   a.sink = sink; a.items = items; a.n_items = n_items; a.max_items = max_items;
-  a.out = reinterpret_cast<__nv_bfloat16*>(out);
+  a.out = out;
+  a.out_f32 = p.fp32_out;
   a.lse = lse;
   a.status = status;
   int grid = num_sms;

@@ -23,9 +23,9 @@ constexpr int kTok = 4;
 
 // Also writes an fp16 copy of dO (dout16, when non-null): the BF16 backward's
 // tensor-core operands are fp16.
-template <typename T>
+template <typename TO, typename T>
 __global__ void __launch_bounds__(kThreads)
-bwd_pre_kernel(const T* __restrict__ out, const T* __restrict__ dout,
+bwd_pre_kernel(const TO* __restrict__ out, const T* __restrict__ dout,
                const float* __restrict__ lse, const float* __restrict__ sink,
                float* __restrict__ dvec, float* __restrict__ part, __half* __restrict__ dout16,
                int ntok, int H) {
@@ -112,14 +112,16 @@ cudaError_t launch_bwd_preprocess(const Resolved& p, const void* out, const void
   const size_t smem = (size_t)kGroups * p.H * sizeof(float);
   {
   ProfScope prof(kKBwdPre, st);
-  if (p.dtype == FLINT_BF16)
-    bwd_pre_kernel<__nv_bfloat16><<<blocks, kThreads, smem, st>>>(
-        (const __nv_bfloat16*)out, (const __nv_bfloat16*)dout, lse, sink, dvec, part, dout16,
-        p.T, p.H);
+  typedef __nv_bfloat16 bf;
+  if (p.dtype == FLINT_BF16 && p.fp32_out)
+    bwd_pre_kernel<float, bf><<<blocks, kThreads, smem, st>>>(
+        (const float*)out, (const bf*)dout, lse, sink, dvec, part, dout16, p.T, p.H);
+  else if (p.dtype == FLINT_BF16)
+    bwd_pre_kernel<bf, bf><<<blocks, kThreads, smem, st>>>(
+        (const bf*)out, (const bf*)dout, lse, sink, dvec, part, dout16, p.T, p.H);
   else
-    bwd_pre_kernel<float><<<blocks, kThreads, smem, st>>>((const float*)out, (const float*)dout,
-                                                          lse, sink, dvec, part, nullptr, p.T,
-                                                          p.H);
+    bwd_pre_kernel<float, float><<<blocks, kThreads, smem, st>>>(
+        (const float*)out, (const float*)dout, lse, sink, dvec, part, nullptr, p.T, p.H);
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;

@@ -28,7 +28,7 @@ struct Resolved {
   int T, N, H, Hk, D, G, W, rope;
   float theta, eps, scale;
   int dtype;
-  int fp32_grads;   // dq, dk, dv written as float32 (always for FP32 inputs)
+  int fp32_out;     // out, dq, dk, dv are float32 (always for FP32 inputs)
   int R;            // tokens per 128-row tile = 128 / G
 };
 
@@ -45,7 +45,7 @@ struct WsLayout {
   size_t dq_acc;        // [T,H,D] fp32 gradient w.r.t. q_hat (backward)
   size_t dk_acc;        // [T,Hk,D] fp32 gradient w.r.t. k_hat (backward)
   size_t dout16;        // [T,H,D] fp16 copy of dO (backward, BF16 inputs)
-  size_t v16;           // [T,Hk,D] fp16 copy of v (backward, BF16 inputs)
+  size_t v16;           // [T,Hk,D] fp16 copy of v (BF16 inputs)
   size_t total;
   int max_items_q, max_items_q1, max_items_kv, max_items_any;
   int part_blocks;      // number of partial-sum rows per reduced quantity
@@ -76,15 +76,13 @@ inline WsLayout make_layout(const Resolved& p, bool backward) {
   L.items_kv = backward ? take((size_t)L.max_items_kv * 16) : off;
   L.sched_tmp = take((size_t)L.max_items_any * 20);
   L.part_blocks = kPartBlocks;
+  if (p.dtype == FLINT_BF16) L.v16 = take((size_t)p.T * p.Hk * p.D * 2);
   if (backward) {
     L.dvec = take((size_t)p.H * p.T * 4);
     L.part = take((size_t)kPartBlocks * (p.H + 2 * p.D) * 4);
     L.dq_acc = take((size_t)p.T * p.H * p.D * 4);
     L.dk_acc = take((size_t)p.T * p.Hk * p.D * 4);
-    if (p.dtype == FLINT_BF16) {
-      L.dout16 = take((size_t)p.T * p.H * p.D * 2);
-      L.v16 = take((size_t)p.T * p.Hk * p.D * 2);
-    }
+    if (p.dtype == FLINT_BF16) L.dout16 = take((size_t)p.T * p.H * p.D * 2);
   }
   L.total = off;
   return L;

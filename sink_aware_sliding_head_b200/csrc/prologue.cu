@@ -229,7 +229,7 @@ cudaError_t launch_bwd_epilogue(const Resolved& p, const void* x, const void* w,
   {
   ProfScope prof(kKPrologueBwd, st);
   typedef __nv_bfloat16 bf;
-  if (p.dtype == FLINT_BF16 && p.fp32_grads)
+  if (p.dtype == FLINT_BF16 && p.fp32_out)
     prologue_bwd_kernel<bf, float><<<blocks, kThreads, 0, st>>>(
         (const bf*)x, (const bf*)w, g_hat, (float*)dx, part, p.T, heads, cu, p.N, p.rope, p.theta,
         p.eps);
