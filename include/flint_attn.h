@@ -131,6 +131,31 @@ flint_status_t flint_attn_bwd(const flint_attn_params_t* params,
                               float* dq_norm_w, float* dk_norm_w, float* dsink,
                               void* workspace, size_t workspace_bytes, void* stream);
 
+/* Largest num_q_heads flint_attn_bwd_preprocess_static accepts. */
+#define FLINT_STATIC_MAX_HEADS 128
+
+/* Backward preprocess without a workspace and without allocating: writes
+ * d_rowsum [H,T] fp32 (D_i = dout_i . out_i per row) and dsink [H] fp32, the
+ * same values flint_attn_bwd computes for its own use. The source pages have
+ * no counterpart of this call; it exists for callers that cannot allocate
+ * device memory where they run (a fixed-budget serving loop, a plugin that is
+ * given tensors but no workspace, a path where cudaMalloc/cudaFree would
+ * synchronise the device).
+ *   params: total_tokens, num_q_heads, head_dim (128), dtype, fp32_out (the type
+ *   of out, as for flint_attn_bwd) are read; num_q_heads <= FLINT_STATIC_MAX_HEADS,
+ *   else FLINT_ERR_WORKSPACE before any launch.
+ *   out, dout [T,H,D] (out float32 with fp32_out), lse [H,T] fp32, sink [H] fp32:
+ *   device inputs. d_rowsum [H,T], dsink [H]: device outputs (overwritten).
+ * Its scratch is a fixed 592 KiB array in device memory, held by every GPU that
+ * loads the library until exit and shared by all calls: calls whose kernels
+ * overlap on the GPU (unordered streams) race on it. The first call on a device
+ * looks the array up with that device current; make it before any stream
+ * capture on that device. Asynchronous on `stream`. */
+flint_status_t flint_attn_bwd_preprocess_static(const flint_attn_params_t* params,
+                                                const void* out, const void* dout,
+                                                const float* lse, const float* sink,
+                                                float* d_rowsum, float* dsink, void* stream);
+
 /* Synchronises `stream`, reads and clears the device status word in
  * `workspace` (written by bounded device waits), and returns FLINT_OK or
  * FLINT_ERR_TIMEOUT (FLINT_ERR_CUDA if the stream itself reports an error). */

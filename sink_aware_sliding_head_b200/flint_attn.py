@@ -27,7 +27,8 @@ STATUS = {0: "FLINT_OK", 1: "FLINT_ERR_INVALID_ARG", 2: "FLINT_ERR_UNSUPPORTED",
 EXPORTED = ["flint_attn_workspace_bytes", "flint_attn_fwd", "flint_attn_bwd",
             "flint_attn_check_status", "flint_status_string", "flint_attn_version",
             "flint_attn_profile_enable", "flint_attn_profile_collect",
-            "flint_attn_profile_reset", "flint_attn_launch_count"]
+            "flint_attn_profile_reset", "flint_attn_launch_count",
+            "flint_attn_bwd_preprocess_static"]
 
 
 class Params(ctypes.Structure):
@@ -90,6 +91,8 @@ def load_library(path: str = LIB_PATH):
     lib.flint_attn_profile_reset.restype = None
     lib.flint_attn_launch_count.argtypes = []
     lib.flint_attn_launch_count.restype = ctypes.c_longlong
+    lib.flint_attn_bwd_preprocess_static.argtypes = [P] + [vp] * 6 + [vp]
+    lib.flint_attn_bwd_preprocess_static.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -231,6 +234,29 @@ def profile_collect():
 def launch_count() -> int:
     """Kernels the library has launched since it was loaded."""
     return int(load_library().flint_attn_launch_count())
+
+
+def bwd_preprocess_static(out, dout, lse, sink, fp32_out=False, d_rowsum=None, dsink=None,
+                          stream=None):
+    """D = rowsum(dout * out) [H,T] and d_sink [H] through the no-allocation entry point.
+
+    For callers that cannot allocate device memory where they run: the library
+    uses a fixed scratch array of its own instead of a caller workspace (see
+    ``flint_attn_bwd_preprocess_static`` in include/flint_attn.h for its limits).
+    """
+    lib = load_library()
+    T, H, D = out.shape
+    p = make_params(T, 1, H, 1, 0, False, 0.0, _dtype_code(dout), head_dim=D,
+                    fp32_out=fp32_out)
+    if d_rowsum is None:
+        d_rowsum = torch.empty(H, T, dtype=torch.float32, device=out.device)
+    if dsink is None:
+        dsink = torch.empty(H, dtype=torch.float32, device=out.device)
+    code = lib.flint_attn_bwd_preprocess_static(ctypes.byref(p), _ptr(out), _ptr(dout), _ptr(lse),
+                                                _ptr(sink), _ptr(d_rowsum), _ptr(dsink),
+                                                _stream_ptr(stream))
+    _check(code, "flint_attn_bwd_preprocess_static")
+    return d_rowsum, dsink
 
 
 def version() -> str:
