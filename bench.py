@@ -50,6 +50,9 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="target CPU time of the oracle baseline sample")
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="run the workload as one document of this many tokens (smaller "
+                         "cases for profiler captures); 0 keeps the workload's size")
     return ap.parse_args(argv)
 
 
@@ -276,6 +279,10 @@ def main(argv=None):
             pg.barrier()
 
     w = WORKLOADS[args.workload]
+    if args.tokens > 0:
+        import dataclasses
+        w = dataclasses.replace(w, name=f"{w.name}@{args.tokens}", doc_lens=(args.tokens,),
+                                total_tokens=args.tokens, drawn_len_range=None)
     cpu = fi.make_inputs(w, seed=w.seed + rank, with_grad_out=True)
     pairs, ff, fb = flops_of(cpu["doc_lens"], w.window, w.num_q_heads)
     flops_step = ff + fb

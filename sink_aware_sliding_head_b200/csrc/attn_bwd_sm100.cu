@@ -15,8 +15,13 @@
 // and dO, and P, dS rounded to fp16 - fp16's 10-bit mantissa keeps the bf16
 // rounding of these intermediates from dominating the gradient error.
 //
-// Two persistent kernels share one warp layout (warps 0-3: elementwise math,
-// thread = TMEM lane; warp 4: TMA; warp 5: MMA issue + TMEM owner):
+// Two persistent kernels share one warp layout: warps 0-7 do the elementwise
+// math as two warpgroups that split the 128 columns of each tile (there is no
+// row reduction in the backward, so the halves are independent; thread = TMEM
+// lane), warp 8 issues TMA, warp 9 issues MMAs and owns TMEM. Each warpgroup
+// writes its fp16 P/dS half into the first 32 of the 64 TMEM columns it has
+// just read itself (columns [64c, 64c+32) for warpgroup c), so the TMEM A
+// operand of the following MMA skips from column 32 to 64 halfway through K.
 //  * dkv: key-major. A CTA owns 128 keys of one KV head and streams the
 //    128-row query tiles (R tokens x G heads) that see them. Per tile:
 //    S^T = K Q^T and dP^T = V dO^T (TMEM), then P^T and dS^T in fp16 overwrite
@@ -34,9 +39,10 @@ namespace flint {
 
 namespace {
 
-constexpr int kThreads = 192;
-constexpr int kWarpTma = 4;
-constexpr int kWarpMma = 5;
+constexpr int kThreads = 320;
+constexpr int kWarpTma = 8;
+constexpr int kWarpMma = 9;
+constexpr int kMathWarps = 8;
 constexpr uint32_t kChunkBytes = 128 * 64 * 2;
 constexpr uint32_t kTileBytes = 2 * kChunkBytes;
 constexpr float kLog2e = 1.4426950408889634f;
@@ -62,25 +68,10 @@ __device__ __forceinline__ uint64_t kmajor_desc(uint32_t tile_base, int kk) {
 __device__ __forceinline__ uint64_t mnmajor_desc(uint32_t tile_base, int kk) {
   return make_sdesc(tile_base + kk * 2048, kChunkBytes, 1024);
 }
-
-// 128 fp32 TMEM columns of this thread's lane -> v[128]
-__device__ __forceinline__ void tmem_row128(uint32_t taddr, float (&v)[128]) {
-  uint32_t u0[32], u1[32], u2[32], u3[32];
-  tmem_ld32(taddr + 0, u0);
-  tmem_ld32(taddr + 32, u1);
-  tmem_ld32(taddr + 64, u2);
-  tmem_ld32(taddr + 96, u3);
-  tc_wait_ld_dep(u0);
-  tc_wait_ld_dep(u1);
-  tc_wait_ld_dep(u2);
-  tc_wait_ld_dep(u3);
-#pragma unroll
-  for (int e = 0; e < 32; ++e) {
-    v[e] = __uint_as_float(u0[e]);
-    v[32 + e] = __uint_as_float(u1[e]);
-    v[64 + e] = __uint_as_float(u2[e]);
-    v[96 + e] = __uint_as_float(u3[e]);
-  }
+// TMEM column of the fp16 A-operand slice kk (16 K-elements = 8 columns) of a
+// region whose two 64-element halves sit at columns [0,32) and [64,96).
+__device__ __forceinline__ uint32_t split_a_col(int kk) {
+  return kk < 4 ? kk * 8 : 64 + (kk - 4) * 8;
 }
 
 __device__ __forceinline__ float2 unpack_f16x2(uint32_t u) {
@@ -145,12 +136,12 @@ attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_q,
     }
     mbar_init(smem_u32(&bars->s_full), 1);
     mbar_init(smem_u32(&bars->dp_full), 1);
-    mbar_init(smem_u32(&bars->p_full), 4);
-    mbar_init(smem_u32(&bars->ds_full), 4);
+    mbar_init(smem_u32(&bars->p_full), kMathWarps);
+    mbar_init(smem_u32(&bars->ds_full), kMathWarps);
     mbar_init(smem_u32(&bars->dv_done), 1);
     mbar_init(smem_u32(&bars->dk_done), 1);
     mbar_init(smem_u32(&bars->acc_full), 1);
-    mbar_init(smem_u32(&bars->acc_empty), 4);
+    mbar_init(smem_u32(&bars->acc_empty), kMathWarps);
     mbar_init(smem_u32(&bars->drain), 1);
     fence_mbar_init();
   }
@@ -263,7 +254,7 @@ attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_q,
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            mma_ts(tmem + 256, tmem + 0 + kk * 8, mnmajor_desc(dot, kk), idesc_ts,
+            mma_ts(tmem + 256, tmem + split_a_col(kk), mnmajor_desc(dot, kk), idesc_ts,
                    (m > 0 || kk > 0) ? 1u : 0u);
           mma_commit(smem_u32(&bars->dv_done));
           ++dv_count;
@@ -273,7 +264,7 @@ attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_q,
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            mma_ts(tmem + 384, tmem + 128 + kk * 8, mnmajor_desc(qt, kk), idesc_ts,
+            mma_ts(tmem + 384, tmem + 128 + split_a_col(kk), mnmajor_desc(qt, kk), idesc_ts,
                    (m > 0 || kk > 0) ? 1u : 0u);
           mma_commit(smem_u32(&bars->dk_done));
           ++dk_count;
@@ -291,8 +282,10 @@ attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_q,
     }
   } else {
     // ---------------------------------------------------------------- math warps
-    const int kl = warp * 32 + lane;               // key row of the tile = TMEM lane
-    const uint32_t t_row = tmem + ((uint32_t)(warp * 32) << 16);
+    const int wg = warp >> 2;                      // column half: query rows [64wg, 64wg+64)
+    const int kl = (warp & 3) * 32 + lane;         // key row of the tile = TMEM lane
+    const uint32_t t_row = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+    const uint32_t c0 = 64 * wg;                   // first column of this warpgroup
     uint32_t item_count = 0, s_cnt = 0, dp_cnt = 0, tile_count = 0;
     bool ok = true;
     for (int idx = blockIdx.x; idx < n_items && ok; idx += gridDim.x) {
@@ -312,17 +305,17 @@ attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_q,
         ++s_cnt;
         if (!ok) break;
         tc_fence_after();
-        uint32_t pk[64];
-#pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
+        // P^T for query rows [c0, c0+64): 2^(s*scale - lse2), masked, fp16
+        uint32_t pk[32];
+        {
           uint32_t u0[32], u1[32];
-          tmem_ld32(t_row + hf * 64, u0);
-          tmem_ld32(t_row + hf * 64 + 32, u1);
+          tmem_ld32(t_row + c0, u0);
+          tmem_ld32(t_row + c0 + 32, u1);
           tc_wait_ld_dep(u0);
           tc_wait_ld_dep(u1);
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
-            const int c = hf * 64 + 2 * e;
+            const int c = c0 + 2 * e;
             const float s0 = __uint_as_float(e < 16 ? u0[2 * e] : u1[2 * e - 32]);
             const float s1 = __uint_as_float(e < 16 ? u0[2 * e + 1] : u1[2 * e - 31]);
             float p0 = ex2_approx(fmaf(s0, a.scale_log2, -st[c]));
@@ -334,11 +327,10 @@ attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_q,
               p0 = v0 ? p0 : 0.f;
               p1 = v1 ? p1 : 0.f;
             }
-            pk[hf * 32 + e] = pack_f16x2(p0, p1);
+            pk[e] = pack_f16x2(p0, p1);
           }
         }
-        tmem_st32(t_row + 0, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
-        tmem_st32(t_row + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
+        tmem_st32(t_row + c0, pk);
         tc_wait_st();
         tc_fence_before();
         __syncwarp();
@@ -347,24 +339,21 @@ attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_q,
         ++dp_cnt;
         if (!ok) break;
         tc_fence_after();
-#pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
+        {
           uint32_t u0[32], u1[32], ds[32];
-          tmem_ld32(t_row + 128 + hf * 64, u0);
-          tmem_ld32(t_row + 128 + hf * 64 + 32, u1);
+          tmem_ld32(t_row + 128 + c0, u0);
+          tmem_ld32(t_row + 128 + c0 + 32, u1);
           tc_wait_ld_dep(u0);
           tc_wait_ld_dep(u1);
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
-            const int c = hf * 64 + 2 * e;
+            const int c = c0 + 2 * e;
             const float d0 = __uint_as_float(e < 16 ? u0[2 * e] : u1[2 * e - 32]);
             const float d1 = __uint_as_float(e < 16 ? u0[2 * e + 1] : u1[2 * e - 31]);
-            const float2 p = unpack_f16x2(pk[hf * 32 + e]);
+            const float2 p = unpack_f16x2(pk[e]);
             ds[e] = pack_f16x2(p.x * (d0 - st[128 + c]), p.y * (d1 - st[128 + c + 1]));
           }
-          // dS^T columns [hf*32, hf*32+32) of the fp16 region; this thread's
-          // dP^T row for these keys was fully read above.
-          tmem_st32(t_row + 128 + hf * 32, ds);
+          tmem_st32(t_row + 128 + c0, ds);
         }
         tc_wait_st();
         tc_fence_before();
@@ -376,44 +365,59 @@ attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_q,
       if (!ok) break;
       tc_fence_after();
       {
-        const size_t rb = ((size_t)j * a.Hk + it.g) * kHeadDim;
-        {  // dV: fp32 or bf16
-          float acc[128];
-          tmem_row128(t_row + 256, acc);
+        // this warpgroup writes columns [c0, c0+64) of the key row's dV, then dK
+        const size_t rb = ((size_t)j * a.Hk + it.g) * kHeadDim + c0;
+        {
+          uint32_t v0[32], v1[32];
+          tmem_ld32(t_row + 256 + c0, v0);
+          tmem_ld32(t_row + 256 + c0 + 32, v1);
+          tc_wait_ld_dep(v0);
+          tc_wait_ld_dep(v1);
           if (valid_key) {
 #pragma unroll
-            for (int c = 0; c < 128; c += 8) {
+            for (int hh = 0; hh < 2; ++hh) {
+              const uint32_t* vv = hh ? v1 : v0;
               if (a.dv_f32) {
-                float* dvrow = reinterpret_cast<float*>(a.dv) + rb;
-                *reinterpret_cast<float4*>(dvrow + c) =
-                    make_float4(acc[c], acc[c + 1], acc[c + 2], acc[c + 3]);
-                *reinterpret_cast<float4*>(dvrow + c + 4) =
-                    make_float4(acc[c + 4], acc[c + 5], acc[c + 6], acc[c + 7]);
+                float* dvrow = reinterpret_cast<float*>(a.dv) + rb + hh * 32;
+#pragma unroll
+                for (int c = 0; c < 32; c += 4)
+                  *reinterpret_cast<uint4*>(dvrow + c) =
+                      make_uint4(vv[c], vv[c + 1], vv[c + 2], vv[c + 3]);
               } else {
-                __nv_bfloat16* dvrow = reinterpret_cast<__nv_bfloat16*>(a.dv) + rb;
-                uint4 pkv;
-                pkv.x = pack_bf16x2(acc[c + 0], acc[c + 1]);
-                pkv.y = pack_bf16x2(acc[c + 2], acc[c + 3]);
-                pkv.z = pack_bf16x2(acc[c + 4], acc[c + 5]);
-                pkv.w = pack_bf16x2(acc[c + 6], acc[c + 7]);
-                *reinterpret_cast<uint4*>(dvrow + c) = pkv;
+                __nv_bfloat16* dvrow = reinterpret_cast<__nv_bfloat16*>(a.dv) + rb + hh * 32;
+#pragma unroll
+                for (int c = 0; c < 32; c += 8) {
+                  uint4 pkv;
+                  pkv.x = pack_bf16x2(__uint_as_float(vv[c]), __uint_as_float(vv[c + 1]));
+                  pkv.y = pack_bf16x2(__uint_as_float(vv[c + 2]), __uint_as_float(vv[c + 3]));
+                  pkv.z = pack_bf16x2(__uint_as_float(vv[c + 4]), __uint_as_float(vv[c + 5]));
+                  pkv.w = pack_bf16x2(__uint_as_float(vv[c + 6]), __uint_as_float(vv[c + 7]));
+                  *reinterpret_cast<uint4*>(dvrow + c) = pkv;
+                }
               }
             }
           }
         }
-        {  // dK_hat (scaled) into the fp32 workspace
-          float dkv[128];
-          tmem_row128(t_row + 384, dkv);
+        {
+          uint32_t k0[32], k1[32];
+          tmem_ld32(t_row + 384 + c0, k0);
+          tmem_ld32(t_row + 384 + c0 + 32, k1);
+          tc_wait_ld_dep(k0);
+          tc_wait_ld_dep(k1);
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(smem_u32(&bars->acc_empty));
           if (valid_key) {
-            float* dkrow = a.dk_acc + rb;
 #pragma unroll
-            for (int c = 0; c < 128; c += 4)
-              *reinterpret_cast<float4*>(dkrow + c) =
-                  make_float4(dkv[c] * a.scale, dkv[c + 1] * a.scale, dkv[c + 2] * a.scale,
-                              dkv[c + 3] * a.scale);
+            for (int hh = 0; hh < 2; ++hh) {
+              const uint32_t* kv = hh ? k1 : k0;
+              float* dkrow = a.dk_acc + rb + hh * 32;
+#pragma unroll
+              for (int c = 0; c < 32; c += 4)
+                *reinterpret_cast<float4*>(dkrow + c) = make_float4(
+                    __uint_as_float(kv[c]) * a.scale, __uint_as_float(kv[c + 1]) * a.scale,
+                    __uint_as_float(kv[c + 2]) * a.scale, __uint_as_float(kv[c + 3]) * a.scale);
+            }
           }
         }
       }
@@ -483,10 +487,10 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q,
     }
     mbar_init(smem_u32(&bars->s_full), 1);
     mbar_init(smem_u32(&bars->dp_full), 1);
-    mbar_init(smem_u32(&bars->ds_full), 4);
+    mbar_init(smem_u32(&bars->ds_full), kMathWarps);
     mbar_init(smem_u32(&bars->dq_done), 1);
     mbar_init(smem_u32(&bars->acc_full), 1);
-    mbar_init(smem_u32(&bars->acc_empty), 4);
+    mbar_init(smem_u32(&bars->acc_empty), kMathWarps);
     mbar_init(smem_u32(&bars->drain), 1);
     fence_mbar_init();
   }
@@ -576,7 +580,7 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q,
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            mma_ts(tmem + 256, tmem + 0 + kk * 8, mnmajor_desc(kt, kk), idesc_ts,
+            mma_ts(tmem + 256, tmem + split_a_col(kk), mnmajor_desc(kt, kk), idesc_ts,
                    (n > 0 || kk > 0) ? 1u : 0u);
           mma_commit(smem_u32(&bars->dq_done));
           ++dq_count;
@@ -594,40 +598,52 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q,
     }
   } else {
     // ---------------------------------------------------------------- math warps
-    const int r = warp * 32 + lane;                // query row of the tile = TMEM lane
-    const uint32_t t_row = tmem + ((uint32_t)(warp * 32) << 16);
+    const int wg = warp >> 2;                      // column half: keys [64wg, 64wg+64)
+    const int r = (warp & 3) * 32 + lane;          // query row of the tile = TMEM lane
+    const uint32_t t_row = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+    const int c0 = 64 * wg;
     uint32_t item_count = 0, s_cnt = 0, dp_cnt = 0;
     bool ok = true;
     for (int idx = blockIdx.x; idx < n_items && ok; idx += gridDim.x) {
       const QItem it = decode_q(a, idx);
-      const int tok = it.q0 + r / a.G;
-      const int h = it.g * a.G + r % a.G;
+      const int tok = it.q0 + (r >> a.logG);
+      const int h = it.g * a.G + (r & (a.G - 1));
       const bool valid = tok < it.d1;
       const int lo_r = a.W > 0 ? max(it.d0, tok - a.W + 1) : it.d0;
       const float lse2 = valid ? __ldg(a.lse + (size_t)h * a.T + tok) * kLog2e : 0.f;
       const float Di = valid ? __ldg(a.dvec + (size_t)h * a.T + tok) : 0.f;
+      const uint64_t sc2 = f2(a.scale_log2, a.scale_log2);
+      const uint64_t nl2 = f2(-lse2, -lse2);
+      const uint64_t nd2 = f2(-Di, -Di);
       for (int n = 0; n < it.ntiles; ++n) {
         const int ks = it.kend - kTileKeys * (n + 1);
         const bool needs_mask = (ks + kTileKeys - 1 > it.q0) || (ks < it.d0) ||
                                 (a.W > 0 && ks < it.q0 + a.R - a.W);
+        const int c_lo = lo_r - ks, c_hi = tok - ks;
         ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->s_full), s_cnt & 1, wc));
         ++s_cnt;
         if (!ok) break;
         tc_fence_after();
-        uint32_t pk[64];
+        uint32_t pk[32];
         {
-          float sv[128];
-          tmem_row128(t_row + 0, sv);
-          const int c_lo = lo_r - ks, c_hi = tok - ks;
+          uint32_t u0[32], u1[32];
+          tmem_ld32(t_row + c0, u0);
+          tmem_ld32(t_row + c0 + 32, u1);
+          tc_wait_ld_dep(u0);
+          tc_wait_ld_dep(u1);
 #pragma unroll
-          for (int c = 0; c < 128; c += 2) {
-            float p0 = ex2_approx(fmaf(sv[c], a.scale_log2, -lse2));
-            float p1 = ex2_approx(fmaf(sv[c + 1], a.scale_log2, -lse2));
+          for (int e = 0; e < 32; ++e) {
+            const uint32_t a0 = e < 16 ? u0[2 * e] : u1[2 * e - 32];
+            const uint32_t a1 = e < 16 ? u0[2 * e + 1] : u1[2 * e - 31];
+            float x0, x1;
+            f2_split(ffma2(f2(__uint_as_float(a0), __uint_as_float(a1)), sc2, nl2), x0, x1);
+            float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
             if (needs_mask) {
+              const int c = c0 + 2 * e;
               p0 = (valid && c >= c_lo && c <= c_hi) ? p0 : 0.f;
               p1 = (valid && c + 1 >= c_lo && c + 1 <= c_hi) ? p1 : 0.f;
             }
-            pk[c >> 1] = pack_f16x2(p0, p1);
+            pk[e] = pack_f16x2(p0, p1);
           }
         }
         ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->dp_full), dp_cnt & 1, wc));
@@ -635,16 +651,23 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q,
         if (!ok) break;
         tc_fence_after();
         {
-          float dp[128];
-          tmem_row128(t_row + 128, dp);
-          uint32_t ds[64];
+          uint32_t u0[32], u1[32], ds[32];
+          tmem_ld32(t_row + 128 + c0, u0);
+          tmem_ld32(t_row + 128 + c0 + 32, u1);
+          tc_wait_ld_dep(u0);
+          tc_wait_ld_dep(u1);
 #pragma unroll
-          for (int c = 0; c < 128; c += 2) {
-            const float2 p = unpack_f16x2(pk[c >> 1]);
-            ds[c >> 1] = pack_f16x2(p.x * (dp[c] - Di), p.y * (dp[c + 1] - Di));
+          for (int e = 0; e < 32; ++e) {
+            const uint32_t a0 = e < 16 ? u0[2 * e] : u1[2 * e - 32];
+            const uint32_t a1 = e < 16 ? u0[2 * e + 1] : u1[2 * e - 31];
+            float y0, y1;
+            const float2 pr = unpack_f16x2(pk[e]);          // dS = P * (dP - D)
+            f2_split(fmul2(f2(pr.x, pr.y),
+                           fadd2(f2(__uint_as_float(a0), __uint_as_float(a1)), nd2)), y0, y1);
+            ds[e] = pack_f16x2(y0, y1);
           }
-          tmem_st32(t_row + 0, *reinterpret_cast<uint32_t(*)[32]>(&ds[0]));
-          tmem_st32(t_row + 32, *reinterpret_cast<uint32_t(*)[32]>(&ds[32]));
+          // dS for keys [c0, c0+64) into columns [c0, c0+32): read above by this thread
+          tmem_st32(t_row + c0, ds);
         }
         tc_wait_st();
         tc_fence_before();
@@ -656,18 +679,25 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q,
       if (!ok) break;
       tc_fence_after();
       {
-        float acc[128];
-        tmem_row128(t_row + 256, acc);
+        uint32_t u0[32], u1[32];
+        tmem_ld32(t_row + 256 + c0, u0);
+        tmem_ld32(t_row + 256 + c0 + 32, u1);
+        tc_wait_ld_dep(u0);
+        tc_wait_ld_dep(u1);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&bars->acc_empty));
         if (valid) {
-          float* row = a.dq_acc + ((size_t)tok * a.H + h) * kHeadDim;
+          float* row = a.dq_acc + ((size_t)tok * a.H + h) * kHeadDim + c0;
 #pragma unroll
-          for (int c = 0; c < 128; c += 4)
-            *reinterpret_cast<float4*>(row + c) = make_float4(acc[c] * a.scale, acc[c + 1] * a.scale,
-                                                              acc[c + 2] * a.scale,
-                                                              acc[c + 3] * a.scale);
+          for (int hh = 0; hh < 2; ++hh) {
+            const uint32_t* uu = hh ? u1 : u0;
+#pragma unroll
+            for (int c = 0; c < 32; c += 4)
+              *reinterpret_cast<float4*>(row + hh * 32 + c) = make_float4(
+                  __uint_as_float(uu[c]) * a.scale, __uint_as_float(uu[c + 1]) * a.scale,
+                  __uint_as_float(uu[c + 2]) * a.scale, __uint_as_float(uu[c + 3]) * a.scale);
+          }
         }
       }
       ++item_count;
