@@ -55,6 +55,7 @@ struct BwdArgs {
   const int4* items;
   const int* n_items;
   int max_items;
+  int* next_item;    // zeroed before the launch: dynamic item counter
   float* dq_acc;
   float* dk_acc;
   void* dv;          // float or bf16, per dv_f32
@@ -87,6 +88,7 @@ struct __align__(8) KvBars {
   uint64_t qd_full[2], qd_empty[2];
   uint64_t s_full, dp_full, p_full, ds_full, dv_done, dk_done, acc_full, acc_empty;
   uint64_t drain;
+  ItemRing ring;
 };
 constexpr uint32_t kKvOffK = 0;
 constexpr uint32_t kKvOffV = kTileBytes;
@@ -143,6 +145,7 @@ attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_q,
     mbar_init(smem_u32(&bars->acc_full), 1);
     mbar_init(smem_u32(&bars->acc_empty), kMathWarps);
     mbar_init(smem_u32(&bars->drain), 1);
+    ring_init(&bars->ring, kMathWarps + 1);
     fence_mbar_init();
   }
   if (warp == kWarpMma) {
@@ -156,11 +159,21 @@ attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_q,
   const int n_items = min(*a.n_items, a.max_items);
 
   if (warp == kWarpTma) {
-    // TMA issue from lane 0; the whole warp stages each query tile's per-row
+    // Lane 0 takes items from the global counter and issues TMA; the whole warp
+    // stages each query tile's per-row
     // log2-LSE and D into shared memory and completes qd_full's second arrival.
     uint32_t item_count = 0, qd_iter = 0, kv_arm = 0, qd_arm[2] = {0, 0};
     bool ok = true;
-    for (int idx = blockIdx.x; idx < n_items && ok; idx += gridDim.x) {
+    while (ok) {
+      int idx = -1;
+      if (lane == 0) {
+        idx = atomicAdd(a.next_item, 1);
+        if (idx >= n_items) idx = -1;
+        ok = ring_push(&bars->ring, item_count, idx, wc);
+      }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      idx = __shfl_sync(0xffffffffu, idx, 0);
+      if (!ok || idx < 0) break;
       const KvItem it = decode_kv(a, idx);
       if (lane == 0) {
         if (item_count > 0) ok = mbar_wait(smem_u32(&bars->kv_empty), (item_count - 1) & 1, wc);
@@ -214,41 +227,57 @@ attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_q,
       if (qd_arm[1]) mbar_wait(smem_u32(&bars->qd_full[1]), (qd_arm[1] - 1) & 1, drain);
     }
   } else if (warp == kWarpMma) {
+    // Issue order for query tile m: dV(m), S^T(m+1), dK(m), dP^T(m+1), so the
+    // softmax part of tile m+1 overlaps dK(m) and dP^T(m+1). S^T(m+1) and
+    // dP^T(m+1) overwrite the regions holding P^T(m) and dS^T(m); each waits
+    // for the completion of the MMA that reads them.
     if (lane == 0) {
       const uint32_t idesc_ss = make_idesc_f16(128, 128, 0, 0);
       const uint32_t idesc_ts = make_idesc_f16(128, 128, 0, 1);
       uint32_t item_count = 0, qd_iter = 0, dv_count = 0, dk_count = 0, p_cnt = 0, ds_cnt = 0;
       bool ok = true;
       const uint32_t kt = sbase + kKvOffK, vt = sbase + kKvOffV;
-      for (int idx = blockIdx.x; idx < n_items && ok; idx += gridDim.x) {
+      auto issue_s = [&](uint32_t qt) {
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ss(tmem + 0, kmajor_desc(kt, kk), kmajor_desc(qt, kk), idesc_ss, kk > 0);
+        mma_commit(smem_u32(&bars->s_full));
+      };
+      auto issue_dp = [&](uint32_t dot) {
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ss(tmem + 128, kmajor_desc(vt, kk), kmajor_desc(dot, kk), idesc_ss, kk > 0);
+        mma_commit(smem_u32(&bars->dp_full));
+      };
+      while (ok) {
+        int idx = -1;
+        ok = ring_pop1(&bars->ring, item_count, &idx, wc);
+        if (!ok || idx < 0) break;
         const KvItem it = decode_kv(a, idx);
         ok = mbar_wait(smem_u32(&bars->kv_full), item_count & 1, wc);
         if (!ok) break;
-        tc_fence_after();
-        for (int m = 0; m < it.nq && ok; ++m, ++qd_iter) {
-          const uint32_t s = qd_iter & 1, ph = (qd_iter >> 1) & 1;
-          const uint32_t qt = sbase + kKvOffQ + s * kTileBytes;
-          const uint32_t dot = sbase + kKvOffDO + s * kTileBytes;
-          ok = mbar_wait(smem_u32(&bars->qd_full[s]), ph, wc);
-          if (!ok) break;
-          if (dv_count > 0) ok = mbar_wait(smem_u32(&bars->dv_done), (dv_count - 1) & 1, wc);
+        {  // S^T and dP^T of the item's first query tile
+          const uint32_t s0 = qd_iter & 1, ph0 = (qd_iter >> 1) & 1;
+          ok = mbar_wait(smem_u32(&bars->qd_full[s0]), ph0, wc);
+          if (ok && dv_count > 0) ok = mbar_wait(smem_u32(&bars->dv_done), (dv_count - 1) & 1, wc);
           if (!ok) break;
           tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_ss(tmem + 0, kmajor_desc(kt, kk), kmajor_desc(qt, kk), idesc_ss, kk > 0);
-          mma_commit(smem_u32(&bars->s_full));
+          issue_s(sbase + kKvOffQ + s0 * kTileBytes);
           if (dk_count > 0) ok = mbar_wait(smem_u32(&bars->dk_done), (dk_count - 1) & 1, wc);
           if (!ok) break;
           tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_ss(tmem + 128, kmajor_desc(vt, kk), kmajor_desc(dot, kk), idesc_ss, kk > 0);
-          mma_commit(smem_u32(&bars->dp_full));
+          issue_dp(sbase + kKvOffDO + s0 * kTileBytes);
+        }
+        for (int m = 0; m < it.nq && ok; ++m, ++qd_iter) {
+          const uint32_t s = qd_iter & 1;
+          const uint32_t qt = sbase + kKvOffQ + s * kTileBytes;
+          const uint32_t dot = sbase + kKvOffDO + s * kTileBytes;
+          const bool has_next = m + 1 < it.nq;
+          const uint32_t s2 = (qd_iter + 1) & 1, ph2 = ((qd_iter + 1) >> 1) & 1;
+          // dV(m) += P^T(m) dO(m)
           ok = mbar_wait(smem_u32(&bars->p_full), p_cnt & 1, wc);
           ++p_cnt;
-          if (!ok) break;
-          if (m == 0 && item_count > 0)
+          if (ok && m == 0 && item_count > 0)
             ok = mbar_wait(smem_u32(&bars->acc_empty), (item_count - 1) & 1, wc);
           if (!ok) break;
           tc_fence_after();
@@ -258,6 +287,15 @@ attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_q,
                    (m > 0 || kk > 0) ? 1u : 0u);
           mma_commit(smem_u32(&bars->dv_done));
           ++dv_count;
+          // S^T(m+1) once dV(m) has read P^T(m)
+          if (has_next) {
+            ok = mbar_wait(smem_u32(&bars->qd_full[s2]), ph2, wc);
+            if (ok) ok = mbar_wait(smem_u32(&bars->dv_done), (dv_count - 1) & 1, wc);
+            if (!ok) break;
+            tc_fence_after();
+            issue_s(sbase + kKvOffQ + s2 * kTileBytes);
+          }
+          // dK(m) += dS^T(m) Q(m)
           ok = mbar_wait(smem_u32(&bars->ds_full), ds_cnt & 1, wc);
           ++ds_cnt;
           if (!ok) break;
@@ -269,6 +307,13 @@ attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_q,
           mma_commit(smem_u32(&bars->dk_done));
           ++dk_count;
           mma_commit(smem_u32(&bars->qd_empty[s]));
+          // dP^T(m+1) once dK(m) has read dS^T(m)
+          if (has_next) {
+            ok = mbar_wait(smem_u32(&bars->dk_done), (dk_count - 1) & 1, wc);
+            if (!ok) break;
+            tc_fence_after();
+            issue_dp(sbase + kKvOffDO + s2 * kTileBytes);
+          }
         }
         if (!ok) break;
         mma_commit(smem_u32(&bars->kv_empty));
@@ -288,7 +333,10 @@ attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_q,
     const uint32_t c0 = 64 * wg;                   // first column of this warpgroup
     uint32_t item_count = 0, s_cnt = 0, dp_cnt = 0, tile_count = 0;
     bool ok = true;
-    for (int idx = blockIdx.x; idx < n_items && ok; idx += gridDim.x) {
+    while (ok) {
+      int idx = -1;
+      ok = ring_pop(&bars->ring, item_count, &idx, wc);
+      if (!ok || idx < 0) break;
       const KvItem it = decode_kv(a, idx);
       const int j = it.k0 + kl;
       const bool valid_key = j < it.d1;
@@ -318,8 +366,9 @@ attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_q,
             const int c = c0 + 2 * e;
             const float s0 = __uint_as_float(e < 16 ? u0[2 * e] : u1[2 * e - 32]);
             const float s1 = __uint_as_float(e < 16 ? u0[2 * e + 1] : u1[2 * e - 31]);
-            float p0 = ex2_approx(fmaf(s0, a.scale_log2, -st[c]));
-            float p1 = ex2_approx(fmaf(s1, a.scale_log2, -st[c + 1]));
+            const float2 l2 = *reinterpret_cast<const float2*>(st + c);
+            float p0 = ex2_approx(fmaf(s0, a.scale_log2, -l2.x));
+            float p1 = ex2_approx(fmaf(s1, a.scale_log2, -l2.y));
             if (needs_mask) {
               const int t0 = qs + (c >> a.logG), t1 = qs + ((c + 1) >> a.logG);
               const bool v0 = valid_key && j <= t0 && t0 < it.d1 && (a.W <= 0 || t0 - j < a.W);
@@ -351,7 +400,8 @@ attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_q,
             const float d0 = __uint_as_float(e < 16 ? u0[2 * e] : u1[2 * e - 32]);
             const float d1 = __uint_as_float(e < 16 ? u0[2 * e + 1] : u1[2 * e - 31]);
             const float2 p = unpack_f16x2(pk[e]);
-            ds[e] = pack_f16x2(p.x * (d0 - st[128 + c]), p.y * (d1 - st[128 + c + 1]));
+            const float2 dd = *reinterpret_cast<const float2*>(st + 128 + c);
+            ds[e] = pack_f16x2(p.x * (d0 - dd.x), p.y * (d1 - dd.y));
           }
           tmem_st32(t_row + 128 + c0, ds);
         }
@@ -742,6 +792,7 @@ cudaError_t launch_attn_bwd_sm100_impl(const CUtensorMap& tq, const CUtensorMap&
   a.status = status;
 
   a.items = items_kv; a.n_items = n_kv; a.max_items = max_kv;
+  a.next_item = status + 4;
   int grid = num_sms < max_kv ? num_sms : max_kv;
   {
     ProfScope prof(kKBwdDkvSm100, st);
@@ -751,6 +802,7 @@ cudaError_t launch_attn_bwd_sm100_impl(const CUtensorMap& tq, const CUtensorMap&
   if (e != cudaSuccess) return e;
 
   a.items = items_q; a.n_items = n_q; a.max_items = max_q;
+  a.next_item = status + 5;
   grid = num_sms < max_q ? num_sms : max_q;
   ProfScope prof(kKBwdDqSm100, st);
   attn_bwd_dq_kernel<<<grid > 0 ? grid : 1, kThreads, kQSmem, st>>>(tq, tk, tv, tdo, a);

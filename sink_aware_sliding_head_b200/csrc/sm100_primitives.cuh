@@ -75,6 +75,52 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const W
   }
 }
 
+// ---------------------------------------------------------------- dynamic work items
+// A persistent CTA takes its next work item from a global counter (one
+// atomicAdd by the TMA thread) and hands the index to its other roles through
+// a small ring in shared memory. Over a list sorted heaviest first this is
+// greedy longest-processing-time scheduling. Index -1 ends the CTA's loop.
+constexpr int kItemSlots = 4;
+struct ItemRing {
+  int idx[kItemSlots];
+  uint64_t full[kItemSlots];    // 1 arrival: the fetching thread
+  uint64_t empty[kItemSlots];   // one arrival per consuming warp
+};
+__device__ __forceinline__ void ring_init(ItemRing* r, uint32_t consumers) {
+  for (int s = 0; s < kItemSlots; ++s) {
+    mbar_init(smem_u32(&r->full[s]), 1);
+    mbar_init(smem_u32(&r->empty[s]), consumers);
+  }
+}
+// Fetching thread: publish the k-th item index of this CTA (k counts from 0).
+__device__ __forceinline__ bool ring_push(ItemRing* r, uint32_t k, int idx, const WaitCtx& w) {
+  const uint32_t s = k % kItemSlots;
+  if (k >= (uint32_t)kItemSlots &&
+      !mbar_wait(smem_u32(&r->empty[s]), ((k / kItemSlots) - 1) & 1, w))
+    return false;
+  r->idx[s] = idx;
+  mbar_arrive(smem_u32(&r->full[s]));       // release: the index is visible after the wait
+  return true;
+}
+// Consuming warp (all lanes): read the k-th item index; lane 0 frees the slot.
+__device__ __forceinline__ bool ring_pop(ItemRing* r, uint32_t k, int* idx, const WaitCtx& w) {
+  const uint32_t s = k % kItemSlots;
+  const bool ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&r->full[s]), (k / kItemSlots) & 1, w));
+  if (!ok) return false;
+  *idx = *reinterpret_cast<volatile int*>(&r->idx[s]);
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(smem_u32(&r->empty[s]));
+  return true;
+}
+// Single consuming thread (e.g. the MMA issuer) that stands for its warp.
+__device__ __forceinline__ bool ring_pop1(ItemRing* r, uint32_t k, int* idx, const WaitCtx& w) {
+  const uint32_t s = k % kItemSlots;
+  if (!mbar_wait(smem_u32(&r->full[s]), (k / kItemSlots) & 1, w)) return false;
+  *idx = *reinterpret_cast<volatile int*>(&r->idx[s]);
+  mbar_arrive(smem_u32(&r->empty[s]));
+  return true;
+}
+
 // ---------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* m) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
