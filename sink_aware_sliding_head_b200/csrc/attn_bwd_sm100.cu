@@ -29,7 +29,9 @@
 //    operands. dK and dV stay in TMEM for the whole key tile, so the G heads
 //    of a group are summed without atomics. TMEM: S^T, dP^T, dV, dK = 512 cols.
 //  * dq: query-major. A CTA owns one 128-row query tile and streams its key
-//    tiles: S = Q K^T, dP = dO V^T, dS (fp16) over S, dQ += dS K. TMEM 384 cols.
+//    tiles: S = Q K^T, dP = dO V^T, dS (fp16) over S, dQ += dS K. TMEM: two S
+//    buffers, dP, dQ = 512 cols; S of the next key tile is computed while the
+//    math warps finish the current one.
 // Before an MMA overwrites a TMEM region that a previous MMA reads as its A
 // operand, the issuer waits for that MMA's completion barrier.
 #include "common.cuh"
@@ -487,8 +489,10 @@ attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_q,
 struct __align__(8) QBars {
   uint64_t qd_full, qd_empty;
   uint64_t kv_full[2], kv_empty[2];
-  uint64_t s_full, dp_full, ds_full, dq_done, acc_full, acc_empty;
+  uint64_t s_full[2], dq_done[2];     // per S buffer
+  uint64_t dp_full, ds_full, acc_full, acc_empty;
   uint64_t drain;
+  ItemRing ring;
 };
 constexpr uint32_t kQOffQ = 0;
 constexpr uint32_t kQOffDO = kTileBytes;
@@ -498,6 +502,8 @@ constexpr uint32_t kQOffBar = kQOffV + 2 * kTileBytes;
 constexpr uint32_t kQOffTmem = kQOffBar + sizeof(QBars);
 constexpr uint32_t kQOffAbort = kQOffTmem + 16;
 constexpr uint32_t kQSmem = kQOffAbort + 16 + 1024;
+// TMEM columns: S double-buffered, dP, dQ accumulator
+constexpr uint32_t kQColS0 = 0, kQColDP = 256, kQColDQ = 384;
 
 struct QItem {
   int q0, d0, d1, g, kend, kbeg, ntiles;
@@ -512,6 +518,8 @@ __device__ __forceinline__ QItem decode_q(const BwdArgs& a, int idx) {
   return r;
 }
 
+// Tiles are numbered per CTA across items (t = 0, 1, ...): tile t uses S
+// buffer t % 2 and K/V stage t % 2.
 __global__ void __launch_bounds__(kThreads, 1)
 attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q,
                    const __grid_constant__ CUtensorMap tm_k,
@@ -534,14 +542,15 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q,
     for (int s = 0; s < 2; ++s) {
       mbar_init(smem_u32(&bars->kv_full[s]), 1);
       mbar_init(smem_u32(&bars->kv_empty[s]), 1);
+      mbar_init(smem_u32(&bars->s_full[s]), 1);
+      mbar_init(smem_u32(&bars->dq_done[s]), 1);
     }
-    mbar_init(smem_u32(&bars->s_full), 1);
     mbar_init(smem_u32(&bars->dp_full), 1);
     mbar_init(smem_u32(&bars->ds_full), kMathWarps);
-    mbar_init(smem_u32(&bars->dq_done), 1);
     mbar_init(smem_u32(&bars->acc_full), 1);
     mbar_init(smem_u32(&bars->acc_empty), kMathWarps);
     mbar_init(smem_u32(&bars->drain), 1);
+    ring_init(&bars->ring, kMathWarps + 1);
     fence_mbar_init();
   }
   if (warp == kWarpMma) {
@@ -556,9 +565,13 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q,
 
   if (warp == kWarpTma) {
     if (lane == 0) {
-      uint32_t item_count = 0, kv_iter = 0, qd_arm = 0, kv_arm[2] = {0, 0};
+      uint32_t item_count = 0, kv_iter = 0, qd_arm = 0, kv_arm0 = 0, kv_arm1 = 0;
       bool ok = true;
-      for (int idx = blockIdx.x; idx < n_items && ok; idx += gridDim.x) {
+      while (ok) {
+        int idx = atomicAdd(a.next_item, 1);
+        if (idx >= n_items) idx = -1;
+        ok = ring_push(&bars->ring, item_count, idx, wc);
+        if (!ok || idx < 0) break;
         const QItem it = decode_q(a, idx);
         if (item_count > 0) ok = mbar_wait(smem_u32(&bars->qd_empty), (item_count - 1) & 1, wc);
         if (!ok) break;
@@ -576,7 +589,7 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q,
           if (!ok) break;
           const uint32_t kf = smem_u32(&bars->kv_full[s]);
           mbar_arrive_expect_tx(kf, 2 * kTileBytes);
-          ++kv_arm[s];
+          if (s == 0) ++kv_arm0; else ++kv_arm1;
           for (int c = 0; c < 2; ++c) {
             tma_load_3d(sbase + kQOffK + s * kTileBytes + c * kChunkBytes, &tm_k, kf, c * 64, it.g,
                         ks);
@@ -589,52 +602,69 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q,
       volatile int no_abort = 0;
       const WaitCtx drain{&no_abort, a.status, kStatusTimeoutBwdQ};
       if (qd_arm) mbar_wait(smem_u32(&bars->qd_full), (qd_arm - 1) & 1, drain);
-      if (kv_arm[0]) mbar_wait(smem_u32(&bars->kv_full[0]), (kv_arm[0] - 1) & 1, drain);
-      if (kv_arm[1]) mbar_wait(smem_u32(&bars->kv_full[1]), (kv_arm[1] - 1) & 1, drain);
+      if (kv_arm0) mbar_wait(smem_u32(&bars->kv_full[0]), (kv_arm0 - 1) & 1, drain);
+      if (kv_arm1) mbar_wait(smem_u32(&bars->kv_full[1]), (kv_arm1 - 1) & 1, drain);
     }
   } else if (warp == kWarpMma) {
+    // Per tile t: dP(t), S(t+1) (into the other S buffer, once dQ(t-1) has read
+    // it), dQ(t). P of tile t+1 is then computed while dQ(t) and dP(t+1) run.
     if (lane == 0) {
       const uint32_t idesc_ss = make_idesc_f16(128, 128, 0, 0);
       const uint32_t idesc_ts = make_idesc_f16(128, 128, 0, 1);
-      uint32_t item_count = 0, kv_iter = 0, dq_count = 0, ds_cnt = 0;
+      uint32_t item_count = 0, t = 0, ds_cnt = 0, dq_cnt0 = 0, dq_cnt1 = 0;
       bool ok = true;
       const uint32_t qt = sbase + kQOffQ, dot = sbase + kQOffDO;
-      for (int idx = blockIdx.x; idx < n_items && ok; idx += gridDim.x) {
+      // S(tt) = Q K(tt)^T into buffer tt % 2, after the dQ that last read it.
+      auto issue_s = [&](uint32_t tt) -> bool {
+        const uint32_t b = tt & 1, st = tt & 1, ph = (tt >> 1) & 1;
+        if (!mbar_wait(smem_u32(&bars->kv_full[st]), ph, wc)) return false;
+        const uint32_t cnt = b ? dq_cnt1 : dq_cnt0;
+        if (cnt > 0 && !mbar_wait(smem_u32(&bars->dq_done[b]), (cnt - 1) & 1, wc)) return false;
+        tc_fence_after();
+        const uint32_t kt = sbase + kQOffK + st * kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ss(tmem + kQColS0 + b * 128, kmajor_desc(qt, kk), kmajor_desc(kt, kk), idesc_ss,
+                 kk > 0);
+        mma_commit(smem_u32(&bars->s_full[b]));
+        return true;
+      };
+      while (ok) {
+        int idx = -1;
+        ok = ring_pop1(&bars->ring, item_count, &idx, wc);
+        if (!ok || idx < 0) break;
         const QItem it = decode_q(a, idx);
         ok = mbar_wait(smem_u32(&bars->qd_full), item_count & 1, wc);
         if (!ok) break;
         tc_fence_after();
-        for (int n = 0; n < it.ntiles && ok; ++n, ++kv_iter) {
-          const uint32_t s = kv_iter & 1, ph = (kv_iter >> 1) & 1;
-          const uint32_t kt = sbase + kQOffK + s * kTileBytes;
-          const uint32_t vt = sbase + kQOffV + s * kTileBytes;
-          ok = mbar_wait(smem_u32(&bars->kv_full[s]), ph, wc);
-          if (!ok) break;
-          if (dq_count > 0) ok = mbar_wait(smem_u32(&bars->dq_done), (dq_count - 1) & 1, wc);
-          if (!ok) break;
-          tc_fence_after();
+        ok = issue_s(t);
+        for (int n = 0; n < it.ntiles && ok; ++n, ++t) {
+          const uint32_t st = t & 1;
+          const uint32_t vt = sbase + kQOffV + st * kTileBytes;
+          const uint32_t kt = sbase + kQOffK + st * kTileBytes;
+          // dP(t) = dO V(t)^T; the math warps finished reading dP(t-1) before ds_full(t-1)
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            mma_ss(tmem + 0, kmajor_desc(qt, kk), kmajor_desc(kt, kk), idesc_ss, kk > 0);
-          mma_commit(smem_u32(&bars->s_full));
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_ss(tmem + 128, kmajor_desc(dot, kk), kmajor_desc(vt, kk), idesc_ss, kk > 0);
+            mma_ss(tmem + kQColDP, kmajor_desc(dot, kk), kmajor_desc(vt, kk), idesc_ss, kk > 0);
           mma_commit(smem_u32(&bars->dp_full));
+          if (n + 1 < it.ntiles) {
+            ok = issue_s(t + 1);
+            if (!ok) break;
+          }
           ok = mbar_wait(smem_u32(&bars->ds_full), ds_cnt & 1, wc);
           ++ds_cnt;
-          if (!ok) break;
-          if (n == 0 && item_count > 0)
+          if (ok && n == 0 && item_count > 0)
             ok = mbar_wait(smem_u32(&bars->acc_empty), (item_count - 1) & 1, wc);
           if (!ok) break;
           tc_fence_after();
+          const uint32_t b = t & 1;
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            mma_ts(tmem + 256, tmem + split_a_col(kk), mnmajor_desc(kt, kk), idesc_ts,
-                   (n > 0 || kk > 0) ? 1u : 0u);
-          mma_commit(smem_u32(&bars->dq_done));
-          ++dq_count;
-          mma_commit(smem_u32(&bars->kv_empty[s]));
+            mma_ts(tmem + kQColDQ, tmem + kQColS0 + b * 128 + split_a_col(kk), mnmajor_desc(kt, kk),
+                   idesc_ts, (n > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(smem_u32(&bars->dq_done[b]));
+          if (b) ++dq_cnt1; else ++dq_cnt0;
+          mma_commit(smem_u32(&bars->kv_empty[st]));
         }
         if (!ok) break;
         mma_commit(smem_u32(&bars->qd_empty));
@@ -652,9 +682,12 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q,
     const int r = (warp & 3) * 32 + lane;          // query row of the tile = TMEM lane
     const uint32_t t_row = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     const int c0 = 64 * wg;
-    uint32_t item_count = 0, s_cnt = 0, dp_cnt = 0;
+    uint32_t item_count = 0, t = 0;
     bool ok = true;
-    for (int idx = blockIdx.x; idx < n_items && ok; idx += gridDim.x) {
+    while (ok) {
+      int idx = -1;
+      ok = ring_pop(&bars->ring, item_count, &idx, wc);
+      if (!ok || idx < 0) break;
       const QItem it = decode_q(a, idx);
       const int tok = it.q0 + (r >> a.logG);
       const int h = it.g * a.G + (r & (a.G - 1));
@@ -665,20 +698,21 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q,
       const uint64_t sc2 = f2(a.scale_log2, a.scale_log2);
       const uint64_t nl2 = f2(-lse2, -lse2);
       const uint64_t nd2 = f2(-Di, -Di);
-      for (int n = 0; n < it.ntiles; ++n) {
+      for (int n = 0; n < it.ntiles; ++n, ++t) {
+        const uint32_t b = t & 1;
+        const uint32_t s_col = kQColS0 + b * 128;
         const int ks = it.kend - kTileKeys * (n + 1);
         const bool needs_mask = (ks + kTileKeys - 1 > it.q0) || (ks < it.d0) ||
                                 (a.W > 0 && ks < it.q0 + a.R - a.W);
         const int c_lo = lo_r - ks, c_hi = tok - ks;
-        ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->s_full), s_cnt & 1, wc));
-        ++s_cnt;
+        ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->s_full[b]), (t >> 1) & 1, wc));
         if (!ok) break;
         tc_fence_after();
         uint32_t pk[32];
         {
           uint32_t u0[32], u1[32];
-          tmem_ld32(t_row + c0, u0);
-          tmem_ld32(t_row + c0 + 32, u1);
+          tmem_ld32(t_row + s_col + c0, u0);
+          tmem_ld32(t_row + s_col + c0 + 32, u1);
           tc_wait_ld_dep(u0);
           tc_wait_ld_dep(u1);
 #pragma unroll
@@ -696,14 +730,13 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q,
             pk[e] = pack_f16x2(p0, p1);
           }
         }
-        ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->dp_full), dp_cnt & 1, wc));
-        ++dp_cnt;
+        ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->dp_full), t & 1, wc));
         if (!ok) break;
         tc_fence_after();
         {
           uint32_t u0[32], u1[32], ds[32];
-          tmem_ld32(t_row + 128 + c0, u0);
-          tmem_ld32(t_row + 128 + c0 + 32, u1);
+          tmem_ld32(t_row + kQColDP + c0, u0);
+          tmem_ld32(t_row + kQColDP + c0 + 32, u1);
           tc_wait_ld_dep(u0);
           tc_wait_ld_dep(u1);
 #pragma unroll
@@ -716,8 +749,8 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q,
                            fadd2(f2(__uint_as_float(a0), __uint_as_float(a1)), nd2)), y0, y1);
             ds[e] = pack_f16x2(y0, y1);
           }
-          // dS for keys [c0, c0+64) into columns [c0, c0+32): read above by this thread
-          tmem_st32(t_row + c0, ds);
+          // dS for keys [c0, c0+64) into S-buffer columns [c0, c0+32), read above
+          tmem_st32(t_row + s_col + c0, ds);
         }
         tc_wait_st();
         tc_fence_before();
@@ -730,8 +763,8 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q,
       tc_fence_after();
       {
         uint32_t u0[32], u1[32];
-        tmem_ld32(t_row + 256 + c0, u0);
-        tmem_ld32(t_row + 256 + c0 + 32, u1);
+        tmem_ld32(t_row + kQColDQ + c0, u0);
+        tmem_ld32(t_row + kQColDQ + c0 + 32, u1);
         tc_wait_ld_dep(u0);
         tc_wait_ld_dep(u1);
         tc_fence_before();
