@@ -177,6 +177,12 @@ int flint_attn_profile_collect(int max_kernels, const char** names, double* tota
 void flint_attn_profile_reset(void);
 long long flint_attn_launch_count(void);
 
+/* Diagnostic: y[i] = the kernels' FMA-pipe evaluation of 2^x[i] (range
+ * reduction + degree-3 minimax polynomial; relative error <= 7.5e-5 for
+ * x >= -125, inputs below -125 are clamped to it). x, y: device fp32 [n],
+ * n even. Asynchronous on `stream`. */
+flint_status_t flint_attn_exp2_poly(const float* x, float* y, int32_t n, void* stream);
+
 /* Static description of a status code. */
 const char* flint_status_string(flint_status_t status);
 

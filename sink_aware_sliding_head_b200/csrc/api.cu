@@ -15,6 +15,7 @@ namespace flint {
 
 cudaError_t launch_reduce_rows(const float* part, int nrows, int width, float* out,
                                cudaStream_t st);
+cudaError_t launch_exp2_poly(const float* x, float* y, int n, cudaStream_t st);
 cudaError_t launch_attn_fwd_sm100_impl(const CUtensorMap& tq, const CUtensorMap& tk,
                                        const CUtensorMap& tv, const Resolved& p, const float* sink,
                                        const int4* items, const int* n_items, int max_items,
@@ -363,6 +364,12 @@ extern "C" long long flint_attn_launch_count(void) {
   Prof& P = prof();
   std::lock_guard<std::mutex> g(P.mu);
   return P.launches_total;
+}
+
+extern "C" flint_status_t flint_attn_exp2_poly(const float* x, float* y, int32_t n, void* stream) {
+  if (n < 0 || (n & 1) || (n > 0 && (!x || !y || !aligned(x, 4) || !aligned(y, 4))))
+    return FLINT_ERR_INVALID_ARG;
+  return cuda_status(launch_exp2_poly(x, y, n, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 extern "C" const char* flint_status_string(flint_status_t s) {

@@ -9,6 +9,7 @@
 // summed per block in a fixed order, and the per-block partials are summed in a
 // fixed order by a second tiny launch, so the result is deterministic.
 #include "common.cuh"
+#include "sm100_primitives.cuh"
 
 namespace flint {
 
@@ -88,7 +89,22 @@ __global__ void convert_f16_kernel(const __nv_bfloat16* __restrict__ src, __half
   }
 }
 
+__global__ void exp2_poly_kernel(const float* __restrict__ x, float* __restrict__ y, int n2) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n2; i += gridDim.x * blockDim.x) {
+    float p0, p1;
+    exp2_fma2(x[2 * i], x[2 * i + 1], p0, p1);
+    y[2 * i] = p0;
+    y[2 * i + 1] = p1;
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_exp2_poly(const float* x, float* y, int n, cudaStream_t st) {
+  if (n <= 0) return cudaSuccess;
+  exp2_poly_kernel<<<(n / 2 + 255) / 256, 256, 0, st>>>(x, y, n / 2);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_convert_f16(const __nv_bfloat16* src, __half* dst, size_t n, cudaStream_t st) {
   const size_t n8 = n / 8;

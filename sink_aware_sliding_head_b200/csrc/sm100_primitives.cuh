@@ -307,6 +307,29 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
 }
+// 2^x for two lanes on the FMA/ALU pipes instead of the MUFU unit:
+// 2^x = 2^n * p(f), n = round(x) (adding 1.5*2^23 leaves n in the low mantissa
+// bits), f = x - n in [-1/2, 1/2], p the degree-3 minimax polynomial for 2^f
+// in relative error (max 7.5e-5; derive_exp2_poly.py), and 2^n applied by
+// adding n to the exponent field. x is clamped to >= -125 so the result stays
+// a normal float (p >= 0.7 keeps the exponent field >= 1); masked -inf inputs
+// give about 2^-125, i.e. zero after rounding to 16 bits.
+__device__ __forceinline__ void exp2_fma2(float x0, float x1, float& p0, float& p1) {
+  constexpr float kRound = 12582912.0f;                  // 1.5 * 2^23
+  constexpr float c0 = 0.99992806f, c1 = 0.69326085f, c2 = 0.24261115f, c3 = 0.05517222f;
+  const uint64_t xc = f2(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
+  const uint64_t t = fadd2(xc, f2(kRound, kRound));
+  const uint64_t nf = fadd2(t, f2(-kRound, -kRound));
+  const uint64_t fr = ffma2(nf, f2(-1.f, -1.f), xc);
+  uint64_t p = ffma2(f2(c3, c3), fr, f2(c2, c2));
+  p = ffma2(p, fr, f2(c1, c1));
+  p = ffma2(p, fr, f2(c0, c0));
+  float t0, t1, q0, q1;
+  f2_split(t, t0, t1);
+  f2_split(p, q0, q1);
+  p0 = __int_as_float(__float_as_int(q0) + (__float_as_int(t0) << 23));
+  p1 = __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
+}
 __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
   __half2 v = __floats2half2_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);

@@ -28,7 +28,7 @@ EXPORTED = ["flint_attn_workspace_bytes", "flint_attn_fwd", "flint_attn_bwd",
             "flint_attn_check_status", "flint_status_string", "flint_attn_version",
             "flint_attn_profile_enable", "flint_attn_profile_collect",
             "flint_attn_profile_reset", "flint_attn_launch_count",
-            "flint_attn_bwd_preprocess_static"]
+            "flint_attn_bwd_preprocess_static", "flint_attn_exp2_poly"]
 
 
 class Params(ctypes.Structure):
@@ -93,6 +93,8 @@ def load_library(path: str = LIB_PATH):
     lib.flint_attn_launch_count.restype = ctypes.c_longlong
     lib.flint_attn_bwd_preprocess_static.argtypes = [P] + [vp] * 6 + [vp]
     lib.flint_attn_bwd_preprocess_static.restype = ctypes.c_int
+    lib.flint_attn_exp2_poly.argtypes = [vp, vp, ctypes.c_int32, vp]
+    lib.flint_attn_exp2_poly.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -257,6 +259,14 @@ def bwd_preprocess_static(out, dout, lse, sink, fp32_out=False, d_rowsum=None, d
                                                 _stream_ptr(stream))
     _check(code, "flint_attn_bwd_preprocess_static")
     return d_rowsum, dsink
+
+
+def exp2_poly(x: torch.Tensor) -> torch.Tensor:
+    """Diagnostic: the kernels' FMA-pipe 2^x evaluated on the device (fp32, even length)."""
+    y = torch.empty_like(x)
+    _check(load_library().flint_attn_exp2_poly(_ptr(x), _ptr(y), x.numel(), _stream_ptr()),
+           "flint_attn_exp2_poly")
+    return y
 
 
 def version() -> str:

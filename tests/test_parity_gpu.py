@@ -247,3 +247,22 @@ def test_bf16_backward_prefix_whole_layer(cuda_lib, wl, n_tok, n_docs):
     ref = fo.flint_attn_bwd(p["q"], p["k"], p["v"], p["w_q"], p["w_k"], p["sink"],
                             p["cu_doc_lens"], wl.window, wl.use_rope, wl.rope_theta, p["dout"])
     check_grads(g, ref)
+
+
+# ----------------------------------------------------------------------- FMA-pipe exp2
+
+def test_fma_pipe_exp2_error_bound(cuda_lib):
+    """The polynomial exp2 used for part of the softmax stays within 7.5e-5 relative."""
+    x = torch.linspace(-125.0, 9.0, 1 << 20, dtype=torch.float64)
+    x = torch.cat([x, torch.rand(1 << 16, dtype=torch.float64) - 0.5])
+    xf = x.float().cuda()
+    y = cuda_lib.exp2_poly(xf).double().cpu()
+    ref = torch.exp2(xf.double().cpu())
+    rel = ((y - ref).abs() / ref).max().item()
+    assert rel <= 7.6e-5, rel
+    # exactly 1 at 0, monotone enough that no value is negative or NaN
+    assert torch.isfinite(y).all() and (y > 0).all()
+    # inputs below -125 (including -inf from the mask) clamp to about 2^-125
+    low = cuda_lib.exp2_poly(torch.tensor([-float("inf"), -1e30, -200.0, -126.5],
+                                          device="cuda")).cpu()
+    assert (low <= 2.0 ** -124).all() and (low > 0).all()
