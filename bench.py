@@ -166,6 +166,25 @@ def traffic_for(kernel, workload):
     return None
 
 
+def aggregate(times_ms, world, flops_step, steps, pg=None):
+    """Whole-job numbers from this rank's CUDA-event times.
+
+    times_ms: this rank's [total, fwd, bwd] milliseconds over `steps` steps. The
+    slowest rank defines the step time (max over ranks through `pg`, any
+    torch.distributed backend); every rank processed its own batch (weak
+    scaling), so the job's throughput is world * flops_step * steps / time.
+    Returns (value TFLOP/s, [total, fwd, bwd] ms maxed over ranks).
+    """
+    t = torch.tensor(list(times_ms), dtype=torch.float64)
+    if pg is not None:
+        dev = torch.device("cuda", torch.cuda.current_device()) if \
+            pg.get_backend() == "nccl" else torch.device("cpu")
+        t = t.to(dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    t = [float(x) for x in t.cpu().tolist()]
+    return world * flops_step * steps / (t[0] * 1e-3) / 1e12, t
+
+
 # --------------------------------------------------------------------------- CPU oracle
 
 def oracle_sample(w, inp, seconds):
@@ -356,13 +375,9 @@ def main(argv=None):
     clk = clocks.stop() if clocks else None
     fwd_ms = sum(e[0].elapsed_time(e[1]) for e in ev)
     bwd_ms = sum(e[1].elapsed_time(e[2]) for e in ev)
-    tot_ms = fwd_ms + bwd_ms
-    t_local = torch.tensor([tot_ms, fwd_ms, bwd_ms], dtype=torch.float64, device=dev)
-    if pg is not None:
-        pg.all_reduce(t_local, op=pg.ReduceOp.MAX)
-    tot_ms, fwd_ms, bwd_ms = [float(x) for x in t_local.tolist()]
+    value, (tot_ms, fwd_ms, bwd_ms) = aggregate([fwd_ms + bwd_ms, fwd_ms, bwd_ms], world,
+                                                flops_step, args.steps, pg)
     ms_step = tot_ms / args.steps
-    value = world * flops_step * args.steps / (tot_ms * 1e-3) / 1e12
 
     # ---- end to end: host (pinned) inputs -> device -> both calls -> host results
     e2e = None
@@ -400,12 +415,9 @@ def main(argv=None):
         e1.record(stream)
         torch.cuda.synchronize(dev)
         barrier()
-        t_e2e = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
-        if pg is not None:
-            pg.all_reduce(t_e2e, op=pg.ReduceOp.MAX)
-        e2e = {"value": world * flops_step * args.steps / (float(t_e2e.item()) * 1e-3) / 1e12,
-               "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-               "ms_per_step": float(t_e2e.item()) / args.steps}
+        e2e_val, (t_e2e,) = aggregate([e0.elapsed_time(e1)], world, flops_step, args.steps, pg)
+        e2e = {"value": e2e_val, "unit": UNIT, "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "ms_per_step": t_e2e / args.steps}
 
     if rank != 0:
         if pg is not None:
