@@ -24,16 +24,20 @@
 // operand of the following MMA skips from column 32 to 64 halfway through K.
 //  * dkv: key-major. A CTA owns 128 keys of one KV head and streams the
 //    128-row query tiles (R tokens x G heads) that see them. Per tile:
-//    S^T = K Q^T and dP^T = V dO^T (TMEM), then P^T and dS^T in fp16 overwrite
-//    their first 64 columns and feed dV += P^T dO and dK += dS^T Q as TMEM A
-//    operands. dK and dV stay in TMEM for the whole key tile, so the G heads
-//    of a group are summed without atomics. TMEM: S^T, dP^T, dV, dK = 512 cols.
+//    S^T = K Q^T and dP^T = V dO^T (TMEM), then P^T and dS^T in fp16 are
+//    written over S^T and feed dV += P^T dO and dK += dS^T Q as TMEM A
+//    operands. The S^T and dP^T regions swap roles every tile, so the next
+//    S^T never waits for an MMA to finish. dK and dV stay in TMEM for the whole
+//    key tile, so the G heads of a group are summed without atomics. TMEM:
+//    2 x 128 rotating columns + dV + dK = 512 cols.
 //  * dq: query-major. A CTA owns one 128-row query tile and streams its key
 //    tiles: S = Q K^T, dP = dO V^T, dS (fp16) over S, dQ += dS K. TMEM: two S
 //    buffers, dP, dQ = 512 cols; S of the next key tile is computed while the
 //    math warps finish the current one.
 // Before an MMA overwrites a TMEM region that a previous MMA reads as its A
 // operand, the issuer waits for that MMA's completion barrier.
+#include <type_traits>
+
 #include "common.cuh"
 #include "sm100_primitives.cuh"
 
@@ -229,26 +233,31 @@ attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_q,
       if (qd_arm[1]) mbar_wait(smem_u32(&bars->qd_full[1]), (qd_arm[1] - 1) & 1, drain);
     }
   } else if (warp == kWarpMma) {
-    // Issue order for query tile m: dV(m), S^T(m+1), dK(m), dP^T(m+1), so the
-    // softmax part of tile m+1 overlaps dK(m) and dP^T(m+1). S^T(m+1) and
-    // dP^T(m+1) overwrite the regions holding P^T(m) and dS^T(m); each waits
-    // for the completion of the MMA that reads them.
+    // TMEM regions R0 = [0,128), R1 = [128,256) rotate between query tiles
+    // (numbered t across items): S^T(t) goes to X_t = R(t&1), dP^T(t) to
+    // Y_t = R(~t&1). The math warps write P^T(t) and dS^T(t) into X_t, so Y_t
+    // is free once they have read dP^T(t) (ds_full). Issue order per tile:
+    // dV(t), S^T(t+1) into Y_t, dK(t), then - after dK(t) has completed, as it
+    // reads X_t - dP^T(t+1) into X_t.
     if (lane == 0) {
       const uint32_t idesc_ss = make_idesc_f16(128, 128, 0, 0);
       const uint32_t idesc_ts = make_idesc_f16(128, 128, 0, 1);
-      uint32_t item_count = 0, qd_iter = 0, dv_count = 0, dk_count = 0, p_cnt = 0, ds_cnt = 0;
+      uint32_t item_count = 0, t = 0, dk_count = 0, p_cnt = 0, ds_cnt = 0;
       bool ok = true;
       const uint32_t kt = sbase + kKvOffK, vt = sbase + kKvOffV;
-      auto issue_s = [&](uint32_t qt) {
+      auto region = [&](uint32_t r) { return tmem + (r & 1) * 128; };
+      auto issue_s = [&](uint32_t tt) {          // S^T(tt) into X_tt
+        const uint32_t qt = sbase + kKvOffQ + (tt & 1) * kTileBytes;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_ss(tmem + 0, kmajor_desc(kt, kk), kmajor_desc(qt, kk), idesc_ss, kk > 0);
+          mma_ss(region(tt), kmajor_desc(kt, kk), kmajor_desc(qt, kk), idesc_ss, kk > 0);
         mma_commit(smem_u32(&bars->s_full));
       };
-      auto issue_dp = [&](uint32_t dot) {
+      auto issue_dp = [&](uint32_t tt) {         // dP^T(tt) into Y_tt
+        const uint32_t dot = sbase + kKvOffDO + (tt & 1) * kTileBytes;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_ss(tmem + 128, kmajor_desc(vt, kk), kmajor_desc(dot, kk), idesc_ss, kk > 0);
+          mma_ss(region(tt + 1), kmajor_desc(vt, kk), kmajor_desc(dot, kk), idesc_ss, kk > 0);
         mma_commit(smem_u32(&bars->dp_full));
       };
       while (ok) {
@@ -259,24 +268,22 @@ attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_q,
         ok = mbar_wait(smem_u32(&bars->kv_full), item_count & 1, wc);
         if (!ok) break;
         {  // S^T and dP^T of the item's first query tile
-          const uint32_t s0 = qd_iter & 1, ph0 = (qd_iter >> 1) & 1;
-          ok = mbar_wait(smem_u32(&bars->qd_full[s0]), ph0, wc);
-          if (ok && dv_count > 0) ok = mbar_wait(smem_u32(&bars->dv_done), (dv_count - 1) & 1, wc);
+          ok = mbar_wait(smem_u32(&bars->qd_full[t & 1]), (t >> 1) & 1, wc);
           if (!ok) break;
           tc_fence_after();
-          issue_s(sbase + kKvOffQ + s0 * kTileBytes);
+          issue_s(t);                            // X_t = Y_{t-1}: free after ds_full(t-1)
           if (dk_count > 0) ok = mbar_wait(smem_u32(&bars->dk_done), (dk_count - 1) & 1, wc);
           if (!ok) break;
           tc_fence_after();
-          issue_dp(sbase + kKvOffDO + s0 * kTileBytes);
+          issue_dp(t);                           // Y_t = X_{t-1}: free after dK(t-1)
         }
-        for (int m = 0; m < it.nq && ok; ++m, ++qd_iter) {
-          const uint32_t s = qd_iter & 1;
+        for (int m = 0; m < it.nq && ok; ++m, ++t) {
+          const uint32_t s = t & 1;
           const uint32_t qt = sbase + kKvOffQ + s * kTileBytes;
           const uint32_t dot = sbase + kKvOffDO + s * kTileBytes;
+          const uint32_t X = region(t);
           const bool has_next = m + 1 < it.nq;
-          const uint32_t s2 = (qd_iter + 1) & 1, ph2 = ((qd_iter + 1) >> 1) & 1;
-          // dV(m) += P^T(m) dO(m)
+          // dV(t) += P^T(t) dO(t)
           ok = mbar_wait(smem_u32(&bars->p_full), p_cnt & 1, wc);
           ++p_cnt;
           if (ok && m == 0 && item_count > 0)
@@ -285,36 +292,29 @@ attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_q,
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            mma_ts(tmem + 256, tmem + split_a_col(kk), mnmajor_desc(dot, kk), idesc_ts,
+            mma_ts(tmem + 256, X + split_a_col(kk), mnmajor_desc(dot, kk), idesc_ts,
                    (m > 0 || kk > 0) ? 1u : 0u);
-          mma_commit(smem_u32(&bars->dv_done));
-          ++dv_count;
-          // S^T(m+1) once dV(m) has read P^T(m)
-          if (has_next) {
-            ok = mbar_wait(smem_u32(&bars->qd_full[s2]), ph2, wc);
-            if (ok) ok = mbar_wait(smem_u32(&bars->dv_done), (dv_count - 1) & 1, wc);
-            if (!ok) break;
-            tc_fence_after();
-            issue_s(sbase + kKvOffQ + s2 * kTileBytes);
-          }
-          // dK(m) += dS^T(m) Q(m)
+          // dS^T(t) written; dP^T(t) read -> Y_t free for S^T(t+1)
           ok = mbar_wait(smem_u32(&bars->ds_full), ds_cnt & 1, wc);
           ++ds_cnt;
+          if (ok && has_next) ok = mbar_wait(smem_u32(&bars->qd_full[(t + 1) & 1]),
+                                             ((t + 1) >> 1) & 1, wc);
           if (!ok) break;
           tc_fence_after();
+          if (has_next) issue_s(t + 1);
+          // dK(t) += dS^T(t) Q(t)
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            mma_ts(tmem + 384, tmem + 128 + split_a_col(kk), mnmajor_desc(qt, kk), idesc_ts,
+            mma_ts(tmem + 384, X + 32 + split_a_col(kk), mnmajor_desc(qt, kk), idesc_ts,
                    (m > 0 || kk > 0) ? 1u : 0u);
           mma_commit(smem_u32(&bars->dk_done));
           ++dk_count;
           mma_commit(smem_u32(&bars->qd_empty[s]));
-          // dP^T(m+1) once dK(m) has read dS^T(m)
           if (has_next) {
             ok = mbar_wait(smem_u32(&bars->dk_done), (dk_count - 1) & 1, wc);
             if (!ok) break;
             tc_fence_after();
-            issue_dp(sbase + kKvOffDO + s2 * kTileBytes);
+            issue_dp(t + 1);
           }
         }
         if (!ok) break;
@@ -355,33 +355,45 @@ attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_q,
         ++s_cnt;
         if (!ok) break;
         tc_fence_after();
-        // P^T for query rows [c0, c0+64): 2^(s*scale - lse2), masked, fp16
+        // TMEM regions of this tile: S^T in X, dP^T in Y (rotating per tile)
+        const uint32_t X = (tile_count & 1) * 128, Y = 128 - X;
+        // P^T for query rows [c0, c0+64): 2^(s*scale - lse2), masked, fp16.
+        // Row c of the tile is token qs + c/G, so the rows that see key j form
+        // one column range [cmin, cmax); masked and unmasked tiles run separate
+        // code so the mask costs nothing on interior tiles.
+        int cmin = 0, cmax = kTileRows;
+        if (needs_mask) {
+          const int qend_j = a.W > 0 ? min(it.d1, j + a.W) : it.d1;
+          cmin = valid_key ? max(0, (j - qs) * a.G) : kTileRows;
+          cmax = valid_key ? min(kTileRows, (qend_j - qs) * a.G) : 0;
+        }
         uint32_t pk[32];
         {
           uint32_t u0[32], u1[32];
-          tmem_ld32(t_row + c0, u0);
-          tmem_ld32(t_row + c0 + 32, u1);
+          tmem_ld32(t_row + X + c0, u0);
+          tmem_ld32(t_row + X + c0 + 32, u1);
           tc_wait_ld_dep(u0);
           tc_wait_ld_dep(u1);
+          auto p_half = [&](auto masked) {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const int c = c0 + 2 * e;
-            const float s0 = __uint_as_float(e < 16 ? u0[2 * e] : u1[2 * e - 32]);
-            const float s1 = __uint_as_float(e < 16 ? u0[2 * e + 1] : u1[2 * e - 31]);
-            const float2 l2 = *reinterpret_cast<const float2*>(st + c);
-            float p0 = ex2_approx(fmaf(s0, a.scale_log2, -l2.x));
-            float p1 = ex2_approx(fmaf(s1, a.scale_log2, -l2.y));
-            if (needs_mask) {
-              const int t0 = qs + (c >> a.logG), t1 = qs + ((c + 1) >> a.logG);
-              const bool v0 = valid_key && j <= t0 && t0 < it.d1 && (a.W <= 0 || t0 - j < a.W);
-              const bool v1 = valid_key && j <= t1 && t1 < it.d1 && (a.W <= 0 || t1 - j < a.W);
-              p0 = v0 ? p0 : 0.f;
-              p1 = v1 ? p1 : 0.f;
+            for (int e = 0; e < 32; ++e) {
+              const int c = c0 + 2 * e;
+              const float s0 = __uint_as_float(e < 16 ? u0[2 * e] : u1[2 * e - 32]);
+              const float s1 = __uint_as_float(e < 16 ? u0[2 * e + 1] : u1[2 * e - 31]);
+              const float2 l2 = *reinterpret_cast<const float2*>(st + c);
+              float p0 = ex2_approx(fmaf(s0, a.scale_log2, -l2.x));
+              float p1 = ex2_approx(fmaf(s1, a.scale_log2, -l2.y));
+              if (decltype(masked)::value) {
+                p0 = (c >= cmin && c < cmax) ? p0 : 0.f;
+                p1 = (c + 1 >= cmin && c + 1 < cmax) ? p1 : 0.f;
+              }
+              pk[e] = pack_f16x2(p0, p1);
             }
-            pk[e] = pack_f16x2(p0, p1);
-          }
+          };
+          if (needs_mask) p_half(std::true_type{});
+          else p_half(std::false_type{});
         }
-        tmem_st32(t_row + c0, pk);
+        tmem_st32(t_row + X + c0, pk);             // P^T into X columns [c0, c0+32)
         tc_wait_st();
         tc_fence_before();
         __syncwarp();
@@ -392,8 +404,8 @@ attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_q,
         tc_fence_after();
         {
           uint32_t u0[32], u1[32], ds[32];
-          tmem_ld32(t_row + 128 + c0, u0);
-          tmem_ld32(t_row + 128 + c0 + 32, u1);
+          tmem_ld32(t_row + Y + c0, u0);
+          tmem_ld32(t_row + Y + c0 + 32, u1);
           tc_wait_ld_dep(u0);
           tc_wait_ld_dep(u1);
 #pragma unroll
@@ -405,7 +417,7 @@ attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_q,
             const float2 dd = *reinterpret_cast<const float2*>(st + 128 + c);
             ds[e] = pack_f16x2(p.x * (d0 - dd.x), p.y * (d1 - dd.y));
           }
-          tmem_st32(t_row + 128 + c0, ds);
+          tmem_st32(t_row + X + c0 + 32, ds);       // dS^T into X columns [c0+32, c0+64)
         }
         tc_wait_st();
         tc_fence_before();
@@ -715,20 +727,25 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q,
           tmem_ld32(t_row + s_col + c0 + 32, u1);
           tc_wait_ld_dep(u0);
           tc_wait_ld_dep(u1);
+          // masked and unmasked key tiles run separate code
+          auto p_half = [&](auto masked) {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const uint32_t a0 = e < 16 ? u0[2 * e] : u1[2 * e - 32];
-            const uint32_t a1 = e < 16 ? u0[2 * e + 1] : u1[2 * e - 31];
-            float x0, x1;
-            f2_split(ffma2(f2(__uint_as_float(a0), __uint_as_float(a1)), sc2, nl2), x0, x1);
-            float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
-            if (needs_mask) {
-              const int c = c0 + 2 * e;
-              p0 = (valid && c >= c_lo && c <= c_hi) ? p0 : 0.f;
-              p1 = (valid && c + 1 >= c_lo && c + 1 <= c_hi) ? p1 : 0.f;
+            for (int e = 0; e < 32; ++e) {
+              const uint32_t a0 = e < 16 ? u0[2 * e] : u1[2 * e - 32];
+              const uint32_t a1 = e < 16 ? u0[2 * e + 1] : u1[2 * e - 31];
+              float x0, x1;
+              f2_split(ffma2(f2(__uint_as_float(a0), __uint_as_float(a1)), sc2, nl2), x0, x1);
+              float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+              if (decltype(masked)::value) {
+                const int c = c0 + 2 * e;
+                p0 = (valid && c >= c_lo && c <= c_hi) ? p0 : 0.f;
+                p1 = (valid && c + 1 >= c_lo && c + 1 <= c_hi) ? p1 : 0.f;
+              }
+              pk[e] = pack_f16x2(p0, p1);
             }
-            pk[e] = pack_f16x2(p0, p1);
-          }
+          };
+          if (needs_mask) p_half(std::true_type{});
+          else p_half(std::false_type{});
         }
         ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->dp_full), t & 1, wc));
         if (!ok) break;

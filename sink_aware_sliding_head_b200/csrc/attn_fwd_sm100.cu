@@ -32,6 +32,8 @@
 //     sum at 1 (the sink's own weight), so there is no extra pass and a row is
 //     never all -inf. The max is updated lazily: O and l are rescaled only when
 //     the max grows by more than 2^8.
+#include <type_traits>
+
 #include "common.cuh"
 #include "sm100_primitives.cuh"
 
@@ -338,31 +340,36 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                                 (a.W > 0 && ks < it.q0 + 2 * a.R - a.W);
         const int c_lo = needs_mask ? lo_r - ks : 0;
         const int c_hi = needs_mask ? tok - ks : 127;
-        // pass 1: row max over the 128 columns, two 64-column halves
+        // pass 1: row max over the 128 columns, two 64-column halves. Masked
+        // and unmasked key tiles run separate code (the mask is free inside).
         float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+        auto pass1 = [&](auto masked) {
 #pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          uint32_t u0[32], u1[32];
-          tmem_ld32(t_row + s_col + hf * 64, u0);
-          tmem_ld32(t_row + s_col + hf * 64 + 32, u1);
-          tc_wait_ld_dep(u0);
-          tc_wait_ld_dep(u1);
-          if (needs_mask) {
+          for (int hf = 0; hf < 2; ++hf) {
+            uint32_t u0[32], u1[32];
+            tmem_ld32(t_row + s_col + hf * 64, u0);
+            tmem_ld32(t_row + s_col + hf * 64 + 32, u1);
+            tc_wait_ld_dep(u0);
+            tc_wait_ld_dep(u1);
+            if (decltype(masked)::value) {
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              const int c0 = hf * 64 + e, c1 = hf * 64 + 32 + e;
-              if (c0 < c_lo || c0 > c_hi) u0[e] = 0xff800000u;   // -inf
-              if (c1 < c_lo || c1 > c_hi) u1[e] = 0xff800000u;
+              for (int e = 0; e < 32; ++e) {
+                const int ca = hf * 64 + e, cb = hf * 64 + 32 + e;
+                if (ca < c_lo || ca > c_hi) u0[e] = 0xff800000u;   // -inf
+                if (cb < c_lo || cb > c_hi) u1[e] = 0xff800000u;
+              }
+            }
+#pragma unroll
+            for (int e = 0; e < 32; e += 4) {
+              mx0 = fmax3(mx0, __uint_as_float(u0[e]), __uint_as_float(u0[e + 1]));
+              mx1 = fmax3(mx1, __uint_as_float(u0[e + 2]), __uint_as_float(u0[e + 3]));
+              mx2 = fmax3(mx2, __uint_as_float(u1[e]), __uint_as_float(u1[e + 1]));
+              mx3 = fmax3(mx3, __uint_as_float(u1[e + 2]), __uint_as_float(u1[e + 3]));
             }
           }
-#pragma unroll
-          for (int e = 0; e < 32; e += 4) {
-            mx0 = fmax3(mx0, __uint_as_float(u0[e]), __uint_as_float(u0[e + 1]));
-            mx1 = fmax3(mx1, __uint_as_float(u0[e + 2]), __uint_as_float(u0[e + 3]));
-            mx2 = fmax3(mx2, __uint_as_float(u1[e]), __uint_as_float(u1[e + 1]));
-            mx3 = fmax3(mx3, __uint_as_float(u1[e + 2]), __uint_as_float(u1[e + 3]));
-          }
-        }
+        };
+        if (needs_mask) pass1(std::true_type{});
+        else pass1(std::false_type{});
         const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
         const float m_tile = mx * a.scale_log2;
         float alpha = 1.f;
@@ -398,37 +405,41 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         const uint64_t sc2 = f2(a.scale_log2, a.scale_log2);
         const uint64_t nm2 = f2(-mb, -mb);
         uint64_t rs2 = f2(0.f, 0.f);
-        // pass 2: P = 2^(s*scale - m) in bf16 over the first 64 columns of S.
+        // pass 2: P = 2^(s*scale - m) in fp16 over the first 64 columns of S.
         // Half hf re-reads S columns [64hf, 64hf+64) and writes P columns
         // [32hf, 32hf+32), which this thread has already read.
+        auto pass2 = [&](auto masked) {
 #pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          uint32_t u0[32], u1[32], pk[32];
-          tmem_ld32(t_row + s_col + hf * 64, u0);
-          tmem_ld32(t_row + s_col + hf * 64 + 32, u1);
-          tc_wait_ld_dep(u0);
-          tc_wait_ld_dep(u1);
-          if (needs_mask) {
+          for (int hf = 0; hf < 2; ++hf) {
+            uint32_t u0[32], u1[32], pk[32];
+            tmem_ld32(t_row + s_col + hf * 64, u0);
+            tmem_ld32(t_row + s_col + hf * 64 + 32, u1);
+            tc_wait_ld_dep(u0);
+            tc_wait_ld_dep(u1);
+            if (decltype(masked)::value) {
+#pragma unroll
+              for (int e = 0; e < 32; ++e) {
+                const int ca = hf * 64 + e, cb = hf * 64 + 32 + e;
+                if (ca < c_lo || ca > c_hi) u0[e] = 0xff800000u;
+                if (cb < c_lo || cb > c_hi) u1[e] = 0xff800000u;
+              }
+            }
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
-              const int c0 = hf * 64 + e, c1 = hf * 64 + 32 + e;
-              if (c0 < c_lo || c0 > c_hi) u0[e] = 0xff800000u;
-              if (c1 < c_lo || c1 > c_hi) u1[e] = 0xff800000u;
+              const uint32_t a0 = e < 16 ? u0[2 * e] : u1[2 * e - 32];
+              const uint32_t a1 = e < 16 ? u0[2 * e + 1] : u1[2 * e - 31];
+              float x0, x1;
+              f2_split(ffma2(f2(__uint_as_float(a0), __uint_as_float(a1)), sc2, nm2), x0, x1);
+              const float p0 = ex2_approx(x0);
+              const float p1 = ex2_approx(x1);
+              rs2 = fadd2(rs2, f2(p0, p1));
+              pk[e] = pack_f16x2(p0, p1);
             }
+            tmem_st32(t_row + s_col + hf * 32, pk);
           }
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const uint32_t a0 = e < 16 ? u0[2 * e] : u1[2 * e - 32];
-            const uint32_t a1 = e < 16 ? u0[2 * e + 1] : u1[2 * e - 31];
-            float x0, x1;
-            f2_split(ffma2(f2(__uint_as_float(a0), __uint_as_float(a1)), sc2, nm2), x0, x1);
-            const float p0 = ex2_approx(x0);
-            const float p1 = ex2_approx(x1);
-            rs2 = fadd2(rs2, f2(p0, p1));
-            pk[e] = pack_f16x2(p0, p1);
-          }
-          tmem_st32(t_row + s_col + hf * 32, pk);
-        }
+        };
+        if (needs_mask) pass2(std::true_type{});
+        else pass2(std::false_type{});
         float rs_lo, rs_hi;
         f2_split(rs2, rs_lo, rs_hi);
         const float rs = rs_lo + rs_hi;
