@@ -23,8 +23,10 @@
 //     (thread = TMEM lane = query row), warp 8 issues TMA loads, warp 9 issues
 //     tcgen05.mma from one thread and owns the TMEM allocation.
 //   * TMEM (512 columns): S0 [0,128), S1 [128,256), O0 [256,384), O1 [384,512).
-//     P_i (bf16, two per column) overwrites the first 64 columns of S_i and is
-//     the A operand of the PV MMA straight from TMEM. Before the next QK MMA of
+//     P_i (fp16, two per column) overwrites the first 64 columns of S_i and is
+//     the A operand of the PV MMA straight from TMEM. The softmax reads S_i
+//     once into registers and releases P_i in two halves (keys 0-63, then
+//     64-127); the PV MMA of the first half runs while the second is computed. Before the next QK MMA of
 //     tile i overwrites S_i, the issuer waits until the PV MMA of tile i has
 //     completed (a commit barrier), so no ordering between MMAs writing
 //     different accumulators is assumed.
@@ -67,7 +69,7 @@ struct FwdArgs {
 struct __align__(8) Barriers {
   uint64_t q_full, q_empty;
   uint64_t k_full[kStages], k_empty[kStages], v_full[kStages], v_empty[kStages];
-  uint64_t s_full[2], p_full[2], pv_done[2], o_full[2], o_empty[2];
+  uint64_t s_full[2], p_half[2], p_full[2], pv_done[2], o_full[2], o_empty[2];
   uint64_t drain;
 };
 
@@ -132,6 +134,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&bars->s_full[i]), 1);
+      mbar_init(smem_u32(&bars->p_half[i]), 4);
       mbar_init(smem_u32(&bars->p_full[i]), 4);
       mbar_init(smem_u32(&bars->pv_done[i]), 1);
       mbar_init(smem_u32(&bars->o_full[i]), 1);
@@ -253,16 +256,23 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
           ok = mbar_wait(smem_u32(&bars->v_full[s]), ph, wc);
           if (ok && has_next) ok = mbar_wait(smem_u32(&bars->k_full[s2]), ph2, wc);
           // ---- tile 0
-          if (ok) ok = mbar_wait(smem_u32(&bars->p_full[0]), pc0 & 1, wc);
-          ++pc0;
+          // keys 0-63 of P as soon as the softmax has written them, then 64-127
+          if (ok) ok = mbar_wait(smem_u32(&bars->p_half[0]), pc0 & 1, wc);
           if (ok && n == 0 && item_count > 0)
             ok = mbar_wait(smem_u32(&bars->o_empty[0]), (item_count - 1) & 1, wc);
           if (!ok) break;
           tc_fence_after();
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
+          for (int kk = 0; kk < 4; ++kk)
             mma_ts(tmem + 256, tmem + 0 + kk * 8, mnmajor_desc(vt, kk), idesc_pv,
                    (n > 0 || kk > 0) ? 1u : 0u);
+          ok = mbar_wait(smem_u32(&bars->p_full[0]), pc0 & 1, wc);
+          ++pc0;
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 4; kk < 8; ++kk)
+            mma_ts(tmem + 256, tmem + 0 + kk * 8, mnmajor_desc(vt, kk), idesc_pv, 1u);
           mma_commit(smem_u32(&bars->pv_done[0]));
           ++pv0;
           if (!has_next) mma_commit(smem_u32(&bars->o_full[0]));
@@ -276,16 +286,23 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
             mma_commit(smem_u32(&bars->s_full[0]));
           }
           // ---- tile 1
-          ok = mbar_wait(smem_u32(&bars->p_full[1]), pc1 & 1, wc);
-          ++pc1;
+          // keys 0-63 of P as soon as the softmax has written them, then 64-127
+          if (ok) ok = mbar_wait(smem_u32(&bars->p_half[1]), pc1 & 1, wc);
           if (ok && n == 0 && item_count > 0)
             ok = mbar_wait(smem_u32(&bars->o_empty[1]), (item_count - 1) & 1, wc);
           if (!ok) break;
           tc_fence_after();
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
+          for (int kk = 0; kk < 4; ++kk)
             mma_ts(tmem + 384, tmem + 128 + kk * 8, mnmajor_desc(vt, kk), idesc_pv,
                    (n > 0 || kk > 0) ? 1u : 0u);
+          ok = mbar_wait(smem_u32(&bars->p_full[1]), pc1 & 1, wc);
+          ++pc1;
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 4; kk < 8; ++kk)
+            mma_ts(tmem + 384, tmem + 128 + kk * 8, mnmajor_desc(vt, kk), idesc_pv, 1u);
           mma_commit(smem_u32(&bars->pv_done[1]));
           ++pv1;
           if (!has_next) mma_commit(smem_u32(&bars->o_full[1]));
@@ -340,36 +357,39 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                                 (a.W > 0 && ks < it.q0 + 2 * a.R - a.W);
         const int c_lo = needs_mask ? lo_r - ks : 0;
         const int c_hi = needs_mask ? tok - ks : 127;
-        // pass 1: row max over the 128 columns, two 64-column halves. Masked
-        // and unmasked key tiles run separate code (the mask is free inside).
+        // The whole row of S (128 columns) is loaded once. Masked and
+        // unmasked key tiles run separate code; masked entries become -inf
+        // in place, so the exponentials below need no mask.
+        uint32_t u0[32], u1[32], u2[32], u3[32];
+        tmem_ld32(t_row + s_col, u0);
+        tmem_ld32(t_row + s_col + 32, u1);
+        tmem_ld32(t_row + s_col + 64, u2);
+        tmem_ld32(t_row + s_col + 96, u3);
+        tc_wait_ld_dep(u0);
+        tc_wait_ld_dep(u1);
+        tc_wait_ld_dep(u2);
+        tc_wait_ld_dep(u3);
         float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
-        auto pass1 = [&](auto masked) {
-#pragma unroll
-          for (int hf = 0; hf < 2; ++hf) {
-            uint32_t u0[32], u1[32];
-            tmem_ld32(t_row + s_col + hf * 64, u0);
-            tmem_ld32(t_row + s_col + hf * 64 + 32, u1);
-            tc_wait_ld_dep(u0);
-            tc_wait_ld_dep(u1);
+        auto row_max = [&](auto masked) {
+          auto one = [&](uint32_t (&u)[32], int c0, float& mxa, float& mxb) {
             if (decltype(masked)::value) {
 #pragma unroll
-              for (int e = 0; e < 32; ++e) {
-                const int ca = hf * 64 + e, cb = hf * 64 + 32 + e;
-                if (ca < c_lo || ca > c_hi) u0[e] = 0xff800000u;   // -inf
-                if (cb < c_lo || cb > c_hi) u1[e] = 0xff800000u;
-              }
+              for (int e = 0; e < 32; ++e)
+                if (c0 + e < c_lo || c0 + e > c_hi) u[e] = 0xff800000u;   // -inf
             }
 #pragma unroll
             for (int e = 0; e < 32; e += 4) {
-              mx0 = fmax3(mx0, __uint_as_float(u0[e]), __uint_as_float(u0[e + 1]));
-              mx1 = fmax3(mx1, __uint_as_float(u0[e + 2]), __uint_as_float(u0[e + 3]));
-              mx2 = fmax3(mx2, __uint_as_float(u1[e]), __uint_as_float(u1[e + 1]));
-              mx3 = fmax3(mx3, __uint_as_float(u1[e + 2]), __uint_as_float(u1[e + 3]));
+              mxa = fmax3(mxa, __uint_as_float(u[e]), __uint_as_float(u[e + 1]));
+              mxb = fmax3(mxb, __uint_as_float(u[e + 2]), __uint_as_float(u[e + 3]));
             }
-          }
+          };
+          one(u0, 0, mx0, mx1);
+          one(u1, 32, mx2, mx3);
+          one(u2, 64, mx0, mx1);
+          one(u3, 96, mx2, mx3);
         };
-        if (needs_mask) pass1(std::true_type{});
-        else pass1(std::false_type{});
+        if (needs_mask) row_max(std::true_type{});
+        else row_max(std::false_type{});
         const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
         const float m_tile = mx * a.scale_log2;
         float alpha = 1.f;
@@ -382,11 +402,34 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
           rescale_o = true;
         }
         l *= alpha;
+        const float mb = (m == -INFINITY) ? 0.f : m;
+        const uint64_t sc2 = f2(a.scale_log2, a.scale_log2);
+        const uint64_t nm2 = f2(-mb, -mb);
+        uint64_t rs2 = f2(0.f, 0.f);
+        // P = 2^(s*scale - m) in fp16, two keys per TMEM column, over the
+        // first 64 columns of S (already read). Keys 0-63 are handed to the
+        // PV MMA before keys 64-127 are computed.
+        auto exp_chunk = [&](const uint32_t (&u)[32], int col) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            float x0, x1;
+            f2_split(ffma2(f2(__uint_as_float(u[2 * e]), __uint_as_float(u[2 * e + 1])), sc2, nm2),
+                     x0, x1);
+            const float p0 = ex2_approx(x0);
+            const float p1 = ex2_approx(x1);
+            rs2 = fadd2(rs2, f2(p0, p1));
+            pk[e] = pack_f16x2(p0, p1);
+          }
+          tmem_st16(t_row + s_col + col, pk);
+        };
+        exp_chunk(u0, 0);
         if (__any_sync(0xffffffffu, rescale_o)) {
           // PV of the previous tile has completed (the QK that produced this
-          // S was issued after it completed), so O is stable here.
+          // S was issued after it completed), so O is stable here. Done once
+          // the first quarter of S is consumed, to stay within registers.
           const uint64_t a2 = f2(alpha, alpha);
-#pragma unroll
+#pragma unroll 1
           for (int c = 0; c < 4; ++c) {
             uint32_t u[32];
             tmem_ld32(t_row + o_col + c * 32, u);
@@ -401,45 +444,13 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
             tmem_st32(t_row + o_col + c * 32, u);
           }
         }
-        const float mb = (m == -INFINITY) ? 0.f : m;
-        const uint64_t sc2 = f2(a.scale_log2, a.scale_log2);
-        const uint64_t nm2 = f2(-mb, -mb);
-        uint64_t rs2 = f2(0.f, 0.f);
-        // pass 2: P = 2^(s*scale - m) in fp16 over the first 64 columns of S.
-        // Half hf re-reads S columns [64hf, 64hf+64) and writes P columns
-        // [32hf, 32hf+32), which this thread has already read.
-        auto pass2 = [&](auto masked) {
-#pragma unroll
-          for (int hf = 0; hf < 2; ++hf) {
-            uint32_t u0[32], u1[32], pk[32];
-            tmem_ld32(t_row + s_col + hf * 64, u0);
-            tmem_ld32(t_row + s_col + hf * 64 + 32, u1);
-            tc_wait_ld_dep(u0);
-            tc_wait_ld_dep(u1);
-            if (decltype(masked)::value) {
-#pragma unroll
-              for (int e = 0; e < 32; ++e) {
-                const int ca = hf * 64 + e, cb = hf * 64 + 32 + e;
-                if (ca < c_lo || ca > c_hi) u0[e] = 0xff800000u;
-                if (cb < c_lo || cb > c_hi) u1[e] = 0xff800000u;
-              }
-            }
-#pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              const uint32_t a0 = e < 16 ? u0[2 * e] : u1[2 * e - 32];
-              const uint32_t a1 = e < 16 ? u0[2 * e + 1] : u1[2 * e - 31];
-              float x0, x1;
-              f2_split(ffma2(f2(__uint_as_float(a0), __uint_as_float(a1)), sc2, nm2), x0, x1);
-              const float p0 = ex2_approx(x0);
-              const float p1 = ex2_approx(x1);
-              rs2 = fadd2(rs2, f2(p0, p1));
-              pk[e] = pack_f16x2(p0, p1);
-            }
-            tmem_st32(t_row + s_col + hf * 32, pk);
-          }
-        };
-        if (needs_mask) pass2(std::true_type{});
-        else pass2(std::false_type{});
+        exp_chunk(u1, 16);
+        tc_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&bars->p_half[i]));
+        exp_chunk(u2, 32);
+        exp_chunk(u3, 48);
         float rs_lo, rs_hi;
         f2_split(rs2, rs_lo, rs_hi);
         const float rs = rs_lo + rs_hi;
