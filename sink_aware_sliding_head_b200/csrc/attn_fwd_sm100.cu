@@ -20,16 +20,18 @@
 //     built on the device; only key tiles inside the window and the document
 //     are visited, and only edge tiles are masked.
 //   * Warp roles: warps 0-3 run the softmax of tile 0, warps 4-7 of tile 1
-//     (thread = TMEM lane = query row), warp 8 issues TMA loads, warp 9 issues
-//     tcgen05.mma from one thread and owns the TMEM allocation.
+//     (thread = TMEM lane = query row), warp 8 issues TMA loads, warp 9 owns
+//     the TMEM allocation and issues tcgen05.mma: the warp runs its loop
+//     converged and one elected lane issues, so descriptors stay warp-uniform
+//     (issued from a lane-0 branch instead, each MMA cost ~75 issue cycles).
 //   * TMEM (512 columns): S0 [0,128), S1 [128,256), O0 [256,384), O1 [384,512).
 //     P_i (fp16, two per column) overwrites the first 64 columns of S_i and is
 //     the A operand of the PV MMA straight from TMEM. The softmax reads S_i
 //     once into registers and releases P_i in two halves (keys 0-63, then
-//     64-127); the PV MMA of the first half runs while the second is computed. Before the next QK MMA of
-//     tile i overwrites S_i, the issuer waits until the PV MMA of tile i has
-//     completed (a commit barrier), so no ordering between MMAs writing
-//     different accumulators is assumed.
+//     64-127); the PV MMA of the first half runs while the second is
+//     computed. Before the next QK MMA of tile i overwrites S_i, the issuer
+//     waits until the PV MMA of tile i has completed (a commit barrier), so no
+//     ordering between MMAs writing different accumulators is assumed.
 //   * Sink folding: the running max starts at the sink logit and the running
 //     sum at 1 (the sink's own weight), so there is no extra pass and a row is
 //     never all -inf. The max is updated lazily: O and l are rescaled only when
@@ -43,7 +45,10 @@ namespace flint {
 
 namespace {
 
-constexpr int kStages = 2;
+// K and V tiles stream through one ring of kSlots 32 KB slots in the order
+// K(0), V(0), K(1), V(1), ...; five slots let the producer run 2.5 key tiles
+// ahead of the MMAs, which covers the load latency of a tile.
+constexpr int kSlots = 5;
 constexpr int kThreads = 320;
 constexpr int kWarpTma = 8;
 constexpr int kWarpMma = 9;
@@ -68,19 +73,19 @@ struct FwdArgs {
 
 struct __align__(8) Barriers {
   uint64_t q_full, q_empty;
-  uint64_t k_full[kStages], k_empty[kStages], v_full[kStages], v_empty[kStages];
+  uint64_t kv_full[kSlots], kv_empty[kSlots];
   uint64_t s_full[2], p_half[2], p_full[2], pv_done[2], o_full[2], o_empty[2];
   uint64_t drain;
 };
 
 // Dynamic shared memory: [Q0 | Q1 | K stages | V stages | barriers | tmem addr | abort flag]
 constexpr uint32_t kOffQ = 0;
-constexpr uint32_t kOffK = 2 * kTileBytes;
-constexpr uint32_t kOffV = kOffK + kStages * kTileBytes;
-constexpr uint32_t kOffBar = kOffV + kStages * kTileBytes;
+constexpr uint32_t kOffKV = 2 * kTileBytes;
+constexpr uint32_t kOffBar = kOffKV + kSlots * kTileBytes;
 constexpr uint32_t kOffTmem = kOffBar + sizeof(Barriers);
 constexpr uint32_t kOffAbort = kOffTmem + 16;
 constexpr uint32_t kSmemBytes = kOffAbort + 16 + 1024;   // + alignment slack
+static_assert(kSmemBytes <= 227 * 1024, "exceeds the shared memory of one CTA");
 
 struct Item {
   int q0, d0, d1, g, kend, kbeg, ntiles;
@@ -126,11 +131,9 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
     *abort_flag = 0;
     mbar_init(smem_u32(&bars->q_full), 1);
     mbar_init(smem_u32(&bars->q_empty), 1);
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(smem_u32(&bars->k_full[s]), 1);
-      mbar_init(smem_u32(&bars->k_empty[s]), 1);
-      mbar_init(smem_u32(&bars->v_full[s]), 1);
-      mbar_init(smem_u32(&bars->v_empty[s]), 1);
+    for (int s = 0; s < kSlots; ++s) {
+      mbar_init(smem_u32(&bars->kv_full[s]), 1);
+      mbar_init(smem_u32(&bars->kv_empty[s]), 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&bars->s_full[i]), 1);
@@ -161,7 +164,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
   if (warp == kWarpTma) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      uint32_t kv_iter = 0, item_count = 0, q_arm = 0, k_arm[kStages] = {}, v_arm[kStages] = {};
+      uint32_t kv_load = 0, item_count = 0, q_arm = 0, arm[kSlots] = {};
       bool ok = true;
       for (int idx = blockIdx.x; idx < n_items && ok; idx += gridDim.x) {
         const Item it = decode(a, idx);
@@ -174,25 +177,17 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
           for (int c = 0; c < 2; ++c)
             tma_load_3d(sbase + kOffQ + i * kTileBytes + c * kChunkBytes, &tm_q, qf, c * 64,
                         it.g * a.G, it.q0 + i * a.R);
-        for (int n = 0; n < it.ntiles && ok; ++n, ++kv_iter) {
-          const int ks = it.kend - kTileKeys * (n + 1);
-          const uint32_t s = kv_iter % kStages, ph = (kv_iter / kStages) & 1;
-          if (kv_iter >= kStages) ok = mbar_wait(smem_u32(&bars->k_empty[s]), ph ^ 1, wc);
+        for (int j = 0; j < 2 * it.ntiles && ok; ++j, ++kv_load) {
+          const int ks = it.kend - kTileKeys * ((j >> 1) + 1);
+          const uint32_t s = kv_load % kSlots, ph = (kv_load / kSlots) & 1;
+          if (kv_load >= kSlots) ok = mbar_wait(smem_u32(&bars->kv_empty[s]), ph ^ 1, wc);
           if (!ok) break;
-          const uint32_t kf = smem_u32(&bars->k_full[s]);
-          mbar_arrive_expect_tx(kf, kTileBytes);
-          ++k_arm[s];
+          const uint32_t f = smem_u32(&bars->kv_full[s]);
+          mbar_arrive_expect_tx(f, kTileBytes);
+          ++arm[s];
+          const CUtensorMap* m = (j & 1) ? &tm_v : &tm_k;
           for (int c = 0; c < 2; ++c)
-            tma_load_3d(sbase + kOffK + s * kTileBytes + c * kChunkBytes, &tm_k, kf, c * 64, it.g,
-                        ks);
-          if (kv_iter >= kStages) ok = mbar_wait(smem_u32(&bars->v_empty[s]), ph ^ 1, wc);
-          if (!ok) break;
-          const uint32_t vf = smem_u32(&bars->v_full[s]);
-          mbar_arrive_expect_tx(vf, kTileBytes);
-          ++v_arm[s];
-          for (int c = 0; c < 2; ++c)
-            tma_load_3d(sbase + kOffV + s * kTileBytes + c * kChunkBytes, &tm_v, vf, c * 64, it.g,
-                        ks);
+            tma_load_3d(sbase + kOffKV + s * kTileBytes + c * kChunkBytes, m, f, c * 64, it.g, ks);
         }
         ++item_count;
       }
@@ -201,10 +196,8 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       volatile int no_abort = 0;
       const WaitCtx drain{&no_abort, a.status, kStatusTimeoutFwd};
       if (q_arm) mbar_wait(smem_u32(&bars->q_full), (q_arm - 1) & 1, drain);
-      for (int s = 0; s < kStages; ++s) {
-        if (k_arm[s]) mbar_wait(smem_u32(&bars->k_full[s]), (k_arm[s] - 1) & 1, drain);
-        if (v_arm[s]) mbar_wait(smem_u32(&bars->v_full[s]), (v_arm[s] - 1) & 1, drain);
-      }
+      for (int s = 0; s < kSlots; ++s)
+        if (arm[s]) mbar_wait(smem_u32(&bars->kv_full[s]), (arm[s] - 1) & 1, drain);
     }
   } else if (warp == kWarpMma) {
     // ------------------------------------------------------------ MMA issuer
@@ -212,122 +205,126 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
     // runs half a period behind tile 0, so each tile's softmax overlaps the
     // other tile's MMAs. QK_i(n+1) overwrites S_i, which holds P_i(n), so it
     // is issued only after PV_i(n) has completed.
-    if (lane == 0) {
+    {
+      const uint32_t leader = elect_one();   // the one lane that issues
       const uint32_t idesc_qk = make_idesc_f16(128, 128, 0, 0);
       const uint32_t idesc_pv = make_idesc_f16(128, 128, 0, 1);
-      uint32_t kv_iter = 0, item_count = 0;
+      uint32_t kv_load = 0, item_count = 0;   // K/V ring loads consumed before this item
       uint32_t pv0 = 0, pv1 = 0, pc0 = 0, pc1 = 0;   // PV commits / P arrivals seen, per tile
       bool ok = true;
       const uint32_t q0t = sbase + kOffQ, q1t = sbase + kOffQ + kTileBytes;
       for (int idx = blockIdx.x; idx < n_items && ok; idx += gridDim.x) {
         const Item it = decode(a, idx);
-        ok = mbar_wait(smem_u32(&bars->q_full), item_count & 1, wc);
+        ok = mbar_wait_warp(smem_u32(&bars->q_full), item_count & 1, wc);
         if (!ok) break;
         tc_fence_after();
         {  // QK of the first key tile for both query tiles
-          const uint32_t s = kv_iter % kStages, ph = (kv_iter / kStages) & 1;
-          ok = mbar_wait(smem_u32(&bars->k_full[s]), ph, wc);
+          const uint32_t s = kv_load % kSlots, ph = (kv_load / kSlots) & 1;   // K(0)
+          ok = mbar_wait_warp(smem_u32(&bars->kv_full[s]), ph, wc);
           if (!ok) break;
-          const uint32_t kt = sbase + kOffK + s * kTileBytes;
-          if (pv0 > 0) ok = mbar_wait(smem_u32(&bars->pv_done[0]), (pv0 - 1) & 1, wc);
-          if (!ok) break;
-          tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_ss(tmem + 0, kmajor_desc(q0t, kk), kmajor_desc(kt, kk), idesc_qk, kk > 0);
-          mma_commit(smem_u32(&bars->s_full[0]));
-          if (pv1 > 0) ok = mbar_wait(smem_u32(&bars->pv_done[1]), (pv1 - 1) & 1, wc);
+          const uint32_t kt = sbase + kOffKV + s * kTileBytes;
+          if (pv0 > 0) ok = mbar_wait_warp(smem_u32(&bars->pv_done[0]), (pv0 - 1) & 1, wc);
           if (!ok) break;
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            mma_ss(tmem + 128, kmajor_desc(q1t, kk), kmajor_desc(kt, kk), idesc_qk, kk > 0);
-          mma_commit(smem_u32(&bars->s_full[1]));
-          mma_commit(smem_u32(&bars->k_empty[s]));
-          if (it.ntiles == 1) mma_commit(smem_u32(&bars->q_empty));
+            mma_ss_w(tmem + 0, kmajor_desc(q0t, kk), kmajor_desc(kt, kk), idesc_qk, kk > 0, leader);
+          mma_commit_w(smem_u32(&bars->s_full[0]), leader);
+          if (pv1 > 0) ok = mbar_wait_warp(smem_u32(&bars->pv_done[1]), (pv1 - 1) & 1, wc);
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ss_w(tmem + 128, kmajor_desc(q1t, kk), kmajor_desc(kt, kk),
+                     idesc_qk, kk > 0, leader);
+          mma_commit_w(smem_u32(&bars->s_full[1]), leader);
+          mma_commit_w(smem_u32(&bars->kv_empty[s]), leader);
+          if (it.ntiles == 1) mma_commit_w(smem_u32(&bars->q_empty), leader);
         }
         for (int n = 0; n < it.ntiles; ++n) {
-          const uint32_t cur = kv_iter + n, nxt = cur + 1;
-          const uint32_t s = cur % kStages, ph = (cur / kStages) & 1;
-          const uint32_t s2 = nxt % kStages, ph2 = (nxt / kStages) & 1;
+          const uint32_t lv = kv_load + 2 * n + 1, lk = lv + 1;       // V(n), K(n+1)
+          const uint32_t s = lv % kSlots, ph = (lv / kSlots) & 1;
+          const uint32_t s2 = lk % kSlots, ph2 = (lk / kSlots) & 1;
           const bool has_next = n + 1 < it.ntiles;
-          const uint32_t vt = sbase + kOffV + s * kTileBytes;
-          const uint32_t kt2 = sbase + kOffK + s2 * kTileBytes;
-          ok = mbar_wait(smem_u32(&bars->v_full[s]), ph, wc);
-          if (ok && has_next) ok = mbar_wait(smem_u32(&bars->k_full[s2]), ph2, wc);
+          const uint32_t vt = sbase + kOffKV + s * kTileBytes;
+          const uint32_t kt2 = sbase + kOffKV + s2 * kTileBytes;
+          ok = mbar_wait_warp(smem_u32(&bars->kv_full[s]), ph, wc);
           // ---- tile 0
           // keys 0-63 of P as soon as the softmax has written them, then 64-127
-          if (ok) ok = mbar_wait(smem_u32(&bars->p_half[0]), pc0 & 1, wc);
+          if (ok) ok = mbar_wait_warp(smem_u32(&bars->p_half[0]), pc0 & 1, wc);
           if (ok && n == 0 && item_count > 0)
-            ok = mbar_wait(smem_u32(&bars->o_empty[0]), (item_count - 1) & 1, wc);
+            ok = mbar_wait_warp(smem_u32(&bars->o_empty[0]), (item_count - 1) & 1, wc);
           if (!ok) break;
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            mma_ts(tmem + 256, tmem + 0 + kk * 8, mnmajor_desc(vt, kk), idesc_pv,
-                   (n > 0 || kk > 0) ? 1u : 0u);
-          ok = mbar_wait(smem_u32(&bars->p_full[0]), pc0 & 1, wc);
+            mma_ts_w(tmem + 256, tmem + 0 + kk * 8, mnmajor_desc(vt, kk), idesc_pv,
+                   (n > 0 || kk > 0) ? 1u : 0u, leader);
+          ok = mbar_wait_warp(smem_u32(&bars->p_full[0]), pc0 & 1, wc);
           ++pc0;
           if (!ok) break;
           tc_fence_after();
 #pragma unroll
           for (int kk = 4; kk < 8; ++kk)
-            mma_ts(tmem + 256, tmem + 0 + kk * 8, mnmajor_desc(vt, kk), idesc_pv, 1u);
-          mma_commit(smem_u32(&bars->pv_done[0]));
+            mma_ts_w(tmem + 256, tmem + 0 + kk * 8, mnmajor_desc(vt, kk), idesc_pv, 1u, leader);
+          mma_commit_w(smem_u32(&bars->pv_done[0]), leader);
           ++pv0;
-          if (!has_next) mma_commit(smem_u32(&bars->o_full[0]));
+          if (!has_next) mma_commit_w(smem_u32(&bars->o_full[0]), leader);
           if (has_next) {
-            ok = mbar_wait(smem_u32(&bars->pv_done[0]), (pv0 - 1) & 1, wc);
+            ok = mbar_wait_warp(smem_u32(&bars->kv_full[s2]), ph2, wc);
+            if (ok) ok = mbar_wait_warp(smem_u32(&bars->pv_done[0]), (pv0 - 1) & 1, wc);
             if (!ok) break;
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
-              mma_ss(tmem + 0, kmajor_desc(q0t, kk), kmajor_desc(kt2, kk), idesc_qk, kk > 0);
-            mma_commit(smem_u32(&bars->s_full[0]));
+              mma_ss_w(tmem + 0, kmajor_desc(q0t, kk), kmajor_desc(kt2, kk),
+                       idesc_qk, kk > 0, leader);
+            mma_commit_w(smem_u32(&bars->s_full[0]), leader);
           }
           // ---- tile 1
           // keys 0-63 of P as soon as the softmax has written them, then 64-127
-          if (ok) ok = mbar_wait(smem_u32(&bars->p_half[1]), pc1 & 1, wc);
+          if (ok) ok = mbar_wait_warp(smem_u32(&bars->p_half[1]), pc1 & 1, wc);
           if (ok && n == 0 && item_count > 0)
-            ok = mbar_wait(smem_u32(&bars->o_empty[1]), (item_count - 1) & 1, wc);
+            ok = mbar_wait_warp(smem_u32(&bars->o_empty[1]), (item_count - 1) & 1, wc);
           if (!ok) break;
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            mma_ts(tmem + 384, tmem + 128 + kk * 8, mnmajor_desc(vt, kk), idesc_pv,
-                   (n > 0 || kk > 0) ? 1u : 0u);
-          ok = mbar_wait(smem_u32(&bars->p_full[1]), pc1 & 1, wc);
+            mma_ts_w(tmem + 384, tmem + 128 + kk * 8, mnmajor_desc(vt, kk), idesc_pv,
+                   (n > 0 || kk > 0) ? 1u : 0u, leader);
+          ok = mbar_wait_warp(smem_u32(&bars->p_full[1]), pc1 & 1, wc);
           ++pc1;
           if (!ok) break;
           tc_fence_after();
 #pragma unroll
           for (int kk = 4; kk < 8; ++kk)
-            mma_ts(tmem + 384, tmem + 128 + kk * 8, mnmajor_desc(vt, kk), idesc_pv, 1u);
-          mma_commit(smem_u32(&bars->pv_done[1]));
+            mma_ts_w(tmem + 384, tmem + 128 + kk * 8, mnmajor_desc(vt, kk), idesc_pv, 1u, leader);
+          mma_commit_w(smem_u32(&bars->pv_done[1]), leader);
           ++pv1;
-          if (!has_next) mma_commit(smem_u32(&bars->o_full[1]));
-          mma_commit(smem_u32(&bars->v_empty[s]));
+          if (!has_next) mma_commit_w(smem_u32(&bars->o_full[1]), leader);
+          mma_commit_w(smem_u32(&bars->kv_empty[s]), leader);
           if (has_next) {
-            ok = mbar_wait(smem_u32(&bars->pv_done[1]), (pv1 - 1) & 1, wc);
+            ok = mbar_wait_warp(smem_u32(&bars->pv_done[1]), (pv1 - 1) & 1, wc);
             if (!ok) break;
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
-              mma_ss(tmem + 128, kmajor_desc(q1t, kk), kmajor_desc(kt2, kk), idesc_qk, kk > 0);
-            mma_commit(smem_u32(&bars->s_full[1]));
-            mma_commit(smem_u32(&bars->k_empty[s2]));
-            if (n + 2 == it.ntiles) mma_commit(smem_u32(&bars->q_empty));
+              mma_ss_w(tmem + 128, kmajor_desc(q1t, kk), kmajor_desc(kt2, kk),
+                       idesc_qk, kk > 0, leader);
+            mma_commit_w(smem_u32(&bars->s_full[1]), leader);
+            mma_commit_w(smem_u32(&bars->kv_empty[s2]), leader);
+            if (n + 2 == it.ntiles) mma_commit_w(smem_u32(&bars->q_empty), leader);
           }
         }
         if (!ok) break;
-        kv_iter += it.ntiles;
+        kv_load += 2 * it.ntiles;
         ++item_count;
       }
       // Every MMA this thread issued has finished before TMEM is released.
-      mma_commit(smem_u32(&bars->drain));
+      mma_commit_w(smem_u32(&bars->drain), leader);
       volatile int no_abort = 0;
       const WaitCtx drain{&no_abort, a.status, kStatusTimeoutFwd};
-      mbar_wait(smem_u32(&bars->drain), 0, drain);
+      mbar_wait_warp(smem_u32(&bars->drain), 0, drain);
     }
   } else {
     // ------------------------------------------------------------ softmax + epilogue

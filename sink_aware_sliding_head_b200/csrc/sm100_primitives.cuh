@@ -75,6 +75,11 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const W
   }
 }
 
+// The same wait taken by a whole warp; every lane gets the same answer.
+__device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, const WaitCtx& w) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity, w));
+}
+
 // ---------------------------------------------------------------- dynamic work items
 // A persistent CTA takes its next work item from a global counter (one
 // atomicAdd by the TMA thread) and hands the index to its other roles through
@@ -105,7 +110,7 @@ __device__ __forceinline__ bool ring_push(ItemRing* r, uint32_t k, int idx, cons
 // Consuming warp (all lanes): read the k-th item index; lane 0 frees the slot.
 __device__ __forceinline__ bool ring_pop(ItemRing* r, uint32_t k, int* idx, const WaitCtx& w) {
   const uint32_t s = k % kItemSlots;
-  const bool ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&r->full[s]), (k / kItemSlots) & 1, w));
+  const bool ok = mbar_wait_warp(smem_u32(&r->full[s]), (k / kItemSlots) & 1, w);
   if (!ok) return false;
   *idx = *reinterpret_cast<volatile int*>(&r->idx[s]);
   __syncwarp();
@@ -192,6 +197,50 @@ __host__ __device__ constexpr uint32_t make_idesc_f16(int M, int N, int a_mn, in
   return (1u << 4)                      // D format F32; A, B format F16 (0)
          | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16) |
          ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// One lane of a fully active warp, the same lane on every call (elect.sync
+// picks the lowest active lane). The issuing warp runs its loop converged and
+// predicates only the issue on this flag, so descriptors and TMEM addresses stay
+// warp-uniform values.
+__device__ __forceinline__ uint32_t elect_one() {
+  uint32_t e;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "elect.sync _|p, 0xffffffff;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(e));
+  return e;
+}
+// Warp-converged forms of the three calls below: only the lane with leader != 0
+// issues.
+__device__ __forceinline__ void mma_ss_w(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                         uint32_t idesc, uint32_t accumulate, uint32_t leader) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "setp.ne.b32 e, %5, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(leader)
+      : "memory");
+}
+__device__ __forceinline__ void mma_ts_w(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
+                                         uint32_t idesc, uint32_t accumulate, uint32_t leader) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "setp.ne.b32 e, %5, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(leader)
+      : "memory");
+}
+__device__ __forceinline__ void mma_commit_w(uint32_t bar, uint32_t leader) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t"
+      "setp.ne.b32 e, %1, 0;\n\t"
+      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}\n" ::"r"(
+          bar), "r"(leader)
+      : "memory");
 }
 
 // D[tmem] (+)= A[smem] * B[smem]^T   (one K=16 step)
