@@ -158,7 +158,9 @@ flint_status_t flint_attn_bwd_preprocess_static(const flint_attn_params_t* param
 
 /* Synchronises `stream`, reads and clears the device status word in
  * `workspace` (written by bounded device waits), and returns FLINT_OK or
- * FLINT_ERR_TIMEOUT (FLINT_ERR_CUDA if the stream itself reports an error). */
+ * FLINT_ERR_TIMEOUT. It returns FLINT_ERR_CUDA if the stream itself reports an
+ * error, or if a backward kernel found its dynamic shared memory not 1024-byte
+ * aligned and did no work (its tiles need that alignment; not expected). */
 flint_status_t flint_attn_check_status(void* workspace, void* stream);
 
 /* ---- Measurement aids (not needed to compute anything) --------------------

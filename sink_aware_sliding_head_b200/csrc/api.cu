@@ -319,7 +319,7 @@ extern "C" flint_status_t flint_attn_check_status(void* workspace, void* stream)
     const int zero = 0;
     if (cudaMemcpy(workspace, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
       return FLINT_ERR_CUDA;
-    return FLINT_ERR_TIMEOUT;
+    return (host & flint::kStatusSmemAlign) ? FLINT_ERR_CUDA : FLINT_ERR_TIMEOUT;
   }
   return FLINT_OK;
 }

@@ -18,7 +18,8 @@
 // Two persistent kernels share one warp layout: warps 0-7 do the elementwise
 // math as two warpgroups that split the 128 columns of each tile (there is no
 // row reduction in the backward, so the halves are independent; thread = TMEM
-// lane), warp 8 issues TMA, warp 9 issues MMAs and owns TMEM. Each warpgroup
+// lane), warp 8 issues TMA, warp 9 issues MMAs (converged, one elected lane
+// issues) and owns TMEM. Each warpgroup
 // writes its fp16 P/dS half into the first 32 of the 64 TMEM columns it has
 // just read itself (columns [64c, 64c+32) for warpgroup c), so the TMEM A
 // operand of the following MMA skips from column 32 to 64 halfway through K.
@@ -89,22 +90,27 @@ __device__ __forceinline__ float2 unpack_f16x2(uint32_t u) {
 // ============================================================================
 // dK / dV : key-major
 // ============================================================================
+constexpr int kQStages = 3;   // Q tiles in flight (its buffer is released last, by dK)
 struct __align__(8) KvBars {
   uint64_t kv_full, kv_empty;
-  uint64_t qd_full[2], qd_empty[2];
+  uint64_t q_full[kQStages], q_empty[kQStages], do_full[2], do_empty[2];
   uint64_t s_full, dp_full, p_full, ds_full, dv_done, dk_done, acc_full, acc_empty;
   uint64_t drain;
   ItemRing ring;
 };
 constexpr uint32_t kKvOffK = 0;
 constexpr uint32_t kKvOffV = kTileBytes;
-constexpr uint32_t kKvOffQ = 2 * kTileBytes;                 // 2 stages
-constexpr uint32_t kKvOffDO = kKvOffQ + 2 * kTileBytes;      // 2 stages
-constexpr uint32_t kKvOffStats = kKvOffDO + 2 * kTileBytes;  // [2][2][128] fp32
+constexpr uint32_t kKvOffQ = 2 * kTileBytes;                        // kQStages stages
+constexpr uint32_t kKvOffDO = kKvOffQ + kQStages * kTileBytes;      // 2 stages
+constexpr uint32_t kKvOffStats = kKvOffDO + 2 * kTileBytes;         // [2][2][128] fp32
 constexpr uint32_t kKvOffBar = kKvOffStats + 2 * 2 * 128 * 4;
 constexpr uint32_t kKvOffTmem = kKvOffBar + sizeof(KvBars);
 constexpr uint32_t kKvOffAbort = kKvOffTmem + 16;
-constexpr uint32_t kKvSmem = kKvOffAbort + 16 + 1024;
+// No alignment slack: the kernel checks that the dynamic shared memory starts
+// on a 1024-byte boundary (the 128-byte swizzle needs it) and reports
+// kStatusSmemAlign otherwise.
+constexpr uint32_t kKvSmem = kKvOffAbort + 16;
+static_assert(kKvSmem <= 227 * 1024, "exceeds the shared memory of one CTA");
 
 struct KvItem {
   int k0, d0, d1, g, qend, nq;
@@ -123,9 +129,12 @@ attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v,
                     const __grid_constant__ CUtensorMap tm_do, const BwdArgs a) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  if (smem_u32(smem_raw) & 1023) {
+    if (threadIdx.x == 0) atomicOr(a.status, kStatusSmemAlign);
+    return;
+  }
+  uint8_t* smem = smem_raw;
   const uint32_t sbase = smem_u32(smem);
   KvBars* bars = reinterpret_cast<KvBars*>(smem + kKvOffBar);
   float* stats = reinterpret_cast<float*>(smem + kKvOffStats);   // [buf][lse2|D][128]
@@ -138,9 +147,13 @@ attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_q,
     *abort_flag = 0;
     mbar_init(smem_u32(&bars->kv_full), 1);
     mbar_init(smem_u32(&bars->kv_empty), 1);
+    for (int s = 0; s < kQStages; ++s) {
+      mbar_init(smem_u32(&bars->q_full[s]), 1);
+      mbar_init(smem_u32(&bars->q_empty[s]), 1);
+    }
     for (int s = 0; s < 2; ++s) {
-      mbar_init(smem_u32(&bars->qd_full[s]), 2);   // TMA bytes + per-row statistics
-      mbar_init(smem_u32(&bars->qd_empty[s]), 1);
+      mbar_init(smem_u32(&bars->do_full[s]), 2);   // TMA bytes + per-row statistics
+      mbar_init(smem_u32(&bars->do_empty[s]), 1);
     }
     mbar_init(smem_u32(&bars->s_full), 1);
     mbar_init(smem_u32(&bars->dp_full), 1);
@@ -166,9 +179,9 @@ attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_q,
 
   if (warp == kWarpTma) {
     // Lane 0 takes items from the global counter and issues TMA; the whole warp
-    // stages each query tile's per-row
-    // log2-LSE and D into shared memory and completes qd_full's second arrival.
-    uint32_t item_count = 0, qd_iter = 0, kv_arm = 0, qd_arm[2] = {0, 0};
+    // stages each query tile's per-row log2-LSE and D into shared memory and
+    // completes do_full's second arrival.
+    uint32_t item_count = 0, qd_iter = 0, kv_arm = 0, q_arm[kQStages] = {}, do_arm[2] = {};
     bool ok = true;
     while (ok) {
       int idx = -1;
@@ -196,32 +209,48 @@ attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_q,
       ok = __shfl_sync(0xffffffffu, ok, 0);
       for (int m = 0; m < it.nq && ok; ++m, ++qd_iter) {
         const int qs = it.k0 + m * a.R;
+        const uint32_t sq = qd_iter % kQStages, phq = (qd_iter / kQStages) & 1;
         const uint32_t s = qd_iter & 1, ph = (qd_iter >> 1) & 1;
-        if (lane == 0 && qd_iter >= 2) ok = mbar_wait(smem_u32(&bars->qd_empty[s]), ph ^ 1, wc);
-        ok = __shfl_sync(0xffffffffu, ok, 0);
-        if (!ok) break;
-        const uint32_t qf = smem_u32(&bars->qd_full[s]);
-        if (lane == 0) {
-          mbar_arrive_expect_tx(qf, 2 * kTileBytes);
-          ++qd_arm[s];
-          for (int c = 0; c < 2; ++c) {
-            tma_load_3d(sbase + kKvOffQ + s * kTileBytes + c * kChunkBytes, &tm_q, qf, c * 64,
-                        it.g * a.G, qs);
-            tma_load_3d(sbase + kKvOffDO + s * kTileBytes + c * kChunkBytes, &tm_do, qf, c * 64,
-                        it.g * a.G, qs);
-          }
-        }
-        float* st = stats + s * 256;
+        // The tile's statistics are read before waiting for its buffer, so the
+        // global-load latency overlaps the wait.
+        float lse2[4], dr[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int r = lane + 32 * e;
           const int tok = qs + (r >> a.logG), h = it.g * a.G + (r & (a.G - 1));
           const bool vr = tok < it.d1;
-          st[r] = vr ? __ldg(a.lse + (size_t)h * a.T + tok) * kLog2e : 0.f;
-          st[128 + r] = vr ? __ldg(a.dvec + (size_t)h * a.T + tok) : 0.f;
+          lse2[e] = vr ? __ldg(a.lse + (size_t)h * a.T + tok) * kLog2e : 0.f;
+          dr[e] = vr ? __ldg(a.dvec + (size_t)h * a.T + tok) : 0.f;
+        }
+        const uint32_t qf = smem_u32(&bars->q_full[sq]), df = smem_u32(&bars->do_full[s]);
+        if (lane == 0) {
+          if (qd_iter >= kQStages) ok = mbar_wait(smem_u32(&bars->q_empty[sq]), phq ^ 1, wc);
+          if (ok) {
+            mbar_arrive_expect_tx(qf, kTileBytes);
+            ++q_arm[sq];
+            for (int c = 0; c < 2; ++c)
+              tma_load_3d(sbase + kKvOffQ + sq * kTileBytes + c * kChunkBytes, &tm_q, qf, c * 64,
+                          it.g * a.G, qs);
+          }
+          if (ok && qd_iter >= 2) ok = mbar_wait(smem_u32(&bars->do_empty[s]), ph ^ 1, wc);
+          if (ok) {
+            mbar_arrive_expect_tx(df, kTileBytes);
+            ++do_arm[s];
+            for (int c = 0; c < 2; ++c)
+              tma_load_3d(sbase + kKvOffDO + s * kTileBytes + c * kChunkBytes, &tm_do, df,
+                          c * 64, it.g * a.G, qs);
+          }
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        float* st = stats + s * 256;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          st[lane + 32 * e] = lse2[e];
+          st[128 + lane + 32 * e] = dr[e];
         }
         __syncwarp();
-        if (lane == 0) mbar_arrive(qf);
+        if (lane == 0) mbar_arrive(df);
       }
       ++item_count;
     }
@@ -229,8 +258,10 @@ attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_q,
       volatile int no_abort = 0;
       const WaitCtx drain{&no_abort, a.status, kStatusTimeoutBwdKV};
       if (kv_arm) mbar_wait(smem_u32(&bars->kv_full), (kv_arm - 1) & 1, drain);
-      if (qd_arm[0]) mbar_wait(smem_u32(&bars->qd_full[0]), (qd_arm[0] - 1) & 1, drain);
-      if (qd_arm[1]) mbar_wait(smem_u32(&bars->qd_full[1]), (qd_arm[1] - 1) & 1, drain);
+      for (int s = 0; s < kQStages; ++s)
+        if (q_arm[s]) mbar_wait(smem_u32(&bars->q_full[s]), (q_arm[s] - 1) & 1, drain);
+      for (int s = 0; s < 2; ++s)
+        if (do_arm[s]) mbar_wait(smem_u32(&bars->do_full[s]), (do_arm[s] - 1) & 1, drain);
     }
   } else if (warp == kWarpMma) {
     // TMEM regions R0 = [0,128), R1 = [128,256) rotate between query tiles
@@ -239,7 +270,8 @@ attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_q,
     // is free once they have read dP^T(t) (ds_full). Issue order per tile:
     // dV(t), S^T(t+1) into Y_t, dK(t), then - after dK(t) has completed, as it
     // reads X_t - dP^T(t+1) into X_t.
-    if (lane == 0) {
+    {
+      const uint32_t leader = elect_one();   // the one lane that issues
       const uint32_t idesc_ss = make_idesc_f16(128, 128, 0, 0);
       const uint32_t idesc_ts = make_idesc_f16(128, 128, 0, 1);
       uint32_t item_count = 0, t = 0, dk_count = 0, p_cnt = 0, ds_cnt = 0;
@@ -247,85 +279,92 @@ attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_q,
       const uint32_t kt = sbase + kKvOffK, vt = sbase + kKvOffV;
       auto region = [&](uint32_t r) { return tmem + (r & 1) * 128; };
       auto issue_s = [&](uint32_t tt) {          // S^T(tt) into X_tt
-        const uint32_t qt = sbase + kKvOffQ + (tt & 1) * kTileBytes;
+        const uint32_t qt = sbase + kKvOffQ + (tt % kQStages) * kTileBytes;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_ss(region(tt), kmajor_desc(kt, kk), kmajor_desc(qt, kk), idesc_ss, kk > 0);
-        mma_commit(smem_u32(&bars->s_full));
+          mma_ss_w(region(tt), kmajor_desc(kt, kk), kmajor_desc(qt, kk), idesc_ss, kk > 0, leader);
+        mma_commit_w(smem_u32(&bars->s_full), leader);
       };
       auto issue_dp = [&](uint32_t tt) {         // dP^T(tt) into Y_tt
         const uint32_t dot = sbase + kKvOffDO + (tt & 1) * kTileBytes;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_ss(region(tt + 1), kmajor_desc(vt, kk), kmajor_desc(dot, kk), idesc_ss, kk > 0);
-        mma_commit(smem_u32(&bars->dp_full));
+          mma_ss_w(region(tt + 1), kmajor_desc(vt, kk), kmajor_desc(dot, kk), idesc_ss, kk > 0,
+                   leader);
+        mma_commit_w(smem_u32(&bars->dp_full), leader);
       };
       while (ok) {
         int idx = -1;
-        ok = ring_pop1(&bars->ring, item_count, &idx, wc);
+        ok = ring_pop(&bars->ring, item_count, &idx, wc);
         if (!ok || idx < 0) break;
         const KvItem it = decode_kv(a, idx);
-        ok = mbar_wait(smem_u32(&bars->kv_full), item_count & 1, wc);
+        ok = mbar_wait_warp(smem_u32(&bars->kv_full), item_count & 1, wc);
         if (!ok) break;
         {  // S^T and dP^T of the item's first query tile
-          ok = mbar_wait(smem_u32(&bars->qd_full[t & 1]), (t >> 1) & 1, wc);
+          ok = mbar_wait_warp(smem_u32(&bars->q_full[t % kQStages]), (t / kQStages) & 1, wc);
           if (!ok) break;
           tc_fence_after();
           issue_s(t);                            // X_t = Y_{t-1}: free after ds_full(t-1)
-          if (dk_count > 0) ok = mbar_wait(smem_u32(&bars->dk_done), (dk_count - 1) & 1, wc);
+          if (dk_count > 0) ok = mbar_wait_warp(smem_u32(&bars->dk_done), (dk_count - 1) & 1, wc);
+          if (ok) ok = mbar_wait_warp(smem_u32(&bars->do_full[t & 1]), (t >> 1) & 1, wc);
           if (!ok) break;
           tc_fence_after();
           issue_dp(t);                           // Y_t = X_{t-1}: free after dK(t-1)
         }
         for (int m = 0; m < it.nq && ok; ++m, ++t) {
-          const uint32_t s = t & 1;
-          const uint32_t qt = sbase + kKvOffQ + s * kTileBytes;
+          const uint32_t s = t & 1, sq = t % kQStages;
+          const uint32_t qt = sbase + kKvOffQ + sq * kTileBytes;
           const uint32_t dot = sbase + kKvOffDO + s * kTileBytes;
           const uint32_t X = region(t);
           const bool has_next = m + 1 < it.nq;
           // dV(t) += P^T(t) dO(t)
-          ok = mbar_wait(smem_u32(&bars->p_full), p_cnt & 1, wc);
+          ok = mbar_wait_warp(smem_u32(&bars->p_full), p_cnt & 1, wc);
           ++p_cnt;
           if (ok && m == 0 && item_count > 0)
-            ok = mbar_wait(smem_u32(&bars->acc_empty), (item_count - 1) & 1, wc);
+            ok = mbar_wait_warp(smem_u32(&bars->acc_empty), (item_count - 1) & 1, wc);
           if (!ok) break;
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            mma_ts(tmem + 256, X + split_a_col(kk), mnmajor_desc(dot, kk), idesc_ts,
-                   (m > 0 || kk > 0) ? 1u : 0u);
+            mma_ts_w(tmem + 256, X + split_a_col(kk), mnmajor_desc(dot, kk), idesc_ts,
+                     (m > 0 || kk > 0) ? 1u : 0u, leader);
           // dS^T(t) written; dP^T(t) read -> Y_t free for S^T(t+1)
-          ok = mbar_wait(smem_u32(&bars->ds_full), ds_cnt & 1, wc);
+          ok = mbar_wait_warp(smem_u32(&bars->ds_full), ds_cnt & 1, wc);
           ++ds_cnt;
-          if (ok && has_next) ok = mbar_wait(smem_u32(&bars->qd_full[(t + 1) & 1]),
-                                             ((t + 1) >> 1) & 1, wc);
+          if (ok && has_next) ok = mbar_wait_warp(smem_u32(&bars->q_full[(t + 1) % kQStages]),
+                                                  ((t + 1) / kQStages) & 1, wc);
           if (!ok) break;
           tc_fence_after();
+          // dO(t) and its statistics: dV(t) (issued) is their last reader on the
+          // tensor cores, and the math warps are done with them (ds_full).
+          mma_commit_w(smem_u32(&bars->do_empty[s]), leader);
           if (has_next) issue_s(t + 1);
           // dK(t) += dS^T(t) Q(t)
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            mma_ts(tmem + 384, X + 32 + split_a_col(kk), mnmajor_desc(qt, kk), idesc_ts,
-                   (m > 0 || kk > 0) ? 1u : 0u);
-          mma_commit(smem_u32(&bars->dk_done));
+            mma_ts_w(tmem + 384, X + 32 + split_a_col(kk), mnmajor_desc(qt, kk), idesc_ts,
+                     (m > 0 || kk > 0) ? 1u : 0u, leader);
+          mma_commit_w(smem_u32(&bars->dk_done), leader);
           ++dk_count;
-          mma_commit(smem_u32(&bars->qd_empty[s]));
+          mma_commit_w(smem_u32(&bars->q_empty[sq]), leader);
           if (has_next) {
-            ok = mbar_wait(smem_u32(&bars->dk_done), (dk_count - 1) & 1, wc);
+            ok = mbar_wait_warp(smem_u32(&bars->dk_done), (dk_count - 1) & 1, wc);
+            if (ok)
+              ok = mbar_wait_warp(smem_u32(&bars->do_full[(t + 1) & 1]), ((t + 1) >> 1) & 1, wc);
             if (!ok) break;
             tc_fence_after();
             issue_dp(t + 1);
           }
         }
         if (!ok) break;
-        mma_commit(smem_u32(&bars->kv_empty));
-        mma_commit(smem_u32(&bars->acc_full));
+        mma_commit_w(smem_u32(&bars->kv_empty), leader);
+        mma_commit_w(smem_u32(&bars->acc_full), leader);
         ++item_count;
       }
-      mma_commit(smem_u32(&bars->drain));
+      mma_commit_w(smem_u32(&bars->drain), leader);
       volatile int no_abort = 0;
       const WaitCtx drain{&no_abort, a.status, kStatusTimeoutBwdKV};
-      mbar_wait(smem_u32(&bars->drain), 0, drain);
+      mbar_wait_warp(smem_u32(&bars->drain), 0, drain);
     }
   } else {
     // ---------------------------------------------------------------- math warps
@@ -348,8 +387,8 @@ attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_q,
         const float* st = stats + stg * 256;
         const bool needs_mask = (it.k0 + kTileKeys - 1 > qs) || (it.k0 + kTileKeys > it.d1) ||
                                 (qs + a.R > it.d1) || (a.W > 0 && qs + a.R - 1 - it.k0 >= a.W);
-        // the tile's statistics are in shared memory once qd_full completes
-        ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->qd_full[stg]), ph, wc));
+        // the tile's statistics are in shared memory once do_full completes
+        ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->do_full[stg]), ph, wc));
         if (!ok) break;
         ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->s_full), s_cnt & 1, wc));
         ++s_cnt;
@@ -498,9 +537,12 @@ attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_q,
 // ============================================================================
 // dQ : query-major
 // ============================================================================
+// K and V tiles stream through one ring of kQSlots 32 KB slots in the order
+// K(0), V(0), K(1), V(1), ...; V(t) is released by dP(t), K(t) by dQ(t).
+constexpr int kQSlots = 5;
 struct __align__(8) QBars {
   uint64_t qd_full, qd_empty;
-  uint64_t kv_full[2], kv_empty[2];
+  uint64_t kv_full[kQSlots], kv_empty[kQSlots];
   uint64_t s_full[2], dq_done[2];     // per S buffer
   uint64_t dp_full, ds_full, acc_full, acc_empty;
   uint64_t drain;
@@ -508,12 +550,12 @@ struct __align__(8) QBars {
 };
 constexpr uint32_t kQOffQ = 0;
 constexpr uint32_t kQOffDO = kTileBytes;
-constexpr uint32_t kQOffK = 2 * kTileBytes;                  // 2 stages
-constexpr uint32_t kQOffV = kQOffK + 2 * kTileBytes;         // 2 stages
-constexpr uint32_t kQOffBar = kQOffV + 2 * kTileBytes;
+constexpr uint32_t kQOffKV = 2 * kTileBytes;                 // kQSlots slots
+constexpr uint32_t kQOffBar = kQOffKV + kQSlots * kTileBytes;
 constexpr uint32_t kQOffTmem = kQOffBar + sizeof(QBars);
 constexpr uint32_t kQOffAbort = kQOffTmem + 16;
-constexpr uint32_t kQSmem = kQOffAbort + 16 + 1024;
+constexpr uint32_t kQSmem = kQOffAbort + 16;   // no slack: the base is checked instead
+static_assert(kQSmem <= 227 * 1024, "exceeds the shared memory of one CTA");
 // TMEM columns: S double-buffered, dP, dQ accumulator
 constexpr uint32_t kQColS0 = 0, kQColDP = 256, kQColDQ = 384;
 
@@ -537,9 +579,12 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q,
                    const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v,
                    const __grid_constant__ CUtensorMap tm_do, const BwdArgs a) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  if (smem_u32(smem_raw) & 1023) {
+    if (threadIdx.x == 0) atomicOr(a.status, kStatusSmemAlign);
+    return;
+  }
+  uint8_t* smem = smem_raw;
   const uint32_t sbase = smem_u32(smem);
   QBars* bars = reinterpret_cast<QBars*>(smem + kQOffBar);
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + kQOffTmem);
@@ -551,9 +596,11 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q,
     *abort_flag = 0;
     mbar_init(smem_u32(&bars->qd_full), 1);
     mbar_init(smem_u32(&bars->qd_empty), 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < kQSlots; ++s) {
       mbar_init(smem_u32(&bars->kv_full[s]), 1);
       mbar_init(smem_u32(&bars->kv_empty[s]), 1);
+    }
+    for (int s = 0; s < 2; ++s) {
       mbar_init(smem_u32(&bars->s_full[s]), 1);
       mbar_init(smem_u32(&bars->dq_done[s]), 1);
     }
@@ -577,7 +624,7 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q,
 
   if (warp == kWarpTma) {
     if (lane == 0) {
-      uint32_t item_count = 0, kv_iter = 0, qd_arm = 0, kv_arm0 = 0, kv_arm1 = 0;
+      uint32_t item_count = 0, kv_load = 0, qd_arm = 0, arm[kQSlots] = {};
       bool ok = true;
       while (ok) {
         int idx = atomicAdd(a.next_item, 1);
@@ -594,33 +641,32 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q,
           tma_load_3d(sbase + kQOffQ + c * kChunkBytes, &tm_q, qf, c * 64, it.g * a.G, it.q0);
           tma_load_3d(sbase + kQOffDO + c * kChunkBytes, &tm_do, qf, c * 64, it.g * a.G, it.q0);
         }
-        for (int n = 0; n < it.ntiles && ok; ++n, ++kv_iter) {
-          const int ks = it.kend - kTileKeys * (n + 1);
-          const uint32_t s = kv_iter & 1, ph = (kv_iter >> 1) & 1;
-          if (kv_iter >= 2) ok = mbar_wait(smem_u32(&bars->kv_empty[s]), ph ^ 1, wc);
+        for (int j = 0; j < 2 * it.ntiles && ok; ++j, ++kv_load) {
+          const int ks = it.kend - kTileKeys * ((j >> 1) + 1);
+          const uint32_t s = kv_load % kQSlots, ph = (kv_load / kQSlots) & 1;
+          if (kv_load >= kQSlots) ok = mbar_wait(smem_u32(&bars->kv_empty[s]), ph ^ 1, wc);
           if (!ok) break;
-          const uint32_t kf = smem_u32(&bars->kv_full[s]);
-          mbar_arrive_expect_tx(kf, 2 * kTileBytes);
-          if (s == 0) ++kv_arm0; else ++kv_arm1;
-          for (int c = 0; c < 2; ++c) {
-            tma_load_3d(sbase + kQOffK + s * kTileBytes + c * kChunkBytes, &tm_k, kf, c * 64, it.g,
+          const uint32_t f = smem_u32(&bars->kv_full[s]);
+          mbar_arrive_expect_tx(f, kTileBytes);
+          ++arm[s];
+          const CUtensorMap* m = (j & 1) ? &tm_v : &tm_k;
+          for (int c = 0; c < 2; ++c)
+            tma_load_3d(sbase + kQOffKV + s * kTileBytes + c * kChunkBytes, m, f, c * 64, it.g,
                         ks);
-            tma_load_3d(sbase + kQOffV + s * kTileBytes + c * kChunkBytes, &tm_v, kf, c * 64, it.g,
-                        ks);
-          }
         }
         ++item_count;
       }
       volatile int no_abort = 0;
       const WaitCtx drain{&no_abort, a.status, kStatusTimeoutBwdQ};
       if (qd_arm) mbar_wait(smem_u32(&bars->qd_full), (qd_arm - 1) & 1, drain);
-      if (kv_arm0) mbar_wait(smem_u32(&bars->kv_full[0]), (kv_arm0 - 1) & 1, drain);
-      if (kv_arm1) mbar_wait(smem_u32(&bars->kv_full[1]), (kv_arm1 - 1) & 1, drain);
+      for (int s = 0; s < kQSlots; ++s)
+        if (arm[s]) mbar_wait(smem_u32(&bars->kv_full[s]), (arm[s] - 1) & 1, drain);
     }
   } else if (warp == kWarpMma) {
     // Per tile t: dP(t), S(t+1) (into the other S buffer, once dQ(t-1) has read
     // it), dQ(t). P of tile t+1 is then computed while dQ(t) and dP(t+1) run.
-    if (lane == 0) {
+    {
+      const uint32_t leader = elect_one();   // the one lane that issues
       const uint32_t idesc_ss = make_idesc_f16(128, 128, 0, 0);
       const uint32_t idesc_ts = make_idesc_f16(128, 128, 0, 1);
       uint32_t item_count = 0, t = 0, ds_cnt = 0, dq_cnt0 = 0, dq_cnt1 = 0;
@@ -628,65 +674,73 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q,
       const uint32_t qt = sbase + kQOffQ, dot = sbase + kQOffDO;
       // S(tt) = Q K(tt)^T into buffer tt % 2, after the dQ that last read it.
       auto issue_s = [&](uint32_t tt) -> bool {
-        const uint32_t b = tt & 1, st = tt & 1, ph = (tt >> 1) & 1;
-        if (!mbar_wait(smem_u32(&bars->kv_full[st]), ph, wc)) return false;
+        const uint32_t b = tt & 1, lk = 2 * tt;                 // K(tt) in the ring
+        const uint32_t st = lk % kQSlots, ph = (lk / kQSlots) & 1;
+        if (!mbar_wait_warp(smem_u32(&bars->kv_full[st]), ph, wc)) return false;
         const uint32_t cnt = b ? dq_cnt1 : dq_cnt0;
-        if (cnt > 0 && !mbar_wait(smem_u32(&bars->dq_done[b]), (cnt - 1) & 1, wc)) return false;
+        if (cnt > 0 && !mbar_wait_warp(smem_u32(&bars->dq_done[b]), (cnt - 1) & 1, wc))
+          return false;
         tc_fence_after();
-        const uint32_t kt = sbase + kQOffK + st * kTileBytes;
+        const uint32_t kt = sbase + kQOffKV + st * kTileBytes;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_ss(tmem + kQColS0 + b * 128, kmajor_desc(qt, kk), kmajor_desc(kt, kk), idesc_ss,
-                 kk > 0);
-        mma_commit(smem_u32(&bars->s_full[b]));
+          mma_ss_w(tmem + kQColS0 + b * 128, kmajor_desc(qt, kk), kmajor_desc(kt, kk), idesc_ss,
+                 kk > 0, leader);
+        mma_commit_w(smem_u32(&bars->s_full[b]), leader);
         return true;
       };
       while (ok) {
         int idx = -1;
-        ok = ring_pop1(&bars->ring, item_count, &idx, wc);
+        ok = ring_pop(&bars->ring, item_count, &idx, wc);
         if (!ok || idx < 0) break;
         const QItem it = decode_q(a, idx);
-        ok = mbar_wait(smem_u32(&bars->qd_full), item_count & 1, wc);
+        ok = mbar_wait_warp(smem_u32(&bars->qd_full), item_count & 1, wc);
         if (!ok) break;
         tc_fence_after();
         ok = issue_s(t);
         for (int n = 0; n < it.ntiles && ok; ++n, ++t) {
-          const uint32_t st = t & 1;
-          const uint32_t vt = sbase + kQOffV + st * kTileBytes;
-          const uint32_t kt = sbase + kQOffK + st * kTileBytes;
+          const uint32_t sk = (2 * t) % kQSlots, lv = 2 * t + 1;   // K(t), V(t) in the ring
+          const uint32_t sv = lv % kQSlots;
+          const uint32_t vt = sbase + kQOffKV + sv * kTileBytes;
+          const uint32_t kt = sbase + kQOffKV + sk * kTileBytes;
+          ok = mbar_wait_warp(smem_u32(&bars->kv_full[sv]), (lv / kQSlots) & 1, wc);
+          if (!ok) break;
+          tc_fence_after();
           // dP(t) = dO V(t)^T; the math warps finished reading dP(t-1) before ds_full(t-1)
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            mma_ss(tmem + kQColDP, kmajor_desc(dot, kk), kmajor_desc(vt, kk), idesc_ss, kk > 0);
-          mma_commit(smem_u32(&bars->dp_full));
+            mma_ss_w(tmem + kQColDP, kmajor_desc(dot, kk), kmajor_desc(vt, kk), idesc_ss, kk > 0,
+                     leader);
+          mma_commit_w(smem_u32(&bars->dp_full), leader);
+          mma_commit_w(smem_u32(&bars->kv_empty[sv]), leader);   // V(t) done after dP(t)
           if (n + 1 < it.ntiles) {
             ok = issue_s(t + 1);
             if (!ok) break;
           }
-          ok = mbar_wait(smem_u32(&bars->ds_full), ds_cnt & 1, wc);
+          ok = mbar_wait_warp(smem_u32(&bars->ds_full), ds_cnt & 1, wc);
           ++ds_cnt;
           if (ok && n == 0 && item_count > 0)
-            ok = mbar_wait(smem_u32(&bars->acc_empty), (item_count - 1) & 1, wc);
+            ok = mbar_wait_warp(smem_u32(&bars->acc_empty), (item_count - 1) & 1, wc);
           if (!ok) break;
           tc_fence_after();
           const uint32_t b = t & 1;
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            mma_ts(tmem + kQColDQ, tmem + kQColS0 + b * 128 + split_a_col(kk), mnmajor_desc(kt, kk),
-                   idesc_ts, (n > 0 || kk > 0) ? 1u : 0u);
-          mma_commit(smem_u32(&bars->dq_done[b]));
+            mma_ts_w(tmem + kQColDQ, tmem + kQColS0 + b * 128 + split_a_col(kk),
+                     mnmajor_desc(kt, kk), idesc_ts, (n > 0 || kk > 0) ? 1u : 0u, leader);
+          mma_commit_w(smem_u32(&bars->dq_done[b]), leader);
           if (b) ++dq_cnt1; else ++dq_cnt0;
-          mma_commit(smem_u32(&bars->kv_empty[st]));
+          mma_commit_w(smem_u32(&bars->kv_empty[sk]), leader);   // K(t) done after dQ(t)
         }
         if (!ok) break;
-        mma_commit(smem_u32(&bars->qd_empty));
-        mma_commit(smem_u32(&bars->acc_full));
+        mma_commit_w(smem_u32(&bars->qd_empty), leader);
+        mma_commit_w(smem_u32(&bars->acc_full), leader);
         ++item_count;
       }
-      mma_commit(smem_u32(&bars->drain));
+      mma_commit_w(smem_u32(&bars->drain), leader);
       volatile int no_abort = 0;
       const WaitCtx drain{&no_abort, a.status, kStatusTimeoutBwdQ};
-      mbar_wait(smem_u32(&bars->drain), 0, drain);
+      mbar_wait_warp(smem_u32(&bars->drain), 0, drain);
     }
   } else {
     // ---------------------------------------------------------------- math warps

@@ -21,6 +21,7 @@ enum : int {
   kStatusTimeoutFwd = 1,
   kStatusTimeoutBwdKV = 2,
   kStatusTimeoutBwdQ = 4,
+  kStatusSmemAlign = 8,        // dynamic shared memory not 1024-byte aligned
 };
 
 // Parameters after validation and defaulting.
