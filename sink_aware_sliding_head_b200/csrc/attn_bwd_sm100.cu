@@ -94,7 +94,7 @@ constexpr int kQStages = 3;   // Q tiles in flight (its buffer is released last,
 struct __align__(8) KvBars {
   uint64_t kv_full, kv_empty;
   uint64_t q_full[kQStages], q_empty[kQStages], do_full[2], do_empty[2];
-  uint64_t s_full, dp_full, p_full, ds_full, dv_done, dk_done, acc_full, acc_empty;
+  uint64_t s_full, dp_full, p_full, dp_free, ds_full, dk_done, acc_full, acc_empty;
   uint64_t drain;
   ItemRing ring;
 };
@@ -159,7 +159,7 @@ attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_q,
     mbar_init(smem_u32(&bars->dp_full), 1);
     mbar_init(smem_u32(&bars->p_full), kMathWarps);
     mbar_init(smem_u32(&bars->ds_full), kMathWarps);
-    mbar_init(smem_u32(&bars->dv_done), 1);
+    mbar_init(smem_u32(&bars->dp_free), kMathWarps);
     mbar_init(smem_u32(&bars->dk_done), 1);
     mbar_init(smem_u32(&bars->acc_full), 1);
     mbar_init(smem_u32(&bars->acc_empty), kMathWarps);
@@ -267,14 +267,15 @@ attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_q,
     // TMEM regions R0 = [0,128), R1 = [128,256) rotate between query tiles
     // (numbered t across items): S^T(t) goes to X_t = R(t&1), dP^T(t) to
     // Y_t = R(~t&1). The math warps write P^T(t) and dS^T(t) into X_t, so Y_t
-    // is free once they have read dP^T(t) (ds_full). Issue order per tile:
-    // dV(t), S^T(t+1) into Y_t, dK(t), then - after dK(t) has completed, as it
+    // is free once they have loaded dP^T(t) into registers (dp_free, early in
+    // their dS step). Issue order per tile: dV(t), S^T(t+1) into Y_t (runs
+    // while dS(t) is computed), dK(t), then - after dK(t) has completed, as it
     // reads X_t - dP^T(t+1) into X_t.
     {
       const uint32_t leader = elect_one();   // the one lane that issues
       const uint32_t idesc_ss = make_idesc_f16(128, 128, 0, 0);
       const uint32_t idesc_ts = make_idesc_f16(128, 128, 0, 1);
-      uint32_t item_count = 0, t = 0, dk_count = 0, p_cnt = 0, ds_cnt = 0;
+      uint32_t item_count = 0, t = 0, dk_count = 0, p_cnt = 0, ds_cnt = 0, dpf_cnt = 0;
       bool ok = true;
       const uint32_t kt = sbase + kKvOffK, vt = sbase + kKvOffV;
       auto region = [&](uint32_t r) { return tmem + (r & 1) * 128; };
@@ -328,17 +329,24 @@ attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_q,
           for (int kk = 0; kk < 8; ++kk)
             mma_ts_w(tmem + 256, X + split_a_col(kk), mnmajor_desc(dot, kk), idesc_ts,
                      (m > 0 || kk > 0) ? 1u : 0u, leader);
-          // dS^T(t) written; dP^T(t) read -> Y_t free for S^T(t+1)
+          // dP^T(t) read by the math warps -> Y_t free for S^T(t+1)
+          if (has_next) {
+            ok = mbar_wait_warp(smem_u32(&bars->dp_free), dpf_cnt & 1, wc);
+            if (ok) ok = mbar_wait_warp(smem_u32(&bars->q_full[(t + 1) % kQStages]),
+                                        ((t + 1) / kQStages) & 1, wc);
+            if (!ok) break;
+            tc_fence_after();
+            issue_s(t + 1);
+          }
+          ++dpf_cnt;
+          // dS^T(t) written
           ok = mbar_wait_warp(smem_u32(&bars->ds_full), ds_cnt & 1, wc);
           ++ds_cnt;
-          if (ok && has_next) ok = mbar_wait_warp(smem_u32(&bars->q_full[(t + 1) % kQStages]),
-                                                  ((t + 1) / kQStages) & 1, wc);
           if (!ok) break;
           tc_fence_after();
           // dO(t) and its statistics: dV(t) (issued) is their last reader on the
           // tensor cores, and the math warps are done with them (ds_full).
           mma_commit_w(smem_u32(&bars->do_empty[s]), leader);
-          if (has_next) issue_s(t + 1);
           // dK(t) += dS^T(t) Q(t)
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
@@ -447,6 +455,10 @@ attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_q,
           tmem_ld32(t_row + Y + c0 + 32, u1);
           tc_wait_ld_dep(u0);
           tc_wait_ld_dep(u1);
+          // dP^T(t) is in registers: Y may take S^T(t+1)
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(smem_u32(&bars->dp_free));
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
             const int c = c0 + 2 * e;
