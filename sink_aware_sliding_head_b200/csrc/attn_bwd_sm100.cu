@@ -137,7 +137,7 @@ attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_q,
   uint8_t* smem = smem_raw;
   const uint32_t sbase = smem_u32(smem);
   KvBars* bars = reinterpret_cast<KvBars*>(smem + kKvOffBar);
-  float* stats = reinterpret_cast<float*>(smem + kKvOffStats);   // [buf][lse2|D][128]
+  float* stats = reinterpret_cast<float*>(smem + kKvOffStats);   // [buf][-lse2|D][128]
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + kKvOffTmem);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kKvOffAbort);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -179,7 +179,7 @@ attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_q,
 
   if (warp == kWarpTma) {
     // Lane 0 takes items from the global counter and issues TMA; the whole warp
-    // stages each query tile's per-row log2-LSE and D into shared memory and
+    // stages each query tile's per-row -log2-LSE and D into shared memory and
     // completes do_full's second arrival.
     uint32_t item_count = 0, qd_iter = 0, kv_arm = 0, q_arm[kQStages] = {}, do_arm[2] = {};
     bool ok = true;
@@ -219,7 +219,7 @@ attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_q,
           const int r = lane + 32 * e;
           const int tok = qs + (r >> a.logG), h = it.g * a.G + (r & (a.G - 1));
           const bool vr = tok < it.d1;
-          lse2[e] = vr ? __ldg(a.lse + (size_t)h * a.T + tok) * kLog2e : 0.f;
+          lse2[e] = vr ? -__ldg(a.lse + (size_t)h * a.T + tok) * kLog2e : 0.f;   // negated
           dr[e] = vr ? __ldg(a.dvec + (size_t)h * a.T + tok) : 0.f;
         }
         const uint32_t qf = smem_u32(&bars->q_full[sq]), df = smem_u32(&bars->do_full[s]);
@@ -404,6 +404,7 @@ attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_q,
         tc_fence_after();
         // TMEM regions of this tile: S^T in X, dP^T in Y (rotating per tile)
         const uint32_t X = (tile_count & 1) * 128, Y = 128 - X;
+        const uint64_t sc2 = f2(a.scale_log2, a.scale_log2);
         // P^T for query rows [c0, c0+64): 2^(s*scale - lse2), masked, fp16.
         // Row c of the tile is token qs + c/G, so the rows that see key j form
         // one column range [cmin, cmax); masked and unmasked tiles run separate
@@ -427,9 +428,14 @@ attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_q,
               const int c = c0 + 2 * e;
               const float s0 = __uint_as_float(e < 16 ? u0[2 * e] : u1[2 * e - 32]);
               const float s1 = __uint_as_float(e < 16 ? u0[2 * e + 1] : u1[2 * e - 31]);
-              const float2 l2 = *reinterpret_cast<const float2*>(st + c);
-              float p0 = ex2_approx(fmaf(s0, a.scale_log2, -l2.x));
-              float p1 = ex2_approx(fmaf(s1, a.scale_log2, -l2.y));
+              const uint64_t nl2 = *reinterpret_cast<const uint64_t*>(st + c);   // -lse2 pair
+              float x0, x1;
+              f2_split(ffma2(f2(s0, s1), sc2, nl2), x0, x1);
+              // one pair in four on the FMA pipe (polynomial 2^x), the rest on
+              // the special-function unit, which alone would bound this loop
+              float p0, p1;
+              if ((e & 3) == 3) exp2_fma2(x0, x1, p0, p1);
+              else { p0 = ex2_approx(x0); p1 = ex2_approx(x1); }
               if (decltype(masked)::value) {
                 p0 = (c >= cmin && c < cmax) ? p0 : 0.f;
                 p1 = (c + 1 >= cmin && c + 1 < cmax) ? p1 : 0.f;
@@ -801,7 +807,11 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q,
               const uint32_t a1 = e < 16 ? u0[2 * e + 1] : u1[2 * e - 31];
               float x0, x1;
               f2_split(ffma2(f2(__uint_as_float(a0), __uint_as_float(a1)), sc2, nl2), x0, x1);
-              float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+              // one pair in four on the FMA pipe (polynomial 2^x), the rest on
+              // the special-function unit, which alone would bound this loop
+              float p0, p1;
+              if ((e & 3) == 3) exp2_fma2(x0, x1, p0, p1);
+              else { p0 = ex2_approx(x0); p1 = ex2_approx(x1); }
               if (decltype(masked)::value) {
                 const int c = c0 + 2 * e;
                 p0 = (valid && c >= c_lo && c <= c_hi) ? p0 : 0.f;
