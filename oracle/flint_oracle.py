@@ -377,3 +377,52 @@ class RowOracle:
         dx, _ = prologue_backward(self.k[j:j + 1, kv:kv + 1, :], self.w_k, dk_hat[None, None, :],
                                   self.pos[j:j + 1], self.use_rope, self.theta, self.eps)
         return dx[0, 0], dv
+
+
+# ----------------------------------------------------------------------------
+# Decode: one new token per sequence attending over its KV cache
+# ----------------------------------------------------------------------------
+
+def decode(q, k_new, v_new, w_q, w_k, sink, cache_lens, k_cache, v_cache, window,
+           use_rope, rope_theta, eps=1e-6, scale=None, store=None):
+    """The layer's forward for the next token of B cached sequences.
+
+    Same definition as ``flint_attn_fwd``, restricted to one query row: sequence
+    b has ``cache_lens[b]`` = p tokens cached (positions 0..p-1), so the new token
+    sits at position p (RoPE angle and causal index). Its normalised, rotated key
+    and its value are written into slot p of the caches first, and attention
+    reads the caches: the query sees slots j with max(0, p - W + 1) <= j <= p
+    (W <= 0: all of 0..p), plus the sink category.
+
+    q [B, H, D], k_new / v_new [B, Hk, D] are the raw projections of the new
+    token; the caches are [B, Hk, C, D] (head-major per sequence) and hold
+    normalised, rotated keys. ``store`` maps a row to the value the cache holds
+    after the write (rounding to the cache dtype); None keeps it exact.
+    Returns out [B, H, D], lse [B, H] and the updated caches.
+    """
+    q, k_new, v_new, w_q, w_k, sink = map(_f64, (q, k_new, v_new, w_q, w_k, sink))
+    kc = _f64(k_cache).copy()
+    vc = _f64(v_cache).copy()
+    lens = np.asarray(_f64(cache_lens), dtype=np.int64)
+    B, H, D = q.shape
+    Hk = k_new.shape[1]
+    if scale is None:
+        scale = 1.0 / np.sqrt(D)
+    keep = (lambda x: x) if store is None else store
+    out = np.zeros((B, H, D))
+    lse = np.zeros((B, H))
+    for b in range(B):
+        p = int(lens[b])
+        pos = np.array([p])
+        q_hat = prologue(q[b][None], w_q, pos, use_rope, rope_theta, eps)[0]      # [H, D]
+        k_hat = prologue(k_new[b][None], w_k, pos, use_rope, rope_theta, eps)[0]  # [Hk, D]
+        kc[b, :, p, :] = keep(k_hat)
+        vc[b, :, p, :] = keep(v_new[b])
+        lo, _ = visible_keys(p, 0, window)
+        for h in range(H):
+            g = _group(h, H, Hk)
+            z = scale * (kc[b, g, lo:p + 1, :] @ q_hat[h])                       # [n]
+            pr, _, l = _sink_softmax(z[None, None, :], sink[h:h + 1])
+            out[b, h] = pr[0, 0] @ vc[b, g, lo:p + 1, :]
+            lse[b, h] = l[0, 0]
+    return out, lse, kc, vc

@@ -361,3 +361,65 @@ def test_config_constants_golden():
     q[:] = 0
     _, lse = fo.flint_attn_fwd(q, k, v, wq, wk, sink, cu, c["sliding_window"], True, 1e4)
     np.testing.assert_allclose(lse[0], np.log(np.exp(sink[0]) + np.array(n)), atol=1e-12)
+
+
+# ----------------------------------------------------------------------------
+# Decode (one new token per sequence over a KV cache)
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("W,rope", [(0, False), (1, True), (5, True), (64, False)])
+def test_decode_equals_last_row_of_the_layer(W, rope):
+    """Decoding token p over a cache of tokens 0..p-1 is row p of the whole layer."""
+    H, Hk, D, C = 4, 2, 16, 40
+    lens = [1, 9, 23, 37]                  # tokens per sequence, the last one is new
+    rng = np.random.default_rng(11 + W)
+    wq = 1 + 0.1 * rng.standard_normal(D)
+    wk = 1 + 0.1 * rng.standard_normal(D)
+    sink = rng.standard_normal(H)
+    B = len(lens)
+    q_new = np.zeros((B, H, D)); k_new = np.zeros((B, Hk, D)); v_new = np.zeros((B, Hk, D))
+    kc = rng.standard_normal((B, Hk, C, D)); vc = rng.standard_normal((B, Hk, C, D))
+    rows, lses = [], []
+    for b, L in enumerate(lens):
+        q = rng.standard_normal((L, H, D)); k = rng.standard_normal((L, Hk, D))
+        v = rng.standard_normal((L, Hk, D))
+        cu = np.array([0, L])
+        O, lse = fo.flint_attn_fwd(q, k, v, wq, wk, sink, cu, W, rope, 1e4)
+        rows.append(O[L - 1]); lses.append(lse[:, L - 1])
+        k_hat = fo.prologue(k, wk, np.arange(L), rope, 1e4, 1e-6)
+        kc[b, :, :L - 1, :] = k_hat[:L - 1].transpose(1, 0, 2)
+        vc[b, :, :L - 1, :] = v[:L - 1].transpose(1, 0, 2)
+        q_new[b], k_new[b], v_new[b] = q[L - 1], k[L - 1], v[L - 1]
+        want_k = k_hat[L - 1]
+    lens_cached = np.array(lens) - 1
+    out, lse, kc2, vc2 = fo.decode(q_new, k_new, v_new, wq, wk, sink, lens_cached, kc, vc,
+                                   W, rope, 1e4)
+    np.testing.assert_allclose(out, np.stack(rows), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse, np.stack(lses), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(kc2[B - 1, :, lens_cached[-1], :], want_k, rtol=0, atol=1e-12)
+    # slots other than the new one are untouched
+    for b, p in enumerate(lens_cached):
+        mask = np.ones(C, bool); mask[p] = False
+        assert np.array_equal(kc2[b][:, mask], kc[b][:, mask])
+        assert np.array_equal(vc2[b][:, p], v_new[b])
+
+
+def test_decode_window_one_closed_form():
+    """W = 1: only the new key is visible; O = (1 - p_sink) v_new, LSE = log(e^s + e^z)."""
+    H, Hk, D, C = 4, 1, 8, 10
+    rng = np.random.default_rng(5)
+    B = 3
+    q = rng.standard_normal((B, H, D)); k = rng.standard_normal((B, Hk, D))
+    v = rng.standard_normal((B, Hk, D))
+    wq = np.ones(D); wk = np.ones(D); sink = rng.standard_normal(H)
+    kc = rng.standard_normal((B, Hk, C, D)); vc = rng.standard_normal((B, Hk, C, D))
+    lens = np.array([0, 4, 9])
+    out, lse, _, _ = fo.decode(q, k, v, wq, wk, sink, lens, kc, vc, 1, False, 1e4)
+    for b in range(B):
+        qh = q[b] / np.sqrt(np.mean(q[b] ** 2, axis=-1, keepdims=True) + 1e-6)
+        kh = k[b, 0] / np.sqrt(np.mean(k[b, 0] ** 2) + 1e-6)
+        for h in range(H):
+            z = qh[h] @ kh / math.sqrt(D)
+            ps = math.exp(sink[h]) / (math.exp(sink[h]) + math.exp(z))
+            np.testing.assert_allclose(out[b, h], (1 - ps) * v[b, 0], rtol=0, atol=1e-12)
+            assert abs(lse[b, h] - math.log(math.exp(sink[h]) + math.exp(z))) < 1e-12
