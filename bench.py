@@ -35,6 +35,8 @@ METRIC = "sink-attention fwd/bwd TFLOP/s (masked FLOPs) and % of B200 BF16 tenso
 UNIT = "TFLOP/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 WORKLOADS = {w.name: w for w in fi.WORKLOADS}
+DECODE_WORKLOADS = {w.name: w for w in [fi.DECODE_SLIDING_BF16]}
+DECODE_METRIC = "decode step: KV-cache bytes read per second (one new token per sequence)"
 DEFAULT_WORKLOAD = fi.FULL_BF16.name
 L2_FLUSH_BYTES = 256 << 20
 
@@ -45,7 +47,10 @@ def parse_args(argv=None):
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="flint", choices=["flint", "reference"])
-    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
+                    choices=sorted(WORKLOADS) + sorted(DECODE_WORKLOADS),
+                    help="the default is the fwd+bwd layer the headline metric is quoted "
+                         "on; decode_* workloads time flint_attn_decode instead")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
@@ -273,8 +278,227 @@ def run_reference(args):
 
 # --------------------------------------------------------------------------- GPU arm
 
+def decode_config(w, lens, kv_bytes):
+    return {"workload": f"{w.name} decode step", "batch": w.batch,
+            "cache_capacity": w.cache_capacity, "cache_lens": f"drawn U{list(w.lens_range)}",
+            "mean_cache_len": sum(int(x) for x in lens) / len(lens),
+            "heads_q": w.num_q_heads, "heads_kv": w.num_kv_heads, "head_dim": w.head_dim,
+            "window": w.window if w.window > 0 else "unbounded", "rope": bool(w.use_rope),
+            "kv_bytes_per_step": kv_bytes,
+            "l2": "K/V windows (~0.5 GB) larger than L2, plus a 256 MB L2 flush before every step",
+            "parallelism": "replicas (one independent batch per GPU)"}
+
+
+def oracle_decode_sample(w, inp, seconds):
+    """Time the FP64 decode oracle on leading sequences for ~seconds; returns (bytes, s, desc)."""
+    from oracle import flint_oracle as fo   # test infrastructure: CPU baseline leg only
+
+    def run(nb):
+        sl = slice(0, nb)
+        t0 = time.perf_counter()
+        fo.decode(inp["q"][sl], inp["k"][sl], inp["v"][sl], inp["w_q"], inp["w_k"], inp["sink"],
+                  inp["cache_lens"][sl], inp["k_cache"][sl], inp["v_cache"][sl], w.window,
+                  w.use_rope, w.rope_theta)
+        dt = time.perf_counter() - t0
+        return fi.decode_kv_bytes(inp["cache_lens"][sl].tolist(), w.window, w.num_kv_heads), dt
+
+    b0, t0 = run(1)
+    nb = max(1, min(w.batch, int(seconds / max(t0, 1e-3))))
+    b, t = run(nb)
+    return b, t, (f"oracle decode (FP64 NumPy) on the first {nb} of {w.batch} sequences of "
+                  f"{w.name}; K/V bytes of those sequences")
+
+
+def run_reference_decode(args):
+    if int(os.environ.get("RANK", "0")) != 0:
+        return
+    w = DECODE_WORKLOADS[args.workload]
+    inp = fi.make_decode_inputs(w)
+    lens = inp["cache_lens"].tolist()
+    per_step = max(1.0, min(10.0, 120.0 / max(1, args.steps + args.warmup)))
+    tb, tt, desc = 0, 0.0, ""
+    for i in range(args.warmup + args.steps):
+        b, t, desc = oracle_decode_sample(w, inp, per_step)
+        if i >= args.warmup:
+            tb += b
+            tt += t
+    value = tb / tt / 1e9
+    line = {"impl": "reference", "metric": DECODE_METRIC, "value": value, "unit": "GB/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * tt / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": decode_config(w, lens, fi.decode_kv_bytes(lens, w.window, w.num_kv_heads)),
+            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": blas_threads(),
+                             "kind": "oracle", "sample": desc},
+            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_decode(args):
+    """flint_attn_decode on the serving shape: K/V bytes read per second."""
+    from sink_aware_sliding_head_b200 import flint_attn as fa
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=dev)
+        pg = dist
+    w = DECODE_WORKLOADS[args.workload]
+    cpu = fi.make_decode_inputs(w, seed=w.seed + rank)
+    lens = cpu["cache_lens"].tolist()
+    kv_bytes = fi.decode_kv_bytes(lens, w.window, w.num_kv_heads)
+    d = {k: v.to(dev) for k, v in cpu.items()}
+    B, H, D = d["q"].shape
+    p = fa.decode_params(B, w.cache_capacity, H, w.num_kv_heads, w.window, w.use_rope,
+                         w.rope_theta)
+    lib = fa.load_library()
+    import ctypes
+    ws = torch.empty(lib.flint_attn_decode_workspace_bytes(ctypes.byref(p)),
+                     dtype=torch.uint8, device=dev)
+    out = torch.empty(B, H, D, dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(B, H, dtype=torch.float32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def call(src):
+        # writing the new token's slot again with the same values keeps every step identical
+        fa.decode(src["q"], src["k"], src["v"], src["w_q"], src["w_k"], src["sink"],
+                  src["cache_lens"], d["k_cache"], d["v_cache"], w.window, w.use_rope,
+                  w.rope_theta, out=out, lse=lse, workspace=ws)
+
+    for _ in range(max(3, args.warmup)):
+        flush.zero_()
+        call(d)
+    torch.cuda.synchronize(dev)
+    code = lib.flint_attn_check_status(fa._ptr(ws), fa._stream_ptr())
+    if code != 0:
+        raise RuntimeError(f"device status {fa.STATUS.get(code, code)} during warm-up")
+    # timed region: plain calls (a decode step is ~0.1 ms, so per-kernel profiling
+    # events would distort it); the per-kernel split comes from a separate pass
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    clocks = ClockSampler() if rank == 0 else None
+    if clocks:
+        clocks.start()
+    n0 = fa.launch_count()
+    if pg is not None:
+        pg.barrier()
+    torch.cuda.synchronize(dev)
+    for i in range(args.steps):
+        flush.zero_()
+        ev[i][0].record(stream)
+        call(d)
+        ev[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    if pg is not None:
+        pg.barrier()
+    launches = fa.launch_count() - n0
+    clk = clocks.stop(local) if clocks else None
+    t_ms = sum(e[0].elapsed_time(e[1]) for e in ev)
+    fa.profile_reset()
+    fa.profile_collect()
+    fa.profile_reset()
+    fa.profile_enable(True)
+    for i in range(min(args.steps, 50)):
+        flush.zero_()
+        call(d)
+    torch.cuda.synchronize(dev)
+    fa.profile_enable(False)
+    kern = fa.profile_collect()
+    t = torch.tensor([t_ms], dtype=torch.float64)
+    if pg is not None:
+        t = t.to(dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    t_ms = float(t.cpu()[0])
+    value = world * kv_bytes * args.steps / (t_ms * 1e-3) / 1e9
+
+    # end to end: the new tokens' q, k, v and cache_lens in from pinned host memory,
+    # out and LSE back, every step (the caches are device-resident serving state)
+    names_in = ["q", "k", "v", "w_q", "w_k", "sink", "cache_lens"]
+    host_in = {k: cpu[k].pin_memory() for k in names_in}
+    dev_in = {k: torch.empty_like(d[k]) for k in names_in}
+    host_out = {"out": torch.empty(out.shape, dtype=out.dtype, pin_memory=True),
+                "lse": torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)}
+    h2d = sum(x.numel() * x.element_size() for x in host_in.values())
+    d2h = sum(x.numel() * x.element_size() for x in host_out.values())
+
+    def e2e_step():
+        for k in names_in:
+            dev_in[k].copy_(host_in[k], non_blocking=True)
+        call(dev_in)
+        host_out["out"].copy_(out, non_blocking=True)
+        host_out["lse"].copy_(lse, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64)
+    if pg is not None:
+        te = te.to(dev)
+        pg.all_reduce(te, op=pg.ReduceOp.MAX)
+    te_ms = float(te.cpu()[0])
+    if rank != 0:
+        if pg is not None:
+            pg.destroy_process_group()
+        return
+    peaks, peak_src = read_peaks()
+    attn = kern.get("decode", (0.0, 0))
+    per_launch = attn[0] / max(attn[1], 1)
+    achieved = kv_bytes / (per_launch * 1e-3) / 1e9 if attn[1] else None
+    roofline = {"kernel": "decode", "bound": "hbm", "achieved": achieved,
+                "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": (achieved or 0.0) / peaks["hbm_gbs"],
+                "peak_kind": f"HBM copy bandwidth ({peak_src})",
+                "traffic": traffic_for("decode", w.name),
+                "algorithmic_bytes_per_launch": kv_bytes, "ms_per_launch": per_launch,
+                "source": "decode.cu"}
+    cpu_baseline = None
+    if world == 1 and not args.no_cpu_baseline:
+        b, tc, desc = oracle_decode_sample(w, cpu, min(args.cpu_seconds, 10.0))
+        cpu_baseline = {"value": b / tc / 1e9, "unit": "GB/s", "cores": blas_threads(),
+                        "kind": "oracle", "sample": desc, "seconds": tc}
+    line = {
+        "metric": DECODE_METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) caches and new-token q/k/v, FP32 sinks)",
+        "config": decode_config(w, lens, kv_bytes),
+        "tokens_per_s": world * B * args.steps / (t_ms * 1e-3),
+        "roofline": roofline,
+        "kernels": {k: {"ms_per_launch": v[0] / v[1], "launches_profiled": v[1]}
+                    for k, v in kern.items() if v[1] > 0},
+        "gpu_launches": launches, "clocks": clk,
+        "e2e": {"value": world * kv_bytes * args.steps / (te_ms * 1e-3) / 1e9, "unit": "GB/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": te_ms / args.steps},
+        "cpu_baseline": cpu_baseline,
+    }
+    print(json.dumps(line), flush=True)
+    if pg is not None:
+        pg.destroy_process_group()
+
+
 def main(argv=None):
     args = parse_args(argv)
+    if args.workload in DECODE_WORKLOADS:
+        if args.impl == "reference":
+            run_reference_decode(args)
+        else:
+            run_decode(args)
+        return
     if args.impl == "reference":
         run_reference(args)
         return

@@ -165,3 +165,76 @@ def visible_pairs(doc_lens, window: int) -> int:
             # rows 0..W-1 see i+1 keys, the rest see W keys
             total += W * (W + 1) // 2 + (L - W) * W
     return total
+
+
+# ----------------------------------------------------------------------------
+# Decode over a KV cache (one new token per sequence)
+# ----------------------------------------------------------------------------
+
+@dataclasses.dataclass(frozen=True)
+class DecodeWorkload:
+    """B sequences, each with ``cache_lens[b]`` tokens cached and one new token.
+
+    The caches are [B, Hk, C, D] (head-major per sequence). Cached keys are
+    drawn as N(0, 1) rows: they stand for normalised keys, whose channels have
+    unit mean square before the norm weight.
+    """
+
+    name: str
+    batch: int
+    cache_capacity: int
+    num_q_heads: int
+    num_kv_heads: int
+    window: int
+    use_rope: bool
+    rope_theta: float
+    lens_range: tuple                  # cache_lens drawn uniformly in [lo, hi] inclusive
+    head_dim: int = 128
+    sink_std: float = 1.0
+    seed: int = 0
+
+
+# Serving shape of a sliding layer: 64 sequences with 4096-8191 cached tokens,
+# 4096-token window, 32/4 heads (the decode-step counterpart of the sliding
+# configurations above).
+DECODE_SLIDING_BF16 = DecodeWorkload(
+    name="decode_bf16_B64_C8192_H32x4_W4096", batch=64, cache_capacity=8192,
+    num_q_heads=32, num_kv_heads=4, window=4096, use_rope=True, rope_theta=1e6,
+    lens_range=(4096, 8191))
+
+
+def make_decode_inputs(w: DecodeWorkload, seed: Optional[int] = None, lens=None):
+    """Draw one decode step: cache_lens, q, k, v (new tokens), w_q, w_k, sink, caches.
+
+    Draw order: cache_lens (unless given), q, k, v, w_q, w_k, sink, k_cache,
+    v_cache. All draws are FP32 from one CPU generator, cast to bf16 (sinks
+    stay FP32, cache_lens int32).
+    """
+    gen = torch.Generator(device="cpu")
+    gen.manual_seed(w.seed if seed is None else seed)
+    B, C, H, Hk, D = w.batch, w.cache_capacity, w.num_q_heads, w.num_kv_heads, w.head_dim
+    if lens is None:
+        lo, hi = w.lens_range
+        lens = torch.randint(lo, hi + 1, (B,), generator=gen, dtype=torch.int64)
+    cache_lens = torch.as_tensor(list(lens), dtype=torch.int32)
+    bf = torch.bfloat16
+    out = {"cache_lens": cache_lens}
+    out["q"] = torch.randn(B, H, D, generator=gen, dtype=torch.float32).to(bf)
+    out["k"] = torch.randn(B, Hk, D, generator=gen, dtype=torch.float32).to(bf)
+    out["v"] = torch.randn(B, Hk, D, generator=gen, dtype=torch.float32).to(bf)
+    out["w_q"] = (1.0 + 0.1 * torch.randn(D, generator=gen, dtype=torch.float32)).to(bf)
+    out["w_k"] = (1.0 + 0.1 * torch.randn(D, generator=gen, dtype=torch.float32)).to(bf)
+    out["sink"] = w.sink_std * torch.randn(H, generator=gen, dtype=torch.float32)
+    out["k_cache"] = torch.randn(B, Hk, C, D, generator=gen, dtype=torch.float32).to(bf)
+    out["v_cache"] = torch.randn(B, Hk, C, D, generator=gen, dtype=torch.float32).to(bf)
+    return out
+
+
+def decode_kv_bytes(cache_lens, window: int, num_kv_heads: int, head_dim: int = 128) -> int:
+    """Bytes of K and V (bf16) the decode step reads: every visible slot, once."""
+    total = 0
+    for p in cache_lens:
+        p = int(p)
+        n = p + 1 if window <= 0 else min(p + 1, int(window))
+        total += n
+    return total * num_kv_heads * head_dim * 2 * 2

@@ -131,6 +131,58 @@ flint_status_t flint_attn_bwd(const flint_attn_params_t* params,
                               float* dq_norm_w, float* dk_norm_w, float* dsink,
                               void* workspace, size_t workspace_bytes, void* stream);
 
+/* ---- Decode over a KV cache ----------------------------------------------
+ * The forward of one NEW token per sequence, for serving (the pages mention
+ * serving kernels on the Flint layers page, module docstring, and a KV cache
+ * through use_cache on the Flint config page). It computes exactly what
+ * flint_attn_fwd computes for the last token of each sequence, with the earlier
+ * tokens' keys and values taken from caches instead of recomputed:
+ *   sequence b has cache_lens[b] = p tokens cached (positions 0..p-1); its new
+ *   token is at position p. q_hat = RoPE_p(RMSNorm(q)) and k_hat =
+ *   RoPE_p(RMSNorm(k)) as in the forward; k_hat and v are first written into
+ *   slot p of k_cache / v_cache (rounded to bf16), then the new query attends
+ *   to slots j with max(0, p - W + 1) <= j <= p (W <= 0: 0..p), plus the sink:
+ *   LSE = ln(e^{sink_h} + sum_j e^{z_j}), O = sum_j e^{z_j - LSE} v_j.
+ * Layouts: q [B, H, D]; k, v [B, Hk, D] (raw projections of the new token,
+ *   bfloat16); q_norm_w, k_norm_w [D] bf16; sink [H] fp32; cache_lens [B] int32
+ *   (device); k_cache, v_cache [B, Hk, C, D] bfloat16, head-major per sequence
+ *   (slot j of KV head g of sequence b at ((b * Hk + g) * C + j) * D); k_cache
+ *   holds normalised, rotated keys. out [B, H, D] (bf16, or float32 with
+ *   fp32_out); lse [B, H] fp32 (natural log).
+ * Only dtype FLINT_BF16 is supported (FLINT_ERR_UNSUPPORTED otherwise); H/Hk
+ *   must be <= 16. Slot p must exist (0 <= p < C): a sequence whose cache_lens
+ *   entry is out of range is skipped on the device (out and lse are left
+ *   untouched, nothing is written to its cache) and the status word records it;
+ *   flint_attn_check_status() then returns FLINT_ERR_INVALID_ARG.
+ * The caches are read and written in place; the call does not allocate.
+ * Asynchronous on `stream`. */
+typedef struct {
+  int32_t batch;            /* B >= 1 sequences, one new token each */
+  int32_t cache_capacity;   /* C >= 1 slots per (sequence, KV head) */
+  int32_t num_q_heads;      /* H */
+  int32_t num_kv_heads;     /* Hk; H % Hk == 0, H / Hk <= 16 */
+  int32_t head_dim;         /* D; must be 128 */
+  int32_t window;           /* > 0: keys p-W+1..p visible; <= 0: unbounded */
+  int32_t use_rope;         /* NeoX RoPE at position p */
+  float rope_theta;
+  float rms_eps;            /* 1e-6 in the Flint config */
+  float softmax_scale;      /* 0 => 1/sqrt(head_dim) */
+  flint_dtype_t dtype;      /* FLINT_BF16 */
+  int32_t fp32_out;         /* out in float32 instead of bf16 */
+} flint_decode_params_t;
+
+/* Bytes of device workspace flint_attn_decode needs (0 if the params are
+ * invalid). 256-byte aligned; not used after the call's kernels finish. */
+size_t flint_attn_decode_workspace_bytes(const flint_decode_params_t* params);
+
+flint_status_t flint_attn_decode(const flint_decode_params_t* params,
+                                 const void* q, const void* k, const void* v,
+                                 const void* q_norm_w, const void* k_norm_w,
+                                 const float* sink, const int32_t* cache_lens,
+                                 void* k_cache, void* v_cache,
+                                 void* out, float* lse,
+                                 void* workspace, size_t workspace_bytes, void* stream);
+
 /* Largest num_q_heads flint_attn_bwd_preprocess_static accepts. */
 #define FLINT_STATIC_MAX_HEADS 128
 
@@ -158,9 +210,11 @@ flint_status_t flint_attn_bwd_preprocess_static(const flint_attn_params_t* param
 
 /* Synchronises `stream`, reads and clears the device status word in
  * `workspace` (written by bounded device waits), and returns FLINT_OK or
- * FLINT_ERR_TIMEOUT. It returns FLINT_ERR_CUDA if the stream itself reports an
- * error, or if a backward kernel found its dynamic shared memory not 1024-byte
- * aligned and did no work (its tiles need that alignment; not expected). */
+ * FLINT_ERR_TIMEOUT (FLINT_ERR_INVALID_ARG for a flint_attn_decode workspace
+ * whose call met an out-of-range cache_lens entry). It returns FLINT_ERR_CUDA
+ * if the stream itself reports an error, or if a backward kernel found its
+ * dynamic shared memory not 1024-byte aligned and did no work (its tiles need
+ * that alignment; not expected). */
 flint_status_t flint_attn_check_status(void* workspace, void* stream);
 
 /* ---- Measurement aids (not needed to compute anything) --------------------

@@ -34,7 +34,8 @@ namespace {
 const char* const kKernelNames[kNumKernelIds] = {
     "prologue_rmsnorm_rope", "build_worklist", "attn_fwd_sm100", "attn_fwd_fp32",
     "bwd_preprocess", "reduce_rows", "attn_bwd_dkv_sm100", "attn_bwd_dq_sm100",
-    "attn_bwd_dq_fp32", "attn_bwd_dkv_fp32", "prologue_bwd", "convert_f16"};
+    "attn_bwd_dq_fp32", "attn_bwd_dkv_fp32", "prologue_bwd", "convert_f16",
+    "decode"};
 constexpr int kMaxSlots = 1 << 15;
 struct Prof {
   std::mutex mu;
@@ -308,6 +309,78 @@ extern "C" flint_status_t flint_attn_bwd(const flint_attn_params_t* params, cons
   return FLINT_OK;
 }
 
+// ------------------------------------------------------------------ decode
+namespace {
+struct DecodeLayout {
+  size_t status, counters, part_o, part_ml, total;   // status and counters are contiguous
+};
+size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
+
+flint_status_t resolve_decode(const flint_decode_params_t* d, DecodeLayout* L) {
+  if (!d) return FLINT_ERR_INVALID_ARG;
+  if (d->dtype != FLINT_BF16) return d->dtype == FLINT_FP32 ? FLINT_ERR_UNSUPPORTED
+                                                           : FLINT_ERR_INVALID_ARG;
+  if (d->head_dim != kHeadDim) return FLINT_ERR_UNSUPPORTED;
+  if (d->batch < 1 || d->cache_capacity < 1 || d->num_q_heads < 1 || d->num_kv_heads < 1 ||
+      d->num_q_heads % d->num_kv_heads != 0)
+    return FLINT_ERR_INVALID_ARG;
+  if (d->num_q_heads / d->num_kv_heads > 16) return FLINT_ERR_UNSUPPORTED;
+  if (!(d->rms_eps >= 0.f) || !(d->softmax_scale >= 0.f) ||
+      (d->use_rope && !(d->rope_theta > 0.f)))
+    return FLINT_ERR_INVALID_ARG;
+  const size_t B = d->batch, H = d->num_q_heads;
+  const size_t S = decode_splits(d->cache_capacity, d->window);
+  L->status = 0;
+  L->counters = 64 * sizeof(int);
+  L->part_o = round256(L->counters + B * d->num_kv_heads * sizeof(int));
+  L->part_ml = L->part_o + round256(B * H * S * kHeadDim * sizeof(float));
+  L->total = L->part_ml + round256(B * H * S * 2 * sizeof(float));
+  return FLINT_OK;
+}
+}  // namespace
+
+extern "C" size_t flint_attn_decode_workspace_bytes(const flint_decode_params_t* params) {
+  DecodeLayout L;
+  return resolve_decode(params, &L) == FLINT_OK ? L.total : 0;
+}
+
+extern "C" flint_status_t flint_attn_decode(const flint_decode_params_t* params, const void* q,
+                                            const void* k, const void* v, const void* q_norm_w,
+                                            const void* k_norm_w, const float* sink,
+                                            const int32_t* cache_lens, void* k_cache,
+                                            void* v_cache, void* out, float* lse,
+                                            void* workspace, size_t workspace_bytes,
+                                            void* stream) {
+  DecodeLayout L;
+  flint_status_t s = resolve_decode(params, &L);
+  if (s != FLINT_OK) return s;
+  const void* vec16[] = {q, k, v, q_norm_w, k_norm_w, k_cache, v_cache, out};
+  for (const void* ptr : vec16)
+    if (!ptr || !aligned(ptr, 16)) return FLINT_ERR_INVALID_ARG;
+  if (!sink || !aligned(sink, 4) || !cache_lens || !aligned(cache_lens, 4) || !lse ||
+      !aligned(lse, 4))
+    return FLINT_ERR_INVALID_ARG;
+  if (!workspace || !aligned(workspace, 256)) return FLINT_ERR_INVALID_ARG;
+  if (workspace_bytes < L.total) return FLINT_ERR_WORKSPACE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  int* status = at<int>(workspace, L.status);
+  FLINT_TRY(cudaMemsetAsync(status, 0, L.part_o, st));    // status word and split counters
+  DecodeLaunch D;
+  D.B = params->batch; D.C = params->cache_capacity;
+  D.H = params->num_q_heads; D.Hk = params->num_kv_heads;
+  D.W = params->window; D.rope = params->use_rope ? 1 : 0; D.out_f32 = params->fp32_out ? 1 : 0;
+  D.theta = params->rope_theta; D.eps = params->rms_eps;
+  D.scale = params->softmax_scale > 0.f ? params->softmax_scale
+                                        : 1.0f / sqrtf((float)kHeadDim);
+  D.q = q; D.k = k; D.v = v; D.wq = q_norm_w; D.wk = k_norm_w;
+  D.sink = sink; D.lens = cache_lens; D.kc = k_cache; D.vc = v_cache;
+  D.counters = at<int>(workspace, L.counters);
+  D.part_o = at<float>(workspace, L.part_o);
+  D.part_ml = at<float>(workspace, L.part_ml);
+  D.out = out; D.lse = lse; D.status = status;
+  return cuda_status(launch_decode(D, st));
+}
+
 extern "C" flint_status_t flint_attn_check_status(void* workspace, void* stream) {
   if (!workspace || !aligned(workspace, 256)) return FLINT_ERR_INVALID_ARG;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -319,7 +392,9 @@ extern "C" flint_status_t flint_attn_check_status(void* workspace, void* stream)
     const int zero = 0;
     if (cudaMemcpy(workspace, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
       return FLINT_ERR_CUDA;
-    return (host & flint::kStatusSmemAlign) ? FLINT_ERR_CUDA : FLINT_ERR_TIMEOUT;
+    if (host & flint::kStatusSmemAlign) return FLINT_ERR_CUDA;
+    if (host & flint::kStatusDecodeRange) return FLINT_ERR_INVALID_ARG;
+    return FLINT_ERR_TIMEOUT;
   }
   return FLINT_OK;
 }

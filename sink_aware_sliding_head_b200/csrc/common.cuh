@@ -22,6 +22,7 @@ enum : int {
   kStatusTimeoutBwdKV = 2,
   kStatusTimeoutBwdQ = 4,
   kStatusSmemAlign = 8,        // dynamic shared memory not 1024-byte aligned
+  kStatusDecodeRange = 16,     // a decode cache_lens entry outside [0, cache_capacity)
 };
 
 // Parameters after validation and defaulting.
@@ -154,7 +155,8 @@ __device__ __forceinline__ void store8(float* p, const float (&f)[8]) {
 // on the launching stream (see flint_attn_profile_* in the public header).
 enum KernelId {
   kKPrologue = 0, kKWorklist, kKFwdSm100, kKFwdFp32, kKBwdPre, kKReduce, kKBwdDkvSm100,
-  kKBwdDqSm100, kKBwdDqFp32, kKBwdDkvFp32, kKPrologueBwd, kKConvert, kNumKernelIds
+  kKBwdDqSm100, kKBwdDqFp32, kKBwdDkvFp32, kKPrologueBwd, kKConvert, kKDecode,
+  kNumKernelIds
 };
 struct ProfScope {
   int id;
@@ -173,6 +175,24 @@ cudaError_t launch_build_worklist(const int32_t* cu, const Resolved& p, int mode
 cudaError_t launch_prologue(const Resolved& p, const void* x, const void* w, void* y, int heads,
                             const int32_t* cu, cudaStream_t st, bool out_f16 = false);
 cudaError_t launch_convert_f16(const __nv_bfloat16* src, __half* dst, size_t n, cudaStream_t st);
+
+// Decode over a KV cache (decode.cu). Keys per split CTA of the window.
+constexpr int kChunkKeysDecode = 1024;
+struct DecodeLaunch {
+  int B, C, H, Hk, W, rope, out_f32;
+  float theta, eps, scale;
+  const void *q, *k, *v, *wq, *wk;
+  const float* sink;
+  const int32_t* lens;
+  void *kc, *vc;
+  int* counters;                    // workspace: [B * Hk], zeroed per call
+  float *part_o, *part_ml;          // workspace
+  void* out;
+  float* lse;
+  int* status;
+};
+int decode_splits(int C, int W);    // split CTAs per (sequence, KV head)
+cudaError_t launch_decode(const DecodeLaunch& L, cudaStream_t st);
 cudaError_t launch_attn_fwd_fp32(const Resolved& p, const float* qh, const float* kh,
                                  const float* v, const float* sink, const int32_t* cu, float* out,
                                  float* lse, cudaStream_t st);

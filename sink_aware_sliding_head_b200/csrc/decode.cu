@@ -1,0 +1,488 @@
+// decode.cu - flint_attn_decode: the forward of one new token per sequence
+// over a KV cache (serving).
+//
+// What it computes is flint_attn_fwd's definition restricted to the last row
+// of each sequence (Flint layers page, nemo_automodel.components.models.flint.
+// layers: FlintAttention.forward, causal attention with a zero-value sink
+// category; per-head RMSNorm then NeoX RoPE; Flint config page: the window
+// counts the current token). Sequence b has p = cache_lens[b] tokens cached;
+// the new token's normalised, rotated key and its value go into slot p, and
+// the new query attends to slots max(0, p - W + 1) .. p plus the sink.
+//
+// Decode is bound by HBM: every key costs 512 bytes of K and V and feeds only
+// the G query heads of its group. One kernel, grid (splits, Hk, B); each CTA
+// covers kChunkKeysDecode keys of one (sequence, KV head) window:
+//   * it normalises and rotates the G query rows of its group itself (RMSNorm
+//     + RoPE at position p, a warp per row, kept in fp32 and pre-scaled by
+//     softmax_scale * log2(e)); the CTA whose chunk holds slot p also computes
+//     k_hat and appends k_hat (rounded to bf16) and v to the caches before it
+//     stages them;
+//   * its 4 warps take 16-key steps, each staging its own K and V rows into
+//     shared memory with cp.async (double buffered, coalesced 16-byte copies
+//     of the head-major cache). The two small contractions run on mma.sync
+//     m16n8k16 (bf16 in, fp32 accumulate): S = Q K^T with the G heads as 16
+//     padded rows and q_hat split into bf16 hi + lo parts (two MMAs), and
+//     O += P V with P in bf16. Tensor throughput is not the limit here (16
+//     padded rows per 16 keys), so the per-SM tcgen05/TMEM machinery of the
+//     prefill kernels would add nothing; K fragments come from ldmatrix, V
+//     fragments from ldmatrix.trans, and P is the S accumulator re-packed in
+//     registers. Online softmax with a lazily rescaled running max;
+//   * the warps merge in shared memory and the CTA writes one unnormalised
+//     partial (m, l, O); the last CTA of the (sequence, KV head) to finish (an
+//     atomic counter per pair) folds the sink in once (m = sink, l = 1 before
+//     the partials), normalises and writes out and LSE.
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+#include "sm100_primitives.cuh"
+
+namespace flint {
+
+namespace {
+
+constexpr int kDecWarps = 4;
+constexpr int kDecThreads = 32 * kDecWarps;
+constexpr int kStepKeys = 16;                  // keys per warp step
+constexpr int kRowBytes = 2 * kHeadDim + 16;   // a key row + 16 B: ldmatrix rows hit distinct banks
+constexpr int kStageBytes = 2 * kStepKeys * kRowBytes;              // K and V rows of one step
+constexpr int kDecStages = 2;                                       // steps in flight per warp
+constexpr int kWarpSmem = kDecStages * kStageBytes;
+constexpr int kAttnSmem = kDecWarps * kWarpSmem;
+constexpr int kMergeBytes = kDecWarps * 16 * (kHeadDim + 2) * 4;    // per-warp m, l, O for merging
+static_assert(kMergeBytes <= kAttnSmem && 16 * kHeadDim * 4 <= kAttnSmem,
+              "merge area and q_hat rows must fit in the staging area");
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kRescale = 8.0f;               // log2 units
+
+struct DecArgs {
+  int B, C, H, Hk, G, W, rope, splits, out_f32;
+  float theta, eps, scale_log2;
+  const __nv_bfloat16 *q, *k, *v, *wq, *wk;
+  const float* sink;
+  const int* lens;
+  __nv_bfloat16 *kc, *vc;
+  int* counters;     // [B * Hk], zero at the start of a call
+  float* part_o;     // [B, H, splits, D]
+  float* part_ml;    // [B, H, splits, 2]
+  void* out;
+  float* lse;        // [B, H]
+  int* status;
+};
+
+__device__ __forceinline__ bool pos_ok(const DecArgs& a, int p) { return p >= 0 && p < a.C; }
+
+__device__ __forceinline__ int window_lo(const DecArgs& a, int p) {
+  return a.W > 0 ? max(0, p - a.W + 1) : 0;
+}
+
+// ---------------------------------------------------------------------------
+// Prologue of one row: RMSNorm with weight w, then NeoX RoPE from the table.
+// A warp owns the row, lane l channels 4l..4l+3; channel c's RoPE partner
+// c +- 64 is in lane l ^ 16.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void warp_row_prologue(const __nv_bfloat16* x, const __nv_bfloat16* w,
+                                                  const float* cs, const float* sn, bool rope,
+                                                  float eps, float (&y)[4]) {
+  const int lane = threadIdx.x & 31;
+  const uint2 xr = *reinterpret_cast<const uint2*>(x + 4 * lane);
+  const uint2 wr = *reinterpret_cast<const uint2*>(w + 4 * lane);
+  const __nv_bfloat162* xh = reinterpret_cast<const __nv_bfloat162*>(&xr);
+  const __nv_bfloat162* wh = reinterpret_cast<const __nv_bfloat162*>(&wr);
+  float xv[4], wv[4];
+  xv[0] = __low2float(xh[0]); xv[1] = __high2float(xh[0]);
+  xv[2] = __low2float(xh[1]); xv[3] = __high2float(xh[1]);
+  wv[0] = __low2float(wh[0]); wv[1] = __high2float(wh[0]);
+  wv[2] = __low2float(wh[1]); wv[3] = __high2float(wh[1]);
+  float ss = xv[0] * xv[0] + xv[1] * xv[1] + xv[2] * xv[2] + xv[3] * xv[3];
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  const float r = rsqrtf(ss * (1.0f / kHeadDim) + eps);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) y[e] = xv[e] * r * wv[e];
+  if (rope) {
+    const bool lo_half = lane < 16;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float partner = __shfl_xor_sync(0xffffffffu, y[e], 16);
+      const int j = (4 * lane + e) & (kHeadDim / 2 - 1);
+      y[e] = lo_half ? (y[e] * cs[j] - partner * sn[j]) : (y[e] * cs[j] + partner * sn[j]);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Split attention
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void mma_bf16_16816(float (&c)[4], uint32_t a0, uint32_t a1,
+                                               uint32_t a2, uint32_t a3, uint32_t b0,
+                                               uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
+      "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+// 16-byte global -> shared copy; src_bytes = 0 writes zeros (src still valid).
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, int src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+               "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ uint32_t bf16x2_bits(float lo, float hi) {
+  return pack_bf16x2(lo, hi);
+}
+__device__ __forceinline__ float bf16_round(float x) {
+  return __bfloat162float(__float2bfloat16_rn(x));
+}
+
+__global__ void __launch_bounds__(kDecThreads) decode_attn_kernel(const DecArgs a) {
+  extern __shared__ __align__(128) uint8_t dsmem[];
+  // q_hat rows of the group (log2 units): only until they are in registers, so
+  // they share the staging area
+  float (*qs)[kHeadDim] = reinterpret_cast<float (*)[kHeadDim]>(dsmem);
+  __shared__ float cs[kHeadDim / 2], sn[kHeadDim / 2];
+  __shared__ int last_flag;
+  const int s = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int p = __ldg(a.lens + b);
+  if (!pos_ok(a, p)) {
+    if (s == 0 && g == 0 && threadIdx.x == 0) atomicOr(a.status, kStatusDecodeRange);
+    return;
+  }
+  const int lo = window_lo(a, p);
+  const int k0 = lo + s * kChunkKeysDecode;
+  if (k0 > p) return;                                // this split has no keys
+  const int k1 = min(k0 + kChunkKeysDecode, p + 1);  // keys [k0, k1)
+  const int nsplit = (p - lo + kChunkKeysDecode) / kChunkKeysDecode;
+  const bool owner = k1 == p + 1;                    // this CTA reads slot p
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int gid = lane >> 2, tig = lane & 3;
+  const size_t row0 = ((size_t)b * a.Hk + g) * a.C;  // slot 0 of this (sequence, KV head)
+  const __nv_bfloat16* kbase = a.kc + row0 * kHeadDim;
+  const __nv_bfloat16* vbase = a.vc + row0 * kHeadDim;
+
+  // ---- prologue: RoPE table, the group's q_hat rows, and (owner) the append
+  if (a.rope && threadIdx.x < kHeadDim / 2) {
+    const int j = threadIdx.x;
+    double inv_freq = exp2(-(2.0 * j / kHeadDim) * log2((double)a.theta));
+    double ang = (double)p * inv_freq;
+    const double two_pi = 6.283185307179586476925286766559;
+    ang -= two_pi * rint(ang / two_pi);
+    float sv, cv;
+    sincosf((float)ang, &sv, &cv);
+    cs[j] = cv;
+    sn[j] = sv;
+  }
+  __syncthreads();
+  for (int r = warp; r < a.G; r += kDecWarps) {
+    float y[4];
+    warp_row_prologue(a.q + ((size_t)b * a.H + g * a.G + r) * kHeadDim, a.wq, cs, sn, a.rope,
+                      a.eps, y);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) qs[r][4 * lane + e] = y[e] * a.scale_log2;
+  }
+  if (owner && warp == kDecWarps - 1) {
+    float y[4];
+    const size_t src = ((size_t)b * a.Hk + g) * kHeadDim;
+    warp_row_prologue(a.k + src, a.wk, cs, sn, a.rope, a.eps, y);
+    uint2 kb;
+    kb.x = pack_bf16x2(y[0], y[1]);
+    kb.y = pack_bf16x2(y[2], y[3]);
+    const size_t dst = (row0 + p) * kHeadDim + 4 * lane;
+    *reinterpret_cast<uint2*>(a.kc + dst) = kb;
+    *reinterpret_cast<uint2*>(a.vc + dst) = *reinterpret_cast<const uint2*>(a.v + src + 4 * lane);
+  }
+  __threadfence_block();
+  __syncthreads();                                   // slot p written before it is staged
+
+  // q_hat fragments (rows = heads of the group, zero past G), bf16 hi + lo
+  uint32_t qa_hi[8][4], qa_lo[8][4];
+  {
+    const bool v0 = gid < a.G, v1 = gid + 8 < a.G;
+    const float* q0 = qs[gid];
+    const float* q1 = qs[gid + 8];
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) {
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        // a0: (row gid, k 2tig..+1), a1: (row gid+8, same), a2: (row gid, k+8), a3: (row gid+8, k+8)
+        const int d = kk * 16 + 2 * tig + ((r & 2) ? 8 : 0);
+        const bool hv = (r & 1) ? v1 : v0;
+        const float* qr = (r & 1) ? q1 : q0;
+        float x0 = 0.f, x1 = 0.f;
+        if (hv) {
+          const float2 t = *reinterpret_cast<const float2*>(qr + d);
+          x0 = t.x;
+          x1 = t.y;
+        }
+        const float h0f = bf16_round(x0), h1f = bf16_round(x1);
+        qa_hi[kk][r] = bf16x2_bits(h0f, h1f);
+        qa_lo[kk][r] = bf16x2_bits(x0 - h0f, x1 - h1f);
+      }
+    }
+  }
+
+  __syncthreads();                                   // every warp holds its fragments
+  const uint32_t wsm = smem_u32(dsmem) + warp * kWarpSmem;
+  const int nsteps = (k1 - k0 + kStepKeys - 1) / kStepKeys;
+  auto issue = [&](int step, int buf) {              // stage K and V rows of a step
+    const int kb = k0 + step * kStepKeys;
+    const uint32_t ks = wsm + buf * kStageBytes, vs = ks + kStepKeys * kRowBytes;
+#pragma unroll
+    for (int i = 0; i < (kStepKeys * 16) / 32; ++i) {
+      const int c = lane + 32 * i;                   // 16-byte chunk of the step
+      const int key = c >> 4, part = c & 15;
+      const int j = kb + key;
+      const bool in = j < k1;
+      const size_t off = (size_t)(in ? j : k0) * kHeadDim + part * 8;
+      cp_async16(ks + key * kRowBytes + part * 16, kbase + off, in ? 16 : 0);
+      cp_async16(vs + key * kRowBytes + part * 16, vbase + off, in ? 16 : 0);
+    }
+  };
+
+  float o[16][4];
+#pragma unroll
+  for (int n = 0; n < 16; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;   // rows gid, gid + 8
+
+  // Each iteration commits one group (empty past the last step), so the wait
+  // count below is constant: the group of the step being computed is done.
+#pragma unroll
+  for (int j = 0; j < kDecStages - 1; ++j) {
+    if (warp + kDecWarps * j < nsteps) issue(warp + kDecWarps * j, j);
+    cp_async_commit();
+  }
+  int it = 0;
+  for (int step = warp; step < nsteps; step += kDecWarps, ++it) {
+    const int buf = it % kDecStages;
+    const int ahead = step + kDecWarps * (kDecStages - 1);
+    if (ahead < nsteps) issue(ahead, (it + kDecStages - 1) % kDecStages);
+    cp_async_commit();
+    cp_async_wait<kDecStages - 1>();
+    __syncwarp();
+    const uint32_t ks = wsm + buf * kStageBytes, vs = ks + kStepKeys * kRowBytes;
+    const int kb = k0 + step * kStepKeys;
+
+    // S = q_hat K^T for keys kb .. kb+15 (two 8-key n-tiles)
+    float sc[2][4];
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+      sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
+#pragma unroll
+      for (int kp = 0; kp < 4; ++kp) {               // pairs of 16-dim k-steps
+        uint32_t bk[4];
+        const int key = nt * 8 + (lane & 7);
+        const int col = kp * 32 + (lane >> 3) * 8;   // dims
+        ldsm_x4(ks + key * kRowBytes + col * 2, bk);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int kk = 2 * kp + h;
+          mma_bf16_16816(sc[nt], qa_hi[kk][0], qa_hi[kk][1], qa_hi[kk][2], qa_hi[kk][3],
+                         bk[2 * h], bk[2 * h + 1]);
+          mma_bf16_16816(sc[nt], qa_lo[kk][0], qa_lo[kk][1], qa_lo[kk][2], qa_lo[kk][3],
+                         bk[2 * h], bk[2 * h + 1]);
+        }
+      }
+    }
+    // mask keys past the end of the range; c0,c1 = row gid, c2,c3 = row gid + 8
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+      const int j = kb + nt * 8 + 2 * tig;
+      if (j >= k1) sc[nt][0] = sc[nt][2] = -INFINITY;
+      if (j + 1 >= k1) sc[nt][1] = sc[nt][3] = -INFINITY;
+    }
+    float mx0 = fmaxf(fmaxf(sc[0][0], sc[0][1]), fmaxf(sc[1][0], sc[1][1]));
+    float mx1 = fmaxf(fmaxf(sc[0][2], sc[0][3]), fmaxf(sc[1][2], sc[1][3]));
+    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+    // lazy rescale: the running max moves only when it grows by more than 2^8
+    if (mx0 > m0 + kRescale || m0 == -INFINITY) {
+      const float alpha = (m0 == -INFINITY) ? 0.f : exp2f(m0 - mx0);
+      m0 = mx0;
+      l0 *= alpha;
+#pragma unroll
+      for (int n = 0; n < 16; ++n) { o[n][0] *= alpha; o[n][1] *= alpha; }
+    }
+    if (mx1 > m1 + kRescale || m1 == -INFINITY) {
+      const float alpha = (m1 == -INFINITY) ? 0.f : exp2f(m1 - mx1);
+      m1 = mx1;
+      l1 *= alpha;
+#pragma unroll
+      for (int n = 0; n < 16; ++n) { o[n][2] *= alpha; o[n][3] *= alpha; }
+    }
+    const float mb0 = (m0 == -INFINITY) ? 0.f : m0, mb1 = (m1 == -INFINITY) ? 0.f : m1;
+    float pr[2][4];
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+      pr[nt][0] = ex2_approx(sc[nt][0] - mb0);
+      pr[nt][1] = ex2_approx(sc[nt][1] - mb0);
+      pr[nt][2] = ex2_approx(sc[nt][2] - mb1);
+      pr[nt][3] = ex2_approx(sc[nt][3] - mb1);
+    }
+    // P in bf16 as the A fragment of P V (rows gid / gid+8, keys 2tig.. / 8+2tig..);
+    // the row sums use the same rounded values
+    const uint32_t pa0 = bf16x2_bits(pr[0][0], pr[0][1]);
+    const uint32_t pa1 = bf16x2_bits(pr[0][2], pr[0][3]);
+    const uint32_t pa2 = bf16x2_bits(pr[1][0], pr[1][1]);
+    const uint32_t pa3 = bf16x2_bits(pr[1][2], pr[1][3]);
+    l0 += bf16_round(pr[0][0]) + bf16_round(pr[0][1]) + bf16_round(pr[1][0]) +
+          bf16_round(pr[1][1]);
+    l1 += bf16_round(pr[0][2]) + bf16_round(pr[0][3]) + bf16_round(pr[1][2]) +
+          bf16_round(pr[1][3]);
+    // O += P V: 16 n-tiles of 8 dims, V fragments by ldmatrix.trans
+#pragma unroll
+    for (int np = 0; np < 8; ++np) {                 // pairs of n-tiles
+      uint32_t bv[4];
+      const int key = (lane & 7) + ((lane >> 3) & 1) * 8;
+      const int col = np * 16 + (lane >> 4) * 8;
+      ldsm_x4_t(vs + key * kRowBytes + col * 2, bv);
+      mma_bf16_16816(o[2 * np], pa0, pa1, pa2, pa3, bv[0], bv[1]);
+      mma_bf16_16816(o[2 * np + 1], pa0, pa1, pa2, pa3, bv[2], bv[3]);
+    }
+    __syncwarp();                                    // buffer reusable by a later step
+  }
+  cp_async_wait<0>();                                // only empty groups remain
+  // row sums over the quad
+  l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
+  l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
+  l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+  l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+
+  // merge the warps: per warp [16 rows][m, l, O(128)]
+  __syncthreads();
+  float* ms = reinterpret_cast<float*>(dsmem);
+  float* wrow = ms + (size_t)warp * 16 * (kHeadDim + 2);
+  {
+    float* r0 = wrow + gid * (kHeadDim + 2);
+    float* r1 = wrow + (gid + 8) * (kHeadDim + 2);
+    if (tig == 0) {
+      r0[0] = m0; r0[1] = l0;
+      r1[0] = m1; r1[1] = l1;
+    }
+#pragma unroll
+    for (int n = 0; n < 16; ++n) {                   // C layout: cols 2tig, 2tig+1 of tile n
+      r0[2 + n * 8 + 2 * tig] = o[n][0];
+      r0[2 + n * 8 + 2 * tig + 1] = o[n][1];
+      r1[2 + n * 8 + 2 * tig] = o[n][2];
+      r1[2 + n * 8 + 2 * tig + 1] = o[n][3];
+    }
+  }
+  __syncthreads();
+  const int nw = min(kDecWarps, nsteps);             // warps that saw keys
+  for (int e = threadIdx.x; e < a.G * kHeadDim; e += kDecThreads) {
+    const int r = e / kHeadDim, d = e % kHeadDim;
+    float M = -INFINITY;
+    for (int w = 0; w < nw; ++w) M = fmaxf(M, ms[((size_t)w * 16 + r) * (kHeadDim + 2)]);
+    float L = 0.f, O = 0.f;
+    for (int w = 0; w < nw; ++w) {
+      const float* wr = ms + ((size_t)w * 16 + r) * (kHeadDim + 2);
+      const float f = (wr[0] == -INFINITY) ? 0.f : exp2f(wr[0] - M);
+      L += wr[1] * f;
+      O += wr[2 + d] * f;
+    }
+    const int h = g * a.G + r;
+    const size_t pi = ((size_t)b * a.H + h) * a.splits + s;
+    a.part_o[pi * kHeadDim + d] = O;
+    if (d == 0) {
+      a.part_ml[2 * pi] = M;
+      a.part_ml[2 * pi + 1] = L;
+    }
+  }
+
+  // ---- the last CTA of this (sequence, KV head) combines the splits and the sink
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0)
+    last_flag = atomicAdd(a.counters + (size_t)b * a.Hk + g, 1) == nsplit - 1;
+  __syncthreads();
+  if (!last_flag) return;
+  __threadfence();
+  for (int r = warp; r < a.G; r += kDecWarps) {
+    const int h = g * a.G + r;
+    const size_t pb = ((size_t)b * a.H + h) * a.splits;
+    const float s2 = __ldg(a.sink + h) * kLog2e;      // the sink's logit, log2 units
+    float M = s2;
+    for (int i = 0; i < nsplit; ++i) M = fmaxf(M, __ldcg(a.part_ml + 2 * (pb + i)));
+    float L = exp2f(s2 - M);                         // the sink's own weight
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int i = 0; i < nsplit; ++i) {
+      const float mi = __ldcg(a.part_ml + 2 * (pb + i));
+      const float f = (mi == -INFINITY) ? 0.f : exp2f(mi - M);
+      L += __ldcg(a.part_ml + 2 * (pb + i) + 1) * f;
+      const float4 v = __ldcg(reinterpret_cast<const float4*>(a.part_o + (pb + i) * kHeadDim) +
+                              lane);
+      acc[0] += v.x * f; acc[1] += v.y * f; acc[2] += v.z * f; acc[3] += v.w * f;
+    }
+    const float inv = 1.f / L;
+    const size_t ob = ((size_t)b * a.H + h) * kHeadDim + lane * 4;
+    if (a.out_f32) {
+      *reinterpret_cast<float4*>(reinterpret_cast<float*>(a.out) + ob) =
+          make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
+    } else {
+      uint2 pk;
+      pk.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
+      pk.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
+      *reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(a.out) + ob) = pk;
+    }
+    if (lane == 0) a.lse[(size_t)b * a.H + h] = (M + log2f(L)) * kLn2;
+  }
+  if (threadIdx.x == 0) a.counters[(size_t)b * a.Hk + g] = 0;   // ready for the next call
+}
+
+}  // namespace
+
+int decode_splits(int C, int W) {
+  const int maxkeys = (W > 0) ? (W < C ? W : C) : C;
+  return (maxkeys + kChunkKeysDecode - 1) / kChunkKeysDecode;
+}
+
+cudaError_t launch_decode(const DecodeLaunch& L, cudaStream_t st) {
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(decode_attn_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kAttnSmem);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  DecArgs a;
+  a.B = L.B; a.C = L.C; a.H = L.H; a.Hk = L.Hk; a.G = L.H / L.Hk; a.W = L.W;
+  a.rope = L.rope; a.theta = L.theta; a.eps = L.eps;
+  a.scale_log2 = L.scale * kLog2e;
+  a.splits = decode_splits(L.C, L.W);
+  a.out_f32 = L.out_f32;
+  a.q = static_cast<const __nv_bfloat16*>(L.q);
+  a.k = static_cast<const __nv_bfloat16*>(L.k);
+  a.v = static_cast<const __nv_bfloat16*>(L.v);
+  a.wq = static_cast<const __nv_bfloat16*>(L.wq);
+  a.wk = static_cast<const __nv_bfloat16*>(L.wk);
+  a.sink = L.sink;
+  a.lens = L.lens;
+  a.kc = static_cast<__nv_bfloat16*>(L.kc);
+  a.vc = static_cast<__nv_bfloat16*>(L.vc);
+  a.counters = L.counters; a.part_o = L.part_o; a.part_ml = L.part_ml;
+  a.out = L.out; a.lse = L.lse; a.status = L.status;
+  ProfScope prof(kKDecode, st);
+  decode_attn_kernel<<<dim3(a.splits, a.Hk, a.B), kDecThreads, kAttnSmem, st>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace flint

@@ -28,7 +28,8 @@ EXPORTED = ["flint_attn_workspace_bytes", "flint_attn_fwd", "flint_attn_bwd",
             "flint_attn_check_status", "flint_status_string", "flint_attn_version",
             "flint_attn_profile_enable", "flint_attn_profile_collect",
             "flint_attn_profile_reset", "flint_attn_launch_count",
-            "flint_attn_bwd_preprocess_static", "flint_attn_exp2_poly"]
+            "flint_attn_bwd_preprocess_static", "flint_attn_exp2_poly",
+            "flint_attn_decode_workspace_bytes", "flint_attn_decode"]
 
 
 class Params(ctypes.Structure):
@@ -36,6 +37,24 @@ class Params(ctypes.Structure):
     _fields_ = [
         ("total_tokens", ctypes.c_int32),
         ("num_docs", ctypes.c_int32),
+        ("num_q_heads", ctypes.c_int32),
+        ("num_kv_heads", ctypes.c_int32),
+        ("head_dim", ctypes.c_int32),
+        ("window", ctypes.c_int32),
+        ("use_rope", ctypes.c_int32),
+        ("rope_theta", ctypes.c_float),
+        ("rms_eps", ctypes.c_float),
+        ("softmax_scale", ctypes.c_float),
+        ("dtype", ctypes.c_int32),
+        ("fp32_out", ctypes.c_int32),
+    ]
+
+
+class DecodeParams(ctypes.Structure):
+    """Mirror of ``flint_decode_params_t``."""
+    _fields_ = [
+        ("batch", ctypes.c_int32),
+        ("cache_capacity", ctypes.c_int32),
         ("num_q_heads", ctypes.c_int32),
         ("num_kv_heads", ctypes.c_int32),
         ("head_dim", ctypes.c_int32),
@@ -95,6 +114,11 @@ def load_library(path: str = LIB_PATH):
     lib.flint_attn_bwd_preprocess_static.restype = ctypes.c_int
     lib.flint_attn_exp2_poly.argtypes = [vp, vp, ctypes.c_int32, vp]
     lib.flint_attn_exp2_poly.restype = ctypes.c_int
+    DP = ctypes.POINTER(DecodeParams)
+    lib.flint_attn_decode_workspace_bytes.argtypes = [DP]
+    lib.flint_attn_decode_workspace_bytes.restype = sz
+    lib.flint_attn_decode.argtypes = [DP] + [vp] * 11 + [vp, sz, vp]
+    lib.flint_attn_decode.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -259,6 +283,50 @@ def bwd_preprocess_static(out, dout, lse, sink, fp32_out=False, d_rowsum=None, d
                                                 _stream_ptr(stream))
     _check(code, "flint_attn_bwd_preprocess_static")
     return d_rowsum, dsink
+
+
+def decode_params(batch, cache_capacity, num_q_heads, num_kv_heads, window, use_rope,
+                  rope_theta, rms_eps=1e-6, softmax_scale=0.0, fp32_out=False,
+                  head_dim=128) -> DecodeParams:
+    return DecodeParams(int(batch), int(cache_capacity), int(num_q_heads), int(num_kv_heads),
+                        int(head_dim), int(window), 1 if use_rope else 0, float(rope_theta),
+                        float(rms_eps), float(softmax_scale), FLINT_BF16,
+                        1 if fp32_out else 0)
+
+
+def decode(q, k, v, q_norm_w, k_norm_w, sink, cache_lens, k_cache, v_cache, window, use_rope,
+           rope_theta, rms_eps=1e-6, softmax_scale=0.0, out=None, lse=None, workspace=None,
+           stream=None, check_status=False, fp32_out=False):
+    """One new token per sequence through ``flint_attn_decode``.
+
+    q [B,H,D], k, v [B,Hk,D] bf16 (raw projections of the new tokens); cache_lens
+    [B] int32 on the device; k_cache, v_cache [B,Hk,C,D] bf16, updated in place
+    at slot cache_lens[b]. Returns (out [B,H,D], lse [B,H] fp32).
+    """
+    lib = load_library()
+    B, H, D = q.shape
+    Hk, C = k_cache.shape[1], k_cache.shape[2]
+    p = decode_params(B, C, H, Hk, window, use_rope, rope_theta, rms_eps, softmax_scale,
+                      fp32_out, D)
+    if out is None:
+        out = torch.empty(q.shape, dtype=torch.float32 if fp32_out else q.dtype,
+                          device=q.device)
+    if lse is None:
+        lse = torch.empty(B, H, dtype=torch.float32, device=q.device)
+    if workspace is None:
+        n = lib.flint_attn_decode_workspace_bytes(ctypes.byref(p))
+        if n == 0:
+            raise FlintError(1, "flint_attn_decode_workspace_bytes")
+        workspace = torch.empty(n, dtype=torch.uint8, device=q.device)
+    st = _stream_ptr(stream)
+    code = lib.flint_attn_decode(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(q_norm_w),
+                                 _ptr(k_norm_w), _ptr(sink), _ptr(cache_lens), _ptr(k_cache),
+                                 _ptr(v_cache), _ptr(out), _ptr(lse), _ptr(workspace),
+                                 workspace.numel(), st)
+    _check(code, "flint_attn_decode")
+    if check_status:
+        _check(lib.flint_attn_check_status(_ptr(workspace), st), "flint_attn_decode (device)")
+    return out, lse
 
 
 def exp2_poly(x: torch.Tensor) -> torch.Tensor:

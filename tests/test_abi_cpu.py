@@ -82,3 +82,25 @@ def test_fp32_any_group_size_is_accepted_by_validation(lib):
     # FP32 runs on CUDA cores and takes any H/Hk; only workspace sizing is checked here
     assert fa.workspace_bytes(params(num_q_heads=12, num_kv_heads=1, dtype=fa.FLINT_FP32),
                               False) > 0
+
+
+def test_decode_validation(lib):
+    """flint_attn_decode's workspace size and argument errors, without a GPU."""
+    ok = fa.decode_params(64, 8192, 32, 4, 4096, True, 1e6)
+    n = lib.flint_attn_decode_workspace_bytes(ctypes.byref(ok))
+    # status, split counters and per-split partials (4 splits of 1024 keys for W = 4096)
+    assert n >= 64 * 32 * (128 + 2) * 4 * 4 and n % 256 == 0
+    bad = [fa.decode_params(64, 8192, 32, 4, 4096, True, 1e6, head_dim=64),   # D != 128
+           fa.decode_params(4, 64, 34, 1, 0, False, 1e4),                       # G = 34
+           fa.decode_params(4, 64, 32, 5, 0, False, 1e4),                       # H % Hk
+           fa.decode_params(0, 64, 32, 4, 0, False, 1e4)]                       # B = 0
+    for p in bad:
+        assert lib.flint_attn_decode_workspace_bytes(ctypes.byref(p)) == 0
+    p32 = fa.decode_params(4, 64, 32, 4, 0, False, 1e4)
+    p32.dtype = fa.FLINT_FP32
+    assert lib.flint_attn_decode_workspace_bytes(ctypes.byref(p32)) == 0
+    nul = ctypes.c_void_p(0)
+    code = lib.flint_attn_decode(ctypes.byref(p32), *([nul] * 11), nul, 0, nul)
+    assert code == 2                                     # FLINT_ERR_UNSUPPORTED
+    code = lib.flint_attn_decode(ctypes.byref(ok), *([nul] * 11), nul, 0, nul)
+    assert code == 1                                     # null pointers, before any launch
