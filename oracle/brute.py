@@ -43,8 +43,13 @@ def _norm_rope_row(x, w, pos, use_rope, theta, eps):
 
 
 def forward(q, k, v, w_q, w_k, sink, cu_doc_lens, window, use_rope, theta,
-            eps=1e-6, scale=None):
-    """q [T][H][D], k/v [T][Hk][D] nested lists (or arrays); returns O [T][H][D], LSE [H][T]."""
+            eps=1e-6, scale=None, valid_lens=None):
+    """q [T][H][D], k/v [T][Hk][D] nested lists (or arrays); returns O [T][H][D], LSE [H][T].
+
+    valid_lens[d] (optional): document d's first valid_lens[d] tokens are real,
+    the rest are padding - excluded as keys, and as queries they see no key, so
+    only the sink remains (O = 0, LSE = the sink logit).
+    """
     T = len(q)
     H = len(q[0])
     Hk = len(k[0])
@@ -53,9 +58,12 @@ def forward(q, k, v, w_q, w_k, sink, cu_doc_lens, window, use_rope, theta,
     scale = 1.0 / math.sqrt(D) if scale is None else scale
     cu = [int(c) for c in cu_doc_lens]
     doc_start = [0] * T
+    doc_valid = [0] * T                 # first padded token of the token's document
     for d in range(len(cu) - 1):
+        n = cu[d + 1] - cu[d] if valid_lens is None else min(int(valid_lens[d]), cu[d + 1] - cu[d])
         for t in range(cu[d], cu[d + 1]):
             doc_start[t] = cu[d]
+            doc_valid[t] = cu[d] + n
     kh = [[_norm_rope_row([float(a) for a in k[t][g]], [float(a) for a in w_k],
                           t - doc_start[t], use_rope, theta, eps) for g in range(Hk)]
           for t in range(T)]
@@ -67,7 +75,10 @@ def forward(q, k, v, w_q, w_k, sink, cu_doc_lens, window, use_rope, theta,
             g = h // G
             qh = _norm_rope_row([float(a) for a in q[i][h]], [float(a) for a in w_q],
                                 i - d0, use_rope, theta, eps)
-            keys = [j for j in range(d0, i + 1) if window <= 0 or i - j < window]
+            keys = [j for j in range(d0, i + 1)
+                    if (window <= 0 or i - j < window) and j < doc_valid[i]]
+            if i >= doc_valid[i]:
+                keys = []                   # a padded query sees no key
             logits = []
             for j in range(len(keys)):
                 dot = 0.0

@@ -284,6 +284,68 @@ def flint_attn_bwd(q, k, v, w_q, w_k, sink, cu_doc_lens, window, use_rope,
 
 
 # ----------------------------------------------------------------------------
+# Padding (attention utils page: a BSHD attention_mask; TE takes trailing
+# padding only): document d holds valid_lens[d] real tokens followed by padding
+# ----------------------------------------------------------------------------
+
+def _valid_tokens(cu, valid_lens):
+    """Indices of the real tokens and the cu_doc_lens of the documents they form."""
+    idx, cu_v = [], [0]
+    for d, (a, b) in enumerate(doc_bounds(cu)):
+        n = max(0, min(int(valid_lens[d]), b - a))
+        idx.extend(range(a, a + n))
+        cu_v.append(cu_v[-1] + n)
+    return np.asarray(idx, dtype=np.int64), np.asarray(cu_v, dtype=np.int64)
+
+
+def flint_attn_fwd_padded(q, k, v, w_q, w_k, sink, cu_doc_lens, valid_lens, window, use_rope,
+                          rope_theta, eps=1e-6, scale=None):
+    """Forward with trailing padding in every document.
+
+    Padded tokens are excluded as keys; a padded query sees no key, so its row
+    is the sink alone: O = 0 and LSE = sink_h (the sink stays valid). Padding is
+    trailing, so a real token keeps its position and its visible keys, and the
+    real rows are exactly the layer over the documents' real prefixes.
+    """
+    q, k, v, sink = map(_f64, (q, k, v, sink))
+    cu = np.asarray(_f64(cu_doc_lens), dtype=np.int64)
+    idx, cu_v = _valid_tokens(cu, _f64(valid_lens))
+    T, H, D = q.shape
+    O = np.zeros((T, H, D))
+    lse = np.repeat(sink[:, None], T, axis=1)
+    if len(idx):
+        O_v, lse_v = flint_attn_fwd(q[idx], k[idx], v[idx], w_q, w_k, sink, cu_v, window,
+                                    use_rope, rope_theta, eps, scale)
+        O[idx] = O_v
+        lse[:, idx] = lse_v
+    return O, lse
+
+
+def flint_attn_bwd_padded(q, k, v, w_q, w_k, sink, cu_doc_lens, valid_lens, window, use_rope,
+                          rope_theta, dO, eps=1e-6, scale=None):
+    """Gradients of sum(dO * O) for ``flint_attn_fwd_padded``.
+
+    Padded rows of O are constant, so every gradient at a padded token is zero
+    and padded rows add nothing to d_sink (their D = dO . O is 0) or to the
+    norm-weight gradients.
+    """
+    q, k, v, dO = map(_f64, (q, k, v, dO))
+    cu = np.asarray(_f64(cu_doc_lens), dtype=np.int64)
+    idx, cu_v = _valid_tokens(cu, _f64(valid_lens))
+    D = q.shape[-1]
+    out = {"dq": np.zeros(q.shape), "dk": np.zeros(k.shape), "dv": np.zeros(v.shape),
+           "dw_q": np.zeros(D), "dw_k": np.zeros(D), "dsink": np.zeros(len(_f64(sink)))}
+    if len(idx):
+        g = flint_attn_bwd(q[idx], k[idx], v[idx], w_q, w_k, sink, cu_v, window, use_rope,
+                           rope_theta, dO[idx], eps, scale)
+        for name in ("dq", "dk", "dv"):
+            out[name][idx] = g[name]
+        for name in ("dw_q", "dw_k", "dsink"):
+            out[name] = g[name]
+    return out
+
+
+# ----------------------------------------------------------------------------
 # Sampled rows, for sizes where the whole layer is too slow on a CPU
 # ----------------------------------------------------------------------------
 

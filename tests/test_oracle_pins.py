@@ -423,3 +423,54 @@ def test_decode_window_one_closed_form():
             ps = math.exp(sink[h]) / (math.exp(sink[h]) + math.exp(z))
             np.testing.assert_allclose(out[b, h], (1 - ps) * v[b, 0], rtol=0, atol=1e-12)
             assert abs(lse[b, h] - math.log(math.exp(sink[h]) + math.exp(z))) < 1e-12
+
+
+# ----------------------------------------------------------------------------
+# Padding (trailing padding in every document; BSHD is cu = [0, S, 2S, ...])
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("lens,valid,H,Hk,D,window,rope", [
+    ([10, 10, 10], [10, 4, 0], 4, 2, 8, 0, True),      # BSHD, S = 10
+    ([7, 12, 5], [3, 12, 1], 2, 1, 8, 3, True),         # THD with per-document padding
+    ([16], [9], 4, 4, 8, 1, False),
+])
+def test_padded_matches_bruteforce(lens, valid, H, Hk, D, window, rope):
+    q, k, v, wq, wk, sink, cu, _ = rand_case(lens, H, Hk, D, seed=sum(valid) + D)
+    O, lse = fo.flint_attn_fwd_padded(q, k, v, wq, wk, sink, cu, valid, window, rope, 1e4)
+    Ob, lseb = brute.forward(q, k, v, wq, wk, sink, cu, window, rope, 1e4, valid_lens=valid)
+    np.testing.assert_allclose(O, np.array(Ob), atol=1e-12, rtol=0)
+    np.testing.assert_allclose(lse, np.array(lseb), atol=1e-12, rtol=0)
+    # padded rows: the sink alone
+    for d, (a, b) in enumerate(zip(cu[:-1], cu[1:])):
+        for t in range(a + valid[d], b):
+            assert np.all(O[t] == 0.0)
+            np.testing.assert_array_equal(lse[:, t], sink)
+
+
+def test_padded_backward_finite_differences():
+    """Gradients of the padded layer, including zeros at every padded token."""
+    lens, valid, H, Hk, D = [6, 5], [4, 2], 2, 1, 8
+    q, k, v, wq, wk, sink, cu, dO = rand_case(lens, H, Hk, D, seed=2)
+    g = fo.flint_attn_bwd_padded(q, k, v, wq, wk, sink, cu, valid, 3, True, 1e4, dO)
+
+    def loss(q_, k_, v_, wq_, wk_, s_):
+        O, _ = fo.flint_attn_fwd_padded(q_, k_, v_, wq_, wk_, s_, cu, valid, 3, True, 1e4)
+        return float(np.sum(O * dO))
+
+    args = [q, k, v, wq, wk, sink]
+    names = ["dq", "dk", "dv", "dw_q", "dw_k", "dsink"]
+    h = 1e-6
+    for ai, name in enumerate(names):
+        x = args[ai]
+        fd = np.zeros_like(x)
+        it = np.nditer(x, flags=["multi_index"])
+        for _ in it:
+            i = it.multi_index
+            xp = x.copy(); xp[i] += h
+            xm = x.copy(); xm[i] -= h
+            ap = list(args); ap[ai] = xp
+            am = list(args); am[ai] = xm
+            fd[i] = (loss(*ap) - loss(*am)) / (2 * h)
+        np.testing.assert_allclose(g[name], fd, rtol=1e-6, atol=1e-8)
+    for t in (4, 5, 6 + 2, 6 + 3, 6 + 4):                # padded tokens
+        assert np.all(g["dq"][t] == 0) and np.all(g["dk"][t] == 0) and np.all(g["dv"][t] == 0)
