@@ -131,6 +131,38 @@ flint_status_t flint_attn_bwd(const flint_attn_params_t* params,
                               float* dq_norm_w, float* dk_norm_w, float* dsink,
                               void* workspace, size_t workspace_bytes, void* stream);
 
+/* ---- Padding ------------------------------------------------------------
+ * flint_attn_fwd / flint_attn_bwd with trailing padding in every document: a
+ * BSHD attention_mask as the attention utils page
+ * (nemo_automodel.components.attention.utils) hands it to TE, which takes
+ * trailing padding only. BSHD [B, S] is cu_doc_lens = [0, S, 2S, ..., B*S].
+ *   valid_lens [num_docs] int32 (device): document d's first valid_lens[d]
+ *   tokens are real (clamped to [0, length]); the rest are padding.
+ * Padded queries and keys are excluded while the sink stays valid (Flint
+ * layers page, FlintAttention.forward): a padded row gets out = 0 and
+ * lse = sink_h; real rows see only real keys; every gradient row at a padded
+ * token (dq, dk, dv) is zero, and padded rows add nothing to dsink or the
+ * norm-weight gradients. RoPE positions still count from the document start,
+ * so real tokens are unaffected by the padding after them. Same workspace as
+ * the unpadded calls; dtype FLINT_BF16 only (FLINT_ERR_UNSUPPORTED for
+ * FLINT_FP32). Other arguments as in flint_attn_fwd / flint_attn_bwd. */
+flint_status_t flint_attn_fwd_padded(const flint_attn_params_t* params,
+                                     const void* q, const void* k, const void* v,
+                                     const void* q_norm_w, const void* k_norm_w,
+                                     const float* sink, const int32_t* cu_doc_lens,
+                                     const int32_t* valid_lens, void* out, float* lse,
+                                     void* workspace, size_t workspace_bytes, void* stream);
+
+flint_status_t flint_attn_bwd_padded(const flint_attn_params_t* params,
+                                     const void* q, const void* k, const void* v,
+                                     const void* q_norm_w, const void* k_norm_w,
+                                     const float* sink, const int32_t* cu_doc_lens,
+                                     const int32_t* valid_lens, const void* out,
+                                     const float* lse, const void* dout,
+                                     void* dq, void* dk, void* dv,
+                                     float* dq_norm_w, float* dk_norm_w, float* dsink,
+                                     void* workspace, size_t workspace_bytes, void* stream);
+
 /* ---- Decode over a KV cache ----------------------------------------------
  * The forward of one NEW token per sequence, for serving (the pages mention
  * serving kernels on the Flint layers page, module docstring, and a KV cache

@@ -35,7 +35,7 @@ const char* const kKernelNames[kNumKernelIds] = {
     "prologue_rmsnorm_rope", "build_worklist", "attn_fwd_sm100", "attn_fwd_fp32",
     "bwd_preprocess", "reduce_rows", "attn_bwd_dkv_sm100", "attn_bwd_dq_sm100",
     "attn_bwd_dq_fp32", "attn_bwd_dkv_fp32", "prologue_bwd", "convert_f16",
-    "decode"};
+    "decode", "pad_fill"};
 constexpr int kMaxSlots = 1 << 15;
 struct Prof {
   std::mutex mu;
@@ -187,11 +187,13 @@ extern "C" size_t flint_attn_workspace_bytes(const flint_attn_params_t* params, 
   return make_layout(p, backward != 0).total;
 }
 
-extern "C" flint_status_t flint_attn_fwd(const flint_attn_params_t* params, const void* q,
-                                         const void* k, const void* v, const void* q_norm_w,
-                                         const void* k_norm_w, const float* sink,
-                                         const int32_t* cu_doc_lens, void* out, float* lse,
-                                         void* workspace, size_t workspace_bytes, void* stream) {
+namespace {
+// valid: per-document count of real tokens (trailing padding), or nullptr.
+flint_status_t fwd_impl(const flint_attn_params_t* params, const void* q, const void* k,
+                        const void* v, const void* q_norm_w, const void* k_norm_w,
+                        const float* sink, const int32_t* cu_doc_lens, const int32_t* valid,
+                        void* out, float* lse, void* workspace, size_t workspace_bytes,
+                        void* stream) {
   Resolved p;
   flint_status_t s = resolve(params, &p);
   if (s != FLINT_OK) return s;
@@ -219,7 +221,7 @@ extern "C" flint_status_t flint_attn_fwd(const flint_attn_params_t* params, cons
                                             st));
   }
   int4* items = at<int4>(workspace, L.items_q);
-  FLINT_TRY(launch_build_worklist(cu_doc_lens, p, kModeQuery, 2 * p.R, items, status + 1,
+  FLINT_TRY(launch_build_worklist(cu_doc_lens, valid, p, kModeQuery, 2 * p.R, items, status + 1,
                                   at<void>(workspace, L.sched_tmp), L.max_items_q, st));
   __half* v16 = at<__half>(workspace, L.v16);
   FLINT_TRY(launch_convert_f16(static_cast<const __nv_bfloat16*>(v), v16,
@@ -230,18 +232,18 @@ extern "C" flint_status_t flint_attn_fwd(const flint_attn_params_t* params, cons
       !encode_3d(&tk, kh, p.T, p.Hk, 1, kTileKeys, f16t) ||
       !encode_3d(&tv, v16, p.T, p.Hk, 1, kTileKeys, f16t))
     return FLINT_ERR_CUDA;
-  return cuda_status(launch_attn_fwd_sm100_impl(tq, tk, tv, p, sink, items, status + 1,
-                                                L.max_items_q, out, lse, status, sm_count(), st));
+  FLINT_TRY(launch_attn_fwd_sm100_impl(tq, tk, tv, p, sink, items, status + 1, L.max_items_q,
+                                       out, lse, status, sm_count(), st));
+  if (valid) FLINT_TRY(launch_pad_fill_fwd(p, cu_doc_lens, valid, sink, out, lse, st));
+  return FLINT_OK;
 }
 
-extern "C" flint_status_t flint_attn_bwd(const flint_attn_params_t* params, const void* q,
-                                         const void* k, const void* v, const void* q_norm_w,
-                                         const void* k_norm_w, const float* sink,
-                                         const int32_t* cu_doc_lens, const void* out,
-                                         const float* lse, const void* dout, void* dq, void* dk,
-                                         void* dv, float* dq_norm_w, float* dk_norm_w,
-                                         float* dsink, void* workspace, size_t workspace_bytes,
-                                         void* stream) {
+flint_status_t bwd_impl(const flint_attn_params_t* params, const void* q, const void* k,
+                        const void* v, const void* q_norm_w, const void* k_norm_w,
+                        const float* sink, const int32_t* cu_doc_lens, const int32_t* valid,
+                        const void* out, const float* lse, const void* dout, void* dq, void* dk,
+                        void* dv, float* dq_norm_w, float* dk_norm_w, float* dsink,
+                        void* workspace, size_t workspace_bytes, void* stream) {
   Resolved p;
   flint_status_t s = resolve(params, &p);
   if (s != FLINT_OK) return s;
@@ -283,10 +285,10 @@ extern "C" flint_status_t flint_attn_bwd(const flint_attn_params_t* params, cons
     int4* items_kv = at<int4>(workspace, L.items_kv);
     int4* items_q1 = at<int4>(workspace, L.items_q1);
     void* tmp = at<void>(workspace, L.sched_tmp);
-    FLINT_TRY(launch_build_worklist(cu_doc_lens, p, kModeKey, kTileKeys, items_kv, status + 2, tmp,
-                                    L.max_items_kv, st));
-    FLINT_TRY(launch_build_worklist(cu_doc_lens, p, kModeQuery, p.R, items_q1, status + 3, tmp,
-                                    L.max_items_q1, st));
+    FLINT_TRY(launch_build_worklist(cu_doc_lens, valid, p, kModeKey, kTileKeys, items_kv,
+                                    status + 2, tmp, L.max_items_kv, st));
+    FLINT_TRY(launch_build_worklist(cu_doc_lens, valid, p, kModeQuery, p.R, items_q1, status + 3,
+                                    tmp, L.max_items_q1, st));
     FLINT_TRY(launch_convert_f16(static_cast<const __nv_bfloat16*>(v), v16,
                                  (size_t)p.T * p.Hk * kHeadDim, st));
     const CUtensorMapDataType f16t = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
@@ -299,6 +301,8 @@ extern "C" flint_status_t flint_attn_bwd(const flint_attn_params_t* params, cons
     FLINT_TRY(launch_attn_bwd_sm100_impl(tq, tk, tv, tdo, p, lse, dvec, items_kv, status + 2,
                                          L.max_items_kv, items_q1, status + 3, L.max_items_q1,
                                          dq_acc, dk_acc, dv, status, sm_count(), st));
+    if (valid)
+      FLINT_TRY(launch_pad_fill_bwd(p, cu_doc_lens, valid, dq_acc, dk_acc, dv, p.fp32_out, st));
   }
   float* part_q = part + (size_t)kPartBlocks * p.H;
   float* part_k = part_q + (size_t)kPartBlocks * kHeadDim;
@@ -307,6 +311,59 @@ extern "C" flint_status_t flint_attn_bwd(const flint_attn_params_t* params, cons
   FLINT_TRY(launch_bwd_epilogue(p, k, k_norm_w, dk_acc, dk, dk_norm_w, part_k, p.Hk, cu_doc_lens,
                                 st));
   return FLINT_OK;
+}
+
+bool padded_args_ok(const flint_attn_params_t* params, const int32_t* valid_lens) {
+  return params && valid_lens && aligned(valid_lens, 4);
+}
+}  // namespace
+
+extern "C" flint_status_t flint_attn_fwd(const flint_attn_params_t* params, const void* q,
+                                         const void* k, const void* v, const void* q_norm_w,
+                                         const void* k_norm_w, const float* sink,
+                                         const int32_t* cu_doc_lens, void* out, float* lse,
+                                         void* workspace, size_t workspace_bytes, void* stream) {
+  return fwd_impl(params, q, k, v, q_norm_w, k_norm_w, sink, cu_doc_lens, nullptr, out, lse,
+                  workspace, workspace_bytes, stream);
+}
+
+extern "C" flint_status_t flint_attn_bwd(const flint_attn_params_t* params, const void* q,
+                                         const void* k, const void* v, const void* q_norm_w,
+                                         const void* k_norm_w, const float* sink,
+                                         const int32_t* cu_doc_lens, const void* out,
+                                         const float* lse, const void* dout, void* dq, void* dk,
+                                         void* dv, float* dq_norm_w, float* dk_norm_w,
+                                         float* dsink, void* workspace, size_t workspace_bytes,
+                                         void* stream) {
+  return bwd_impl(params, q, k, v, q_norm_w, k_norm_w, sink, cu_doc_lens, nullptr, out, lse,
+                  dout, dq, dk, dv, dq_norm_w, dk_norm_w, dsink, workspace, workspace_bytes,
+                  stream);
+}
+
+extern "C" flint_status_t flint_attn_fwd_padded(const flint_attn_params_t* params, const void* q,
+                                                const void* k, const void* v,
+                                                const void* q_norm_w, const void* k_norm_w,
+                                                const float* sink, const int32_t* cu_doc_lens,
+                                                const int32_t* valid_lens, void* out, float* lse,
+                                                void* workspace, size_t workspace_bytes,
+                                                void* stream) {
+  if (!padded_args_ok(params, valid_lens)) return FLINT_ERR_INVALID_ARG;
+  if (params->dtype == FLINT_FP32) return FLINT_ERR_UNSUPPORTED;
+  return fwd_impl(params, q, k, v, q_norm_w, k_norm_w, sink, cu_doc_lens, valid_lens, out, lse,
+                  workspace, workspace_bytes, stream);
+}
+
+extern "C" flint_status_t flint_attn_bwd_padded(
+    const flint_attn_params_t* params, const void* q, const void* k, const void* v,
+    const void* q_norm_w, const void* k_norm_w, const float* sink, const int32_t* cu_doc_lens,
+    const int32_t* valid_lens, const void* out, const float* lse, const void* dout, void* dq,
+    void* dk, void* dv, float* dq_norm_w, float* dk_norm_w, float* dsink, void* workspace,
+    size_t workspace_bytes, void* stream) {
+  if (!padded_args_ok(params, valid_lens)) return FLINT_ERR_INVALID_ARG;
+  if (params->dtype == FLINT_FP32) return FLINT_ERR_UNSUPPORTED;
+  return bwd_impl(params, q, k, v, q_norm_w, k_norm_w, sink, cu_doc_lens, valid_lens, out, lse,
+                  dout, dq, dk, dv, dq_norm_w, dk_norm_w, dsink, workspace, workspace_bytes,
+                  stream);
 }
 
 // ------------------------------------------------------------------ decode

@@ -155,7 +155,7 @@ __device__ __forceinline__ void store8(float* p, const float (&f)[8]) {
 // on the launching stream (see flint_attn_profile_* in the public header).
 enum KernelId {
   kKPrologue = 0, kKWorklist, kKFwdSm100, kKFwdFp32, kKBwdPre, kKReduce, kKBwdDkvSm100,
-  kKBwdDqSm100, kKBwdDqFp32, kKBwdDkvFp32, kKPrologueBwd, kKConvert, kKDecode,
+  kKBwdDqSm100, kKBwdDqFp32, kKBwdDkvFp32, kKPrologueBwd, kKConvert, kKDecode, kKPadFill,
   kNumKernelIds
 };
 struct ProfScope {
@@ -168,9 +168,17 @@ struct ProfScope {
 
 // ------------------------------------------------------------------ launchers
 // (defined in the .cu files; all return cudaGetLastError() of their launch)
-cudaError_t launch_build_worklist(const int32_t* cu, const Resolved& p, int mode, int span,
-                                  int4* items, int* count, void* tmp, int max_items,
-                                  cudaStream_t st);
+// valid: per-document count of real tokens (trailing padding), or nullptr
+cudaError_t launch_build_worklist(const int32_t* cu, const int32_t* valid, const Resolved& p,
+                                  int mode, int span, int4* items, int* count, void* tmp,
+                                  int max_items, cudaStream_t st);
+// Padding: padded rows get out = 0 and lse = sink (forward), and zero gradient
+// rows dq_acc, dk_acc (fp32 workspace) and dv (backward).
+cudaError_t launch_pad_fill_fwd(const Resolved& p, const int32_t* cu, const int32_t* valid,
+                                const float* sink, void* out, float* lse, cudaStream_t st);
+cudaError_t launch_pad_fill_bwd(const Resolved& p, const int32_t* cu, const int32_t* valid,
+                                float* dq_acc, float* dk_acc, void* dv, int dv_f32,
+                                cudaStream_t st);
 // out_f16: write x_hat as fp16 (backward operands of BF16 inputs) instead of the input type
 cudaError_t launch_prologue(const Resolved& p, const void* x, const void* w, void* y, int heads,
                             const int32_t* cu, cudaStream_t st, bool out_f16 = false);

@@ -11,6 +11,9 @@
 //   3. counting-sorts the items by price, heaviest first (LPT order), so that a
 //      grid of persistent CTAs striding over the list finishes together.
 // Item = int4 {first token, document start, document end, KV head}.
+// With padding (valid != nullptr), document d ends after its valid[d] real
+// tokens: the trailing padding gets no item, so no kernel visits it as a query
+// or a key.
 #include "common.cuh"
 
 namespace flint {
@@ -59,7 +62,8 @@ __device__ __forceinline__ int item_cost(int mode, int start, int d0, int d1, in
 }
 
 __global__ void __launch_bounds__(kThreads)
-build_worklist_kernel(const int32_t* __restrict__ cu, int N, int mode, int span, int W, int R,
+build_worklist_kernel(const int32_t* __restrict__ cu, const int32_t* __restrict__ valid, int N,
+                      int mode, int span, int W, int R,
                       int Hk, int4* __restrict__ items, int* __restrict__ count,
                       int4* __restrict__ tmp_items, int* __restrict__ tmp_cost, int max_items) {
   __shared__ int warp_sums[32];
@@ -77,6 +81,7 @@ build_worklist_kernel(const int32_t* __restrict__ cu, int N, int mode, int span,
     if (d < N) {
       d0 = __ldg(cu + d);
       d1 = __ldg(cu + d + 1);
+      if (valid) d1 = d0 + max(0, min(__ldg(valid + d), d1 - d0));
       n = (d1 > d0 ? (d1 - d0 + span - 1) / span : 0) * Hk;
     }
     int ex = block_exclusive_scan(n, warp_sums, &total_s);
@@ -92,7 +97,9 @@ build_worklist_kernel(const int32_t* __restrict__ cu, int N, int mode, int span,
       }
       while (chunk_off[lo + 1] <= f) ++lo;       // skip documents with no items
       const int dd = dc + lo;
-      const int e0 = __ldg(cu + dd), e1 = __ldg(cu + dd + 1);
+      const int e0 = __ldg(cu + dd);
+      int e1 = __ldg(cu + dd + 1);
+      if (valid) e1 = e0 + max(0, min(__ldg(valid + dd), e1 - e0));
       const int local = f - chunk_off[lo];
       const int start = e0 + (local / Hk) * span;
       const int g = local % Hk;
@@ -138,14 +145,14 @@ build_worklist_kernel(const int32_t* __restrict__ cu, int N, int mode, int span,
 
 }  // namespace
 
-cudaError_t launch_build_worklist(const int32_t* cu, const Resolved& p, int mode, int span,
-                                  int4* items, int* count, void* tmp, int max_items,
-                                  cudaStream_t st) {
+cudaError_t launch_build_worklist(const int32_t* cu, const int32_t* valid, const Resolved& p,
+                                  int mode, int span, int4* items, int* count, void* tmp,
+                                  int max_items, cudaStream_t st) {
   int4* tmp_items = reinterpret_cast<int4*>(tmp);
   int* tmp_cost = reinterpret_cast<int*>(tmp_items + max_items);
   ProfScope prof(kKWorklist, st);
-  build_worklist_kernel<<<1, kThreads, 0, st>>>(cu, p.N, mode, span, p.W, p.R, p.Hk, items, count,
-                                                tmp_items, tmp_cost, max_items);
+  build_worklist_kernel<<<1, kThreads, 0, st>>>(cu, valid, p.N, mode, span, p.W, p.R, p.Hk, items,
+                                                count, tmp_items, tmp_cost, max_items);
   return cudaGetLastError();
 }
 

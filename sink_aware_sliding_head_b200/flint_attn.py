@@ -29,7 +29,8 @@ EXPORTED = ["flint_attn_workspace_bytes", "flint_attn_fwd", "flint_attn_bwd",
             "flint_attn_profile_enable", "flint_attn_profile_collect",
             "flint_attn_profile_reset", "flint_attn_launch_count",
             "flint_attn_bwd_preprocess_static", "flint_attn_exp2_poly",
-            "flint_attn_decode_workspace_bytes", "flint_attn_decode"]
+            "flint_attn_decode_workspace_bytes", "flint_attn_decode",
+            "flint_attn_fwd_padded", "flint_attn_bwd_padded"]
 
 
 class Params(ctypes.Structure):
@@ -94,6 +95,10 @@ def load_library(path: str = LIB_PATH):
     lib.flint_attn_fwd.restype = ctypes.c_int
     lib.flint_attn_bwd.argtypes = [P] + [vp] * 16 + [vp, sz, vp]
     lib.flint_attn_bwd.restype = ctypes.c_int
+    lib.flint_attn_fwd_padded.argtypes = [P] + [vp] * 10 + [vp, sz, vp]
+    lib.flint_attn_fwd_padded.restype = ctypes.c_int
+    lib.flint_attn_bwd_padded.argtypes = [P] + [vp] * 17 + [vp, sz, vp]
+    lib.flint_attn_bwd_padded.restype = ctypes.c_int
     lib.flint_attn_check_status.argtypes = [vp, vp]
     lib.flint_attn_check_status.restype = ctypes.c_int
     lib.flint_status_string.argtypes = [ctypes.c_int]
@@ -174,10 +179,12 @@ def alloc_workspace(params: Params, backward: bool, device=None) -> torch.Tensor
 
 def fwd(q, k, v, q_norm_w, k_norm_w, sink, cu_doc_lens, window, use_rope, rope_theta,
         rms_eps=1e-6, softmax_scale=0.0, out=None, lse=None, workspace=None, stream=None,
-        check_status=False, fp32_out=False):
+        check_status=False, fp32_out=False, valid_lens=None):
     """Forward through ``flint_attn_fwd``. Returns (out [T,H,D], lse [H,T] fp32).
 
     ``fp32_out``: out is float32 (pass it unchanged to ``bwd`` with the same flag).
+    ``valid_lens``: int32 [num_docs] on the device, the real tokens at the start of
+    each document (trailing padding; ``flint_attn_fwd_padded``).
     """
     lib = load_library()
     p = params_for(q, k, cu_doc_lens, window, use_rope, rope_theta, rms_eps, softmax_scale,
@@ -191,9 +198,15 @@ def fwd(q, k, v, q_norm_w, k_norm_w, sink, cu_doc_lens, window, use_rope, rope_t
     if workspace is None:
         workspace = alloc_workspace(p, False, q.device)
     st = _stream_ptr(stream)
-    code = lib.flint_attn_fwd(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(q_norm_w),
-                              _ptr(k_norm_w), _ptr(sink), _ptr(cu_doc_lens), _ptr(out), _ptr(lse),
-                              _ptr(workspace), workspace.numel(), st)
+    if valid_lens is None:
+        code = lib.flint_attn_fwd(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(q_norm_w),
+                                  _ptr(k_norm_w), _ptr(sink), _ptr(cu_doc_lens), _ptr(out),
+                                  _ptr(lse), _ptr(workspace), workspace.numel(), st)
+    else:
+        code = lib.flint_attn_fwd_padded(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v),
+                                         _ptr(q_norm_w), _ptr(k_norm_w), _ptr(sink),
+                                         _ptr(cu_doc_lens), _ptr(valid_lens), _ptr(out),
+                                         _ptr(lse), _ptr(workspace), workspace.numel(), st)
     _check(code, "flint_attn_fwd")
     if check_status:
         _check(lib.flint_attn_check_status(_ptr(workspace), st), "flint_attn_fwd (device)")
@@ -202,8 +215,8 @@ def fwd(q, k, v, q_norm_w, k_norm_w, sink, cu_doc_lens, window, use_rope, rope_t
 
 def bwd(q, k, v, q_norm_w, k_norm_w, sink, cu_doc_lens, out, lse, dout, window, use_rope,
         rope_theta, rms_eps=1e-6, softmax_scale=0.0, grads=None, workspace=None, stream=None,
-        check_status=False, fp32_out=False):
-    """Backward through ``flint_attn_bwd``.
+        check_status=False, fp32_out=False, valid_lens=None):
+    """Backward through ``flint_attn_bwd`` (``flint_attn_bwd_padded`` with ``valid_lens``).
 
     Returns a dict with dq, dk, dv (input dtype, or float32 with ``fp32_out``),
     dw_q, dw_k, dsink (fp32). ``out`` must be the forward's result with the same
@@ -226,11 +239,18 @@ def bwd(q, k, v, q_norm_w, k_norm_w, sink, cu_doc_lens, out, lse, dout, window, 
     if workspace is None:
         workspace = alloc_workspace(p, True, q.device)
     st = _stream_ptr(stream)
-    code = lib.flint_attn_bwd(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(q_norm_w),
-                              _ptr(k_norm_w), _ptr(sink), _ptr(cu_doc_lens), _ptr(out), _ptr(lse),
-                              _ptr(dout), _ptr(grads["dq"]), _ptr(grads["dk"]), _ptr(grads["dv"]),
-                              _ptr(grads["dw_q"]), _ptr(grads["dw_k"]), _ptr(grads["dsink"]),
-                              _ptr(workspace), workspace.numel(), st)
+    g = [_ptr(grads[n]) for n in ("dq", "dk", "dv", "dw_q", "dw_k", "dsink")]
+    if valid_lens is None:
+        code = lib.flint_attn_bwd(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(q_norm_w),
+                                  _ptr(k_norm_w), _ptr(sink), _ptr(cu_doc_lens), _ptr(out),
+                                  _ptr(lse), _ptr(dout), *g, _ptr(workspace), workspace.numel(),
+                                  st)
+    else:
+        code = lib.flint_attn_bwd_padded(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v),
+                                         _ptr(q_norm_w), _ptr(k_norm_w), _ptr(sink),
+                                         _ptr(cu_doc_lens), _ptr(valid_lens), _ptr(out),
+                                         _ptr(lse), _ptr(dout), *g, _ptr(workspace),
+                                         workspace.numel(), st)
     _check(code, "flint_attn_bwd")
     if check_status:
         _check(lib.flint_attn_check_status(_ptr(workspace), st), "flint_attn_bwd (device)")
