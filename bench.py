@@ -63,6 +63,13 @@ def parse_args(argv=None):
 
 # --------------------------------------------------------------------------- helpers
 
+def real_lens(inp):
+    """Real tokens per document (all of it unless the workload has padding)."""
+    if "valid_lens" in inp:
+        return [int(x) for x in inp["valid_lens"]]
+    return list(inp["doc_lens"])
+
+
 def flops_of(doc_lens, window, H, D=128):
     pairs = fi.visible_pairs(doc_lens, window)
     return pairs, 4.0 * D * H * pairs, 10.0 * D * H * pairs
@@ -83,6 +90,8 @@ def config_of(w, pairs, flops_step):
         "workload": f"{w.name} fwd+bwd",
         "tokens": w.total_tokens,
         "docs": "drawn U[128,8192]" if w.doc_lens is None else len(w.doc_lens),
+        "padding": (f"trailing, real tokens per document drawn U{list(w.valid_range)}; "
+                    "masked FLOPs count real tokens only") if w.valid_range else None,
         "heads_q": w.num_q_heads, "heads_kv": w.num_kv_heads, "head_dim": w.head_dim,
         "window": w.window if w.window > 0 else "full causal",
         "rope": bool(w.use_rope), "rope_theta": w.rope_theta if w.use_rope else None,
@@ -200,6 +209,18 @@ def oracle_sample(w, inp, seconds):
     """
     from oracle import flint_oracle as fo   # test infrastructure: CPU baseline leg only
 
+    if "valid_lens" in inp:
+        # the real tokens alone: the padded layer's real rows are exactly this layer
+        idx, cu_v = [], [0]
+        for d, (a, b) in enumerate(zip(inp["cu_doc_lens"][:-1].tolist(),
+                                       inp["cu_doc_lens"][1:].tolist())):
+            n = min(int(inp["valid_lens"][d]), b - a)
+            idx.extend(range(a, a + n))
+            cu_v.append(cu_v[-1] + n)
+        idx = torch.tensor(idx)
+        inp = dict(inp, q=inp["q"][idx], k=inp["k"][idx], v=inp["v"][idx],
+                   dout=inp["dout"][idx], cu_doc_lens=torch.tensor(cu_v, dtype=torch.int32))
+
     def run(n_tok):
         cu = [int(c) for c in inp["cu_doc_lens"]]
         lens, acc = [], 0
@@ -253,7 +274,7 @@ def run_reference(args):
         return
     w = WORKLOADS[args.workload]
     inp = fi.make_inputs(w, with_grad_out=True)
-    pairs, ff, fb = flops_of(inp["doc_lens"], w.window, w.num_q_heads)
+    pairs, ff, fb = flops_of(real_lens(inp), w.window, w.num_q_heads)
     per_step = max(2.0, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
     total_f, total_t, desc = 0.0, 0.0, ""
     for i in range(args.warmup + args.steps):
@@ -527,7 +548,7 @@ def main(argv=None):
         w = dataclasses.replace(w, name=f"{w.name}@{args.tokens}", doc_lens=(args.tokens,),
                                 total_tokens=args.tokens, drawn_len_range=None)
     cpu = fi.make_inputs(w, seed=w.seed + rank, with_grad_out=True)
-    pairs, ff, fb = flops_of(cpu["doc_lens"], w.window, w.num_q_heads)
+    pairs, ff, fb = flops_of(real_lens(cpu), w.window, w.num_q_heads)
     flops_step = ff + fb
     d = {k: (v.to(dev) if torch.is_tensor(v) else v) for k, v in cpu.items()}
     T, H, D = d["q"].shape
@@ -554,13 +575,14 @@ def main(argv=None):
         fa.fwd(src["q"], src["k"], src["v"], src["w_q"], src["w_k"], src["sink"],
                src["cu_doc_lens"], w.window, w.use_rope, w.rope_theta,
                out=out if o is None else o, lse=lse if l is None else l,
-               workspace=ws_f, fp32_out=True)
+               workspace=ws_f, fp32_out=True, valid_lens=src.get("valid_lens"))
 
     def bwd_call(src, o=None, l=None, g=None):
         fa.bwd(src["q"], src["k"], src["v"], src["w_q"], src["w_k"], src["sink"],
                src["cu_doc_lens"], out if o is None else o, lse if l is None else l,
                src["dout"], w.window, w.use_rope, w.rope_theta,
-               grads=grads if g is None else g, workspace=ws_b, fp32_out=True)
+               grads=grads if g is None else g, workspace=ws_b, fp32_out=True,
+               valid_lens=src.get("valid_lens"))
 
     # ---- warm-up (also surfaces device-side timeouts before timing)
     for _ in range(args.warmup):
@@ -615,6 +637,8 @@ def main(argv=None):
     e2e = None
     if not args.no_e2e:
         names_in = ["q", "k", "v", "w_q", "w_k", "sink", "cu_doc_lens", "dout"]
+        if "valid_lens" in cpu:
+            names_in.append("valid_lens")
         host_in = [{k: cpu[k].pin_memory() for k in names_in} for _ in range(2)]
         dev_in = [{k: torch.empty_like(d[k]) for k in names_in} for _ in range(2)]
         dev_out = [{"out": out, "lse": lse, **grads}]

@@ -47,6 +47,7 @@ class Workload:
     drawn_len_range: Optional[tuple] = None   # (lo, hi) inclusive, for drawn lengths
     rms_eps: float = 1e-6
     seed: int = 0
+    valid_range: Optional[tuple] = None       # (lo, hi): real tokens per document, rest padding
 
 
 # The five synthetic Flint layers the library is measured and checked on.
@@ -71,7 +72,16 @@ LONG_FULL_BF16 = Workload(
     num_q_heads=32, num_kv_heads=4, head_dim=128, window=0, use_rope=False,
     rope_theta=1e6, dtype="bf16")
 
-WORKLOADS = [TINY_SLIDING_FP32, SLIDING_BF16, FULL_BF16, PACKED_BF16, LONG_FULL_BF16]
+# BSHD with trailing padding (the attention utils page's attention_mask, trailing
+# as TE takes it): 8 sequences of 8192 slots, 4096-8192 real tokens each, on the
+# sliding-layer shape of the packed workload.
+BSHD_PADDED_BF16 = Workload(
+    name="bshd_padded_bf16_B8_S8192_H32x4_W1024", doc_lens=(8192,) * 8, total_tokens=65536,
+    num_q_heads=32, num_kv_heads=4, head_dim=128, window=1024, use_rope=True,
+    rope_theta=1e6, dtype="bf16", valid_range=(4096, 8192))
+
+WORKLOADS = [TINY_SLIDING_FP32, SLIDING_BF16, FULL_BF16, PACKED_BF16, LONG_FULL_BF16,
+             BSHD_PADDED_BF16]
 
 
 def draw_doc_lens(w: Workload, gen: torch.Generator) -> List[int]:
@@ -111,7 +121,8 @@ def make_inputs(w: Workload, seed: Optional[int] = None, with_grad_out: Optional
 
     Returns a dict of CPU tensors: ``q`` [T,H,D], ``k``/``v`` [T,Hk,D], ``w_q``/``w_k``
     [D] (all in the workload dtype), ``sink`` [H] FP32, ``cu_doc_lens`` int32
-    [N+1], and ``dout`` [T,H,D] when a backward pass is wanted.
+    [N+1], and ``dout`` [T,H,D] when a backward pass is wanted. Padded workloads
+    add ``valid_lens`` int32 [N] (drawn last, so the other draws are unchanged).
     """
     seed = w.seed if seed is None else seed
     with_grad_out = w.backward if with_grad_out is None else with_grad_out
@@ -129,6 +140,10 @@ def make_inputs(w: Workload, seed: Optional[int] = None, with_grad_out: Optional
     out["sink"] = w.sink_std * torch.randn(H, generator=gen, dtype=torch.float32)
     if with_grad_out:
         out["dout"] = torch.randn(T, H, D, generator=gen, dtype=torch.float32).to(dt)
+    if w.valid_range is not None:
+        lo, hi = w.valid_range
+        v = torch.randint(lo, hi + 1, (len(lens),), generator=gen, dtype=torch.int64)
+        out["valid_lens"] = torch.minimum(v, torch.tensor(lens)).to(torch.int32)
     return out
 
 
