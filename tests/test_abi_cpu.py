@@ -104,3 +104,20 @@ def test_decode_validation(lib):
     assert code == 2                                     # FLINT_ERR_UNSUPPORTED
     code = lib.flint_attn_decode(ctypes.byref(ok), *([nul] * 11), nul, 0, nul)
     assert code == 1                                     # null pointers, before any launch
+
+
+def test_header_is_c99_and_links(lib, tmp_path):
+    """A C99 program that includes the public header and links the library."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    exe = tmp_path / "abi_check"
+    libdir = os.path.dirname(fa.LIB_PATH)
+    subprocess.run([gcc, "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"),
+                    os.path.join(ROOT, "tests", "c", "abi_check.c"), "-o", str(exe),
+                    "-L", libdir, "-lflint_attn", f"-Wl,-rpath,{libdir}"], check=True)
+    r = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    assert "c abi ok" in r.stdout
