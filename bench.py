@@ -9,6 +9,13 @@ for the forward and 10*D*H*pairs for the backward (five GEMMs).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
 
+The default workload is the 32768-token full-causal layer (32/4 heads). Other
+workloads: ``--workload bshd_padded_bf16_B8_S8192_H32x4_W1024`` (the padded
+calls, FLOPs over real tokens) and ``--workload decode_bf16_B64_C8192_H32x4_W4096``
+(flint_attn_decode; metric: K/V bytes read per second, roofline against HBM).
+``--impl reference`` times the FP64 oracle on the host cores for the same
+workload and metric.
+
 Multi-GPU (torchrun, one process per GPU): every rank runs its own batch
 (replicas, weak scaling); no data-path collective exists in this path. The
 step time is the max over ranks of CUDA-event time. Rank 0 prints one JSON line.
