@@ -81,7 +81,8 @@ typedef struct {
   int32_t total_tokens;   /* T = cu_doc_lens[num_docs]; 0 <= T < 2^31 / H / D */
   int32_t num_docs;       /* N >= 1; zero-length documents are allowed */
   int32_t num_q_heads;    /* H, a multiple of num_kv_heads */
-  int32_t num_kv_heads;   /* Hk >= 1; G = H / Hk must be 1, 2, 4, 8 or 16 */
+  int32_t num_kv_heads;   /* Hk >= 1; G = H / Hk must be 1, 2, 4, 8 or 16 (tensor-core
+                             paths; FP32 inputs without compute_f16 take any G) */
   int32_t head_dim;       /* D; must be 128 */
   int32_t window;         /* > 0: key j visible from query i iff 0 <= i - j < window
                              (counts the current token); <= 0: full causal */
@@ -92,7 +93,15 @@ typedef struct {
   int32_t dtype;          /* flint_dtype_t */
   int32_t fp32_out;       /* nonzero => out (forward, and as passed to the backward) and
                              dq, dk, dv are float32; zero => same type as q. FP32 inputs
-                             always use float32. */
+                             always use float32 (but see compute_f16). */
+  int32_t compute_f16;    /* FP32 inputs only (else FLINT_ERR_INVALID_ARG): the fp16
+                             attention boundary of attention_compute_dtype='fp16' (Flint
+                             config page: an fp16 QKV/kernel-output boundary inside
+                             otherwise FP32 compute). RMSNorm and RoPE run in FP32; q_hat,
+                             k_hat, v (and dout in the backward) enter the tcgen05
+                             tensor-core path as fp16, and out is written as IEEE fp16
+                             (float32 with fp32_out). dq, dk, dv and the norm-weight and
+                             sink gradients stay float32. G must be 1, 2, 4, 8 or 16. */
 } flint_attn_params_t;
 
 /* Bytes of device workspace a call needs (backward = 0 for flint_attn_fwd,

@@ -89,8 +89,9 @@ flint_status_t resolve(const flint_attn_params_t* in, Resolved* p) {
   if (in->num_q_heads % in->num_kv_heads != 0) return FLINT_ERR_INVALID_ARG;
   if (in->head_dim != kHeadDim) return FLINT_ERR_UNSUPPORTED;
   const int G = in->num_q_heads / in->num_kv_heads;
-  if (in->dtype == FLINT_BF16 && !(G == 1 || G == 2 || G == 4 || G == 8 || G == 16))
-    return FLINT_ERR_UNSUPPORTED;
+  if (in->compute_f16 && in->dtype != FLINT_FP32) return FLINT_ERR_INVALID_ARG;
+  const bool tc = in->dtype == FLINT_BF16 || in->compute_f16;
+  if (tc && !(G == 1 || G == 2 || G == 4 || G == 8 || G == 16)) return FLINT_ERR_UNSUPPORTED;
   if ((long long)in->total_tokens * in->num_q_heads * in->head_dim > 0x7fffffffLL)
     return FLINT_ERR_INVALID_ARG;
   if (!(std::isfinite(in->rms_eps) && in->rms_eps >= 0.f)) return FLINT_ERR_INVALID_ARG;
@@ -110,6 +111,8 @@ flint_status_t resolve(const flint_attn_params_t* in, Resolved* p) {
   p->scale = in->softmax_scale > 0.f ? in->softmax_scale : 1.0f / std::sqrt((float)kHeadDim);
   p->dtype = in->dtype;
   p->fp32_out = (in->fp32_out != 0 || in->dtype == FLINT_FP32) ? 1 : 0;
+  p->tc = tc ? 1 : 0;
+  p->out_f16 = (in->compute_f16 && !in->fp32_out) ? 1 : 0;
   p->R = kTileRows / (G <= 128 ? G : 128);
   if (p->R < 1) p->R = 1;
   return FLINT_OK;
@@ -188,6 +191,14 @@ extern "C" size_t flint_attn_workspace_bytes(const flint_attn_params_t* params, 
 }
 
 namespace {
+// fp16 copy of v, the B operand of the PV / P^T dO MMAs
+cudaError_t convert_v(const Resolved& p, const void* v, __half* v16, cudaStream_t st) {
+  const size_t n = (size_t)p.T * p.Hk * kHeadDim;
+  if (p.dtype == FLINT_BF16)
+    return launch_convert_f16(static_cast<const __nv_bfloat16*>(v), v16, n, st);
+  return launch_convert_f16(static_cast<const float*>(v), v16, n, st);
+}
+
 // valid: per-document count of real tokens (trailing padding), or nullptr.
 flint_status_t fwd_impl(const flint_attn_params_t* params, const void* q, const void* k,
                         const void* v, const void* q_norm_w, const void* k_norm_w,
@@ -212,10 +223,10 @@ flint_status_t fwd_impl(const flint_attn_params_t* params, const void* q, const 
   if (p.T == 0) return FLINT_OK;
   void* qh = at<void>(workspace, L.qhat);
   void* kh = at<void>(workspace, L.khat);
-  const bool f16 = p.dtype == FLINT_BF16;   // tensor-core operands are fp16
+  const bool f16 = p.tc;   // tensor-core operands are fp16
   FLINT_TRY(launch_prologue(p, q, q_norm_w, qh, p.H, cu_doc_lens, st, f16));
   FLINT_TRY(launch_prologue(p, k, k_norm_w, kh, p.Hk, cu_doc_lens, st, f16));
-  if (p.dtype == FLINT_FP32) {
+  if (!p.tc) {
     return cuda_status(launch_attn_fwd_fp32(p, (const float*)qh, (const float*)kh,
                                             (const float*)v, sink, cu_doc_lens, (float*)out, lse,
                                             st));
@@ -224,8 +235,7 @@ flint_status_t fwd_impl(const flint_attn_params_t* params, const void* q, const 
   FLINT_TRY(launch_build_worklist(cu_doc_lens, valid, p, kModeQuery, 2 * p.R, items, status + 1,
                                   at<void>(workspace, L.sched_tmp), L.max_items_q, st));
   __half* v16 = at<__half>(workspace, L.v16);
-  FLINT_TRY(launch_convert_f16(static_cast<const __nv_bfloat16*>(v), v16,
-                               (size_t)p.T * p.Hk * kHeadDim, st));
+  FLINT_TRY(convert_v(p, v, v16, st));
   const CUtensorMapDataType f16t = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
   CUtensorMap tq, tk, tv;
   if (!encode_3d(&tq, qh, p.T, p.H, p.G, p.R, f16t) ||
@@ -271,13 +281,13 @@ flint_status_t bwd_impl(const flint_attn_params_t* params, const void* q, const 
   float* part = at<float>(workspace, L.part);
   float* dq_acc = at<float>(workspace, L.dq_acc);
   float* dk_acc = at<float>(workspace, L.dk_acc);
-  const bool f16 = p.dtype == FLINT_BF16;   // tensor-core operands of the backward are fp16
+  const bool f16 = p.tc;   // tensor-core operands of the backward are fp16
   __half* dout16 = f16 ? at<__half>(workspace, L.dout16) : nullptr;
   __half* v16 = f16 ? at<__half>(workspace, L.v16) : nullptr;
   FLINT_TRY(launch_prologue(p, q, q_norm_w, qh, p.H, cu_doc_lens, st, f16));
   FLINT_TRY(launch_prologue(p, k, k_norm_w, kh, p.Hk, cu_doc_lens, st, f16));
   FLINT_TRY(launch_bwd_preprocess(p, out, dout, lse, sink, dvec, part, dsink, dout16, st));
-  if (p.dtype == FLINT_FP32) {
+  if (!p.tc) {
     FLINT_TRY(launch_attn_bwd_fp32(p, (const float*)qh, (const float*)kh, (const float*)v,
                                    (const float*)dout, lse, dvec, cu_doc_lens, dq_acc, dk_acc,
                                    (float*)dv, st));
@@ -289,8 +299,7 @@ flint_status_t bwd_impl(const flint_attn_params_t* params, const void* q, const 
                                     status + 2, tmp, L.max_items_kv, st));
     FLINT_TRY(launch_build_worklist(cu_doc_lens, valid, p, kModeQuery, p.R, items_q1, status + 3,
                                     tmp, L.max_items_q1, st));
-    FLINT_TRY(launch_convert_f16(static_cast<const __nv_bfloat16*>(v), v16,
-                                 (size_t)p.T * p.Hk * kHeadDim, st));
+    FLINT_TRY(convert_v(p, v, v16, st));
     const CUtensorMapDataType f16t = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
     CUtensorMap tq, tk, tv, tdo;
     if (!encode_3d(&tq, qh, p.T, p.H, p.G, p.R, f16t) ||
@@ -348,7 +357,7 @@ extern "C" flint_status_t flint_attn_fwd_padded(const flint_attn_params_t* param
                                                 void* workspace, size_t workspace_bytes,
                                                 void* stream) {
   if (!padded_args_ok(params, valid_lens)) return FLINT_ERR_INVALID_ARG;
-  if (params->dtype == FLINT_FP32) return FLINT_ERR_UNSUPPORTED;
+  if (params->dtype == FLINT_FP32 && !params->compute_f16) return FLINT_ERR_UNSUPPORTED;
   return fwd_impl(params, q, k, v, q_norm_w, k_norm_w, sink, cu_doc_lens, valid_lens, out, lse,
                   workspace, workspace_bytes, stream);
 }
@@ -360,7 +369,7 @@ extern "C" flint_status_t flint_attn_bwd_padded(
     void* dk, void* dv, float* dq_norm_w, float* dk_norm_w, float* dsink, void* workspace,
     size_t workspace_bytes, void* stream) {
   if (!padded_args_ok(params, valid_lens)) return FLINT_ERR_INVALID_ARG;
-  if (params->dtype == FLINT_FP32) return FLINT_ERR_UNSUPPORTED;
+  if (params->dtype == FLINT_FP32 && !params->compute_f16) return FLINT_ERR_UNSUPPORTED;
   return bwd_impl(params, q, k, v, q_norm_w, k_norm_w, sink, cu_doc_lens, valid_lens, out, lse,
                   dout, dq, dk, dv, dq_norm_w, dk_norm_w, dsink, workspace, workspace_bytes,
                   stream);

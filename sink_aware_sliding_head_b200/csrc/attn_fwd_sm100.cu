@@ -65,8 +65,8 @@ struct FwdArgs {
   const int4* items;
   const int* n_items;
   int max_items;
-  void* out;        // bf16 or float, per out_f32
-  int out_f32;
+  void* out;        // bf16, float (out_f32) or fp16 (out_f16)
+  int out_f32, out_f16;
   float* lse;
   int* status;
 };
@@ -488,14 +488,22 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
               *reinterpret_cast<float4*>(orow + 4 * v4) =
                   make_float4(o[4 * v4], o[4 * v4 + 1], o[4 * v4 + 2], o[4 * v4 + 3]);
           } else {
-            __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.out) + obase + c * 32;
+            // bf16, or IEEE fp16 for the fp16 compute boundary (both 2 bytes)
+            uint16_t* orow = reinterpret_cast<uint16_t*>(a.out) + obase + c * 32;
 #pragma unroll
             for (int v4 = 0; v4 < 4; ++v4) {
               uint4 pk;
-              pk.x = pack_bf16x2(o[v4 * 8 + 0], o[v4 * 8 + 1]);
-              pk.y = pack_bf16x2(o[v4 * 8 + 2], o[v4 * 8 + 3]);
-              pk.z = pack_bf16x2(o[v4 * 8 + 4], o[v4 * 8 + 5]);
-              pk.w = pack_bf16x2(o[v4 * 8 + 6], o[v4 * 8 + 7]);
+              if (a.out_f16) {
+                pk.x = pack_f16x2(o[v4 * 8 + 0], o[v4 * 8 + 1]);
+                pk.y = pack_f16x2(o[v4 * 8 + 2], o[v4 * 8 + 3]);
+                pk.z = pack_f16x2(o[v4 * 8 + 4], o[v4 * 8 + 5]);
+                pk.w = pack_f16x2(o[v4 * 8 + 6], o[v4 * 8 + 7]);
+              } else {
+                pk.x = pack_bf16x2(o[v4 * 8 + 0], o[v4 * 8 + 1]);
+                pk.y = pack_bf16x2(o[v4 * 8 + 2], o[v4 * 8 + 3]);
+                pk.z = pack_bf16x2(o[v4 * 8 + 4], o[v4 * 8 + 5]);
+                pk.w = pack_bf16x2(o[v4 * 8 + 6], o[v4 * 8 + 7]);
+              }
               *reinterpret_cast<uint4*>(orow + v4 * 8) = pk;
             }
           }
@@ -531,7 +539,8 @@ cudaError_t launch_attn_fwd_sm100_impl(const CUtensorMap& tq, const CUtensorMap&
   a.scale_log2 = p.scale * kLog2e;
   a.sink = sink; a.items = items; a.n_items = n_items; a.max_items = max_items;
   a.out = out;
-  a.out_f32 = p.fp32_out;
+  a.out_f32 = p.fp32_out && !p.out_f16;
+  a.out_f16 = p.out_f16;
   a.lse = lse;
   a.status = status;
   int grid = num_sms;

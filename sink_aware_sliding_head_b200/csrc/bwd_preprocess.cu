@@ -22,8 +22,8 @@ constexpr int kThreads = 256;
 constexpr int kGroups = kThreads / 16;
 constexpr int kTok = 4;
 
-// Also writes an fp16 copy of dO (dout16, when non-null): the BF16 backward's
-// tensor-core operands are fp16.
+// Also writes an fp16 copy of dO (dout16, when non-null): the tensor-core
+// backward's operands are fp16.
 template <typename TO, typename T>
 __global__ void __launch_bounds__(kThreads)
 bwd_pre_kernel(const TO* __restrict__ out, const T* __restrict__ dout,
@@ -77,7 +77,8 @@ bwd_pre_kernel(const TO* __restrict__ out, const T* __restrict__ dout,
 }
 
 // dst[i] = fp16(src[i]) for n elements (n a multiple of 8), saturating at +-65504.
-__global__ void convert_f16_kernel(const __nv_bfloat16* __restrict__ src, __half* __restrict__ dst,
+template <typename T>
+__global__ void convert_f16_kernel(const T* __restrict__ src, __half* __restrict__ dst,
                                    size_t n8) {
   for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n8;
        i += (size_t)gridDim.x * blockDim.x) {
@@ -106,14 +107,21 @@ cudaError_t launch_exp2_poly(const float* x, float* y, int n, cudaStream_t st) {
   return cudaGetLastError();
 }
 
-cudaError_t launch_convert_f16(const __nv_bfloat16* src, __half* dst, size_t n, cudaStream_t st) {
+template <typename T>
+static cudaError_t convert_f16(const T* src, __half* dst, size_t n, cudaStream_t st) {
   const size_t n8 = n / 8;
   if (n8 == 0) return cudaSuccess;
   size_t blocks = (n8 + 255) / 256;
   if (blocks > 148 * 16) blocks = 148 * 16;
   ProfScope prof(kKConvert, st);
-  convert_f16_kernel<<<(unsigned)blocks, 256, 0, st>>>(src, dst, n8);
+  convert_f16_kernel<T><<<(unsigned)blocks, 256, 0, st>>>(src, dst, n8);
   return cudaGetLastError();
+}
+cudaError_t launch_convert_f16(const __nv_bfloat16* src, __half* dst, size_t n, cudaStream_t st) {
+  return convert_f16(src, dst, n, st);
+}
+cudaError_t launch_convert_f16(const float* src, __half* dst, size_t n, cudaStream_t st) {
+  return convert_f16(src, dst, n, st);
 }
 
 cudaError_t launch_bwd_preprocess(const Resolved& p, const void* out, const void* dout,
@@ -135,9 +143,13 @@ cudaError_t launch_bwd_preprocess(const Resolved& p, const void* out, const void
   else if (p.dtype == FLINT_BF16)
     bwd_pre_kernel<bf, bf><<<blocks, kThreads, smem, st>>>(
         (const bf*)out, (const bf*)dout, lse, sink, dvec, part, dout16, p.T, p.H);
+  else if (p.out_f16)   // FP32 inputs at the fp16 compute boundary: out is fp16
+    bwd_pre_kernel<__half, float><<<blocks, kThreads, smem, st>>>(
+        (const __half*)out, (const float*)dout, lse, sink, dvec, part, dout16, p.T, p.H);
   else
     bwd_pre_kernel<float, float><<<blocks, kThreads, smem, st>>>(
-        (const float*)out, (const float*)dout, lse, sink, dvec, part, nullptr, p.T, p.H);
+        (const float*)out, (const float*)dout, lse, sink, dvec, part, p.tc ? dout16 : nullptr,
+        p.T, p.H);
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;

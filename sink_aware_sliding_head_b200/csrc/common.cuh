@@ -31,6 +31,8 @@ struct Resolved {
   float theta, eps, scale;
   int dtype;
   int fp32_out;     // out, dq, dk, dv are float32 (always for FP32 inputs)
+  int tc;           // the tcgen05 path with fp16 operands: BF16 inputs, or FP32 + compute_f16
+  int out_f16;      // out is IEEE fp16 (FP32 inputs with compute_f16, without fp32_out)
   int R;            // tokens per 128-row tile = 128 / G
 };
 
@@ -46,8 +48,8 @@ struct WsLayout {
   size_t part;          // fp32 partial sums (d sink, d norm weights)
   size_t dq_acc;        // [T,H,D] fp32 gradient w.r.t. q_hat (backward)
   size_t dk_acc;        // [T,Hk,D] fp32 gradient w.r.t. k_hat (backward)
-  size_t dout16;        // [T,H,D] fp16 copy of dO (backward, BF16 inputs)
-  size_t v16;           // [T,Hk,D] fp16 copy of v (BF16 inputs)
+  size_t dout16;        // [T,H,D] fp16 copy of dO (backward, tensor-core path)
+  size_t v16;           // [T,Hk,D] fp16 copy of v (tensor-core path)
   size_t total;
   int max_items_q, max_items_q1, max_items_kv, max_items_any;
   int part_blocks;      // number of partial-sum rows per reduced quantity
@@ -78,13 +80,13 @@ inline WsLayout make_layout(const Resolved& p, bool backward) {
   L.items_kv = backward ? take((size_t)L.max_items_kv * 16) : off;
   L.sched_tmp = take((size_t)L.max_items_any * 20);
   L.part_blocks = kPartBlocks;
-  if (p.dtype == FLINT_BF16) L.v16 = take((size_t)p.T * p.Hk * p.D * 2);
+  if (p.tc) L.v16 = take((size_t)p.T * p.Hk * p.D * 2);
   if (backward) {
     L.dvec = take((size_t)p.H * p.T * 4);
     L.part = take((size_t)kPartBlocks * (p.H + 2 * p.D) * 4);
     L.dq_acc = take((size_t)p.T * p.H * p.D * 4);
     L.dk_acc = take((size_t)p.T * p.Hk * p.D * 4);
-    if (p.dtype == FLINT_BF16) L.dout16 = take((size_t)p.T * p.H * p.D * 2);
+    if (p.tc) L.dout16 = take((size_t)p.T * p.H * p.D * 2);
   }
   L.total = off;
   return L;
@@ -118,6 +120,16 @@ __device__ __forceinline__ void load8(const __nv_bfloat16* p, float (&f)[8]) {
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     float2 t = __bfloat1622float2(h[i]);
+    f[2 * i] = t.x;
+    f[2 * i + 1] = t.y;
+  }
+}
+__device__ __forceinline__ void load8(const __half* p, float (&f)[8]) {
+  const uint4 u = *reinterpret_cast<const uint4*>(p);
+  const __half2* h = reinterpret_cast<const __half2*>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 t = __half22float2(h[i]);
     f[2 * i] = t.x;
     f[2 * i + 1] = t.y;
   }
@@ -183,6 +195,7 @@ cudaError_t launch_pad_fill_bwd(const Resolved& p, const int32_t* cu, const int3
 cudaError_t launch_prologue(const Resolved& p, const void* x, const void* w, void* y, int heads,
                             const int32_t* cu, cudaStream_t st, bool out_f16 = false);
 cudaError_t launch_convert_f16(const __nv_bfloat16* src, __half* dst, size_t n, cudaStream_t st);
+cudaError_t launch_convert_f16(const float* src, __half* dst, size_t n, cudaStream_t st);
 
 // Decode over a KV cache (decode.cu). Keys per split CTA of the window.
 constexpr int kChunkKeysDecode = 1024;

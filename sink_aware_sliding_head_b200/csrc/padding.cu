@@ -68,7 +68,8 @@ cudaError_t launch_pad_fill_fwd(const Resolved& p, const int32_t* cu, const int3
                                 const float* sink, void* out, float* lse, cudaStream_t st) {
   if (p.T == 0) return cudaSuccess;
   ProfScope prof(kKPadFill, st);
-  pad_fill_fwd_kernel<<<p.T, kThreads, 0, st>>>(p.T, p.N, p.H, cu, valid, sink, out, p.fp32_out,
+  const int out_f32 = p.fp32_out && !p.out_f16;   // else a 2-byte type (zeros alike)
+  pad_fill_fwd_kernel<<<p.T, kThreads, 0, st>>>(p.T, p.N, p.H, cu, valid, sink, out, out_f32,
                                                 lse);
   return cudaGetLastError();
 }

@@ -210,6 +210,10 @@ cudaError_t launch_prologue(const Resolved& p, const void* x, const void* w, voi
   else if (p.dtype == FLINT_BF16)
     prologue_kernel<bf, bf><<<grid, kThreads, 0, st>>>(
         (const bf*)x, (const bf*)w, (bf*)y, p.T, heads, cu, p.N, p.rope, p.theta, p.eps);
+  else if (out_f16)   // FP32 inputs at the fp16 compute boundary
+    prologue_kernel<float, __half><<<grid, kThreads, 0, st>>>(
+        (const float*)x, (const float*)w, (__half*)y, p.T, heads, cu, p.N, p.rope, p.theta,
+        p.eps);
   else
     prologue_kernel<float, float><<<grid, kThreads, 0, st>>>(
         (const float*)x, (const float*)w, (float*)y, p.T, heads, cu, p.N, p.rope, p.theta, p.eps);

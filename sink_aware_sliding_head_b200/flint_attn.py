@@ -48,6 +48,7 @@ class Params(ctypes.Structure):
         ("softmax_scale", ctypes.c_float),
         ("dtype", ctypes.c_int32),
         ("fp32_out", ctypes.c_int32),
+        ("compute_f16", ctypes.c_int32),
     ]
 
 
@@ -130,10 +131,11 @@ def load_library(path: str = LIB_PATH):
 
 def make_params(total_tokens, num_docs, num_q_heads, num_kv_heads, window, use_rope,
                 rope_theta, dtype, head_dim=128, rms_eps=1e-6, softmax_scale=0.0,
-                fp32_out=False) -> Params:
+                fp32_out=False, compute_f16=False) -> Params:
     return Params(int(total_tokens), int(num_docs), int(num_q_heads), int(num_kv_heads),
                   int(head_dim), int(window), 1 if use_rope else 0, float(rope_theta),
-                  float(rms_eps), float(softmax_scale), int(dtype), 1 if fp32_out else 0)
+                  float(rms_eps), float(softmax_scale), int(dtype), 1 if fp32_out else 0,
+                  1 if compute_f16 else 0)
 
 
 def _ptr(t: Optional[torch.Tensor]):
@@ -159,11 +161,11 @@ def _check(code: int, where: str):
 
 
 def params_for(q, k, cu_doc_lens, window, use_rope, rope_theta, rms_eps=1e-6,
-               softmax_scale=0.0, fp32_out=False) -> Params:
+               softmax_scale=0.0, fp32_out=False, compute_f16=False) -> Params:
     T, H, D = q.shape
     return make_params(T, cu_doc_lens.numel() - 1, H, k.shape[1], window, use_rope, rope_theta,
                        _dtype_code(q), head_dim=D, rms_eps=rms_eps, softmax_scale=softmax_scale,
-                       fp32_out=fp32_out)
+                       fp32_out=fp32_out, compute_f16=compute_f16)
 
 
 def workspace_bytes(params: Params, backward: bool) -> int:
@@ -179,20 +181,22 @@ def alloc_workspace(params: Params, backward: bool, device=None) -> torch.Tensor
 
 def fwd(q, k, v, q_norm_w, k_norm_w, sink, cu_doc_lens, window, use_rope, rope_theta,
         rms_eps=1e-6, softmax_scale=0.0, out=None, lse=None, workspace=None, stream=None,
-        check_status=False, fp32_out=False, valid_lens=None):
+        check_status=False, fp32_out=False, valid_lens=None, compute_f16=False):
     """Forward through ``flint_attn_fwd``. Returns (out [T,H,D], lse [H,T] fp32).
 
     ``fp32_out``: out is float32 (pass it unchanged to ``bwd`` with the same flag).
     ``valid_lens``: int32 [num_docs] on the device, the real tokens at the start of
     each document (trailing padding; ``flint_attn_fwd_padded``).
+    ``compute_f16`` (float32 inputs): the fp16 attention boundary; out is float16
+    unless ``fp32_out``.
     """
     lib = load_library()
     p = params_for(q, k, cu_doc_lens, window, use_rope, rope_theta, rms_eps, softmax_scale,
-                   fp32_out)
+                   fp32_out, compute_f16)
     T, H, D = q.shape
     if out is None:
-        out = torch.empty(q.shape, dtype=torch.float32 if fp32_out else q.dtype,
-                          device=q.device)
+        odt = torch.float32 if fp32_out else (torch.float16 if compute_f16 else q.dtype)
+        out = torch.empty(q.shape, dtype=odt, device=q.device)
     if lse is None:
         lse = torch.empty(H, T, dtype=torch.float32, device=q.device)
     if workspace is None:
@@ -215,7 +219,7 @@ def fwd(q, k, v, q_norm_w, k_norm_w, sink, cu_doc_lens, window, use_rope, rope_t
 
 def bwd(q, k, v, q_norm_w, k_norm_w, sink, cu_doc_lens, out, lse, dout, window, use_rope,
         rope_theta, rms_eps=1e-6, softmax_scale=0.0, grads=None, workspace=None, stream=None,
-        check_status=False, fp32_out=False, valid_lens=None):
+        check_status=False, fp32_out=False, valid_lens=None, compute_f16=False):
     """Backward through ``flint_attn_bwd`` (``flint_attn_bwd_padded`` with ``valid_lens``).
 
     Returns a dict with dq, dk, dv (input dtype, or float32 with ``fp32_out``),
@@ -224,7 +228,7 @@ def bwd(q, k, v, q_norm_w, k_norm_w, sink, cu_doc_lens, out, lse, dout, window, 
     """
     lib = load_library()
     p = params_for(q, k, cu_doc_lens, window, use_rope, rope_theta, rms_eps, softmax_scale,
-                   fp32_out)
+                   fp32_out, compute_f16)
     T, H, D = q.shape
     gdt = torch.float32 if (fp32_out or q.dtype == torch.float32) else q.dtype
     if grads is None:

@@ -121,3 +121,13 @@ def test_header_is_c99_and_links(lib, tmp_path):
     r = subprocess.run([str(exe)], capture_output=True, text=True)
     assert r.returncode == 0, r.stderr
     assert "c abi ok" in r.stdout
+
+
+def test_compute_f16_validation(lib):
+    """The fp16 attention boundary is for FP32 inputs and the tensor-core group sizes."""
+    assert fa.workspace_bytes(params(compute_f16=True), False) == 0          # BF16 inputs
+    assert fa.workspace_bytes(params(dtype=fa.FLINT_FP32, compute_f16=True, num_q_heads=12,
+                                     num_kv_heads=1), False) == 0            # G = 12
+    plain = fa.workspace_bytes(params(dtype=fa.FLINT_FP32), True)
+    f16 = fa.workspace_bytes(params(dtype=fa.FLINT_FP32, compute_f16=True), True)
+    assert f16 >= plain + 256 * (32 + 4) * 128 * 2      # fp16 copies of dO and v
