@@ -164,12 +164,16 @@ class ClockSampler:
 
 
 def kernel_source_sha(name):
+    """Fingerprint of a kernel source's code: // comments and blank lines are left out,
+    so recorded profiler counters stay attached to the code they measured."""
     path = os.path.join(ROOT, "sink_aware_sliding_head_b200", "csrc", name)
     try:
-        with open(path, "rb") as f:
-            return hashlib.sha256(f.read()).hexdigest()[:16]
+        with open(path) as f:
+            lines = [ln.split("//", 1)[0].rstrip() for ln in f]
     except OSError:
         return None
+    code = "\n".join(ln for ln in lines if ln)
+    return hashlib.sha256(code.encode()).hexdigest()[:16]
 
 
 def traffic_for(kernel, workload):

@@ -27,14 +27,19 @@
 //    128-row query tiles (R tokens x G heads) that see them. Per tile:
 //    S^T = K Q^T and dP^T = V dO^T (TMEM), then P^T and dS^T in fp16 are
 //    written over S^T and feed dV += P^T dO and dK += dS^T Q as TMEM A
-//    operands. The S^T and dP^T regions swap roles every tile, so the next
-//    S^T never waits for an MMA to finish. dK and dV stay in TMEM for the whole
-//    key tile, so the G heads of a group are summed without atomics. TMEM:
-//    2 x 128 rotating columns + dV + dK = 512 cols.
+//    operands. The S^T and dP^T regions swap roles every tile: the next S^T
+//    goes into this tile's dP^T region as soon as the math warps hold dP^T in
+//    registers, so it runs during their dS step. dK and dV stay in TMEM for the
+//    whole key tile, so the G heads of a group are summed without atomics.
+//    TMEM: 2 x 128 rotating columns + dV + dK = 512 cols. Query tiles stream
+//    through 3 shared-memory stages, dO tiles (with the per-row statistics)
+//    through 2.
 //  * dq: query-major. A CTA owns one 128-row query tile and streams its key
 //    tiles: S = Q K^T, dP = dO V^T, dS (fp16) over S, dQ += dS K. TMEM: two S
 //    buffers, dP, dQ = 512 cols; S of the next key tile is computed while the
-//    math warps finish the current one.
+//    math warps finish the current one. K and V stream through a 5-slot ring.
+// In both P steps one exponential pair in four is evaluated on the FMA pipe
+// (exp2_fma2); the special-function unit alone would bound them.
 // Before an MMA overwrites a TMEM region that a previous MMA reads as its A
 // operand, the issuer waits for that MMA's completion barrier.
 #include <type_traits>
