@@ -596,7 +596,8 @@ __device__ __forceinline__ QItem decode_q(const BwdArgs& a, int idx) {
 }
 
 // Tiles are numbered per CTA across items (t = 0, 1, ...): tile t uses S
-// buffer t % 2 and K/V stage t % 2.
+// buffer t % 2, and K(t), V(t) take ring positions 2t and 2t + 1. An item has
+// at least one key tile (kbeg <= q0 < kend).
 __global__ void __launch_bounds__(kThreads, 1)
 attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q,
                    const __grid_constant__ CUtensorMap tm_k,
@@ -736,6 +737,9 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q,
                      leader);
           mma_commit_w(smem_u32(&bars->dp_full), leader);
           mma_commit_w(smem_u32(&bars->kv_empty[sv]), leader);   // V(t) done after dP(t)
+          // Q and dO are read only by the S and dP MMAs, so the item's last dP frees
+          // them: the next item's Q/dO loads overlap this tile's dS and dQ.
+          if (n + 1 == it.ntiles) mma_commit_w(smem_u32(&bars->qd_empty), leader);
           if (n + 1 < it.ntiles) {
             ok = issue_s(t + 1);
             if (!ok) break;
@@ -756,7 +760,6 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q,
           mma_commit_w(smem_u32(&bars->kv_empty[sk]), leader);   // K(t) done after dQ(t)
         }
         if (!ok) break;
-        mma_commit_w(smem_u32(&bars->qd_empty), leader);
         mma_commit_w(smem_u32(&bars->acc_full), leader);
         ++item_count;
       }
