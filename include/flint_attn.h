@@ -37,7 +37,10 @@
  * Conventions for every call:
  *   - All tensor arguments are DEVICE pointers owned by the caller, contiguous,
  *     row-major, 16-byte aligned. The library allocates no memory and keeps no
- *     state between calls except a cached device property (SM count).
+ *     state between calls except the SM count of each device and each kernel's
+ *     raised dynamic shared-memory limit. That limit is set once per process,
+ *     at the first call, on the device current then: a process drives one
+ *     device (multi-GPU use is one process per GPU).
  *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
  *     stream). Results are ready when the stream is synchronised.
  *   - Argument errors are returned before any launch (no GPU work is queued).
