@@ -13,9 +13,10 @@
 // Design:
 //   * A 128-row tile is R = 128/G tokens x the G query heads of one KV group,
 //     so every K/V tile staged by TMA feeds all G heads of the group (GQA
-//     sharing inside the CTA; no tile is broadcast across CTAs). A CTA works on two such tiles at
-//     once ("tile 0" and "tile 1": 2R consecutive tokens) that share every K/V
-//     tile, so each K/V byte brought on chip serves 256 query rows.
+//     sharing inside the CTA; no tile is broadcast across CTAs). A CTA works
+//     on two such tiles at once ("tile 0" and "tile 1": 2R consecutive tokens)
+//     that share every K/V tile, so each K/V byte brought on chip serves 256
+//     query rows.
 //   * Persistent grid (one CTA per SM) striding over an LPT-sorted work list
 //     built on the device; only key tiles inside the window and the document
 //     are visited, and only edge tiles are masked.
