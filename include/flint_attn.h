@@ -283,6 +283,22 @@ long long flint_attn_launch_count(void);
  * n even. Asynchronous on `stream`. */
 flint_status_t flint_attn_exp2_poly(const float* x, float* y, int32_t n, void* stream);
 
+/* Self-test of failure detection, without a GPU fault. One warp waits, through
+ * the same bounded mbarrier wait that every pipelined kernel uses, on a
+ * shared-memory barrier that completes only if arrive_first != 0, and gives
+ * up after wait_cycles SM clock cycles (1 <= wait_cycles <= 4e9, the kernels'
+ * own limit). status: caller-owned device int32[64], 256-byte aligned, with
+ * status[0] = 0 on entry (the layout of a workspace's status word). A wait
+ * that runs out sets a timeout bit in status[0], so a following
+ * flint_attn_check_status(status, stream) returns FLINT_ERR_TIMEOUT (and
+ * clears the word); status[1] = 1 if the wait completed, 0 if it gave up. The
+ * kernel exits normally either way and the CUDA context stays usable.
+ * Asynchronous on `stream`. FLINT_ERR_INVALID_ARG for a null or misaligned
+ * status pointer or a limit out of range (before any launch); FLINT_ERR_CUDA
+ * if the launch fails. */
+flint_status_t flint_attn_selftest_wait(int64_t wait_cycles, int32_t arrive_first,
+                                        int32_t* status, void* stream);
+
 /* Static description of a status code. */
 const char* flint_status_string(flint_status_t status);
 

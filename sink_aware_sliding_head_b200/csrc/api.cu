@@ -513,6 +513,14 @@ extern "C" flint_status_t flint_attn_exp2_poly(const float* x, float* y, int32_t
   return cuda_status(launch_exp2_poly(x, y, n, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+extern "C" flint_status_t flint_attn_selftest_wait(int64_t wait_cycles, int32_t arrive_first,
+                                                   int32_t* status, void* stream) {
+  if (!status || !aligned(status, 256) || wait_cycles < 1 || wait_cycles > FLINT_WAIT_CYCLES)
+    return FLINT_ERR_INVALID_ARG;
+  return cuda_status(launch_wait_selftest((long long)wait_cycles, arrive_first != 0 ? 1 : 0,
+                                          status, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 extern "C" const char* flint_status_string(flint_status_t s) {
   switch (s) {
     case FLINT_OK: return "ok";

@@ -23,6 +23,7 @@ enum : int {
   kStatusTimeoutBwdQ = 4,
   kStatusSmemAlign = 8,        // dynamic shared memory not 1024-byte aligned
   kStatusDecodeRange = 16,     // a decode cache_lens entry outside [0, cache_capacity)
+  kStatusTimeoutSelftest = 32, // the bounded-wait self-test's wait ran out
 };
 
 // Parameters after validation and defaulting.
@@ -196,6 +197,10 @@ cudaError_t launch_prologue(const Resolved& p, const void* x, const void* w, voi
                             const int32_t* cu, cudaStream_t st, bool out_f16 = false);
 cudaError_t launch_convert_f16(const __nv_bfloat16* src, __half* dst, size_t n, cudaStream_t st);
 cudaError_t launch_convert_f16(const float* src, __half* dst, size_t n, cudaStream_t st);
+// Bounded-wait self-test (selftest.cu): status[0] gets the timeout bit, status[1]
+// 1 if the wait completed and 0 if it gave up.
+cudaError_t launch_wait_selftest(long long limit, int arrive_first, int* status,
+                                 cudaStream_t st);
 
 // Decode over a KV cache (decode.cu). Keys per split CTA of the window.
 constexpr int kChunkKeysDecode = 1024;

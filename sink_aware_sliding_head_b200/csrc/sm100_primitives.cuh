@@ -61,13 +61,16 @@ struct WaitCtx {
   int code;                   // bit recorded in *status on timeout
 };
 
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const WaitCtx& w) {
+// limit: SM clock cycles before the wait gives up (the kernels take the
+// default; the bounded-wait self-test passes a short one).
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const WaitCtx& w,
+                                          long long limit = FLINT_WAIT_CYCLES) {
   if (mbar_try_wait(bar, parity)) return true;
   long long t0 = clock64();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*w.abort_flag) return false;
-    if (clock64() - t0 > FLINT_WAIT_CYCLES) {
+    if (clock64() - t0 > limit) {
       *w.abort_flag = 1;
       atomicOr(w.status, w.code);
       return false;
@@ -76,8 +79,9 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const W
 }
 
 // The same wait taken by a whole warp; every lane gets the same answer.
-__device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, const WaitCtx& w) {
-  return __all_sync(0xffffffffu, mbar_wait(bar, parity, w));
+__device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, const WaitCtx& w,
+                                               long long limit = FLINT_WAIT_CYCLES) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity, w, limit));
 }
 
 // ---------------------------------------------------------------- dynamic work items

@@ -30,7 +30,7 @@ EXPORTED = ["flint_attn_workspace_bytes", "flint_attn_fwd", "flint_attn_bwd",
             "flint_attn_profile_reset", "flint_attn_launch_count",
             "flint_attn_bwd_preprocess_static", "flint_attn_exp2_poly",
             "flint_attn_decode_workspace_bytes", "flint_attn_decode",
-            "flint_attn_fwd_padded", "flint_attn_bwd_padded"]
+            "flint_attn_fwd_padded", "flint_attn_bwd_padded", "flint_attn_selftest_wait"]
 
 
 class Params(ctypes.Structure):
@@ -120,6 +120,8 @@ def load_library(path: str = LIB_PATH):
     lib.flint_attn_bwd_preprocess_static.restype = ctypes.c_int
     lib.flint_attn_exp2_poly.argtypes = [vp, vp, ctypes.c_int32, vp]
     lib.flint_attn_exp2_poly.restype = ctypes.c_int
+    lib.flint_attn_selftest_wait.argtypes = [ctypes.c_int64, ctypes.c_int32, vp, vp]
+    lib.flint_attn_selftest_wait.restype = ctypes.c_int
     DP = ctypes.POINTER(DecodeParams)
     lib.flint_attn_decode_workspace_bytes.argtypes = [DP]
     lib.flint_attn_decode_workspace_bytes.restype = sz
@@ -359,6 +361,20 @@ def exp2_poly(x: torch.Tensor) -> torch.Tensor:
     _check(load_library().flint_attn_exp2_poly(_ptr(x), _ptr(y), x.numel(), _stream_ptr()),
            "flint_attn_exp2_poly")
     return y
+
+
+def selftest_wait(wait_cycles: int, arrive_first: bool, stream=None):
+    """Bounded-wait self-test on the device: (flint_attn_check_status code, completed).
+
+    A wait that nothing completes must give FLINT_ERR_TIMEOUT and completed = False.
+    """
+    lib = load_library()
+    status = torch.zeros(64, dtype=torch.int32, device="cuda")
+    st = _stream_ptr(stream)
+    _check(lib.flint_attn_selftest_wait(int(wait_cycles), 1 if arrive_first else 0,
+                                        _ptr(status), st), "flint_attn_selftest_wait")
+    code = lib.flint_attn_check_status(_ptr(status), st)      # synchronises the stream
+    return code, bool(status[1].item())
 
 
 def version() -> str:

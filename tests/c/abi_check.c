@@ -53,6 +53,7 @@ int main(void) {
   CHECK(flint_attn_decode(&d, NULL, NULL, NULL, NULL, NULL, NULL, NULL, NULL, NULL, NULL, NULL,
                           NULL, 0, NULL) == FLINT_ERR_UNSUPPORTED);
 
+  CHECK(flint_attn_selftest_wait(1000, 0, NULL, NULL) == FLINT_ERR_INVALID_ARG);
   CHECK(strstr(flint_attn_version(), "sm_100a") != NULL);
   CHECK(strlen(flint_status_string(FLINT_ERR_TIMEOUT)) > 0);
   if (fails == 0) printf("c abi ok\n");

@@ -131,3 +131,13 @@ def test_compute_f16_validation(lib):
     plain = fa.workspace_bytes(params(dtype=fa.FLINT_FP32), True)
     f16 = fa.workspace_bytes(params(dtype=fa.FLINT_FP32, compute_f16=True), True)
     assert f16 >= plain + 256 * (32 + 4) * 128 * 2      # fp16 copies of dO and v
+
+
+def test_selftest_wait_validation(lib):
+    """flint_attn_selftest_wait rejects bad arguments before any launch."""
+    P = ctypes.c_void_p
+    f = lib.flint_attn_selftest_wait
+    assert f(1000, 0, P(0), None) == 1                   # null status
+    assert f(1000, 0, P(0x100010), None) == 1            # not 256-byte aligned
+    assert f(0, 0, P(0x100000), None) == 1               # limit below 1 cycle
+    assert f(4_000_000_001, 0, P(0x100000), None) == 1   # above the kernels' own limit

@@ -4,7 +4,8 @@
 memory where they run: it takes only inputs and outputs and keeps its scratch
 in a fixed array inside the library. Its d_sink must equal the one the regular
 ``flint_attn_bwd`` (which uses a caller workspace) returns, call after call.
-This file is collected last on purpose.
+This file is collected after the parity files on purpose, so that under -x a
+failure here stops none of them.
 """
 import pytest
 import torch
