@@ -50,6 +50,10 @@
  *   - Layouts: q, out, dout, dq [T, H, D]; k, v, dk, dv [T, Hk, D];
  *     q_norm_w, k_norm_w [D]; sink, dsink [H] fp32; lse [H, T] fp32;
  *     dq_norm_w, dk_norm_w [D] fp32.
+ *   - An empty batch (T = 0; documents of length 0) is valid: the [T, ...]
+ *     tensors (q, k, v, out, lse, dout, dq, dk, dv) may then be null. The
+ *     forward writes nothing; the backward writes zero dsink and norm-weight
+ *     gradients.
  *   - dtype FLINT_BF16: q, k, v, dout and the norm weights are bfloat16; out,
  *     dq, dk, dv are bfloat16, or float32 with params->fp32_out. The attention
  *     contractions run on tcgen05 tensor cores with FP32 accumulation; their

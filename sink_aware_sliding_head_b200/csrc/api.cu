@@ -208,11 +208,16 @@ flint_status_t fwd_impl(const flint_attn_params_t* params, const void* q, const 
   Resolved p;
   flint_status_t s = resolve(params, &p);
   if (s != FLINT_OK) return s;
-  const void* vec16[] = {q, k, v, q_norm_w, k_norm_w, out};
-  for (const void* ptr : vec16)
+  // With no tokens the [T, ...] tensors are empty and may be null.
+  const bool no_tokens = p.T == 0;
+  const void* tok16[] = {q, k, v, out};
+  for (const void* ptr : tok16)
+    if ((!ptr && !no_tokens) || !aligned(ptr, 16)) return FLINT_ERR_INVALID_ARG;
+  const void* w16[] = {q_norm_w, k_norm_w};
+  for (const void* ptr : w16)
     if (!ptr || !aligned(ptr, 16)) return FLINT_ERR_INVALID_ARG;
-  if (!sink || !aligned(sink, 4) || !cu_doc_lens || !aligned(cu_doc_lens, 4) || !lse ||
-      !aligned(lse, 4))
+  if (!sink || !aligned(sink, 4) || !cu_doc_lens || !aligned(cu_doc_lens, 4) ||
+      (!lse && !no_tokens) || !aligned(lse, 4))
     return FLINT_ERR_INVALID_ARG;
   const WsLayout L = make_layout(p, false);
   if (!workspace || !aligned(workspace, 256)) return FLINT_ERR_INVALID_ARG;
@@ -257,10 +262,16 @@ flint_status_t bwd_impl(const flint_attn_params_t* params, const void* q, const 
   Resolved p;
   flint_status_t s = resolve(params, &p);
   if (s != FLINT_OK) return s;
-  const void* vec16[] = {q, k, v, q_norm_w, k_norm_w, out, dout, dq, dk, dv};
-  for (const void* ptr : vec16)
+  // With no tokens the [T, ...] tensors are empty and may be null.
+  const bool no_tokens = p.T == 0;
+  const void* tok16[] = {q, k, v, out, dout, dq, dk, dv};
+  for (const void* ptr : tok16)
+    if ((!ptr && !no_tokens) || !aligned(ptr, 16)) return FLINT_ERR_INVALID_ARG;
+  const void* w16[] = {q_norm_w, k_norm_w};
+  for (const void* ptr : w16)
     if (!ptr || !aligned(ptr, 16)) return FLINT_ERR_INVALID_ARG;
-  const void* vec4[] = {sink, cu_doc_lens, lse, dq_norm_w, dk_norm_w, dsink};
+  if ((!lse && !no_tokens) || !aligned(lse, 4)) return FLINT_ERR_INVALID_ARG;
+  const void* vec4[] = {sink, cu_doc_lens, dq_norm_w, dk_norm_w, dsink};
   for (const void* ptr : vec4)
     if (!ptr || !aligned(ptr, 4)) return FLINT_ERR_INVALID_ARG;
   const WsLayout L = make_layout(p, true);

@@ -141,3 +141,23 @@ def test_selftest_wait_validation(lib):
     assert f(1000, 0, P(0x100010), None) == 1            # not 256-byte aligned
     assert f(0, 0, P(0x100000), None) == 1               # limit below 1 cycle
     assert f(4_000_000_001, 0, P(0x100000), None) == 1   # above the kernels' own limit
+
+
+def test_empty_batch_accepts_null_token_tensors(lib):
+    """With T = 0 the [T, ...] tensors may be null; validation passes them and stops
+    at the workspace size check (which comes before any CUDA call). With T > 0 the
+    same null pointers are an argument error."""
+    P = ctypes.c_void_p
+    w, ws = P(0x1000), P(0x100000)
+    for T, want in ((0, 3), (256, 1)):
+        p = params(total_tokens=T, num_docs=2)
+        assert lib.flint_attn_fwd(ctypes.byref(p), None, None, None, w, w, w, w, None, None,
+                                  ws, 16, None) == want
+        assert lib.flint_attn_bwd(ctypes.byref(p), None, None, None, w, w, w, w, None, None,
+                                  None, None, None, None, w, w, w, ws, 16, None) == want
+    p = params(total_tokens=0, num_docs=2)
+    # the parameter-sized tensors stay required
+    assert lib.flint_attn_fwd(ctypes.byref(p), None, None, None, None, w, w, w, None, None,
+                              ws, 16, None) == 1
+    assert lib.flint_attn_bwd(ctypes.byref(p), None, None, None, w, w, w, w, None, None,
+                              None, None, None, None, w, w, None, ws, 16, None) == 1
