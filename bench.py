@@ -77,8 +77,34 @@ def real_lens(inp):
     return list(inp["doc_lens"])
 
 
+def visible_pairs(doc_lens, window: int) -> int:
+    """Masked FLOP accounting: (query, key) pairs per head under the causal document
+    mask whose window counts the current token (row i of a document sees min(i + 1, W)
+    keys)."""
+    total = 0
+    for L in doc_lens:
+        L = int(L)
+        if window <= 0 or window >= L:
+            total += L * (L + 1) // 2
+        else:
+            W = int(window)
+            # rows 0..W-1 see i+1 keys, the rest see W keys
+            total += W * (W + 1) // 2 + (L - W) * W
+    return total
+
+
+def decode_kv_bytes(cache_lens, window: int, num_kv_heads: int, head_dim: int = 128) -> int:
+    """Bytes of K and V (bf16) the decode step reads: every visible slot, once."""
+    total = 0
+    for p in cache_lens:
+        p = int(p)
+        n = p + 1 if window <= 0 else min(p + 1, int(window))
+        total += n
+    return total * num_kv_heads * head_dim * 2 * 2
+
+
 def flops_of(doc_lens, window, H, D=128):
-    pairs = fi.visible_pairs(doc_lens, window)
+    pairs = visible_pairs(doc_lens, window)
     return pairs, 4.0 * D * H * pairs, 10.0 * D * H * pairs
 
 
@@ -332,7 +358,7 @@ def oracle_decode_sample(w, inp, seconds):
                   inp["cache_lens"][sl], inp["k_cache"][sl], inp["v_cache"][sl], w.window,
                   w.use_rope, w.rope_theta)
         dt = time.perf_counter() - t0
-        return fi.decode_kv_bytes(inp["cache_lens"][sl].tolist(), w.window, w.num_kv_heads), dt
+        return decode_kv_bytes(inp["cache_lens"][sl].tolist(), w.window, w.num_kv_heads), dt
 
     b0, t0 = run(1)
     nb = max(1, min(w.batch, int(seconds / max(t0, 1e-3))))
@@ -359,7 +385,7 @@ def run_reference_decode(args):
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * tt / args.steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": decode_config(w, lens, fi.decode_kv_bytes(lens, w.window, w.num_kv_heads)),
+            "config": decode_config(w, lens, decode_kv_bytes(lens, w.window, w.num_kv_heads)),
             "cpu_baseline": {"value": value, "unit": "GB/s", "cores": blas_threads(),
                              "kind": "oracle", "sample": desc},
             "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0,
@@ -385,7 +411,7 @@ def run_decode(args):
     w = DECODE_WORKLOADS[args.workload]
     cpu = fi.make_decode_inputs(w, seed=w.seed + rank)
     lens = cpu["cache_lens"].tolist()
-    kv_bytes = fi.decode_kv_bytes(lens, w.window, w.num_kv_heads)
+    kv_bytes = decode_kv_bytes(lens, w.window, w.num_kv_heads)
     d = {k: v.to(dev) for k, v in cpu.items()}
     B, H, D = d["q"].shape
     p = fa.decode_params(B, w.cache_capacity, H, w.num_kv_heads, w.window, w.use_rope,

@@ -168,20 +168,6 @@ def make_custom(doc_lens, num_q_heads, num_kv_heads, head_dim=128, dtype="bf16",
     return out
 
 
-def visible_pairs(doc_lens, window: int) -> int:
-    """Number of (query, key) pairs under the causal (windowed) document mask, per head."""
-    total = 0
-    for L in doc_lens:
-        L = int(L)
-        if window <= 0 or window >= L:
-            total += L * (L + 1) // 2
-        else:
-            W = int(window)
-            # rows 0..W-1 see i+1 keys, the rest see W keys
-            total += W * (W + 1) // 2 + (L - W) * W
-    return total
-
-
 # ----------------------------------------------------------------------------
 # Decode over a KV cache (one new token per sequence)
 # ----------------------------------------------------------------------------
@@ -243,13 +229,3 @@ def make_decode_inputs(w: DecodeWorkload, seed: Optional[int] = None, lens=None)
     out["k_cache"] = torch.randn(B, Hk, C, D, generator=gen, dtype=torch.float32).to(bf)
     out["v_cache"] = torch.randn(B, Hk, C, D, generator=gen, dtype=torch.float32).to(bf)
     return out
-
-
-def decode_kv_bytes(cache_lens, window: int, num_kv_heads: int, head_dim: int = 128) -> int:
-    """Bytes of K and V (bf16) the decode step reads: every visible slot, once."""
-    total = 0
-    for p in cache_lens:
-        p = int(p)
-        n = p + 1 if window <= 0 else min(p + 1, int(window))
-        total += n
-    return total * num_kv_heads * head_dim * 2 * 2
