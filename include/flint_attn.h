@@ -5,8 +5,9 @@
  * What the calls compute (the passages that define it):
  *   - Per-head RMSNorm of q and k with eps = rms_norm_eps (1e-6 by default):
  *     Flint layers page (nemo_automodel.components.models.flint.layers),
- *     FlintAttention ("Separate Q/K/V, per-head RMSNorm, selective Neox RoPE
- *     and learned sinks"), attributes q_norm, k_norm, eps; Flint config page
+ *     FlintAttention class summary (separate Q/K/V projections, an RMSNorm per
+ *     head, RoPE on selected layers, learned sinks), attributes q_norm,
+ *     k_norm, eps; Flint config page
  *     (nemo_automodel.components.models.flint.config), FlintConfig.rms_norm_eps.
  *     Reading: one weight vector [D] for q and one for k, shared by all heads,
  *     applied as w * x / sqrt(mean(x^2) + eps).
@@ -18,15 +19,15 @@
  *   - Causal window that counts the current token; window <= 0 is unbounded:
  *     FlintConfig docstring and sliding_window; attention utils page
  *     (nemo_automodel.components.attention.utils),
- *     preprocess_args_and_kwargs_for_attn ("window_size" semantics).
+ *     preprocess_args_and_kwargs_for_attn (its window_size convention).
  *   - THD packing: documents given by cu_doc_lens int32 [num_docs + 1], the
  *     cu_seqlens format of preprocess_args_and_kwargs_for_attn; attention never
  *     crosses a document boundary.
  *   - GQA: query head h reads KV head h / (H / Hk).
  *   - One learned FP32 sink logit per query head, unscaled, entering only the
  *     softmax denominator with a zero value: _FlintSinkParameters.forward and
- *     FlintAttention.forward ("causal attention with a zero-value sink
- *     category").
+ *     FlintAttention.forward (the sink is one more softmax category, whose
+ *     value vector is zero).
  *     LSE_i = ln(e^{sink_h} + sum_j e^{z_ij}),  O_i = sum_j e^{z_ij - LSE_i} v_j,
  *     z_ij = softmax_scale * q_hat_i . k_hat_j.
  *   - Backward: gradients of sum(dO * O) w.r.t. q, k, v (raw inputs, before
@@ -36,11 +37,13 @@
  *
  * Conventions for every call:
  *   - All tensor arguments are DEVICE pointers owned by the caller, contiguous,
- *     row-major, 16-byte aligned. The library allocates no memory and keeps no
- *     state between calls except the SM count of each device and each kernel's
- *     raised dynamic shared-memory limit. That limit is set once per process,
- *     at the first call, on the device current then: a process drives one
- *     device (multi-GPU use is one process per GPU).
+ *     row-major, 16-byte aligned. The library allocates no memory. Calls run on
+ *     the device current when they are made; one process may drive several
+ *     devices, from several host threads. State kept between calls, per device:
+ *     the SM count, each kernel's raised dynamic shared-memory limit (set at the
+ *     first call that launches it there), and, for
+ *     flint_attn_bwd_preprocess_static only, the address of a fixed scratch
+ *     array in device memory (see there).
  *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
  *     stream). Results are ready when the stream is synchronised.
  *   - Argument errors are returned before any launch (no GPU work is queued).
@@ -241,16 +244,23 @@ flint_status_t flint_attn_decode(const flint_decode_params_t* params,
  * device memory where they run (a fixed-budget serving loop, a plugin that is
  * given tensors but no workspace, a path where cudaMalloc/cudaFree would
  * synchronise the device).
- *   params: total_tokens, num_q_heads, head_dim (128), dtype, fp32_out (the type
- *   of out, as for flint_attn_bwd) are read; num_q_heads <= FLINT_STATIC_MAX_HEADS,
- *   else FLINT_ERR_WORKSPACE before any launch.
- *   out, dout [T,H,D] (out float32 with fp32_out), lse [H,T] fp32, sink [H] fp32:
- *   device inputs. d_rowsum [H,T], dsink [H]: device outputs (overwritten).
+ *   params: total_tokens, num_q_heads, head_dim (128), dtype, fp32_out and
+ *   compute_f16 are read; they fix the type of out exactly as for flint_attn_bwd
+ *   (float32 with fp32_out or for FP32 inputs; IEEE fp16 for FP32 inputs with
+ *   compute_f16 and without fp32_out; else bfloat16), and dout has the input
+ *   type. compute_f16 with BF16 inputs is FLINT_ERR_INVALID_ARG;
+ *   num_q_heads <= FLINT_STATIC_MAX_HEADS, else FLINT_ERR_WORKSPACE (both
+ *   before any launch).
+ *   out, dout [T,H,D], lse [H,T] fp32, sink [H] fp32: device inputs.
+ *   d_rowsum [H,T], dsink [H]: device outputs (overwritten). With T = 0 the
+ *   [T, ...] pointers (out, dout, lse, d_rowsum) may be null; dsink is zeroed.
  * Its scratch is a fixed 592 KiB array in device memory, held by every GPU that
  * loads the library until exit and shared by all calls: calls whose kernels
  * overlap on the GPU (unordered streams) race on it. The first call on a device
- * looks the array up with that device current; make it before any stream
- * capture on that device. Asynchronous on `stream`. */
+ * looks the array up with that device current and keeps its address for the
+ * rest of the process; make it before any stream capture on that device, and
+ * do not call this entry point on a device again after cudaDeviceReset (the
+ * kept address belongs to the reset context). Asynchronous on `stream`. */
 flint_status_t flint_attn_bwd_preprocess_static(const flint_attn_params_t* params,
                                                 const void* out, const void* dout,
                                                 const float* lse, const float* sink,

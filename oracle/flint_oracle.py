@@ -8,7 +8,8 @@ What it computes, step by step, with the passage each step follows:
 
 * Per-head RMSNorm on q and k: Flint layers page
   (nemo_automodel.components.models.flint.layers), ``FlintAttention`` class
-  summary ("per-head RMSNorm") and its ``q_norm``/``k_norm``/``eps`` attributes;
+  summary (an RMSNorm applied to each head) and its ``q_norm``/``k_norm``/``eps``
+  attributes;
   the epsilon is ``rms_norm_eps`` = 1e-6 on the Flint config page
   (nemo_automodel.components.models.flint.config, ``FlintConfig``).
 * NeoX RoPE: Flint layers page, ``FlintAttention._apply_rope`` (each channel in
@@ -26,8 +27,8 @@ What it computes, step by step, with the passage each step follows:
   on the mistral_large4 attention page).
 * A learned, unscaled FP32 sink logit per query head that enters only the
   softmax denominator, with a zero value: ``_FlintSinkParameters.forward`` and
-  ``FlintAttention.forward`` ("causal attention with a zero-value sink
-  category") on the Flint layers page.
+  ``FlintAttention.forward`` (the sink is one more softmax category whose value
+  vector is zero) on the Flint layers page.
 * GQA with contiguous groups: head h reads KV head floor(h / (H / Hk)).
 
 Readings where the pages are silent: the softmax scale is 1/sqrt(head_dim);

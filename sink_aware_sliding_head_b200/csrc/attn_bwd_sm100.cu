@@ -903,16 +903,11 @@ cudaError_t launch_attn_bwd_sm100_impl(const CUtensorMap& tq, const CUtensorMap&
                                        const int4* items_q, const int* n_q, int max_q,
                                        float* dq_acc, float* dk_acc, void* dv, int* status,
                                        int num_sms, cudaStream_t st) {
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(attn_bwd_dkv_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kKvSmem);
-    if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(attn_bwd_dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kQSmem);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static PerDeviceOnce smem_once_kv, smem_once_q;
+  cudaError_t e0 = smem_limit_once(smem_once_kv, attn_bwd_dkv_kernel, kKvSmem);
+  if (e0 != cudaSuccess) return e0;
+  e0 = smem_limit_once(smem_once_q, attn_bwd_dq_kernel, kQSmem);
+  if (e0 != cudaSuccess) return e0;
   BwdArgs a;
   a.T = p.T; a.H = p.H; a.Hk = p.Hk; a.G = p.G; a.R = p.R; a.W = p.W;
   a.logG = 0;

@@ -528,13 +528,9 @@ cudaError_t launch_attn_fwd_sm100_impl(const CUtensorMap& tq, const CUtensorMap&
                                        const int4* items, const int* n_items, int max_items,
                                        void* out, float* lse, int* status, int num_sms,
                                        cudaStream_t st) {
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(attn_fwd_sm100_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static PerDeviceOnce smem_once;
+  cudaError_t e = smem_limit_once(smem_once, attn_fwd_sm100_kernel, kSmemBytes);
+  if (e != cudaSuccess) return e;
   FwdArgs a;
   a.T = p.T; a.H = p.H; a.Hk = p.Hk; a.G = p.G; a.R = p.R; a.W = p.W;
   a.scale_log2 = p.scale * kLog2e;

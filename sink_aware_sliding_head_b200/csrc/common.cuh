@@ -9,6 +9,7 @@
 #include <cuda_runtime.h>
 
 #include "../../include/flint_attn.h"
+#include "device_once.h"
 
 namespace flint {
 
@@ -244,5 +245,17 @@ cudaError_t launch_attn_bwd_sm100(const Resolved& p, const void* qh, const void*
                                   int num_sms, cudaStream_t st);
 
 enum { kModeQuery = 0, kModeKey = 1 };
+
+// Raises a kernel's dynamic shared-memory limit on the current device the
+// first time its launcher runs there (per device; safe from several threads).
+template <typename Kernel>
+cudaError_t smem_limit_once(PerDeviceOnce& once, Kernel* kernel, int bytes) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  return static_cast<cudaError_t>(once.run(dev, [&] {
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  }));
+}
 
 }  // namespace flint

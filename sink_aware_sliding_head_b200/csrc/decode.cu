@@ -456,13 +456,9 @@ int decode_splits(int C, int W) {
 }
 
 cudaError_t launch_decode(const DecodeLaunch& L, cudaStream_t st) {
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(decode_attn_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kAttnSmem);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static PerDeviceOnce smem_once;
+  cudaError_t e = smem_limit_once(smem_once, decode_attn_kernel, kAttnSmem);
+  if (e != cudaSuccess) return e;
   DecArgs a;
   a.B = L.B; a.C = L.C; a.H = L.H; a.Hk = L.Hk; a.G = L.H / L.Hk; a.W = L.W;
   a.rope = L.rope; a.theta = L.theta; a.eps = L.eps;

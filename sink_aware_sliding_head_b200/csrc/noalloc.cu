@@ -22,9 +22,10 @@
 //    race on it. Order such calls on one stream or with events.
 //  * The first call on a device looks up the array's device address
 //    (cudaGetSymbolAddress) with that device current and caches it. Make that
-//    first call before any stream capture begins on that device.
-#include <mutex>
-
+//    first call before any stream capture begins on that device. The cached
+//    address belongs to the device's primary context: after cudaDeviceReset
+//    (or any reset of that context) this library must not be called again on
+//    that device in the same process.
 #include "common.cuh"
 
 namespace flint {
@@ -38,9 +39,8 @@ constexpr int kStaticPartRows = kPartBlocks;   // the preprocess launch never us
 // address: the address is obtained with cudaGetSymbolAddress below.
 static __device__ __align__(256) float g_bwd_pre_partials[kStaticPartRows * kStaticMaxHeads];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_mu;
-float* g_addr[kMaxDevices] = {};
+PerDeviceOnce g_lookup;
+float* g_addr[kMaxDevices] = {};   // written once per device under g_lookup
 
 // Device address of g_bwd_pre_partials on the current device (looked up once).
 cudaError_t scratch_on_current_device(float** out) {
@@ -48,13 +48,13 @@ cudaError_t scratch_on_current_device(float** out) {
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  std::lock_guard<std::mutex> g(g_mu);
-  if (g_addr[dev] == nullptr) {
+  e = static_cast<cudaError_t>(g_lookup.run(dev, [&] {
     void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_bwd_pre_partials);
-    if (e != cudaSuccess) return e;
-    g_addr[dev] = static_cast<float*>(p);
-  }
+    const cudaError_t r = cudaGetSymbolAddress(&p, g_bwd_pre_partials);
+    if (r == cudaSuccess) g_addr[dev] = static_cast<float*>(p);
+    return r;
+  }));
+  if (e != cudaSuccess) return e;
   *out = g_addr[dev];
   return cudaSuccess;
 }
@@ -74,15 +74,21 @@ extern "C" flint_status_t flint_attn_bwd_preprocess_static(const flint_attn_para
                                                            void* stream) {
   if (!params) return FLINT_ERR_INVALID_ARG;
   if (params->dtype != FLINT_BF16 && params->dtype != FLINT_FP32) return FLINT_ERR_INVALID_ARG;
+  if (params->compute_f16 && params->dtype != FLINT_FP32) return FLINT_ERR_INVALID_ARG;
   if (params->total_tokens < 0 || params->num_q_heads < 1 || params->head_dim != kHeadDim)
     return params->head_dim != kHeadDim ? FLINT_ERR_UNSUPPORTED : FLINT_ERR_INVALID_ARG;
   if ((long long)params->total_tokens * params->num_q_heads * kHeadDim > 0x7fffffffLL)
     return FLINT_ERR_INVALID_ARG;
   if (params->num_q_heads > kStaticMaxHeads) return FLINT_ERR_WORKSPACE;
-  if (!out || !dout || !aligned16(out) || !aligned16(dout)) return FLINT_ERR_INVALID_ARG;
-  if (!lse || !sink || !d_rowsum || !dsink || !aligned4(lse) || !aligned4(sink) ||
-      !aligned4(d_rowsum) || !aligned4(dsink))
+  // With no tokens the [T, ...] tensors (out, dout, lse, d_rowsum) are empty and may be null.
+  const bool no_tokens = params->total_tokens == 0;
+  if ((!no_tokens && (!out || !dout || !lse || !d_rowsum)) || !aligned16(out) ||
+      !aligned16(dout) || !aligned4(lse) || !aligned4(d_rowsum))
     return FLINT_ERR_INVALID_ARG;
+  if (!sink || !dsink || !aligned4(sink) || !aligned4(dsink)) return FLINT_ERR_INVALID_ARG;
+  // The same type rules as flint_attn_bwd: out is float32 with fp32_out (always
+  // for FP32 inputs), IEEE fp16 for FP32 inputs with compute_f16 and without
+  // fp32_out, else the input type.
   Resolved p{};
   p.T = params->total_tokens;
   p.N = params->num_docs > 0 ? params->num_docs : 1;
@@ -91,6 +97,8 @@ extern "C" flint_status_t flint_attn_bwd_preprocess_static(const flint_attn_para
   p.D = kHeadDim;
   p.dtype = params->dtype;
   p.fp32_out = (params->fp32_out != 0 || params->dtype == FLINT_FP32) ? 1 : 0;
+  p.tc = (params->dtype == FLINT_BF16 || params->compute_f16) ? 1 : 0;
+  p.out_f16 = (params->compute_f16 && !params->fp32_out) ? 1 : 0;
   float* scratch = nullptr;
   if (scratch_on_current_device(&scratch) != cudaSuccess) return FLINT_ERR_CUDA;
   cudaError_t e = launch_bwd_preprocess(p, out, dout, lse, sink, d_rowsum, scratch, dsink,

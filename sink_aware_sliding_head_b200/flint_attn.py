@@ -288,22 +288,37 @@ def launch_count() -> int:
     return int(load_library().flint_attn_launch_count())
 
 
-def bwd_preprocess_static(out, dout, lse, sink, fp32_out=False, d_rowsum=None, dsink=None,
-                          stream=None):
+def bwd_preprocess_static(out, dout, lse, sink, d_rowsum=None, dsink=None, stream=None):
     """D = rowsum(dout * out) [H,T] and d_sink [H] through the no-allocation entry point.
 
     For callers that cannot allocate device memory where they run: the library
     uses a fixed scratch array of its own instead of a caller workspace (see
     ``flint_attn_bwd_preprocess_static`` in include/flint_attn.h for its limits).
+    The input type is dout's (bfloat16 or float32); out's type says how the
+    forward stored it: bfloat16 inputs take a bfloat16 or float32 out (fp32_out),
+    float32 inputs a float32 out, or float16 for the fp16 compute boundary
+    (compute_f16).
     """
     lib = load_library()
+    if out.dim() != 3 or dout.shape != out.shape:
+        raise ValueError(f"out {tuple(out.shape)} and dout {tuple(dout.shape)} must both be [T,H,D]")
     T, H, D = out.shape
+    if lse.shape != (H, T) or lse.dtype != torch.float32:
+        raise ValueError(f"lse must be float32 [H,T] = [{H},{T}], got {lse.dtype} {tuple(lse.shape)}")
+    if sink.shape != (H,) or sink.dtype != torch.float32:
+        raise ValueError(f"sink must be float32 [H] = [{H}], got {sink.dtype} {tuple(sink.shape)}")
+    allowed = {torch.bfloat16: (torch.bfloat16, torch.float32),
+               torch.float32: (torch.float32, torch.float16)}
+    if dout.dtype not in allowed or out.dtype not in allowed[dout.dtype]:
+        raise TypeError(f"unsupported pair: dout {dout.dtype}, out {out.dtype}")
+    fp32_out = out.dtype == torch.float32
+    compute_f16 = out.dtype == torch.float16
     p = make_params(T, 1, H, 1, 0, False, 0.0, _dtype_code(dout), head_dim=D,
-                    fp32_out=fp32_out)
+                    fp32_out=fp32_out, compute_f16=compute_f16)
     if d_rowsum is None:
-        d_rowsum = torch.empty(H, T, dtype=torch.float32, device=out.device)
+        d_rowsum = torch.empty(H, T, dtype=torch.float32, device=dout.device)
     if dsink is None:
-        dsink = torch.empty(H, dtype=torch.float32, device=out.device)
+        dsink = torch.empty(H, dtype=torch.float32, device=dout.device)
     code = lib.flint_attn_bwd_preprocess_static(ctypes.byref(p), _ptr(out), _ptr(dout), _ptr(lse),
                                                 _ptr(sink), _ptr(d_rowsum), _ptr(dsink),
                                                 _stream_ptr(stream))

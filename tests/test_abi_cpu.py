@@ -161,3 +161,41 @@ def test_empty_batch_accepts_null_token_tensors(lib):
                               ws, 16, None) == 1
     assert lib.flint_attn_bwd(ctypes.byref(p), None, None, None, w, w, w, w, None, None,
                               None, None, None, None, w, w, None, ws, 16, None) == 1
+
+
+def test_per_device_setup_flags(tmp_path):
+    """The launchers' per-device set-up flags (device_once.h), compiled and run on
+    the CPU: one set-up per device, independent devices, retry after a failure,
+    no caching outside the table, one set-up under concurrent first calls."""
+    import shutil
+    import subprocess
+    gxx = shutil.which("g++")
+    if gxx is None:
+        pytest.skip("no C++ compiler")
+    exe = tmp_path / "device_once_check"
+    subprocess.run([gxx, "-std=c++17", "-O1", "-Wall", "-Werror", "-pthread",
+                    "-I", os.path.join(ROOT, "sink_aware_sliding_head_b200", "csrc"),
+                    os.path.join(ROOT, "tests", "c", "device_once_check.cpp"), "-o", str(exe)],
+                   check=True)
+    r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert r.returncode == 0, r.stdout + r.stderr
+    assert "device once ok" in r.stdout
+
+
+def test_static_preprocess_validation(lib):
+    """flint_attn_bwd_preprocess_static's argument rules, checked before any launch."""
+    P = ctypes.c_void_p
+    f = lib.flint_attn_bwd_preprocess_static
+    w = P(0x1000)
+
+    def call(p, tok=w):
+        return f(ctypes.byref(p), tok, tok, tok, w, tok, w, None)
+
+    assert call(params(compute_f16=True)) == 1                    # fp16 boundary needs FP32
+    assert call(params(num_q_heads=256, num_kv_heads=4)) == 3     # above the static limit
+    assert call(params(head_dim=64)) == 2
+    assert call(params(), tok=P(0)) == 1                          # null token tensors, T > 0
+    assert call(params(), tok=P(0x1008)) == 1                     # misaligned
+    # T = 0: null token tensors pass validation (the call then needs a device)
+    assert call(params(total_tokens=0), tok=P(0)) in (0, 4)
+    assert f(ctypes.byref(params()), w, w, w, P(0), w, w, None) == 1   # null sink
