@@ -442,6 +442,65 @@ class RowOracle:
         return dx[0, 0], dv
 
 
+    def dkv_rows(self, keys, kv, chunk=256):
+        """``dkv_row`` for several keys of KV head ``kv`` at once.
+
+        The same definition: every query row (i, h) that sees a key contributes
+        p_ij dO_i to dv_j and scale * p_ij (dO_i . v_j - D_i) q_hat_i to dk_hat_j,
+        with p, D_i = dO_i . O_i and O_i from that row's full visible set. The
+        query rows are taken ``chunk`` at a time as one matrix of logits, so keys
+        with thousands of viewing rows stay affordable. Returns (dk, dv) [n, D].
+        """
+        keys = [int(j) for j in keys]
+        G = self.H // self.Hk
+        heads = list(range(kv * G, (kv + 1) * G))
+        # query tokens that see any of the keys
+        rows = set()
+        for j in keys:
+            d0, d1 = _doc_of(self.cu, j)
+            hi = d1 if self.window <= 0 else min(d1, j + self.window)
+            rows.update(range(j, hi))
+        rows = sorted(rows)
+        pairs = [(i, h) for i in rows for h in heads]
+        K, V = self.k_hat_kv[kv], self.v_kv[kv]
+        kidx = np.asarray(keys)
+        dk_hat = np.zeros((len(keys), self.D))
+        dv = np.zeros((len(keys), self.v.shape[-1]))
+        for c0 in range(0, len(pairs), chunk):
+            part = pairs[c0:c0 + chunk]
+            bounds = [visible_keys(i, _doc_of(self.cu, i)[0], self.window) for i, _ in part]
+            lo = min(b[0] for b in bounds)
+            hi = max(b[1] for b in bounds) + 1
+            qh = np.stack([self._q_hat(i, h) for i, h in part])           # [r, D]
+            dO = np.stack([self._dO_row(i, h) for i, h in part])          # [r, D]
+            s_h = np.array([self.sink[h] for _, h in part])
+            z = self.scale * (qh @ K[lo:hi].T)                            # [r, m]
+            col = np.arange(lo, hi)[None, :]
+            vis = (col >= np.array([b[0] for b in bounds])[:, None]) & \
+                  (col <= np.array([b[1] for b in bounds])[:, None])
+            z = np.where(vis, z, -np.inf)
+            m = np.maximum(np.max(z, axis=1), s_h)
+            e = np.exp(z - m[:, None])
+            Z = np.exp(s_h - m) + np.sum(e, axis=1)
+            p = e / Z[:, None]                                            # [r, m]
+            O = p @ V[lo:hi]                                              # [r, D]
+            Di = np.sum(dO * O, axis=1)                                   # [r]
+            inside = (kidx >= lo) & (kidx < hi)
+            for n in np.nonzero(inside)[0]:
+                j = kidx[n]
+                pj = p[:, j - lo]                                         # [r]
+                dv[n] += pj @ dO
+                dz = pj * (dO @ self.v[j, kv] - Di)
+                dk_hat[n] += self.scale * (dz @ qh)
+        dk = np.zeros_like(dk_hat)
+        for n, j in enumerate(keys):
+            dx, _ = prologue_backward(self.k[j:j + 1, kv:kv + 1, :], self.w_k,
+                                      dk_hat[n][None, None, :], self.pos[j:j + 1],
+                                      self.use_rope, self.theta, self.eps)
+            dk[n] = dx[0, 0]
+        return dk, dv
+
+
 # ----------------------------------------------------------------------------
 # Decode: one new token per sequence attending over its KV cache
 # ----------------------------------------------------------------------------

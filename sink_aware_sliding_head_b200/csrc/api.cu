@@ -20,12 +20,13 @@ cudaError_t launch_exp2_poly(const float* x, float* y, int n, cudaStream_t st);
 cudaError_t launch_attn_fwd_sm100_impl(const CUtensorMap& tq, const CUtensorMap& tk,
                                        const CUtensorMap& tv, const Resolved& p, const float* sink,
                                        const int4* items, const int* n_items, int max_items,
-                                       void* out, float* lse, int* status, int num_sms,
-                                       cudaStream_t st);
+                                       const unsigned* amax_v, void* out, float* lse,
+                                       int* status, int num_sms, cudaStream_t st);
 cudaError_t launch_attn_bwd_sm100_impl(const CUtensorMap& tq, const CUtensorMap& tk,
                                        const CUtensorMap& tv, const CUtensorMap& tdo,
                                        const Resolved& p, const float* lse, const float* dvec,
-                                       const int4* items_kv, const int* n_kv, int max_kv,
+                                       const unsigned* amax, const int4* items_kv,
+                                       const int* n_kv, int max_kv,
                                        const int4* items_q, const int* n_q, int max_q,
                                        float* dq_acc, float* dk_acc, void* dv, int* status,
                                        int num_sms, cudaStream_t st);
@@ -36,7 +37,7 @@ const char* const kKernelNames[kNumKernelIds] = {
     "prologue_rmsnorm_rope", "build_worklist", "attn_fwd_sm100", "attn_fwd_fp32",
     "bwd_preprocess", "reduce_rows", "attn_bwd_dkv_sm100", "attn_bwd_dq_sm100",
     "attn_bwd_dq_fp32", "attn_bwd_dkv_fp32", "prologue_bwd", "convert_f16",
-    "decode", "pad_fill"};
+    "decode", "pad_fill", "absmax"};
 constexpr int kMaxSlots = 1 << 15;
 struct Prof {
   std::mutex mu;
@@ -193,11 +194,13 @@ extern "C" size_t flint_attn_workspace_bytes(const flint_attn_params_t* params, 
 
 namespace {
 // fp16 copy of v, the B operand of the PV / P^T dO MMAs
-cudaError_t convert_v(const Resolved& p, const void* v, __half* v16, cudaStream_t st) {
+// amax_v: the max |v| slot; the copy is v * 2^e (pow2_scale_exp).
+cudaError_t convert_v(const Resolved& p, const void* v, __half* v16, const unsigned* amax_v,
+                      cudaStream_t st) {
   const size_t n = (size_t)p.T * p.Hk * kHeadDim;
   if (p.dtype == FLINT_BF16)
-    return launch_convert_f16(static_cast<const __nv_bfloat16*>(v), v16, n, st);
-  return launch_convert_f16(static_cast<const float*>(v), v16, n, st);
+    return launch_convert_f16(static_cast<const __nv_bfloat16*>(v), v16, n, amax_v, st);
+  return launch_convert_f16(static_cast<const float*>(v), v16, n, amax_v, st);
 }
 
 // valid: per-document count of real tokens (trailing padding), or nullptr.
@@ -241,7 +244,9 @@ flint_status_t fwd_impl(const flint_attn_params_t* params, const void* q, const 
   FLINT_TRY(launch_build_worklist(cu_doc_lens, valid, p, kModeQuery, 2 * p.R, items, status + 1,
                                   at<void>(workspace, L.sched_tmp), L.max_items_q, st));
   __half* v16 = at<__half>(workspace, L.v16);
-  FLINT_TRY(convert_v(p, v, v16, st));
+  unsigned* amax = reinterpret_cast<unsigned*>(status + kSlotAmaxDout);   // [dout, v]
+  FLINT_TRY(launch_absmax(p.dtype, nullptr, 0, v, (size_t)p.T * p.Hk * kHeadDim, amax, st));
+  FLINT_TRY(convert_v(p, v, v16, amax + 1, st));
   const CUtensorMapDataType f16t = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
   CUtensorMap tq, tk, tv;
   if (!encode_3d(&tq, qh, p.T, p.H, p.G, p.R, f16t) ||
@@ -249,7 +254,7 @@ flint_status_t fwd_impl(const flint_attn_params_t* params, const void* q, const 
       !encode_3d(&tv, v16, p.T, p.Hk, 1, kTileKeys, f16t))
     return FLINT_ERR_CUDA;
   FLINT_TRY(launch_attn_fwd_sm100_impl(tq, tk, tv, p, sink, items, status + 1, L.max_items_q,
-                                       out, lse, status, sm_count(), st));
+                                       amax + 1, out, lse, status, sm_count(), st));
   if (valid) FLINT_TRY(launch_pad_fill_fwd(p, cu_doc_lens, valid, sink, out, lse, st));
   return FLINT_OK;
 }
@@ -296,9 +301,14 @@ flint_status_t bwd_impl(const flint_attn_params_t* params, const void* q, const 
   const bool f16 = p.tc;   // tensor-core operands of the backward are fp16
   __half* dout16 = f16 ? at<__half>(workspace, L.dout16) : nullptr;
   __half* v16 = f16 ? at<__half>(workspace, L.v16) : nullptr;
+  unsigned* amax = reinterpret_cast<unsigned*>(status + kSlotAmaxDout);   // [dout, v]
+  if (f16)
+    FLINT_TRY(launch_absmax(p.dtype, dout, (size_t)p.T * p.H * kHeadDim, v,
+                            (size_t)p.T * p.Hk * kHeadDim, amax, st));
   FLINT_TRY(launch_prologue(p, q, q_norm_w, qh, p.H, cu_doc_lens, st, f16));
   FLINT_TRY(launch_prologue(p, k, k_norm_w, kh, p.Hk, cu_doc_lens, st, f16));
-  FLINT_TRY(launch_bwd_preprocess(p, out, dout, lse, sink, dvec, part, dsink, dout16, st));
+  FLINT_TRY(launch_bwd_preprocess(p, out, dout, lse, sink, dvec, part, dsink, dout16,
+                                  f16 ? amax : nullptr, st));
   if (!p.tc) {
     FLINT_TRY(launch_attn_bwd_fp32(p, (const float*)qh, (const float*)kh, (const float*)v,
                                    (const float*)dout, lse, dvec, cu_doc_lens, dq_acc, dk_acc,
@@ -311,7 +321,7 @@ flint_status_t bwd_impl(const flint_attn_params_t* params, const void* q, const 
                                     status + 2, tmp, L.max_items_kv, st));
     FLINT_TRY(launch_build_worklist(cu_doc_lens, valid, p, kModeQuery, p.R, items_q1, status + 3,
                                     tmp, L.max_items_q1, st));
-    FLINT_TRY(convert_v(p, v, v16, st));
+    FLINT_TRY(convert_v(p, v, v16, amax + 1, st));
     const CUtensorMapDataType f16t = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
     CUtensorMap tq, tk, tv, tdo;
     if (!encode_3d(&tq, qh, p.T, p.H, p.G, p.R, f16t) ||
@@ -319,8 +329,9 @@ flint_status_t bwd_impl(const flint_attn_params_t* params, const void* q, const 
         !encode_3d(&tv, v16, p.T, p.Hk, 1, kTileKeys, f16t) ||
         !encode_3d(&tdo, dout16, p.T, p.H, p.G, p.R, f16t))
       return FLINT_ERR_CUDA;
-    FLINT_TRY(launch_attn_bwd_sm100_impl(tq, tk, tv, tdo, p, lse, dvec, items_kv, status + 2,
-                                         L.max_items_kv, items_q1, status + 3, L.max_items_q1,
+    FLINT_TRY(launch_attn_bwd_sm100_impl(tq, tk, tv, tdo, p, lse, dvec, amax, items_kv,
+                                         status + 2, L.max_items_kv, items_q1, status + 3,
+                                         L.max_items_q1,
                                          dq_acc, dk_acc, dv, status, sm_count(), st));
     if (valid)
       FLINT_TRY(launch_pad_fill_bwd(p, cu_doc_lens, valid, dq_acc, dk_acc, dv, p.fp32_out, st));

@@ -63,7 +63,8 @@ struct BwdArgs {
   int T, H, Hk, G, R, W, logG;
   float scale, scale_log2;
   const float* lse;
-  const float* dvec;
+  const float* dvec;      // D * s_dout * s_v (the scales of the fp16 operand copies)
+  const unsigned* amax;   // [max |dout|, max |v|] slots (pow2_scale_exp)
   const int4* items;
   const int* n_items;
   int max_items;
@@ -385,6 +386,9 @@ attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_q,
     const int kl = (warp & 3) * 32 + lane;         // key row of the tile = TMEM lane
     const uint32_t t_row = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     const uint32_t c0 = 64 * wg;                   // first column of this warpgroup
+    // dV carries the scale of the fp16 dO copy, dK that of dO and v
+    const float inv_sdo = slot_scale(a.amax, true);
+    const float dk_mul = a.scale * inv_sdo * slot_scale(a.amax + 1, true);
     uint32_t item_count = 0, s_cnt = 0, dp_cnt = 0, tile_count = 0;
     bool ok = true;
     while (ok) {
@@ -503,21 +507,24 @@ attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_q,
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
               const uint32_t* vv = hh ? v1 : v0;
+              float f[32];
+#pragma unroll
+              for (int c = 0; c < 32; ++c) f[c] = __uint_as_float(vv[c]) * inv_sdo;
               if (a.dv_f32) {
                 float* dvrow = reinterpret_cast<float*>(a.dv) + rb + hh * 32;
 #pragma unroll
                 for (int c = 0; c < 32; c += 4)
-                  *reinterpret_cast<uint4*>(dvrow + c) =
-                      make_uint4(vv[c], vv[c + 1], vv[c + 2], vv[c + 3]);
+                  *reinterpret_cast<float4*>(dvrow + c) =
+                      make_float4(f[c], f[c + 1], f[c + 2], f[c + 3]);
               } else {
                 __nv_bfloat16* dvrow = reinterpret_cast<__nv_bfloat16*>(a.dv) + rb + hh * 32;
 #pragma unroll
                 for (int c = 0; c < 32; c += 8) {
                   uint4 pkv;
-                  pkv.x = pack_bf16x2(__uint_as_float(vv[c]), __uint_as_float(vv[c + 1]));
-                  pkv.y = pack_bf16x2(__uint_as_float(vv[c + 2]), __uint_as_float(vv[c + 3]));
-                  pkv.z = pack_bf16x2(__uint_as_float(vv[c + 4]), __uint_as_float(vv[c + 5]));
-                  pkv.w = pack_bf16x2(__uint_as_float(vv[c + 6]), __uint_as_float(vv[c + 7]));
+                  pkv.x = pack_bf16x2(f[c], f[c + 1]);
+                  pkv.y = pack_bf16x2(f[c + 2], f[c + 3]);
+                  pkv.z = pack_bf16x2(f[c + 4], f[c + 5]);
+                  pkv.w = pack_bf16x2(f[c + 6], f[c + 7]);
                   *reinterpret_cast<uint4*>(dvrow + c) = pkv;
                 }
               }
@@ -541,8 +548,8 @@ attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_q,
 #pragma unroll
               for (int c = 0; c < 32; c += 4)
                 *reinterpret_cast<float4*>(dkrow + c) = make_float4(
-                    __uint_as_float(kv[c]) * a.scale, __uint_as_float(kv[c + 1]) * a.scale,
-                    __uint_as_float(kv[c + 2]) * a.scale, __uint_as_float(kv[c + 3]) * a.scale);
+                    __uint_as_float(kv[c]) * dk_mul, __uint_as_float(kv[c + 1]) * dk_mul,
+                    __uint_as_float(kv[c + 2]) * dk_mul, __uint_as_float(kv[c + 3]) * dk_mul);
             }
           }
         }
@@ -774,6 +781,8 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q,
     const int r = (warp & 3) * 32 + lane;          // query row of the tile = TMEM lane
     const uint32_t t_row = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     const int c0 = 64 * wg;
+    // dQ carries the scales of the fp16 dO and v copies
+    const float dq_mul = a.scale * slot_scale(a.amax, true) * slot_scale(a.amax + 1, true);
     uint32_t item_count = 0, t = 0;
     bool ok = true;
     while (ok) {
@@ -879,8 +888,8 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q,
 #pragma unroll
             for (int c = 0; c < 32; c += 4)
               *reinterpret_cast<float4*>(row + hh * 32 + c) = make_float4(
-                  __uint_as_float(uu[c]) * a.scale, __uint_as_float(uu[c + 1]) * a.scale,
-                  __uint_as_float(uu[c + 2]) * a.scale, __uint_as_float(uu[c + 3]) * a.scale);
+                  __uint_as_float(uu[c]) * dq_mul, __uint_as_float(uu[c + 1]) * dq_mul,
+                  __uint_as_float(uu[c + 2]) * dq_mul, __uint_as_float(uu[c + 3]) * dq_mul);
           }
         }
       }
@@ -899,7 +908,8 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q,
 cudaError_t launch_attn_bwd_sm100_impl(const CUtensorMap& tq, const CUtensorMap& tk,
                                        const CUtensorMap& tv, const CUtensorMap& tdo,
                                        const Resolved& p, const float* lse, const float* dvec,
-                                       const int4* items_kv, const int* n_kv, int max_kv,
+                                       const unsigned* amax, const int4* items_kv,
+                                       const int* n_kv, int max_kv,
                                        const int4* items_q, const int* n_q, int max_q,
                                        float* dq_acc, float* dk_acc, void* dv, int* status,
                                        int num_sms, cudaStream_t st) {
@@ -914,7 +924,7 @@ cudaError_t launch_attn_bwd_sm100_impl(const CUtensorMap& tq, const CUtensorMap&
   while ((1 << a.logG) < p.G) ++a.logG;
   a.scale = p.scale;
   a.scale_log2 = p.scale * kLog2e;
-  a.lse = lse; a.dvec = dvec;
+  a.lse = lse; a.dvec = dvec; a.amax = amax;
   a.dq_acc = dq_acc; a.dk_acc = dk_acc;
   a.dv = dv;
   a.dv_f32 = p.fp32_out || p.dtype == FLINT_FP32;

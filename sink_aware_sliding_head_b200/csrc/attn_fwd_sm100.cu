@@ -66,6 +66,7 @@ struct FwdArgs {
   const int4* items;
   const int* n_items;
   int max_items;
+  const unsigned* amax_v;   // max |v| slot: the fp16 copy of v is v * 2^e
   void* out;        // bf16, float (out_f32) or fp16 (out_f16)
   int out_f32, out_f16;
   float* lse;
@@ -334,6 +335,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
     const int r = wq * 32 + lane;          // row of the tile = TMEM lane
     const uint32_t t_row = tmem + ((uint32_t)(wq * 32) << 16);
     const uint32_t s_col = i * 128, o_col = 256 + i * 128;
+    const float inv_sv = slot_scale(a.amax_v, true);
     uint32_t s_count = 0, item_count = 0;
     bool ok = true;
     for (int idx = blockIdx.x; idx < n_items && ok; idx += gridDim.x) {
@@ -463,7 +465,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->o_full[i]), item_count & 1, wc));
       if (!ok) break;
       tc_fence_after();
-      const float inv_l = 1.f / l;
+      const float inv_l = inv_sv / l;   // 1/l, and the scale of the fp16 copy of v
       const uint64_t il2 = f2(inv_l, inv_l);
       const size_t obase = ((size_t)tok * a.H + h) * kHeadDim;
 #pragma unroll
@@ -526,8 +528,8 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
 cudaError_t launch_attn_fwd_sm100_impl(const CUtensorMap& tq, const CUtensorMap& tk,
                                        const CUtensorMap& tv, const Resolved& p, const float* sink,
                                        const int4* items, const int* n_items, int max_items,
-                                       void* out, float* lse, int* status, int num_sms,
-                                       cudaStream_t st) {
+                                       const unsigned* amax_v, void* out, float* lse,
+                                       int* status, int num_sms, cudaStream_t st) {
   static PerDeviceOnce smem_once;
   cudaError_t e = smem_limit_once(smem_once, attn_fwd_sm100_kernel, kSmemBytes);
   if (e != cudaSuccess) return e;
@@ -535,6 +537,7 @@ cudaError_t launch_attn_fwd_sm100_impl(const CUtensorMap& tq, const CUtensorMap&
   a.T = p.T; a.H = p.H; a.Hk = p.Hk; a.G = p.G; a.R = p.R; a.W = p.W;
   a.scale_log2 = p.scale * kLog2e;
   a.sink = sink; a.items = items; a.n_items = n_items; a.max_items = max_items;
+  a.amax_v = amax_v;
   a.out = out;
   a.out_f32 = p.fp32_out && !p.out_f16;
   a.out_f16 = p.out_f16;

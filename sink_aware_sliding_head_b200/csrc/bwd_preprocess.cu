@@ -24,15 +24,19 @@ constexpr int kTok = 4;
 
 // Also writes an fp16 copy of dO (dout16, when non-null): the tensor-core
 // backward's operands are fp16.
+// amax (nullable): [max|dout|, max|v|] slots; dout16 gets dout * s_dout and dvec
+// D * s_dout * s_v, the scales of the fp16 operands (d_sink uses the plain D).
 template <typename TO, typename T>
 __global__ void __launch_bounds__(kThreads)
 bwd_pre_kernel(const TO* __restrict__ out, const T* __restrict__ dout,
                const float* __restrict__ lse, const float* __restrict__ sink,
                float* __restrict__ dvec, float* __restrict__ part, __half* __restrict__ dout16,
-               int ntok, int H) {
+               const unsigned* __restrict__ amax, int ntok, int H) {
   extern __shared__ float acc[];   // [kGroups][H]
   const int lane16 = threadIdx.x & 15, grp = threadIdx.x >> 4;
   const int c0 = lane16 * 8;
+  const float s_do = slot_scale(amax, false);
+  const float s_d = s_do * slot_scale(amax ? amax + 1 : nullptr, false);
   for (int e = threadIdx.x; e < kGroups * H; e += kThreads) acc[e] = 0.f;
   __syncthreads();
   const int rows = kTok * H;
@@ -50,7 +54,7 @@ bwd_pre_kernel(const TO* __restrict__ out, const T* __restrict__ dout,
         if (dout16) {
           float s8[8];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) s8[e] = sat_f16(b[e]);
+          for (int e = 0; e < 8; ++e) s8[e] = sat_f16(b[e] * s_do);
           store8(dout16 + base, s8);
         }
       } else {
@@ -63,7 +67,7 @@ bwd_pre_kernel(const TO* __restrict__ out, const T* __restrict__ dout,
 #pragma unroll
       for (int o = 8; o >= 1; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
       if (valid && lane16 == 0) {
-        dvec[(size_t)h * ntok + t] = d;
+        dvec[(size_t)h * ntok + t] = d * s_d;
         acc[grp * H + h] -= expf(sink[h] - lse[(size_t)h * ntok + t]) * d;
       }
     }
@@ -76,17 +80,52 @@ bwd_pre_kernel(const TO* __restrict__ out, const T* __restrict__ dout,
   }
 }
 
-// dst[i] = fp16(src[i]) for n elements (n a multiple of 8), saturating at +-65504.
+// dst[i] = fp16(src[i] * 2^e) for n elements (n a multiple of 8), e from the
+// max |src| slot (nullptr: e = 0); saturating at +-65504.
 template <typename T>
 __global__ void convert_f16_kernel(const T* __restrict__ src, __half* __restrict__ dst,
-                                   size_t n8) {
+                                   size_t n8, const unsigned* __restrict__ amax) {
+  const float sc = slot_scale(amax, false);
   for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n8;
        i += (size_t)gridDim.x * blockDim.x) {
     float f[8];
     load8(src + 8 * i, f);
 #pragma unroll
-    for (int e = 0; e < 8; ++e) f[e] = sat_f16(f[e]);
+    for (int e = 0; e < 8; ++e) f[e] = sat_f16(f[e] * sc);
     store8(dst + 8 * i, f);
+  }
+}
+
+// Largest magnitude of two tensors (8 elements per thread and step), one
+// atomicMax per block and tensor on the float bit patterns.
+template <typename T>
+__global__ void __launch_bounds__(256)
+absmax_kernel(const T* __restrict__ x0, size_t n0_8, const T* __restrict__ x1, size_t n1_8,
+              unsigned* __restrict__ amax) {
+  __shared__ float red[2][8];
+  float m0 = 0.f, m1 = 0.f;
+  const size_t stride = (size_t)gridDim.x * blockDim.x;
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n0_8 + n1_8; i += stride) {
+    float f[8];
+    const bool first = i < n0_8;
+    load8(first ? x0 + 8 * i : x1 + 8 * (i - n0_8), f);
+    float m = 0.f;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) m = fmaxf(m, fabsf(f[e]));
+    if (first) m0 = fmaxf(m0, m); else m1 = fmaxf(m1, m);
+  }
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) {
+    m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, o));
+    m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, o));
+  }
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) { red[0][warp] = m0; red[1][warp] = m1; }
+  __syncthreads();
+  if (threadIdx.x < 2) {
+    float m = 0.f;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) m = fmaxf(m, red[threadIdx.x][w]);
+    if (m > 0.f) atomicMax(amax + threadIdx.x, __float_as_uint(m));
   }
 }
 
@@ -108,25 +147,46 @@ cudaError_t launch_exp2_poly(const float* x, float* y, int n, cudaStream_t st) {
 }
 
 template <typename T>
-static cudaError_t convert_f16(const T* src, __half* dst, size_t n, cudaStream_t st) {
+static cudaError_t convert_f16(const T* src, __half* dst, size_t n, const unsigned* amax,
+                               cudaStream_t st) {
   const size_t n8 = n / 8;
   if (n8 == 0) return cudaSuccess;
   size_t blocks = (n8 + 255) / 256;
   if (blocks > 148 * 16) blocks = 148 * 16;
   ProfScope prof(kKConvert, st);
-  convert_f16_kernel<T><<<(unsigned)blocks, 256, 0, st>>>(src, dst, n8);
+  convert_f16_kernel<T><<<(unsigned)blocks, 256, 0, st>>>(src, dst, n8, amax);
   return cudaGetLastError();
 }
-cudaError_t launch_convert_f16(const __nv_bfloat16* src, __half* dst, size_t n, cudaStream_t st) {
-  return convert_f16(src, dst, n, st);
+cudaError_t launch_convert_f16(const __nv_bfloat16* src, __half* dst, size_t n,
+                               const unsigned* amax, cudaStream_t st) {
+  return convert_f16(src, dst, n, amax, st);
 }
-cudaError_t launch_convert_f16(const float* src, __half* dst, size_t n, cudaStream_t st) {
-  return convert_f16(src, dst, n, st);
+cudaError_t launch_convert_f16(const float* src, __half* dst, size_t n, const unsigned* amax,
+                               cudaStream_t st) {
+  return convert_f16(src, dst, n, amax, st);
+}
+
+cudaError_t launch_absmax(int dtype, const void* x0, size_t n0, const void* x1, size_t n1,
+                          unsigned* amax, cudaStream_t st) {
+  const size_t n0_8 = x0 ? n0 / 8 : 0, n1_8 = x1 ? n1 / 8 : 0;
+  if (n0_8 + n1_8 == 0) return cudaSuccess;
+  size_t blocks = (n0_8 + n1_8 + 255) / 256;
+  if (blocks > 148 * 8) blocks = 148 * 8;
+  ProfScope prof(kKAbsmax, st);
+  if (dtype == FLINT_BF16)
+    absmax_kernel<__nv_bfloat16><<<(unsigned)blocks, 256, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(x0), n0_8, static_cast<const __nv_bfloat16*>(x1),
+        n1_8, amax);
+  else
+    absmax_kernel<float><<<(unsigned)blocks, 256, 0, st>>>(
+        static_cast<const float*>(x0), n0_8, static_cast<const float*>(x1), n1_8, amax);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_bwd_preprocess(const Resolved& p, const void* out, const void* dout,
                                   const float* lse, const float* sink, float* dvec, float* part,
-                                  float* dsink, __half* dout16, cudaStream_t st) {
+                                  float* dsink, __half* dout16, const unsigned* amax,
+                                  cudaStream_t st) {
   if (p.T == 0) {
     cudaMemsetAsync(dsink, 0, p.H * sizeof(float), st);
     return cudaGetLastError();
@@ -139,17 +199,17 @@ cudaError_t launch_bwd_preprocess(const Resolved& p, const void* out, const void
   typedef __nv_bfloat16 bf;
   if (p.dtype == FLINT_BF16 && p.fp32_out)
     bwd_pre_kernel<float, bf><<<blocks, kThreads, smem, st>>>(
-        (const float*)out, (const bf*)dout, lse, sink, dvec, part, dout16, p.T, p.H);
+        (const float*)out, (const bf*)dout, lse, sink, dvec, part, dout16, amax, p.T, p.H);
   else if (p.dtype == FLINT_BF16)
     bwd_pre_kernel<bf, bf><<<blocks, kThreads, smem, st>>>(
-        (const bf*)out, (const bf*)dout, lse, sink, dvec, part, dout16, p.T, p.H);
+        (const bf*)out, (const bf*)dout, lse, sink, dvec, part, dout16, amax, p.T, p.H);
   else if (p.out_f16)   // FP32 inputs at the fp16 compute boundary: out is fp16
     bwd_pre_kernel<__half, float><<<blocks, kThreads, smem, st>>>(
-        (const __half*)out, (const float*)dout, lse, sink, dvec, part, dout16, p.T, p.H);
+        (const __half*)out, (const float*)dout, lse, sink, dvec, part, dout16, amax, p.T, p.H);
   else
     bwd_pre_kernel<float, float><<<blocks, kThreads, smem, st>>>(
         (const float*)out, (const float*)dout, lse, sink, dvec, part, p.tc ? dout16 : nullptr,
-        p.T, p.H);
+        p.tc ? amax : nullptr, p.T, p.H);
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;

@@ -27,6 +27,37 @@ enum : int {
   kStatusTimeoutSelftest = 32, // the bounded-wait self-test's wait ran out
 };
 
+// int slots of the workspace's status region (int[64], zeroed at the start of
+// every call): [0] status bits, [1..3] work-list lengths, [4..5] dynamic item
+// counters, [8] and [9] the bit patterns of max |dout| and max |v|.
+enum : int { kSlotAmaxDout = 8, kSlotAmaxV = 9 };
+
+// Operand range of the fp16 tensor-core copies of dout and v. Each copy is
+// multiplied by a power of two 2^e chosen from the tensor's largest magnitude,
+// so that it lands in [4, 8) - the range of the N(0,1) data the kernels are
+// tuned and tested on - and can neither saturate at fp16's 65504 nor lose
+// precision in fp16's subnormal range (below 6.1e-5). Multiplying by a power
+// of two is exact, and the FP32 epilogues divide it out again. amax_bits is
+// the bit pattern of max |x| (non-negative floats order like their bits); an
+// all-zero tensor gets e = 0.
+__host__ __device__ inline int pow2_scale_exp(unsigned amax_bits) {
+  if (amax_bits == 0) return 0;
+  const int E = (int)((amax_bits >> 23) & 0xff);   // floor(log2 max|x|) + 127 (normal)
+  int e = 129 - E;                                  // max|x| * 2^e in [4, 8)
+  return e < -126 ? -126 : (e > 126 ? 126 : e);
+}
+__host__ __device__ inline float exp2_int(int e) {   // 2^e for -126 <= e <= 127
+  union { unsigned u; float f; } c;
+  c.u = (unsigned)(e + 127) << 23;
+  return c.f;
+}
+// 2^e read from a device slot written by launch_absmax (nullptr: 1).
+__device__ __forceinline__ float slot_scale(const unsigned* amax, bool inverse) {
+  if (!amax) return 1.f;
+  const int e = pow2_scale_exp(*reinterpret_cast<const volatile unsigned*>(amax));
+  return exp2_int(inverse ? -e : e);
+}
+
 // Parameters after validation and defaulting.
 struct Resolved {
   int T, N, H, Hk, D, G, W, rope;
@@ -170,6 +201,7 @@ __device__ __forceinline__ void store8(float* p, const float (&f)[8]) {
 enum KernelId {
   kKPrologue = 0, kKWorklist, kKFwdSm100, kKFwdFp32, kKBwdPre, kKReduce, kKBwdDkvSm100,
   kKBwdDqSm100, kKBwdDqFp32, kKBwdDkvFp32, kKPrologueBwd, kKConvert, kKDecode, kKPadFill,
+  kKAbsmax,
   kNumKernelIds
 };
 struct ProfScope {
@@ -196,8 +228,16 @@ cudaError_t launch_pad_fill_bwd(const Resolved& p, const int32_t* cu, const int3
 // out_f16: write x_hat as fp16 (backward operands of BF16 inputs) instead of the input type
 cudaError_t launch_prologue(const Resolved& p, const void* x, const void* w, void* y, int heads,
                             const int32_t* cu, cudaStream_t st, bool out_f16 = false);
-cudaError_t launch_convert_f16(const __nv_bfloat16* src, __half* dst, size_t n, cudaStream_t st);
-cudaError_t launch_convert_f16(const float* src, __half* dst, size_t n, cudaStream_t st);
+// dst = fp16(src * 2^e), e from the max |src| in *amax (nullptr: e = 0).
+cudaError_t launch_convert_f16(const __nv_bfloat16* src, __half* dst, size_t n,
+                               const unsigned* amax, cudaStream_t st);
+cudaError_t launch_convert_f16(const float* src, __half* dst, size_t n, const unsigned* amax,
+                               cudaStream_t st);
+// amax[0] = bits of max |x0| over n0 elements, amax[1] = bits of max |x1| over n1
+// (both raised with atomicMax, so the slots must start at zero); x0 or x1 may be
+// null (n = 0). n0, n1 multiples of 8. dtype: FLINT_BF16 or FLINT_FP32 for both.
+cudaError_t launch_absmax(int dtype, const void* x0, size_t n0, const void* x1, size_t n1,
+                          unsigned* amax, cudaStream_t st);
 // Bounded-wait self-test (selftest.cu): status[0] gets the timeout bit, status[1]
 // 1 if the wait completed and 0 if it gave up.
 cudaError_t launch_wait_selftest(long long limit, int arrive_first, int* status,
@@ -227,23 +267,17 @@ cudaError_t launch_attn_bwd_fp32(const Resolved& p, const float* qh, const float
                                  const float* v, const float* dout, const float* lse,
                                  const float* dvec, const int32_t* cu, float* dq_acc,
                                  float* dk_acc, float* dv, cudaStream_t st);
+// D = rowsum(dout * out) into dvec, d_sink, and (dout16 non-null) the fp16 copy of
+// dout. amax (nullable): the [max|dout|, max|v|] slots; when given, dout16 is
+// dout * s_dout and dvec holds D * s_dout * s_v (the scales of the fp16
+// operands), while d_sink is formed from the unscaled D.
 cudaError_t launch_bwd_preprocess(const Resolved& p, const void* out, const void* dout,
                                   const float* lse, const float* sink, float* dvec, float* part,
-                                  float* dsink, __half* dout16, cudaStream_t st);
+                                  float* dsink, __half* dout16, const unsigned* amax,
+                                  cudaStream_t st);
 cudaError_t launch_bwd_epilogue(const Resolved& p, const void* x, const void* w,
                                 const float* g_hat, void* dx, float* dw, float* part, int heads,
                                 const int32_t* cu, cudaStream_t st);
-cudaError_t launch_attn_fwd_sm100(const Resolved& p, const void* qh, const void* kh,
-                                  const void* v, const float* sink, const int4* items,
-                                  const int* n_items, int max_items, void* out, float* lse,
-                                  int* status, int num_sms, cudaStream_t st);
-cudaError_t launch_attn_bwd_sm100(const Resolved& p, const void* qh, const void* kh,
-                                  const void* v, const void* dout, const float* lse,
-                                  const float* dvec, const int4* items_kv, const int* n_kv,
-                                  int max_kv, const int4* items_q, const int* n_q, int max_q,
-                                  float* dq_acc, float* dk_acc, void* dv, int* status,
-                                  int num_sms, cudaStream_t st);
-
 enum { kModeQuery = 0, kModeKey = 1 };
 
 // Raises a kernel's dynamic shared-memory limit on the current device the

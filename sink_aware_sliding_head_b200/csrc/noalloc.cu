@@ -102,6 +102,6 @@ extern "C" flint_status_t flint_attn_bwd_preprocess_static(const flint_attn_para
   float* scratch = nullptr;
   if (scratch_on_current_device(&scratch) != cudaSuccess) return FLINT_ERR_CUDA;
   cudaError_t e = launch_bwd_preprocess(p, out, dout, lse, sink, d_rowsum, scratch, dsink,
-                                        nullptr, reinterpret_cast<cudaStream_t>(stream));
+                                        nullptr, nullptr, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? FLINT_OK : FLINT_ERR_CUDA;
 }

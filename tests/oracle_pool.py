@@ -1,0 +1,41 @@
+"""Whole-layer oracle comparisons split by document, run in worker processes.
+
+Test infrastructure. Documents of a THD pack are independent (positions restart
+per document, attention never crosses a boundary; the oracle pins check this
+pack invariance for the forward and the backward), so the FP64 oracle of a
+packed layer is the oracle of each document on its own, with d_sink and the
+norm-weight gradients summed over documents. Each worker evaluates one document
+and compares it with the GPU's rows there, returning only error statistics, so
+multi-GB layers stay affordable. Start the pool with the ``spawn`` method.
+"""
+import numpy as np
+from threadpoolctl import threadpool_limits
+
+from oracle import flint_oracle as fo
+
+ELEMENTWISE = ("out", "lse", "dq", "dk", "dv")
+SUMS = ("dsink", "dw_q", "dw_k")
+
+
+def doc_check(task):
+    """task: (inputs of one document as float32 arrays, GPU results for its rows,
+    window, use_rope, rope_theta). Returns ({name: (max_abs, sum_err2, sum_ref2,
+    n_nonfinite)}, {sum name: this document's oracle value})."""
+    inp, gpu, window, rope, theta = task
+    L = inp["q"].shape[0]
+    cu = np.array([0, L])
+    with threadpool_limits(limits=2):     # the pool already runs one document per core
+        O, lse = fo.flint_attn_fwd(inp["q"], inp["k"], inp["v"], inp["w_q"], inp["w_k"],
+                                   inp["sink"], cu, window, rope, theta)
+        R = fo.flint_attn_bwd(inp["q"], inp["k"], inp["v"], inp["w_q"], inp["w_k"],
+                              inp["sink"], cu, window, rope, theta, inp["dout"])
+    ref = {"out": O, "lse": lse, "dq": R["dq"], "dk": R["dk"], "dv": R["dv"]}
+    stats = {}
+    for name in ELEMENTWISE:
+        g = np.asarray(gpu[name], dtype=np.float64)
+        r = ref[name]
+        bad = int(np.sum(~np.isfinite(g)))
+        err = g - r
+        stats[name] = (float(np.max(np.abs(err))) if err.size else 0.0,
+                       float(np.sum(err * err)), float(np.sum(r * r)), bad)
+    return stats, {name: R[name] for name in SUMS}

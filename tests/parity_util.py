@@ -68,11 +68,24 @@ DSINK_REL = 2e-4
 DW_REL = 2e-3
 
 
-def check_grads(g, ref, dtype="bf16"):
+def report_sums(g, ref, label=""):
+    """Print the raw errors of the row sums (d_sink, dw_q, dw_k) against the plain
+    2e-2 bar, whatever bar the test asserts (run pytest with -s to see them)."""
+    for name in ["dsink", "dw_q", "dw_k"]:
+        err = f64(g[name]) - np.asarray(ref[name], np.float64)
+        mx = float(np.max(np.abs(err)))
+        rms = float(np.sqrt(np.mean(err ** 2)) / max(np.sqrt(np.mean(np.square(ref[name]))), 1e-300))
+        print(f"SUMS {label} {name}: max_abs {mx:.3e} ({mx / BF16_MAX_ABS:.2f} of 2e-2), "
+              f"rel_rms {rms:.2e}, max|ref| {float(np.max(np.abs(ref[name]))):.3e}", flush=True)
+
+
+def check_grads(g, ref, dtype="bf16", label=""):
     """Elementwise gradients at the stated bar; d_sink and norm-weight gradients as sums."""
     for name in ["dq", "dk", "dv"]:
         compare(g[name], ref[name], dtype, name)
     bf = dtype == "bf16"
+    if bf:
+        report_sums(g, ref, label)
     compare(g["dsink"], ref["dsink"], dtype, "dsink", reduction=DSINK_REL if bf else 0.0)
     for name in ["dw_q", "dw_k"]:
         compare(g[name], ref[name], dtype, name, reduction=DW_REL if bf else 0.0)

@@ -214,6 +214,28 @@ def test_pack_invariance():
     np.testing.assert_allclose(lse[:, a:b], la, atol=1e-13)
 
 
+def test_pack_invariance_backward():
+    """Per-document gradients equal the packed layer's rows, and d_sink / the norm-weight
+    gradients of the pack are the sums over its documents (what the per-document
+    whole-layer comparisons in the GPU tests rely on)."""
+    H, Hk, D = 4, 2, 16
+    q, k, v, wq, wk, sink, cu, dO = rand_case([9, 0, 21, 6], H, Hk, D, seed=9)
+    g = fo.flint_attn_bwd(q, k, v, wq, wk, sink, cu, 8, True, 1e4, dO)
+    sums = {n: np.zeros_like(g[n]) for n in ("dsink", "dw_q", "dw_k")}
+    cu = [int(c) for c in cu]
+    for a, b in zip(cu[:-1], cu[1:]):
+        if b == a:
+            continue
+        gd = fo.flint_attn_bwd(q[a:b], k[a:b], v[a:b], wq, wk, sink, np.array([0, b - a]), 8,
+                               True, 1e4, dO[a:b])
+        for n in ("dq", "dk", "dv"):
+            np.testing.assert_allclose(gd[n], g[n][a:b], atol=1e-13)
+        for n in sums:
+            sums[n] += gd[n]
+    for n in sums:
+        np.testing.assert_allclose(sums[n], g[n], atol=1e-12)
+
+
 # --------------------------------------------------------------------------
 # GQA
 # --------------------------------------------------------------------------
@@ -340,6 +362,22 @@ def test_row_oracle_matches_whole_layer():
             dk, dv = ro.dkv_row(j, kv)
             np.testing.assert_allclose(dk, g["dk"][j, kv], atol=1e-12)
             np.testing.assert_allclose(dv, g["dv"][j, kv], atol=1e-12)
+
+
+def test_row_oracle_batched_key_rows_match_whole_layer():
+    """RowOracle.dkv_rows (query rows taken as chunks of a logit matrix) equals the
+    whole-layer backward, for keys seen by many rows, small chunks included."""
+    H, Hk, D = 4, 2, 16
+    q, k, v, wq, wk, sink, cu, dO = rand_case([40, 0, 33], H, Hk, D, seed=41)
+    for W, rope in [(9, True), (0, False)]:
+        g = fo.flint_attn_bwd(q, k, v, wq, wk, sink, cu, W, rope, 1e4, dO)
+        ro = fo.RowOracle(q, k, v, wq, wk, sink, cu, W, rope, 1e4, dO=dO)
+        keys = [0, 5, 39, 40, 41, 72]
+        for kv in range(Hk):
+            for chunk in (3, 64, 1000):
+                dk, dv = ro.dkv_rows(keys, kv, chunk=chunk)
+                np.testing.assert_allclose(dk, g["dk"][keys, kv], atol=1e-12)
+                np.testing.assert_allclose(dv, g["dv"][keys, kv], atol=1e-12)
 
 
 def test_config_constants_golden():

@@ -1,0 +1,119 @@
+"""Full-size parity beyond sampled rows.
+
+* The packed THD sliding layer (65536 tokens, W = 1024) forward and backward,
+  every element of out, LSE, dq, dk, dv and d_sink / the norm-weight gradients
+  over all tokens, against the whole-layer FP64 oracle (evaluated per document
+  in worker processes; see oracle_pool.py).
+* The S = 32768 full-causal forward on 4096 rows that cover every row position
+  of the kernel's tile pair (32 tokens x 8 heads of a KV group) at many points
+  of the sequence.
+* The S = 131072 full-causal backward on key rows that 1000-2000 query tokens
+  (x 8 heads) see, so long dK/dV accumulations are compared at full size.
+All run through the C ABI in the launch configuration bench.py times.
+"""
+import multiprocessing as mp
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import flint_inputs as fi
+import oracle_pool
+from oracle import flint_oracle as fo
+from parity_util import (BF16_MAX_ABS, BF16_REL_RMS, DSINK_REL, DW_REL, compare, report_sums,
+                         run_bwd, run_fwd, to_dev)
+
+pytestmark = pytest.mark.gpu
+
+
+def _np32(t):
+    return t.detach().to("cpu", torch.float32).numpy()
+
+
+def test_packed_whole_layer_every_element(cuda_lib):
+    wl = fi.PACKED_BF16
+    cpu = fi.make_inputs(wl)
+    d = to_dev(cpu)
+    out, lse = run_fwd(cuda_lib, d, wl.window, wl.use_rope, wl.rope_theta, fp32_out=True)
+    g = run_bwd(cuda_lib, d, out, lse, wl.window, wl.use_rope, wl.rope_theta)
+    torch.cuda.synchronize()
+    gpu = {"out": out, "lse": lse, "dq": g["dq"], "dk": g["dk"], "dv": g["dv"]}
+    cu = [int(c) for c in cpu["cu_doc_lens"]]
+    tasks = []
+    for a, b in zip(cu[:-1], cu[1:]):
+        if b == a:
+            continue
+        inp = {n: _np32(cpu[n][a:b]) for n in ("q", "k", "v", "dout")}
+        inp.update({n: _np32(cpu[n]) for n in ("w_q", "w_k", "sink")})
+        res = {n: _np32(gpu[n][a:b]) for n in ("out", "dq", "dk", "dv")}
+        res["lse"] = _np32(lse[:, a:b])
+        tasks.append((inp, res, wl.window, wl.use_rope, wl.rope_theta))
+    tasks.sort(key=lambda t: -t[0]["q"].shape[0])          # longest documents first
+    workers = max(1, min(len(tasks), os.cpu_count() or 1, 16))
+    with mp.get_context("spawn").Pool(workers) as pool:
+        results = pool.map(oracle_pool.doc_check, tasks, chunksize=1)
+    for name in oracle_pool.ELEMENTWISE:
+        mx = max(r[0][name][0] for r in results)
+        e2 = sum(r[0][name][1] for r in results)
+        r2 = sum(r[0][name][2] for r in results)
+        bad = sum(r[0][name][3] for r in results)
+        rel = float(np.sqrt(e2 / r2))
+        print(f"WHOLE packed {name}: max_abs {mx:.3e} rel_rms {rel:.2e}", flush=True)
+        assert bad == 0, f"{name}: {bad} non-finite values"
+        assert mx <= BF16_MAX_ABS, f"{name}: max_abs {mx:.3e}"
+        assert rel <= BF16_REL_RMS, f"{name}: rel_rms {rel:.3e}"
+    ref = {n: sum(r[1][n] for r in results) for n in oracle_pool.SUMS}
+    report_sums(g, ref, "packed whole layer")
+    compare(g["dsink"], ref["dsink"], "bf16", "dsink", reduction=DSINK_REL)
+    for name in ("dw_q", "dw_k"):
+        compare(g[name], ref[name], "bf16", name, reduction=DW_REL)
+
+
+def tile_position_rows(T, H, G=8, pair_tokens=32, per_position=16, seed=7):
+    """(token, head) rows covering every (token mod 32, head mod 8) position of the
+    forward's tile pair, each at per_position places spread over the sequence."""
+    rng = np.random.default_rng(seed)
+    rows = []
+    n_pairs = T // pair_tokens
+    for off in range(pair_tokens):
+        for hm in range(G):
+            bases = rng.choice(n_pairs, size=per_position, replace=False)
+            for b in bases:
+                rows.append((int(b) * pair_tokens + off, int(rng.integers(0, H // G)) * G + hm))
+    return rows
+
+
+def test_full_forward_every_tile_position(cuda_lib):
+    wl = fi.FULL_BF16
+    cpu = fi.make_inputs(wl, with_grad_out=False)
+    d = to_dev(cpu)
+    out, lse = run_fwd(cuda_lib, d, wl.window, wl.use_rope, wl.rope_theta)
+    torch.cuda.synchronize()
+    rows = tile_position_rows(wl.total_tokens, wl.num_q_heads)
+    assert len(rows) == 4096
+    ro = fo.RowOracle(cpu["q"], cpu["k"], cpu["v"], cpu["w_q"], cpu["w_k"], cpu["sink"],
+                      cpu["cu_doc_lens"], wl.window, wl.use_rope, wl.rope_theta)
+    ref = [ro.forward_row(t, h) for t, h in rows]
+    idx_t = torch.tensor([t for t, _ in rows], device=out.device)
+    idx_h = torch.tensor([h for _, h in rows], device=out.device)
+    compare(out[idx_t, idx_h], np.stack([r[0] for r in ref]), "bf16", "out rows",
+            out_bf16=True)
+    compare(lse[idx_h, idx_t], np.array([r[1] for r in ref]), "bf16", "lse rows")
+
+
+def test_long_backward_keys_with_many_viewers(cuda_lib):
+    wl = fi.LONG_FULL_BF16
+    cpu = fi.make_inputs(wl)
+    d = to_dev(cpu)
+    out, lse = run_fwd(cuda_lib, d, wl.window, wl.use_rope, wl.rope_theta, fp32_out=True)
+    g = run_bwd(cuda_lib, d, out, lse, wl.window, wl.use_rope, wl.rope_theta)
+    torch.cuda.synchronize()
+    T = wl.total_tokens
+    keys = [T - 1000, T - 1001, T - 1500, T - 2000]       # 1000-2000 viewing tokens x 8 heads
+    ro = fo.RowOracle(cpu["q"], cpu["k"], cpu["v"], cpu["w_q"], cpu["w_k"], cpu["sink"],
+                      cpu["cu_doc_lens"], wl.window, wl.use_rope, wl.rope_theta, dO=cpu["dout"])
+    for kv in (0, wl.num_kv_heads - 1):
+        dk, dv = ro.dkv_rows(keys, kv)
+        compare(g["dk"][keys, kv], dk, "bf16", f"dk rows kv{kv}")
+        compare(g["dv"][keys, kv], dv, "bf16", f"dv rows kv{kv}")
