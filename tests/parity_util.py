@@ -61,11 +61,19 @@ def run_fwd(fa, d, window, rope, theta, check=True, fp32_out=False):
                   window, rope, theta, check_status=check, fp32_out=fp32_out)
 
 
-# Sums over rows (BF16 inputs, 16-bit tensor-core operands): the per-row
-# relative error of the logits and of normalising fp16 P by an FP32 sum is
-# ~2^-12, of the fp16 dq_hat/dk_hat rows ~1e-3, so these bars scale with size.
+# Sums over rows (BF16 inputs, 16-bit tensor-core operands).
+# d_sink is held to the plain bar (max-abs 2e-2) except on the degenerate W = 1
+# layer, where |d_sink| reaches ~166 and the measured max-abs error is 2.5e-2:
+# there the bar is 2e-2 + DSINK_REL * max|d_sink|.
+# dw_q and dw_k sum g * x * r over all T * H rows; their relative error is
+# that of the dq_hat / dk_hat rows (rel-RMS ~5e-4, the fp16 operands' unit
+# roundoff 2^-11 = 4.9e-4), so on values of 30-300 the plain 2e-2 is out of
+# reach for any 16-bit-operand kernel (measured max-abs 1e-2 .. 0.156, i.e.
+# 0.5x .. 7.8x the plain bar, rel-RMS <= 6.3e-4 in every case). They are held
+# to 2e-2 + DW_REL * max|dw| (DW_REL about twice that unit roundoff) and
+# rel-RMS 1e-2; report_sums prints the raw errors next to the plain bar.
 DSINK_REL = 2e-4
-DW_REL = 2e-3
+DW_REL = 1e-3
 
 
 def report_sums(g, ref, label=""):
@@ -79,14 +87,16 @@ def report_sums(g, ref, label=""):
               f"rel_rms {rms:.2e}, max|ref| {float(np.max(np.abs(ref[name]))):.3e}", flush=True)
 
 
-def check_grads(g, ref, dtype="bf16", label=""):
-    """Elementwise gradients at the stated bar; d_sink and norm-weight gradients as sums."""
+def check_grads(g, ref, dtype="bf16", label="", window=None):
+    """Elementwise gradients and d_sink at the stated bar (d_sink: size-scaled only
+    for window == 1); norm-weight gradients as sums over all rows (see DW_REL)."""
     for name in ["dq", "dk", "dv"]:
         compare(g[name], ref[name], dtype, name)
     bf = dtype == "bf16"
     if bf:
         report_sums(g, ref, label)
-    compare(g["dsink"], ref["dsink"], dtype, "dsink", reduction=DSINK_REL if bf else 0.0)
+    compare(g["dsink"], ref["dsink"], dtype, "dsink",
+            reduction=DSINK_REL if (bf and window == 1) else 0.0)
     for name in ["dw_q", "dw_k"]:
         compare(g[name], ref[name], dtype, name, reduction=DW_REL if bf else 0.0)
 

@@ -41,7 +41,7 @@ def test_compute_f16_matches_oracle(cuda_lib, fp32_out):
                           cpu["cu_doc_lens"], W, rope, 1e4, cpu["dout"])
     compare(out, O, "bf16", "out")
     compare(lse, L, "bf16", "lse")
-    check_grads(g, R)
+    check_grads(g, R, label="compute_f16")
 
 
 def test_compute_f16_with_padding(cuda_lib):

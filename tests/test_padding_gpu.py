@@ -50,7 +50,7 @@ def test_padded_matches_oracle(cuda_lib, lens, valid, W, rope):
                                  cpu["dout"])
     compare(out, O, "bf16", "out")
     compare(lse, L, "bf16", "lse")
-    check_grads(g, R)
+    check_grads(g, R, label="padded")
     cu = [int(c) for c in cpu["cu_doc_lens"]]
     rows = padded_rows(cu, valid)
     assert rows

@@ -154,7 +154,7 @@ def test_bf16_backward_small(cuda_lib, lens, H, Hk, W, rope):
     torch.cuda.synchronize()
     ref = fo.flint_attn_bwd(cpu["q"], cpu["k"], cpu["v"], cpu["w_q"], cpu["w_k"], cpu["sink"],
                             cpu["cu_doc_lens"], W, rope, 1e6, cpu["dout"])
-    check_grads(g, ref)
+    check_grads(g, ref, label=f"small {lens} H{H}/{Hk} W{W}", window=W)
 
 
 def test_bf16_backward_bf16_io(cuda_lib):
@@ -246,7 +246,7 @@ def test_bf16_backward_prefix_whole_layer(cuda_lib, wl, n_tok, n_docs):
     compare(lse, L, "bf16", "lse")
     ref = fo.flint_attn_bwd(p["q"], p["k"], p["v"], p["w_q"], p["w_k"], p["sink"],
                             p["cu_doc_lens"], wl.window, wl.use_rope, wl.rope_theta, p["dout"])
-    check_grads(g, ref)
+    check_grads(g, ref, label=f"{wl.name} prefix {n_tok}", window=wl.window)
 
 
 # ----------------------------------------------------------------------- FMA-pipe exp2

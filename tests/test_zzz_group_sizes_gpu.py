@@ -35,4 +35,4 @@ def test_group_size(cuda_lib, lens, H, Hk, W, rope):
     compare(lse, L, "bf16", "lse")
     ref = fo.flint_attn_bwd(cpu["q"], cpu["k"], cpu["v"], cpu["w_q"], cpu["w_k"], cpu["sink"],
                             cpu["cu_doc_lens"], W, rope, 1e6, cpu["dout"])
-    check_grads(g, ref)
+    check_grads(g, ref, label=f"group size {H // Hk}")
