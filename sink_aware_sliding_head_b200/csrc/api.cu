@@ -233,8 +233,7 @@ flint_status_t fwd_impl(const flint_attn_params_t* params, const void* q, const 
   void* qh = at<void>(workspace, L.qhat);
   void* kh = at<void>(workspace, L.khat);
   const bool f16 = p.tc;   // tensor-core operands are fp16
-  FLINT_TRY(launch_prologue(p, q, q_norm_w, qh, p.H, cu_doc_lens, st, f16));
-  FLINT_TRY(launch_prologue(p, k, k_norm_w, kh, p.Hk, cu_doc_lens, st, f16));
+  FLINT_TRY(launch_prologue_qk(p, q, q_norm_w, qh, k, k_norm_w, kh, cu_doc_lens, st, f16));
   if (!p.tc) {
     return cuda_status(launch_attn_fwd_fp32(p, (const float*)qh, (const float*)kh,
                                             (const float*)v, sink, cu_doc_lens, (float*)out, lse,
@@ -305,8 +304,7 @@ flint_status_t bwd_impl(const flint_attn_params_t* params, const void* q, const 
   if (f16)
     FLINT_TRY(launch_absmax(p.dtype, dout, (size_t)p.T * p.H * kHeadDim, v,
                             (size_t)p.T * p.Hk * kHeadDim, amax, st));
-  FLINT_TRY(launch_prologue(p, q, q_norm_w, qh, p.H, cu_doc_lens, st, f16));
-  FLINT_TRY(launch_prologue(p, k, k_norm_w, kh, p.Hk, cu_doc_lens, st, f16));
+  FLINT_TRY(launch_prologue_qk(p, q, q_norm_w, qh, k, k_norm_w, kh, cu_doc_lens, st, f16));
   FLINT_TRY(launch_bwd_preprocess(p, out, dout, lse, sink, dvec, part, dsink, dout16,
                                   f16 ? amax : nullptr, st));
   if (!p.tc) {
@@ -316,11 +314,10 @@ flint_status_t bwd_impl(const flint_attn_params_t* params, const void* q, const 
   } else {
     int4* items_kv = at<int4>(workspace, L.items_kv);
     int4* items_q1 = at<int4>(workspace, L.items_q1);
-    void* tmp = at<void>(workspace, L.sched_tmp);
-    FLINT_TRY(launch_build_worklist(cu_doc_lens, valid, p, kModeKey, kTileKeys, items_kv,
-                                    status + 2, tmp, L.max_items_kv, st));
-    FLINT_TRY(launch_build_worklist(cu_doc_lens, valid, p, kModeQuery, p.R, items_q1, status + 3,
-                                    tmp, L.max_items_q1, st));
+    FLINT_TRY(launch_build_worklists2(cu_doc_lens, valid, p, kModeKey, kTileKeys, items_kv,
+                                      status + 2, at<void>(workspace, L.sched_tmp),
+                                      L.max_items_kv, kModeQuery, p.R, items_q1, status + 3,
+                                      at<void>(workspace, L.sched_tmp2), L.max_items_q1, st));
     FLINT_TRY(convert_v(p, v, v16, amax + 1, st));
     const CUtensorMapDataType f16t = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
     CUtensorMap tq, tk, tv, tdo;

@@ -17,9 +17,10 @@
 //     on two such tiles at once ("tile 0" and "tile 1": 2R consecutive tokens)
 //     that share every K/V tile, so each K/V byte brought on chip serves 256
 //     query rows.
-//   * Persistent grid (one CTA per SM) striding over an LPT-sorted work list
-//     built on the device; only key tiles inside the window and the document
-//     are visited, and only edge tiles are masked.
+//   * Persistent grid (one CTA per SM) taking items from an LPT-sorted work
+//     list built on the device through a global counter (greedy LPT: a CTA
+//     asks for its next item when it is ready for it); only key tiles inside
+//     the window and the document are visited, and only edge tiles are masked.
 //   * Warp roles: warps 0-3 run the softmax of tile 0, warps 4-7 of tile 1
 //     (thread = TMEM lane = query row), warp 8 issues TMA loads, warp 9 owns
 //     the TMEM allocation and issues tcgen05.mma: the warp runs its loop
@@ -66,6 +67,7 @@ struct FwdArgs {
   const int4* items;
   const int* n_items;
   int max_items;
+  int* next_item;   // zeroed before the launch: dynamic item counter
   const unsigned* amax_v;   // max |v| slot: the fp16 copy of v is v * 2^e
   void* out;        // bf16, float (out_f32) or fp16 (out_f16)
   int out_f32, out_f16;
@@ -78,6 +80,7 @@ struct __align__(8) Barriers {
   uint64_t kv_full[kSlots], kv_empty[kSlots];
   uint64_t s_full[2], p_half[2], p_full[2], pv_done[2], o_full[2], o_empty[2];
   uint64_t drain;
+  ItemRing ring;
 };
 
 // Dynamic shared memory: [Q0 | Q1 | K stages | V stages | barriers | tmem addr | abort flag]
@@ -146,6 +149,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       mbar_init(smem_u32(&bars->o_empty[i]), 4);
     }
     mbar_init(smem_u32(&bars->drain), 1);
+    ring_init(&bars->ring, 9);   // the MMA warp and the 8 softmax warps consume
     fence_mbar_init();
   }
   if (warp == kWarpMma) {
@@ -168,7 +172,13 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
     if (lane == 0) {
       uint32_t kv_load = 0, item_count = 0, q_arm = 0, arm[kSlots] = {};
       bool ok = true;
-      for (int idx = blockIdx.x; idx < n_items && ok; idx += gridDim.x) {
+      while (ok) {
+        // greedy LPT over the heaviest-first list: the next item goes to the
+        // CTA that asks first; -1 ends every role's loop
+        int idx = atomicAdd(a.next_item, 1);
+        if (idx >= n_items) idx = -1;
+        ok = ring_push(&bars->ring, item_count, idx, wc);
+        if (!ok || idx < 0) break;
         const Item it = decode(a, idx);
         if (item_count > 0) ok = mbar_wait(smem_u32(&bars->q_empty), (item_count - 1) & 1, wc);
         if (!ok) break;
@@ -215,7 +225,10 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       uint32_t pv0 = 0, pv1 = 0, pc0 = 0, pc1 = 0;   // PV commits / P arrivals seen, per tile
       bool ok = true;
       const uint32_t q0t = sbase + kOffQ, q1t = sbase + kOffQ + kTileBytes;
-      for (int idx = blockIdx.x; idx < n_items && ok; idx += gridDim.x) {
+      while (ok) {
+        int idx = -1;
+        ok = ring_pop(&bars->ring, item_count, &idx, wc);
+        if (!ok || idx < 0) break;
         const Item it = decode(a, idx);
         ok = mbar_wait_warp(smem_u32(&bars->q_full), item_count & 1, wc);
         if (!ok) break;
@@ -338,7 +351,10 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
     const float inv_sv = slot_scale(a.amax_v, true);
     uint32_t s_count = 0, item_count = 0;
     bool ok = true;
-    for (int idx = blockIdx.x; idx < n_items && ok; idx += gridDim.x) {
+    while (ok) {
+      int idx = -1;
+      ok = ring_pop(&bars->ring, item_count, &idx, wc);
+      if (!ok || idx < 0) break;
       const Item it = decode(a, idx);
       const int tok = it.q0 + i * a.R + r / a.G;
       const int h = it.g * a.G + r % a.G;
@@ -537,6 +553,7 @@ cudaError_t launch_attn_fwd_sm100_impl(const CUtensorMap& tq, const CUtensorMap&
   a.T = p.T; a.H = p.H; a.Hk = p.Hk; a.G = p.G; a.R = p.R; a.W = p.W;
   a.scale_log2 = p.scale * kLog2e;
   a.sink = sink; a.items = items; a.n_items = n_items; a.max_items = max_items;
+  a.next_item = status + 4;
   a.amax_v = amax_v;
   a.out = out;
   a.out_f32 = p.fp32_out && !p.out_f16;

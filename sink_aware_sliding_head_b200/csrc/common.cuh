@@ -77,6 +77,7 @@ struct WsLayout {
   size_t items_q1;      // int4 work items, query-major single tiles (backward dQ)
   size_t items_kv;      // int4 work items, key-major (backward dK/dV)
   size_t sched_tmp;     // int4 + int per item, scratch for the LPT sort
+  size_t sched_tmp2;    // the same for the backward's second list (built concurrently)
   size_t dvec;          // [H,T] fp32 rowsum(dO * O)      (backward)
   size_t part;          // fp32 partial sums (d sink, d norm weights)
   size_t dq_acc;        // [T,H,D] fp32 gradient w.r.t. q_hat (backward)
@@ -112,6 +113,7 @@ inline WsLayout make_layout(const Resolved& p, bool backward) {
   L.items_q1 = backward ? take((size_t)L.max_items_q1 * 16) : off;
   L.items_kv = backward ? take((size_t)L.max_items_kv * 16) : off;
   L.sched_tmp = take((size_t)L.max_items_any * 20);
+  L.sched_tmp2 = backward ? take((size_t)L.max_items_any * 20) : off;
   L.part_blocks = kPartBlocks;
   if (p.tc) L.v16 = take((size_t)p.T * p.Hk * p.D * 2);
   if (backward) {
@@ -218,6 +220,11 @@ struct ProfScope {
 cudaError_t launch_build_worklist(const int32_t* cu, const int32_t* valid, const Resolved& p,
                                   int mode, int span, int4* items, int* count, void* tmp,
                                   int max_items, cudaStream_t st);
+// Two lists in one launch (one block each); tmp0 and tmp1 must not overlap.
+cudaError_t launch_build_worklists2(const int32_t* cu, const int32_t* valid, const Resolved& p,
+                                    int mode0, int span0, int4* items0, int* count0, void* tmp0,
+                                    int max0, int mode1, int span1, int4* items1, int* count1,
+                                    void* tmp1, int max1, cudaStream_t st);
 // Padding: padded rows get out = 0 and lse = sink (forward), and zero gradient
 // rows dq_acc, dk_acc (fp32 workspace) and dv (backward).
 cudaError_t launch_pad_fill_fwd(const Resolved& p, const int32_t* cu, const int32_t* valid,
@@ -225,9 +232,11 @@ cudaError_t launch_pad_fill_fwd(const Resolved& p, const int32_t* cu, const int3
 cudaError_t launch_pad_fill_bwd(const Resolved& p, const int32_t* cu, const int32_t* valid,
                                 float* dq_acc, float* dk_acc, void* dv, int dv_f32,
                                 cudaStream_t st);
-// out_f16: write x_hat as fp16 (backward operands of BF16 inputs) instead of the input type
-cudaError_t launch_prologue(const Resolved& p, const void* x, const void* w, void* y, int heads,
-                            const int32_t* cu, cudaStream_t st, bool out_f16 = false);
+// q_hat [T,H,D] and k_hat [T,Hk,D] in one launch. out_f16: write them as fp16 (the
+// tensor-core operands) instead of the input type.
+cudaError_t launch_prologue_qk(const Resolved& p, const void* q, const void* wq, void* qh,
+                               const void* k, const void* wk, void* kh, const int32_t* cu,
+                               cudaStream_t st, bool out_f16);
 // dst = fp16(src * 2^e), e from the max |src| in *amax (nullptr: e = 0).
 cudaError_t launch_convert_f16(const __nv_bfloat16* src, __half* dst, size_t n,
                                const unsigned* amax, cudaStream_t st);

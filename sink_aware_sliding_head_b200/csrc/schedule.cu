@@ -8,12 +8,13 @@
 //   2. prices each item by the number of tiles it will visit (key tiles for
 //      query-major items, 128-row query tiles for key-major ones) - tiles
 //      wholly outside the window or another document are never listed;
-//   3. counting-sorts the items by price, heaviest first (LPT order), so that a
-//      grid of persistent CTAs striding over the list finishes together.
+//   3. counting-sorts the items by price, heaviest first, so that persistent
+//      CTAs that take items in list order through a global counter schedule
+//      them greedily longest-first (LPT) and finish together.
 // Item = int4 {first token, document start, document end, KV head}.
 // With padding (valid != nullptr), document d ends after its valid[d] real
 // tokens: the trailing padding gets no item, so no kernel visits it as a query
-// or a key.
+// or a key. The backward's two lists are built by the two blocks of one launch.
 #include "common.cuh"
 
 namespace flint {
@@ -61,11 +62,12 @@ __device__ __forceinline__ int item_cost(int mode, int start, int d0, int d1, in
   return (qend - start + R - 1) / R;
 }
 
-__global__ void __launch_bounds__(kThreads)
-build_worklist_kernel(const int32_t* __restrict__ cu, const int32_t* __restrict__ valid, int N,
-                      int mode, int span, int W, int R,
-                      int Hk, int4* __restrict__ items, int* __restrict__ count,
-                      int4* __restrict__ tmp_items, int* __restrict__ tmp_cost, int max_items) {
+// One list, built by the whole (1024-thread) block.
+__device__ void build_list(const int32_t* __restrict__ cu, const int32_t* __restrict__ valid,
+                           int N, int mode, int span, int W, int R, int Hk,
+                           int4* __restrict__ items, int* __restrict__ count,
+                           int4* __restrict__ tmp_items, int* __restrict__ tmp_cost,
+                           int max_items) {
   __shared__ int warp_sums[32];
   __shared__ int total_s;
   __shared__ int chunk_off[kThreads + 1];
@@ -143,16 +145,52 @@ build_worklist_kernel(const int32_t* __restrict__ cu, const int32_t* __restrict_
   if (threadIdx.x == 0) *count = n_items;
 }
 
+struct ListSpec {
+  int mode, span;
+  int4* items;
+  int* count;
+  int4* tmp_items;
+  int* tmp_cost;
+  int max_items;
+};
+
+// Block b builds list b (gridDim.x lists, at most 2), independently.
+__global__ void __launch_bounds__(kThreads)
+build_worklist_kernel(const int32_t* __restrict__ cu, const int32_t* __restrict__ valid, int N,
+                      int W, int R, int Hk, ListSpec l0, ListSpec l1) {
+  const ListSpec& L = blockIdx.x == 0 ? l0 : l1;
+  build_list(cu, valid, N, L.mode, L.span, W, R, Hk, L.items, L.count, L.tmp_items, L.tmp_cost,
+             L.max_items);
+}
+
+ListSpec spec(int mode, int span, int4* items, int* count, void* tmp, int max_items) {
+  ListSpec l;
+  l.mode = mode; l.span = span; l.items = items; l.count = count;
+  l.tmp_items = reinterpret_cast<int4*>(tmp);
+  l.tmp_cost = reinterpret_cast<int*>(l.tmp_items + max_items);
+  l.max_items = max_items;
+  return l;
+}
+
 }  // namespace
 
 cudaError_t launch_build_worklist(const int32_t* cu, const int32_t* valid, const Resolved& p,
                                   int mode, int span, int4* items, int* count, void* tmp,
                                   int max_items, cudaStream_t st) {
-  int4* tmp_items = reinterpret_cast<int4*>(tmp);
-  int* tmp_cost = reinterpret_cast<int*>(tmp_items + max_items);
+  const ListSpec l = spec(mode, span, items, count, tmp, max_items);
   ProfScope prof(kKWorklist, st);
-  build_worklist_kernel<<<1, kThreads, 0, st>>>(cu, valid, p.N, mode, span, p.W, p.R, p.Hk, items,
-                                                count, tmp_items, tmp_cost, max_items);
+  build_worklist_kernel<<<1, kThreads, 0, st>>>(cu, valid, p.N, p.W, p.R, p.Hk, l, l);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_build_worklists2(const int32_t* cu, const int32_t* valid, const Resolved& p,
+                                    int mode0, int span0, int4* items0, int* count0, void* tmp0,
+                                    int max0, int mode1, int span1, int4* items1, int* count1,
+                                    void* tmp1, int max1, cudaStream_t st) {
+  const ListSpec l0 = spec(mode0, span0, items0, count0, tmp0, max0);
+  const ListSpec l1 = spec(mode1, span1, items1, count1, tmp1, max1);
+  ProfScope prof(kKWorklist, st);
+  build_worklist_kernel<<<2, kThreads, 0, st>>>(cu, valid, p.N, p.W, p.R, p.Hk, l0, l1);
   return cudaGetLastError();
 }
 

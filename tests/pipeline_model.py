@@ -284,7 +284,8 @@ def _ring_bars(sim):
 
 
 # ============================================================================
-# Forward (attn_fwd_sm100_kernel): items are query-tile pairs, static striding
+# Forward (attn_fwd_sm100_kernel): items are query-tile pairs, taken through the
+# item ring like the backward kernels'
 # ============================================================================
 
 def forward(sim, items, mut=None):
@@ -295,13 +296,18 @@ def forward(sim, items, mut=None):
     for i in range(2):
         sim.bar(f"s_full{i}"), sim.bar(f"p_half{i}", 4), sim.bar(f"p_full{i}", 4)
         sim.bar(f"pv_done{i}"), sim.bar(f"o_full{i}"), sim.bar(f"o_empty{i}", 4)
+    _ring_bars(sim)
+    seq = list(items) + [None]
 
     def kv_tag(load):
         return ("V" if load & 1 else "K", load // 2)
 
     def producer():
         kv_load = 0
-        for item, nt in enumerate(items):
+        for item, nt in enumerate(seq):
+            yield from _ring_push(item, ("idx", item))
+            if nt is None:
+                return
             if item > 0:
                 yield ("wait", "q_empty", item - 1)
             yield ("expect_tx", "q_full", 2)
@@ -322,7 +328,10 @@ def forward(sim, items, mut=None):
             return ("mma", [([f"smem:Q{i}"], ("Q", item, i)), ([f"smem:kv{slot}"], ("K", g))],
                     tmem(f"S{i}", ALL_CHUNKS), ("S", i, g), False)
 
-        for item, nt in enumerate(items):
+        for item, nt in enumerate(seq):
+            yield from _ring_pop(item, ("idx", item))
+            if nt is None:
+                return
             g0 = kv_load // 2
             yield ("wait", "q_full", item)
             s = kv_load % K_SLOTS
@@ -378,7 +387,10 @@ def forward(sim, items, mut=None):
     def softmax(i, q):
         s_count, kv_load = 0, 0
         quarter = [q]
-        for item, nt in enumerate(items):
+        for item, nt in enumerate(seq):
+            yield from _ring_pop(item, ("idx", item))
+            if nt is None:
+                return
             g0 = kv_load // 2
             for n in range(nt):
                 g = g0 + n
