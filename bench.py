@@ -79,7 +79,7 @@ def real_lens(inp):
 
 def visible_pairs(doc_lens, window: int) -> int:
     """Masked FLOP accounting: (query, key) pairs per head under the causal document
-    mask whose window counts the current token (row i of a document sees min(i + 1, W)
+    mask whose window includes the current token (row i of a document sees min(i + 1, W)
     keys)."""
     total = 0
     for L in doc_lens:

@@ -16,7 +16,7 @@
  *     FlintConfig docstring. Frequencies theta^(-2j/D); positions restart at 0
  *     in every document (FlintAttention.forward, position_ids for THD).
  *     RMSNorm is applied first, then RoPE.
- *   - Causal window that counts the current token; window <= 0 is unbounded:
+ *   - Causal window that includes the current token; window <= 0 is unbounded:
  *     FlintConfig docstring and sliding_window; attention utils page
  *     (nemo_automodel.components.attention.utils),
  *     preprocess_args_and_kwargs_for_attn (its window_size convention).
@@ -95,7 +95,7 @@ typedef struct {
                              paths; FP32 inputs without compute_f16 take any G) */
   int32_t head_dim;       /* D; must be 128 */
   int32_t window;         /* > 0: key j visible from query i iff 0 <= i - j < window
-                             (counts the current token); <= 0: full causal */
+                             (the current token included); <= 0: full causal */
   int32_t use_rope;       /* nonzero: NeoX RoPE on all D channels after RMSNorm */
   float rope_theta;       /* RoPE base (> 0 when use_rope) */
   float rms_eps;          /* RMSNorm epsilon (Flint: 1e-6) */

@@ -13,7 +13,7 @@ Per query token i of document [d0, d1), head h (KV head h // (H/Hk)):
   visible keys: d0 <= j <= i and (W <= 0 or i - j < W)
                                              (FlintConfig docstring; attention utils
                                               page, preprocess_args_and_kwargs_for_attn)
-  softmax over {z_ij} and the unscaled sink logit s_h; the sink's value is zero
+  softmax over {z_ij} and the sink logit s_h (not scaled); the sink's value is zero
                                              (FlintAttention.forward,
                                               _FlintSinkParameters.forward)
 """

@@ -18,7 +18,7 @@ What it computes, step by step, with the passage each step follows:
   layers (Flint config page, ``FlintConfig`` docstring; ``use_rope`` on the
   layers page). Positions are document-local for THD (``FlintAttention.forward``,
   ``position_ids``).
-* Causal window that counts the current token (``FlintConfig`` docstring;
+* Causal window that includes the current token (``FlintConfig`` docstring;
   attention utils page, ``preprocess_args_and_kwargs_for_attn``: a positive
   left window counts visible keys including the current token, negative or
   None is unbounded).
@@ -70,7 +70,7 @@ def doc_positions(cu_doc_lens):
 def visible_keys(i, d0, window):
     """Key range [lo, i] visible from query token i of a document starting at d0.
 
-    The window counts the current token: key j is visible iff d0 <= j <= i and
+    The window includes the current token: key j is visible iff d0 <= j <= i and
     (window <= 0 or i - j < window).
     """
     lo = d0 if window <= 0 else max(d0, i - window + 1)

@@ -17,6 +17,7 @@ namespace flint {
 cudaError_t launch_reduce_rows(const float* part, int nrows, int width, float* out,
                                cudaStream_t st);
 cudaError_t launch_exp2_poly(const float* x, float* y, int n, cudaStream_t st);
+int fwd_kv_box_tokens();
 cudaError_t launch_attn_fwd_sm100_impl(const CUtensorMap& tq, const CUtensorMap& tk,
                                        const CUtensorMap& tv, const Resolved& p, const float* sink,
                                        const int4* items, const int* n_items, int max_items,
@@ -248,9 +249,10 @@ flint_status_t fwd_impl(const flint_attn_params_t* params, const void* q, const 
   FLINT_TRY(convert_v(p, v, v16, amax + 1, st));
   const CUtensorMapDataType f16t = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
   CUtensorMap tq, tk, tv;
+  const int kv_box = fwd_kv_box_tokens();
   if (!encode_3d(&tq, qh, p.T, p.H, p.G, p.R, f16t) ||
-      !encode_3d(&tk, kh, p.T, p.Hk, 1, kTileKeys, f16t) ||
-      !encode_3d(&tv, v16, p.T, p.Hk, 1, kTileKeys, f16t))
+      !encode_3d(&tk, kh, p.T, p.Hk, 1, kv_box, f16t) ||
+      !encode_3d(&tv, v16, p.T, p.Hk, 1, kv_box, f16t))
     return FLINT_ERR_CUDA;
   FLINT_TRY(launch_attn_fwd_sm100_impl(tq, tk, tv, p, sink, items, status + 1, L.max_items_q,
                                        amax + 1, out, lse, status, sm_count(), st));

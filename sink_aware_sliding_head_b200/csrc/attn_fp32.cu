@@ -7,7 +7,7 @@
 // FlintAttention.forward and _FlintSinkParameters.forward): for query row
 // (t, h) of document [d0, d1), visible keys j satisfy d0 <= j <= t and
 // (W <= 0 or t - j < W) (window counting the current token, FlintConfig
-// docstring); z_tj = scale * q_hat . k_hat; the unscaled sink logit s_h joins
+// docstring); z_tj = scale * q_hat . k_hat; the sink logit s_h, not scaled, joins
 // the softmax denominator with a zero value.
 //   forward : running max starts at s_h and the running sum at 1 (the sink's
 //             own weight), then O = acc / l, LSE = m + ln l.

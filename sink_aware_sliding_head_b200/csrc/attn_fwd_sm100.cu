@@ -4,9 +4,10 @@
 // accumulation, output in bf16 or fp32.
 //
 // What it computes (Flint layers page, nemo_automodel.components.models.flint.
-// layers, FlintAttention.forward: causal attention with a zero-value sink
-// category; _FlintSinkParameters.forward: unscaled FP32 sink logits; Flint
-// config page: the window counts the current token):
+// layers, FlintAttention.forward: causal attention in which the sink is one
+// more softmax category with a zero value vector; _FlintSinkParameters.forward:
+// FP32 sink logits, not scaled; Flint config page: the window includes the
+// current token):
 //   O_i = sum_j e^{z_ij - LSE_i} v_j,  LSE_i = ln(e^{s_h} + sum_j e^{z_ij}),
 //   over keys j of the same document with 0 <= i - j < W (W <= 0: unbounded).
 //
@@ -540,6 +541,9 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
 }
 
 }  // namespace
+
+// Keys per K/V box of the forward's tensor maps (one key tile).
+int fwd_kv_box_tokens() { return kTileKeys; }
 
 cudaError_t launch_attn_fwd_sm100_impl(const CUtensorMap& tq, const CUtensorMap& tk,
                                        const CUtensorMap& tv, const Resolved& p, const float* sink,

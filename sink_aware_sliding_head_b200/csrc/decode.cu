@@ -3,9 +3,9 @@
 //
 // What it computes is flint_attn_fwd's definition restricted to the last row
 // of each sequence (Flint layers page, nemo_automodel.components.models.flint.
-// layers: FlintAttention.forward, causal attention with a zero-value sink
-// category; per-head RMSNorm then NeoX RoPE; Flint config page: the window
-// counts the current token). Sequence b has p = cache_lens[b] tokens cached;
+// layers: FlintAttention.forward, causal attention in which the sink is one
+// more softmax category with a zero value vector; per-head RMSNorm then NeoX
+// RoPE; Flint config page: the window includes the current token). Sequence b has p = cache_lens[b] tokens cached;
 // the new token's normalised, rotated key and its value go into slot p, and
 // the new query attends to slots max(0, p - W + 1) .. p plus the sink.
 //

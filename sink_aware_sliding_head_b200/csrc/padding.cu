@@ -4,7 +4,8 @@
 // Padded queries and keys are excluded while the sink stays valid (attention
 // utils page, nemo_automodel.components.attention.utils: the BSHD
 // attention_mask, with trailing padding as TE takes it; Flint layers page,
-// FlintAttention.forward: the zero-value sink category). A padded query sees no
+// FlintAttention.forward: the sink is a softmax category with a zero value
+// vector, so it stays in every row). A padded query sees no
 // key, so its row is the sink alone: O = 0, LSE = sink_h. Nothing downstream
 // depends on a padded token, so its gradients are zero. The work lists give
 // padded tokens no item, so the attention kernels never write these rows; the

@@ -46,41 +46,40 @@ __device__ void build_rope_table(const int32_t* __restrict__ cu, int N, int T, i
   __syncthreads();
 }
 
-// q and k in one launch: a block owns kTok tokens and normalises their q rows
-// (heads0 per token) and then their k rows (heads1 per token), sharing the
-// RoPE table of the tokens.
+// q and k in one launch: the first nblk0 blocks normalise kTok tokens of x0
+// (heads0 rows per token) each, the rest kTok tokens of x1 (heads1 rows).
 template <typename T, typename TO>
 __global__ void __launch_bounds__(kThreads)
 prologue_kernel(const T* __restrict__ x0, const T* __restrict__ w0, TO* __restrict__ y0,
                 int heads0, const T* __restrict__ x1, const T* __restrict__ w1,
-                TO* __restrict__ y1, int heads1, int ntok, const int32_t* __restrict__ cu,
-                int N, int rope, float theta, float eps) {
+                TO* __restrict__ y1, int heads1, int nblk0, int ntok,
+                const int32_t* __restrict__ cu, int N, int rope, float theta, float eps) {
   __shared__ float cs[kTok][kHalf], sn[kTok][kHalf];
   __shared__ int pos_s[kTok];
-  const int t0 = blockIdx.x * kTok;
+  const bool second = (int)blockIdx.x >= nblk0;
+  const T* __restrict__ x = second ? x1 : x0;
+  const T* __restrict__ w = second ? w1 : w0;
+  TO* __restrict__ y = second ? y1 : y0;
+  const int heads = second ? heads1 : heads0;
+  const int t0 = (second ? blockIdx.x - nblk0 : blockIdx.x) * kTok;
   if (rope) build_rope_table(cu, N, ntok, t0, theta, cs, sn, pos_s);
   const int lane16 = threadIdx.x & 15;
   const int grp = threadIdx.x >> 4;
   const int c0 = lane16 * 8;
-  float wv0[8], wv1[8];
-  load8(w0 + c0, wv0);
-  if (heads1 > 0) load8(w1 + c0, wv1);
-  const int rows0 = kTok * heads0;
-  const int rows = rows0 + kTok * heads1;
+  float wv[8];
+  load8(w + c0, wv);
+  const int rows = kTok * heads;
   // Every half-warp runs the same number of iterations so the full-warp
   // shuffles below always see both halves; invalid rows load zeros, store nothing.
   const int iters = (rows + kThreads / 16 - 1) / (kThreads / 16);
   for (int it = 0; it < iters; ++it) {
     const int rr = grp + it * (kThreads / 16);
-    const bool second = rr >= rows0;
-    const int r1 = second ? rr - rows0 : rr;
-    const int heads = second ? heads1 : heads0;
-    const int tok = heads > 0 ? r1 / heads : 0;
+    const int tok = rr / heads;
     const int t = t0 + tok;
     const bool valid = rr < rows && t < ntok;
-    const size_t base = valid ? ((size_t)t * heads + (r1 % heads)) * kHeadDim + c0 : 0;
+    const size_t base = valid ? ((size_t)t * heads + (rr % heads)) * kHeadDim + c0 : 0;
     float v[8];
-    if (valid) load8((second ? x1 : x0) + base, v);
+    if (valid) load8(x + base, v);
     else {
 #pragma unroll
       for (int e = 0; e < 8; ++e) v[e] = 0.f;
@@ -92,7 +91,7 @@ prologue_kernel(const T* __restrict__ x0, const T* __restrict__ w0, TO* __restri
     for (int o = 8; o >= 1; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
     const float r = rsqrtf(ss * (1.0f / kHeadDim) + eps);
 #pragma unroll
-    for (int e = 0; e < 8; ++e) v[e] = v[e] * r * (second ? wv1[e] : wv0[e]);
+    for (int e = 0; e < 8; ++e) v[e] = v[e] * r * wv[e];
     if (rope) {
       float o8[8];
       const bool lo_half = lane16 < 8;
@@ -107,7 +106,7 @@ prologue_kernel(const T* __restrict__ x0, const T* __restrict__ w0, TO* __restri
 #pragma unroll
       for (int e = 0; e < 8; ++e) v[e] = o8[e];
     }
-    if (valid) store8((second ? y1 : y0) + base, v);
+    if (valid) store8(y + base, v);
   }
 }
 
@@ -211,25 +210,26 @@ cudaError_t launch_prologue_qk(const Resolved& p, const void* q, const void* wq,
                                const void* k, const void* wk, void* kh, const int32_t* cu,
                                cudaStream_t st, bool out_f16) {
   if (p.T == 0) return cudaSuccess;
-  dim3 grid((p.T + kTok - 1) / kTok);
+  const int nblk = (p.T + kTok - 1) / kTok;   // per tensor
+  dim3 grid(2 * nblk);
   ProfScope prof(kKPrologue, st);
   typedef __nv_bfloat16 bf;
   if (p.dtype == FLINT_BF16 && out_f16)
     prologue_kernel<bf, __half><<<grid, kThreads, 0, st>>>(
         (const bf*)q, (const bf*)wq, (__half*)qh, p.H, (const bf*)k, (const bf*)wk, (__half*)kh,
-        p.Hk, p.T, cu, p.N, p.rope, p.theta, p.eps);
+        p.Hk, nblk, p.T, cu, p.N, p.rope, p.theta, p.eps);
   else if (p.dtype == FLINT_BF16)
     prologue_kernel<bf, bf><<<grid, kThreads, 0, st>>>(
         (const bf*)q, (const bf*)wq, (bf*)qh, p.H, (const bf*)k, (const bf*)wk, (bf*)kh, p.Hk,
-        p.T, cu, p.N, p.rope, p.theta, p.eps);
+        nblk, p.T, cu, p.N, p.rope, p.theta, p.eps);
   else if (out_f16)   // FP32 inputs at the fp16 compute boundary
     prologue_kernel<float, __half><<<grid, kThreads, 0, st>>>(
         (const float*)q, (const float*)wq, (__half*)qh, p.H, (const float*)k, (const float*)wk,
-        (__half*)kh, p.Hk, p.T, cu, p.N, p.rope, p.theta, p.eps);
+        (__half*)kh, p.Hk, nblk, p.T, cu, p.N, p.rope, p.theta, p.eps);
   else
     prologue_kernel<float, float><<<grid, kThreads, 0, st>>>(
         (const float*)q, (const float*)wq, (float*)qh, p.H, (const float*)k, (const float*)wk,
-        (float*)kh, p.Hk, p.T, cu, p.N, p.rope, p.theta, p.eps);
+        (float*)kh, p.Hk, nblk, p.T, cu, p.N, p.rope, p.theta, p.eps);
   return cudaGetLastError();
 }
 

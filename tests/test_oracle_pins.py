@@ -391,7 +391,7 @@ def test_config_constants_golden():
     assert SLIDING_BF16.num_kv_heads == c["num_key_value_heads"]
     for w in WORKLOADS:
         assert w.rms_eps == c["rms_norm_eps"]
-    # the default window of 513 counts the current token: 512 earlier keys + itself
+    # the default window of 513 includes the current token: 512 earlier keys + itself
     lens = [600]
     n = [min(p + 1, c["sliding_window"]) for p in range(600)]
     assert n[-1] == 513
