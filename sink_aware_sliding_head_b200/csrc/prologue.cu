@@ -31,11 +31,13 @@ __device__ void build_rope_table(const int32_t* __restrict__ cu, int N, int T, i
     int t = t0 + threadIdx.x;
     pos_s[threadIdx.x] = (t < T) ? t - __ldg(cu + doc_of(cu, N, t)) : 0;
   }
+  __shared__ double inv_freq[kHalf];
+  if (threadIdx.x < kHalf)
+    inv_freq[threadIdx.x] = exp2(-(2.0 * threadIdx.x / kHeadDim) * log2((double)theta));
   __syncthreads();
   for (int e = threadIdx.x; e < kTok * kHalf; e += blockDim.x) {
     int tok = e / kHalf, j = e % kHalf;
-    double inv_freq = exp2(-(2.0 * j / kHeadDim) * log2((double)theta));
-    double a = (double)pos_s[tok] * inv_freq;
+    double a = (double)pos_s[tok] * inv_freq[j];
     const double two_pi = 6.283185307179586476925286766559;
     a -= two_pi * rint(a / two_pi);
     float s, c;
@@ -194,14 +196,29 @@ prologue_bwd_kernel(const T* __restrict__ x, const T* __restrict__ w,
   }
 }
 
-// out[c] = sum over rows b < nrows of part[b * width + c], in a fixed order.
-__global__ void reduce_rows_kernel(const float* __restrict__ part, int nrows, int width,
-                                   float* __restrict__ out) {
-  const int c = blockIdx.x * blockDim.x + threadIdx.x;
-  if (c >= width) return;
+// out[c] = sum over rows b < nrows of part[b * width + c], in a fixed order: a
+// block of 32 warps owns 32 columns (one per lane, so loads are coalesced), warp
+// w adds rows w, w + 32, ... in turn, and one warp then adds the 32 warp sums in
+// warp order. The result does not depend on timing (deterministic).
+constexpr int kRedWarps = 32;
+__global__ void __launch_bounds__(32 * kRedWarps)
+reduce_rows_kernel(const float* __restrict__ part, int nrows, int width,
+                   float* __restrict__ out) {
+  __shared__ float red[kRedWarps][33];
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int c = blockIdx.x * 32 + lane;
   float s = 0.f;
-  for (int b = 0; b < nrows; ++b) s += part[(size_t)b * width + c];
-  out[c] = s;
+  if (c < width) {
+#pragma unroll 4
+    for (int b = w; b < nrows; b += kRedWarps) s += part[(size_t)b * width + c];
+  }
+  red[w][lane] = s;
+  __syncthreads();
+  if (w == 0 && c < width) {
+    float t = 0.f;
+    for (int i = 0; i < kRedWarps; ++i) t += red[i][lane];
+    out[c] = t;
+  }
 }
 
 }  // namespace
@@ -262,14 +279,14 @@ cudaError_t launch_bwd_epilogue(const Resolved& p, const void* x, const void* w,
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   ProfScope prof(kKReduce, st);
-  reduce_rows_kernel<<<1, kHeadDim, 0, st>>>(part, blocks, kHeadDim, dw);
+  reduce_rows_kernel<<<(kHeadDim + 31) / 32, 32 * kRedWarps, 0, st>>>(part, blocks, kHeadDim, dw);
   return cudaGetLastError();
 }
 
 cudaError_t launch_reduce_rows(const float* part, int nrows, int width, float* out,
                                cudaStream_t st) {
   ProfScope prof(kKReduce, st);
-  reduce_rows_kernel<<<(width + 127) / 128, 128, 0, st>>>(part, nrows, width, out);
+  reduce_rows_kernel<<<(width + 31) / 32, 32 * kRedWarps, 0, st>>>(part, nrows, width, out);
   return cudaGetLastError();
 }
 
