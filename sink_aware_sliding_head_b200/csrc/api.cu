@@ -245,7 +245,8 @@ flint_status_t fwd_impl(const flint_attn_params_t* params, const void* q, const 
                                   at<void>(workspace, L.sched_tmp), L.max_items_q, st));
   __half* v16 = at<__half>(workspace, L.v16);
   unsigned* amax = reinterpret_cast<unsigned*>(status + kSlotAmaxDout);   // [dout, v]
-  FLINT_TRY(launch_absmax(p.dtype, nullptr, 0, v, (size_t)p.T * p.Hk * kHeadDim, amax, st));
+  FLINT_TRY(launch_absmax(p.dtype, nullptr, 0, v, (size_t)p.T * p.Hk * kHeadDim, amax,
+                          cu_doc_lens, valid, p.N, p.H, p.Hk, st));
   FLINT_TRY(convert_v(p, v, v16, amax + 1, st));
   const CUtensorMapDataType f16t = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
   CUtensorMap tq, tk, tv;
@@ -305,7 +306,8 @@ flint_status_t bwd_impl(const flint_attn_params_t* params, const void* q, const 
   unsigned* amax = reinterpret_cast<unsigned*>(status + kSlotAmaxDout);   // [dout, v]
   if (f16)
     FLINT_TRY(launch_absmax(p.dtype, dout, (size_t)p.T * p.H * kHeadDim, v,
-                            (size_t)p.T * p.Hk * kHeadDim, amax, st));
+                            (size_t)p.T * p.Hk * kHeadDim, amax, cu_doc_lens, valid, p.N, p.H,
+                            p.Hk, st));
   FLINT_TRY(launch_prologue_qk(p, q, q_norm_w, qh, k, k_norm_w, kh, cu_doc_lens, st, f16));
   FLINT_TRY(launch_bwd_preprocess(p, out, dout, lse, sink, dvec, part, dsink, dout16,
                                   f16 ? amax : nullptr, st));

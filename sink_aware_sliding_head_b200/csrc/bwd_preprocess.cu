@@ -97,17 +97,26 @@ __global__ void convert_f16_kernel(const T* __restrict__ src, __half* __restrict
 }
 
 // Largest magnitude of two tensors (8 elements per thread and step), one
-// atomicMax per block and tensor on the float bit patterns.
+// atomicMax per block and tensor on the float bit patterns. With padding (valid
+// non-null), rows of padding tokens are skipped: whatever a caller leaves there
+// must not set the scale of the real rows. row8_0 / row8_1: 8-element groups
+// per token of x0 / x1.
 template <typename T>
 __global__ void __launch_bounds__(256)
 absmax_kernel(const T* __restrict__ x0, size_t n0_8, const T* __restrict__ x1, size_t n1_8,
-              unsigned* __restrict__ amax) {
+              unsigned* __restrict__ amax, const int32_t* __restrict__ cu,
+              const int32_t* __restrict__ valid, int N, int row8_0, int row8_1) {
   __shared__ float red[2][8];
   float m0 = 0.f, m1 = 0.f;
   const size_t stride = (size_t)gridDim.x * blockDim.x;
   for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n0_8 + n1_8; i += stride) {
     float f[8];
     const bool first = i < n0_8;
+    if (valid) {
+      const int t = (int)(first ? i / row8_0 : (i - n0_8) / row8_1);
+      const int d = doc_of(cu, N, t);
+      if (t - __ldg(cu + d) >= __ldg(valid + d)) continue;   // a padding token
+    }
     load8(first ? x0 + 8 * i : x1 + 8 * (i - n0_8), f);
     float m = 0.f;
 #pragma unroll
@@ -167,19 +176,22 @@ cudaError_t launch_convert_f16(const float* src, __half* dst, size_t n, const un
 }
 
 cudaError_t launch_absmax(int dtype, const void* x0, size_t n0, const void* x1, size_t n1,
-                          unsigned* amax, cudaStream_t st) {
+                          unsigned* amax, const int32_t* cu, const int32_t* valid, int N,
+                          int heads0, int heads1, cudaStream_t st) {
   const size_t n0_8 = x0 ? n0 / 8 : 0, n1_8 = x1 ? n1 / 8 : 0;
   if (n0_8 + n1_8 == 0) return cudaSuccess;
   size_t blocks = (n0_8 + n1_8 + 255) / 256;
   if (blocks > 148 * 8) blocks = 148 * 8;
   ProfScope prof(kKAbsmax, st);
+  const int r0 = heads0 * kHeadDim / 8, r1 = heads1 * kHeadDim / 8;   // 8-groups per token
   if (dtype == FLINT_BF16)
     absmax_kernel<__nv_bfloat16><<<(unsigned)blocks, 256, 0, st>>>(
         static_cast<const __nv_bfloat16*>(x0), n0_8, static_cast<const __nv_bfloat16*>(x1),
-        n1_8, amax);
+        n1_8, amax, cu, valid, N, r0 > 0 ? r0 : 1, r1 > 0 ? r1 : 1);
   else
     absmax_kernel<float><<<(unsigned)blocks, 256, 0, st>>>(
-        static_cast<const float*>(x0), n0_8, static_cast<const float*>(x1), n1_8, amax);
+        static_cast<const float*>(x0), n0_8, static_cast<const float*>(x1), n1_8, amax, cu,
+        valid, N, r0 > 0 ? r0 : 1, r1 > 0 ? r1 : 1);
   return cudaGetLastError();
 }
 

@@ -245,8 +245,11 @@ cudaError_t launch_convert_f16(const float* src, __half* dst, size_t n, const un
 // amax[0] = bits of max |x0| over n0 elements, amax[1] = bits of max |x1| over n1
 // (both raised with atomicMax, so the slots must start at zero); x0 or x1 may be
 // null (n = 0). n0, n1 multiples of 8. dtype: FLINT_BF16 or FLINT_FP32 for both.
+// x0 is [T, heads0, D] and x1 [T, heads1, D]; with valid non-null (padding),
+// the rows of padding tokens (documents per cu, N) are left out.
 cudaError_t launch_absmax(int dtype, const void* x0, size_t n0, const void* x1, size_t n1,
-                          unsigned* amax, cudaStream_t st);
+                          unsigned* amax, const int32_t* cu, const int32_t* valid, int N,
+                          int heads0, int heads1, cudaStream_t st);
 // Bounded-wait self-test (selftest.cu): status[0] gets the timeout bit, status[1]
 // 1 if the wait completed and 0 if it gave up.
 cudaError_t launch_wait_selftest(long long limit, int arrive_first, int* status,

@@ -112,3 +112,34 @@ def test_fp32_padding_is_unsupported(cuda_lib):
         cuda_lib.fwd(d["q"], d["k"], d["v"], d["w_q"], d["w_k"], d["sink"], d["cu_doc_lens"],
                      0, False, 1e4, valid_lens=vd)
     assert e.value.code == 2
+
+
+def test_padding_contents_do_not_touch_real_rows(cuda_lib):
+    """Whatever finite values a caller leaves in the padding (here +-3e7, far outside
+    fp16's range) must not change the real rows: padded tokens are excluded from the
+    attention and from the choice of the fp16 operand scales of v and dO."""
+    lens, valid, W, rope, theta = [300, 300, 300], [300, 150, 1], 0, True, 1e6
+    cpu = fi.make_custom(lens, 32, 4, dtype="bf16", seed=12)
+    cu = [int(c) for c in cpu["cu_doc_lens"]]
+    pad = padded_rows(cu, valid)
+    gen = torch.Generator().manual_seed(5)
+    for name in ("q", "k", "v", "dout"):
+        t = cpu[name]
+        noise = torch.sign(torch.randn(len(pad), *t.shape[1:], generator=gen)) * 3e7
+        t[pad] = noise.to(t.dtype)
+    d = to_dev(cpu)
+    vd = torch.tensor(valid, dtype=torch.int32, device="cuda")
+    out, lse, g = run_padded(cuda_lib, d, vd, W, rope, theta)
+    O, L = fo.flint_attn_fwd_padded(cpu["q"], cpu["k"], cpu["v"], cpu["w_q"], cpu["w_k"],
+                                    cpu["sink"], cpu["cu_doc_lens"], valid, W, rope, theta)
+    R = fo.flint_attn_bwd_padded(cpu["q"], cpu["k"], cpu["v"], cpu["w_q"], cpu["w_k"],
+                                 cpu["sink"], cpu["cu_doc_lens"], valid, W, rope, theta,
+                                 cpu["dout"])
+    real = [t for t in range(cu[-1]) if t not in set(pad)]
+    compare(out[real], O[real], "bf16", "out")
+    compare(lse[:, real], L[:, real], "bf16", "lse")
+    for name in ("dq", "dk", "dv"):
+        compare(g[name][real], R[name][real], "bf16", name)
+        assert torch.all(g[name][pad] == 0), name
+    assert torch.all(out[pad] == 0)
+    compare(g["dsink"], R["dsink"], "bf16", "dsink")
