@@ -442,6 +442,42 @@ class RowOracle:
         return dx[0, 0], dv
 
 
+    def forward_rows(self, tokens, chunk=256):
+        """``forward_row`` for every head of several query tokens at once.
+
+        The same definition: each row (t, h) takes its own visible keys, the
+        unscaled sink logit joins its softmax denominator with a zero value, and
+        O and LSE follow. Rows are taken ``chunk`` at a time as one matrix of
+        logits per KV head. Returns O [n, H, D] and LSE [H, n].
+        """
+        tokens = [int(t) for t in tokens]
+        G = self.H // self.Hk
+        O = np.zeros((len(tokens), self.H, self.v.shape[-1]))
+        L = np.zeros((self.H, len(tokens)))
+        for kv in range(self.Hk):
+            K, V = self.k_hat_kv[kv], self.v_kv[kv]
+            pairs = [(n, t, h) for n, t in enumerate(tokens) for h in range(kv * G, (kv + 1) * G)]
+            for c0 in range(0, len(pairs), chunk):
+                part = pairs[c0:c0 + chunk]
+                bounds = [visible_keys(t, _doc_of(self.cu, t)[0], self.window) for _, t, _ in part]
+                lo = min(b[0] for b in bounds)
+                hi = max(b[1] for b in bounds) + 1
+                qh = np.stack([self._q_hat(t, h) for _, t, h in part])
+                s_h = np.array([self.sink[h] for _, _, h in part])
+                z = self.scale * (qh @ K[lo:hi].T)
+                col = np.arange(lo, hi)[None, :]
+                vis = (col >= np.array([b[0] for b in bounds])[:, None]) & \
+                      (col <= np.array([b[1] for b in bounds])[:, None])
+                z = np.where(vis, z, -np.inf)
+                m = np.maximum(np.max(z, axis=1), s_h)
+                e = np.exp(z - m[:, None])
+                Z = np.exp(s_h - m) + np.sum(e, axis=1)
+                o = (e @ V[lo:hi]) / Z[:, None]
+                for r, (n, _, h) in enumerate(part):
+                    O[n, h] = o[r]
+                    L[h, n] = m[r] + np.log(Z[r])
+        return O, L
+
     def dkv_rows(self, keys, kv, chunk=256):
         """``dkv_row`` for several keys of KV head ``kv`` at once.
 

@@ -39,3 +39,39 @@ def doc_check(task):
         stats[name] = (float(np.max(np.abs(err))) if err.size else 0.0,
                        float(np.sum(err * err)), float(np.sum(r * r)), bad)
     return stats, {name: R[name] for name in SUMS}
+
+
+# ---------------------------------------------------------------------------
+# Whole-layer forward of a long single-document layer, rows split across workers.
+# Rows of the forward are independent, so each worker computes its share of
+# query rows with RowOracle.forward_rows. Every worker draws the workload's
+# inputs itself from their seed (the same generator the test used), so nothing
+# large crosses the process boundary but the GPU rows it checks.
+# ---------------------------------------------------------------------------
+_ROW_ORACLE = None
+
+
+def init_forward_rows(workload_name):
+    global _ROW_ORACLE
+    import flint_inputs as fi
+    wl = {w.name: w for w in fi.WORKLOADS}[workload_name]
+    cpu = fi.make_inputs(wl, with_grad_out=False)
+    with threadpool_limits(limits=2):
+        _ROW_ORACLE = fo.RowOracle(cpu["q"], cpu["k"], cpu["v"], cpu["w_q"], cpu["w_k"],
+                                   cpu["sink"], cpu["cu_doc_lens"], wl.window, wl.use_rope,
+                                   wl.rope_theta)
+
+
+def forward_rows_check(task):
+    """task: (first token, end token, GPU out rows [n, H, D], GPU lse [H, n]).
+    Returns {"out"/"lse": (max_abs, sum_err2, sum_ref2, n_nonfinite)}."""
+    t0, t1, out, lse = task
+    with threadpool_limits(limits=2):
+        O, L = _ROW_ORACLE.forward_rows(range(t0, t1))
+    stats = {}
+    for name, g, r in (("out", out, O), ("lse", lse, L)):
+        g = np.asarray(g, dtype=np.float64)
+        err = g - r
+        stats[name] = (float(np.max(np.abs(err))), float(np.sum(err * err)), float(np.sum(r * r)),
+                       int(np.sum(~np.isfinite(g))))
+    return stats

@@ -364,6 +364,21 @@ def test_row_oracle_matches_whole_layer():
             np.testing.assert_allclose(dv, g["dv"][j, kv], atol=1e-12)
 
 
+def test_row_oracle_batched_forward_rows_match_whole_layer():
+    """RowOracle.forward_rows (query rows taken as chunks of a logit matrix) equals
+    the whole-layer forward, for rows of several documents, small chunks included."""
+    H, Hk, D = 4, 2, 16
+    q, k, v, wq, wk, sink, cu, _ = rand_case([40, 0, 33, 5], H, Hk, D, seed=42)
+    for W, rope in [(9, True), (0, False)]:
+        O, L = fo.flint_attn_fwd(q, k, v, wq, wk, sink, cu, W, rope, 1e4)
+        ro = fo.RowOracle(q, k, v, wq, wk, sink, cu, W, rope, 1e4)
+        toks = [0, 1, 17, 39, 40, 41, 72, 73, 77]
+        for chunk in (3, 64, 1000):
+            o, l = ro.forward_rows(toks, chunk=chunk)
+            np.testing.assert_allclose(o, O[toks], atol=1e-13)
+            np.testing.assert_allclose(l, L[:, toks], atol=1e-13)
+
+
 def test_row_oracle_batched_key_rows_match_whole_layer():
     """RowOracle.dkv_rows (query rows taken as chunks of a logit matrix) equals the
     whole-layer backward, for keys seen by many rows, small chunks included."""

@@ -4,9 +4,10 @@
   every element of out, LSE, dq, dk, dv and d_sink / the norm-weight gradients
   over all tokens, against the whole-layer FP64 oracle (evaluated per document
   in worker processes; see oracle_pool.py).
-* The S = 32768 full-causal forward on 4096 rows that cover every row position
-  of the kernel's tile pair (32 tokens x 8 heads of a KV group) at many points
-  of the sequence.
+* The S = 32768 full-causal forward, every element of out and LSE against the
+  oracle (rows split across worker processes), and 4096 rows that cover every
+  row position of the kernel's tile pair (32 tokens x 8 heads of a KV group)
+  at many points of the sequence, in bfloat16 output.
 * The S = 131072 full-causal backward on key rows that 1000-2000 query tokens
   (x 8 heads) see, so long dK/dV accumulations are compared at full size.
 All run through the C ABI in the launch configuration bench.py times.
@@ -100,6 +101,29 @@ def test_full_forward_every_tile_position(cuda_lib):
     compare(out[idx_t, idx_h], np.stack([r[0] for r in ref]), "bf16", "out rows",
             out_bf16=True)
     compare(lse[idx_h, idx_t], np.array([r[1] for r in ref]), "bf16", "lse rows")
+
+
+def test_full_forward_whole_layer_every_element(cuda_lib):
+    wl = fi.FULL_BF16
+    cpu = fi.make_inputs(wl, with_grad_out=False)
+    d = to_dev(cpu)
+    out, lse = run_fwd(cuda_lib, d, wl.window, wl.use_rope, wl.rope_theta, fp32_out=True)
+    torch.cuda.synchronize()
+    T, step = wl.total_tokens, 512
+    tasks = [(t0, t0 + step, _np32(out[t0:t0 + step]), _np32(lse[:, t0:t0 + step]))
+             for t0 in range(T - step, -1, -step)]          # the longest rows first
+    workers = max(1, min(len(tasks), os.cpu_count() or 1, 16))
+    with mp.get_context("spawn").Pool(workers, initializer=oracle_pool.init_forward_rows,
+                                      initargs=(wl.name,)) as pool:
+        results = pool.map(oracle_pool.forward_rows_check, tasks, chunksize=1)
+    for name in ("out", "lse"):
+        mx = max(r[name][0] for r in results)
+        rel = float(np.sqrt(sum(r[name][1] for r in results) / sum(r[name][2] for r in results)))
+        bad = sum(r[name][3] for r in results)
+        print(f"WHOLE full forward {name}: max_abs {mx:.3e} rel_rms {rel:.2e}", flush=True)
+        assert bad == 0, f"{name}: {bad} non-finite values"
+        assert mx <= BF16_MAX_ABS, f"{name}: max_abs {mx:.3e}"
+        assert rel <= BF16_REL_RMS, f"{name}: rel_rms {rel:.3e}"
 
 
 def test_long_backward_keys_with_many_viewers(cuda_lib):
