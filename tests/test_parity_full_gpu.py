@@ -8,8 +8,9 @@
   oracle (rows split across worker processes), and 4096 rows that cover every
   row position of the kernel's tile pair (32 tokens x 8 heads of a KV group)
   at many points of the sequence, in bfloat16 output.
-* The S = 131072 full-causal backward on key rows that 1000-2000 query tokens
-  (x 8 heads) see, so long dK/dV accumulations are compared at full size.
+* The S = 131072 full-causal forward on 1024 tokens x all 32 heads covering
+  every tile-row position, and its backward on key rows that 1000-2000 query
+  tokens (x 8 heads) see, so long dK/dV accumulations are compared at full size.
 All run through the C ABI in the launch configuration bench.py times.
 """
 import multiprocessing as mp
@@ -110,8 +111,17 @@ def test_full_forward_whole_layer_every_element(cuda_lib):
     out, lse = run_fwd(cuda_lib, d, wl.window, wl.use_rope, wl.rope_theta, fp32_out=True)
     torch.cuda.synchronize()
     T, step = wl.total_tokens, 512
-    tasks = [(t0, t0 + step, _np32(out[t0:t0 + step]), _np32(lse[:, t0:t0 + step]))
-             for t0 in range(T - step, -1, -step)]          # the longest rows first
+    chunks = [list(range(t0, t0 + step)) for t0 in range(T - step, -1, -step)]  # longest first
+    _check_rows_in_pool(wl, out, lse, chunks, "full forward (every row)")
+
+
+def _check_rows_in_pool(wl, out, lse, chunks, label):
+    """Compare the GPU's out / lse rows of every token in `chunks` (lists of tokens, all
+    heads) with the oracle, one chunk per task in spawned workers."""
+    tasks = []
+    for toks in chunks:
+        idx = torch.tensor(toks, device=out.device)
+        tasks.append((toks, _np32(out[idx]), _np32(lse[:, idx])))
     workers = max(1, min(len(tasks), os.cpu_count() or 1, 16))
     with mp.get_context("spawn").Pool(workers, initializer=oracle_pool.init_forward_rows,
                                       initargs=(wl.name,)) as pool:
@@ -120,10 +130,28 @@ def test_full_forward_whole_layer_every_element(cuda_lib):
         mx = max(r[name][0] for r in results)
         rel = float(np.sqrt(sum(r[name][1] for r in results) / sum(r[name][2] for r in results)))
         bad = sum(r[name][3] for r in results)
-        print(f"WHOLE full forward {name}: max_abs {mx:.3e} rel_rms {rel:.2e}", flush=True)
+        print(f"WHOLE {label} {name}: max_abs {mx:.3e} rel_rms {rel:.2e}", flush=True)
         assert bad == 0, f"{name}: {bad} non-finite values"
         assert mx <= BF16_MAX_ABS, f"{name}: max_abs {mx:.3e}"
         assert rel <= BF16_REL_RMS, f"{name}: rel_rms {rel:.3e}"
+
+
+def test_long_forward_every_tile_position(cuda_lib):
+    """The 131072-token forward on 1024 tokens x all 32 heads: every (token mod 32,
+    head) position of the kernel's tile pair at 32 places spread over the sequence."""
+    wl = fi.LONG_FULL_BF16
+    cpu = fi.make_inputs(wl, with_grad_out=False)
+    d = to_dev(cpu)
+    out, lse = run_fwd(cuda_lib, d, wl.window, wl.use_rope, wl.rope_theta, fp32_out=True)
+    torch.cuda.synchronize()
+    del d
+    rng = np.random.default_rng(11)
+    n_pairs = wl.total_tokens // 32
+    toks = sorted({int(b) * 32 + off for off in range(32)
+                   for b in rng.choice(n_pairs, size=32, replace=False)}, reverse=True)
+    assert len(toks) == 1024 and toks[0] < wl.total_tokens
+    chunks = [toks[i:i + 64] for i in range(0, len(toks), 64)]
+    _check_rows_in_pool(wl, out, lse, chunks, "long forward (tile positions)")
 
 
 def test_long_backward_keys_with_many_viewers(cuda_lib):
