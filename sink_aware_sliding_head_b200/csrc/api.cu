@@ -31,6 +31,22 @@ cudaError_t launch_attn_bwd_sm100_impl(const CUtensorMap& tq, const CUtensorMap&
                                        const int4* items_q, const int* n_q, int max_q,
                                        float* dq_acc, float* dk_acc, void* dv, int* status,
                                        int num_sms, cudaStream_t st);
+int x3_kv_box_tokens_fwd();
+int x3_q_box_rows_dkv();
+int x3_kv_box_tokens_dq();
+cudaError_t launch_attn_fwd_x3(const CUtensorMap& tq, const CUtensorMap& tk,
+                               const CUtensorMap& tv, const Resolved& p, const float* sink,
+                               const int4* items, const int* n_items, int max_items,
+                               const unsigned* amax, float* out, float* lse, int* status,
+                               int num_sms, cudaStream_t st);
+cudaError_t launch_attn_bwd_x3(const CUtensorMap& tq64, const CUtensorMap& tk128,
+                               const CUtensorMap& tdo64, const CUtensorMap& tk64,
+                               const CUtensorMap& tv64, const Resolved& p, const float* lse,
+                               const float* dvec, const unsigned* amax, const __half* qs,
+                               const __half* dos, const __half* vs, const int4* items_kv,
+                               const int* n_kv, int max_kv, const int4* items_q, const int* n_q,
+                               int max_q, float* dq_acc, float* dk_acc, float* dv, int* status,
+                               int num_sms, cudaStream_t st);
 
 // ------------------------------------------------------------------ kernel timing
 namespace {
@@ -38,7 +54,8 @@ const char* const kKernelNames[kNumKernelIds] = {
     "prologue_rmsnorm_rope", "build_worklist", "attn_fwd_sm100", "attn_fwd_fp32",
     "bwd_preprocess", "reduce_rows", "attn_bwd_dkv_sm100", "attn_bwd_dq_sm100",
     "attn_bwd_dq_fp32", "attn_bwd_dkv_fp32", "prologue_bwd", "convert_f16",
-    "decode", "pad_fill", "absmax"};
+    "decode", "pad_fill", "absmax", "attn_fwd_x3_sm100", "attn_bwd_dkv_x3_sm100",
+    "attn_bwd_dq_x3_sm100"};
 constexpr int kMaxSlots = 1 << 15;
 struct Prof {
   std::mutex mu;
@@ -94,7 +111,8 @@ flint_status_t resolve(const flint_attn_params_t* in, Resolved* p) {
   const int G = in->num_q_heads / in->num_kv_heads;
   if (in->compute_f16 && in->dtype != FLINT_FP32) return FLINT_ERR_INVALID_ARG;
   const bool tc = in->dtype == FLINT_BF16 || in->compute_f16;
-  if (tc && !(G == 1 || G == 2 || G == 4 || G == 8 || G == 16)) return FLINT_ERR_UNSUPPORTED;
+  const bool g_tc = G == 1 || G == 2 || G == 4 || G == 8 || G == 16;
+  if (tc && !g_tc) return FLINT_ERR_UNSUPPORTED;
   if ((long long)in->total_tokens * in->num_q_heads * in->head_dim > 0x7fffffffLL)
     return FLINT_ERR_INVALID_ARG;
   if (!(std::isfinite(in->rms_eps) && in->rms_eps >= 0.f)) return FLINT_ERR_INVALID_ARG;
@@ -115,6 +133,9 @@ flint_status_t resolve(const flint_attn_params_t* in, Resolved* p) {
   p->dtype = in->dtype;
   p->fp32_out = (in->fp32_out != 0 || in->dtype == FLINT_FP32) ? 1 : 0;
   p->tc = tc ? 1 : 0;
+  // FP32 inputs take the split tensor-core path wherever its tiles fit the group
+  // size; other group sizes run the CUDA-core kernels.
+  p->x3 = (!tc && g_tc) ? 1 : 0;
   p->out_f16 = (in->compute_f16 && !in->fp32_out) ? 1 : 0;
   p->R = kTileRows / (G <= 128 ? G : 128);
   if (p->R < 1) p->R = 1;
@@ -213,6 +234,8 @@ flint_status_t fwd_impl(const flint_attn_params_t* params, const void* q, const 
   Resolved p;
   flint_status_t s = resolve(params, &p);
   if (s != FLINT_OK) return s;
+  // padding needs a tensor-core path (the CUDA-core FP32 kernels have none)
+  if (valid && !p.tc && !p.x3) return FLINT_ERR_UNSUPPORTED;
   // With no tokens the [T, ...] tensors are empty and may be null.
   const bool no_tokens = p.T == 0;
   const void* tok16[] = {q, k, v, out};
@@ -233,8 +256,31 @@ flint_status_t fwd_impl(const flint_attn_params_t* params, const void* q, const 
   if (p.T == 0) return FLINT_OK;
   void* qh = at<void>(workspace, L.qhat);
   void* kh = at<void>(workspace, L.khat);
-  const bool f16 = p.tc;   // tensor-core operands are fp16
-  FLINT_TRY(launch_prologue_qk(p, q, q_norm_w, qh, k, k_norm_w, kh, cu_doc_lens, st, f16));
+  unsigned* amax = reinterpret_cast<unsigned*>(status + kSlotAmaxDout);   // [dout, v]
+  if (p.x3) {
+    FLINT_TRY(launch_prologue_qk(p, q, q_norm_w, qh, k, k_norm_w, kh, cu_doc_lens, st,
+                                 kHatSplit));
+    int4* items = at<int4>(workspace, L.items_q);
+    FLINT_TRY(launch_build_worklist(cu_doc_lens, valid, p, kModeQuery, p.R, items, status + 1,
+                                    at<void>(workspace, L.sched_tmp), L.max_items_q, st));
+    __half* vs = at<__half>(workspace, L.v16);
+    FLINT_TRY(launch_absmax(p.dtype, nullptr, 0, v, (size_t)p.T * p.Hk * kHeadDim, amax,
+                            cu_doc_lens, valid, p.N, p.H, p.Hk, st));
+    FLINT_TRY(launch_convert_split(static_cast<const float*>(v), vs, p.T, p.Hk, amax + 1, st));
+    const CUtensorMapDataType f16t = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    CUtensorMap tq, tk, tv;
+    const int kv_box = x3_kv_box_tokens_fwd();
+    if (!encode_3d(&tq, qh, p.T, 2 * p.H, p.G, p.R, f16t) ||
+        !encode_3d(&tk, kh, p.T, 2 * p.Hk, 1, kv_box, f16t) ||
+        !encode_3d(&tv, vs, p.T, 2 * p.Hk, 1, kv_box, f16t))
+      return FLINT_ERR_CUDA;
+    FLINT_TRY(launch_attn_fwd_x3(tq, tk, tv, p, sink, items, status + 1, L.max_items_q, amax,
+                                 static_cast<float*>(out), lse, status, sm_count(), st));
+    if (valid) FLINT_TRY(launch_pad_fill_fwd(p, cu_doc_lens, valid, sink, out, lse, st));
+    return FLINT_OK;
+  }
+  FLINT_TRY(launch_prologue_qk(p, q, q_norm_w, qh, k, k_norm_w, kh, cu_doc_lens, st,
+                               p.tc ? kHatF16 : kHatInput));
   if (!p.tc) {
     return cuda_status(launch_attn_fwd_fp32(p, (const float*)qh, (const float*)kh,
                                             (const float*)v, sink, cu_doc_lens, (float*)out, lse,
@@ -244,7 +290,6 @@ flint_status_t fwd_impl(const flint_attn_params_t* params, const void* q, const 
   FLINT_TRY(launch_build_worklist(cu_doc_lens, valid, p, kModeQuery, 2 * p.R, items, status + 1,
                                   at<void>(workspace, L.sched_tmp), L.max_items_q, st));
   __half* v16 = at<__half>(workspace, L.v16);
-  unsigned* amax = reinterpret_cast<unsigned*>(status + kSlotAmaxDout);   // [dout, v]
   FLINT_TRY(launch_absmax(p.dtype, nullptr, 0, v, (size_t)p.T * p.Hk * kHeadDim, amax,
                           cu_doc_lens, valid, p.N, p.H, p.Hk, st));
   FLINT_TRY(convert_v(p, v, v16, amax + 1, st));
@@ -270,6 +315,8 @@ flint_status_t bwd_impl(const flint_attn_params_t* params, const void* q, const 
   Resolved p;
   flint_status_t s = resolve(params, &p);
   if (s != FLINT_OK) return s;
+  // padding needs a tensor-core path (the CUDA-core FP32 kernels have none)
+  if (valid && !p.tc && !p.x3) return FLINT_ERR_UNSUPPORTED;
   // With no tokens the [T, ...] tensors are empty and may be null.
   const bool no_tokens = p.T == 0;
   const void* tok16[] = {q, k, v, out, dout, dq, dk, dv};
@@ -300,7 +347,7 @@ flint_status_t bwd_impl(const flint_attn_params_t* params, const void* q, const 
   float* part = at<float>(workspace, L.part);
   float* dq_acc = at<float>(workspace, L.dq_acc);
   float* dk_acc = at<float>(workspace, L.dk_acc);
-  const bool f16 = p.tc;   // tensor-core operands of the backward are fp16
+  const bool f16 = p.tc || p.x3;   // tensor-core operands of the backward are fp16
   __half* dout16 = f16 ? at<__half>(workspace, L.dout16) : nullptr;
   __half* v16 = f16 ? at<__half>(workspace, L.v16) : nullptr;
   unsigned* amax = reinterpret_cast<unsigned*>(status + kSlotAmaxDout);   // [dout, v]
@@ -308,10 +355,35 @@ flint_status_t bwd_impl(const flint_attn_params_t* params, const void* q, const 
     FLINT_TRY(launch_absmax(p.dtype, dout, (size_t)p.T * p.H * kHeadDim, v,
                             (size_t)p.T * p.Hk * kHeadDim, amax, cu_doc_lens, valid, p.N, p.H,
                             p.Hk, st));
-  FLINT_TRY(launch_prologue_qk(p, q, q_norm_w, qh, k, k_norm_w, kh, cu_doc_lens, st, f16));
+  FLINT_TRY(launch_prologue_qk(p, q, q_norm_w, qh, k, k_norm_w, kh, cu_doc_lens, st,
+                               p.x3 ? kHatSplit : (p.tc ? kHatF16 : kHatInput)));
   FLINT_TRY(launch_bwd_preprocess(p, out, dout, lse, sink, dvec, part, dsink, dout16,
-                                  f16 ? amax : nullptr, st));
-  if (!p.tc) {
+                                  f16 ? amax : nullptr, st, p.x3));
+  if (p.x3) {
+    int4* items_kv = at<int4>(workspace, L.items_kv);
+    int4* items_q1 = at<int4>(workspace, L.items_q1);
+    FLINT_TRY(launch_build_worklists2(cu_doc_lens, valid, p, kModeKey, kTileKeys, items_kv,
+                                      status + 2, at<void>(workspace, L.sched_tmp),
+                                      L.max_items_kv, kModeQuery, p.R, items_q1, status + 3,
+                                      at<void>(workspace, L.sched_tmp2), L.max_items_q1, st));
+    FLINT_TRY(launch_convert_split(static_cast<const float*>(v), v16, p.T, p.Hk, amax + 1, st));
+    const CUtensorMapDataType f16t = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    const int rows64 = x3_q_box_rows_dkv(), keys_dq = x3_kv_box_tokens_dq();
+    CUtensorMap tq64, tk128, tdo64, tk64, tv64;
+    if (!encode_3d(&tq64, qh, p.T, 2 * p.H, p.G, rows64 / p.G, f16t) ||
+        !encode_3d(&tk128, kh, p.T, 2 * p.Hk, 1, kTileKeys, f16t) ||
+        !encode_3d(&tdo64, dout16, p.T, 2 * p.H, p.G, rows64 / p.G, f16t) ||
+        !encode_3d(&tk64, kh, p.T, 2 * p.Hk, 1, keys_dq, f16t) ||
+        !encode_3d(&tv64, v16, p.T, 2 * p.Hk, 1, keys_dq, f16t))
+      return FLINT_ERR_CUDA;
+    FLINT_TRY(launch_attn_bwd_x3(tq64, tk128, tdo64, tk64, tv64, p, lse, dvec, amax,
+                                 static_cast<const __half*>(qh), dout16, v16, items_kv,
+                                 status + 2, L.max_items_kv, items_q1, status + 3,
+                                 L.max_items_q1, dq_acc, dk_acc, static_cast<float*>(dv), status,
+                                 sm_count(), st));
+    if (valid)
+      FLINT_TRY(launch_pad_fill_bwd(p, cu_doc_lens, valid, dq_acc, dk_acc, dv, 1, st));
+  } else if (!p.tc) {
     FLINT_TRY(launch_attn_bwd_fp32(p, (const float*)qh, (const float*)kh, (const float*)v,
                                    (const float*)dout, lse, dvec, cu_doc_lens, dq_acc, dk_acc,
                                    (float*)dv, st));
@@ -381,7 +453,6 @@ extern "C" flint_status_t flint_attn_fwd_padded(const flint_attn_params_t* param
                                                 void* workspace, size_t workspace_bytes,
                                                 void* stream) {
   if (!padded_args_ok(params, valid_lens)) return FLINT_ERR_INVALID_ARG;
-  if (params->dtype == FLINT_FP32 && !params->compute_f16) return FLINT_ERR_UNSUPPORTED;
   return fwd_impl(params, q, k, v, q_norm_w, k_norm_w, sink, cu_doc_lens, valid_lens, out, lse,
                   workspace, workspace_bytes, stream);
 }
@@ -393,7 +464,6 @@ extern "C" flint_status_t flint_attn_bwd_padded(
     void* dk, void* dv, float* dq_norm_w, float* dk_norm_w, float* dsink, void* workspace,
     size_t workspace_bytes, void* stream) {
   if (!padded_args_ok(params, valid_lens)) return FLINT_ERR_INVALID_ARG;
-  if (params->dtype == FLINT_FP32 && !params->compute_f16) return FLINT_ERR_UNSUPPORTED;
   return bwd_impl(params, q, k, v, q_norm_w, k_norm_w, sink, cu_doc_lens, valid_lens, out, lse,
                   dout, dq, dk, dv, dq_norm_w, dk_norm_w, dsink, workspace, workspace_bytes,
                   stream);

@@ -26,12 +26,14 @@ constexpr int kTok = 4;
 // backward's operands are fp16.
 // amax (nullable): [max|dout|, max|v|] slots; dout16 gets dout * s_dout and dvec
 // D * s_dout * s_v, the scales of the fp16 operands (d_sink uses the plain D).
+// split: dout16 is [T, 2H, D], hi = fp16(dout * s_dout) in row (t, h) and
+// lo = fp16(dout * s_dout - hi) in row (t, H + h).
 template <typename TO, typename T>
 __global__ void __launch_bounds__(kThreads)
 bwd_pre_kernel(const TO* __restrict__ out, const T* __restrict__ dout,
                const float* __restrict__ lse, const float* __restrict__ sink,
                float* __restrict__ dvec, float* __restrict__ part, __half* __restrict__ dout16,
-               const unsigned* __restrict__ amax, int ntok, int H) {
+               const unsigned* __restrict__ amax, int ntok, int H, int split) {
   extern __shared__ float acc[];   // [kGroups][H]
   const int lane16 = threadIdx.x & 15, grp = threadIdx.x >> 4;
   const int c0 = lane16 * 8;
@@ -51,7 +53,18 @@ bwd_pre_kernel(const TO* __restrict__ out, const T* __restrict__ dout,
         const size_t base = ((size_t)t * H + h) * kHeadDim + c0;
         load8(out + base, a);
         load8(dout + base, b);
-        if (dout16) {
+        if (dout16 && split) {
+          float hi[8], lo[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const float x = b[e] * s_do;   // |x| < 8: no saturation needed
+            hi[e] = __half2float(__float2half_rn(x));
+            lo[e] = x - hi[e];
+          }
+          const size_t hb = ((size_t)t * 2 * H + h) * kHeadDim + c0;
+          store8(dout16 + hb, hi);
+          store8(dout16 + hb + (size_t)H * kHeadDim, lo);
+        } else if (dout16) {
           float s8[8];
 #pragma unroll
           for (int e = 0; e < 8; ++e) s8[e] = sat_f16(b[e] * s_do);
@@ -93,6 +106,32 @@ __global__ void convert_f16_kernel(const T* __restrict__ src, __half* __restrict
 #pragma unroll
     for (int e = 0; e < 8; ++e) f[e] = sat_f16(f[e] * sc);
     store8(dst + 8 * i, f);
+  }
+}
+
+// Split copy: x [T][heads][D] -> dst [T][2 heads][D], hi = fp16(x * 2^e) and
+// lo = fp16(x * 2^e - hi); one thread per 8 consecutive channels.
+__global__ void convert_split_kernel(const float* __restrict__ src, __half* __restrict__ dst,
+                                     size_t n8, int heads, const unsigned* __restrict__ amax) {
+  const float sc = slot_scale(amax, false);
+  const int row8 = kHeadDim / 8;
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n8;
+       i += (size_t)gridDim.x * blockDim.x) {
+    const size_t row = i / row8;              // t * heads + h
+    const int c = (int)(i % row8) * 8;
+    const size_t t = row / heads;
+    const int h = (int)(row % heads);
+    float f[8], hi[8], lo[8];
+    load8(src + 8 * i, f);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const float x = f[e] * sc;
+      hi[e] = __half2float(__float2half_rn(x));
+      lo[e] = x - hi[e];
+    }
+    const size_t hb = (t * 2 * heads + h) * kHeadDim + c;
+    store8(dst + hb, hi);
+    store8(dst + hb + (size_t)heads * kHeadDim, lo);
   }
 }
 
@@ -175,6 +214,17 @@ cudaError_t launch_convert_f16(const float* src, __half* dst, size_t n, const un
   return convert_f16(src, dst, n, amax, st);
 }
 
+cudaError_t launch_convert_split(const float* src, __half* dst, int T, int heads,
+                                 const unsigned* amax, cudaStream_t st) {
+  const size_t n8 = (size_t)T * heads * kHeadDim / 8;
+  if (n8 == 0) return cudaSuccess;
+  size_t blocks = (n8 + 255) / 256;
+  if (blocks > 148 * 16) blocks = 148 * 16;
+  ProfScope prof(kKConvert, st);
+  convert_split_kernel<<<(unsigned)blocks, 256, 0, st>>>(src, dst, n8, heads, amax);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_absmax(int dtype, const void* x0, size_t n0, const void* x1, size_t n1,
                           unsigned* amax, const int32_t* cu, const int32_t* valid, int N,
                           int heads0, int heads1, cudaStream_t st) {
@@ -198,7 +248,7 @@ cudaError_t launch_absmax(int dtype, const void* x0, size_t n0, const void* x1, 
 cudaError_t launch_bwd_preprocess(const Resolved& p, const void* out, const void* dout,
                                   const float* lse, const float* sink, float* dvec, float* part,
                                   float* dsink, __half* dout16, const unsigned* amax,
-                                  cudaStream_t st) {
+                                  cudaStream_t st, int split) {
   if (p.T == 0) {
     cudaMemsetAsync(dsink, 0, p.H * sizeof(float), st);
     return cudaGetLastError();
@@ -211,17 +261,17 @@ cudaError_t launch_bwd_preprocess(const Resolved& p, const void* out, const void
   typedef __nv_bfloat16 bf;
   if (p.dtype == FLINT_BF16 && p.fp32_out)
     bwd_pre_kernel<float, bf><<<blocks, kThreads, smem, st>>>(
-        (const float*)out, (const bf*)dout, lse, sink, dvec, part, dout16, amax, p.T, p.H);
+        (const float*)out, (const bf*)dout, lse, sink, dvec, part, dout16, amax, p.T, p.H, 0);
   else if (p.dtype == FLINT_BF16)
     bwd_pre_kernel<bf, bf><<<blocks, kThreads, smem, st>>>(
-        (const bf*)out, (const bf*)dout, lse, sink, dvec, part, dout16, amax, p.T, p.H);
+        (const bf*)out, (const bf*)dout, lse, sink, dvec, part, dout16, amax, p.T, p.H, 0);
   else if (p.out_f16)   // FP32 inputs at the fp16 compute boundary: out is fp16
     bwd_pre_kernel<__half, float><<<blocks, kThreads, smem, st>>>(
-        (const __half*)out, (const float*)dout, lse, sink, dvec, part, dout16, amax, p.T, p.H);
+        (const __half*)out, (const float*)dout, lse, sink, dvec, part, dout16, amax, p.T, p.H, 0);
   else
     bwd_pre_kernel<float, float><<<blocks, kThreads, smem, st>>>(
-        (const float*)out, (const float*)dout, lse, sink, dvec, part, p.tc ? dout16 : nullptr,
-        p.tc ? amax : nullptr, p.T, p.H);
+        (const float*)out, (const float*)dout, lse, sink, dvec, part,
+        (p.tc || split) ? dout16 : nullptr, (p.tc || split) ? amax : nullptr, p.T, p.H, split);
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;

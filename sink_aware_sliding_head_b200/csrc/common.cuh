@@ -66,13 +66,16 @@ struct Resolved {
   int fp32_out;     // out, dq, dk, dv are float32 (always for FP32 inputs)
   int tc;           // the tcgen05 path with fp16 operands: BF16 inputs, or FP32 + compute_f16
   int out_f16;      // out is IEEE fp16 (FP32 inputs with compute_f16, without fp32_out)
+  int x3;           // the tcgen05 path for FP32 inputs: operands split into fp16 hi + lo
+                    // parts, three MMAs per product (no compute_f16; G in {1,2,4,8,16})
   int R;            // tokens per 128-row tile = 128 / G
 };
 
 // Offsets (bytes) of every region of the workspace. All regions are 256-byte aligned.
 struct WsLayout {
   size_t status;        // int[64]: [0] status bits, [1..3] work-list lengths
-  size_t qhat, khat;    // normalised+rotated q [T,H,D], k [T,Hk,D] (dtype)
+  size_t qhat, khat;    // normalised+rotated q [T,H,D], k [T,Hk,D] (dtype; for the
+                        // split path fp16 [T,2H,D], [T,2Hk,D]: hi rows, then lo rows)
   size_t items_q;       // int4 work items, query-major (forward: pairs of tiles)
   size_t items_q1;      // int4 work items, query-major single tiles (backward dQ)
   size_t items_kv;      // int4 work items, key-major (backward dK/dV)
@@ -82,8 +85,9 @@ struct WsLayout {
   size_t part;          // fp32 partial sums (d sink, d norm weights)
   size_t dq_acc;        // [T,H,D] fp32 gradient w.r.t. q_hat (backward)
   size_t dk_acc;        // [T,Hk,D] fp32 gradient w.r.t. k_hat (backward)
-  size_t dout16;        // [T,H,D] fp16 copy of dO (backward, tensor-core path)
-  size_t v16;           // [T,Hk,D] fp16 copy of v (tensor-core path)
+  size_t dout16;        // [T,H,D] fp16 copy of dO (backward, tensor-core path; [T,2H,D]
+                        // hi and lo parts on the split path)
+  size_t v16;           // [T,Hk,D] fp16 copy of v (tensor-core path; [T,2Hk,D] split)
   size_t total;
   int max_items_q, max_items_q1, max_items_kv, max_items_any;
   int part_blocks;      // number of partial-sum rows per reduced quantity
@@ -103,7 +107,8 @@ inline WsLayout make_layout(const Resolved& p, bool backward) {
   L.status = take(64 * sizeof(int));
   L.qhat = take((size_t)p.T * p.H * p.D * eb);
   L.khat = take((size_t)p.T * p.Hk * p.D * eb);
-  L.max_items_q = p.Hk * ((p.T + 2 * p.R - 1) / (2 * p.R) + p.N);
+  const int span_fwd = p.x3 ? p.R : 2 * p.R;   // tokens per forward item
+  L.max_items_q = p.Hk * ((p.T + span_fwd - 1) / span_fwd + p.N);
   L.max_items_q1 = p.Hk * ((p.T + p.R - 1) / p.R + p.N);
   L.max_items_kv = p.Hk * ((p.T + kTileKeys - 1) / kTileKeys + p.N);
   L.max_items_any = L.max_items_q1;
@@ -115,13 +120,14 @@ inline WsLayout make_layout(const Resolved& p, bool backward) {
   L.sched_tmp = take((size_t)L.max_items_any * 20);
   L.sched_tmp2 = backward ? take((size_t)L.max_items_any * 20) : off;
   L.part_blocks = kPartBlocks;
-  if (p.tc) L.v16 = take((size_t)p.T * p.Hk * p.D * 2);
+  const size_t parts = p.x3 ? 2 : 1;   // the split path keeps hi and lo fp16 parts
+  if (p.tc || p.x3) L.v16 = take((size_t)p.T * p.Hk * p.D * 2 * parts);
   if (backward) {
     L.dvec = take((size_t)p.H * p.T * 4);
     L.part = take((size_t)kPartBlocks * (p.H + 2 * p.D) * 4);
     L.dq_acc = take((size_t)p.T * p.H * p.D * 4);
     L.dk_acc = take((size_t)p.T * p.Hk * p.D * 4);
-    if (p.tc) L.dout16 = take((size_t)p.T * p.H * p.D * 2);
+    if (p.tc || p.x3) L.dout16 = take((size_t)p.T * p.H * p.D * 2 * parts);
   }
   L.total = off;
   return L;
@@ -203,7 +209,7 @@ __device__ __forceinline__ void store8(float* p, const float (&f)[8]) {
 enum KernelId {
   kKPrologue = 0, kKWorklist, kKFwdSm100, kKFwdFp32, kKBwdPre, kKReduce, kKBwdDkvSm100,
   kKBwdDqSm100, kKBwdDqFp32, kKBwdDkvFp32, kKPrologueBwd, kKConvert, kKDecode, kKPadFill,
-  kKAbsmax,
+  kKAbsmax, kKFwdX3, kKBwdDkvX3, kKBwdDqX3,
   kNumKernelIds
 };
 struct ProfScope {
@@ -232,11 +238,18 @@ cudaError_t launch_pad_fill_fwd(const Resolved& p, const int32_t* cu, const int3
 cudaError_t launch_pad_fill_bwd(const Resolved& p, const int32_t* cu, const int32_t* valid,
                                 float* dq_acc, float* dk_acc, void* dv, int dv_f32,
                                 cudaStream_t st);
-// q_hat [T,H,D] and k_hat [T,Hk,D] in one launch. out_f16: write them as fp16 (the
-// tensor-core operands) instead of the input type.
+// q_hat [T,H,D] and k_hat [T,Hk,D] in one launch, written as
+enum { kHatInput = 0,    // the input type
+       kHatF16 = 1,      // fp16 (the tensor-core operands)
+       kHatSplit = 2 };  // fp16 hi and lo parts, [T,2H,D] and [T,2Hk,D] (FP32 inputs)
 cudaError_t launch_prologue_qk(const Resolved& p, const void* q, const void* wq, void* qh,
                                const void* k, const void* wk, void* kh, const int32_t* cu,
-                               cudaStream_t st, bool out_f16);
+                               cudaStream_t st, int hat_mode);
+// Split copy of an FP32 tensor x [T,heads,D]: dst [T,2*heads,D] fp16 holds
+// hi = fp16(x * 2^e) in rows [0,heads) of each token and lo = fp16(x * 2^e - hi)
+// in rows [heads, 2*heads); e from the max |x| slot (nullptr: e = 0).
+cudaError_t launch_convert_split(const float* src, __half* dst, int T, int heads,
+                                 const unsigned* amax, cudaStream_t st);
 // dst = fp16(src * 2^e), e from the max |src| in *amax (nullptr: e = 0).
 cudaError_t launch_convert_f16(const __nv_bfloat16* src, __half* dst, size_t n,
                                const unsigned* amax, cudaStream_t st);
@@ -282,11 +295,12 @@ cudaError_t launch_attn_bwd_fp32(const Resolved& p, const float* qh, const float
 // D = rowsum(dout * out) into dvec, d_sink, and (dout16 non-null) the fp16 copy of
 // dout. amax (nullable): the [max|dout|, max|v|] slots; when given, dout16 is
 // dout * s_dout and dvec holds D * s_dout * s_v (the scales of the fp16
-// operands), while d_sink is formed from the unscaled D.
+// operands), while d_sink is formed from the unscaled D. split: dout16 is
+// [T,2H,D] with the hi and lo fp16 parts of dout * s_dout (FP32 inputs).
 cudaError_t launch_bwd_preprocess(const Resolved& p, const void* out, const void* dout,
                                   const float* lse, const float* sink, float* dvec, float* part,
                                   float* dsink, __half* dout16, const unsigned* amax,
-                                  cudaStream_t st);
+                                  cudaStream_t st, int split = 0);
 cudaError_t launch_bwd_epilogue(const Resolved& p, const void* x, const void* w,
                                 const float* g_hat, void* dx, float* dw, float* part, int heads,
                                 const int32_t* cu, cudaStream_t st);

@@ -50,7 +50,9 @@ __device__ void build_rope_table(const int32_t* __restrict__ cu, int N, int T, i
 
 // q and k in one launch: the first nblk0 blocks normalise kTok tokens of x0
 // (heads0 rows per token) each, the rest kTok tokens of x1 (heads1 rows).
-template <typename T, typename TO>
+// kSplit (TO = __half): y is [T, 2*heads, D]; row (t, h) gets hi = fp16(x) and
+// row (t, heads + h) lo = fp16(x - hi), the two parts of the split path.
+template <typename T, typename TO, bool kSplit = false>
 __global__ void __launch_bounds__(kThreads)
 prologue_kernel(const T* __restrict__ x0, const T* __restrict__ w0, TO* __restrict__ y0,
                 int heads0, const T* __restrict__ x1, const T* __restrict__ w1,
@@ -108,7 +110,21 @@ prologue_kernel(const T* __restrict__ x0, const T* __restrict__ w0, TO* __restri
 #pragma unroll
       for (int e = 0; e < 8; ++e) v[e] = o8[e];
     }
-    if (valid) store8(y + base, v);
+    if (valid) {
+      if constexpr (kSplit) {
+        const size_t hb = ((size_t)t * 2 * heads + (rr % heads)) * kHeadDim + c0;
+        float hi[8], lo[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          hi[e] = __half2float(__float2half_rn(v[e]));
+          lo[e] = v[e] - hi[e];   // exact in fp32; rounded once to fp16 by store8
+        }
+        store8(y + hb, hi);
+        store8(y + hb + (size_t)heads * kHeadDim, lo);
+      } else {
+        store8(y + base, v);
+      }
+    }
   }
 }
 
@@ -225,7 +241,8 @@ reduce_rows_kernel(const float* __restrict__ part, int nrows, int width,
 
 cudaError_t launch_prologue_qk(const Resolved& p, const void* q, const void* wq, void* qh,
                                const void* k, const void* wk, void* kh, const int32_t* cu,
-                               cudaStream_t st, bool out_f16) {
+                               cudaStream_t st, int hat_mode) {
+  const bool out_f16 = hat_mode == kHatF16;
   if (p.T == 0) return cudaSuccess;
   const int nblk = (p.T + kTok - 1) / kTok;   // per tensor
   dim3 grid(2 * nblk);
@@ -239,6 +256,10 @@ cudaError_t launch_prologue_qk(const Resolved& p, const void* q, const void* wq,
     prologue_kernel<bf, bf><<<grid, kThreads, 0, st>>>(
         (const bf*)q, (const bf*)wq, (bf*)qh, p.H, (const bf*)k, (const bf*)wk, (bf*)kh, p.Hk,
         nblk, p.T, cu, p.N, p.rope, p.theta, p.eps);
+  else if (hat_mode == kHatSplit)   // FP32 inputs on the split path
+    prologue_kernel<float, __half, true><<<grid, kThreads, 0, st>>>(
+        (const float*)q, (const float*)wq, (__half*)qh, p.H, (const float*)k, (const float*)wk,
+        (__half*)kh, p.Hk, nblk, p.T, cu, p.N, p.rope, p.theta, p.eps);
   else if (out_f16)   // FP32 inputs at the fp16 compute boundary
     prologue_kernel<float, __half><<<grid, kThreads, 0, st>>>(
         (const float*)q, (const float*)wq, (__half*)qh, p.H, (const float*)k, (const float*)wk,

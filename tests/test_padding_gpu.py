@@ -104,8 +104,9 @@ def test_bshd_8192_equals_the_layer_on_the_real_tokens(cuda_lib):
         assert torch.all(g_p[name][rows] == 0), name
 
 
-def test_fp32_padding_is_unsupported(cuda_lib):
-    cpu = fi.make_custom([64], 8, 1, dtype="fp32", seed=1)
+def test_fp32_padding_needs_a_tensor_core_group_size(cuda_lib):
+    """FP32 inputs with G = 3 run the CUDA-core kernels, which have no padded form."""
+    cpu = fi.make_custom([64], 3, 1, dtype="fp32", seed=1)
     d = to_dev(cpu)
     vd = torch.tensor([10], dtype=torch.int32, device="cuda")
     with pytest.raises(cuda_lib.FlintError) as e:
