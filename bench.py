@@ -580,6 +580,10 @@ def main(argv=None):
             pg.barrier()
 
     w = WORKLOADS[args.workload]
+    # FP32 inputs run the split tensor-core kernels (fp16 hi/lo operands, three MMAs
+    # per product); BF16 inputs the fp16-operand ones
+    split = w.dtype == "fp32"
+    fwd_name = "attn_fwd_x3_sm100" if split else "attn_fwd_sm100"
     if args.tokens > 0:
         import dataclasses
         w = dataclasses.replace(w, name=f"{w.name}@{args.tokens}", doc_lens=(args.tokens,),
@@ -764,7 +768,7 @@ def main(argv=None):
         kf = fa.profile_collect()
         clk_f = clocks_f.stop() if clocks_f else None
         call_ms = sum(e[0].elapsed_time(e[1]) for e in fo_ev) / args.steps
-        kms = kf.get("attn_fwd_sm100", (0.0, 0))
+        kms = kf.get(fwd_name, (0.0, 0))
         fwd_only = {
             "ms_per_call": call_ms,
             "call_tflops": ff / (call_ms * 1e-3) / 1e12,
@@ -781,11 +785,16 @@ def main(argv=None):
 
     # ---- roofline of the dominant kernel (live CUDA-event time per launch)
     peaks, peak_src = read_peaks()
-    eb = 2                                  # bf16 inputs; the prologue writes fp16 q_hat / k_hat
-    algo = {  # algorithmic work per launch
+    # bytes per element of the prologue's rows: bf16 in, fp16 q_hat / k_hat out; or
+    # FP32 in, fp16 hi + lo parts out
+    eb = 4 if split else 2
+    algo = {  # algorithmic (useful) work per launch
         "attn_fwd_sm100": ("tensor", 4.0 * D * H * pairs),
         "attn_bwd_dkv_sm100": ("tensor", 8.0 * D * H * pairs),
         "attn_bwd_dq_sm100": ("tensor", 2.0 * D * H * pairs),
+        "attn_fwd_x3_sm100": ("tensor", 4.0 * D * H * pairs),
+        "attn_bwd_dkv_x3_sm100": ("tensor", 8.0 * D * H * pairs),
+        "attn_bwd_dq_x3_sm100": ("tensor", 2.0 * D * H * pairs),
     }
     dom = max(kern.items(), key=lambda kv: kv[1][0])
     dname, (dms, dn) = dom
@@ -793,14 +802,20 @@ def main(argv=None):
     roofline = None
     if dname in algo:
         achieved = algo[dname][1] / (per_launch_ms * 1e-3) / 1e12
-        peak = peaks["bf16_tflops"]
-        src = {"attn_fwd_sm100": "attn_fwd_sm100.cu"}.get(dname, "attn_bwd_sm100.cu")
+        # the split kernels issue three f16 MMAs per useful product: their useful-work
+        # ceiling is a third of the f16/bf16 tensor peak
+        mmas = 3.0 if "_x3_" in dname else 1.0
+        peak = peaks["bf16_tflops"] / mmas
+        src = {"attn_fwd_sm100": "attn_fwd_sm100.cu"}.get(
+            dname, "attn_x3_sm100.cu" if mmas > 1 else "attn_bwd_sm100.cu")
         roofline = {"kernel": dname, "bound": "tensor", "achieved": achieved, "peak": peak,
                     "unit": "TFLOP/s", "frac": achieved / peak,
-                    "peak_kind": f"bf16 burst ({peak_src}); the kernel runs inside a "
-                                 "power-capped step, see frac_of_sustained",
-                    "frac_of_sustained": achieved / peaks["bf16_tflops_sustained"],
-                    "peak_sustained": peaks["bf16_tflops_sustained"],
+                    "peak_kind": f"bf16 burst ({peak_src})" +
+                                 (" / 3 (three MMAs per product)" if mmas > 1 else "") +
+                                 "; the kernel runs inside a power-capped step, see "
+                                 "frac_of_sustained",
+                    "frac_of_sustained": achieved * mmas / peaks["bf16_tflops_sustained"],
+                    "peak_sustained": peaks["bf16_tflops_sustained"] / mmas,
                     "traffic": traffic_for(dname, w.name),
                     "algorithmic_flops_per_launch": algo[dname][1],
                     "ms_per_launch": per_launch_ms, "source": src}
@@ -824,7 +839,7 @@ def main(argv=None):
     kernels = {k: {"ms_per_step": v[0] / args.steps, "launches": v[1],
                    "share": v[0] / max(sum(x[0] for x in kern.values()), 1e-9)}
                for k, v in kern.items() if v[1] > 0}
-    fwd_attn = kern.get("attn_fwd_sm100", (0.0, 0))
+    fwd_attn = kern.get(fwd_name, (0.0, 0))
     fwd_kernel_tflops = (4.0 * D * H * pairs * fwd_attn[1] / (fwd_attn[0] * 1e-3) / 1e12
                          if fwd_attn[1] else None)
 
@@ -837,7 +852,7 @@ def main(argv=None):
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
         "data": "synthetic (seeded N(0,1) q/k/v/dO, norm weights 1+0.1N, FP32 sinks)",
         "config": config_of(w, pairs, flops_step),
         "fwd_tflops": world * ff * args.steps / (fwd_ms * 1e-3) / 1e12,

@@ -80,8 +80,15 @@ BSHD_PADDED_BF16 = Workload(
     num_q_heads=32, num_kv_heads=4, head_dim=128, window=1024, use_rope=True,
     rope_theta=1e6, dtype="bf16", valid_range=(4096, 8192))
 
+# The full-causal layer with FP32 inputs (FP32 attention_compute_dtype, the Flint
+# config page's default): the split tensor-core path at the headline layer's size.
+FULL_FP32 = Workload(
+    name="full_fp32_S32768_H32x4", doc_lens=(32768,), total_tokens=32768,
+    num_q_heads=32, num_kv_heads=4, head_dim=128, window=0, use_rope=False,
+    rope_theta=1e6, dtype="fp32", sink_std=2.0, backward=False)
+
 WORKLOADS = [TINY_SLIDING_FP32, SLIDING_BF16, FULL_BF16, PACKED_BF16, LONG_FULL_BF16,
-             BSHD_PADDED_BF16]
+             BSHD_PADDED_BF16, FULL_FP32]
 
 
 def draw_doc_lens(w: Workload, gen: torch.Generator) -> List[int]:

@@ -63,8 +63,14 @@
  *     operands (q_hat, k_hat, v, P, and in the backward dout and dS) are IEEE
  *     fp16, whose 10-bit mantissa keeps their rounding well below bf16's.
  *     |v| and |dout| must stay below 65504 (larger values saturate).
- *     dtype FLINT_FP32: all tensors are float32 and every step runs in FP32 on
- *     CUDA cores.
+ *     dtype FLINT_FP32: all tensors are float32. With G = 1, 2, 4, 8 or 16 the
+ *     attention contractions run on tcgen05 tensor cores at FP32 accuracy:
+ *     each operand x enters as two fp16 parts, hi = fp16(x) and
+ *     lo = fp16(x - hi), and each product takes three MMAs (hi*hi + hi*lo +
+ *     lo*hi) with FP32 accumulation; v and dout are scaled by powers of two
+ *     (as above), so any float32 magnitude is taken. RMSNorm, RoPE, the
+ *     softmax and every reduction run in FP32. Other group sizes run every
+ *     step in FP32 on CUDA cores (no padded calls there).
  */
 #ifndef FLINT_ATTN_H
 #define FLINT_ATTN_H
@@ -92,7 +98,8 @@ typedef struct {
   int32_t num_docs;       /* N >= 1; zero-length documents are allowed */
   int32_t num_q_heads;    /* H, a multiple of num_kv_heads */
   int32_t num_kv_heads;   /* Hk >= 1; G = H / Hk must be 1, 2, 4, 8 or 16 (tensor-core
-                             paths; FP32 inputs without compute_f16 take any G) */
+                             paths; FP32 inputs without compute_f16 take any G, other
+                             values on CUDA cores) */
   int32_t head_dim;       /* D; must be 128 */
   int32_t window;         /* > 0: key j visible from query i iff 0 <= i - j < window
                              (the current token included); <= 0: full causal */
@@ -163,8 +170,9 @@ flint_status_t flint_attn_bwd(const flint_attn_params_t* params,
  * token (dq, dk, dv) is zero, and padded rows add nothing to dsink or the
  * norm-weight gradients. RoPE positions still count from the document start,
  * so real tokens are unaffected by the padding after them. Same workspace as
- * the unpadded calls; dtype FLINT_BF16 only (FLINT_ERR_UNSUPPORTED for
- * FLINT_FP32). Other arguments as in flint_attn_fwd / flint_attn_bwd. */
+ * the unpadded calls; the tensor-core paths only (FLINT_ERR_UNSUPPORTED for
+ * FLINT_FP32 inputs whose G is not 1, 2, 4, 8 or 16). Other arguments as in
+ * flint_attn_fwd / flint_attn_bwd. */
 flint_status_t flint_attn_fwd_padded(const flint_attn_params_t* params,
                                      const void* q, const void* k, const void* v,
                                      const void* q_norm_w, const void* k_norm_w,
