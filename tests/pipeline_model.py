@@ -1,8 +1,9 @@
 """Model checker for the mbarrier protocols of the pipelined attention kernels.
 
-TEST INFRASTRUCTURE. The forward kernel (csrc/attn_fwd_sm100.cu) and the two
-backward kernels (csrc/attn_bwd_sm100.cu: dK/dV key-major, dQ query-major)
-coordinate a TMA producer thread, an MMA issuing thread and eight math warps
+TEST INFRASTRUCTURE. The forward kernel (csrc/attn_fwd_sm100.cu), the two
+backward kernels (csrc/attn_bwd_sm100.cu: dK/dV key-major, dQ query-major) and
+their FP32-input counterparts (csrc/attn_x3_sm100.cu) coordinate a TMA producer
+thread, an MMA issuing thread and four or eight math warps
 through shared-memory mbarriers. This module restates, role by role, the waits,
 arrivals, commits and buffer accesses of each kernel's normal path (the abort
 and drain paths are left out) and runs them under random interleavings:
@@ -277,10 +278,10 @@ def _ring_pop(k, idx_tag):
     yield ("arrive", f"ring_empty{s}")
 
 
-def _ring_bars(sim):
+def _ring_bars(sim, consumers=MATH_WARPS + 1):
     for s in range(ITEM_SLOTS):
         sim.bar(f"ring_full{s}", 1)
-        sim.bar(f"ring_empty{s}", MATH_WARPS + 1)
+        sim.bar(f"ring_empty{s}", consumers)
 
 
 # ============================================================================
@@ -678,7 +679,432 @@ def backward_dq(sim, items, mut=None):
         sim.role(f"math{w}", math(w >> 2, w & 3))
 
 
-KERNELS = {"forward": forward, "backward_dkv": backward_dkv, "backward_dq": backward_dq}
+# ============================================================================
+# FP32 inputs on the tensor cores (csrc/attn_x3_sm100.cu): every operand has a hi
+# and a lo part. An MMA below stands for the group of MMAs (three per product)
+# that the kernel issues between two barrier operations.
+# ============================================================================
+
+X3_KV_SLOTS_FWD = 5
+X3_KV_SLOTS_DQ = 12
+X3_DRAIN_TILES = 2   # the dK/dV kernel drains every 16 tiles; 2 exercises more drains
+PARTS = ("Kh", "Kl", "Vh", "Vl")
+
+
+def forward_x3(sim, items, mut=None):
+    """attn_fwd_x3_kernel: one query tile per item, two S buffers, 4 softmax warps."""
+    sim.bar("q_full"), sim.bar("q_empty")
+    for s in range(X3_KV_SLOTS_FWD):
+        sim.bar(f"kv_full{s}"), sim.bar(f"kv_empty{s}")
+    for b in range(2):
+        sim.bar(f"s_full{b}"), sim.bar(f"p_half{b}", 4), sim.bar(f"p_full{b}", 4)
+        sim.bar(f"pv_done{b}")
+    sim.bar("o_full"), sim.bar("o_empty", 4)
+    _ring_bars(sim, 5)
+    seq = list(items) + [None]
+    NS = X3_KV_SLOTS_FWD
+
+    def producer():
+        kv_load = 0
+        for item, nt in enumerate(seq):
+            yield from _ring_push(item, ("idx", item))
+            if nt is None:
+                return
+            if item > 0:
+                yield ("wait", "q_empty", item - 1)
+            yield ("expect_tx", "q_full", 2)
+            yield ("tma", ["smem:Qh"], ("Qh", item), "q_full")
+            yield ("tma", ["smem:Ql"], ("Ql", item), "q_full")
+            for j in range(4 * nt):
+                s = kv_load % NS
+                if kv_load >= NS:
+                    yield ("wait", f"kv_empty{s}", kv_load // NS - 1)
+                yield ("expect_tx", f"kv_full{s}", 1)
+                yield ("tma", [f"smem:kv{s}"], (PARTS[j & 3], kv_load // 4), f"kv_full{s}")
+                kv_load += 1
+
+    def mma():
+        t, kv_base, pv = 0, 0, [0, 0]
+
+        def slot_read(pos):
+            return ([f"smem:kv{pos % NS}"], (PARTS[pos & 3], pos // 4))
+
+        def issue_qk(n, tt, item, last):
+            b, pos = tt & 1, kv_base + 4 * n
+            yield ("wait", f"kv_full{pos % NS}", pos // NS)
+            yield ("wait", f"kv_full{(pos + 1) % NS}", (pos + 1) // NS)
+            # implied by the 5-slot ring (K(t+2) lands in the slot of V_lo(t), which
+            # PV(t) releases on completion), kept as in the kernel
+            if pv[b] > 0:
+                yield ("wait", f"pv_done{b}", pv[b] - 1)
+            yield ("mma", [(["smem:Qh"], ("Qh", item)), (["smem:Ql"], ("Ql", item)),
+                           slot_read(pos), slot_read(pos + 1)],
+                   tmem(f"S{b}", ALL_CHUNKS), ("S", tt), False)
+            yield ("commit", f"s_full{b}")
+            yield ("commit", f"kv_empty{pos % NS}")
+            yield ("commit", f"kv_empty{(pos + 1) % NS}")
+            if last:
+                yield ("commit", "q_empty")
+
+        for item, nt in enumerate(seq):
+            yield from _ring_pop(item, ("idx", item))
+            if nt is None:
+                return
+            yield ("wait", "q_full", item)
+            yield from issue_qk(0, t, item, nt == 1)
+            if nt > 1:
+                yield from issue_qk(1, t + 1, item, nt == 2)
+            for n in range(nt):
+                tt = t + n
+                b = tt & 1
+                pos = kv_base + 4 * n + 2
+                yield ("wait", f"kv_full{pos % NS}", pos // NS)
+                yield ("wait", f"kv_full{(pos + 1) % NS}", (pos + 1) // NS)
+                yield ("wait", f"p_half{b}", tt >> 1)
+                if n == 0 and item > 0:
+                    yield ("wait", "o_empty", item - 1)
+                o = tmem("O", ALL_CHUNKS)
+                # keys 0-63: P' hi in chunks 0-1, lo in chunks 2-3 of the S buffer
+                yield ("mma", [(tmem(f"S{b}", [0, 1, 2, 3]), ("P", tt)), slot_read(pos),
+                               slot_read(pos + 1)], o, ("O", item), n > 0)
+                if mut != "x3f_pv_without_p_full":
+                    yield ("wait", f"p_full{b}", tt >> 1)
+                yield ("mma", [(tmem(f"S{b}", [4, 5, 6, 7]), ("P", tt)), slot_read(pos),
+                               slot_read(pos + 1)], o, ("O", item), True)
+                yield ("commit", f"pv_done{b}")
+                pv[b] += 1
+                yield ("commit", f"kv_empty{pos % NS}")
+                yield ("commit", f"kv_empty{(pos + 1) % NS}")
+                if n + 1 == nt:
+                    yield ("commit", "o_full")
+                if n + 2 < nt:
+                    yield from issue_qk(n + 2, tt + 2, item, n + 3 == nt)
+            kv_base += 4 * nt
+            t += nt
+
+    def softmax(q):
+        quarter = [q]
+        t = 0
+        for item, nt in enumerate(seq):
+            yield from _ring_pop(item, ("idx", item))
+            if nt is None:
+                return
+            for n in range(nt):
+                tt = t + n
+                b = tt & 1
+                yield ("wait", f"s_full{b}", tt >> 1)
+                yield ("read", tmem(f"S{b}", ALL_CHUNKS, quarter), ("S", tt))
+                yield ("write", tmem(f"S{b}", [0, 2], quarter), ("P", tt))    # keys 0-31
+                if n > 0 and sim.rng.random() < 0.5:       # lazy rescale of O
+                    if mut != "x3f_rescale_without_pv_done":
+                        yield ("wait", f"pv_done{(tt - 1) & 1}", (tt - 1) >> 1)
+                    o = tmem("O", ALL_CHUNKS, quarter)
+                    yield ("read", o, ("O", item))
+                    yield ("write", o, ("O", item))
+                yield ("write", tmem(f"S{b}", [1, 3], quarter), ("P", tt))    # keys 32-63
+                yield ("arrive", f"p_half{b}")
+                yield ("write", tmem(f"S{b}", [4, 6, 5, 7], quarter), ("P", tt))
+                yield ("arrive", f"p_full{b}")
+            t += nt
+            yield ("wait", "o_full", item)
+            yield ("read", tmem("O", ALL_CHUNKS, quarter), ("O", item))
+            yield ("arrive", "o_empty")
+
+    sim.role("tma", producer())
+    sim.role("mma", mma())
+    for w in range(4):
+        sim.role(f"softmax{w}", softmax(w))
+
+
+def backward_dkv_x3(sim, items, mut=None):
+    """attn_bwd_dkv_x3_kernel: V's parts in TMEM, 64-row query tiles, drains of dV/dK."""
+    sim.bar("kv_full"), sim.bar("kv_empty")
+    for s in range(Q_STAGES_DKV):
+        sim.bar(f"q_full{s}"), sim.bar(f"q_empty{s}")
+    for s in range(2):
+        sim.bar(f"do_full{s}", 2), sim.bar(f"do_empty{s}")
+    for b in ("s_full", "dp_full", "dv_done", "dk_done", "acc_full"):
+        sim.bar(b)
+    for b in ("v_full", "p_full", "ds_full", "acc_empty"):
+        sim.bar(b, MATH_WARPS)
+    _ring_bars(sim)
+    seq = list(items) + [None]
+    QS = Q_STAGES_DKV
+
+    def producer():
+        qd = 0
+        for item, nq in enumerate(seq):
+            yield from _ring_push(item, ("idx", item))
+            if nq is None:
+                return
+            if item > 0:
+                yield ("wait", "kv_empty", item - 1)
+            yield ("expect_tx", "kv_full", 2)
+            yield ("tma", ["smem:Kh"], ("Kh", item), "kv_full")
+            yield ("tma", ["smem:Kl"], ("Kl", item), "kv_full")
+            for m in range(nq):
+                sq, s = qd % QS, qd & 1
+                if qd >= QS:
+                    yield ("wait", f"q_empty{sq}", qd // QS - 1)
+                yield ("expect_tx", f"q_full{sq}", 2)
+                yield ("tma", [f"smem:Q{sq}h"], ("Qh", qd), f"q_full{sq}")
+                yield ("tma", [f"smem:Q{sq}l"], ("Ql", qd), f"q_full{sq}")
+                if qd >= 2:
+                    yield ("wait", f"do_empty{s}", qd // 2 - 1)
+                yield ("expect_tx", f"do_full{s}", 2)
+                yield ("tma", [f"smem:dO{s}h"], ("dOh", qd), f"do_full{s}")
+                yield ("tma", [f"smem:dO{s}l"], ("dOl", qd), f"do_full{s}")
+                yield ("write", [f"smem:stats{s}"], ("st", qd))
+                yield ("arrive", f"do_full{s}")
+                qd += 1
+
+    def q_read(tt):
+        return [([f"smem:Q{tt % QS}h"], ("Qh", tt)), ([f"smem:Q{tt % QS}l"], ("Ql", tt))]
+
+    def do_read(tt):
+        return [([f"smem:dO{tt & 1}h"], ("dOh", tt)), ([f"smem:dO{tt & 1}l"], ("dOl", tt))]
+
+    X, Y = tmem("X", range(4)), tmem("Y", range(4))
+
+    def mma():
+        t, p_cnt, ds_cnt, dv_cnt, dk_cnt, drains = 0, 0, 0, 0, 0, 0
+
+        def issue_s(tt, item):
+            yield ("mma", [(["smem:Kh"], ("Kh", item)), (["smem:Kl"], ("Kl", item))] + q_read(tt),
+                   X, ("ST", tt), False)
+            yield ("commit", "s_full")
+
+        def issue_dp(tt, item):
+            yield ("mma", [(tmem("V", ALL_CHUNKS), ("V", item))] + do_read(tt),
+                   Y, ("dPT", tt), False)
+            yield ("commit", "dp_full")
+
+        for item, nq in enumerate(seq):
+            yield from _ring_pop(item, ("idx", item))
+            if nq is None:
+                return
+            yield ("wait", "kv_full", item)
+            yield ("wait", f"q_full{t % QS}", t // QS)
+            if dv_cnt > 0:
+                yield ("wait", "dv_done", dv_cnt - 1)
+            yield from issue_s(t, item)
+            yield ("wait", "v_full", item)
+            yield ("wait", f"do_full{t & 1}", t >> 1)
+            if dk_cnt > 0:
+                yield ("wait", "dk_done", dk_cnt - 1)
+            yield from issue_dp(t, item)
+            for m in range(nq):
+                has_next = m + 1 < nq
+                c_first = m % X3_DRAIN_TILES == 0
+                c_last = (m + 1) % X3_DRAIN_TILES == 0 or not has_next
+                yield ("wait", "p_full", p_cnt)
+                p_cnt += 1
+                # implied by p_full (a math warp arrives on it only after its own drain),
+                # kept as in the kernel
+                if c_first and drains > 0:
+                    yield ("wait", "acc_empty", drains - 1)
+                yield ("mma", [(X, ("PT", t))] + do_read(t), tmem("dV", ALL_CHUNKS),
+                       ("dV", drains), not c_first)
+                yield ("commit", "dv_done")
+                dv_cnt += 1
+                if has_next:
+                    if mut != "x3k_s_without_dv_done":
+                        yield ("wait", "dv_done", dv_cnt - 1)
+                    yield ("wait", f"q_full{(t + 1) % QS}", (t + 1) // QS)
+                    yield from issue_s(t + 1, item)
+                yield ("wait", "ds_full", ds_cnt)
+                ds_cnt += 1
+                yield ("commit", f"do_empty{t & 1}")
+                yield ("mma", [(Y, ("dST", t))] + q_read(t), tmem("dK", ALL_CHUNKS),
+                       ("dK", drains), not c_first)
+                yield ("commit", "dk_done")
+                dk_cnt += 1
+                yield ("commit", f"q_empty{t % QS}")
+                if c_last:
+                    yield ("commit", "acc_full")
+                    drains += 1
+                if has_next:
+                    yield ("wait", "dk_done", dk_cnt - 1)
+                    yield ("wait", f"do_full{(t + 1) & 1}", (t + 1) >> 1)
+                    yield from issue_dp(t + 1, item)
+                t += 1
+            yield ("commit", "kv_empty")
+
+    def math(wg, q):
+        quarter = [q]
+        mine = [2 * wg, 2 * wg + 1]                # query columns [32wg, 32wg+32)
+        chans = [4 * wg + c for c in range(4)]     # channels [64wg, 64wg+64)
+        t, drains = 0, 0
+        early_v = False
+        for item, nq in enumerate(seq):
+            yield from _ring_pop(item, ("idx", item))
+            if nq is None:
+                return
+            if not early_v:
+                # V's parts: warpgroup 0 the hi part (chunks 0-3), 1 the lo part (4-7)
+                yield ("write", tmem("V", chans, quarter), ("V", item))
+                yield ("arrive", "v_full")
+            early_v = False
+            for m in range(nq):
+                has_next = m + 1 < nq
+                yield ("wait", f"do_full{t & 1}", t >> 1)
+                yield ("wait", "s_full", t)
+                yield ("read", tmem("X", mine, quarter), ("ST", t))
+                yield ("read", [f"smem:stats{t & 1}"], ("st", t))
+                yield ("write", tmem("X", mine, quarter), ("PT", t))
+                yield ("arrive", "p_full")
+                if mut == "x3k_v_before_last_dp" and not has_next and seq[item + 1]:
+                    # planted: the next item's V while this item's last dP^T may still run
+                    yield ("write", tmem("V", chans, quarter), ("V", item + 1))
+                    yield ("arrive", "v_full")
+                    early_v = True
+                yield ("wait", "dp_full", t)
+                yield ("read", tmem("Y", mine, quarter), ("dPT", t))
+                yield ("read", [f"smem:stats{t & 1}"], ("st", t))
+                yield ("write", tmem("Y", mine, quarter), ("dST", t))
+                yield ("arrive", "ds_full")
+                if (m + 1) % X3_DRAIN_TILES == 0 or not has_next:
+                    yield ("wait", "acc_full", drains)
+                    yield ("read", tmem("dV", chans, quarter), ("dV", drains))
+                    yield ("read", tmem("dK", chans, quarter), ("dK", drains))
+                    yield ("arrive", "acc_empty")
+                    drains += 1
+                t += 1
+
+    sim.role("tma", producer())
+    sim.role("mma", mma())
+    for w in range(MATH_WARPS):
+        sim.role(f"math{w}", math(w >> 2, w & 3))
+
+
+def backward_dq_x3(sim, items, mut=None):
+    """attn_bwd_dq_x3_kernel: Q's and dO's parts in TMEM, 64-key tiles, rotating regions."""
+    NS = X3_KV_SLOTS_DQ
+    for s in range(NS):
+        sim.bar(f"kv_full{s}"), sim.bar(f"kv_empty{s}")
+    for b in ("s_full", "dp_full", "dq_done", "acc_full"):
+        sim.bar(b)
+    for b in ("qd_full", "dp_free", "ds_full", "acc_empty"):
+        sim.bar(b, MATH_WARPS)
+    _ring_bars(sim)
+    seq = list(items) + [None]
+
+    def region(tt):
+        return "R" + str(tt & 1)
+
+    def producer():
+        kv_load = 0
+        for item, nt in enumerate(seq):
+            yield from _ring_push(item, ("idx", item))
+            if nt is None:
+                return
+            for j in range(4 * nt):
+                s = kv_load % NS
+                if kv_load >= NS:
+                    yield ("wait", f"kv_empty{s}", kv_load // NS - 1)
+                yield ("expect_tx", f"kv_full{s}", 1)
+                yield ("tma", [f"smem:kv{s}"], (PARTS[j & 3], kv_load // 4), f"kv_full{s}")
+                kv_load += 1
+
+    def mma():
+        t, kv_base, dpf_cnt, ds_cnt, dq_cnt = 0, 0, 0, 0, 0
+
+        def slot_read(pos):
+            return ([f"smem:kv{pos % NS}"], (PARTS[pos & 3], pos // 4))
+
+        def issue_s(n, tt, item):
+            pos = kv_base + 4 * n
+            yield ("wait", f"kv_full{pos % NS}", pos // NS)
+            yield ("wait", f"kv_full{(pos + 1) % NS}", (pos + 1) // NS)
+            yield ("mma", [(tmem("QD", range(8)), ("Q", item)), slot_read(pos),
+                           slot_read(pos + 1)], tmem(region(tt), range(4)), ("S", tt), False)
+            yield ("commit", "s_full")
+
+        def issue_dp(n, tt, item):
+            pos = kv_base + 4 * n + 2
+            yield ("wait", f"kv_full{pos % NS}", pos // NS)
+            yield ("wait", f"kv_full{(pos + 1) % NS}", (pos + 1) // NS)
+            yield ("mma", [(tmem("QD", range(8, 16)), ("dO", item)), slot_read(pos),
+                           slot_read(pos + 1)], tmem(region(tt + 1), range(4)), ("dP", tt),
+                   False)
+            yield ("commit", "dp_full")
+            yield ("commit", f"kv_empty{pos % NS}")
+            yield ("commit", f"kv_empty{(pos + 1) % NS}")
+
+        for item, nt in enumerate(seq):
+            yield from _ring_pop(item, ("idx", item))
+            if nt is None:
+                return
+            yield ("wait", "qd_full", item)
+            if t > 0:
+                yield ("wait", "dp_free", dpf_cnt - 1)
+            yield from issue_s(0, t, item)
+            if dq_cnt > 0:
+                yield ("wait", "dq_done", dq_cnt - 1)
+            yield from issue_dp(0, t, item)
+            for n in range(nt):
+                tt = t + n
+                has_next = n + 1 < nt
+                if has_next:
+                    if mut != "x3d_s_without_dp_free":
+                        yield ("wait", "dp_free", dpf_cnt)
+                    yield from issue_s(n + 1, tt + 1, item)
+                dpf_cnt += 1
+                yield ("wait", "ds_full", ds_cnt)
+                ds_cnt += 1
+                if n == 0 and item > 0:
+                    yield ("wait", "acc_empty", item - 1)
+                pos = kv_base + 4 * n
+                yield ("mma", [(tmem(region(tt), range(4)), ("dS", tt)), slot_read(pos),
+                               slot_read(pos + 1)], tmem("dQ", ALL_CHUNKS), ("dQ", item), n > 0)
+                yield ("commit", "dq_done")
+                dq_cnt += 1
+                yield ("commit", f"kv_empty{pos % NS}")
+                yield ("commit", f"kv_empty{(pos + 1) % NS}")
+                if has_next:
+                    if mut != "x3d_dp_without_dq_done":
+                        yield ("wait", "dq_done", dq_cnt - 1)
+                    yield from issue_dp(n + 1, tt + 1, item)
+            yield ("commit", "acc_full")
+            kv_base += 4 * nt
+            t += nt
+
+    def math(wg, q):
+        quarter = [q]
+        mine = [2 * wg, 2 * wg + 1]                # keys [32wg, 32wg+32) of a tile
+        t = 0
+        for item, nt in enumerate(seq):
+            yield from _ring_pop(item, ("idx", item))
+            if nt is None:
+                return
+            # Q's parts (warpgroup 0, chunks 0-7) or dO's (warpgroup 1, chunks 8-15)
+            yield ("write", tmem("QD", range(8 * wg, 8 * wg + 8), quarter),
+                   ("dO" if wg else "Q", item))
+            yield ("arrive", "qd_full")
+            for n in range(nt):
+                X, Y = region(t), region(t + 1)
+                yield ("wait", "s_full", t)
+                yield ("read", tmem(X, mine, quarter), ("S", t))
+                yield ("wait", "dp_full", t)
+                yield ("read", tmem(Y, mine, quarter), ("dP", t))
+                yield ("arrive", "dp_free")
+                yield ("write", tmem(X, mine, quarter), ("dS", t))
+                yield ("arrive", "ds_full")
+                t += 1
+            if mut != "x3d_epilogue_without_acc_full":
+                yield ("wait", "acc_full", item)
+            yield ("read", tmem("dQ", [4 * wg + c for c in range(4)], quarter), ("dQ", item))
+            yield ("arrive", "acc_empty")
+
+    sim.role("tma", producer())
+    sim.role("mma", mma())
+    for w in range(MATH_WARPS):
+        sim.role(f"math{w}", math(w >> 2, w & 3))
+
+
+KERNELS = {"forward": forward, "backward_dkv": backward_dkv, "backward_dq": backward_dq,
+           "forward_x3": forward_x3, "backward_dkv_x3": backward_dkv_x3,
+           "backward_dq_x3": backward_dq_x3}
 
 # planted mistakes: (kernel, mutation)
 MUTATIONS = [
@@ -691,6 +1117,13 @@ MUTATIONS = [
     ("backward_dq", "dq_s_without_dq_done"),
     ("backward_dq", "dq_qd_empty_before_last_dp"),
     ("backward_dq", "dq_k_released_after_dp"),
+    ("forward_x3", "x3f_pv_without_p_full"),
+    ("forward_x3", "x3f_rescale_without_pv_done"),
+    ("backward_dkv_x3", "x3k_s_without_dv_done"),
+    ("backward_dkv_x3", "x3k_v_before_last_dp"),
+    ("backward_dq_x3", "x3d_s_without_dp_free"),
+    ("backward_dq_x3", "x3d_dp_without_dq_done"),
+    ("backward_dq_x3", "x3d_epilogue_without_acc_full"),
 ]
 
 

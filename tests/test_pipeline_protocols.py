@@ -1,4 +1,4 @@
-"""The mbarrier protocols of the three pipelined kernels, model-checked on the CPU.
+"""The mbarrier protocols of the six pipelined kernels, model-checked on the CPU.
 
 ``tests/pipeline_model.py`` restates each kernel's roles (TMA producer, MMA
 issuer, eight math warps) with their waits, arrivals, commits and buffer
@@ -17,6 +17,9 @@ ITEM_LISTS = {
     "forward": [[1], [3], [1, 1, 1, 1], [2, 5, 1, 3], [6, 1, 2]],
     "backward_dkv": [[1], [4], [1, 1, 1, 1, 1], [3, 1, 5, 2]],
     "backward_dq": [[1], [4], [1, 1, 1, 1, 1, 1], [3, 1, 5, 2, 1]],
+    "forward_x3": [[1], [3], [1, 1, 1, 1], [2, 5, 1, 3], [6, 1, 2]],
+    "backward_dkv_x3": [[1], [4], [1, 1, 1, 1, 1], [3, 1, 5, 2]],
+    "backward_dq_x3": [[1], [4], [1, 1, 1, 1, 1, 1], [3, 1, 5, 2, 1]],
 }
 SEEDS = 30
 
