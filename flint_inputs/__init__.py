@@ -85,7 +85,7 @@ BSHD_PADDED_BF16 = Workload(
 FULL_FP32 = Workload(
     name="full_fp32_S32768_H32x4", doc_lens=(32768,), total_tokens=32768,
     num_q_heads=32, num_kv_heads=4, head_dim=128, window=0, use_rope=False,
-    rope_theta=1e6, dtype="fp32", sink_std=2.0, backward=False)
+    rope_theta=1e6, dtype="fp32", sink_std=2.0)
 
 WORKLOADS = [TINY_SLIDING_FP32, SLIDING_BF16, FULL_BF16, PACKED_BF16, LONG_FULL_BF16,
              BSHD_PADDED_BF16, FULL_FP32]

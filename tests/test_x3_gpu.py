@@ -153,3 +153,31 @@ def test_split_path_with_padding(cuda_lib):
     _compare_all(out, lse, g, O, L, R, "padded")
     assert torch.all(out[120:300] == 0)
     assert torch.all(g["dq"][120:300] == 0) and torch.all(g["dv"][120:300] == 0)
+
+
+def test_split_path_full_size_sampled(cuda_lib):
+    """The 32768-token full-causal layer with FP32 inputs: sampled rows of every output
+    against the row oracle at max-abs 1e-4, including the keys at the document start,
+    which every one of the 32768 x 8 query rows of their group sees (the longest
+    accumulation of the dK/dV kernel)."""
+    wl = fi.FULL_FP32
+    cpu = fi.make_inputs(wl)
+    d = to_dev(cpu)
+    out, lse, g, k = _run(cuda_lib, cpu, wl.window, wl.use_rope, wl.rope_theta)
+    for name in SPLIT_KERNELS:
+        assert k[name][1] == 1, name
+    ro = fo.RowOracle(cpu["q"], cpu["k"], cpu["v"], cpu["w_q"], cpu["w_k"], cpu["sink"],
+                      cpu["cu_doc_lens"], wl.window, wl.use_rope, wl.rope_theta, dO=cpu["dout"])
+    T = wl.total_tokens
+    toks = [0, 1, 127, 128, 255, 4095, 16383, 16384, T - 129, T - 1]
+    O, L = ro.forward_rows(toks)
+    _check("full fp32 out rows", out[toks], O)
+    _check("full fp32 lse rows", lse[:, toks], L)
+    rng = np.random.default_rng(3)
+    rows = [(t, int(rng.integers(0, wl.num_q_heads))) for t in toks]
+    _check("full fp32 dq rows", torch.stack([g["dq"][t, h] for t, h in rows]),
+           np.stack([ro.dq_row(t, h) for t, h in rows]))
+    for kv, keys in ((0, [0, 1, 127, 128, 16383]), (3, [T - 130, T - 1])):
+        dk, dv = ro.dkv_rows(keys, kv)
+        _check(f"full fp32 dk rows kv{kv}", g["dk"][keys, kv], dk)
+        _check(f"full fp32 dv rows kv{kv}", g["dv"][keys, kv], dv)
