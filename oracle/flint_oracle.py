@@ -478,7 +478,7 @@ class RowOracle:
                     L[h, n] = m[r] + np.log(Z[r])
         return O, L
 
-    def dkv_rows(self, keys, kv, chunk=256):
+    def dkv_rows(self, keys, kv, chunk=256, tokens=None):
         """``dkv_row`` for several keys of KV head ``kv`` at once.
 
         The same definition: every query row (i, h) that sees a key contributes
@@ -486,6 +486,12 @@ class RowOracle:
         with p, D_i = dO_i . O_i and O_i from that row's full visible set. The
         query rows are taken ``chunk`` at a time as one matrix of logits, so keys
         with thousands of viewing rows stay affordable. Returns (dk, dv) [n, D].
+
+        ``tokens`` (optional): only query rows whose token is in this collection
+        contribute. dv_j and dk_hat_j are sums over rows and the transpose of the
+        prologue is linear in dk_hat_j, so the results for a partition of the
+        viewing tokens add up to the whole (a long layer's rows can be split
+        across processes).
         """
         keys = [int(j) for j in keys]
         G = self.H // self.Hk
@@ -496,6 +502,8 @@ class RowOracle:
             d0, d1 = _doc_of(self.cu, j)
             hi = d1 if self.window <= 0 else min(d1, j + self.window)
             rows.update(range(j, hi))
+        if tokens is not None:
+            rows &= {int(t) for t in tokens}
         rows = sorted(rows)
         pairs = [(i, h) for i in rows for h in heads]
         K, V = self.k_hat_kv[kv], self.v_kv[kv]

@@ -75,3 +75,33 @@ def forward_rows_check(task):
         stats[name] = (float(np.max(np.abs(err))), float(np.sum(err * err)), float(np.sum(r * r)),
                        int(np.sum(~np.isfinite(g))))
     return stats
+
+
+# ---------------------------------------------------------------------------
+# Key rows of a long layer, their viewing query rows split across workers.
+# RowOracle.dkv_rows restricted to a part of the query tokens gives that part's
+# share of dk and dv (the shares add up: pinned on the CPU), so each worker takes
+# a range of query tokens; every worker draws the inputs from their seed.
+# ---------------------------------------------------------------------------
+_DKV_ORACLE = None
+
+
+def init_dkv_rows(workload_name):
+    global _DKV_ORACLE
+    import dataclasses
+    import flint_inputs as fi
+    wl = {w.name: w for w in fi.WORKLOADS}[workload_name]
+    wl = dataclasses.replace(wl, backward=True)
+    cpu = fi.make_inputs(wl, with_grad_out=True)
+    with threadpool_limits(limits=1):
+        _DKV_ORACLE = fo.RowOracle(cpu["q"], cpu["k"], cpu["v"], cpu["w_q"], cpu["w_k"],
+                                   cpu["sink"], cpu["cu_doc_lens"], wl.window, wl.use_rope,
+                                   wl.rope_theta, dO=cpu["dout"])
+
+
+def dkv_rows_part(task):
+    """task: (keys, kv, first query token, end query token). Returns this token
+    range's share of (dk, dv) [n, D] for the keys."""
+    keys, kv, t0, t1 = task
+    with threadpool_limits(limits=1):
+        return _DKV_ORACLE.dkv_rows(keys, kv, tokens=range(t0, t1))

@@ -395,6 +395,30 @@ def test_row_oracle_batched_key_rows_match_whole_layer():
                 np.testing.assert_allclose(dv, g["dv"][keys, kv], atol=1e-12)
 
 
+def test_row_oracle_key_rows_split_by_query_tokens_add_up():
+    """dkv_rows restricted to the query tokens of each part of a partition adds up to
+    the whole-layer backward (how a long layer's rows are split across processes)."""
+    H, Hk, D = 4, 2, 16
+    q, k, v, wq, wk, sink, cu, dO = rand_case([60, 21], H, Hk, D, seed=43)
+    for W, rope in [(0, True), (13, False)]:
+        g = fo.flint_attn_bwd(q, k, v, wq, wk, sink, cu, W, rope, 1e4, dO)
+        ro = fo.RowOracle(q, k, v, wq, wk, sink, cu, W, rope, 1e4, dO=dO)
+        keys = [0, 1, 30, 59, 60]
+        parts = [range(0, 7), range(7, 31), [31, 33, 35], [32, 34] + list(range(36, 81))]
+        for kv in range(Hk):
+            dk = np.zeros((len(keys), D))
+            dv = np.zeros((len(keys), D))
+            for part in parts:
+                a, b = ro.dkv_rows(keys, kv, chunk=5, tokens=part)
+                dk += a
+                dv += b
+            np.testing.assert_allclose(dk, g["dk"][keys, kv], atol=1e-12)
+            np.testing.assert_allclose(dv, g["dv"][keys, kv], atol=1e-12)
+            # a part that no viewing query falls in contributes nothing
+            a, b = ro.dkv_rows([59], kv, tokens=range(0, 59))
+            assert not np.any(a) and not np.any(b)
+
+
 def test_config_constants_golden():
     """Constants the Flint pages print, as used by the workloads."""
     with open(os.path.join(GOLDEN, "flint_config_constants.json")) as f:

@@ -11,6 +11,8 @@
 * The S = 131072 full-causal forward on 1024 tokens x all 32 heads covering
   every tile-row position, and its backward on key rows that 1000-2000 query
   tokens (x 8 heads) see, so long dK/dV accumulations are compared at full size.
+* dK and dV of the first keys of the S = 32768 and S = 131072 layers, which every
+  query row of their group sees: the longest accumulations of the dK/dV kernel.
 All run through the C ABI in the launch configuration bench.py times.
 """
 import multiprocessing as mp
@@ -169,3 +171,54 @@ def test_long_backward_keys_with_many_viewers(cuda_lib):
         dk, dv = ro.dkv_rows(keys, kv)
         compare(g["dk"][keys, kv], dk, "bf16", f"dk rows kv{kv}")
         compare(g["dv"][keys, kv], dv, "bf16", f"dv rows kv{kv}")
+
+
+def _first_keys_check(cuda_lib, wl, keys, workers):
+    """dK, dV of keys at the start of a full-causal document, which every query row of
+    their group sees (the longest dK/dV accumulations of the layer), against the row
+    oracle with the viewing query tokens split across spawned workers."""
+    import dataclasses
+    wl = dataclasses.replace(wl, backward=True)
+    cpu = fi.make_inputs(wl, with_grad_out=True)
+    d = to_dev(cpu)
+    out, lse = run_fwd(cuda_lib, d, wl.window, wl.use_rope, wl.rope_theta, fp32_out=True)
+    g = run_bwd(cuda_lib, d, out, lse, wl.window, wl.use_rope, wl.rope_theta)
+    torch.cuda.synchronize()
+    gk = g["dk"][keys, 0].clone()
+    gv = g["dv"][keys, 0].clone()
+    del d, out, lse, g, cpu
+    T = wl.total_tokens
+    # row i costs ~i (its visible keys): equal-cost token ranges split at T * sqrt(k / n)
+    n = 8 * workers
+    bounds = sorted({0, T} | {int(T * np.sqrt(k / n)) for k in range(1, n)})
+    tasks = [(keys, 0, a, b) for a, b in zip(bounds[:-1], bounds[1:]) if b > a]
+    tasks.reverse()                                       # the costly ranges first
+    with mp.get_context("spawn").Pool(workers, initializer=oracle_pool.init_dkv_rows,
+                                      initargs=(wl.name,)) as pool:
+        parts = pool.map(oracle_pool.dkv_rows_part, tasks, chunksize=1)
+    dk = sum(p[0] for p in parts)
+    dv = sum(p[1] for p in parts)
+    compare(gk, dk, "bf16", f"{wl.name} dk of keys {keys}")
+    compare(gv, dv, "bf16", f"{wl.name} dv of keys {keys}")
+    print(f"FIRST KEYS {wl.name}: dk max-abs {float(np.max(np.abs(gk.double().cpu().numpy() - dk))):.3e}"
+          f", dv {float(np.max(np.abs(gv.double().cpu().numpy() - dv))):.3e}")
+
+
+def _workers(gb_each):
+    """Worker processes: at most 16, one per core, and as many as host memory holds."""
+    try:
+        ram_gb = os.sysconf("SC_PAGE_SIZE") * os.sysconf("SC_PHYS_PAGES") / 2 ** 30
+    except (ValueError, OSError):
+        ram_gb = 64.0
+    return max(1, min(os.cpu_count() or 1, 16, int(ram_gb * 0.6 // gb_each)))
+
+
+def test_full_backward_first_keys(cuda_lib):
+    """The S = 32768 layer's first keys: 32768 x 8 viewing query rows each."""
+    _first_keys_check(cuda_lib, fi.FULL_BF16, [0, 1, 2, 127, 128], _workers(2))
+
+
+def test_long_backward_first_keys(cuda_lib):
+    """The S = 131072 layer's first keys: 131072 x 8 viewing query rows each
+    (the oracle's ~1.7e13 FLOPs take about 2.5 minutes on 16 cores)."""
+    _first_keys_check(cuda_lib, fi.LONG_FULL_BF16, [0, 1, 128], _workers(6))
