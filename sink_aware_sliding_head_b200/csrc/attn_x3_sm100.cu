@@ -23,7 +23,7 @@
 // global counter, bounded mbarrier waits, one elected lane issues MMAs):
 //  * fwd_x3: one 128-row query tile (R tokens x the G heads of a KV group) per
 //    item; K and V tiles of 128 keys stream through a ring of five 32 KB slots
-//    (one fp16 part per slot). TMEM: two S buffers (QK of the next key tile
+//    (one fp16 part per slot, K one tile ahead of V). TMEM: two S buffers (QK of the next key tile
 //    runs while the softmax works on this one) and O. P' = 2^kPBias P is split
 //    into hi/lo over the S buffer it came from and is the TMEM A operand of PV.
 //  * dkv_x3: key-major, 128 keys of one KV head per item, streaming 64-row
@@ -165,8 +165,24 @@ __device__ __forceinline__ FItem decode_f(const X3Args& a, int idx) {
   return r;
 }
 
-// Tiles are numbered per CTA across items (t): tile t uses S buffer t & 1, and
-// its K_hi, K_lo, V_hi, V_lo parts take ring positions 4t .. 4t + 3.
+// An item's K and V parts go through the ring with K one key tile ahead of V:
+// K(0), then K(n+1), V(n) for n = 0, 1, ..., and V(nt-1) last (hi part, then
+// lo part, each). K(n+2) then lands in slots that QK(n+1) and PV(n-1) free, so
+// QK(n+2) never waits for a load, and V(n+1) loads while QK(n+2) runs. Load
+// positions within the item (in single-part loads; the lo part follows):
+__device__ __forceinline__ uint32_t fwd_pos_k(uint32_t n) { return n == 0 ? 0u : 4 * n - 2; }
+__device__ __forceinline__ uint32_t fwd_pos_v(uint32_t n, uint32_t nt) {
+  return n + 1 < nt ? 4 * n + 4 : 4 * n + 2;
+}
+// Which tile (and whether K or V) the item's pj-th part pair is.
+__device__ __forceinline__ void fwd_pair(int pj, int nt, int& tile, bool& is_v) {
+  if (pj == 0) { tile = 0; is_v = false; return; }
+  const int r = pj - 1;
+  if (r < 2 * (nt - 1)) { tile = (r >> 1) + ((r & 1) ? 0 : 1); is_v = (r & 1) != 0; }
+  else { tile = nt - 1; is_v = true; }
+}
+
+// Tiles are numbered per CTA across items (t): tile t uses S buffer t & 1.
 __global__ void __launch_bounds__(kFThreads, 1)
 attn_fwd_x3_kernel(const __grid_constant__ CUtensorMap tm_q,
                    const __grid_constant__ CUtensorMap tm_k,
@@ -235,14 +251,17 @@ attn_fwd_x3_kernel(const __grid_constant__ CUtensorMap tm_q,
             tma_load_3d(sbase + kFOffQ + part * kPart128 + c * kChunk128, &tm_q, qf, c * 64,
                         part * a.H + it.g * a.G, it.q0);
         for (int j = 0; j < 4 * it.ntiles && ok; ++j, ++kv_load) {
-          const int ks = it.kend - kTileKeys * ((j >> 2) + 1);
+          int tile;
+          bool is_v;
+          fwd_pair(j >> 1, it.ntiles, tile, is_v);
+          const int ks = it.kend - kTileKeys * (tile + 1);
           const uint32_t s = kv_load % kFSlots, ph = (kv_load / kFSlots) & 1;
           if (kv_load >= kFSlots) ok = mbar_wait(smem_u32(&bars->kv_empty[s]), ph ^ 1, wc);
           if (!ok) break;
           const uint32_t f = smem_u32(&bars->kv_full[s]);
           mbar_arrive_expect_tx(f, kPart128);
           ++arm[s];
-          const CUtensorMap* m = (j & 2) ? &tm_v : &tm_k;
+          const CUtensorMap* m = is_v ? &tm_v : &tm_k;
           const int y = (j & 1) ? a.Hk + it.g : it.g;   // lo part rows follow the hi rows
           for (int c = 0; c < 2; ++c)
             tma_load_3d(sbase + kFOffKV + s * kPart128 + c * kChunk128, m, f, c * 64, y, ks);
@@ -272,7 +291,7 @@ attn_fwd_x3_kernel(const __grid_constant__ CUtensorMap tm_q,
     };
     // S(tt) = Q K(tt)^T for tile n of the item; last: the item's last QK frees Q.
     auto issue_qk = [&](uint32_t n, uint32_t tt, bool last) -> bool {
-      const uint32_t b = tt & 1, pos = kv_base + 4 * n;
+      const uint32_t b = tt & 1, pos = kv_base + fwd_pos_k(n);
       if (!wait_full(pos) || !wait_full(pos + 1)) return false;
       if (pv_cnt[b] > 0 &&
           !mbar_wait_warp(smem_u32(&bars->pv_done[b]), (pv_cnt[b] - 1) & 1, wc))
@@ -307,7 +326,7 @@ attn_fwd_x3_kernel(const __grid_constant__ CUtensorMap tm_q,
       if (ok && nt > 1) ok = issue_qk(1, t + 1, nt == 2);
       for (uint32_t n = 0; n < nt && ok; ++n) {
         const uint32_t tt = t + n, b = tt & 1, ph = (tt >> 1) & 1;
-        const uint32_t pos = kv_base + 4 * n + 2;               // V_hi, V_lo
+        const uint32_t pos = kv_base + fwd_pos_v(n, nt);        // V_hi, V_lo
         ok = wait_full(pos) && wait_full(pos + 1);
         if (ok) ok = mbar_wait_warp(smem_u32(&bars->p_half[b]), ph, wc);
         if (ok && n == 0 && item_count > 0)

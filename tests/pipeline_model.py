@@ -715,30 +715,41 @@ def forward_x3(sim, items, mut=None):
             yield ("expect_tx", "q_full", 2)
             yield ("tma", ["smem:Qh"], ("Qh", item), "q_full")
             yield ("tma", ["smem:Ql"], ("Ql", item), "q_full")
-            for j in range(4 * nt):
-                s = kv_load % NS
-                if kv_load >= NS:
-                    yield ("wait", f"kv_empty{s}", kv_load // NS - 1)
-                yield ("expect_tx", f"kv_full{s}", 1)
-                yield ("tma", [f"smem:kv{s}"], (PARTS[j & 3], kv_load // 4), f"kv_full{s}")
-                kv_load += 1
+            # K one key tile ahead of V: K(0), then K(n+1), V(n), ..., V(nt-1)
+            order = [("K", 0)]
+            for n in range(nt):
+                if n + 1 < nt:
+                    order.append(("K", n + 1))
+                order.append(("V", n))
+            for kind, n in order:
+                for part in ("h", "l"):
+                    s = kv_load % NS
+                    if kv_load >= NS:
+                        yield ("wait", f"kv_empty{s}", kv_load // NS - 1)
+                    yield ("expect_tx", f"kv_full{s}", 1)
+                    yield ("tma", [f"smem:kv{s}"], (kind + part, item, n), f"kv_full{s}")
+                    kv_load += 1
 
     def mma():
         t, kv_base, pv = 0, 0, [0, 0]
 
-        def slot_read(pos):
-            return ([f"smem:kv{pos % NS}"], (PARTS[pos & 3], pos // 4))
+        def pos_k(n):
+            return 0 if n == 0 else 4 * n - 2
+
+        def pos_v(n, nt):
+            return 4 * n + 4 if n + 1 < nt else 4 * n + 2
+
+        def slot_read(pos, tag):
+            return ([f"smem:kv{pos % NS}"], tag)
 
         def issue_qk(n, tt, item, last):
-            b, pos = tt & 1, kv_base + 4 * n
+            b, pos = tt & 1, kv_base + pos_k(n)
             yield ("wait", f"kv_full{pos % NS}", pos // NS)
             yield ("wait", f"kv_full{(pos + 1) % NS}", (pos + 1) // NS)
-            # implied by the 5-slot ring (K(t+2) lands in the slot of V_lo(t), which
-            # PV(t) releases on completion), kept as in the kernel
-            if pv[b] > 0:
+            if pv[b] > 0 and mut != "x3f_qk_without_pv_done":
                 yield ("wait", f"pv_done{b}", pv[b] - 1)
             yield ("mma", [(["smem:Qh"], ("Qh", item)), (["smem:Ql"], ("Ql", item)),
-                           slot_read(pos), slot_read(pos + 1)],
+                           slot_read(pos, ("Kh", item, n)), slot_read(pos + 1, ("Kl", item, n))],
                    tmem(f"S{b}", ALL_CHUNKS), ("S", tt), False)
             yield ("commit", f"s_full{b}")
             yield ("commit", f"kv_empty{pos % NS}")
@@ -757,7 +768,8 @@ def forward_x3(sim, items, mut=None):
             for n in range(nt):
                 tt = t + n
                 b = tt & 1
-                pos = kv_base + 4 * n + 2
+                pos = kv_base + pos_v(n, nt)
+                vh, vl = slot_read(pos, ("Vh", item, n)), slot_read(pos + 1, ("Vl", item, n))
                 yield ("wait", f"kv_full{pos % NS}", pos // NS)
                 yield ("wait", f"kv_full{(pos + 1) % NS}", (pos + 1) // NS)
                 yield ("wait", f"p_half{b}", tt >> 1)
@@ -765,12 +777,12 @@ def forward_x3(sim, items, mut=None):
                     yield ("wait", "o_empty", item - 1)
                 o = tmem("O", ALL_CHUNKS)
                 # keys 0-63: P' hi in chunks 0-1, lo in chunks 2-3 of the S buffer
-                yield ("mma", [(tmem(f"S{b}", [0, 1, 2, 3]), ("P", tt)), slot_read(pos),
-                               slot_read(pos + 1)], o, ("O", item), n > 0)
+                yield ("mma", [(tmem(f"S{b}", [0, 1, 2, 3]), ("P", tt)), vh, vl], o,
+                       ("O", item), n > 0)
                 if mut != "x3f_pv_without_p_full":
                     yield ("wait", f"p_full{b}", tt >> 1)
-                yield ("mma", [(tmem(f"S{b}", [4, 5, 6, 7]), ("P", tt)), slot_read(pos),
-                               slot_read(pos + 1)], o, ("O", item), True)
+                yield ("mma", [(tmem(f"S{b}", [4, 5, 6, 7]), ("P", tt)), vh, vl], o,
+                       ("O", item), True)
                 yield ("commit", f"pv_done{b}")
                 pv[b] += 1
                 yield ("commit", f"kv_empty{pos % NS}")
@@ -1118,6 +1130,7 @@ MUTATIONS = [
     ("backward_dq", "dq_qd_empty_before_last_dp"),
     ("backward_dq", "dq_k_released_after_dp"),
     ("forward_x3", "x3f_pv_without_p_full"),
+    ("forward_x3", "x3f_qk_without_pv_done"),
     ("forward_x3", "x3f_rescale_without_pv_done"),
     ("backward_dkv_x3", "x3k_s_without_dv_done"),
     ("backward_dkv_x3", "x3k_v_before_last_dp"),
