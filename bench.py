@@ -60,6 +60,9 @@ def parse_args(argv=None):
                          "on; decode_* workloads time flint_attn_decode instead")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--graph", action="store_true",
+                    help="also time the step replayed from a CUDA graph (the forward and "
+                         "backward calls captured once), reported under 'graph'")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--tokens", type=int, default=0,
@@ -668,6 +671,43 @@ def main(argv=None):
                                                 flops_step, args.steps, pg)
     ms_step = tot_ms / args.steps
 
+    # ---- the same step replayed from a CUDA graph (both calls captured once): the
+    # launch overhead of the ~17 kernels per step drops out
+    graph = None
+    if args.graph:
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            fwd_call(d)
+            bwd_call(d)
+        stream.wait_stream(side)
+        torch.cuda.synchronize(dev)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            fwd_call(d)
+            bwd_call(d)
+        for _ in range(args.warmup):
+            flush.zero_()
+            g.replay()
+        torch.cuda.synchronize(dev)
+        gev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)]
+               for _ in range(args.steps)]
+        barrier()
+        torch.cuda.synchronize(dev)
+        for i in range(args.steps):
+            flush.zero_()
+            gev[i][0].record(stream)
+            g.replay()
+            gev[i][1].record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+        g_val, (g_ms,) = aggregate([sum(e[0].elapsed_time(e[1]) for e in gev)], world,
+                                   flops_step, args.steps, pg)
+        graph = {"value": g_val, "unit": UNIT, "ms_per_step": g_ms / args.steps,
+                 "note": "flint_attn_fwd + flint_attn_bwd captured once in a CUDA graph and "
+                         "replayed, same inputs, same L2 flush before each step"}
+        del g
+
     # ---- end to end: host (pinned) inputs -> device -> both calls -> host results.
     # Every step copies its inputs in and all its results (O, LSE, dq, dk, dv,
     # dw_q, dw_k, d_sink) out. The copies run on their own streams, double
@@ -890,6 +930,7 @@ def main(argv=None):
         "gpu_launches": launches,
         "clocks": clk,
         "e2e": e2e,
+        "graph": graph,
         "cpu_baseline": cpu_baseline,
     }
     print(json.dumps(line), flush=True)
