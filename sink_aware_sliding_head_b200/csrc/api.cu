@@ -489,7 +489,7 @@ flint_status_t resolve_decode(const flint_decode_params_t* d, DecodeLayout* L) {
       (d->use_rope && !(d->rope_theta > 0.f)))
     return FLINT_ERR_INVALID_ARG;
   const size_t B = d->batch, H = d->num_q_heads;
-  const size_t S = decode_splits(d->cache_capacity, d->window);
+  const size_t S = decode_splits_max(d->cache_capacity, d->window);
   L->status = 0;
   L->counters = 64 * sizeof(int);
   L->part_o = round256(L->counters + B * d->num_kv_heads * sizeof(int));
@@ -529,6 +529,7 @@ extern "C" flint_status_t flint_attn_decode(const flint_decode_params_t* params,
   D.B = params->batch; D.C = params->cache_capacity;
   D.H = params->num_q_heads; D.Hk = params->num_kv_heads;
   D.W = params->window; D.rope = params->use_rope ? 1 : 0; D.out_f32 = params->fp32_out ? 1 : 0;
+  D.num_sms = sm_count();
   D.theta = params->rope_theta; D.eps = params->rms_eps;
   D.scale = params->softmax_scale > 0.f ? params->softmax_scale
                                         : 1.0f / sqrtf((float)kHeadDim);

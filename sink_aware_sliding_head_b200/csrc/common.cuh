@@ -268,10 +268,11 @@ cudaError_t launch_absmax(int dtype, const void* x0, size_t n0, const void* x1, 
 cudaError_t launch_wait_selftest(long long limit, int arrive_first, int* status,
                                  cudaStream_t st);
 
-// Decode over a KV cache (decode.cu). Keys per split CTA of the window.
-constexpr int kChunkKeysDecode = 1024;
+// Decode over a KV cache (decode.cu). A (sequence, KV head) window is split into
+// chunks of at least kMinChunkKeysDecode keys (a multiple of the 16-key step).
+constexpr int kMinChunkKeysDecode = 256;
 struct DecodeLaunch {
-  int B, C, H, Hk, W, rope, out_f32;
+  int B, C, H, Hk, W, rope, out_f32, num_sms;
   float theta, eps, scale;
   const void *q, *k, *v, *wq, *wk;
   const float* sink;
@@ -283,7 +284,10 @@ struct DecodeLaunch {
   float* lse;
   int* status;
 };
-int decode_splits(int C, int W);    // split CTAs per (sequence, KV head)
+// Split CTAs per (sequence, KV head): the most any call with capacity C and window W
+// launches (the workspace is sized for it), and the count a launch uses.
+int decode_splits_max(int C, int W);
+int decode_splits(int B, int Hk, int C, int W, int num_sms);
 cudaError_t launch_decode(const DecodeLaunch& L, cudaStream_t st);
 cudaError_t launch_attn_fwd_fp32(const Resolved& p, const float* qh, const float* kh,
                                  const float* v, const float* sink, const int32_t* cu, float* out,

@@ -11,7 +11,9 @@
 //
 // Decode is bound by HBM: every key costs 512 bytes of K and V and feeds only
 // the G query heads of its group. One kernel, grid (splits, Hk, B); each CTA
-// covers kChunkKeysDecode keys of one (sequence, KV head) window:
+// covers one chunk of one (sequence, KV head) window (the splits divide the
+// largest window evenly in multiples of 16 keys; their number aims at about
+// five CTAs per SM, see decode_splits):
 //   * it normalises and rotates the G query rows of its group itself (RMSNorm
 //     + RoPE at position p, a warp per row, kept in fp32 and pre-scaled by
 //     softmax_scale * log2(e)); the CTA whose chunk holds slot p also computes
@@ -56,7 +58,7 @@ constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescale = 8.0f;               // log2 units
 
 struct DecArgs {
-  int B, C, H, Hk, G, W, rope, splits, out_f32;
+  int B, C, H, Hk, G, W, rope, splits, chunk, out_f32;   // splits: stride of the partials
   float theta, eps, scale_log2;
   const __nv_bfloat16 *q, *k, *v, *wq, *wk;
   const float* sink;
@@ -167,10 +169,10 @@ __global__ void __launch_bounds__(kDecThreads) decode_attn_kernel(const DecArgs 
     return;
   }
   const int lo = window_lo(a, p);
-  const int k0 = lo + s * kChunkKeysDecode;
+  const int k0 = lo + s * a.chunk;
   if (k0 > p) return;                                // this split has no keys
-  const int k1 = min(k0 + kChunkKeysDecode, p + 1);  // keys [k0, k1)
-  const int nsplit = (p - lo + kChunkKeysDecode) / kChunkKeysDecode;
+  const int k1 = min(k0 + a.chunk, p + 1);           // keys [k0, k1)
+  const int nsplit = (p - lo + a.chunk) / a.chunk;
   const bool owner = k1 == p + 1;                    // this CTA reads slot p
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int gid = lane >> 2, tig = lane & 3;
@@ -450,9 +452,31 @@ __global__ void __launch_bounds__(kDecThreads) decode_attn_kernel(const DecArgs 
 
 }  // namespace
 
-int decode_splits(int C, int W) {
-  const int maxkeys = (W > 0) ? (W < C ? W : C) : C;
-  return (maxkeys + kChunkKeysDecode - 1) / kChunkKeysDecode;
+namespace {
+int max_window_keys(int C, int W) { return (W > 0) ? (W < C ? W : C) : C; }
+// Keys per chunk when the largest window is divided into s splits: even shares,
+// rounded up to the 16-key step.
+int chunk_keys(int C, int W, int s) {
+  const int per = (max_window_keys(C, W) + s - 1) / s;
+  return (per + kStepKeys - 1) / kStepKeys * kStepKeys;
+}
+}  // namespace
+
+int decode_splits_max(int C, int W) {
+  return (max_window_keys(C, W) + kMinChunkKeysDecode - 1) / kMinChunkKeysDecode;
+}
+
+// About five CTAs per SM over all (sequence, KV head) pairs: at three resident CTAs
+// per SM that is two waves, the second nearly full. Measured on the 64-sequence,
+// window-4096 serving shape (256 pairs, 148 SMs): 3 splits of 1376 keys 4235 GB/s of
+// K and V, 4 of 1024 4100, 5 of 832 4040, 2 of 2048 3690.
+int decode_splits(int B, int Hk, int C, int W, int num_sms) {
+  const long long pairs = (long long)B * Hk;
+  long long s = pairs > 0 ? (5LL * num_sms + pairs / 2) / pairs : 1;
+  const int smax = decode_splits_max(C, W);
+  if (s < 1) s = 1;
+  if (s > smax) s = smax;
+  return (int)s;
 }
 
 cudaError_t launch_decode(const DecodeLaunch& L, cudaStream_t st) {
@@ -463,7 +487,9 @@ cudaError_t launch_decode(const DecodeLaunch& L, cudaStream_t st) {
   a.B = L.B; a.C = L.C; a.H = L.H; a.Hk = L.Hk; a.G = L.H / L.Hk; a.W = L.W;
   a.rope = L.rope; a.theta = L.theta; a.eps = L.eps;
   a.scale_log2 = L.scale * kLog2e;
-  a.splits = decode_splits(L.C, L.W);
+  a.splits = decode_splits_max(L.C, L.W);            // stride of the partials
+  const int launched = decode_splits(L.B, L.Hk, L.C, L.W, L.num_sms);
+  a.chunk = chunk_keys(L.C, L.W, launched);
   a.out_f32 = L.out_f32;
   a.q = static_cast<const __nv_bfloat16*>(L.q);
   a.k = static_cast<const __nv_bfloat16*>(L.k);
@@ -477,7 +503,7 @@ cudaError_t launch_decode(const DecodeLaunch& L, cudaStream_t st) {
   a.counters = L.counters; a.part_o = L.part_o; a.part_ml = L.part_ml;
   a.out = L.out; a.lse = L.lse; a.status = L.status;
   ProfScope prof(kKDecode, st);
-  decode_attn_kernel<<<dim3(a.splits, a.Hk, a.B), kDecThreads, kAttnSmem, st>>>(a);
+  decode_attn_kernel<<<dim3(launched, a.Hk, a.B), kDecThreads, kAttnSmem, st>>>(a);
   return cudaGetLastError();
 }
 
