@@ -1,7 +1,7 @@
-// attn_fp32.cu - sink-aware attention in FP32 on CUDA cores, for FP32 inputs.
-//
-// TF32 tensor cores keep 10 mantissa bits, too few for FP32 parity, so FP32
-// inputs take this path: plain FP32 FMA with online softmax.
+// attn_fp32.cu - sink-aware attention in FP32 on CUDA cores, for FP32 inputs
+// whose group size G has no tensor-core tile (G not 1, 2, 4, 8 or 16; the others
+// take the split tensor-core path of attn_x3_sm100.cu): plain FP32 FMA with
+// online softmax.
 //
 // Definition (Flint layers page, nemo_automodel.components.models.flint.layers,
 // FlintAttention.forward and _FlintSinkParameters.forward): for query row
