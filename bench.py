@@ -158,6 +158,15 @@ class ClockSampler:
                  "-lms", "200"], stdout=self.f, stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
+            return
+        # nvidia-smi's start-up (driver and NVML initialisation) can hold up this
+        # process's launches for a second or more; a step that short would time the
+        # stall. Start timing once the first sample is written (at most 10 s).
+        t_end = time.time() + 10.0
+        while time.time() < t_end and self.proc.poll() is None:
+            if os.path.getsize(self.path) > 0:
+                break
+            time.sleep(0.02)
 
     def stop(self, device_index=None):
         if self.proc is None:

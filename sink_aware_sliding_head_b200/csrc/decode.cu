@@ -22,13 +22,17 @@
 //   * its 4 warps take 16-key steps, each staging its own K and V rows into
 //     shared memory with cp.async (double buffered, coalesced 16-byte copies
 //     of the head-major cache). The two small contractions run on mma.sync
-//     m16n8k16 (bf16 in, fp32 accumulate): S = Q K^T with the G heads as 16
-//     padded rows and q_hat split into bf16 hi + lo parts (two MMAs), and
-//     O += P V with P in bf16. Tensor throughput is not the limit here (16
-//     padded rows per 16 keys), so the per-SM tcgen05/TMEM machinery of the
-//     prefill kernels would add nothing; K fragments come from ldmatrix, V
-//     fragments from ldmatrix.trans, and P is the S accumulator re-packed in
-//     registers. Online softmax with a lazily rescaled running max;
+//     m16n8k16 (bf16 in, fp32 accumulate) with q_hat split into bf16 hi + lo
+//     parts. For G <= 8, S = Q K^T takes the hi parts as rows 0-7 and the lo
+//     parts as rows 8-15 of one A operand (each lane adds its two halves), and
+//     the PV product runs transposed, O^T += V^T P^T, so the 8 heads are the
+//     MMA's N and the P fragment a lane holds is already the B operand; for
+//     9 <= G <= 16 the heads are the 16 rows of both products. Tensor
+//     throughput is not the limit here, so the per-SM tcgen05/TMEM machinery
+//     of the prefill kernels would add nothing; K fragments come from
+//     ldmatrix, V fragments from ldmatrix.trans, and P is the S accumulator
+//     re-packed in registers. Online softmax with a lazily rescaled running
+//     max;
 //   * the warps merge in shared memory and the CTA writes one unnormalised
 //     partial (m, l, O); the last CTA of the (sequence, KV head) to finish (an
 //     atomic counter per pair) folds the sink in once (m = sink, l = 1 before
@@ -154,8 +158,20 @@ __device__ __forceinline__ uint32_t bf16x2_bits(float lo, float hi) {
 __device__ __forceinline__ float bf16_round(float x) {
   return __bfloat162float(__float2bfloat16_rn(x));
 }
+// the two bf16 halves of a packed pair as floats
+__device__ __forceinline__ float bf16_lo(uint32_t x) { return __uint_as_float(x << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t x) { return __uint_as_float(x & 0xffff0000u); }
 
-__global__ void __launch_bounds__(kDecThreads) decode_attn_kernel(const DecArgs a) {
+// kPack (G <= 8): the 16 rows of the S MMA's A operand hold q_hat's bf16 hi
+// parts (rows 0-7) and lo parts (rows 8-15) of the same heads, so one MMA
+// gives both partial products and a lane adds its own c0 + c2 (c1 + c3); the
+// PV product then runs transposed (O^T += V^T P^T: the 8 heads are the MMA's
+// N, and the P fragment a lane holds is already the B operand). This halves
+// the MMAs, the exponentials and the O registers of the padded layout.
+// Otherwise (9 <= G <= 16) the rows are the heads and the hi and lo parts take
+// one MMA each.
+template <bool kPack>
+__global__ void __launch_bounds__(kDecThreads, 3) decode_attn_kernel(const DecArgs a) {
   extern __shared__ __align__(128) uint8_t dsmem[];
   // q_hat rows of the group (log2 units): only until they are in registers, so
   // they share the staging area
@@ -214,8 +230,9 @@ __global__ void __launch_bounds__(kDecThreads) decode_attn_kernel(const DecArgs 
   __threadfence_block();
   __syncthreads();                                   // slot p written before it is staged
 
-  // q_hat fragments (rows = heads of the group, zero past G), bf16 hi + lo
-  uint32_t qa_hi[8][4], qa_lo[8][4];
+  // q_hat fragments, bf16 hi + lo parts (zero past G)
+  constexpr int kQParts = kPack ? 1 : 2;
+  uint32_t qa[kQParts][8][4];
   {
     const bool v0 = gid < a.G, v1 = gid + 8 < a.G;
     const float* q0 = qs[gid];
@@ -224,10 +241,11 @@ __global__ void __launch_bounds__(kDecThreads) decode_attn_kernel(const DecArgs 
     for (int kk = 0; kk < 8; ++kk) {
 #pragma unroll
       for (int r = 0; r < 4; ++r) {
-        // a0: (row gid, k 2tig..+1), a1: (row gid+8, same), a2: (row gid, k+8), a3: (row gid+8, k+8)
+        // a0: (row gid, k 2tig..+1), a1: (row gid+8, same), a2: (row gid, k+8),
+        // a3: (row gid+8, k+8)
         const int d = kk * 16 + 2 * tig + ((r & 2) ? 8 : 0);
-        const bool hv = (r & 1) ? v1 : v0;
-        const float* qr = (r & 1) ? q1 : q0;
+        const bool hv = (kPack || !(r & 1)) ? v0 : v1;
+        const float* qr = (kPack || !(r & 1)) ? q0 : q1;
         float x0 = 0.f, x1 = 0.f;
         if (hv) {
           const float2 t = *reinterpret_cast<const float2*>(qr + d);
@@ -235,8 +253,12 @@ __global__ void __launch_bounds__(kDecThreads) decode_attn_kernel(const DecArgs 
           x1 = t.y;
         }
         const float h0f = bf16_round(x0), h1f = bf16_round(x1);
-        qa_hi[kk][r] = bf16x2_bits(h0f, h1f);
-        qa_lo[kk][r] = bf16x2_bits(x0 - h0f, x1 - h1f);
+        if constexpr (kPack) {
+          qa[0][kk][r] = (r & 1) ? bf16x2_bits(x0 - h0f, x1 - h1f) : bf16x2_bits(h0f, h1f);
+        } else {
+          qa[0][kk][r] = bf16x2_bits(h0f, h1f);
+          qa[1][kk][r] = bf16x2_bits(x0 - h0f, x1 - h1f);
+        }
       }
     }
   }
@@ -259,10 +281,13 @@ __global__ void __launch_bounds__(kDecThreads) decode_attn_kernel(const DecArgs 
     }
   };
 
-  float o[16][4];
+  // kPack: O^T, 8 m-tiles of 16 dims x the 8 heads (lane: dims mt*16 + gid and
+  // + 8, heads 2tig, 2tig+1); otherwise O, 16 n-tiles of 8 dims x 16 head rows
+  constexpr int kOTiles = kPack ? 8 : 16;
+  float o[kOTiles][4];
 #pragma unroll
-  for (int n = 0; n < 16; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
-  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;   // rows gid, gid + 8
+  for (int n = 0; n < kOTiles; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;   // rows (heads) gid, gid + 8
 
   // Each iteration commits one group (empty past the last step), so the wait
   // count below is constant: the group of the step being computed is done.
@@ -282,24 +307,57 @@ __global__ void __launch_bounds__(kDecThreads) decode_attn_kernel(const DecArgs 
     const uint32_t ks = wsm + buf * kStageBytes, vs = ks + kStepKeys * kRowBytes;
     const int kb = k0 + step * kStepKeys;
 
-    // S = q_hat K^T for keys kb .. kb+15 (two 8-key n-tiles)
+    // S = q_hat K^T for keys kb .. kb+15 (two 8-key n-tiles); sc[nt][0..1] row
+    // gid, sc[nt][2..3] row gid + 8 (heads 8-15, !kPack only)
     float sc[2][4];
+    if constexpr (kPack) {
+      // even and odd k-steps accumulate apart: four independent chains of four
+      float acc[2][2][4];
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
-      sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+          acc[nt][h][0] = acc[nt][h][1] = acc[nt][h][2] = acc[nt][h][3] = 0.f;
 #pragma unroll
       for (int kp = 0; kp < 4; ++kp) {               // pairs of 16-dim k-steps
-        uint32_t bk[4];
-        const int key = nt * 8 + (lane & 7);
-        const int col = kp * 32 + (lane >> 3) * 8;   // dims
-        ldsm_x4(ks + key * kRowBytes + col * 2, bk);
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int kk = 2 * kp + h;
-          mma_bf16_16816(sc[nt], qa_hi[kk][0], qa_hi[kk][1], qa_hi[kk][2], qa_hi[kk][3],
-                         bk[2 * h], bk[2 * h + 1]);
-          mma_bf16_16816(sc[nt], qa_lo[kk][0], qa_lo[kk][1], qa_lo[kk][2], qa_lo[kk][3],
-                         bk[2 * h], bk[2 * h + 1]);
+        for (int nt = 0; nt < 2; ++nt) {
+          uint32_t bk[4];
+          const int key = nt * 8 + (lane & 7);
+          const int col = kp * 32 + (lane >> 3) * 8;   // dims
+          ldsm_x4(ks + key * kRowBytes + col * 2, bk);
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int kk = 2 * kp + h;
+            mma_bf16_16816(acc[nt][h], qa[0][kk][0], qa[0][kk][1], qa[0][kk][2], qa[0][kk][3],
+                           bk[2 * h], bk[2 * h + 1]);
+          }
+        }
+      }
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {               // hi part (row gid) + lo part (row gid + 8)
+        sc[nt][0] = (acc[nt][0][0] + acc[nt][1][0]) + (acc[nt][0][2] + acc[nt][1][2]);
+        sc[nt][1] = (acc[nt][0][1] + acc[nt][1][1]) + (acc[nt][0][3] + acc[nt][1][3]);
+        sc[nt][2] = sc[nt][3] = -INFINITY;
+      }
+    } else {
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
+#pragma unroll
+        for (int kp = 0; kp < 4; ++kp) {             // pairs of 16-dim k-steps
+          uint32_t bk[4];
+          const int key = nt * 8 + (lane & 7);
+          const int col = kp * 32 + (lane >> 3) * 8; // dims
+          ldsm_x4(ks + key * kRowBytes + col * 2, bk);
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int kk = 2 * kp + h;
+            mma_bf16_16816(sc[nt], qa[0][kk][0], qa[0][kk][1], qa[0][kk][2], qa[0][kk][3],
+                           bk[2 * h], bk[2 * h + 1]);
+            mma_bf16_16816(sc[nt], qa[1][kk][0], qa[1][kk][1], qa[1][kk][2], qa[1][kk][3],
+                           bk[2 * h], bk[2 * h + 1]);
+          }
         }
       }
     }
@@ -311,54 +369,87 @@ __global__ void __launch_bounds__(kDecThreads) decode_attn_kernel(const DecArgs 
       if (j + 1 >= k1) sc[nt][1] = sc[nt][3] = -INFINITY;
     }
     float mx0 = fmaxf(fmaxf(sc[0][0], sc[0][1]), fmaxf(sc[1][0], sc[1][1]));
-    float mx1 = fmaxf(fmaxf(sc[0][2], sc[0][3]), fmaxf(sc[1][2], sc[1][3]));
     mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
     mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
-    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
-    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
     // lazy rescale: the running max moves only when it grows by more than 2^8
-    if (mx0 > m0 + kRescale || m0 == -INFINITY) {
-      const float alpha = (m0 == -INFINITY) ? 0.f : exp2f(m0 - mx0);
-      m0 = mx0;
-      l0 *= alpha;
+    if constexpr (kPack) {
+      float alpha = 1.f;                             // head gid's factor (< 2^-8 when it moves)
+      if (mx0 > m0 + kRescale || m0 == -INFINITY) {
+        alpha = (m0 == -INFINITY) ? 0.f : exp2f(m0 - mx0);
+        m0 = mx0;
+        l0 *= alpha;
+      }
+      if (__any_sync(0xffffffffu, alpha != 1.f)) {
+        // this lane's O^T columns are heads 2tig and 2tig+1, whose factors the
+        // lanes gid = 2tig (lane 8tig) and gid = 2tig+1 (lane 8tig+4) hold
+        const float a_lo = __shfl_sync(0xffffffffu, alpha, 8 * tig);
+        const float a_hi = __shfl_sync(0xffffffffu, alpha, 8 * tig + 4);
 #pragma unroll
-      for (int n = 0; n < 16; ++n) { o[n][0] *= alpha; o[n][1] *= alpha; }
-    }
-    if (mx1 > m1 + kRescale || m1 == -INFINITY) {
-      const float alpha = (m1 == -INFINITY) ? 0.f : exp2f(m1 - mx1);
-      m1 = mx1;
-      l1 *= alpha;
+        for (int n = 0; n < kOTiles; ++n) {
+          o[n][0] *= a_lo; o[n][1] *= a_hi; o[n][2] *= a_lo; o[n][3] *= a_hi;
+        }
+      }
+    } else {
+      if (mx0 > m0 + kRescale || m0 == -INFINITY) {
+        const float alpha = (m0 == -INFINITY) ? 0.f : exp2f(m0 - mx0);
+        m0 = mx0;
+        l0 *= alpha;
 #pragma unroll
-      for (int n = 0; n < 16; ++n) { o[n][2] *= alpha; o[n][3] *= alpha; }
+        for (int n = 0; n < kOTiles; ++n) { o[n][0] *= alpha; o[n][1] *= alpha; }
+      }
+      float mx1 = fmaxf(fmaxf(sc[0][2], sc[0][3]), fmaxf(sc[1][2], sc[1][3]));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+      if (mx1 > m1 + kRescale || m1 == -INFINITY) {
+        const float alpha = (m1 == -INFINITY) ? 0.f : exp2f(m1 - mx1);
+        m1 = mx1;
+        l1 *= alpha;
+#pragma unroll
+        for (int n = 0; n < kOTiles; ++n) { o[n][2] *= alpha; o[n][3] *= alpha; }
+      }
     }
     const float mb0 = (m0 == -INFINITY) ? 0.f : m0, mb1 = (m1 == -INFINITY) ? 0.f : m1;
-    float pr[2][4];
-#pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
-      pr[nt][0] = ex2_approx(sc[nt][0] - mb0);
-      pr[nt][1] = ex2_approx(sc[nt][1] - mb0);
-      pr[nt][2] = ex2_approx(sc[nt][2] - mb1);
-      pr[nt][3] = ex2_approx(sc[nt][3] - mb1);
+    // P in bf16: the A fragment of P V (rows gid / gid+8, keys 2tig.. / 8+2tig..)
+    // or, kPack, pa0 / pa2 as the B fragment of V^T P^T; the row sums use the
+    // same rounded values
+    uint32_t pa0, pa1 = 0u, pa2, pa3 = 0u;
+    {
+      const float p00 = ex2_approx(sc[0][0] - mb0), p01 = ex2_approx(sc[0][1] - mb0);
+      const float p10 = ex2_approx(sc[1][0] - mb0), p11 = ex2_approx(sc[1][1] - mb0);
+      pa0 = bf16x2_bits(p00, p01);
+      pa2 = bf16x2_bits(p10, p11);
+      l0 += (bf16_lo(pa0) + bf16_hi(pa0)) + (bf16_lo(pa2) + bf16_hi(pa2));
     }
-    // P in bf16 as the A fragment of P V (rows gid / gid+8, keys 2tig.. / 8+2tig..);
-    // the row sums use the same rounded values
-    const uint32_t pa0 = bf16x2_bits(pr[0][0], pr[0][1]);
-    const uint32_t pa1 = bf16x2_bits(pr[0][2], pr[0][3]);
-    const uint32_t pa2 = bf16x2_bits(pr[1][0], pr[1][1]);
-    const uint32_t pa3 = bf16x2_bits(pr[1][2], pr[1][3]);
-    l0 += bf16_round(pr[0][0]) + bf16_round(pr[0][1]) + bf16_round(pr[1][0]) +
-          bf16_round(pr[1][1]);
-    l1 += bf16_round(pr[0][2]) + bf16_round(pr[0][3]) + bf16_round(pr[1][2]) +
-          bf16_round(pr[1][3]);
-    // O += P V: 16 n-tiles of 8 dims, V fragments by ldmatrix.trans
+    if constexpr (!kPack) {
+      const float p02 = ex2_approx(sc[0][2] - mb1), p03 = ex2_approx(sc[0][3] - mb1);
+      const float p12 = ex2_approx(sc[1][2] - mb1), p13 = ex2_approx(sc[1][3] - mb1);
+      pa1 = bf16x2_bits(p02, p03);
+      pa3 = bf16x2_bits(p12, p13);
+      l1 += (bf16_lo(pa1) + bf16_hi(pa1)) + (bf16_lo(pa3) + bf16_hi(pa3));
+    }
+    if constexpr (kPack) {
+      // O^T += V^T P^T: V^T (16 dims x 16 keys) is the A operand by
+      // ldmatrix.trans, and the B operand P^T (keys 2tig.., head gid) is the
+      // lane's own pa0 / pa2
 #pragma unroll
-    for (int np = 0; np < 8; ++np) {                 // pairs of n-tiles
-      uint32_t bv[4];
-      const int key = (lane & 7) + ((lane >> 3) & 1) * 8;
-      const int col = np * 16 + (lane >> 4) * 8;
-      ldsm_x4_t(vs + key * kRowBytes + col * 2, bv);
-      mma_bf16_16816(o[2 * np], pa0, pa1, pa2, pa3, bv[0], bv[1]);
-      mma_bf16_16816(o[2 * np + 1], pa0, pa1, pa2, pa3, bv[2], bv[3]);
+      for (int mt = 0; mt < 8; ++mt) {
+        uint32_t av[4];
+        const int key = (lane & 7) + ((lane >> 4) & 1) * 8;
+        const int col = mt * 16 + ((lane >> 3) & 1) * 8;
+        ldsm_x4_t(vs + key * kRowBytes + col * 2, av);
+        mma_bf16_16816(o[mt], av[0], av[1], av[2], av[3], pa0, pa2);
+      }
+    } else {
+      // O += P V: 16 n-tiles of 8 dims, V fragments by ldmatrix.trans
+#pragma unroll
+      for (int np = 0; np < 8; ++np) {               // pairs of n-tiles
+        uint32_t bv[4];
+        const int key = (lane & 7) + ((lane >> 3) & 1) * 8;
+        const int col = np * 16 + (lane >> 4) * 8;
+        ldsm_x4_t(vs + key * kRowBytes + col * 2, bv);
+        mma_bf16_16816(o[2 * np], pa0, pa1, pa2, pa3, bv[0], bv[1]);
+        mma_bf16_16816(o[2 * np + 1], pa0, pa1, pa2, pa3, bv[2], bv[3]);
+      }
     }
     __syncwarp();                                    // buffer reusable by a later step
   }
@@ -366,8 +457,10 @@ __global__ void __launch_bounds__(kDecThreads) decode_attn_kernel(const DecArgs 
   // row sums over the quad
   l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
   l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
-  l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
-  l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+  if (!kPack) {
+    l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+  }
 
   // merge the warps: per warp [16 rows][m, l, O(128)]
   __syncthreads();
@@ -378,14 +471,27 @@ __global__ void __launch_bounds__(kDecThreads) decode_attn_kernel(const DecArgs 
     float* r1 = wrow + (gid + 8) * (kHeadDim + 2);
     if (tig == 0) {
       r0[0] = m0; r0[1] = l0;
-      r1[0] = m1; r1[1] = l1;
+      if (!kPack) { r1[0] = m1; r1[1] = l1; }
     }
+    if constexpr (kPack) {
+      float* h0 = wrow + (2 * tig) * (kHeadDim + 2) + 2;       // head 2tig
+      float* h1 = h0 + (kHeadDim + 2);                         // head 2tig + 1
 #pragma unroll
-    for (int n = 0; n < 16; ++n) {                   // C layout: cols 2tig, 2tig+1 of tile n
-      r0[2 + n * 8 + 2 * tig] = o[n][0];
-      r0[2 + n * 8 + 2 * tig + 1] = o[n][1];
-      r1[2 + n * 8 + 2 * tig] = o[n][2];
-      r1[2 + n * 8 + 2 * tig + 1] = o[n][3];
+      for (int mt = 0; mt < 8; ++mt) {
+        const int d = mt * 16 + gid;
+        h0[d] = o[mt][0];
+        h1[d] = o[mt][1];
+        h0[d + 8] = o[mt][2];
+        h1[d + 8] = o[mt][3];
+      }
+    } else {
+#pragma unroll
+      for (int n = 0; n < 16; ++n) {                 // C layout: cols 2tig, 2tig+1 of tile n
+        r0[2 + n * 8 + 2 * tig] = o[n][0];
+        r0[2 + n * 8 + 2 * tig + 1] = o[n][1];
+        r1[2 + n * 8 + 2 * tig] = o[n][2];
+        r1[2 + n * 8 + 2 * tig + 1] = o[n][3];
+      }
     }
   }
   __syncthreads();
@@ -480,8 +586,10 @@ int decode_splits(int B, int Hk, int C, int W, int num_sms) {
 }
 
 cudaError_t launch_decode(const DecodeLaunch& L, cudaStream_t st) {
-  static PerDeviceOnce smem_once;
-  cudaError_t e = smem_limit_once(smem_once, decode_attn_kernel, kAttnSmem);
+  static PerDeviceOnce smem_once_pack, smem_once_full;
+  const bool pack = L.H / L.Hk <= 8;
+  cudaError_t e = pack ? smem_limit_once(smem_once_pack, decode_attn_kernel<true>, kAttnSmem)
+                       : smem_limit_once(smem_once_full, decode_attn_kernel<false>, kAttnSmem);
   if (e != cudaSuccess) return e;
   DecArgs a;
   a.B = L.B; a.C = L.C; a.H = L.H; a.Hk = L.Hk; a.G = L.H / L.Hk; a.W = L.W;
@@ -503,7 +611,11 @@ cudaError_t launch_decode(const DecodeLaunch& L, cudaStream_t st) {
   a.counters = L.counters; a.part_o = L.part_o; a.part_ml = L.part_ml;
   a.out = L.out; a.lse = L.lse; a.status = L.status;
   ProfScope prof(kKDecode, st);
-  decode_attn_kernel<<<dim3(launched, a.Hk, a.B), kDecThreads, kAttnSmem, st>>>(a);
+  const dim3 grid(launched, a.Hk, a.B);
+  if (pack)
+    decode_attn_kernel<true><<<grid, kDecThreads, kAttnSmem, st>>>(a);
+  else
+    decode_attn_kernel<false><<<grid, kDecThreads, kAttnSmem, st>>>(a);
   return cudaGetLastError();
 }
 

@@ -67,6 +67,10 @@ def check_cache(cpu, kc, vc, KC, rows):
     (32, 4, 600, 1, True, [0, 5, 599]),
     (32, 2, 300, 64, True, [5, 299, 150]),          # G = 16
     (4, 4, 200, 0, True, [0, 199, 77]),             # G = 1
+    (8, 4, 300, 0, True, [0, 299, 100]),            # G = 2
+    (16, 4, 400, 200, False, [399, 250, 0]),        # G = 4
+    (6, 2, 250, 0, True, [249, 3, 130]),            # G = 3 (rows past G padded)
+    (18, 2, 260, 100, True, [259, 40]),             # G = 9: heads on all 16 rows
     (32, 4, 1100, 1000, False, [1099, 513, 1024]),  # windows spanning several splits
 ])
 def test_decode_matches_oracle(cuda_lib, H, Hk, C, W, rope, lens):
