@@ -45,8 +45,9 @@
 //    math warps finish the current one. K and V stream through a 5-slot ring.
 // In both P steps one exponential pair in four is evaluated on the FMA pipe
 // (exp2_fma2); the special-function unit alone would bound them.
-// Before an MMA overwrites a TMEM region that a previous MMA reads as its A
-// operand, the issuer waits for that MMA's completion barrier.
+// An MMA that overwrites a TMEM region a previous MMA reads as its A operand
+// is issued right behind it without a completion wait: tcgen05.mma operations
+// issued by one thread are performed in issue order.
 #include <type_traits>
 
 #include "common.cuh"
@@ -105,7 +106,7 @@ constexpr int kQStages = 3;   // Q tiles in flight (its buffer is released last,
 struct __align__(8) KvBars {
   uint64_t kv_full, kv_empty;
   uint64_t q_full[kQStages], q_empty[kQStages], do_full[2], do_empty[2];
-  uint64_t s_full, dp_full, p_full, dp_free, ds_full, dk_done, acc_full, acc_empty;
+  uint64_t s_full, dp_full, p_full, dp_free, ds_full, acc_full, acc_empty;
   uint64_t drain;
   ItemRing ring;
 };
@@ -171,7 +172,6 @@ attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_q,
     mbar_init(smem_u32(&bars->p_full), kMathWarps);
     mbar_init(smem_u32(&bars->ds_full), kMathWarps);
     mbar_init(smem_u32(&bars->dp_free), kMathWarps);
-    mbar_init(smem_u32(&bars->dk_done), 1);
     mbar_init(smem_u32(&bars->acc_full), 1);
     mbar_init(smem_u32(&bars->acc_empty), kMathWarps);
     mbar_init(smem_u32(&bars->drain), 1);
@@ -280,13 +280,13 @@ attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_q,
     // Y_t = R(~t&1). The math warps write P^T(t) and dS^T(t) into X_t, so Y_t
     // is free once they have loaded dP^T(t) into registers (dp_free, early in
     // their dS step). Issue order per tile: dV(t), S^T(t+1) into Y_t (runs
-    // while dS(t) is computed), dK(t), then - after dK(t) has completed, as it
-    // reads X_t - dP^T(t+1) into X_t.
+    // while dS(t) is computed), dK(t), then dP^T(t+1) into X_t, right behind
+    // the dK(t) that reads X_t (MMAs are performed in issue order).
     {
       const uint32_t leader = elect_one();   // the one lane that issues
       const uint32_t idesc_ss = make_idesc_f16(128, 128, 0, 0);
       const uint32_t idesc_ts = make_idesc_f16(128, 128, 0, 1);
-      uint32_t item_count = 0, t = 0, dk_count = 0, p_cnt = 0, ds_cnt = 0, dpf_cnt = 0;
+      uint32_t item_count = 0, t = 0, p_cnt = 0, ds_cnt = 0, dpf_cnt = 0;
       bool ok = true;
       const uint32_t kt = sbase + kKvOffK, vt = sbase + kKvOffV;
       auto region = [&](uint32_t r) { return tmem + (r & 1) * 128; };
@@ -317,11 +317,10 @@ attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_q,
           if (!ok) break;
           tc_fence_after();
           issue_s(t);                            // X_t = Y_{t-1}: free after ds_full(t-1)
-          if (dk_count > 0) ok = mbar_wait_warp(smem_u32(&bars->dk_done), (dk_count - 1) & 1, wc);
-          if (ok) ok = mbar_wait_warp(smem_u32(&bars->do_full[t & 1]), (t >> 1) & 1, wc);
+          ok = mbar_wait_warp(smem_u32(&bars->do_full[t & 1]), (t >> 1) & 1, wc);
           if (!ok) break;
           tc_fence_after();
-          issue_dp(t);                           // Y_t = X_{t-1}: free after dK(t-1)
+          issue_dp(t);                           // Y_t = X_{t-1}: behind dK(t-1), its reader
         }
         for (int m = 0; m < it.nq && ok; ++m, ++t) {
           const uint32_t s = t & 1, sq = t % kQStages;
@@ -363,13 +362,9 @@ attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_q,
           for (int kk = 0; kk < 8; ++kk)
             mma_ts_w(tmem + 384, X + 32 + split_a_col(kk), mnmajor_desc(qt, kk), idesc_ts,
                      (m > 0 || kk > 0) ? 1u : 0u, leader);
-          mma_commit_w(smem_u32(&bars->dk_done), leader);
-          ++dk_count;
           mma_commit_w(smem_u32(&bars->q_empty[sq]), leader);
           if (has_next) {
-            ok = mbar_wait_warp(smem_u32(&bars->dk_done), (dk_count - 1) & 1, wc);
-            if (ok)
-              ok = mbar_wait_warp(smem_u32(&bars->do_full[(t + 1) & 1]), ((t + 1) >> 1) & 1, wc);
+            ok = mbar_wait_warp(smem_u32(&bars->do_full[(t + 1) & 1]), ((t + 1) >> 1) & 1, wc);
             if (!ok) break;
             tc_fence_after();
             issue_dp(t + 1);
@@ -578,7 +573,7 @@ constexpr int kQSlots = 5;
 struct __align__(8) QBars {
   uint64_t qd_full, qd_empty;
   uint64_t kv_full[kQSlots], kv_empty[kQSlots];
-  uint64_t s_full[2], dq_done[2];     // per S buffer
+  uint64_t s_full[2];                 // per S buffer
   uint64_t dp_full, ds_full, acc_full, acc_empty;
   uint64_t drain;
   ItemRing ring;
@@ -638,7 +633,6 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q,
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(smem_u32(&bars->s_full[s]), 1);
-      mbar_init(smem_u32(&bars->dq_done[s]), 1);
     }
     mbar_init(smem_u32(&bars->dp_full), 1);
     mbar_init(smem_u32(&bars->ds_full), kMathWarps);
@@ -699,23 +693,21 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q,
         if (arm[s]) mbar_wait(smem_u32(&bars->kv_full[s]), (arm[s] - 1) & 1, drain);
     }
   } else if (warp == kWarpMma) {
-    // Per tile t: dP(t), S(t+1) (into the other S buffer, once dQ(t-1) has read
-    // it), dQ(t). P of tile t+1 is then computed while dQ(t) and dP(t+1) run.
+    // Per tile t: dP(t), S(t+1) (into the other S buffer, right behind the dQ(t-1)
+    // that reads it: MMAs are performed in issue order), dQ(t). P of tile t+1 is
+    // then computed while dQ(t) and dP(t+1) run.
     {
       const uint32_t leader = elect_one();   // the one lane that issues
       const uint32_t idesc_ss = make_idesc_f16(128, 128, 0, 0);
       const uint32_t idesc_ts = make_idesc_f16(128, 128, 0, 1);
-      uint32_t item_count = 0, t = 0, ds_cnt = 0, dq_cnt0 = 0, dq_cnt1 = 0;
+      uint32_t item_count = 0, t = 0, ds_cnt = 0;
       bool ok = true;
       const uint32_t qt = sbase + kQOffQ, dot = sbase + kQOffDO;
-      // S(tt) = Q K(tt)^T into buffer tt % 2, after the dQ that last read it.
+      // S(tt) = Q K(tt)^T into buffer tt % 2, issued after the dQ that last read it.
       auto issue_s = [&](uint32_t tt) -> bool {
         const uint32_t b = tt & 1, lk = 2 * tt;                 // K(tt) in the ring
         const uint32_t st = lk % kQSlots, ph = (lk / kQSlots) & 1;
         if (!mbar_wait_warp(smem_u32(&bars->kv_full[st]), ph, wc)) return false;
-        const uint32_t cnt = b ? dq_cnt1 : dq_cnt0;
-        if (cnt > 0 && !mbar_wait_warp(smem_u32(&bars->dq_done[b]), (cnt - 1) & 1, wc))
-          return false;
         tc_fence_after();
         const uint32_t kt = sbase + kQOffKV + st * kTileBytes;
 #pragma unroll
@@ -767,8 +759,6 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q,
           for (int kk = 0; kk < 8; ++kk)
             mma_ts_w(tmem + kQColDQ, tmem + kQColS0 + b * 128 + split_a_col(kk),
                      mnmajor_desc(kt, kk), idesc_ts, (n > 0 || kk > 0) ? 1u : 0u, leader);
-          mma_commit_w(smem_u32(&bars->dq_done[b]), leader);
-          if (b) ++dq_cnt1; else ++dq_cnt0;
           mma_commit_w(smem_u32(&bars->kv_empty[sk]), leader);   // K(t) done after dQ(t)
         }
         if (!ok) break;

@@ -32,9 +32,12 @@
 //     the A operand of the PV MMA straight from TMEM. The softmax reads S_i
 //     once into registers and releases P_i in two halves (keys 0-63, then
 //     64-127); the PV MMA of the first half runs while the second is
-//     computed. Before the next QK MMA of tile i overwrites S_i, the issuer
-//     waits until the PV MMA of tile i has completed (a commit barrier), so no
-//     ordering between MMAs writing different accumulators is assumed.
+//     computed. The next QK MMA of tile i, which overwrites S_i, is issued
+//     right behind the PV MMA that reads P_i from it: tcgen05.mma operations
+//     issued by one thread are performed in issue order, so the PV has read
+//     its operand before the QK writes (no completion wait on this chain; the
+//     commit that signals the new S also covers the PV, so O and P_i are
+//     settled when the softmax sees it).
 //   * Sink folding: the running max starts at the sink logit and the running
 //     sum at 1 (the sink's own weight), so there is no extra pass and a row is
 //     never all -inf. The max is updated lazily: O and l are rescaled only when
@@ -79,7 +82,7 @@ struct FwdArgs {
 struct __align__(8) Barriers {
   uint64_t q_full, q_empty;
   uint64_t kv_full[kSlots], kv_empty[kSlots];
-  uint64_t s_full[2], p_half[2], p_full[2], pv_done[2], o_full[2], o_empty[2];
+  uint64_t s_full[2], p_half[2], p_full[2], o_full[2], o_empty[2];
   uint64_t drain;
   ItemRing ring;
 };
@@ -145,7 +148,6 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       mbar_init(smem_u32(&bars->s_full[i]), 1);
       mbar_init(smem_u32(&bars->p_half[i]), 4);
       mbar_init(smem_u32(&bars->p_full[i]), 4);
-      mbar_init(smem_u32(&bars->pv_done[i]), 1);
       mbar_init(smem_u32(&bars->o_full[i]), 1);
       mbar_init(smem_u32(&bars->o_empty[i]), 4);
     }
@@ -223,7 +225,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       const uint32_t idesc_qk = make_idesc_f16(128, 128, 0, 0);
       const uint32_t idesc_pv = make_idesc_f16(128, 128, 0, 1);
       uint32_t kv_load = 0, item_count = 0;   // K/V ring loads consumed before this item
-      uint32_t pv0 = 0, pv1 = 0, pc0 = 0, pc1 = 0;   // PV commits / P arrivals seen, per tile
+      uint32_t pc0 = 0, pc1 = 0;                     // P arrivals seen, per tile
       bool ok = true;
       const uint32_t q0t = sbase + kOffQ, q1t = sbase + kOffQ + kTileBytes;
       while (ok) {
@@ -239,16 +241,10 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
           ok = mbar_wait_warp(smem_u32(&bars->kv_full[s]), ph, wc);
           if (!ok) break;
           const uint32_t kt = sbase + kOffKV + s * kTileBytes;
-          if (pv0 > 0) ok = mbar_wait_warp(smem_u32(&bars->pv_done[0]), (pv0 - 1) & 1, wc);
-          if (!ok) break;
-          tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
             mma_ss_w(tmem + 0, kmajor_desc(q0t, kk), kmajor_desc(kt, kk), idesc_qk, kk > 0, leader);
           mma_commit_w(smem_u32(&bars->s_full[0]), leader);
-          if (pv1 > 0) ok = mbar_wait_warp(smem_u32(&bars->pv_done[1]), (pv1 - 1) & 1, wc);
-          if (!ok) break;
-          tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
             mma_ss_w(tmem + 128, kmajor_desc(q1t, kk), kmajor_desc(kt, kk),
@@ -283,12 +279,9 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
 #pragma unroll
           for (int kk = 4; kk < 8; ++kk)
             mma_ts_w(tmem + 256, tmem + 0 + kk * 8, mnmajor_desc(vt, kk), idesc_pv, 1u, leader);
-          mma_commit_w(smem_u32(&bars->pv_done[0]), leader);
-          ++pv0;
           if (!has_next) mma_commit_w(smem_u32(&bars->o_full[0]), leader);
           if (has_next) {
             ok = mbar_wait_warp(smem_u32(&bars->kv_full[s2]), ph2, wc);
-            if (ok) ok = mbar_wait_warp(smem_u32(&bars->pv_done[0]), (pv0 - 1) & 1, wc);
             if (!ok) break;
             tc_fence_after();
 #pragma unroll
@@ -315,14 +308,9 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
 #pragma unroll
           for (int kk = 4; kk < 8; ++kk)
             mma_ts_w(tmem + 384, tmem + 128 + kk * 8, mnmajor_desc(vt, kk), idesc_pv, 1u, leader);
-          mma_commit_w(smem_u32(&bars->pv_done[1]), leader);
-          ++pv1;
           if (!has_next) mma_commit_w(smem_u32(&bars->o_full[1]), leader);
           mma_commit_w(smem_u32(&bars->kv_empty[s]), leader);
           if (has_next) {
-            ok = mbar_wait_warp(smem_u32(&bars->pv_done[1]), (pv1 - 1) & 1, wc);
-            if (!ok) break;
-            tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
               mma_ss_w(tmem + 128, kmajor_desc(q1t, kk), kmajor_desc(kt2, kk),
@@ -442,9 +430,10 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         };
         exp_chunk(u0, 0);
         if (__any_sync(0xffffffffu, rescale_o)) {
-          // PV of the previous tile has completed (the QK that produced this
-          // S was issued after it completed), so O is stable here. Done once
-          // the first quarter of S is consumed, to stay within registers.
+          // PV of the previous tile has completed (the commit that signalled
+          // this S was issued after it and covers it), so O is stable here.
+          // Done once the first quarter of S is consumed, to stay within
+          // registers.
           const uint64_t a2 = f2(alpha, alpha);
 #pragma unroll 1
           for (int c = 0; c < 4; ++c) {

@@ -24,10 +24,13 @@ Violations: a deadlock (no role can move and nothing is in flight); a write
 into a cell that an unfinished operation reads or writes (except an MMA
 accumulating into the accumulator that earlier MMAs of the same chain write);
 a read of a cell while a write to it is in flight, or whose content is not the
-tile the reader expects; phase aliasing; arrivals past a barrier's count. The
-model flags an MMA that overwrites TMEM an earlier unfinished MMA reads, even
-though MMAs from one thread run in order: the kernels do not rely on that order
-and wait for the reader's completion instead.
+tile the reader expects; phase aliasing; arrivals past a barrier's count.
+MMAs from the one issuing thread are performed in issue order, so a model may
+declare (``Sim.mma_in_order``) that an MMA overwrites cells an earlier,
+unfinished MMA reads: the BF16 kernels issue an MMA into a TMEM region right
+behind the MMA that reads it (the forward's next QK behind the PV that reads P,
+dP^T behind dK, S behind dQ). The FP32-input kernels wait for the reader's
+completion instead, and for them that overlap is flagged.
 
 ``MUTATIONS`` plants known mistakes in the restated protocols, so that tests can
 show the checker finds them.
@@ -109,6 +112,7 @@ class Sim:
         self.roles = {}            # name -> [generator, blocked (bar, k) or None]
         self.tma = []              # in-flight TMA loads
         self.mma = deque()         # issued MMAs and commit markers, in issue order
+        self.mma_in_order = False  # an MMA may overwrite what earlier MMAs still read
         self.steps = 0
 
     # -- setup
@@ -136,7 +140,9 @@ class Sim:
     def _write_begin(self, names, tag, op, who, accumulate=False):
         for n in names:
             c = self.cell(n)
-            if c.readers:
+            in_order = (self.mma_in_order and op.kind == "mma"
+                        and all(r.kind == "mma" for r in c.readers))
+            if c.readers and not in_order:
                 raise ProtocolError(f"{who} writes {n} while an unfinished operation reads it")
             if c.writers:
                 chain = accumulate and c.next_tag == tag and all(
@@ -291,12 +297,13 @@ def _ring_bars(sim, consumers=MATH_WARPS + 1):
 
 def forward(sim, items, mut=None):
     """items: key tiles per item (>= 1). Tiles i = 0, 1 of the pair."""
+    sim.mma_in_order = True
     sim.bar("q_full"), sim.bar("q_empty")
     for s in range(K_SLOTS):
         sim.bar(f"kv_full{s}"), sim.bar(f"kv_empty{s}")
     for i in range(2):
         sim.bar(f"s_full{i}"), sim.bar(f"p_half{i}", 4), sim.bar(f"p_full{i}", 4)
-        sim.bar(f"pv_done{i}"), sim.bar(f"o_full{i}"), sim.bar(f"o_empty{i}", 4)
+        sim.bar(f"o_full{i}"), sim.bar(f"o_empty{i}", 4)
     _ring_bars(sim)
     seq = list(items) + [None]
 
@@ -323,7 +330,7 @@ def forward(sim, items, mut=None):
                 kv_load += 1
 
     def mma():
-        kv_load, pv, pc = 0, [0, 0], [0, 0]
+        kv_load, pc = 0, [0, 0]
 
         def qk(i, item, slot, g):
             return ("mma", [([f"smem:Q{i}"], ("Q", item, i)), ([f"smem:kv{slot}"], ("K", g))],
@@ -338,8 +345,6 @@ def forward(sim, items, mut=None):
             s = kv_load % K_SLOTS
             yield ("wait", f"kv_full{s}", kv_load // K_SLOTS)
             for i in range(2):
-                if pv[i] > 0 and mut != "fwd_qk_without_pv_done":
-                    yield ("wait", f"pv_done{i}", pv[i] - 1)
                 yield qk(i, item, s, g0)
                 yield ("commit", f"s_full{i}")
             yield ("commit", f"kv_empty{s}")
@@ -363,21 +368,24 @@ def forward(sim, items, mut=None):
                         yield ("commit", f"o_full{i}")
                     yield ("wait", f"p_full{i}", pc[i])
                     pc[i] += 1
+                    if mut == "fwd_qk_before_pv" and has_next:
+                        # the next QK overtakes the PV that still has to read P
+                        if i == 0:
+                            yield ("wait", f"kv_full{s2}", lk // K_SLOTS)
+                        yield qk(i, item, s2, g + 1)
                     yield ("mma", [(tmem(f"S{i}", [2, 3]), ("P", i, g)),
                                    ([f"smem:kv{s}"], ("V", g))], o, ("O", i, item), True)
-                    yield ("commit", f"pv_done{i}")
-                    pv[i] += 1
                     if not has_next and mut != "fwd_o_full_before_last_pv":
                         yield ("commit", f"o_full{i}")
                     if i == 1:
                         yield ("commit", f"kv_empty{s}")
                     if has_next:
-                        if i == 0:
+                        if i == 0 and mut != "fwd_qk_before_pv":
                             yield ("wait", f"kv_full{s2}", lk // K_SLOTS)
-                        yield ("wait", f"pv_done{i}", pv[i] - 1)
                         if mut == "fwd_q_empty_before_last_qk" and i == 1 and n + 2 == nt:
                             yield ("commit", "q_empty")
-                        yield qk(i, item, s2, g + 1)
+                        if mut != "fwd_qk_before_pv":
+                            yield qk(i, item, s2, g + 1)
                         yield ("commit", f"s_full{i}")
                         if i == 1:
                             yield ("commit", f"kv_empty{s2}")
@@ -431,7 +439,8 @@ def backward_dkv(sim, items, mut=None):
         sim.bar(f"q_full{s}"), sim.bar(f"q_empty{s}")
     for s in range(2):
         sim.bar(f"do_full{s}", 2), sim.bar(f"do_empty{s}")
-    sim.bar("s_full"), sim.bar("dp_full"), sim.bar("dk_done"), sim.bar("acc_full")
+    sim.mma_in_order = True
+    sim.bar("s_full"), sim.bar("dp_full"), sim.bar("acc_full")
     for b in ("p_full", "ds_full", "dp_free", "acc_empty"):
         sim.bar(b, MATH_WARPS)
     _ring_bars(sim)
@@ -466,7 +475,7 @@ def backward_dkv(sim, items, mut=None):
                 qd += 1
 
     def mma():
-        t, dk_count, p_cnt, ds_cnt, dpf_cnt = 0, 0, 0, 0, 0
+        t, p_cnt, ds_cnt, dpf_cnt = 0, 0, 0, 0
 
         def issue_s(tt, item):
             yield ("mma", [(["smem:K"], ("K", item)),
@@ -486,8 +495,6 @@ def backward_dkv(sim, items, mut=None):
             yield ("wait", "kv_full", item)
             yield ("wait", f"q_full{t % Q_STAGES_DKV}", t // Q_STAGES_DKV)
             yield from issue_s(t, item)
-            if dk_count > 0:
-                yield ("wait", "dk_done", dk_count - 1)
             yield ("wait", f"do_full{t & 1}", t >> 1)
             yield from issue_dp(t, item)
             for m in range(nq):
@@ -517,11 +524,8 @@ def backward_dkv(sim, items, mut=None):
                 yield ("mma", [(tmem(X, [2, 3, 6, 7]), ("dST", t)),
                                ([f"smem:Q{t % Q_STAGES_DKV}"], ("Q", t))],
                        tmem("dK", ALL_CHUNKS), ("dK", item), m > 0)
-                yield ("commit", "dk_done")
-                dk_count += 1
                 yield ("commit", f"q_empty{t % Q_STAGES_DKV}")
                 if has_next:
-                    yield ("wait", "dk_done", dk_count - 1)
                     yield ("wait", f"do_full{(t + 1) & 1}", (t + 1) >> 1)
                     yield from issue_dp(t + 1, item)
                 t += 1
@@ -569,11 +573,12 @@ def backward_dkv(sim, items, mut=None):
 # ============================================================================
 
 def backward_dq(sim, items, mut=None):
+    sim.mma_in_order = True
     sim.bar("qd_full"), sim.bar("qd_empty")
     for s in range(K_SLOTS):
         sim.bar(f"kv_full{s}"), sim.bar(f"kv_empty{s}")
     for b in range(2):
-        sim.bar(f"s_full{b}"), sim.bar(f"dq_done{b}")
+        sim.bar(f"s_full{b}")
     sim.bar("dp_full"), sim.bar("acc_full")
     sim.bar("ds_full", MATH_WARPS), sim.bar("acc_empty", MATH_WARPS)
     _ring_bars(sim)
@@ -602,14 +607,12 @@ def backward_dq(sim, items, mut=None):
                 kv_load += 1
 
     def mma():
-        t, ds_cnt, dq_cnt = 0, 0, [0, 0]
+        t, ds_cnt = 0, 0
 
         def issue_s(tt, item):
             b, lk = tt & 1, 2 * tt
             st = lk % K_SLOTS
             yield ("wait", f"kv_full{st}", lk // K_SLOTS)
-            if dq_cnt[b] > 0 and mut != "dq_s_without_dq_done":
-                yield ("wait", f"dq_done{b}", dq_cnt[b] - 1)
             yield ("mma", [(["smem:Q"], ("Q", item)), ([f"smem:kv{st}"], ("K", tt))],
                    tmem(f"S{b}", ALL_CHUNKS), ("S", tt), False)
             yield ("commit", f"s_full{b}")
@@ -636,7 +639,8 @@ def backward_dq(sim, items, mut=None):
                     yield ("commit", f"kv_empty{sk}")
                 if n + 1 < nt:
                     yield from issue_s(t + 1, item)
-                yield ("wait", "ds_full", ds_cnt)
+                if mut != "dq_dq_without_ds_full":
+                    yield ("wait", "ds_full", ds_cnt)
                 ds_cnt += 1
                 if n == 0 and item > 0:
                     yield ("wait", "acc_empty", item - 1)
@@ -645,8 +649,6 @@ def backward_dq(sim, items, mut=None):
                 yield ("mma", [(tmem(f"S{b}", [0, 1, 4, 5]), ("dS", t)),
                                ([f"smem:kv{sk}"], ("K", t))],
                        tmem("dQ", ALL_CHUNKS), ("dQ", item), n > 0)
-                yield ("commit", f"dq_done{b}")
-                dq_cnt[b] += 1
                 if mut != "dq_k_released_after_dp":
                     yield ("commit", f"kv_empty{sk}")
                 t += 1
@@ -1123,10 +1125,10 @@ MUTATIONS = [
     ("forward", "fwd_q_empty_before_last_qk"),
     ("forward", "fwd_p_half_early"),
     ("forward", "fwd_o_full_before_last_pv"),
-    ("forward", "fwd_qk_without_pv_done"),
+    ("forward", "fwd_qk_before_pv"),
     ("backward_dkv", "dkv_s_without_dp_free"),
     ("backward_dkv", "dkv_do_empty_before_ds"),
-    ("backward_dq", "dq_s_without_dq_done"),
+    ("backward_dq", "dq_dq_without_ds_full"),
     ("backward_dq", "dq_qd_empty_before_last_dp"),
     ("backward_dq", "dq_k_released_after_dp"),
     ("forward_x3", "x3f_pv_without_p_full"),

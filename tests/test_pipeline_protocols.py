@@ -9,6 +9,8 @@ operation still reads, and no read of anything but the expected tile, over item
 lists with one-tile items, long items and mixes of both. Each planted mistake
 (a release moved too early, a wait left out) must be caught.
 """
+import random
+
 import pytest
 
 import pipeline_model as pm
@@ -34,7 +36,7 @@ def test_protocol_holds_under_random_schedules(kernel):
 @pytest.mark.parametrize("kernel,mutation", pm.MUTATIONS, ids=[m for _, m in pm.MUTATIONS])
 def test_planted_protocol_mistake_is_caught(kernel, mutation):
     for items in ITEM_LISTS[kernel]:
-        for seed in range(60):
+        for seed in range(200):
             try:
                 pm.check(kernel, items, seed, mutation)
             except pm.ProtocolError:
@@ -59,7 +61,6 @@ def test_barrier_model_follows_the_parity_rule():
 
 
 def test_deadlock_is_reported():
-    import random
     sim = pm.Sim(random.Random(0))
     sim.bar("never")
 
@@ -69,3 +70,23 @@ def test_deadlock_is_reported():
     sim.role("w", waiter())
     with pytest.raises(pm.ProtocolError, match="deadlock"):
         sim.run()
+
+
+@pytest.mark.parametrize("kernel", ["forward", "backward_dkv", "backward_dq"])
+def test_bf16_kernels_rely_on_in_order_mma_issue(kernel):
+    """The BF16 kernels issue an MMA into a TMEM region right behind the MMA that
+    reads it (the forward's next QK behind the PV that reads P; dP^T behind dK;
+    S behind dQ), relying on tcgen05.mma operations of one thread being
+    performed in issue order. Without that rule the same schedules must fail,
+    and only on that overlap."""
+    flagged = 0
+    for seed in range(20):
+        sim = pm.Sim(random.Random(seed))
+        pm.KERNELS[kernel](sim, [3], None)
+        sim.mma_in_order = False
+        try:
+            sim.run()
+        except pm.ProtocolError as e:
+            assert "while an unfinished operation reads it" in str(e)
+            flagged += 1
+    assert flagged > 0
