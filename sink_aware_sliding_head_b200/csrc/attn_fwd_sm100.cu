@@ -30,8 +30,8 @@
 //   * TMEM (512 columns): S0 [0,128), S1 [128,256), O0 [256,384), O1 [384,512).
 //     P_i (fp16, two per column) overwrites the first 64 columns of S_i and is
 //     the A operand of the PV MMA straight from TMEM. The softmax reads S_i
-//     once into registers and releases P_i in two halves (keys 0-63, then
-//     64-127); the PV MMA of the first half runs while the second is
+//     once into registers and releases P_i in two parts (keys 0-95, then
+//     96-127); the PV MMAs of the first part run while the rest is
 //     computed. The next QK MMA of tile i, which overwrites S_i, is issued
 //     right behind the PV MMA that reads P_i from it: tcgen05.mma operations
 //     issued by one thread are performed in issue order, so the PV has read
@@ -262,14 +262,14 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
           const uint32_t kt2 = sbase + kOffKV + s2 * kTileBytes;
           ok = mbar_wait_warp(smem_u32(&bars->kv_full[s]), ph, wc);
           // ---- tile 0
-          // keys 0-63 of P as soon as the softmax has written them, then 64-127
+          // keys 0-95 of P as soon as the softmax has written them, then 96-127
           if (ok) ok = mbar_wait_warp(smem_u32(&bars->p_half[0]), pc0 & 1, wc);
           if (ok && n == 0 && item_count > 0)
             ok = mbar_wait_warp(smem_u32(&bars->o_empty[0]), (item_count - 1) & 1, wc);
           if (!ok) break;
           tc_fence_after();
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
+          for (int kk = 0; kk < 6; ++kk)
             mma_ts_w(tmem + 256, tmem + 0 + kk * 8, mnmajor_desc(vt, kk), idesc_pv,
                    (n > 0 || kk > 0) ? 1u : 0u, leader);
           ok = mbar_wait_warp(smem_u32(&bars->p_full[0]), pc0 & 1, wc);
@@ -277,7 +277,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
           if (!ok) break;
           tc_fence_after();
 #pragma unroll
-          for (int kk = 4; kk < 8; ++kk)
+          for (int kk = 6; kk < 8; ++kk)
             mma_ts_w(tmem + 256, tmem + 0 + kk * 8, mnmajor_desc(vt, kk), idesc_pv, 1u, leader);
           if (!has_next) mma_commit_w(smem_u32(&bars->o_full[0]), leader);
           if (has_next) {
@@ -291,14 +291,14 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
             mma_commit_w(smem_u32(&bars->s_full[0]), leader);
           }
           // ---- tile 1
-          // keys 0-63 of P as soon as the softmax has written them, then 64-127
+          // keys 0-95 of P as soon as the softmax has written them, then 96-127
           if (ok) ok = mbar_wait_warp(smem_u32(&bars->p_half[1]), pc1 & 1, wc);
           if (ok && n == 0 && item_count > 0)
             ok = mbar_wait_warp(smem_u32(&bars->o_empty[1]), (item_count - 1) & 1, wc);
           if (!ok) break;
           tc_fence_after();
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
+          for (int kk = 0; kk < 6; ++kk)
             mma_ts_w(tmem + 384, tmem + 128 + kk * 8, mnmajor_desc(vt, kk), idesc_pv,
                    (n > 0 || kk > 0) ? 1u : 0u, leader);
           ok = mbar_wait_warp(smem_u32(&bars->p_full[1]), pc1 & 1, wc);
@@ -306,7 +306,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
           if (!ok) break;
           tc_fence_after();
 #pragma unroll
-          for (int kk = 4; kk < 8; ++kk)
+          for (int kk = 6; kk < 8; ++kk)
             mma_ts_w(tmem + 384, tmem + 128 + kk * 8, mnmajor_desc(vt, kk), idesc_pv, 1u, leader);
           if (!has_next) mma_commit_w(smem_u32(&bars->o_full[1]), leader);
           mma_commit_w(smem_u32(&bars->kv_empty[s]), leader);
@@ -412,8 +412,9 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         const uint64_t nm2 = f2(-mb, -mb);
         uint64_t rs2 = f2(0.f, 0.f);
         // P = 2^(s*scale - m) in fp16, two keys per TMEM column, over the
-        // first 64 columns of S (already read). Keys 0-63 are handed to the
-        // PV MMA before keys 64-127 are computed.
+        // first 64 columns of S (already read). Keys 0-95 are handed to the
+        // PV MMAs before keys 96-127 are computed, so only two PV MMAs are left
+        // on the tile's chain after the softmax.
         auto exp_chunk = [&](const uint32_t (&u)[32], int col) {
           uint32_t pk[16];
 #pragma unroll
@@ -451,11 +452,11 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
           }
         }
         exp_chunk(u1, 16);
+        exp_chunk(u2, 32);
         tc_wait_st();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&bars->p_half[i]));
-        exp_chunk(u2, 32);
         exp_chunk(u3, 48);
         float rs_lo, rs_hi;
         f2_split(rs2, rs_lo, rs_hi);

@@ -362,7 +362,7 @@ def forward(sim, items, mut=None):
                     if n == 0 and item > 0:
                         yield ("wait", f"o_empty{i}", item - 1)
                     o = tmem(f"O{i}", ALL_CHUNKS)
-                    yield ("mma", [(tmem(f"S{i}", [0, 1]), ("P", i, g)),
+                    yield ("mma", [(tmem(f"S{i}", [0, 1, 2]), ("P", i, g)),
                                    ([f"smem:kv{s}"], ("V", g))], o, ("O", i, item), n > 0)
                     if mut == "fwd_o_full_before_last_pv" and not has_next:
                         yield ("commit", f"o_full{i}")
@@ -373,7 +373,7 @@ def forward(sim, items, mut=None):
                         if i == 0:
                             yield ("wait", f"kv_full{s2}", lk // K_SLOTS)
                         yield qk(i, item, s2, g + 1)
-                    yield ("mma", [(tmem(f"S{i}", [2, 3]), ("P", i, g)),
+                    yield ("mma", [(tmem(f"S{i}", [3]), ("P", i, g)),
                                    ([f"smem:kv{s}"], ("V", g))], o, ("O", i, item), True)
                     if not has_next and mut != "fwd_o_full_before_last_pv":
                         yield ("commit", f"o_full{i}")
@@ -413,10 +413,10 @@ def forward(sim, items, mut=None):
                     yield ("write", o, ("O", i, item))
                 if mut == "fwd_p_half_early":
                     yield ("arrive", f"p_half{i}")
-                yield ("write", tmem(f"S{i}", [1], quarter), ("P", i, g))
+                yield ("write", tmem(f"S{i}", [1, 2], quarter), ("P", i, g))
                 if mut != "fwd_p_half_early":
                     yield ("arrive", f"p_half{i}")
-                yield ("write", tmem(f"S{i}", [2, 3], quarter), ("P", i, g))
+                yield ("write", tmem(f"S{i}", [3], quarter), ("P", i, g))
                 yield ("arrive", f"p_full{i}")
             yield ("wait", f"o_full{i}", item)
             yield ("read", tmem(f"O{i}", ALL_CHUNKS, quarter), ("O", i, item))
