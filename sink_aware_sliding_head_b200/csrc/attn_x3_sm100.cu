@@ -42,8 +42,9 @@
 //    sit in TMEM as A operands (written by the math warps), K and V tiles of 64
 //    keys stream through a ring of 16 KB slots. Two 64-column regions rotate
 //    between S/dS and dP as in the dK/dV kernel of the fp16 path.
-// Before an MMA overwrites a TMEM region that an earlier MMA reads, the issuer
-// waits for that MMA's completion barrier.
+// An MMA that overwrites a TMEM region an earlier MMA reads is issued right
+// behind it without a completion wait: tcgen05.mma operations issued by one
+// thread are performed in issue order.
 #include <type_traits>
 
 #include "common.cuh"
@@ -277,13 +278,14 @@ attn_fwd_x3_kernel(const __grid_constant__ CUtensorMap tm_q,
   } else if (warp == kFWarpMma) {
     // ------------------------------------------------------------ MMA issuer
     // Order: QK(t), QK(t+1); then per tile PV(t) and QK(t+2). QK(t+2) reuses
-    // the S buffer whose P(t) PV(t) reads, so it waits for PV(t) to complete.
+    // the S buffer whose P(t) PV(t) reads and is issued right behind it (MMAs
+    // are performed in issue order); pv_done tells the softmax when PV(t) has
+    // completed (it rescales O).
     const uint32_t leader = elect_one();
     const uint32_t idesc_qk = make_idesc_f16(128, 128, 0, 0);
     const uint32_t idesc_pv = make_idesc_f16(128, 128, 0, 1);
     const uint32_t qh = sbase + kFOffQ, ql = sbase + kFOffQ + kPart128;
     uint32_t item_count = 0, t = 0, kv_base = 0;
-    uint32_t pv_cnt[2] = {0, 0};
     bool ok = true;
     auto slot = [&](uint32_t pos) { return sbase + kFOffKV + (pos % kFSlots) * kPart128; };
     auto wait_full = [&](uint32_t pos) {
@@ -293,9 +295,6 @@ attn_fwd_x3_kernel(const __grid_constant__ CUtensorMap tm_q,
     auto issue_qk = [&](uint32_t n, uint32_t tt, bool last) -> bool {
       const uint32_t b = tt & 1, pos = kv_base + fwd_pos_k(n);
       if (!wait_full(pos) || !wait_full(pos + 1)) return false;
-      if (pv_cnt[b] > 0 &&
-          !mbar_wait_warp(smem_u32(&bars->pv_done[b]), (pv_cnt[b] - 1) & 1, wc))
-        return false;
       tc_fence_after();
       const uint32_t kh = slot(pos), kl = slot(pos + 1), d = tmem + b * 128;
 #pragma unroll
@@ -355,7 +354,6 @@ attn_fwd_x3_kernel(const __grid_constant__ CUtensorMap tm_q,
           mma_ts_w(o, ah, mndesc128(vh, kk), idesc_pv, 1u, leader);
         }
         mma_commit_w(smem_u32(&bars->pv_done[b]), leader);
-        ++pv_cnt[b];
         mma_commit_w(smem_u32(&bars->kv_empty[pos % kFSlots]), leader);
         mma_commit_w(smem_u32(&bars->kv_empty[(pos + 1) % kFSlots]), leader);
         if (n + 1 == nt) mma_commit_w(smem_u32(&bars->o_full), leader);
@@ -561,7 +559,7 @@ constexpr int kDrainTiles = 16;
 struct __align__(8) KBars {
   uint64_t kv_full, kv_empty;
   uint64_t q_full[kKQStages], q_empty[kKQStages], do_full[2], do_empty[2];
-  uint64_t v_full, s_full, dp_full, p_full, ds_full, dv_done, dk_done, acc_full, acc_empty;
+  uint64_t v_full, s_full, dp_full, p_full, ds_full, acc_full, acc_empty;
   uint64_t drain;
   ItemRing ring;
 };
@@ -626,8 +624,6 @@ attn_bwd_dkv_x3_kernel(const __grid_constant__ CUtensorMap tm_q,
     mbar_init(smem_u32(&bars->dp_full), 1);
     mbar_init(smem_u32(&bars->p_full), kBMathWarps);
     mbar_init(smem_u32(&bars->ds_full), kBMathWarps);
-    mbar_init(smem_u32(&bars->dv_done), 1);
-    mbar_init(smem_u32(&bars->dk_done), 1);
     mbar_init(smem_u32(&bars->acc_full), 1);
     mbar_init(smem_u32(&bars->acc_empty), kBMathWarps);
     mbar_init(smem_u32(&bars->drain), 1);
@@ -731,14 +727,14 @@ attn_bwd_dkv_x3_kernel(const __grid_constant__ CUtensorMap tm_q,
     }
   } else if (warp == kBWarpMma) {
     // Per query tile t: S^T(t) into X, dP^T(t) into Y; the math warps write
-    // P'^T(t) over X and dS^T(t) over Y. Issue order: dV(t), S^T(t+1) (after
-    // dV(t) has completed: it reads X), dK(t), dP^T(t+1) (after dK(t): Y).
+    // P'^T(t) over X and dS^T(t) over Y. Issue order: dV(t), S^T(t+1) (right
+    // behind dV(t), which reads X), dK(t), dP^T(t+1) (behind dK(t): Y).
     const uint32_t leader = elect_one();
     const uint32_t idesc_s = make_idesc_f16(128, kQRows, 0, 0);
     const uint32_t idesc_acc = make_idesc_f16(128, 128, 0, 1);
     const uint32_t kh = sbase + kKOffK, kl = sbase + kKOffK + kPart128;
     const uint32_t X = tmem + kKColX, Y = tmem + kKColY;
-    uint32_t item_count = 0, t = 0, p_cnt = 0, ds_cnt = 0, dv_cnt = 0, dk_cnt = 0, drains = 0;
+    uint32_t item_count = 0, t = 0, p_cnt = 0, ds_cnt = 0, drains = 0;
     bool ok = true;
     auto qstage = [&](uint32_t tt) { return sbase + kKOffQ + (tt % kKQStages) * 2 * kPart64; };
     auto dostage = [&](uint32_t tt) { return sbase + kKOffDO + (tt & 1) * 2 * kPart64; };
@@ -776,13 +772,11 @@ attn_bwd_dkv_x3_kernel(const __grid_constant__ CUtensorMap tm_q,
       ok = mbar_wait_warp(smem_u32(&bars->kv_full), item_count & 1, wc);
       if (ok) ok = mbar_wait_warp(smem_u32(&bars->q_full[t % kKQStages]),
                                   (t / kKQStages) & 1, wc);
-      if (ok && dv_cnt > 0) ok = mbar_wait_warp(smem_u32(&bars->dv_done), (dv_cnt - 1) & 1, wc);
       if (!ok) break;
       tc_fence_after();
       issue_s(t);
       ok = mbar_wait_warp(smem_u32(&bars->v_full), item_count & 1, wc);
       if (ok) ok = mbar_wait_warp(smem_u32(&bars->do_full[t & 1]), (t >> 1) & 1, wc);
-      if (ok && dk_cnt > 0) ok = mbar_wait_warp(smem_u32(&bars->dk_done), (dk_cnt - 1) & 1, wc);
       if (!ok) break;
       tc_fence_after();
       issue_dp(t);
@@ -807,12 +801,9 @@ attn_bwd_dkv_x3_kernel(const __grid_constant__ CUtensorMap tm_q,
           mma_ts_w(tmem + kKColDV, al, mndesc64(dh, kk), idesc_acc, 1u, leader);
           mma_ts_w(tmem + kKColDV, ah, mndesc64(dh, kk), idesc_acc, 1u, leader);
         }
-        mma_commit_w(smem_u32(&bars->dv_done), leader);
-        ++dv_cnt;
         if (has_next) {
-          ok = mbar_wait_warp(smem_u32(&bars->dv_done), (dv_cnt - 1) & 1, wc);
-          if (ok) ok = mbar_wait_warp(smem_u32(&bars->q_full[(t + 1) % kKQStages]),
-                                      ((t + 1) / kKQStages) & 1, wc);
+          ok = mbar_wait_warp(smem_u32(&bars->q_full[(t + 1) % kKQStages]),
+                              ((t + 1) / kKQStages) & 1, wc);
           if (!ok) break;
           tc_fence_after();
           issue_s(t + 1);
@@ -832,17 +823,13 @@ attn_bwd_dkv_x3_kernel(const __grid_constant__ CUtensorMap tm_q,
           mma_ts_w(tmem + kKColDK, al, mndesc64(qh, kk), idesc_acc, 1u, leader);
           mma_ts_w(tmem + kKColDK, ah, mndesc64(qh, kk), idesc_acc, 1u, leader);
         }
-        mma_commit_w(smem_u32(&bars->dk_done), leader);
-        ++dk_cnt;
         mma_commit_w(smem_u32(&bars->q_empty[t % kKQStages]), leader);
         if (c_last) {
           mma_commit_w(smem_u32(&bars->acc_full), leader);
           ++drains;
         }
         if (has_next) {
-          ok = mbar_wait_warp(smem_u32(&bars->dk_done), (dk_cnt - 1) & 1, wc);
-          if (ok) ok = mbar_wait_warp(smem_u32(&bars->do_full[(t + 1) & 1]),
-                                      ((t + 1) >> 1) & 1, wc);
+          ok = mbar_wait_warp(smem_u32(&bars->do_full[(t + 1) & 1]), ((t + 1) >> 1) & 1, wc);
           if (!ok) break;
           tc_fence_after();
           issue_dp(t + 1);
@@ -1034,7 +1021,7 @@ constexpr int kDSlots = 12;
 constexpr int kDKeys = 64;       // keys per tile of the dQ kernel
 struct __align__(8) DBars {
   uint64_t kv_full[kDSlots], kv_empty[kDSlots];
-  uint64_t qd_full, s_full, dp_full, dp_free, ds_full, dq_done, acc_full, acc_empty;
+  uint64_t qd_full, s_full, dp_full, dp_free, ds_full, acc_full, acc_empty;
   uint64_t drain;
   ItemRing ring;
 };
@@ -1065,7 +1052,8 @@ __device__ __forceinline__ DItem decode_d(const X3Args& a, int idx) {
 // Tiles are numbered per CTA across items (t). Region R(t & 1) holds S(t) and
 // then dS(t)'s parts; R(~t & 1) holds dP(t). S(t+1) goes into dP(t)'s region
 // once the math warps hold dP(t) in registers (dp_free), dP(t+1) into S(t)'s
-// region once dQ(t), which reads dS(t) there, has completed.
+// region right behind dQ(t), which reads dS(t) there (MMAs are performed in
+// issue order).
 __global__ void __launch_bounds__(kBThreads, 1)
 attn_bwd_dq_x3_kernel(const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const X3Args a) {
@@ -1093,7 +1081,6 @@ attn_bwd_dq_x3_kernel(const __grid_constant__ CUtensorMap tm_k,
     mbar_init(smem_u32(&bars->dp_full), 1);
     mbar_init(smem_u32(&bars->dp_free), kBMathWarps);
     mbar_init(smem_u32(&bars->ds_full), kBMathWarps);
-    mbar_init(smem_u32(&bars->dq_done), 1);
     mbar_init(smem_u32(&bars->acc_full), 1);
     mbar_init(smem_u32(&bars->acc_empty), kBMathWarps);
     mbar_init(smem_u32(&bars->drain), 1);
@@ -1142,11 +1129,11 @@ attn_bwd_dq_x3_kernel(const __grid_constant__ CUtensorMap tm_k,
     }
   } else if (warp == kBWarpMma) {
     // Per tile t: S(t+1) (after dp_free(t)), dQ(t) (after ds_full(t)), then
-    // dP(t+1) (after dQ(t) has completed).
+    // dP(t+1) right behind dQ(t).
     const uint32_t leader = elect_one();
     const uint32_t idesc_s = make_idesc_f16(128, kDKeys, 0, 0);
     const uint32_t idesc_acc = make_idesc_f16(128, 128, 0, 1);
-    uint32_t item_count = 0, t = 0, kv_base = 0, dpf_cnt = 0, ds_cnt = 0, dq_cnt = 0;
+    uint32_t item_count = 0, t = 0, kv_base = 0, dpf_cnt = 0, ds_cnt = 0;
     bool ok = true;
     auto slot = [&](uint32_t pos) { return sbase + kDOffKV + (pos % kDSlots) * kPart64; };
     auto wait_full = [&](uint32_t pos) {
@@ -1199,11 +1186,10 @@ attn_bwd_dq_x3_kernel(const __grid_constant__ CUtensorMap tm_k,
       const uint32_t nt = (uint32_t)it.ntiles;
       // Q and dO of this item in TMEM (written after the previous item's MMAs
       // completed); R(t) held dP(t-1), which the math warps have read; R(t+1)
-      // held dS(t-1), which dQ(t-1) has read.
+      // held dS(t-1), which dQ(t-1), issued before, reads.
       ok = mbar_wait_warp(smem_u32(&bars->qd_full), item_count & 1, wc);
       if (ok && t > 0) ok = mbar_wait_warp(smem_u32(&bars->dp_free), (dpf_cnt - 1) & 1, wc);
       if (ok) ok = issue_s(0, t);
-      if (ok && dq_cnt > 0) ok = mbar_wait_warp(smem_u32(&bars->dq_done), (dq_cnt - 1) & 1, wc);
       if (ok) ok = issue_dp(0, t);
       for (uint32_t n = 0; n < nt && ok; ++n) {
         const uint32_t tt = t + n;
@@ -1231,14 +1217,9 @@ attn_bwd_dq_x3_kernel(const __grid_constant__ CUtensorMap tm_k,
           mma_ts_w(tmem + kDColDQ, al, mndesc64(kh, kk), idesc_acc, 1u, leader);
           mma_ts_w(tmem + kDColDQ, ah, mndesc64(kh, kk), idesc_acc, 1u, leader);
         }
-        mma_commit_w(smem_u32(&bars->dq_done), leader);
-        ++dq_cnt;
         mma_commit_w(smem_u32(&bars->kv_empty[pos % kDSlots]), leader);
         mma_commit_w(smem_u32(&bars->kv_empty[(pos + 1) % kDSlots]), leader);
-        if (has_next) {
-          ok = mbar_wait_warp(smem_u32(&bars->dq_done), (dq_cnt - 1) & 1, wc);
-          if (ok) ok = issue_dp(n + 1, tt + 1);
-        }
+        if (has_next) ok = issue_dp(n + 1, tt + 1);
       }
       if (!ok) break;
       mma_commit_w(smem_u32(&bars->acc_full), leader);

@@ -27,10 +27,10 @@ a read of a cell while a write to it is in flight, or whose content is not the
 tile the reader expects; phase aliasing; arrivals past a barrier's count.
 MMAs from the one issuing thread are performed in issue order, so a model may
 declare (``Sim.mma_in_order``) that an MMA overwrites cells an earlier,
-unfinished MMA reads: the BF16 kernels issue an MMA into a TMEM region right
-behind the MMA that reads it (the forward's next QK behind the PV that reads P,
-dP^T behind dK, S behind dQ). The FP32-input kernels wait for the reader's
-completion instead, and for them that overlap is flagged.
+unfinished MMA reads: every kernel issues an MMA into a TMEM region right
+behind the MMA that reads it (the forwards' next QK behind the PV that reads P;
+dP^T behind dK and, in the FP32-input kernel, S^T behind dV; S or dP behind
+dQ). Any other overlap is flagged.
 
 ``MUTATIONS`` plants known mistakes in the restated protocols, so that tests can
 show the checker finds them.
@@ -695,6 +695,7 @@ PARTS = ("Kh", "Kl", "Vh", "Vl")
 
 def forward_x3(sim, items, mut=None):
     """attn_fwd_x3_kernel: one query tile per item, two S buffers, 4 softmax warps."""
+    sim.mma_in_order = True
     sim.bar("q_full"), sim.bar("q_empty")
     for s in range(X3_KV_SLOTS_FWD):
         sim.bar(f"kv_full{s}"), sim.bar(f"kv_empty{s}")
@@ -733,7 +734,7 @@ def forward_x3(sim, items, mut=None):
                     kv_load += 1
 
     def mma():
-        t, kv_base, pv = 0, 0, [0, 0]
+        t, kv_base = 0, 0
 
         def pos_k(n):
             return 0 if n == 0 else 4 * n - 2
@@ -748,8 +749,6 @@ def forward_x3(sim, items, mut=None):
             b, pos = tt & 1, kv_base + pos_k(n)
             yield ("wait", f"kv_full{pos % NS}", pos // NS)
             yield ("wait", f"kv_full{(pos + 1) % NS}", (pos + 1) // NS)
-            if pv[b] > 0 and mut != "x3f_qk_without_pv_done":
-                yield ("wait", f"pv_done{b}", pv[b] - 1)
             yield ("mma", [(["smem:Qh"], ("Qh", item)), (["smem:Ql"], ("Ql", item)),
                            slot_read(pos, ("Kh", item, n)), slot_read(pos + 1, ("Kl", item, n))],
                    tmem(f"S{b}", ALL_CHUNKS), ("S", tt), False)
@@ -781,17 +780,19 @@ def forward_x3(sim, items, mut=None):
                 # keys 0-63: P' hi in chunks 0-1, lo in chunks 2-3 of the S buffer
                 yield ("mma", [(tmem(f"S{b}", [0, 1, 2, 3]), ("P", tt)), vh, vl], o,
                        ("O", item), n > 0)
+                if mut == "x3f_qk_before_pv" and n + 2 < nt:
+                    # the QK into this S buffer overtakes the PV that still reads P
+                    yield from issue_qk(n + 2, tt + 2, item, n + 3 == nt)
                 if mut != "x3f_pv_without_p_full":
                     yield ("wait", f"p_full{b}", tt >> 1)
                 yield ("mma", [(tmem(f"S{b}", [4, 5, 6, 7]), ("P", tt)), vh, vl], o,
                        ("O", item), True)
                 yield ("commit", f"pv_done{b}")
-                pv[b] += 1
                 yield ("commit", f"kv_empty{pos % NS}")
                 yield ("commit", f"kv_empty{(pos + 1) % NS}")
                 if n + 1 == nt:
                     yield ("commit", "o_full")
-                if n + 2 < nt:
+                if n + 2 < nt and mut != "x3f_qk_before_pv":
                     yield from issue_qk(n + 2, tt + 2, item, n + 3 == nt)
             kv_base += 4 * nt
             t += nt
@@ -832,12 +833,13 @@ def forward_x3(sim, items, mut=None):
 
 def backward_dkv_x3(sim, items, mut=None):
     """attn_bwd_dkv_x3_kernel: V's parts in TMEM, 64-row query tiles, drains of dV/dK."""
+    sim.mma_in_order = True
     sim.bar("kv_full"), sim.bar("kv_empty")
     for s in range(Q_STAGES_DKV):
         sim.bar(f"q_full{s}"), sim.bar(f"q_empty{s}")
     for s in range(2):
         sim.bar(f"do_full{s}", 2), sim.bar(f"do_empty{s}")
-    for b in ("s_full", "dp_full", "dv_done", "dk_done", "acc_full"):
+    for b in ("s_full", "dp_full", "acc_full"):
         sim.bar(b)
     for b in ("v_full", "p_full", "ds_full", "acc_empty"):
         sim.bar(b, MATH_WARPS)
@@ -881,7 +883,7 @@ def backward_dkv_x3(sim, items, mut=None):
     X, Y = tmem("X", range(4)), tmem("Y", range(4))
 
     def mma():
-        t, p_cnt, ds_cnt, dv_cnt, dk_cnt, drains = 0, 0, 0, 0, 0, 0
+        t, p_cnt, ds_cnt, drains = 0, 0, 0, 0
 
         def issue_s(tt, item):
             yield ("mma", [(["smem:Kh"], ("Kh", item)), (["smem:Kl"], ("Kl", item))] + q_read(tt),
@@ -899,13 +901,9 @@ def backward_dkv_x3(sim, items, mut=None):
                 return
             yield ("wait", "kv_full", item)
             yield ("wait", f"q_full{t % QS}", t // QS)
-            if dv_cnt > 0:
-                yield ("wait", "dv_done", dv_cnt - 1)
             yield from issue_s(t, item)
             yield ("wait", "v_full", item)
             yield ("wait", f"do_full{t & 1}", t >> 1)
-            if dk_cnt > 0:
-                yield ("wait", "dk_done", dk_cnt - 1)
             yield from issue_dp(t, item)
             for m in range(nq):
                 has_next = m + 1 < nq
@@ -917,13 +915,13 @@ def backward_dkv_x3(sim, items, mut=None):
                 # kept as in the kernel
                 if c_first and drains > 0:
                     yield ("wait", "acc_empty", drains - 1)
+                if mut == "x3k_s_before_dv" and has_next:
+                    # S^T(t+1) into X ahead of the dV(t) that reads P^T(t) there
+                    yield ("wait", f"q_full{(t + 1) % QS}", (t + 1) // QS)
+                    yield from issue_s(t + 1, item)
                 yield ("mma", [(X, ("PT", t))] + do_read(t), tmem("dV", ALL_CHUNKS),
                        ("dV", drains), not c_first)
-                yield ("commit", "dv_done")
-                dv_cnt += 1
-                if has_next:
-                    if mut != "x3k_s_without_dv_done":
-                        yield ("wait", "dv_done", dv_cnt - 1)
+                if has_next and mut != "x3k_s_before_dv":
                     yield ("wait", f"q_full{(t + 1) % QS}", (t + 1) // QS)
                     yield from issue_s(t + 1, item)
                 yield ("wait", "ds_full", ds_cnt)
@@ -931,14 +929,11 @@ def backward_dkv_x3(sim, items, mut=None):
                 yield ("commit", f"do_empty{t & 1}")
                 yield ("mma", [(Y, ("dST", t))] + q_read(t), tmem("dK", ALL_CHUNKS),
                        ("dK", drains), not c_first)
-                yield ("commit", "dk_done")
-                dk_cnt += 1
                 yield ("commit", f"q_empty{t % QS}")
                 if c_last:
                     yield ("commit", "acc_full")
                     drains += 1
                 if has_next:
-                    yield ("wait", "dk_done", dk_cnt - 1)
                     yield ("wait", f"do_full{(t + 1) & 1}", (t + 1) >> 1)
                     yield from issue_dp(t + 1, item)
                 t += 1
@@ -993,10 +988,11 @@ def backward_dkv_x3(sim, items, mut=None):
 
 def backward_dq_x3(sim, items, mut=None):
     """attn_bwd_dq_x3_kernel: Q's and dO's parts in TMEM, 64-key tiles, rotating regions."""
+    sim.mma_in_order = True
     NS = X3_KV_SLOTS_DQ
     for s in range(NS):
         sim.bar(f"kv_full{s}"), sim.bar(f"kv_empty{s}")
-    for b in ("s_full", "dp_full", "dq_done", "acc_full"):
+    for b in ("s_full", "dp_full", "acc_full"):
         sim.bar(b)
     for b in ("qd_full", "dp_free", "ds_full", "acc_empty"):
         sim.bar(b, MATH_WARPS)
@@ -1021,7 +1017,7 @@ def backward_dq_x3(sim, items, mut=None):
                 kv_load += 1
 
     def mma():
-        t, kv_base, dpf_cnt, ds_cnt, dq_cnt = 0, 0, 0, 0, 0
+        t, kv_base, dpf_cnt, ds_cnt = 0, 0, 0, 0
 
         def slot_read(pos):
             return ([f"smem:kv{pos % NS}"], (PARTS[pos & 3], pos // 4))
@@ -1053,8 +1049,6 @@ def backward_dq_x3(sim, items, mut=None):
             if t > 0:
                 yield ("wait", "dp_free", dpf_cnt - 1)
             yield from issue_s(0, t, item)
-            if dq_cnt > 0:
-                yield ("wait", "dq_done", dq_cnt - 1)
             yield from issue_dp(0, t, item)
             for n in range(nt):
                 tt = t + n
@@ -1069,15 +1063,14 @@ def backward_dq_x3(sim, items, mut=None):
                 if n == 0 and item > 0:
                     yield ("wait", "acc_empty", item - 1)
                 pos = kv_base + 4 * n
+                if mut == "x3d_dp_before_dq" and has_next:
+                    # dP(t+1) into R(t) ahead of the dQ(t) that reads dS(t) there
+                    yield from issue_dp(n + 1, tt + 1, item)
                 yield ("mma", [(tmem(region(tt), range(4)), ("dS", tt)), slot_read(pos),
                                slot_read(pos + 1)], tmem("dQ", ALL_CHUNKS), ("dQ", item), n > 0)
-                yield ("commit", "dq_done")
-                dq_cnt += 1
                 yield ("commit", f"kv_empty{pos % NS}")
                 yield ("commit", f"kv_empty{(pos + 1) % NS}")
-                if has_next:
-                    if mut != "x3d_dp_without_dq_done":
-                        yield ("wait", "dq_done", dq_cnt - 1)
+                if has_next and mut != "x3d_dp_before_dq":
                     yield from issue_dp(n + 1, tt + 1, item)
             yield ("commit", "acc_full")
             kv_base += 4 * nt
@@ -1132,12 +1125,12 @@ MUTATIONS = [
     ("backward_dq", "dq_qd_empty_before_last_dp"),
     ("backward_dq", "dq_k_released_after_dp"),
     ("forward_x3", "x3f_pv_without_p_full"),
-    ("forward_x3", "x3f_qk_without_pv_done"),
+    ("forward_x3", "x3f_qk_before_pv"),
     ("forward_x3", "x3f_rescale_without_pv_done"),
-    ("backward_dkv_x3", "x3k_s_without_dv_done"),
+    ("backward_dkv_x3", "x3k_s_before_dv"),
     ("backward_dkv_x3", "x3k_v_before_last_dp"),
     ("backward_dq_x3", "x3d_s_without_dp_free"),
-    ("backward_dq_x3", "x3d_dp_without_dq_done"),
+    ("backward_dq_x3", "x3d_dp_before_dq"),
     ("backward_dq_x3", "x3d_epilogue_without_acc_full"),
 ]
 

@@ -72,13 +72,13 @@ def test_deadlock_is_reported():
         sim.run()
 
 
-@pytest.mark.parametrize("kernel", ["forward", "backward_dkv", "backward_dq"])
-def test_bf16_kernels_rely_on_in_order_mma_issue(kernel):
-    """The BF16 kernels issue an MMA into a TMEM region right behind the MMA that
-    reads it (the forward's next QK behind the PV that reads P; dP^T behind dK;
-    S behind dQ), relying on tcgen05.mma operations of one thread being
-    performed in issue order. Without that rule the same schedules must fail,
-    and only on that overlap."""
+@pytest.mark.parametrize("kernel", sorted(ITEM_LISTS))
+def test_kernels_rely_on_in_order_mma_issue(kernel):
+    """Every kernel issues an MMA into a TMEM region right behind the MMA that
+    reads it (the forwards' next QK behind the PV that reads P; dP^T behind dK;
+    S^T behind dV; S or dP behind dQ), relying on tcgen05.mma operations of one
+    thread being performed in issue order. Without that rule the same schedules
+    must fail, and only on that overlap."""
     flagged = 0
     for seed in range(20):
         sim = pm.Sim(random.Random(seed))
