@@ -18,7 +18,9 @@
 //     + RoPE at position p, a warp per row, kept in fp32 and pre-scaled by
 //     softmax_scale * log2(e)); the CTA whose chunk holds slot p also computes
 //     k_hat and appends k_hat (rounded to bf16) and v to the caches before it
-//     stages them;
+//     stages them. The raw rows are requested together with cache_lens[b], and
+//     each warp's first K/V step is staged before the rows are normalised, so
+//     a CTA's fixed start-up latency overlaps its first loads;
 //   * its 4 warps take 16-key steps, each staging its own K and V rows into
 //     shared memory with cp.async (double buffered, coalesced 16-byte copies
 //     of the head-major cache). The two small contractions run on mma.sync
@@ -55,7 +57,7 @@ constexpr int kDecStages = 2;                                       // steps in 
 constexpr int kWarpSmem = kDecStages * kStageBytes;
 constexpr int kAttnSmem = kDecWarps * kWarpSmem;
 constexpr int kMergeBytes = kDecWarps * 16 * (kHeadDim + 2) * 4;    // per-warp m, l, O for merging
-static_assert(kMergeBytes <= kAttnSmem && 16 * kHeadDim * 4 <= kAttnSmem,
+static_assert(kMergeBytes <= kAttnSmem && 16 * kHeadDim * 4 <= kStageBytes,
               "merge area and q_hat rows must fit in the staging area");
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
@@ -87,12 +89,11 @@ __device__ __forceinline__ int window_lo(const DecArgs& a, int p) {
 // A warp owns the row, lane l channels 4l..4l+3; channel c's RoPE partner
 // c +- 64 is in lane l ^ 16.
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ void warp_row_prologue(const __nv_bfloat16* x, const __nv_bfloat16* w,
-                                                  const float* cs, const float* sn, bool rope,
-                                                  float eps, float (&y)[4]) {
+// xr, wr: the lane's 4 bf16 channels of the row and of the weight.
+__device__ __forceinline__ void warp_row_prologue(uint2 xr, uint2 wr, const float* cs,
+                                                  const float* sn, bool rope, float eps,
+                                                  float (&y)[4]) {
   const int lane = threadIdx.x & 31;
-  const uint2 xr = *reinterpret_cast<const uint2*>(x + 4 * lane);
-  const uint2 wr = *reinterpret_cast<const uint2*>(w + 4 * lane);
   const __nv_bfloat162* xh = reinterpret_cast<const __nv_bfloat162*>(&xr);
   const __nv_bfloat162* wh = reinterpret_cast<const __nv_bfloat162*>(&wr);
   float xv[4], wv[4];
@@ -173,12 +174,36 @@ __device__ __forceinline__ float bf16_hi(uint32_t x) { return __uint_as_float(x 
 template <bool kPack>
 __global__ void __launch_bounds__(kDecThreads, 3) decode_attn_kernel(const DecArgs a) {
   extern __shared__ __align__(128) uint8_t dsmem[];
-  // q_hat rows of the group (log2 units): only until they are in registers, so
-  // they share the staging area
-  float (*qs)[kHeadDim] = reinterpret_cast<float (*)[kHeadDim]>(dsmem);
+  // q_hat rows of the group (log2 units), only until they are in registers: in
+  // warp 0's second staging buffer, which is first filled inside the step loop,
+  // so each warp's first step can be staged while the rows are computed
+  float (*qs)[kHeadDim] = reinterpret_cast<float (*)[kHeadDim]>(dsmem + kStageBytes);
   __shared__ float cs[kHeadDim / 2], sn[kHeadDim / 2];
   __shared__ int last_flag;
   const int s = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int gid = lane >> 2, tig = lane & 3;
+  // The raw rows this CTA normalises (the warp's query rows, and the new key and
+  // value for the CTA that appends them) are requested with cache_lens[b], so
+  // the loads overlap instead of following one another.
+  constexpr int kRowsPerWarp = 16 / kDecWarps;       // G <= 16
+  const size_t src = ((size_t)b * a.Hk + g) * kHeadDim;
+  uint2 xq[kRowsPerWarp], xk = make_uint2(0u, 0u), xv = make_uint2(0u, 0u);
+#pragma unroll
+  for (int i = 0; i < kRowsPerWarp; ++i) {
+    const int r = warp + kDecWarps * i;
+    xq[i] = make_uint2(0u, 0u);
+    if (r < a.G)
+      xq[i] = *reinterpret_cast<const uint2*>(a.q + ((size_t)b * a.H + g * a.G + r) * kHeadDim +
+                                              4 * lane);
+  }
+  const uint2 wq = *reinterpret_cast<const uint2*>(a.wq + 4 * lane);
+  uint2 wk = make_uint2(0u, 0u);
+  if (warp == kDecWarps - 1) {
+    xk = *reinterpret_cast<const uint2*>(a.k + src + 4 * lane);
+    xv = *reinterpret_cast<const uint2*>(a.v + src + 4 * lane);
+    wk = *reinterpret_cast<const uint2*>(a.wk + 4 * lane);
+  }
   const int p = __ldg(a.lens + b);
   if (!pos_ok(a, p)) {
     if (s == 0 && g == 0 && threadIdx.x == 0) atomicOr(a.status, kStatusDecodeRange);
@@ -190,11 +215,31 @@ __global__ void __launch_bounds__(kDecThreads, 3) decode_attn_kernel(const DecAr
   const int k1 = min(k0 + a.chunk, p + 1);           // keys [k0, k1)
   const int nsplit = (p - lo + a.chunk) / a.chunk;
   const bool owner = k1 == p + 1;                    // this CTA reads slot p
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int gid = lane >> 2, tig = lane & 3;
   const size_t row0 = ((size_t)b * a.Hk + g) * a.C;  // slot 0 of this (sequence, KV head)
   const __nv_bfloat16* kbase = a.kc + row0 * kHeadDim;
   const __nv_bfloat16* vbase = a.vc + row0 * kHeadDim;
+
+  const uint32_t wsm = smem_u32(dsmem) + warp * kWarpSmem;
+  const int nsteps = (k1 - k0 + kStepKeys - 1) / kStepKeys;
+  auto issue = [&](int step, int buf) {              // stage K and V rows of a step
+    const int kb = k0 + step * kStepKeys;
+    const uint32_t ks = wsm + buf * kStageBytes, vs = ks + kStepKeys * kRowBytes;
+#pragma unroll
+    for (int i = 0; i < (kStepKeys * 16) / 32; ++i) {
+      const int c = lane + 32 * i;                   // 16-byte chunk of the step
+      const int key = c >> 4, part = c & 15;
+      const int j = kb + key;
+      const bool in = j < k1;
+      const size_t off = (size_t)(in ? j : k0) * kHeadDim + part * 8;
+      cp_async16(ks + key * kRowBytes + part * 16, kbase + off, in ? 16 : 0);
+      cp_async16(vs + key * kRowBytes + part * 16, vbase + off, in ? 16 : 0);
+    }
+  };
+  // Each warp's first step goes into its first buffer now, unless it holds slot
+  // p, which is staged only after the new key and value are written there.
+  static_assert(kDecStages == 2, "one step staged ahead");
+  const bool first_early = warp < nsteps && !(owner && p < k0 + (warp + 1) * kStepKeys);
+  if (first_early) issue(warp, 0);
 
   // ---- prologue: RoPE table, the group's q_hat rows, and (owner) the append
   if (a.rope && threadIdx.x < kHeadDim / 2) {
@@ -209,23 +254,25 @@ __global__ void __launch_bounds__(kDecThreads, 3) decode_attn_kernel(const DecAr
     sn[j] = sv;
   }
   __syncthreads();
-  for (int r = warp; r < a.G; r += kDecWarps) {
-    float y[4];
-    warp_row_prologue(a.q + ((size_t)b * a.H + g * a.G + r) * kHeadDim, a.wq, cs, sn, a.rope,
-                      a.eps, y);
 #pragma unroll
-    for (int e = 0; e < 4; ++e) qs[r][4 * lane + e] = y[e] * a.scale_log2;
+  for (int i = 0; i < kRowsPerWarp; ++i) {
+    const int r = warp + kDecWarps * i;
+    if (r < a.G) {
+      float y[4];
+      warp_row_prologue(xq[i], wq, cs, sn, a.rope, a.eps, y);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) qs[r][4 * lane + e] = y[e] * a.scale_log2;
+    }
   }
   if (owner && warp == kDecWarps - 1) {
     float y[4];
-    const size_t src = ((size_t)b * a.Hk + g) * kHeadDim;
-    warp_row_prologue(a.k + src, a.wk, cs, sn, a.rope, a.eps, y);
+    warp_row_prologue(xk, wk, cs, sn, a.rope, a.eps, y);
     uint2 kb;
     kb.x = pack_bf16x2(y[0], y[1]);
     kb.y = pack_bf16x2(y[2], y[3]);
     const size_t dst = (row0 + p) * kHeadDim + 4 * lane;
     *reinterpret_cast<uint2*>(a.kc + dst) = kb;
-    *reinterpret_cast<uint2*>(a.vc + dst) = *reinterpret_cast<const uint2*>(a.v + src + 4 * lane);
+    *reinterpret_cast<uint2*>(a.vc + dst) = xv;
   }
   __threadfence_block();
   __syncthreads();                                   // slot p written before it is staged
@@ -264,22 +311,6 @@ __global__ void __launch_bounds__(kDecThreads, 3) decode_attn_kernel(const DecAr
   }
 
   __syncthreads();                                   // every warp holds its fragments
-  const uint32_t wsm = smem_u32(dsmem) + warp * kWarpSmem;
-  const int nsteps = (k1 - k0 + kStepKeys - 1) / kStepKeys;
-  auto issue = [&](int step, int buf) {              // stage K and V rows of a step
-    const int kb = k0 + step * kStepKeys;
-    const uint32_t ks = wsm + buf * kStageBytes, vs = ks + kStepKeys * kRowBytes;
-#pragma unroll
-    for (int i = 0; i < (kStepKeys * 16) / 32; ++i) {
-      const int c = lane + 32 * i;                   // 16-byte chunk of the step
-      const int key = c >> 4, part = c & 15;
-      const int j = kb + key;
-      const bool in = j < k1;
-      const size_t off = (size_t)(in ? j : k0) * kHeadDim + part * 8;
-      cp_async16(ks + key * kRowBytes + part * 16, kbase + off, in ? 16 : 0);
-      cp_async16(vs + key * kRowBytes + part * 16, vbase + off, in ? 16 : 0);
-    }
-  };
 
   // kPack: O^T, 8 m-tiles of 16 dims x the 8 heads (lane: dims mt*16 + gid and
   // + 8, heads 2tig, 2tig+1); otherwise O, 16 n-tiles of 8 dims x 16 head rows
@@ -290,12 +321,10 @@ __global__ void __launch_bounds__(kDecThreads, 3) decode_attn_kernel(const DecAr
   float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;   // rows (heads) gid, gid + 8
 
   // Each iteration commits one group (empty past the last step), so the wait
-  // count below is constant: the group of the step being computed is done.
-#pragma unroll
-  for (int j = 0; j < kDecStages - 1; ++j) {
-    if (warp + kDecWarps * j < nsteps) issue(warp + kDecWarps * j, j);
-    cp_async_commit();
-  }
+  // count below is constant: the group of the step being computed is done. The
+  // first group holds the warp's first step, staged early or now.
+  if (warp < nsteps && !first_early) issue(warp, 0);
+  cp_async_commit();
   int it = 0;
   for (int step = warp; step < nsteps; step += kDecWarps, ++it) {
     const int buf = it % kDecStages;
