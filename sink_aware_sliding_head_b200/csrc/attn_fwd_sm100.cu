@@ -218,8 +218,8 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
     // ------------------------------------------------------------ MMA issuer
     // Issue order per key tile n: PV0(n), QK0(n+1), PV1(n), QK1(n+1). Tile 1
     // runs half a period behind tile 0, so each tile's softmax overlaps the
-    // other tile's MMAs. QK_i(n+1) overwrites S_i, which holds P_i(n), so it
-    // is issued only after PV_i(n) has completed.
+    // other tile's MMAs. QK_i(n+1) overwrites S_i, which holds P_i(n); it is
+    // issued right behind PV_i(n), the MMAs being performed in issue order.
     {
       const uint32_t leader = elect_one();   // the one lane that issues
       const uint32_t idesc_qk = make_idesc_f16(128, 128, 0, 0);
