@@ -43,8 +43,8 @@
 //    tiles: S = Q K^T, dP = dO V^T, dS (fp16) over S, dQ += dS K. TMEM: two S
 //    buffers, dP, dQ = 512 cols; S of the next key tile is computed while the
 //    math warps finish the current one. K and V stream through a 5-slot ring.
-// In both P steps one exponential pair in four is evaluated on the FMA pipe
-// (exp2_fma2); the special-function unit alone would bound them.
+// In the P steps one exponential pair in four (dK/dV) or eight (dQ) is evaluated
+// on the FMA pipe (exp2_fma2); the special-function unit alone would bound them.
 // An MMA that overwrites a TMEM region a previous MMA reads as its A operand
 // is issued right behind it without a completion wait: tcgen05.mma operations
 // issued by one thread are performed in issue order.
@@ -819,10 +819,11 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q,
               const uint32_t a1 = e < 16 ? u0[2 * e + 1] : u1[2 * e - 31];
               float x0, x1;
               f2_split(ffma2(f2(__uint_as_float(a0), __uint_as_float(a1)), sc2, nl2), x0, x1);
-              // one pair in four on the FMA pipe (polynomial 2^x), the rest on
-              // the special-function unit, which alone would bound this loop
+              // one pair in eight on the FMA pipe (polynomial 2^x), the rest on
+              // the special-function unit (one in four, or two, measured slower
+              // here; the dK/dV kernel prefers one in four)
               float p0, p1;
-              if ((e & 3) == 3) exp2_fma2(x0, x1, p0, p1);
+              if ((e & 7) == 7) exp2_fma2(x0, x1, p0, p1);
               else { p0 = ex2_approx(x0); p1 = ex2_approx(x1); }
               if (decltype(masked)::value) {
                 const int c = c0 + 2 * e;
