@@ -48,3 +48,39 @@ def test_flops_per_pair():
 def test_decode_kv_bytes_equals_brute_force(lens, W):
     slots = sum(hi - lo + 1 for lo, hi in (fo.visible_keys(p, 0, W) for p in lens))
     assert bench.decode_kv_bytes(lens, W, 4) == slots * 4 * 128 * 2 * 2
+
+
+def test_clock_sampler_starts_timing_after_its_first_sample(tmp_path, monkeypatch):
+    """The clock sampler's start() returns only once nvidia-smi has written its
+    first sample: a slow start-up (driver and NVML initialisation) must not fall
+    inside a timed region. A stand-in nvidia-smi that needs 0.4 s before its first
+    line checks that, and stop() parses the samples it wrote."""
+    import os
+    import stat
+    import time
+    fake = tmp_path / "nvidia-smi"
+    fake.write_text("#!/bin/sh\nsleep 0.4\n"
+                    "while true; do\n"
+                    "  echo '0, 1500, 1965, 700.5, Active, Not Active, Not Active, Not Active, Active'\n"
+                    "  sleep 0.05\n"
+                    "done\n")
+    fake.chmod(fake.stat().st_mode | stat.S_IEXEC)
+    monkeypatch.setenv("PATH", f"{tmp_path}{os.pathsep}{os.environ.get('PATH', '')}")
+    sampler = bench.ClockSampler()
+    t0 = time.time()
+    sampler.start()
+    waited = time.time() - t0
+    assert waited >= 0.35, waited
+    assert os.path.getsize(sampler.path) > 0
+    time.sleep(0.1)
+    clocks = sampler.stop()
+    assert clocks["sm_mhz"] == 1500.0 and clocks["sm_max_mhz"] == 1965.0
+    assert clocks["reasons"] == ["sw_power_cap"] and clocks["samples_under_load"] >= 1
+
+
+def test_clock_sampler_without_nvidia_smi(tmp_path, monkeypatch):
+    """No nvidia-smi on PATH: start() returns at once and stop() reports nothing."""
+    monkeypatch.setenv("PATH", str(tmp_path))
+    sampler = bench.ClockSampler()
+    sampler.start()
+    assert sampler.stop() is None
