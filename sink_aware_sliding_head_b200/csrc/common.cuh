@@ -285,9 +285,8 @@ struct DecodeLaunch {
   int* status;
 };
 // Split CTAs per (sequence, KV head): the most any call with capacity C and window W
-// launches (the workspace is sized for it), and the count a launch uses.
+// launches (the workspace is sized for it).
 int decode_splits_max(int C, int W);
-int decode_splits(int B, int Hk, int C, int W, int num_sms);
 cudaError_t launch_decode(const DecodeLaunch& L, cudaStream_t st);
 cudaError_t launch_attn_fwd_fp32(const Resolved& p, const float* qh, const float* kh,
                                  const float* v, const float* sink, const int32_t* cu, float* out,

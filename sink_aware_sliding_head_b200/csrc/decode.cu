@@ -12,8 +12,9 @@
 // Decode is bound by HBM: every key costs 512 bytes of K and V and feeds only
 // the G query heads of its group. One kernel, grid (splits, Hk, B); each CTA
 // covers one chunk of one (sequence, KV head) window (the splits divide the
-// largest window evenly in multiples of 16 keys; their number aims at about
-// five CTAs per SM, see decode_splits):
+// largest window evenly in multiples of 16 keys; about five CTAs per SM, or for
+// batches with 1 to 1.5 times as many pairs as resident CTA slots two full
+// waves of one- and two-split pairs, see decode_split_plan):
 //   * it normalises and rotates the G query rows of its group itself (RMSNorm
 //     + RoPE at position p, a warp per row, kept in fp32 and pre-scaled by
 //     softmax_scale * log2(e)); the CTA whose chunk holds slot p also computes
@@ -64,7 +65,8 @@ constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescale = 8.0f;               // log2 units
 
 struct DecArgs {
-  int B, C, H, Hk, G, W, rope, splits, chunk, out_f32;   // splits: stride of the partials
+  int B, C, H, Hk, G, W, rope, splits, out_f32;   // splits: stride of the partials
+  int chunk_a, chunk_b, pair_split;  // keys per chunk: pairs < pair_split chunk_a, the rest chunk_b
   float theta, eps, scale_log2;
   const __nv_bfloat16 *q, *k, *v, *wq, *wk;
   const float* sink;
@@ -210,10 +212,11 @@ __global__ void __launch_bounds__(kDecThreads, 3) decode_attn_kernel(const DecAr
     return;
   }
   const int lo = window_lo(a, p);
-  const int k0 = lo + s * a.chunk;
+  const int chunk = (b * a.Hk + g < a.pair_split) ? a.chunk_a : a.chunk_b;
+  const int k0 = lo + s * chunk;
   if (k0 > p) return;                                // this split has no keys
-  const int k1 = min(k0 + a.chunk, p + 1);           // keys [k0, k1)
-  const int nsplit = (p - lo + a.chunk) / a.chunk;
+  const int k1 = min(k0 + chunk, p + 1);             // keys [k0, k1)
+  const int nsplit = (p - lo + chunk) / chunk;
   const bool owner = k1 == p + 1;                    // this CTA reads slot p
   const size_t row0 = ((size_t)b * a.Hk + g) * a.C;  // slot 0 of this (sequence, KV head)
   const __nv_bfloat16* kbase = a.kc + row0 * kHeadDim;
@@ -601,18 +604,43 @@ int decode_splits_max(int C, int W) {
   return (max_window_keys(C, W) + kMinChunkKeysDecode - 1) / kMinChunkKeysDecode;
 }
 
-// About five CTAs per SM over all (sequence, KV head) pairs: at three resident CTAs
-// per SM that is two waves, the second nearly full. Measured on the 64-sequence,
-// window-4096 serving shape (256 pairs, 148 SMs): 3 splits of 1376 keys 4235 GB/s of
-// K and V, 4 of 1024 4100, 5 of 832 4040, 2 of 2048 3690.
-int decode_splits(int B, int Hk, int C, int W, int num_sms) {
-  const long long pairs = (long long)B * Hk;
-  long long s = pairs > 0 ? (5LL * num_sms + pairs / 2) / pairs : 1;
+namespace {
+constexpr int kDecResident = 3;   // CTAs per SM (shared memory and registers alike)
+
+// The split plan: the first pair_split pairs take s splits, the rest grid_x.
+//   * Fewer pairs than resident CTA slots: about five CTAs per SM, one split
+//     count for all pairs (at three resident CTAs per SM two waves, the second
+//     nearly full). Measured on the 64-sequence, window-4096 serving shape (256
+//     pairs, 148 SMs): 3 splits of 1376 keys 4235 GB/s of K and V, 4 of 1024
+//     4100, 5 of 832 4040, 2 of 2048 3690 with the padded kernel; a two-wave plan
+//     as below 4503-4506 against 4623.
+//   * Between one and one and a half times as many pairs as slots: exactly two
+//     waves, the first pairs with one split and the rest with two (the larger
+//     chunks all launch in the first wave). 148 sequences (592 pairs): 5613-5663
+//     GB/s against 5181-5224 for one split each (1.33 waves); 120 sequences (480
+//     pairs): 5400 against 5285 for two splits each (2.16 waves).
+struct SplitPlan {
+  int s, pair_split, grid_x;
+};
+SplitPlan decode_split_plan(int B, int Hk, int C, int W, int num_sms) {
+  const long long P = (long long)B * Hk;
   const int smax = decode_splits_max(C, W);
-  if (s < 1) s = 1;
-  if (s > smax) s = smax;
-  return (int)s;
+  if (P <= 0) return {1, 0, 1};
+  if (P < (long long)kDecResident * num_sms) {
+    long long s = (5LL * num_sms + P / 2) / P;
+    if (s < 1) s = 1;
+    if (s > smax) s = smax;
+    return {(int)s, (int)P, (int)s};
+  }
+  const long long S = (long long)kDecResident * num_sms, T = 2 * S;
+  long long s = T / P, r = T % P;
+  // only while the larger chunks all start in the first wave (P <= 1.5 slots);
+  // beyond, one split each (800 pairs: 6020 GB/s against 5936 for the plan)
+  if (s < 1 || P - r > S) { s = 1; r = 0; }
+  if (s >= smax) { s = smax; r = 0; }
+  return {(int)s, (int)(P - r), (int)(s + (r > 0 ? 1 : 0))};
 }
+}  // namespace
 
 cudaError_t launch_decode(const DecodeLaunch& L, cudaStream_t st) {
   static PerDeviceOnce smem_once_pack, smem_once_full;
@@ -625,8 +653,11 @@ cudaError_t launch_decode(const DecodeLaunch& L, cudaStream_t st) {
   a.rope = L.rope; a.theta = L.theta; a.eps = L.eps;
   a.scale_log2 = L.scale * kLog2e;
   a.splits = decode_splits_max(L.C, L.W);            // stride of the partials
-  const int launched = decode_splits(L.B, L.Hk, L.C, L.W, L.num_sms);
-  a.chunk = chunk_keys(L.C, L.W, launched);
+  const SplitPlan plan = decode_split_plan(L.B, L.Hk, L.C, L.W, L.num_sms);
+  a.chunk_a = chunk_keys(L.C, L.W, plan.s);
+  a.chunk_b = chunk_keys(L.C, L.W, plan.grid_x);
+  a.pair_split = plan.pair_split;
+  const int launched = plan.grid_x;
   a.out_f32 = L.out_f32;
   a.q = static_cast<const __nv_bfloat16*>(L.q);
   a.k = static_cast<const __nv_bfloat16*>(L.k);
